@@ -1,0 +1,227 @@
+"""B200-native Kimi Delta Attention (KDA) gated delta-rule recurrence.
+
+Thin ctypes binding over ``libkda.so`` (C ABI in ``include/kda.h``). This module only marshals
+arguments: it checks tensor dtypes and shapes, allocates outputs with PyTorch (PyTorch is used
+for device memory and streams only) and passes raw device pointers plus the current CUDA stream
+to the library. Every step of the recurrence runs in the library's CUDA kernels; there is no CPU
+path. Calling any function without the built library, or with CPU tensors, raises.
+
+Functions mirror the C entry points:
+    fwd(q, k, v, log_g, beta, h0=None, cu_seqlens=None, ...)  -> (o, hT)     [kda_fwd]
+    decode_step(q, k, v, log_g, beta, S, o=None)               -> o          [kda_decode_step]
+    get_device_error(stream=None)                                             [kda_get_device_error]
+"""
+
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+__all__ = ["fwd", "decode_step", "get_device_error", "fwd_workspace_size", "KdaError",
+           "library_path", "lib", "CHUNK_AUTO", "CHUNK_PER_TOKEN", "CHUNK_64"]
+
+_PKG = Path(__file__).resolve().parent
+_LIB_PATH = _PKG / "libkda.so"
+
+CHUNK_AUTO, CHUNK_PER_TOKEN, CHUNK_64 = 0, 1, 64
+KDA_F32, KDA_BF16 = 0, 1
+STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_CUDA",
+          4: "KDA_ERR_TIMEOUT", 5: "KDA_ERR_BAD_SEQLENS", 6: "KDA_ERR_RANGE"}
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        super().__init__("%s: %s%s" % (where, STATUS.get(status, str(status)),
+                                       (" (" + detail + ")") if detail else ""))
+
+
+class FwdDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("num_seqs", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("chunk_size", ctypes.c_int)]
+
+
+_lib = None
+
+
+def library_path() -> Path:
+    return _LIB_PATH
+
+
+def lib():
+    """Load libkda.so (once). Raises if it has not been built: there is no fallback."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not _LIB_PATH.exists():
+        raise RuntimeError("libkda.so is missing at %s; build it with "
+                           "`python -m gated_delta_rule_144_b200.build`" % _LIB_PATH)
+    L = ctypes.CDLL(str(_LIB_PATH))
+    p, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.kda_fwd.argtypes = [ctypes.POINTER(FwdDesc), p, p, p, p, p, p, p, p, p, p, sz, p]
+    L.kda_fwd.restype = i32
+    L.kda_fwd_workspace_size.argtypes = [ctypes.POINTER(FwdDesc)]
+    L.kda_fwd_workspace_size.restype = sz
+    L.kda_decode_step.argtypes = [i32, i32, i32, i32, i32, p, p, p, p, p, p, p, p]
+    L.kda_decode_step.restype = i32
+    L.kda_get_device_error.argtypes = [p]
+    L.kda_get_device_error.restype = i32
+    L.kda_status_string.argtypes = [i32]
+    L.kda_status_string.restype = ctypes.c_char_p
+    L.kda_last_error.argtypes = []
+    L.kda_last_error.restype = ctypes.c_char_p
+    L.kda_version.argtypes = []
+    L.kda_version.restype = i32
+    _lib = L
+    return L
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise KdaError(status, where, lib().kda_last_error().decode(errors="replace"))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_F32
+    raise TypeError("q/k/v/beta must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _dev(t, name, dtype=None, shape=None, device=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.device.type != "cuda":
+        raise ValueError("%s must be a CUDA tensor (the library has no CPU path)" % name)
+    if device is not None and t.device != device:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return t
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def fwd_workspace_size(B, T, H, dk, dv, num_seqs, dtype=torch.bfloat16, chunk_size=0) -> int:
+    d = FwdDesc(B, T, H, dk, dv, num_seqs, KDA_BF16 if dtype == torch.bfloat16 else KDA_F32,
+                chunk_size)
+    return int(lib().kda_fwd_workspace_size(ctypes.byref(d)))
+
+
+def fwd(q, k, v, log_g, beta, h0=None, cu_seqlens=None, *, chunk_size: int = CHUNK_AUTO,
+        output_final_state: bool = True, o=None, hT=None, workspace=None, stream=None):
+    """Prefill (``kda_fwd``): the recurrence over whole sequences or packed documents.
+
+    q, k, log_g: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H]; q/k/v/beta share one dtype
+    (bf16 or fp32), log_g is fp32. h0: [N, H, dk, dv] fp32 or None. cu_seqlens: int32 [N + 1]
+    on the device (B must be 1) or None. Returns (o [B, T, H, dv], hT [N, H, dk, dv] fp32 or
+    None). Outputs may be passed in preallocated.
+    """
+    lib()
+    _dev(q, "q")
+    dev = q.device
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, dk]")
+    B, T, H, dk = q.shape
+    dt = q.dtype
+    _dtype_code(q)
+    _dev(k, "k", dt, (B, T, H, dk), dev)
+    _dev(log_g, "log_g", torch.float32, (B, T, H, dk), dev)
+    _dev(v, "v", dt, None, dev)
+    if v.dim() != 4 or tuple(v.shape[:3]) != (B, T, H):
+        raise ValueError("v must be [B, T, H, dv]")
+    dv = v.shape[3]
+    _dev(beta, "beta", dt, (B, T, H), dev)
+    if cu_seqlens is not None:
+        _dev(cu_seqlens, "cu_seqlens", torch.int32, None, dev)
+        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+            raise ValueError("cu_seqlens must be a 1-D int32 tensor of N + 1 offsets")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    _dev(h0, "h0", torch.float32, (N, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    else:
+        _dev(o, "o", dt, (B, T, H, dv), dev)
+    if output_final_state:
+        if hT is None:
+            hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+        else:
+            _dev(hT, "hT", torch.float32, (N, H, dk, dv), dev)
+    else:
+        hT = None
+    desc = FwdDesc(B, T, H, dk, dv, N, _dtype_code(q), chunk_size)
+    need = int(lib().kda_fwd_workspace_size(ctypes.byref(desc)))
+    if need > 0:
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        _dev(workspace, "workspace", torch.uint8, None, dev)
+        if workspace.numel() < need:
+            raise ValueError("workspace needs %d bytes" % need)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    with torch.cuda.device(dev):
+        st = lib().kda_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(log_g),
+                           _ptr(beta), _ptr(h0), _ptr(cu_seqlens), _ptr(o), _ptr(hT),
+                           _ptr(workspace), ws_bytes, _stream(stream, dev))
+    _check(st, "kda_fwd")
+    return o, hT
+
+
+def decode_step(q, k, v, log_g, beta, S, *, o=None, stream=None):
+    """One decode token for N sequences (``kda_decode_step``); S is updated in place.
+
+    q, k, log_g: [N, H, dk]; v: [N, H, dv]; beta: [N, H]; S: [N, H, dk, dv] fp32.
+    Returns o [N, H, dv] in the dtype of q.
+    """
+    lib()
+    _dev(q, "q")
+    dev = q.device
+    if q.dim() != 3:
+        raise ValueError("q must be [N, H, dk]")
+    N, H, dk = q.shape
+    dt = q.dtype
+    _dtype_code(q)
+    _dev(k, "k", dt, (N, H, dk), dev)
+    _dev(log_g, "log_g", torch.float32, (N, H, dk), dev)
+    _dev(v, "v", dt, None, dev)
+    if v.dim() != 3 or tuple(v.shape[:2]) != (N, H):
+        raise ValueError("v must be [N, H, dv]")
+    dv = v.shape[2]
+    _dev(beta, "beta", dt, (N, H), dev)
+    _dev(S, "S", torch.float32, (N, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=dt, device=dev)
+    else:
+        _dev(o, "o", dt, (N, H, dv), dev)
+    with torch.cuda.device(dev):
+        st = lib().kda_decode_step(N, H, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+                                   _ptr(log_g), _ptr(beta), _ptr(S), _ptr(o),
+                                   _stream(stream, dev))
+    _check(st, "kda_decode_step")
+    return o
+
+
+def get_device_error(stream=None, device=None) -> int:
+    """Synchronise and return (then clear) the library's sticky device error code (0 = none)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        return int(lib().kda_get_device_error(_stream(stream, dev)))

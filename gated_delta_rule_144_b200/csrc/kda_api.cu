@@ -1,0 +1,228 @@
+// C ABI of libkda.so: argument validation, path selection and the device error word.
+// Declarations and the contract of every entry point are in include/kda.h.
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "kda.h"
+#include "kda_internal.cuh"
+
+namespace {
+
+// Sticky device error word (one per device context; see kda_get_device_error).
+__device__ unsigned g_device_error = 0;
+
+thread_local char t_last_error[512] = "";
+
+kda_status_t fail(kda_status_t st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+kda_status_t cuda_fail(cudaError_t e, const char* what) {
+    return fail(KDA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int kMaxDevices = 64;
+unsigned* g_err_addr[kMaxDevices] = {};
+std::mutex g_err_mu;
+
+// Device address of the error word on the current device (looked up once per device).
+kda_status_t device_error_word(unsigned** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(KDA_ERR_UNSUPPORTED, "device %d", dev);
+    std::lock_guard<std::mutex> lock(g_err_mu);
+    if (!g_err_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_device_error);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+        g_err_addr[dev] = static_cast<unsigned*>(p);
+    }
+    *out = g_err_addr[dev];
+    return KDA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+kda_status_t check_ptr(const void* p, const char* name, bool required) {
+    if (!p) return required ? fail(KDA_ERR_INVALID_ARG, "%s is NULL", name) : KDA_OK;
+    if (!aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return KDA_OK;
+}
+
+enum class Path { kPerToken, kChunk64 };
+
+kda_status_t check_fwd_desc(const kda_fwd_desc_t* d, bool has_cu, Path* path) {
+    if (!d) return fail(KDA_ERR_INVALID_ARG, "desc is NULL");
+    if (d->B < 1 || d->T < 0 || d->H < 1 || d->dk < 1 || d->dv < 1 || d->num_seqs < 0)
+        return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d H=%d dk=%d dv=%d N=%d", d->B, d->T,
+                    d->H, d->dk, d->dv, d->num_seqs);
+    if (d->dtype != KDA_F32 && d->dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARG, "unknown dtype %d", (int)d->dtype);
+    if (has_cu) {
+        if (d->B != 1) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens requires B == 1");
+    } else if (d->num_seqs != d->B) {
+        return fail(KDA_ERR_INVALID_ARG, "num_seqs (%d) must equal B (%d) without cu_seqlens",
+                    d->num_seqs, d->B);
+    }
+    if ((int64_t)d->B * d->T * d->H > (int64_t)1 << 40)
+        return fail(KDA_ERR_INVALID_ARG, "problem too large");
+    const bool tc_shape =
+        d->dtype == KDA_BF16 && d->dk == 128 && d->dv == 128 && kda::chunk64_available();
+    switch (d->chunk_size) {
+        case KDA_CHUNK_AUTO:
+            *path = tc_shape ? Path::kChunk64 : Path::kPerToken;
+            break;
+        case KDA_CHUNK_PER_TOKEN:
+            *path = Path::kPerToken;
+            break;
+        case KDA_CHUNK_64:
+            if (d->dtype == KDA_F32) {
+                *path = Path::kPerToken;  // fp32 inputs always take the exact path
+                break;
+            }
+            if (!tc_shape)
+                return fail(KDA_ERR_UNSUPPORTED,
+                            "chunk_size 64 needs bf16 with dk = dv = 128 (and the chunked kernel)");
+            *path = Path::kChunk64;
+            break;
+        default:
+            if (d->dtype == KDA_F32 && d->chunk_size > 0) {
+                *path = Path::kPerToken;
+                break;
+            }
+            return fail(KDA_ERR_UNSUPPORTED, "chunk_size %d", d->chunk_size);
+    }
+    if (*path == Path::kPerToken && (d->dk > 256 || d->dv > 256))
+        return fail(KDA_ERR_UNSUPPORTED, "per-token path supports dk, dv <= 256");
+    return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kda_version(void) { return 100; }
+
+const char* kda_last_error(void) { return t_last_error; }
+
+const char* kda_status_string(kda_status_t s) {
+    switch (s) {
+        case KDA_OK: return "ok";
+        case KDA_ERR_INVALID_ARG: return "invalid argument";
+        case KDA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case KDA_ERR_CUDA: return "CUDA runtime error";
+        case KDA_ERR_TIMEOUT: return "device pipeline wait timed out";
+        case KDA_ERR_BAD_SEQLENS: return "malformed cu_seqlens";
+        case KDA_ERR_RANGE: return "decay too steep for the chunked path";
+    }
+    return "unknown status";
+}
+
+size_t kda_fwd_workspace_size(const kda_fwd_desc_t* desc) {
+    (void)desc;
+    return 0;
+}
+
+kda_status_t kda_fwd(const kda_fwd_desc_t* d, const void* q, const void* k, const void* v,
+                     const float* log_g, const void* beta, const float* h0,
+                     const int32_t* cu_seqlens, void* o, float* hT, void* workspace,
+                     size_t workspace_bytes, kda_stream_t stream) {
+    t_last_error[0] = 0;
+    (void)workspace;
+    (void)workspace_bytes;
+    Path path;
+    kda_status_t st = check_fwd_desc(d, cu_seqlens != nullptr, &path);
+    if (st != KDA_OK) return st;
+    const bool tokens = (int64_t)d->B * d->T > 0;
+    const bool has_units = d->num_seqs > 0;
+    if ((st = check_ptr(q, "q", tokens)) || (st = check_ptr(k, "k", tokens)) ||
+        (st = check_ptr(v, "v", tokens)) || (st = check_ptr(log_g, "log_g", tokens)) ||
+        (st = check_ptr(beta, "beta", false)) || (st = check_ptr(o, "o", tokens)) ||
+        (st = check_ptr(h0, "h0", false)) || (st = check_ptr(hT, "hT", false)) ||
+        (st = check_ptr(cu_seqlens, "cu_seqlens", false)))
+        return st;
+    if (tokens && !beta) return fail(KDA_ERR_INVALID_ARG, "beta is NULL");
+    if (!has_units) return KDA_OK;
+
+    kda::FwdParams p{};
+    p.q = q; p.k = k; p.v = v; p.log_g = log_g; p.beta = beta; p.h0 = h0;
+    p.cu_seqlens = cu_seqlens; p.o = o; p.hT = hT;
+    p.B = d->B; p.T = d->T; p.H = d->H; p.dk = d->dk; p.dv = d->dv; p.N = d->num_seqs;
+    p.bf16 = d->dtype == KDA_BF16;
+    if ((st = device_error_word(&p.err)) != KDA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = path == Path::kChunk64 ? kda::launch_chunk64(p, s)
+                                           : kda::launch_recurrent(p, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_fwd launch");
+    return KDA_OK;
+}
+
+kda_status_t kda_decode_step(int N, int H, int dk, int dv, kda_dtype_t dtype, const void* q,
+                             const void* k, const void* v, const float* log_g, const void* beta,
+                             float* S_inout, void* o, kda_stream_t stream) {
+    t_last_error[0] = 0;
+    if (N < 0 || H < 1 || dk < 1 || dv < 1)
+        return fail(KDA_ERR_INVALID_ARG, "bad sizes N=%d H=%d dk=%d dv=%d", N, H, dk, dv);
+    if (dtype != KDA_F32 && dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (dk > 256 || dv > 256) return fail(KDA_ERR_UNSUPPORTED, "decode supports dk, dv <= 256");
+    kda_status_t st;
+    const bool any = N > 0;
+    if ((st = check_ptr(q, "q", any)) || (st = check_ptr(k, "k", any)) ||
+        (st = check_ptr(v, "v", any)) || (st = check_ptr(log_g, "log_g", any)) ||
+        (st = check_ptr(beta, "beta", any)) || (st = check_ptr(S_inout, "S_inout", any)) ||
+        (st = check_ptr(o, "o", any)))
+        return st;
+    if (!any) return KDA_OK;
+    unsigned* err = nullptr;
+    if ((st = device_error_word(&err)) != KDA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (dk == 128 && dv == 128) {
+        kda::DecodeParams p{q, k, v, log_g, beta, S_inout, o, N, H, dk, dv,
+                            dtype == KDA_BF16, err};
+        e = kda::launch_decode_d128(p, s);
+    } else {
+        // general sizes: the per-token walk over one token, state read from and written to S
+        kda::FwdParams p{};
+        p.q = q; p.k = k; p.v = v; p.log_g = log_g; p.beta = beta; p.h0 = S_inout;
+        p.cu_seqlens = nullptr; p.o = o; p.hT = S_inout;
+        p.B = N; p.T = 1; p.H = H; p.dk = dk; p.dv = dv; p.N = N;
+        p.bf16 = dtype == KDA_BF16;
+        p.err = err;
+        e = kda::launch_recurrent(p, s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step launch");
+    return KDA_OK;
+}
+
+kda_status_t kda_get_device_error(kda_stream_t stream) {
+    t_last_error[0] = 0;
+    unsigned* err = nullptr;
+    kda_status_t st = device_error_word(&err);
+    if (st != KDA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned host = 0;
+    cudaError_t e = cudaMemcpyAsync(&host, err, sizeof(host), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+    if (host != 0) {
+        const unsigned zero = 0;
+        e = cudaMemcpyAsync(err, &zero, sizeof(zero), cudaMemcpyHostToDevice, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+        return fail(static_cast<kda_status_t>(host), "device reported: %s",
+                    kda_status_string(static_cast<kda_status_t>(host)));
+    }
+    return KDA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,140 @@
+// Single-token decode for dk = dv = 128: the bandwidth-bound state update, in place.
+//
+// One token per sequence (metrale glm5next_layer page: KDA decode with a per-sequence
+// KdaSeqState), recurrence from the GLM-5.3-Flash model card's Kimi Delta Attention snippet.
+// The fp32 state (64 KiB per sequence-head) is read once and written once; every other byte is
+// small. With S' = diag(g) S,
+//     m = k^T S',  p = q^T S',  delta = beta (v - m),  o = p + (q.k) delta,  S <- S' + k delta^T
+// (o equals q^T of the written state because q^T (S' + k delta^T) = p + (q.k) delta^T).
+//
+// Layout of the work: a 128-thread block owns one (sequence, head); warp w owns value columns
+// [32w, 32w + 32). Lane l covers row phase l / 8 (rows r = l/8 + 4i, i < 32) and the four
+// columns 32w + 4 (l % 8) .. + 3, so each warp load instruction reads four 128-byte row segments
+// (fully coalesced 16-byte loads) and every lane keeps its 32 float4 of S in registers between
+// the read and the write. The key-axis reduction is 32 rows in-thread, then a butterfly over the
+// four row phases (shuffle xor 8, 16). Loads and stores of S use the streaming cache hint: the
+// state is touched once per step.
+
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kRowsPerLane = 32;
+
+__device__ __forceinline__ float4 load_v4(const __nv_bfloat16* p) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    float4 r;
+    r.x = __uint_as_float(u.x << 16);
+    r.y = __uint_as_float(u.x & 0xffff0000u);
+    r.z = __uint_as_float(u.y << 16);
+    r.w = __uint_as_float(u.y & 0xffff0000u);
+    return r;
+}
+__device__ __forceinline__ float4 load_v4(const float* p) {
+    return *reinterpret_cast<const float4*>(p);
+}
+__device__ __forceinline__ void store_v4(__nv_bfloat16* p, float4 x) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(x.x, x.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(x.z, x.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+}
+__device__ __forceinline__ void store_v4(float* p, float4 x) {
+    *reinterpret_cast<float4*>(p) = x;
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(128)
+decode_d128_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                   const Tin* __restrict__ v, const float* __restrict__ log_g,
+                   const Tin* __restrict__ beta, float* __restrict__ S, Tin* __restrict__ o) {
+    __shared__ float s_q[kD], s_k[kD], s_g[kD];
+    const int unit = blockIdx.x;  // n * H + h
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int phase = lane >> 3;                  // row phase 0..3
+    const int col = warp * 32 + (lane & 7) * 4;   // first of this lane's four columns
+
+    float4* Sp = reinterpret_cast<float4*>(S + (size_t)unit * kD * kD);
+    float4 s[kRowsPerLane];
+#pragma unroll
+    for (int i = 0; i < kRowsPerLane; ++i) {
+        const int r = phase + 4 * i;
+        s[i] = __ldcs(Sp + (r * kD + col) / 4);
+    }
+
+    const size_t vec = (size_t)unit * kD;
+    s_q[tid] = load_elem(q, vec + tid);
+    s_k[tid] = load_elem(k, vec + tid);
+    s_g[tid] = expf(log_g[vec + tid]);
+    const float4 vv = load_v4(v + vec + col);
+    const float b = load_elem(beta, unit);
+    __syncthreads();
+
+    float4 m = make_float4(0.f, 0.f, 0.f, 0.f), p = m;
+    float qk = 0.f;
+#pragma unroll
+    for (int i = 0; i < kRowsPerLane; ++i) {
+        const int r = phase + 4 * i;
+        const float g = s_g[r], kr = s_k[r], qr = s_q[r];
+        s[i].x *= g; s[i].y *= g; s[i].z *= g; s[i].w *= g;
+        m.x = fmaf(kr, s[i].x, m.x); m.y = fmaf(kr, s[i].y, m.y);
+        m.z = fmaf(kr, s[i].z, m.z); m.w = fmaf(kr, s[i].w, m.w);
+        p.x = fmaf(qr, s[i].x, p.x); p.y = fmaf(qr, s[i].y, p.y);
+        p.z = fmaf(qr, s[i].z, p.z); p.w = fmaf(qr, s[i].w, p.w);
+        qk = fmaf(qr, kr, qk);
+    }
+#pragma unroll
+    for (int off = 8; off <= 16; off <<= 1) {
+        m.x += __shfl_xor_sync(0xffffffffu, m.x, off);
+        m.y += __shfl_xor_sync(0xffffffffu, m.y, off);
+        m.z += __shfl_xor_sync(0xffffffffu, m.z, off);
+        m.w += __shfl_xor_sync(0xffffffffu, m.w, off);
+        p.x += __shfl_xor_sync(0xffffffffu, p.x, off);
+        p.y += __shfl_xor_sync(0xffffffffu, p.y, off);
+        p.z += __shfl_xor_sync(0xffffffffu, p.z, off);
+        p.w += __shfl_xor_sync(0xffffffffu, p.w, off);
+        qk += __shfl_xor_sync(0xffffffffu, qk, off);
+    }
+    float4 d;
+    d.x = b * (vv.x - m.x); d.y = b * (vv.y - m.y);
+    d.z = b * (vv.z - m.z); d.w = b * (vv.w - m.w);
+    if (phase == 0) {
+        float4 out;
+        out.x = fmaf(qk, d.x, p.x); out.y = fmaf(qk, d.y, p.y);
+        out.z = fmaf(qk, d.z, p.z); out.w = fmaf(qk, d.w, p.w);
+        store_v4(o + vec + col, out);
+    }
+#pragma unroll
+    for (int i = 0; i < kRowsPerLane; ++i) {
+        const int r = phase + 4 * i;
+        const float kr = s_k[r];
+        s[i].x = fmaf(kr, d.x, s[i].x); s[i].y = fmaf(kr, d.y, s[i].y);
+        s[i].z = fmaf(kr, d.z, s[i].z); s[i].w = fmaf(kr, d.w, s[i].w);
+        __stcs(Sp + (r * kD + col) / 4, s[i]);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_d128(const DecodeParams& p, cudaStream_t stream) {
+    const int64_t units = (int64_t)p.N * p.H;
+    if (units == 0) return cudaSuccess;
+    if (units > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    if (p.bf16)
+        decode_d128_kernel<__nv_bfloat16><<<(unsigned)units, 128, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(p.q), static_cast<const __nv_bfloat16*>(p.k),
+            static_cast<const __nv_bfloat16*>(p.v), p.log_g,
+            static_cast<const __nv_bfloat16*>(p.beta), p.S, static_cast<__nv_bfloat16*>(p.o));
+    else
+        decode_d128_kernel<float><<<(unsigned)units, 128, 0, stream>>>(
+            static_cast<const float*>(p.q), static_cast<const float*>(p.k),
+            static_cast<const float*>(p.v), p.log_g, static_cast<const float*>(p.beta), p.S,
+            static_cast<float*>(p.o));
+    return cudaGetLastError();
+}
+
+}  // namespace kda

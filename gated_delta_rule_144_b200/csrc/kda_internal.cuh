@@ -1,0 +1,67 @@
+// Private declarations shared by the translation units of libkda.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kda {
+
+// Codes the kernels store into the sticky device error word (same values as kda_status_t).
+enum DeviceError : unsigned {
+    DEV_OK = 0,
+    DEV_TIMEOUT = 4,
+    DEV_BAD_SEQLENS = 5,
+    DEV_RANGE = 6,
+};
+
+// The first error sticks; later ones are dropped.
+__device__ __forceinline__ void set_device_error(unsigned* err, unsigned code) {
+    atomicCAS(err, 0u, code);
+}
+
+struct FwdParams {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* log_g;
+    const void* beta;
+    const float* h0;          // nullable
+    const int32_t* cu_seqlens;  // nullable (device)
+    void* o;
+    float* hT;                // nullable
+    int B, T, H, dk, dv, N;
+    bool bf16;
+    unsigned* err;            // device error word
+};
+
+struct DecodeParams {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* log_g;
+    const void* beta;
+    float* S;
+    void* o;
+    int N, H, dk, dv;
+    bool bf16;
+    unsigned* err;
+};
+
+// Launchers (host). Each returns the launch status of its kernel(s).
+cudaError_t launch_recurrent(const FwdParams& p, cudaStream_t stream);
+cudaError_t launch_decode_d128(const DecodeParams& p, cudaStream_t stream);
+cudaError_t launch_chunk64(const FwdParams& p, cudaStream_t stream);
+bool chunk64_available();
+
+// Element loads shared by the CUDA-core kernels.
+__device__ __forceinline__ float load_elem(const float* p, int64_t i) { return p[i]; }
+__device__ __forceinline__ float load_elem(const __nv_bfloat16* p, int64_t i) {
+    return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void store_elem(float* p, int64_t i, float x) { p[i] = x; }
+__device__ __forceinline__ void store_elem(__nv_bfloat16* p, int64_t i, float x) {
+    p[i] = __float2bfloat16_rn(x);
+}
+
+}  // namespace kda

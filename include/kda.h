@@ -1,0 +1,149 @@
+/*
+ * kda.h - C ABI of libkda.so, the B200 (sm_100a) implementation of the Kimi Delta Attention
+ * (KDA) gated delta-rule recurrence used by GLM-5.3's linear_attention layers.
+ *
+ * The operation (GLM-5.3-Flash model card, the Kimi Delta Attention snippet of
+ * Glm5NextTextLinearAttention): every (sequence, head) keeps a state S of shape [dk, dv], row c
+ * being key channel c. For each token t, in order,
+ *
+ *     S      = diag(g_t) S                 g_t = exp(log_g_t), one gate per key channel
+ *     m      = k_t^T S
+ *     delta  = beta_t (v_t - m)
+ *     S      = S + k_t delta^T
+ *     o_t    = S^T q_t                     (read-out after the write; no 1/sqrt(dk) scale)
+ *
+ * Packed variable-length input restarts the state at every document boundary (NeMo AutoModel
+ * glm5_next layers page: `_torch_recurrent_kda(q, k, v, g, beta, cu_seqlens)` "packed
+ * boundaries reset the recurrent state"; `Glm5NextLinearAttention.forward` runs KDA "without
+ * crossing documents"). The gate arrives in log space as float32, as returned by
+ * `Glm5NextKDAFp32Params.forward` ("log-decay gates [batch, sequence, heads, head_dim]").
+ * Decode advances a per-sequence state by one token (metrale glm5next_layer page: KDA decode
+ * takes a KdaSeqState).
+ *
+ * Conventions for every entry point
+ *   - All tensors are dense, contiguous, row-major, in DEVICE memory unless stated otherwise, and
+ *     every base pointer must be 16-byte aligned.
+ *   - The caller owns all memory. The library allocates nothing, keeps no per-call state and is
+ *     safe to call from several host threads on different streams.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default stream).
+ *   - Problems visible on the host (null or misaligned pointers, bad sizes, unsupported
+ *     combinations) return an error before anything is launched. Problems only the device can
+ *     see (malformed cu_seqlens, a pipeline wait that timed out) are recorded in a sticky device
+ *     error word that kda_get_device_error() reports and clears.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* kda_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, negative or inconsistent size       */
+    KDA_ERR_UNSUPPORTED = 2,  /* valid request this build has no kernel for (see kda_fwd)     */
+    KDA_ERR_CUDA = 3,         /* a CUDA runtime call failed; kda_last_error() has the text     */
+    KDA_ERR_TIMEOUT = 4,      /* device: a bounded pipeline wait expired (kernel gave up)      */
+    KDA_ERR_BAD_SEQLENS = 5,  /* device: cu_seqlens not non-decreasing from 0 to T             */
+    KDA_ERR_RANGE = 6         /* device: decay too steep for the chunked path (see kda_fwd)    */
+} kda_status_t;
+
+typedef enum {
+    KDA_F32 = 0,   /* float32 */
+    KDA_BF16 = 1   /* bfloat16 */
+} kda_dtype_t;
+
+/* Algorithm selector for kda_fwd (field `chunk_size`). */
+enum {
+    KDA_CHUNK_AUTO = 0,      /* 64 for bf16 with dk = dv = 128, else the per-token walk */
+    KDA_CHUNK_PER_TOKEN = 1, /* per-token walk: exact fp32 recurrence, any dtype, dk,dv <= 256 */
+    KDA_CHUNK_64 = 64        /* chunked WY/UT form on tcgen05 tensor cores: bf16, dk = dv = 128 */
+};
+
+/*
+ * Problem description for kda_fwd.
+ *   B, T, H, dk, dv : batch, tokens per row, heads, key and value head dims.
+ *   num_seqs        : number of independent sequences N. Without cu_seqlens N must equal B;
+ *                     with cu_seqlens, B must be 1 and N = len(cu_seqlens) - 1.
+ *   dtype           : element type of q, k, v, beta and o. log_g, h0 and hT are always float32.
+ *   chunk_size      : KDA_CHUNK_AUTO, KDA_CHUNK_PER_TOKEN or KDA_CHUNK_64. For float32 inputs
+ *                     any value selects the per-token walk (the exact path).
+ */
+typedef struct {
+    int B, T, H, dk, dv;
+    int num_seqs;
+    kda_dtype_t dtype;
+    int chunk_size;
+} kda_fwd_desc_t;
+
+/*
+ * kda_fwd - prefill: run the recurrence over whole sequences or packed documents.
+ *
+ *   q, k    : [B, T, H, dk]  dtype           v, o : [B, T, H, dv] dtype
+ *   log_g   : [B, T, H, dk]  float32 (log of the per-channel decay; must be <= 0 and finite)
+ *   beta    : [B, T, H]      dtype
+ *   h0      : [N, H, dk, dv] float32, or NULL for a zero initial state
+ *   cu_seqlens : int32 [N + 1], device, or NULL. Offsets into the packed token axis of a B = 1
+ *             row; must start at 0, be non-decreasing and end at T. Empty documents are allowed
+ *             (their final state equals their initial state).
+ *   o       : output, written for every token.
+ *   hT      : [N, H, dk, dv] float32 final state of every sequence/document, or NULL to skip.
+ *   workspace, workspace_bytes : scratch owned by the caller; at least
+ *             kda_fwd_workspace_size(desc) bytes (may be NULL when that is 0).
+ *
+ * The chunked path (KDA_CHUNK_64) computes in bf16 tensor-core products with fp32 accumulation
+ * and an fp32 state. Its within-chunk factorisation needs the summed decay of any 8 consecutive
+ * tokens of a 16-token sub-chunk to stay above -80 nats per key channel (e.g. log_g >= -10
+ * everywhere); otherwise a factor would leave the float32 range. The kernel detects that case,
+ * records KDA_ERR_RANGE in the device error word and still finishes; the per-token path
+ * (KDA_CHUNK_PER_TOKEN) has no such limit.
+ * Returns KDA_OK once the work is enqueued. T = 0 or N = 0 is a valid no-op (hT = h0 or 0).
+ */
+kda_status_t kda_fwd(const kda_fwd_desc_t* desc, const void* q, const void* k, const void* v,
+                     const float* log_g, const void* beta, const float* h0,
+                     const int32_t* cu_seqlens, void* o, float* hT, void* workspace,
+                     size_t workspace_bytes, kda_stream_t stream);
+
+/* Scratch bytes kda_fwd needs for `desc` (0 when it needs none). Host-only, no CUDA calls. */
+size_t kda_fwd_workspace_size(const kda_fwd_desc_t* desc);
+
+/*
+ * kda_decode_step - advance N sequences by one token each, updating the state in place.
+ *
+ *   q, k, log_g : [N, H, dk] (q, k in dtype, log_g float32)    v, o : [N, H, dv] dtype
+ *   beta        : [N, H] dtype
+ *   S_inout     : [N, H, dk, dv] float32, read and overwritten with the new state.
+ *   o           : output [N, H, dv].
+ * S_inout must not alias any other argument. dk, dv <= 256.
+ */
+kda_status_t kda_decode_step(int N, int H, int dk, int dv, kda_dtype_t dtype, const void* q,
+                             const void* k, const void* v, const float* log_g, const void* beta,
+                             float* S_inout, void* o, kda_stream_t stream);
+
+/*
+ * kda_get_device_error - synchronise `stream`, then return and clear the sticky device error
+ * word (KDA_OK, KDA_ERR_BAD_SEQLENS, KDA_ERR_TIMEOUT or KDA_ERR_RANGE), or KDA_ERR_CUDA if
+ * the synchronisation itself failed. The word is per device and shared by all streams.
+ */
+kda_status_t kda_get_device_error(kda_stream_t stream);
+
+/* Static description of a status code. */
+const char* kda_status_string(kda_status_t status);
+
+/* Text of the last error raised on this host thread ("" if none). Valid until the next call. */
+const char* kda_last_error(void);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,119 @@
+"""C-ABI checks that need no GPU: the library loads, exports what include/kda.h declares, and
+rejects bad arguments on the host before any launch.
+
+Every call here fails host-side validation (NULL, misaligned or inconsistent arguments), so these
+tests launch nothing even when a GPU is present; fake pointers are never dereferenced.
+"""
+
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import gated_delta_rule_144_b200 as kda
+from gated_delta_rule_144_b200 import build as kbuild
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+@pytest.fixture(scope="module")
+def L():
+    kbuild.build()
+    return kda.lib()
+
+
+def _declared_functions():
+    text = (ROOT / "include" / "kda.h").read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for must in ("kda_fwd", "kda_decode_step", "kda_get_device_error", "kda_status_string",
+                 "kda_fwd_workspace_size", "kda_last_error", "kda_version"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings_and_version(L):
+    assert L.kda_version() >= 100
+    for code in range(7):
+        assert L.kda_status_string(code)
+    assert L.kda_status_string(99) == b"unknown status"
+
+
+def _desc(**kw):
+    d = dict(B=1, T=64, H=2, dk=128, dv=128, num_seqs=1, dtype=kda.KDA_BF16, chunk_size=0)
+    d.update(kw)
+    return kda.FwdDesc(**d)
+
+
+FAKE = 0x100000  # aligned fake address: only ever passed alongside an argument that fails
+
+
+def _fwd(L, desc, q=FAKE, k=FAKE, v=FAKE, g=FAKE, b=FAKE, h0=None, cu=None, o=FAKE, hT=None):
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    return L.kda_fwd(None if desc is None else ctypes.byref(desc), P(q), P(k), P(v), P(g),
+                     P(b), P(h0), P(cu), P(o), P(hT), None, 0, None)
+
+
+@pytest.mark.parametrize("case", [
+    ("null desc", None, {}),
+    ("negative T", _desc(T=-1), {}),
+    ("zero heads", _desc(H=0), {}),
+    ("N != B without cu_seqlens", _desc(B=2, num_seqs=1), {}),
+    ("cu_seqlens with B > 1", _desc(B=2, num_seqs=2), {"cu": FAKE}),
+    ("bad dtype", _desc(dtype=7), {}),
+    ("null q", _desc(), {"q": None}),
+    ("null beta", _desc(), {"b": None}),
+    ("null o", _desc(), {"o": None}),
+    ("misaligned k", _desc(), {"k": FAKE + 2}),
+    ("misaligned h0", _desc(), {"h0": FAKE + 8}),
+    ("misaligned cu_seqlens", _desc(num_seqs=1), {"cu": FAKE + 4, "q": FAKE + 1}),
+], ids=lambda c: c[0])
+def test_fwd_rejects_on_host(L, case):
+    _, desc, kw = case
+    st = _fwd(L, desc, **kw)
+    assert st == 1, (st, L.kda_last_error())
+    assert L.kda_last_error()
+
+
+def test_fwd_unsupported_combinations(L):
+    # chunked tensor-core path is bf16 with dk = dv = 128 only
+    assert _fwd(L, _desc(dk=64, chunk_size=64), q=None) in (1, 2)
+    assert _fwd(L, _desc(chunk_size=48), q=FAKE + 1) in (1, 2)
+    st = _fwd(L, _desc(dk=64, dv=64, chunk_size=64))
+    assert st == 2
+    st = _fwd(L, _desc(dk=512, dv=64, chunk_size=1))
+    assert st == 2
+
+
+def test_decode_rejects_on_host(L):
+    P = ctypes.c_void_p
+    args = lambda **kw: [kw.get(n, P(FAKE)) for n in ("q", "k", "v", "g", "b", "S", "o")]
+    assert L.kda_decode_step(-1, 1, 128, 128, 1, *args(), None) == 1
+    assert L.kda_decode_step(1, 0, 128, 128, 1, *args(), None) == 1
+    assert L.kda_decode_step(1, 1, 128, 128, 5, *args(), None) == 1
+    assert L.kda_decode_step(1, 1, 512, 128, 1, *args(), None) == 2
+    assert L.kda_decode_step(1, 1, 128, 128, 1, *args(S=None), None) == 1
+    assert L.kda_decode_step(1, 1, 128, 128, 1, *args(o=P(FAKE + 4)), None) == 1
+
+
+def test_workspace_size_is_host_only(L):
+    d = _desc()
+    assert L.kda_fwd_workspace_size(ctypes.byref(d)) >= 0
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 4, 1, 8)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        kda.fwd(q, q, q, q, torch.zeros(1, 4, 1))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        kda.decode_step(q[0], q[0], q[0], q[0], torch.zeros(4, 1), torch.zeros(4, 1, 8, 8))
