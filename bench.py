@@ -1,0 +1,519 @@
+#!/usr/bin/env python
+"""Benchmark: KDA prefill tokens/s (H=32, d=128) and decode GB/s on B200, against the roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload W]
+
+One step = one kda_fwd call (every prefill stage of the hot path: load and gate, decayed
+operands, intra-chunk products, UT transform, WY factors, the chunk-serial state pass,
+document resets and state I/O) over one batch of the headline workload, long-t65536: B=2,
+T=65536, H=32, dk=dv=128, bf16 q/k/v/beta, fp32 log g = -softplus(N(2,1)), fp32 h0 ~ N(0,0.02^2).
+Inputs are resident in HBM and larger than L2 (6.4 GB), so no flush is needed between steps.
+`value` is tokens/s over all ranks (each rank runs its own batch: weak scaling, no collective
+on the data path). The decode step (256 sequences x 32 heads, state in place) and the packed
+8-document prefill are timed in the same run and reported under "secondary".
+
+--impl reference times the float64 CPU oracle (the reference arm for this build) on a bounded
+sample of the same workload on the host cores; under torchrun only rank 0 runs it.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import torch  # noqa: E402
+
+METRIC = "KDA prefill tokens/s (H=32,d=128) & decode GB/s; % of B200 roofline"
+PROFILE_TRAFFIC = ROOT / "profiles" / "traffic.json"
+
+# Algorithmic bytes per token-head at d = 128 (q, k, v bf16; log g fp32; beta bf16; o bf16)
+BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 4 + 2 + 128 * 2
+STATE_BYTES = 128 * 128 * 4
+# Chunked-form flops per token-head at d = 128, C = 64: 10 C d + 6 d^2 (full tiles)
+FLOPS_PER_TOKEN_HEAD = 10 * 64 * 128 + 6 * 128 * 128
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def env_rank():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def measured_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ helpers
+
+KERNEL_SOURCES = {
+    "kda_decode_d128": ["kda_decode.cu", "kda_internal.cuh"],
+    "kda_recurrent": ["kda_recurrent.cu", "kda_internal.cuh"],
+    "kda_chunk64": ["kda_chunk64.cu", "kda_sm100.cuh", "kda_internal.cuh"],
+}
+
+
+def source_digest(kernel: str):
+    """Digest of the sources a kernel is built from (its profile is stale once they change)."""
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES.get(kernel, []):
+        p = ROOT / "gated_delta_rule_144_b200" / "csrc" / name
+        h.update(name.encode())
+        h.update(p.read_bytes() if p.exists() else b"")
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel: str, workload: str):
+    """dram read+write bytes per launch from the committed ncu summary, if it is current."""
+    if not PROFILE_TRAFFIC.exists():
+        return None
+    try:
+        d = json.loads(PROFILE_TRAFFIC.read_text())
+        e = d.get(kernel)
+        if not e or e.get("source_digest") != source_digest(kernel) \
+                or e.get("workload") != workload:
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except (ValueError, KeyError):
+        return None
+
+
+def time_launches(fn, steps, stream):
+    """Per-launch CUDA-event timing on the launching stream. Returns (total_ms, [ms...])."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s, e in ev:
+        s.record(stream)
+        fn()
+        e.record(stream)
+    t1.record(stream)
+    t1.synchronize()
+    return t0.elapsed_time(t1), [s.elapsed_time(e) for s, e in ev]
+
+
+def max_over_ranks(x: float, world: int, device):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int, device):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------------------ our arm
+
+def prefill_bytes(inp) -> int:
+    th = inp["T"] * inp["B"] * inp["H"]
+    states = inp["N"] * inp["H"] * STATE_BYTES
+    return th * BYTES_PER_TOKEN_HEAD + states * (2 if inp["h0"] is not None else 1)
+
+
+def run_ours(args):
+    import gated_delta_rule_144_b200 as kda
+    from gated_delta_rule_144_b200 import synth
+
+    rank, local, world = env_rank()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    stream = torch.cuda.current_stream(dev)
+    wl = synth.WORKLOADS[args.workload]
+
+    # ---- headline: prefill on the workload, one batch per rank
+    inp = synth.prefill_inputs(wl, device=dev, seed=1000 + wl.index + 7919 * rank)
+    B, T, H, dk, dv, N = inp["B"], inp["T"], inp["H"], inp["dk"], inp["dv"], inp["N"]
+    o = torch.empty((B, T, H, dv), dtype=inp["q"].dtype, device=dev)
+    hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+
+    def step():
+        kda.fwd(inp["q"], inp["k"], inp["v"], inp["log_g"], inp["beta"], h0=inp["h0"],
+                cu_seqlens=inp["cu_seqlens"], o=o, hT=hT, chunk_size=args.chunk_size)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if kda.get_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    total_ms, per = time_launches(step, args.steps, stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    if kda.get_device_error() != 0:
+        raise RuntimeError("device error in the timed region")
+
+    ms_max = max_over_ranks(total_ms, world, dev)
+    tokens_rank = B * T
+    tokens_all = sum_over_ranks(float(tokens_rank), world, dev)
+    value = tokens_all * args.steps / (ms_max / 1e3)
+    launch_ms = statistics.fmean(per)
+    hbm_peak, tc_peak, peak_kind = measured_peaks()
+    bytes_launch = prefill_bytes(inp)
+    achieved = bytes_launch / (launch_ms / 1e3) / 1e9
+    algo = kda.fwd_algorithm(B, T, H, dk, dv, N, inp["q"].dtype, args.chunk_size,
+                             varlen=inp["cu_seqlens"] is not None)
+    kernel_name = "kda_chunk64" if algo == kda.CHUNK_64 else "kda_recurrent"
+    traffic = committed_traffic(kernel_name, wl.name)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
+                "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                "traffic": traffic, "peak_kind": peak_kind, "kernel": kernel_name,
+                "algorithmic_bytes_per_launch": bytes_launch,
+                "avg_launch_ms": round(launch_ms, 4),
+                "flops_per_launch": FLOPS_PER_TOKEN_HEAD * B * T * H,
+                "tensor_frac_if_tc": round(FLOPS_PER_TOKEN_HEAD * B * T * H /
+                                           (launch_ms / 1e3) / (tc_peak * 1e12), 4)}
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(kda, inp, args, stream, world, dev)
+
+    secondary = {}
+    if not args.no_secondary:
+        secondary = run_secondary(kda, synth, args, dev, stream, world, rank)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, args)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
+                       "global_batch": B * world, "seq_len": T, "h0": inp["h0"] is not None,
+                       "log_g": "-softplus(N(%g,1))" % wl.decay_mu,
+                       "parallelism": "dp%d" % world, "l2": "inputs larger than L2",
+                       "chunk_size": args.chunk_size, "path": kernel_name},
+            "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
+            "clocks": clk, "cpu_baseline": cpu, "secondary": secondary,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(kda, inp, args, stream, world, dev):
+    """Same metric through kda.fwd with pinned host inputs copied in and o, hT copied out."""
+    keys = ("q", "k", "v", "log_g", "beta", "h0", "cu_seqlens")
+    host = {k: (inp[k].cpu().pin_memory() if inp[k] is not None else None) for k in keys}
+    d_in = {k: (torch.empty_like(inp[k]) if inp[k] is not None else None) for k in keys}
+    B, T, H, dv, N, dk = inp["B"], inp["T"], inp["H"], inp["dv"], inp["N"], inp["dk"]
+    o = torch.empty((B, T, H, dv), dtype=inp["q"].dtype, device=dev)
+    hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hT_h = torch.empty(hT.shape, dtype=hT.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+    d2h = o.numel() * o.element_size() + hT.numel() * hT.element_size()
+
+    def step():
+        for k in keys:
+            if host[k] is not None:
+                d_in[k].copy_(host[k], non_blocking=True)
+        kda.fwd(d_in["q"], d_in["k"], d_in["v"], d_in["log_g"], d_in["beta"], h0=d_in["h0"],
+                cu_seqlens=d_in["cu_seqlens"], o=o, hT=hT, chunk_size=args.chunk_size)
+        o_h.copy_(o, non_blocking=True)
+        hT_h.copy_(hT, non_blocking=True)
+
+    steps = max(1, min(args.steps, args.e2e_steps))
+    step()
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms, _ = time_launches(step, steps, stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(total_ms, world, dev)
+    tokens_all = sum_over_ranks(float(B * T), world, dev)
+    return {"value": round(tokens_all * steps / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 3)}
+
+
+def run_secondary(kda, synth, args, dev, stream, world, rank):
+    out = {}
+    hbm_peak, _, _ = measured_peaks()
+    # decode: 256 sequences x 32 heads, fp32 128x128 state updated in place every step
+    d = synth.decode_inputs("decode-n256", device=dev, seed=1003 + 7919 * rank)
+    od = torch.empty_like(d["v"])
+
+    def dstep():
+        kda.decode_step(d["q"], d["k"], d["v"], d["log_g"], d["beta"], d["S"], o=od)
+
+    for _ in range(max(3, args.warmup)):
+        dstep()
+    torch.cuda.synchronize()
+    barrier(world)
+    steps = max(args.steps, 20)
+    total_ms, per = time_launches(dstep, steps, stream)
+    barrier(world)
+    ms = max_over_ranks(total_ms, world, dev) / steps
+    state = d["S"].numel() * 4
+    io = sum(d[k].numel() * d[k].element_size() for k in ("q", "k", "v", "log_g", "beta"))
+    io += od.numel() * od.element_size()
+    by = 2 * state + io
+    gbs = by / (ms / 1e3) / 1e9
+    out["decode"] = {"workload": "decode-n256", "N": 256, "H": 32, "dk": 128, "dv": 128,
+                     "bytes_per_step": by, "ms_per_step": round(ms, 4),
+                     "GB/s": round(gbs * world, 1), "GB/s_per_gpu": round(gbs, 1),
+                     "roofline_frac": round(gbs / hbm_peak, 4), "peak": hbm_peak,
+                     "kernel": "kda_decode_d128",
+                     "traffic": committed_traffic("kda_decode_d128", "decode-n256")}
+    del d, od
+    # packed 8-document prefill (H = 32)
+    p = synth.prefill_inputs("packed-8docs", device=dev, seed=1002 + 7919 * rank)
+    o = torch.empty_like(p["v"])
+    hT = torch.empty((p["N"], p["H"], 128, 128), dtype=torch.float32, device=dev)
+
+    def pstep():
+        kda.fwd(p["q"], p["k"], p["v"], p["log_g"], p["beta"], cu_seqlens=p["cu_seqlens"],
+                o=o, hT=hT, chunk_size=args.chunk_size)
+
+    for _ in range(max(3, args.warmup)):
+        pstep()
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms, per = time_launches(pstep, args.steps, stream)
+    barrier(world)
+    ms = max_over_ranks(total_ms, world, dev) / args.steps
+    by = prefill_bytes(p)
+    out["packed_prefill"] = {"workload": "packed-8docs", "lengths": p["lengths"],
+                             "tokens": p["T"], "ms_per_step": round(ms, 4),
+                             "tokens/s": round(p["T"] * world / (ms / 1e3), 1),
+                             "roofline_frac": round(by / (ms / 1e3) / 1e9 / hbm_peak, 4)}
+    if kda.get_device_error() != 0:
+        raise RuntimeError("device error in the secondary runs")
+    return out
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+
+def oracle_sample(wl, tokens):
+    """Bounded sample of the workload for the float64 oracle: one sequence, all heads."""
+    from gated_delta_rule_144_b200 import synth
+    inp = synth.prefill_inputs(wl, device="cpu", B=1, T=tokens)
+    f = lambda t: None if t is None else t.float().numpy()
+    return {k: f(inp[k]) for k in ("q", "k", "v", "log_g", "beta", "h0")}, inp
+
+
+def cpu_baseline(wl, args):
+    import oracle
+    tokens = args.cpu_tokens
+    arrays, inp = oracle_sample(wl, tokens)
+    t0 = time.perf_counter()
+    oracle.kda_fwd(arrays["q"], arrays["k"], arrays["v"], arrays["log_g"], arrays["beta"],
+                   h0=arrays["h0"])
+    dt = time.perf_counter() - t0
+    return {"value": round(tokens / dt, 1), "unit": "tokens/s", "cores": oracle.max_threads(),
+            "kind": "oracle",
+            "sample": "one sequence of %s, first %d tokens, all %d heads (%.1f s)" % (
+                wl.name, tokens, inp["H"], dt)}
+
+
+def run_reference(args):
+    rank, _, world = env_rank()
+    if rank != 0:
+        return
+    import oracle
+    from gated_delta_rule_144_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    tokens = args.ref_tokens
+    arrays, inp = oracle_sample(wl, tokens)
+    run = lambda: oracle.kda_fwd(arrays["q"], arrays["k"], arrays["v"], arrays["log_g"],
+                                 arrays["beta"], h0=arrays["h0"])
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = time.perf_counter() - t0
+    value = tokens * args.steps / dt
+    sample = "one sequence of %s, first %d tokens, all %d heads, per step" % (
+        wl.name, tokens, inp["H"])
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 1),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "dk": wl.dk,
+                       "dv": wl.dv, "sample_tokens": tokens},
+            "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s",
+                             "cores": oracle.max_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_profile_case(args):
+    """Warm-up plus K launches of one kernel, no timing: the command the ncu captures run."""
+    import gated_delta_rule_144_b200 as kda
+    from gated_delta_rule_144_b200 import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if args.profile_case == "decode":
+        d = synth.decode_inputs("decode-n256", device=dev)
+        fn = lambda: kda.decode_step(d["q"], d["k"], d["v"], d["log_g"], d["beta"], d["S"])
+    else:
+        name = args.workload if args.profile_case == "prefill" else "packed-8docs"
+        kw = {} if args.profile_tokens <= 0 else {"T": args.profile_tokens}
+        p = synth.prefill_inputs(name, device=dev, **kw)
+        fn = lambda: kda.fwd(p["q"], p["k"], p["v"], p["log_g"], p["beta"], h0=p["h0"],
+                             cu_seqlens=p["cu_seqlens"], chunk_size=args.chunk_size)
+    for _ in range(args.warmup + args.steps):
+        fn()
+    torch.cuda.synchronize()
+    st = kda.get_device_error()
+    print(json.dumps({"profile_case": args.profile_case, "launches": args.warmup + args.steps,
+                      "device_error": st}))
+    if st != 0:
+        sys.exit(1)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[1])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="long-t65536")
+    ap.add_argument("--chunk-size", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-tokens", type=int, default=32768)
+    ap.add_argument("--ref-tokens", type=int, default=4096)
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=["prefill", "decode", "packed"], default=None,
+                    help="run only warm-up + steps launches of one case (for ncu captures)")
+    ap.add_argument("--profile-tokens", type=int, default=0,
+                    help="with --profile-case prefill: tokens per sequence (0 = workload's)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        log("warm-up raised to 3 (minimum)")
+        args.warmup = 3
+    _, _, world = env_rank()
+    if args.gpus != world and world > 1:
+        log("note: --gpus %d but WORLD_SIZE %d; using WORLD_SIZE" % (args.gpus, world))
+    if args.profile_case:
+        run_profile_case(args)
+    elif args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
