@@ -19,7 +19,8 @@ from pathlib import Path
 
 import torch
 
-__all__ = ["fwd", "decode_step", "get_device_error", "fwd_workspace_size", "KdaError",
+__all__ = ["fwd", "decode_step", "get_device_error", "fwd_workspace_size", "fwd_algorithm",
+           "KdaError",
            "library_path", "lib", "CHUNK_AUTO", "CHUNK_PER_TOKEN", "CHUNK_64"]
 
 _PKG = Path(__file__).resolve().parent
@@ -63,6 +64,8 @@ def lib():
     p, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     L.kda_fwd.argtypes = [ctypes.POINTER(FwdDesc), p, p, p, p, p, p, p, p, p, p, sz, p]
     L.kda_fwd.restype = i32
+    L.kda_fwd_algorithm.argtypes = [ctypes.POINTER(FwdDesc), i32]
+    L.kda_fwd_algorithm.restype = i32
     L.kda_fwd_workspace_size.argtypes = [ctypes.POINTER(FwdDesc)]
     L.kda_fwd_workspace_size.restype = sz
     L.kda_decode_step.argtypes = [i32, i32, i32, i32, i32, p, p, p, p, p, p, p, p]
@@ -118,6 +121,17 @@ def _stream(stream, device):
     if stream is None:
         stream = torch.cuda.current_stream(device)
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def fwd_algorithm(B, T, H, dk, dv, num_seqs, dtype=torch.bfloat16, chunk_size=0,
+                  varlen=False) -> int:
+    """Path kda_fwd would take: CHUNK_PER_TOKEN or CHUNK_64 (raises KdaError if rejected)."""
+    d = FwdDesc(B, T, H, dk, dv, num_seqs, KDA_BF16 if dtype == torch.bfloat16 else KDA_F32,
+                chunk_size)
+    r = int(lib().kda_fwd_algorithm(ctypes.byref(d), int(varlen)))
+    if r < 0:
+        _check(-r, "kda_fwd_algorithm")
+    return r
 
 
 def fwd_workspace_size(B, T, H, dk, dv, num_seqs, dtype=torch.bfloat16, chunk_size=0) -> int:

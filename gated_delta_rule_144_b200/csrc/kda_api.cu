@@ -126,6 +126,13 @@ const char* kda_status_string(kda_status_t s) {
     return "unknown status";
 }
 
+int kda_fwd_algorithm(const kda_fwd_desc_t* desc, int has_cu_seqlens) {
+    Path path;
+    const kda_status_t st = check_fwd_desc(desc, has_cu_seqlens != 0, &path);
+    if (st != KDA_OK) return -(int)st;
+    return path == Path::kChunk64 ? KDA_CHUNK_64 : KDA_CHUNK_PER_TOKEN;
+}
+
 size_t kda_fwd_workspace_size(const kda_fwd_desc_t* desc) {
     (void)desc;
     return 0;

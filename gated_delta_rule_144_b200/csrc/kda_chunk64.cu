@@ -1,10 +1,853 @@
-// Chunked prefill on tcgen05 tensor cores (dk = dv = 128, bf16 operands, fp32 state).
+// Chunked KDA prefill on tcgen05 tensor cores: dk = dv = 128, bf16 operands, fp32 state.
+//
+// The recurrence (GLM-5.3-Flash model card, Kimi Delta Attention snippet) is evaluated 64 tokens
+// at a time in the WY / UT-transform form of the decay-weighted delta rule. Per chunk of rows r
+// (one head), with a_t = exp(log_g_t) per key channel and Gamma the within-chunk cumulative log
+// decay:
+//
+//   A_kk[r,i] = sum_c k_rc k_ic e^{Gamma_rc - Gamma_ic}  (i < r)    A_qk: same with q_r, i <= r
+//   T  = (I + diag(beta) A_kk)^-1 diag(beta)                          (UT transform, fp32)
+//   W  = T (k e^{Gamma}),   U~ = T v                                  (WY factors)
+//   Q~ = q e^{Gamma} - A_qk W,   O~ = A_qk U~
+//   U  = U~ - W S,   o = O~ + Q~ S,   S <- diag(e^{Gamma_end}) S + (k e^{Gamma_end-Gamma})^T U
+//
+// which equals the per-token recurrence exactly (tests/chunk_model.py checks the algebra in
+// float64). A_kk and A_qk come from ONE tensor-core product R C^T of separable factors that stay
+// inside the float32 range whatever the chunk's total decay: rows of R are anchored at the middle
+// of their own 16-token block, diagonal-block columns at the middle of theirs, and the columns a
+// later block needs are anchored at that later block's middle (those factors are <= 1).
+//
+// Work split: one CTA per (sequence or document, head, half of the value columns). The value
+// columns of S evolve independently, so each CTA owns S[:, 64 half : 64 half + 64] in TMEM (fp32)
+// for the whole sequence and recomputes the chunk's intra-chunk terms for its half.
+// Packed documents (cu_seqlens) start from their own h0 (or zero) and never share a chunk.
+//
+// Pipeline per chunk (256 threads; thread 0 issues TMA and MMAs):
+//   TMA q, k, log g, v  ->  elementwise decay factors (CUDA cores)  ->  MMA R C^T  ->
+//   assemble A_kk, A_qk  ->  UT solve (fp32, blocked)  ->  MMA T [K+ | V]  ->  MMA A_qk [W | U~]
+//   ->  MMA [W; Q~] S  ->  U, o  ->  MMA S += K_end^T U.
+// The next chunk's TMA overlaps everything after the elementwise pass. Every mbarrier wait is
+// bounded; on expiry the CTA records KDA_ERR_TIMEOUT, drains its own outstanding copies and MMAs,
+// frees TMEM and exits.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstdlib>
+#include <mutex>
+
 #include "kda_internal.cuh"
+#include "kda_sm100.cuh"
 
 namespace kda {
+namespace {
 
-bool chunk64_available() { return false; }
+using namespace sm100;
 
-cudaError_t launch_chunk64(const FwdParams&, cudaStream_t) { return cudaErrorNotSupported; }
+constexpr int kC = 64;        // tokens per chunk
+constexpr int kD = 128;       // dk = dv
+constexpr int kDV = 64;       // value columns per CTA
+constexpr int kSplit = kD / kDV;
+constexpr int kThreads = 256;
+constexpr int kLds = 68;      // row stride (floats) of the fp32 solve buffers
+
+// ---- shared memory map (bytes from a 1024-aligned base)
+constexpr uint32_t OFF_Q = 0;            // q   [64][128] bf16 row-major (TMA)
+constexpr uint32_t OFF_K = 16384;        // k   [64][128] bf16 row-major (TMA)
+constexpr uint32_t OFF_G = 32768;        // log g [64][128] f32 row-major (TMA)
+constexpr uint32_t OFF_V = 65536;        // v   2 x [64][64] bf16, 128B-swizzled (TMA)
+constexpr uint32_t OFF_R = 81920;        // R   [128][128] bf16 (K-major A of R C^T)
+constexpr uint32_t OFF_C = OFF_R + 32768;  // C [160][128] bf16 (K-major B of R C^T)
+//   after R C^T completes, the R/C region is reused:
+constexpr uint32_t OFF_LB = OFF_R;              // L = diag(beta) A_kk, f32 [64][kLds]
+constexpr uint32_t OFF_MB = OFF_R + 17408;      // (I + L)^-1, f32 [64][kLds]
+constexpr uint32_t OFF_YB = OFF_R + 34816;      // solve scratch, f32 3 x [16][17]
+constexpr uint32_t OFF_T = OFF_R + 38912;       // T  [64][64] bf16 (K-major A)
+constexpr uint32_t OFF_AQK = OFF_R + 47104;     // A_qk [64][64] bf16 (K-major A)
+constexpr uint32_t OFF_UT = OFF_R + 55296;      // U~ [64][64] bf16 (MN-major B)
+constexpr uint32_t OFF_S16 = OFF_R;             // S  [128][64] bf16 (MN-major B), state pass
+constexpr uint32_t OFF_U16 = OFF_R + 16384;     // U  [64][64] bf16 (MN-major B), state pass
+constexpr uint32_t OFF_KP = OFF_C + 40960;      // K+ [64][128] bf16 (MN-major B)
+constexpr uint32_t OFF_W = OFF_KP + 16384;      // W  [64][128] bf16 (K-major A / MN-major B)
+constexpr uint32_t OFF_QT = OFF_W + 16384;      // Q+ then Q~ [64][128] bf16 (K-major A)
+constexpr uint32_t OFF_KE = OFF_QT + 16384;     // K_end [64][128] bf16 (MN-major A)
+constexpr uint32_t OFF_MISC = OFF_KE + 16384;
+constexpr uint32_t OFF_BETA = OFF_MISC;         // f32 [64]
+constexpr uint32_t OFF_DECAY = OFF_MISC + 256;  // f32 [128]
+constexpr uint32_t OFF_LOUP = OFF_MISC + 768;   // f32 [4][2][128]
+constexpr uint32_t OFF_BAR = OFF_MISC + 4864;   // 4 mbarriers
+constexpr uint32_t OFF_TMEM = OFF_BAR + 32;     // TMEM base address
+constexpr uint32_t kSmemUsed = OFF_TMEM + 16;
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
+static_assert(OFF_UT + 8192 <= OFF_C + 40960, "solve buffers overflow the R/C region");
+static_assert(OFF_S16 + 16384 <= OFF_T, "state-pass tiles overlap the solve outputs");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+// ---- TMEM columns (fp32, 128 lanes)
+constexpr uint32_t TM_A = 0;     // R C^T          [128 x 160]
+constexpr uint32_t TM_W = 160;   // W (lanes +0) and A_qk W (lanes +16), M=64 layout [64 x 128]
+constexpr uint32_t TM_U = 288;   // U~ (lanes +0) and O~ (lanes +16), M=64 layout [64 x 64]
+constexpr uint32_t TM_B = 352;   // W S (lanes +0) and Q~ S (lanes +16) [64 x 64]
+constexpr uint32_t TM_S = 416;   // state S [128 x 64] fp32
+constexpr uint32_t kTmemCols = 512;
+
+constexpr uint32_t kTxBytes = 16384 + 16384 + 32768 + 8192;
+constexpr uint32_t kLaneHi = 16u << 16;   // second M=64 tile interleaved at lane +16
+
+// row offset, inside C[64:], of the columns row block a needs from earlier blocks
+__device__ __forceinline__ int cross_off(int a) { return a == 1 ? 0 : (a == 2 ? 16 : 48); }
+
+struct ChunkArgs {
+    const __nv_bfloat16* beta;
+    const float* h0;
+    const int32_t* cu;
+    __nv_bfloat16* o;
+    float* hT;
+    int T, H, N;
+    long long budget;
+    int debug_stall;   // failure-injection hook: wait on a barrier nothing ever signals
+    unsigned* err;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(x, y);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+__device__ __forceinline__ void st32(uint8_t* base, uint32_t off, uint32_t v) {
+    *reinterpret_cast<uint32_t*>(base + off) = v;
+}
+__device__ __forceinline__ uint32_t ld32(const uint8_t* base, uint32_t off) {
+    return *reinterpret_cast<const uint32_t*>(base + off);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
+               const ChunkArgs args) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int qd = warp & 3, hf = warp >> 2;
+    const int split = blockIdx.x % kSplit;
+    const int unit = blockIdx.x / kSplit;
+    const int n = unit / args.H, h = unit % args.H;
+    const int dv0 = split * kDV;
+
+    long long t0, t1;
+    if (args.cu) {
+        t0 = args.cu[n];
+        t1 = args.cu[n + 1];
+        const bool bad_ends = (n == 0 && t0 != 0) || (n == args.N - 1 && t1 != args.T);
+        if (t1 < t0 || t0 < 0 || t1 > args.T || bad_ends) {
+            if (tid == 0) set_device_error(args.err, DEV_BAD_SEQLENS);
+            return;
+        }
+    } else {
+        t0 = (long long)n * args.T;
+        t1 = t0 + args.T;
+    }
+    const int nchunks = (int)((t1 - t0 + kC - 1) / kC);
+
+    float* beta_s = reinterpret_cast<float*>(sm + OFF_BETA);
+    float* decay_s = reinterpret_cast<float*>(sm + OFF_DECAY);
+    float* loup_s = reinterpret_cast<float*>(sm + OFF_LOUP);
+    uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
+    const uint32_t bar_tma = sb + OFF_BAR, bar_mma = sb + OFF_BAR + 8, bar_b4 = sb + OFF_BAR + 16;
+    const uint32_t bar_never = sb + OFF_BAR + 24;   // never signalled (failure-injection hook)
+
+    if (tid == 0) {
+        mbar_init(bar_tma, 1);
+        mbar_init(bar_mma, 1);
+        mbar_init(bar_b4, 1);
+        mbar_init(bar_never, 1);
+        fence_mbar_init();
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_g);
+        prefetch_tmap(&tm_v);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_s), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_s;
+    const uint32_t lane_q = (uint32_t)(32 * qd) << 16;   // this warp's TMEM lane quarter
+    const size_t state_base = ((size_t)n * args.H + h) * kD * kD;
+
+    // initial state: TMEM lane c = 32 qd + lane holds S[c][dv0 + 32 hf .. + 32)
+    {
+        float v[32];
+        const int c = 32 * qd + lane;
+        if (args.h0) {
+            const float4* src =
+                reinterpret_cast<const float4*>(args.h0 + state_base + (size_t)c * kD + dv0 + 32 * hf);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 x = src[i];
+                v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        }
+        tmem_st32(tbase + lane_q + TM_S + 32 * hf, v);
+        tmem_st_wait();
+    }
+
+    auto issue_tma = [&](int c) {
+        const int row0 = (int)(t0 + (long long)kC * c);
+        mbar_arrive_expect_tx(bar_tma, kTxBytes);
+        tma_load_3d(sb + OFF_Q, &tm_q, bar_tma, 0, h, row0);
+        tma_load_3d(sb + OFF_K, &tm_k, bar_tma, 0, h, row0);
+        tma_load_3d(sb + OFF_G, &tm_g, bar_tma, 0, h, row0);
+        tma_load_3d(sb + OFF_V + (c & 1) * 8192, &tm_v, bar_tma, dv0, h, row0);
+    };
+
+    bool tma_pending = false, mma_pending = false, b4_pending = false;
+    int tma_chunk = 0;   // chunk whose TMA is in flight when tma_pending
+    int b4_chunk = 0;    // chunk whose state update is in flight when b4_pending
+    uint32_t mma_phase = 0;
+    bool aborted = false;
+    // every thread waits; all agree on the outcome
+    auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
+        const bool ok = mbar_wait(bar, parity, args.budget);
+        return __syncthreads_or(!ok) == 0;
+    };
+
+    if (tid == 0 && nchunks > 0) issue_tma(0);
+    tma_pending = nchunks > 0;
+    // Failure injection (KDA_DEBUG_STALL_WAIT): a wait on a barrier that nothing signals, with a
+    // copy in flight, must expire, report KDA_ERR_TIMEOUT and wind down cleanly.
+    if (args.debug_stall && !wait_all(bar_never, 0)) aborted = true;
+
+    const __nv_bfloat16* qs = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_Q);
+    const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_K);
+    const float* gs = reinterpret_cast<const float*>(sm + OFF_G);
+
+    for (int c = 0; c < nchunks && !aborted; ++c) {
+        const long long row0 = t0 + (long long)kC * c;
+        const int L = (int)min((long long)kC, t1 - row0);
+
+        // ---------------------------------------------------------------- inputs of chunk c
+        if (!wait_all(bar_tma, c & 1)) { aborted = true; break; }
+        tma_pending = false;
+        if (b4_pending) {   // previous chunk's state update still reads U and K_end
+            if (!wait_all(bar_b4, b4_chunk & 1)) { aborted = true; break; }
+            b4_pending = false;
+        }
+        if (tid < kC)
+            beta_s[tid] = tid < L ? __bfloat162float(args.beta[(row0 + tid) * args.H + h]) : 0.f;
+
+        // ---------------------------------------------------------------- decay factors (pass 1)
+        // thread: block b = qd (rows 16b .. 16b+15), key channels ch, ch+1
+        const int b = qd;
+        const int ch = 64 * hf + 2 * lane;
+        float av[16][2], sg[16][2];
+        {
+#pragma unroll
+            for (int lr = 0; lr < 16; ++lr) {
+                const int r = 16 * b + lr;
+                float2 g = *reinterpret_cast<const float2*>(gs + r * kD + ch);
+                if (r >= L) g = make_float2(0.f, 0.f);
+                av[lr][0] = __expf(g.x);
+                av[lr][1] = __expf(g.y);
+            }
+            // exclusive suffix products to the block end (sg) and to row 7 (sfx, rows 0..7)
+            float sfx[8][2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                sg[15][j] = 1.f;
+#pragma unroll
+                for (int lr = 14; lr >= 0; --lr) sg[lr][j] = sg[lr + 1][j] * av[lr + 1][j];
+                sfx[7][j] = 1.f;
+#pragma unroll
+                for (int lr = 6; lr >= 0; --lr) sfx[lr][j] = sfx[lr + 1][j] * av[lr + 1][j];
+            }
+            float lo[2], up[2], pfx[2] = {1.f, 1.f}, pp[2] = {1.f, 1.f};
+            bool range_bad = false;
+#pragma unroll
+            for (int lr = 0; lr < 16; ++lr) {
+                const int r = 16 * b + lr;
+                const float2 kk = unpack_bf16(ld32(reinterpret_cast<const uint8_t*>(ks), (r * kD + ch) * 2));
+                const float2 qq = unpack_bf16(ld32(reinterpret_cast<const uint8_t*>(qs), (r * kD + ch) * 2));
+                const float kx[2] = {r < L ? kk.x : 0.f, r < L ? kk.y : 0.f};
+                const float qx[2] = {qq.x, qq.y};
+                float rho[2], kap[2];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    pp[j] *= av[lr][j];
+                    if (lr == 7) lo[j] = pp[j];
+                    if (lr >= 8) {
+                        pfx[j] = (lr == 8) ? av[8][j] : pfx[j] * av[lr][j];
+                        rho[j] = pfx[j];
+                        kap[j] = __frcp_rn(pfx[j]);
+                        range_bad |= pfx[j] < 1e-30f;
+                    } else {
+                        rho[j] = __frcp_rn(sfx[lr][j]);
+                        kap[j] = sfx[lr][j];
+                        range_bad |= sfx[lr][j] < 1e-30f;
+                    }
+                }
+                st32(sm, OFF_R + sw128_off(128, r, ch), pack_bf16(kx[0] * rho[0], kx[1] * rho[1]));
+                st32(sm, OFF_R + sw128_off(128, 64 + r, ch),
+                     pack_bf16(qx[0] * rho[0], qx[1] * rho[1]));
+                st32(sm, OFF_C + sw128_off(160, r, ch), pack_bf16(kx[0] * kap[0], kx[1] * kap[1]));
+            }
+            up[0] = sg[7][0];
+            up[1] = sg[7][1];
+            if (range_bad) set_device_error(args.err, DEV_RANGE);
+            loup_s[(b * 2 + 0) * kD + ch] = lo[0];
+            loup_s[(b * 2 + 0) * kD + ch + 1] = lo[1];
+            loup_s[(b * 2 + 1) * kD + ch] = up[0];
+            loup_s[(b * 2 + 1) * kD + ch + 1] = up[1];
+        }
+        __syncthreads();
+
+        // block totals P_b = Lo_b Up_b; columns later blocks need; chunk-level factors
+        float Pb[4][2], Lob[4][2];
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                Lob[bb][j] = loup_s[(bb * 2) * kD + ch + j];
+                Pb[bb][j] = Lob[bb][j] * loup_s[(bb * 2 + 1) * kD + ch + j];
+            }
+        float Fb[2], Gb[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            Fb[j] = 1.f;
+            Gb[j] = 1.f;
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                if (bb < b) Fb[j] *= Pb[bb][j];
+                if (bb > b) Gb[j] *= Pb[bb][j];
+            }
+        }
+        if (b == 0) {
+            decay_s[ch] = Pb[0][0] * Pb[1][0] * Pb[2][0] * Pb[3][0];
+            decay_s[ch + 1] = Pb[0][1] * Pb[1][1] * Pb[2][1] * Pb[3][1];
+        }
+        // cross columns: for each later row block a, k_i e^{Gamma_m(a) - Gamma_i}
+#pragma unroll
+        for (int a = 1; a < 4; ++a) {
+            if (a <= b) continue;
+            float X[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                X[j] = Lob[a][j];
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb)
+                    if (bb > b && bb < a) X[j] *= Pb[bb][j];
+            }
+#pragma unroll
+            for (int lr = 0; lr < 16; ++lr) {
+                const int r = 16 * b + lr;
+                const float2 kk = unpack_bf16(ld32(reinterpret_cast<const uint8_t*>(ks), (r * kD + ch) * 2));
+                const float k0 = r < L ? kk.x : 0.f, k1 = r < L ? kk.y : 0.f;
+                st32(sm, OFF_C + sw128_off(160, 64 + cross_off(a) + r, ch),
+                     pack_bf16(k0 * sg[lr][0] * X[0], k1 * sg[lr][1] * X[1]));
+            }
+        }
+        fence_proxy_async();
+        __syncthreads();
+
+        // ---------------------------------------------------------------- MMA: R C^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, 160, 0, 0);
+#pragma unroll
+            for (int s = 0; s < kD / 16; ++s) {
+                const int k0 = 16 * s;
+                const uint64_t ad = sw128_desc(sb + OFF_R + (k0 >> 6) * 16384 + (k0 & 63) * 2, 16, 1024);
+                const uint64_t bd = sw128_desc(sb + OFF_C + (k0 >> 6) * 20480 + (k0 & 63) * 2, 16, 1024);
+                umma_f16(tbase + TM_A, ad, bd, id, s > 0);
+            }
+            umma_commit(bar_mma);
+        }
+        mma_pending = true;
+
+        // ---------------------------------------------------------------- pass 2: K+, Q+, K_end
+        {
+            float pp[2] = {1.f, 1.f};
+#pragma unroll
+            for (int lr = 0; lr < 16; ++lr) {
+                const int r = 16 * b + lr;
+                const float2 kk = unpack_bf16(ld32(reinterpret_cast<const uint8_t*>(ks), (r * kD + ch) * 2));
+                const float2 qq = unpack_bf16(ld32(reinterpret_cast<const uint8_t*>(qs), (r * kD + ch) * 2));
+                const float k0 = r < L ? kk.x : 0.f, k1 = r < L ? kk.y : 0.f;
+                pp[0] *= av[lr][0];
+                pp[1] *= av[lr][1];
+                const float e0 = Fb[0] * pp[0], e1 = Fb[1] * pp[1];
+                st32(sm, OFF_KP + sw128_off(64, r, ch), pack_bf16(k0 * e0, k1 * e1));
+                st32(sm, OFF_QT + sw128_off(64, r, ch), pack_bf16(qq.x * e0, qq.y * e1));
+                st32(sm, OFF_KE + sw128_off(64, r, ch),
+                     pack_bf16(k0 * sg[lr][0] * Gb[0], k1 * sg[lr][1] * Gb[1]));
+            }
+        }
+        fence_proxy_async();
+        __syncthreads();   // q, k, log g of chunk c fully consumed
+        if (tid == 0 && c + 1 < nchunks) issue_tma(c + 1);
+        tma_pending = c + 1 < nchunks;
+        tma_chunk = c + 1;
+
+        // ---------------------------------------------------------------- assemble A_kk, A_qk
+        if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
+        ++mma_phase;
+        mma_pending = false;
+        tc_fence_after();
+        {
+            float* Lb = reinterpret_cast<float*>(sm + OFF_LB);
+            const bool is_q = qd >= 2;
+            const int r = 32 * (qd & 1) + lane;
+            const int a = r >> 4;
+            const float br = beta_s[r];
+            if (hf == 0) {
+                // diagonal block (and zeros for the blocks after it)
+                float v[32];
+                tmem_ld32(tbase + lane_q + TM_A + 32 * (qd & 1), v);
+                tmem_ld_wait();
+                const bool second = (a & 1) != 0;   // this row's block inside the 32 columns
+#pragma unroll
+                for (int j = 0; j < 16; j += 2) {
+                    const int i = 16 * a + j;
+                    float x0 = second ? v[16 + j] : v[j];
+                    float x1 = second ? v[17 + j] : v[j + 1];
+                    if (is_q) {
+                        x0 = (i <= r) ? x0 : 0.f;
+                        x1 = (i + 1 <= r) ? x1 : 0.f;
+                        st32(sm, OFF_AQK + sw128_off(64, r, i), pack_bf16(x0, x1));
+                    } else {
+                        Lb[r * kLds + i] = (i < r) ? br * x0 : 0.f;
+                        Lb[r * kLds + i + 1] = (i + 1 < r) ? br * x1 : 0.f;
+                    }
+                }
+                for (int i = 16 * (a + 1); i < kC; i += 2) {
+                    if (is_q) {
+                        st32(sm, OFF_AQK + sw128_off(64, r, i), 0u);
+                    } else {
+                        Lb[r * kLds + i] = 0.f;
+                        Lb[r * kLds + i + 1] = 0.f;
+                    }
+                }
+            } else {
+                // columns from earlier blocks
+                float v[32];
+                auto put = [&](int i, float x0, float x1) {
+                    if (is_q) {
+                        st32(sm, OFF_AQK + sw128_off(64, r, i), pack_bf16(x0, x1));
+                    } else {
+                        Lb[r * kLds + i] = br * x0;
+                        Lb[r * kLds + i + 1] = br * x1;
+                    }
+                };
+                if ((qd & 1) == 0) {
+                    float w[16];
+                    tmem_ld16(tbase + lane_q + TM_A + 64, w);   // row block 1: i in block 0
+                    tmem_ld_wait();
+                    if (a == 1) {
+#pragma unroll
+                        for (int j = 0; j < 16; j += 2) put(j, w[j], w[j + 1]);
+                    }
+                } else {
+                    tmem_ld32(tbase + lane_q + TM_A + 80, v);   // row block 2: i in 0..31
+                    tmem_ld_wait();
+                    if (a == 2) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2) put(j, v[j], v[j + 1]);
+                    }
+                    tmem_ld32(tbase + lane_q + TM_A + 112, v);  // row block 3: i in 0..31
+                    tmem_ld_wait();
+                    if (a == 3) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2) put(j, v[j], v[j + 1]);
+                    }
+                    float w[16];
+                    tmem_ld16(tbase + lane_q + TM_A + 144, w);  // row block 3: i in 32..47
+                    tmem_ld_wait();
+                    if (a == 3) {
+#pragma unroll
+                        for (int j = 0; j < 16; j += 2) put(32 + j, w[j], w[j + 1]);
+                    }
+                }
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---------------------------------------------------------------- UT solve (fp32)
+        {
+            const float* Lb = reinterpret_cast<const float*>(sm + OFF_LB);
+            float* Mb = reinterpret_cast<float*>(sm + OFF_MB);
+            float* Yb = reinterpret_cast<float*>(sm + OFF_YB);
+            // diagonal 16x16 blocks: forward substitution, one column per thread
+            if (tid < 64) {
+                const int base = 16 * (tid >> 4), j = tid & 15;
+                float acc[16], x[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    x[k] = (k == j) ? 1.f : (k < j ? 0.f : -acc[k]);
+#pragma unroll
+                    for (int i = k + 1; i < 16; ++i)
+                        acc[i] = fmaf(Lb[(base + i) * kLds + base + k], x[k], acc[i]);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) Mb[(base + i) * kLds + base + j] = x[i];
+            }
+            __syncthreads();
+            // off-diagonal blocks by distance d = a - b:
+            //   Y = sum_{kk in blocks b..a-1} L[a-block rows][kk] M[kk][b-block cols],  M_ab = -M_aa Y
+#pragma unroll 1
+            for (int d = 1; d < 4; ++d) {
+                const int npairs = 4 - d;
+                for (int e = tid; e < npairs * 256; e += kThreads) {
+                    const int pi = e >> 8, p = (e >> 4) & 15, qq = e & 15;
+                    const int bb = pi, aa = pi + d;
+                    float s = 0.f;
+                    for (int kk = 16 * bb; kk < 16 * aa; ++kk)
+                        s = fmaf(Lb[(16 * aa + p) * kLds + kk], Mb[kk * kLds + 16 * bb + qq], s);
+                    Yb[(pi * 16 + p) * 17 + qq] = s;
+                }
+                __syncthreads();
+                for (int e = tid; e < npairs * 256; e += kThreads) {
+                    const int pi = e >> 8, p = (e >> 4) & 15, qq = e & 15;
+                    const int bb = pi, aa = pi + d;
+                    float s = 0.f;
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        s = fmaf(Mb[(16 * aa + p) * kLds + 16 * aa + k], Yb[(pi * 16 + k) * 17 + qq], s);
+                    Mb[(16 * aa + p) * kLds + 16 * bb + qq] = -s;
+                }
+                __syncthreads();
+            }
+            // T = M diag(beta), lower triangle, bf16 K-major
+            {
+                const int r = tid >> 2, seg = tid & 3;
+#pragma unroll
+                for (int j = 0; j < 16; j += 2) {
+                    const int i = 16 * seg + j;
+                    const float x0 = (i <= r) ? Mb[r * kLds + i] * beta_s[i] : 0.f;
+                    const float x1 = (i + 1 <= r) ? Mb[r * kLds + i + 1] * beta_s[i + 1] : 0.f;
+                    st32(sm, OFF_T + sw128_off(64, r, i), pack_bf16(x0, x1));
+                }
+            }
+        }
+        fence_proxy_async();
+        __syncthreads();
+
+        // ---------------------------------------------------------------- MMA: W = T K+, U~ = T V
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t idw = idesc_bf16(64, 128, 0, 1), idu = idesc_bf16(64, 64, 0, 1);
+#pragma unroll
+            for (int s = 0; s < kC / 16; ++s) {
+                const uint64_t ad = sw128_desc(sb + OFF_T + 32 * s, 16, 1024);
+                const uint64_t bw = sw128_desc(sb + OFF_KP + 2048 * s, 8192, 1024);
+                const uint64_t bu = sw128_desc(sb + OFF_V + (c & 1) * 8192 + 2048 * s, 8192, 1024);
+                umma_f16(tbase + TM_W, ad, bw, idw, s > 0);
+                umma_f16(tbase + TM_U, ad, bu, idu, s > 0);
+            }
+            umma_commit(bar_mma);
+        }
+        mma_pending = true;
+        if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
+        ++mma_phase;
+        mma_pending = false;
+        tc_fence_after();
+        {
+            // lanes 0..15 of each quarter hold rows r = 16 qd + lane of the M=64 results
+            float v[32];
+            const int r = 16 * qd + (lane & 15);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const int c0 = 64 * hf + 32 * part;
+                tmem_ld32(tbase + lane_q + TM_W + c0, v);
+                tmem_ld_wait();
+                if (lane < 16) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2)
+                        st32(sm, OFF_W + sw128_off(64, r, c0 + j), pack_bf16(v[j], v[j + 1]));
+                }
+            }
+            tmem_ld32(tbase + lane_q + TM_U + 32 * hf, v);
+            tmem_ld_wait();
+            if (lane < 16) {
+#pragma unroll
+                for (int j = 0; j < 32; j += 2)
+                    st32(sm, OFF_UT + sw128_off(64, r, 32 * hf + j), pack_bf16(v[j], v[j + 1]));
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---------------------------------------------------------------- MMA: A_qk W, A_qk U~
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t idw = idesc_bf16(64, 128, 0, 1), idu = idesc_bf16(64, 64, 0, 1);
+#pragma unroll
+            for (int s = 0; s < kC / 16; ++s) {
+                const uint64_t ad = sw128_desc(sb + OFF_AQK + 32 * s, 16, 1024);
+                const uint64_t bw = sw128_desc(sb + OFF_W + 2048 * s, 8192, 1024);
+                const uint64_t bu = sw128_desc(sb + OFF_UT + 2048 * s, 8192, 1024);
+                umma_f16(tbase + TM_W + kLaneHi, ad, bw, idw, s > 0);
+                umma_f16(tbase + TM_U + kLaneHi, ad, bu, idu, s > 0);
+            }
+            umma_commit(bar_mma);
+        }
+        mma_pending = true;
+        if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
+        ++mma_phase;
+        mma_pending = false;
+        tc_fence_after();
+        {
+            // lanes 16..31 hold rows r = 16 qd + lane - 16 of A_qk W: Q~ = Q+ - A_qk W
+            float v[32];
+            const int r = 16 * qd + (lane & 15);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const int c0 = 64 * hf + 32 * part;
+                tmem_ld32(tbase + lane_q + TM_W + c0, v);
+                tmem_ld_wait();
+                if (lane >= 16) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        const uint32_t off = OFF_QT + sw128_off(64, r, c0 + j);
+                        const float2 qp = unpack_bf16(ld32(sm, off));
+                        st32(sm, off, pack_bf16(qp.x - v[j], qp.y - v[j + 1]));
+                    }
+                }
+            }
+        }
+        // ---------------------------------------------------------------- state pass
+        {
+            // S (fp32, TMEM) -> bf16 operand; then decay the TMEM copy for the update
+            float v[32];
+            const int cc = 32 * qd + lane;
+            tmem_ld32(tbase + lane_q + TM_S + 32 * hf, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; j += 2)
+                st32(sm, OFF_S16 + sw128_off(128, cc, 32 * hf + j), pack_bf16(v[j], v[j + 1]));
+            const float dcy = decay_s[cc];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= dcy;
+            tmem_st32(tbase + lane_q + TM_S + 32 * hf, v);
+            tmem_st_wait();
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(64, 64, 0, 1);
+#pragma unroll
+            for (int s = 0; s < kD / 16; ++s) {
+                const int k0 = 16 * s;
+                const uint64_t aw = sw128_desc(sb + OFF_W + (k0 >> 6) * 8192 + (k0 & 63) * 2, 16, 1024);
+                const uint64_t aq = sw128_desc(sb + OFF_QT + (k0 >> 6) * 8192 + (k0 & 63) * 2, 16, 1024);
+                const uint64_t bs = sw128_desc(sb + OFF_S16 + 2048 * s, 16384, 1024);
+                umma_f16(tbase + TM_B, aw, bs, id, s > 0);
+                umma_f16(tbase + TM_B + kLaneHi, aq, bs, id, s > 0);
+            }
+            umma_commit(bar_mma);
+        }
+        mma_pending = true;
+        if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
+        ++mma_phase;
+        mma_pending = false;
+        tc_fence_after();
+        {
+            float ws[32], ut[32];
+            const int r = 16 * qd + (lane & 15);
+            tmem_ld32(tbase + lane_q + TM_B + 32 * hf, ws);
+            tmem_ld32(tbase + lane_q + TM_U + 32 * hf, ut);
+            tmem_ld_wait();
+            if (lane < 16) {
+                // U = U~ - W S
+#pragma unroll
+                for (int j = 0; j < 32; j += 2)
+                    st32(sm, OFF_U16 + sw128_off(64, r, 32 * hf + j),
+                         pack_bf16(ut[j] - ws[j], ut[j + 1] - ws[j + 1]));
+            } else if (r < L) {
+                // o = O~ + Q~ S
+                uint4* dst = reinterpret_cast<uint4*>(
+                    args.o + ((size_t)(row0 + r) * args.H + h) * kD + dv0 + 32 * hf);
+#pragma unroll
+                for (int j = 0; j < 32; j += 8) {
+                    uint4 u;
+                    u.x = pack_bf16(ut[j] + ws[j], ut[j + 1] + ws[j + 1]);
+                    u.y = pack_bf16(ut[j + 2] + ws[j + 2], ut[j + 3] + ws[j + 3]);
+                    u.z = pack_bf16(ut[j + 4] + ws[j + 4], ut[j + 5] + ws[j + 5]);
+                    u.w = pack_bf16(ut[j + 6] + ws[j + 6], ut[j + 7] + ws[j + 7]);
+                    dst[j / 8] = u;
+                }
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, 64, 1, 1);
+#pragma unroll
+            for (int s = 0; s < kC / 16; ++s) {
+                const uint64_t ae = sw128_desc(sb + OFF_KE + 2048 * s, 8192, 1024);
+                const uint64_t bu = sw128_desc(sb + OFF_U16 + 2048 * s, 8192, 1024);
+                umma_f16(tbase + TM_S, ae, bu, id, 1);
+            }
+            umma_commit(bar_b4);
+        }
+        b4_pending = true;
+        b4_chunk = c;
+    }
+
+    if (aborted) {
+        if (tid == 0) set_device_error(args.err, DEV_TIMEOUT);
+        // wind down: let this CTA's own copies and MMAs finish before TMEM and smem go away
+        const long long drain = 1ll << 31;
+        if (tma_pending) mbar_wait(bar_tma, tma_chunk & 1, drain);
+        if (mma_pending) mbar_wait(bar_mma, mma_phase & 1, drain);
+        if (b4_pending) mbar_wait(bar_b4, b4_chunk & 1, drain);
+        __syncthreads();
+    } else {
+        if (b4_pending) {
+            if (!wait_all(bar_b4, b4_chunk & 1)) {
+                if (tid == 0) set_device_error(args.err, DEV_TIMEOUT);
+                mbar_wait(bar_b4, b4_chunk & 1, 1ll << 31);
+            }
+        }
+        tc_fence_after();
+        if (args.hT) {
+            float v[32];
+            const int cc = 32 * qd + lane;
+            tmem_ld32(tbase + lane_q + TM_S + 32 * hf, v);
+            tmem_ld_wait();
+            float4* dst = reinterpret_cast<float4*>(args.hT + state_base + (size_t)cc * kD + dv0 + 32 * hf);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, kTmemCols);
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+bool g_attr_set = false;
+std::mutex g_attr_mu;
+
+cudaError_t get_encoder() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode ? cudaSuccess : cudaErrorNotSupported;
+}
+
+// [rows, H, 128] row-major tensor, one head's 64-row tile per box
+cudaError_t make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
+                     int rows, int H, int box_inner, CUtensorMapSwizzle sw) {
+    const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)rows};
+    const cuuint64_t strides[2] = {(cuuint64_t)kD * elem_bytes, (cuuint64_t)H * kD * elem_bytes};
+    const cuuint32_t box[3] = {(cuuint32_t)box_inner, 1, (cuuint32_t)kC};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = g_encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+int debug_stall() {
+    static int v = [] {
+        const char* s = std::getenv("KDA_DEBUG_STALL_WAIT");
+        return (s && *s && *s != '0') ? 1 : 0;
+    }();
+    return v;
+}
+
+long long wait_budget() {
+    static long long budget = [] {
+        const char* s = std::getenv("KDA_DEBUG_WAIT_CYCLES");
+        if (s && *s) {
+            const long long v = std::atoll(s);
+            if (v > 0) return v;
+        }
+        return 1ll << 31;   // about one second of SM clock
+    }();
+    return budget;
+}
+
+}  // namespace
+
+// Compiled in for sm_100a. Availability of the driver's tensor-map encoder is checked at launch
+// (a missing encoder surfaces as a CUDA error there), so path selection stays host-only.
+bool chunk64_available() { return true; }
+
+cudaError_t launch_chunk64(const FwdParams& p, cudaStream_t stream) {
+    cudaError_t e = get_encoder();
+    if (e != cudaSuccess) return e;
+    const int rows = p.B * p.T;
+    const int units = p.N * p.H;
+    if (units == 0) return cudaSuccess;
+    if (rows <= 0) {
+        // no tokens: hT = h0 (or zero); the per-token launcher handles it without TMA
+        return launch_recurrent(p, stream);
+    }
+    CUtensorMap mq, mk, mg, mv;
+    if ((e = make_map(&mq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, kD,
+                      CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
+        (e = make_map(&mk, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, kD,
+                      CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
+        (e = make_map(&mg, p.log_g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, p.H, kD,
+                      CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
+        (e = make_map(&mv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, kDV,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
+        return e;
+    {
+        std::lock_guard<std::mutex> lock(g_attr_mu);
+        if (!g_attr_set) {
+            e = cudaFuncSetAttribute(chunk64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kSmemBytes);
+            if (e != cudaSuccess) return e;
+            g_attr_set = true;
+        }
+    }
+    ChunkArgs a;
+    a.beta = static_cast<const __nv_bfloat16*>(p.beta);
+    a.h0 = p.h0;
+    a.cu = p.cu_seqlens;
+    a.o = static_cast<__nv_bfloat16*>(p.o);
+    a.hT = p.hT;
+    a.T = p.T;
+    a.H = p.H;
+    a.N = p.N;
+    a.budget = wait_budget();
+    a.debug_stall = debug_stall();
+    a.err = p.err;
+    const long long grid = (long long)units * kSplit;
+    if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    chunk64_kernel<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(mq, mk, mg, mv, a);
+    return cudaGetLastError();
+}
 
 }  // namespace kda

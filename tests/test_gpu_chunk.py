@@ -1,0 +1,149 @@
+"""GPU parity of the chunked tcgen05 prefill (bf16, dk = dv = 128) against the float64 oracle.
+
+Sizes escalate from one chunk to the full workloads. Metric: relative L2 over all elements of o
+and of the final states, bound 5e-3 (bf16 inputs).
+"""
+
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_144_b200 as kda
+import oracle
+from gated_delta_rule_144_b200 import synth
+from kda_testutil import TOL_BF16, host, oracle_fwd, rel_l2, require_cuda, to
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    require_cuda()
+    yield
+
+
+def _run(inp, chunk_size=64):
+    g = to(inp, DEV)
+    o, hT = kda.fwd(g["q"], g["k"], g["v"], g["log_g"], g["beta"], h0=g.get("h0"),
+                    cu_seqlens=g.get("cu_seqlens"), chunk_size=chunk_size)
+    torch.cuda.synchronize()
+    st = kda.get_device_error()
+    return o, hT, st
+
+
+def _check(inp, tol=TOL_BF16):
+    o, hT, st = _run(inp)
+    assert st == 0, "device error %d" % st
+    o_ref, h_ref = oracle_fwd(inp)
+    eo, eh = rel_l2(host(o), o_ref), rel_l2(host(hT), h_ref)
+    print("rel-L2 o %.3e hT %.3e" % (eo, eh))
+    assert eo <= tol and eh <= tol, (eo, eh)
+    return eo, eh
+
+
+def test_chunk_path_is_selected():
+    assert kda.fwd_algorithm(1, 64, 1, 128, 128, 1) == kda.CHUNK_64
+
+
+def test_one_full_chunk():
+    _check(synth.prefill_inputs("prefill-t4096", T=64, H=1, seed=11))
+
+
+def test_partial_chunks_batch_and_h0():
+    _check(synth.prefill_inputs("prefill-t4096", B=2, T=200, H=3, h0_std=0.1, seed=12))
+
+
+@pytest.mark.parametrize("T", [1, 63, 65, 127, 129, 333])
+def test_ragged_lengths(T):
+    _check(synth.prefill_inputs("long-t65536", B=1, T=T, H=2, seed=13 + T))
+
+
+def test_prefill_t4096_h16_full():
+    """The T=4096, H=16 bf16 workload at full size."""
+    _check(synth.prefill_inputs("prefill-t4096"))
+
+
+def test_packed_edge_documents():
+    lengths = [1, 63, 64, 65, 0, 130, 7, 200]
+    _check(synth.prefill_inputs("packed-8docs", lengths=lengths, H=4, h0_std=0.05, seed=14))
+
+
+def test_packed_8docs_full():
+    """The packed 8-document workload (H = 32) at full size, every token and state."""
+    _check(synth.prefill_inputs("packed-8docs"))
+
+
+def test_chunked_equals_per_token_path():
+    inp = synth.prefill_inputs("packed-8docs", lengths=[300, 17, 129], H=8, h0_std=0.02,
+                               seed=15)
+    o1, h1, st1 = _run(inp, 64)
+    o2, h2, st2 = _run(inp, 1)
+    assert st1 == 0 and st2 == 0
+    assert rel_l2(host(o1), host(o2)) <= TOL_BF16
+    assert rel_l2(host(h1), host(h2)) <= TOL_BF16
+
+
+@pytest.mark.parametrize("name", ["long-t65536", "long-t65536-slow"])
+def test_long_context_full_size_sampled_heads(name):
+    """B=2, T=65536, H=32 with h0: the GPU runs the whole batch; the oracle recomputes four
+    (sequence, head) chains end to end (every token's output and the final state)."""
+    inp = synth.prefill_inputs(name, device=DEV)
+    o, hT, st = _run(inp)
+    assert st == 0
+    picks = [(0, 0), (0, 31), (1, 7), (1, 20)]
+    f = lambda t: t.float().cpu().numpy()
+    worst = (0.0, 0.0)
+    for n, h in picks:
+        sl = lambda t: f(t[n:n + 1, :, h:h + 1])
+        o_ref, h_ref = oracle.kda_fwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]),
+                                      sl(inp["log_g"]), f(inp["beta"][n:n + 1, :, h:h + 1]),
+                                      h0=f(inp["h0"][n:n + 1, h:h + 1]))
+        eo = rel_l2(f(o[n:n + 1, :, h:h + 1]), o_ref)
+        eh = rel_l2(f(hT[n:n + 1, h:h + 1]), h_ref)
+        worst = (max(worst[0], eo), max(worst[1], eh))
+    print("worst rel-L2 o %.3e hT %.3e" % worst)
+    assert worst[0] <= TOL_BF16 and worst[1] <= TOL_BF16, worst
+
+
+def test_steep_decay_is_reported_as_range_error():
+    """log g = -30 per token leaves the chunk factorisation's float32 range: KDA_ERR_RANGE."""
+    inp = synth.prefill_inputs("prefill-t4096", T=64, H=1, seed=16)
+    inp["log_g"] = torch.full_like(inp["log_g"], -30.0)
+    _, _, st = _run(inp)
+    assert st == 6
+    # the per-token path has no such limit
+    o, hT, st = _run(inp, chunk_size=1)
+    assert st == 0
+    o_ref, h_ref = oracle_fwd(inp)
+    assert rel_l2(host(o), o_ref) <= TOL_BF16
+
+
+def test_expired_wait_reports_timeout_and_context_survives():
+    """Failure injection: with KDA_DEBUG_STALL_WAIT set, every CTA waits (bounded by a 2M-cycle
+    budget, about a millisecond) on a barrier that nothing signals while its first copy is in
+    flight. The kernel must report KDA_ERR_TIMEOUT, drain its own copy, free TMEM and return;
+    the context must stay usable. Runs in a child process: the hooks are read once per process."""
+    code = (
+        "import torch, gated_delta_rule_144_b200 as kda\n"
+        "from gated_delta_rule_144_b200 import synth\n"
+        "inp = synth.prefill_inputs('prefill-t4096', T=512, H=2, device='cuda:0')\n"
+        "kda.fwd(inp['q'], inp['k'], inp['v'], inp['log_g'], inp['beta'], chunk_size=64)\n"
+        "st = kda.get_device_error()\n"
+        "o, hT = kda.fwd(inp['q'], inp['k'], inp['v'], inp['log_g'], inp['beta'], chunk_size=1)\n"
+        "torch.cuda.synchronize()\n"
+        "print('STATUS', st, int(kda.get_device_error()))\n")
+    env = dict(os.environ, KDA_DEBUG_WAIT_CYCLES="2000000", KDA_DEBUG_STALL_WAIT="1")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], env=env, cwd=root, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = [x for x in r.stdout.splitlines() if x.startswith("STATUS")][-1]
+    st, after = map(int, line.split()[1:])
+    assert st == 4
+    assert after == 0        # the context stays usable: the exact path runs clean afterwards
