@@ -49,53 +49,60 @@ constexpr int kD = 128;       // dk = dv
 constexpr int kDV = 64;       // value columns per CTA
 constexpr int kSplit = kD / kDV;
 constexpr int kThreads = 256;
-constexpr int kLds = 68;      // row stride (floats) of the fp32 solve buffers
 
 // ---- shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_Q = 0;            // q   [64][128] bf16 row-major (TMA)
 constexpr uint32_t OFF_K = 16384;        // k   [64][128] bf16 row-major (TMA)
 constexpr uint32_t OFF_G = 32768;        // log g [64][128] f32 row-major (TMA)
-constexpr uint32_t OFF_V = 65536;        // v   2 x [64][64] bf16, 128B-swizzled (TMA)
-constexpr uint32_t OFF_R = 81920;        // R   [128][128] bf16 (K-major A of R C^T)
+constexpr uint32_t OFF_V = 65536;        // v   2 x [64][32] bf16, 64B-swizzled halves (TMA)
+constexpr uint32_t OFF_R = 73728;        // R   [128][128] bf16 (K-major A of R C^T)
 constexpr uint32_t OFF_C = OFF_R + 32768;  // C [160][128] bf16 (K-major B of R C^T)
 //   after R C^T completes, the R/C region is reused:
-constexpr uint32_t OFF_LB = OFF_R;              // L = diag(beta) A_kk, f32 [64][kLds]
-constexpr uint32_t OFF_MB = OFF_R + 17408;      // (I + L)^-1, f32 [64][kLds]
-constexpr uint32_t OFF_YB = OFF_R + 34816;      // solve scratch, f32 3 x [16][17]
-constexpr uint32_t OFF_T = OFF_R + 38912;       // T  [64][64] bf16 (K-major A)
-constexpr uint32_t OFF_AQK = OFF_R + 47104;     // A_qk [64][64] bf16 (K-major A)
-constexpr uint32_t OFF_UT = OFF_R + 55296;      // U~ [64][64] bf16 (MN-major B)
-constexpr uint32_t OFF_S16 = OFF_R;             // S  [128][64] bf16 (MN-major B), state pass
-constexpr uint32_t OFF_U16 = OFF_R + 16384;     // U  [64][64] bf16 (MN-major B), state pass
-constexpr uint32_t OFF_KP = OFF_C + 40960;      // K+ [64][128] bf16 (MN-major B)
+constexpr uint32_t OFF_LB = OFF_R;              // L = diag(beta) A_kk, f32 [64][kLdl]
+constexpr uint32_t OFF_MB = OFF_R + 17408;      // (I + L)^-1, f32 [64][kLdm]
+constexpr uint32_t OFF_YS = OFF_R + 35840;      // per-warp 16x16 scratch of the solve
+constexpr uint32_t OFF_T = OFF_R + 39936;       // T  [64][64] bf16 (K-major A)
+constexpr uint32_t OFF_UT = OFF_R + 48128;      // U~ 2 x [64][32] bf16 (MN-major B halves)
+constexpr uint32_t OFF_S16 = OFF_R;             // S  2 x [128][32] bf16 (MN-major B halves)
+constexpr uint32_t OFF_U16 = OFF_R + 16384;     // U  [64][64] bf16 (MN-major B)
+constexpr uint32_t OFF_AQK = OFF_C + 40960;     // A_qk [64][64] bf16 (K-major A), own region
+constexpr uint32_t OFF_KP = OFF_AQK + 8192;     // K+ [64][128] bf16 (MN-major B)
 constexpr uint32_t OFF_W = OFF_KP + 16384;      // W  [64][128] bf16 (K-major A / MN-major B)
 constexpr uint32_t OFF_QT = OFF_W + 16384;      // Q+ then Q~ [64][128] bf16 (K-major A)
 constexpr uint32_t OFF_KE = OFF_QT + 16384;     // K_end [64][128] bf16 (MN-major A)
 constexpr uint32_t OFF_MISC = OFF_KE + 16384;
 constexpr uint32_t OFF_BETA = OFF_MISC;         // f32 [64]
 constexpr uint32_t OFF_DECAY = OFF_MISC + 256;  // f32 [128]
-constexpr uint32_t OFF_LOUP = OFF_MISC + 768;   // f32 [4][2][128]
-constexpr uint32_t OFF_BAR = OFF_MISC + 4864;   // 4 mbarriers
-constexpr uint32_t OFF_TMEM = OFF_BAR + 32;     // TMEM base address
+constexpr uint32_t OFF_LOUP = OFF_MISC + 768;   // f32 [4 blocks][2 halves][128]
+constexpr uint32_t OFF_BAR = OFF_MISC + 4864;   // 5 mbarriers
+constexpr uint32_t OFF_TMEM = OFF_BAR + 64;     // TMEM base address
 constexpr uint32_t kSmemUsed = OFF_TMEM + 16;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
+constexpr int kLdl = 68;   // row stride (floats) of L: conflict-free A-fragment loads
+constexpr int kLdm = 72;   // row stride (floats) of M: conflict-free B-fragment loads
 static_assert(OFF_UT + 8192 <= OFF_C + 40960, "solve buffers overflow the R/C region");
-static_assert(OFF_S16 + 16384 <= OFF_T, "state-pass tiles overlap the solve outputs");
+static_assert(OFF_U16 + 8192 <= OFF_T, "state-pass tiles overlap the solve outputs");
+static_assert(OFF_YS + 3 * 16 * 17 * 4 <= OFF_T, "solve scratch overlaps T");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-// ---- TMEM columns (fp32, 128 lanes)
+// ---- TMEM columns (fp32, 128 lanes). M=64 results use lanes {0-15, 32-47, ...} ("lo") and
+// the interleaved {16-31, 48-63, ...} ("hi"); every M=64 product is split in two along N so
+// that both lane halves of every warp carry data.
 constexpr uint32_t TM_A = 0;     // R C^T          [128 x 160]
-constexpr uint32_t TM_W = 160;   // W (lanes +0) and A_qk W (lanes +16), M=64 layout [64 x 128]
-constexpr uint32_t TM_U = 288;   // U~ (lanes +0) and O~ (lanes +16), M=64 layout [64 x 64]
-constexpr uint32_t TM_B = 352;   // W S (lanes +0) and Q~ S (lanes +16) [64 x 64]
+constexpr uint32_t TM_W = 160;   // W: cols 0-63 lo, 64-127 hi                     (64 cols)
+constexpr uint32_t TM_U = 224;   // U~: value cols 0-31 lo, 32-63 hi                (32 cols)
+constexpr uint32_t TM_W2 = 256;  // A_qk W, same split as W                         (64 cols)
+constexpr uint32_t TM_U2 = 320;  // O~ = A_qk U~, same split as U~                  (32 cols)
+constexpr uint32_t TM_B = 352;   // W S (+0) and Q~ S (+32), split as U~            (64 cols)
 constexpr uint32_t TM_S = 416;   // state S [128 x 64] fp32
 constexpr uint32_t kTmemCols = 512;
 
-constexpr uint32_t kTxBytes = 16384 + 16384 + 32768 + 8192;
+constexpr uint32_t kTxIn = 16384 + 16384 + 32768;
+constexpr uint32_t kTxV = 8192;
 constexpr uint32_t kLaneHi = 16u << 16;   // second M=64 tile interleaved at lane +16
 
 // row offset, inside C[64:], of the columns row block a needs from earlier blocks
-__device__ __forceinline__ int cross_off(int a) { return a == 1 ? 0 : (a == 2 ? 16 : 48); }
+__host__ __device__ constexpr int cross_off(int a) { return a == 1 ? 0 : (a == 2 ? 16 : 48); }
 
 struct ChunkArgs {
     const __nv_bfloat16* beta;
@@ -116,12 +123,20 @@ __device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
     return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
 }
-__device__ __forceinline__ void st32(uint8_t* base, uint32_t off, uint32_t v) {
-    *reinterpret_cast<uint32_t*>(base + off) = v;
+__device__ __forceinline__ float4 ld_bf16x4(const uint8_t* p) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y);
+    return make_float4(a.x, a.y, b.x, b.y);
 }
-__device__ __forceinline__ uint32_t ld32(const uint8_t* base, uint32_t off) {
-    return *reinterpret_cast<const uint32_t*>(base + off);
+__device__ __forceinline__ void st_bf16x4(uint8_t* p, float a, float b, float c, float d) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16(a, b), pack_bf16(c, d));
 }
+// 8 consecutive fp32 values -> one 16-byte chunk of bf16
+__device__ __forceinline__ void st_bf16x8(uint8_t* p, const float* v) {
+    *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                              pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+}
+__device__ __forceinline__ uint32_t f2tf(float x) { return __float_as_uint(x); }
 
 __global__ void __launch_bounds__(kThreads, 1)
 chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -132,7 +147,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                              ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int qd = warp & 3, hf = warp >> 2;
+    const int qd = warp & 3, hf = warp >> 2;          // TMEM lane quarter, column half
     const int split = blockIdx.x % kSplit;
     const int unit = blockIdx.x / kSplit;
     const int n = unit / args.H, h = unit % args.H;
@@ -157,11 +172,12 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     float* decay_s = reinterpret_cast<float*>(sm + OFF_DECAY);
     float* loup_s = reinterpret_cast<float*>(sm + OFF_LOUP);
     uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
-    const uint32_t bar_tma = sb + OFF_BAR, bar_mma = sb + OFF_BAR + 8, bar_b4 = sb + OFF_BAR + 16;
-    const uint32_t bar_never = sb + OFF_BAR + 24;   // never signalled (failure-injection hook)
+    const uint32_t bar_in = sb + OFF_BAR, bar_v = bar_in + 8, bar_mma = bar_in + 16;
+    const uint32_t bar_b4 = bar_in + 24, bar_never = bar_in + 32;
 
     if (tid == 0) {
-        mbar_init(bar_tma, 1);
+        mbar_init(bar_in, 1);
+        mbar_init(bar_v, 1);
         mbar_init(bar_mma, 1);
         mbar_init(bar_b4, 1);
         mbar_init(bar_never, 1);
@@ -175,6 +191,10 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tmem_alloc(smem_u32(tmem_s), kTmemCols);
         tmem_relinquish();
     }
+    // A_qk lives in its own region: its strictly-upper blocks are zeroed once and never written
+    reinterpret_cast<uint4*>(sm + OFF_AQK)[tid] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4*>(sm + OFF_AQK)[tid + kThreads] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -187,8 +207,8 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         float v[32];
         const int c = 32 * qd + lane;
         if (args.h0) {
-            const float4* src =
-                reinterpret_cast<const float4*>(args.h0 + state_base + (size_t)c * kD + dv0 + 32 * hf);
+            const float4* src = reinterpret_cast<const float4*>(args.h0 + state_base +
+                                                                (size_t)c * kD + dv0 + 32 * hf);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const float4 x = src[i];
@@ -202,160 +222,181 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tmem_st_wait();
     }
 
-    auto issue_tma = [&](int c) {
+    auto issue_in = [&](int c) {
         const int row0 = (int)(t0 + (long long)kC * c);
-        mbar_arrive_expect_tx(bar_tma, kTxBytes);
-        tma_load_3d(sb + OFF_Q, &tm_q, bar_tma, 0, h, row0);
-        tma_load_3d(sb + OFF_K, &tm_k, bar_tma, 0, h, row0);
-        tma_load_3d(sb + OFF_G, &tm_g, bar_tma, 0, h, row0);
-        tma_load_3d(sb + OFF_V + (c & 1) * 8192, &tm_v, bar_tma, dv0, h, row0);
+        mbar_arrive_expect_tx(bar_in, kTxIn);
+        tma_load_3d(sb + OFF_Q, &tm_q, bar_in, 0, h, row0);
+        tma_load_3d(sb + OFF_K, &tm_k, bar_in, 0, h, row0);
+        tma_load_3d(sb + OFF_G, &tm_g, bar_in, 0, h, row0);
+    };
+    auto issue_v = [&](int c) {
+        const int row0 = (int)(t0 + (long long)kC * c);
+        mbar_arrive_expect_tx(bar_v, kTxV);
+        tma_load_3d(sb + OFF_V, &tm_v, bar_v, dv0, h, row0);
+        tma_load_3d(sb + OFF_V + 4096, &tm_v, bar_v, dv0 + 32, h, row0);
     };
 
-    bool tma_pending = false, mma_pending = false, b4_pending = false;
-    int tma_chunk = 0;   // chunk whose TMA is in flight when tma_pending
-    int b4_chunk = 0;    // chunk whose state update is in flight when b4_pending
+    // outstanding asynchronous work, drained before exit if a wait expires
+    bool in_pending = false, v_pending = false, mma_pending = false, b4_pending = false;
+    int in_chunk = 0, v_chunk = 0, b4_chunk = 0;
     uint32_t mma_phase = 0;
     bool aborted = false;
-    // every thread waits; all agree on the outcome
     auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
         const bool ok = mbar_wait(bar, parity, args.budget);
-        return __syncthreads_or(!ok) == 0;
+        return __syncthreads_or(!ok) == 0;   // every thread agrees on the outcome
     };
 
-    if (tid == 0 && nchunks > 0) issue_tma(0);
-    tma_pending = nchunks > 0;
-    // Failure injection (KDA_DEBUG_STALL_WAIT): a wait on a barrier that nothing signals, with a
-    // copy in flight, must expire, report KDA_ERR_TIMEOUT and wind down cleanly.
+    if (nchunks > 0) {
+        if (tid == 0) {
+            issue_in(0);
+            issue_v(0);
+        }
+        in_pending = v_pending = true;
+    }
+    // Failure injection (KDA_DEBUG_STALL_WAIT): a wait on a barrier that nothing signals, with
+    // copies in flight, must expire, report KDA_ERR_TIMEOUT and wind down cleanly.
     if (args.debug_stall && !wait_all(bar_never, 0)) aborted = true;
 
-    const __nv_bfloat16* qs = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_Q);
-    const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_K);
+    const uint8_t* qs = sm + OFF_Q;
+    const uint8_t* ks = sm + OFF_K;
     const float* gs = reinterpret_cast<const float*>(sm + OFF_G);
+
+    // elementwise thread mapping: 16-row block pb, half hh (rows 0-7 / 8-15), channels ch0..+3
+    const int pb = warp >> 1, hh = warp & 1;
+    const int ch0 = 4 * lane;
+    const int rbase = 16 * pb + 8 * hh;
+    const uint32_t lh4 = (uint32_t)(((lane & 15) >> 1) << 4);   // 16-byte chunk within a row
+    const uint32_t lo8 = (uint32_t)((lane & 1) * 8);
+    // byte offset of (row 8*rb8 + j, channels ch0..ch0+3) in a 128-column tile of R rows
+    auto toff = [&](int R, int rb8, int j) -> uint32_t {
+        return (uint32_t)((lane >> 4) * R * 128 + rb8 * 1024 + j * 128) + (lh4 ^ (uint32_t)(j << 4)) +
+               lo8;
+    };
 
     for (int c = 0; c < nchunks && !aborted; ++c) {
         const long long row0 = t0 + (long long)kC * c;
         const int L = (int)min((long long)kC, t1 - row0);
 
         // ---------------------------------------------------------------- inputs of chunk c
-        if (!wait_all(bar_tma, c & 1)) { aborted = true; break; }
-        tma_pending = false;
-        if (b4_pending) {   // previous chunk's state update still reads U and K_end
+        if (!wait_all(bar_in, c & 1)) { aborted = true; break; }
+        in_pending = false;
+        if (b4_pending) {   // the previous state update still reads U and K_end
             if (!wait_all(bar_b4, b4_chunk & 1)) { aborted = true; break; }
             b4_pending = false;
         }
         if (tid < kC)
             beta_s[tid] = tid < L ? __bfloat162float(args.beta[(row0 + tid) * args.H + h]) : 0.f;
 
-        // ---------------------------------------------------------------- decay factors (pass 1)
-        // thread: block b = qd (rows 16b .. 16b+15), key channels ch, ch+1
-        const int b = qd;
-        const int ch = 64 * hf + 2 * lane;
-        float av[16][2], sg[16][2];
+        // ---------------------------------------------------------------- decay products
+        float pre[8][4], suf[8][4];
+        bool range_bad = false;
         {
+            float a[8][4];
 #pragma unroll
-            for (int lr = 0; lr < 16; ++lr) {
-                const int r = 16 * b + lr;
-                float2 g = *reinterpret_cast<const float2*>(gs + r * kD + ch);
-                if (r >= L) g = make_float2(0.f, 0.f);
-                av[lr][0] = __expf(g.x);
-                av[lr][1] = __expf(g.y);
+            for (int j = 0; j < 8; ++j) {
+                const int r = rbase + j;
+                const float4 g = *reinterpret_cast<const float4*>(gs + r * kD + ch0);
+                const bool ok = r < L;
+                a[j][0] = ok ? __expf(g.x) : 1.f;
+                a[j][1] = ok ? __expf(g.y) : 1.f;
+                a[j][2] = ok ? __expf(g.z) : 1.f;
+                a[j][3] = ok ? __expf(g.w) : 1.f;
             }
-            // exclusive suffix products to the block end (sg) and to row 7 (sfx, rows 0..7)
-            float sfx[8][2];
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                sg[15][j] = 1.f;
+            for (int i = 0; i < 4; ++i) {
+                float run = 1.f;
 #pragma unroll
-                for (int lr = 14; lr >= 0; --lr) sg[lr][j] = sg[lr + 1][j] * av[lr + 1][j];
-                sfx[7][j] = 1.f;
-#pragma unroll
-                for (int lr = 6; lr >= 0; --lr) sfx[lr][j] = sfx[lr + 1][j] * av[lr + 1][j];
-            }
-            float lo[2], up[2], pfx[2] = {1.f, 1.f}, pp[2] = {1.f, 1.f};
-            bool range_bad = false;
-#pragma unroll
-            for (int lr = 0; lr < 16; ++lr) {
-                const int r = 16 * b + lr;
-                const float2 kk = unpack_bf16(ld32(reinterpret_cast<const uint8_t*>(ks), (r * kD + ch) * 2));
-                const float2 qq = unpack_bf16(ld32(reinterpret_cast<const uint8_t*>(qs), (r * kD + ch) * 2));
-                const float kx[2] = {r < L ? kk.x : 0.f, r < L ? kk.y : 0.f};
-                const float qx[2] = {qq.x, qq.y};
-                float rho[2], kap[2];
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    pp[j] *= av[lr][j];
-                    if (lr == 7) lo[j] = pp[j];
-                    if (lr >= 8) {
-                        pfx[j] = (lr == 8) ? av[8][j] : pfx[j] * av[lr][j];
-                        rho[j] = pfx[j];
-                        kap[j] = __frcp_rn(pfx[j]);
-                        range_bad |= pfx[j] < 1e-30f;
-                    } else {
-                        rho[j] = __frcp_rn(sfx[lr][j]);
-                        kap[j] = sfx[lr][j];
-                        range_bad |= sfx[lr][j] < 1e-30f;
-                    }
+                for (int j = 0; j < 8; ++j) {
+                    run *= a[j][i];
+                    pre[j][i] = run;          // prod_{t <= j} within this half block
                 }
-                st32(sm, OFF_R + sw128_off(128, r, ch), pack_bf16(kx[0] * rho[0], kx[1] * rho[1]));
-                st32(sm, OFF_R + sw128_off(128, 64 + r, ch),
-                     pack_bf16(qx[0] * rho[0], qx[1] * rho[1]));
-                st32(sm, OFF_C + sw128_off(160, r, ch), pack_bf16(kx[0] * kap[0], kx[1] * kap[1]));
+                suf[7][i] = 1.f;
+#pragma unroll
+                for (int j = 6; j >= 0; --j) suf[j][i] = suf[j + 1][i] * a[j + 1][i];
             }
-            up[0] = sg[7][0];
-            up[1] = sg[7][1];
-            if (range_bad) set_device_error(args.err, DEV_RANGE);
-            loup_s[(b * 2 + 0) * kD + ch] = lo[0];
-            loup_s[(b * 2 + 0) * kD + ch + 1] = lo[1];
-            loup_s[(b * 2 + 1) * kD + ch] = up[0];
-            loup_s[(b * 2 + 1) * kD + ch + 1] = up[1];
+            *reinterpret_cast<float4*>(loup_s + (pb * 2 + hh) * kD + ch0) =
+                make_float4(pre[7][0], pre[7][1], pre[7][2], pre[7][3]);
         }
         __syncthreads();
-
-        // block totals P_b = Lo_b Up_b; columns later blocks need; chunk-level factors
-        float Pb[4][2], Lob[4][2];
+        // half totals of every block: Lo_b (rows 0-7), Up_b (rows 8-15), P_b = Lo_b Up_b.
+        // F = prod_{b < pb} P_b, G = prod_{b > pb} P_b; XA[a] = Lo_a prod_{pb < b < a} P_b is the
+        // factor that carries a column of this block to the middle of a later block a.
+        float F[4], G[4], own[4], XA[3][4];   // own: Up_pb (lower half) or Lo_pb (upper half)
+        {
+            float dec[4];
 #pragma unroll
-        for (int bb = 0; bb < 4; ++bb)
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                Lob[bb][j] = loup_s[(bb * 2) * kD + ch + j];
-                Pb[bb][j] = Lob[bb][j] * loup_s[(bb * 2 + 1) * kD + ch + j];
+            for (int i = 0; i < 4; ++i) {
+                F[i] = 1.f;
+                G[i] = 1.f;
+                dec[i] = 1.f;
+                XA[0][i] = XA[1][i] = XA[2][i] = 0.f;
             }
-        float Fb[2], Gb[2];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            Fb[j] = 1.f;
-            Gb[j] = 1.f;
+            float between[4] = {1.f, 1.f, 1.f, 1.f};
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb) {
-                if (bb < b) Fb[j] *= Pb[bb][j];
-                if (bb > b) Gb[j] *= Pb[bb][j];
+                const float4 lo4 = *reinterpret_cast<const float4*>(loup_s + (bb * 2) * kD + ch0);
+                const float4 up4 = *reinterpret_cast<const float4*>(loup_s + (bb * 2 + 1) * kD + ch0);
+                const float lo[4] = {lo4.x, lo4.y, lo4.z, lo4.w};
+                const float up[4] = {up4.x, up4.y, up4.z, up4.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float Pb = lo[i] * up[i];
+                    dec[i] *= Pb;
+                    if (bb < pb) F[i] *= Pb;
+                    if (bb > pb) {
+                        G[i] *= Pb;
+                        if (bb >= 1) XA[bb - 1][i] = lo[i] * between[i];
+                        between[i] *= Pb;
+                    }
+                    if (bb == pb) own[i] = hh == 0 ? up[i] : lo[i];
+                }
+            }
+            if (pb == 0 && hh == 0)
+                *reinterpret_cast<float4*>(decay_s + ch0) = make_float4(dec[0], dec[1], dec[2], dec[3]);
+        }
+
+        // ---------------------------------------------------------------- R and C operands
+        //   rho_r = e^{Gamma_r - Gamma_m}, kappa_r = e^{Gamma_m - Gamma_r} (m: block middle)
+        //   sigma_r = e^{Gamma_end(b) - Gamma_r}, cross columns k sigma X_a, X_a <= 1
+        const int rb8 = 2 * pb + hh;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int r = rbase + j;
+            float4 k4 = ld_bf16x4(ks + (r * kD + ch0) * 2);
+            const float4 q4 = ld_bf16x4(qs + (r * kD + ch0) * 2);
+            if (r >= L) k4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            const float kk[4] = {k4.x, k4.y, k4.z, k4.w}, qq[4] = {q4.x, q4.y, q4.z, q4.w};
+            float rho[4], kap[4], sig[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (hh == 0) {
+                    rho[i] = __fdividef(1.f, suf[j][i]);
+                    kap[i] = suf[j][i];
+                    sig[i] = suf[j][i] * own[i];
+                    range_bad |= suf[j][i] < 1e-30f;
+                } else {
+                    rho[i] = pre[j][i];
+                    kap[i] = __fdividef(1.f, pre[j][i]);
+                    sig[i] = suf[j][i];
+                    range_bad |= pre[j][i] < 1e-30f;
+                }
+            }
+            st_bf16x4(sm + OFF_R + toff(128, rb8, j), kk[0] * rho[0], kk[1] * rho[1],
+                      kk[2] * rho[2], kk[3] * rho[3]);
+            st_bf16x4(sm + OFF_R + toff(128, rb8 + 8, j), qq[0] * rho[0], qq[1] * rho[1],
+                      qq[2] * rho[2], qq[3] * rho[3]);
+            st_bf16x4(sm + OFF_C + toff(160, rb8, j), kk[0] * kap[0], kk[1] * kap[1],
+                      kk[2] * kap[2], kk[3] * kap[3]);
+#pragma unroll
+            for (int a = 1; a < 4; ++a) {
+                if (a <= pb) continue;
+                const float* xa = XA[a - 1];
+                st_bf16x4(sm + OFF_C + toff(160, rb8 + 8 + cross_off(a) / 8, j),
+                          kk[0] * sig[0] * xa[0], kk[1] * sig[1] * xa[1], kk[2] * sig[2] * xa[2],
+                          kk[3] * sig[3] * xa[3]);
             }
         }
-        if (b == 0) {
-            decay_s[ch] = Pb[0][0] * Pb[1][0] * Pb[2][0] * Pb[3][0];
-            decay_s[ch + 1] = Pb[0][1] * Pb[1][1] * Pb[2][1] * Pb[3][1];
-        }
-        // cross columns: for each later row block a, k_i e^{Gamma_m(a) - Gamma_i}
-#pragma unroll
-        for (int a = 1; a < 4; ++a) {
-            if (a <= b) continue;
-            float X[2];
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                X[j] = Lob[a][j];
-#pragma unroll
-                for (int bb = 0; bb < 4; ++bb)
-                    if (bb > b && bb < a) X[j] *= Pb[bb][j];
-            }
-#pragma unroll
-            for (int lr = 0; lr < 16; ++lr) {
-                const int r = 16 * b + lr;
-                const float2 kk = unpack_bf16(ld32(reinterpret_cast<const uint8_t*>(ks), (r * kD + ch) * 2));
-                const float k0 = r < L ? kk.x : 0.f, k1 = r < L ? kk.y : 0.f;
-                st32(sm, OFF_C + sw128_off(160, 64 + cross_off(a) + r, ch),
-                     pack_bf16(k0 * sg[lr][0] * X[0], k1 * sg[lr][1] * X[1]));
-            }
-        }
+        if (range_bad) set_device_error(args.err, DEV_RANGE);
         fence_proxy_async();
         __syncthreads();
 
@@ -366,37 +407,42 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
             for (int s = 0; s < kD / 16; ++s) {
                 const int k0 = 16 * s;
-                const uint64_t ad = sw128_desc(sb + OFF_R + (k0 >> 6) * 16384 + (k0 & 63) * 2, 16, 1024);
-                const uint64_t bd = sw128_desc(sb + OFF_C + (k0 >> 6) * 20480 + (k0 & 63) * 2, 16, 1024);
+                const uint64_t ad =
+                    sw128_desc(sb + OFF_R + (k0 >> 6) * 16384 + (k0 & 63) * 2, 16, 1024);
+                const uint64_t bd =
+                    sw128_desc(sb + OFF_C + (k0 >> 6) * 20480 + (k0 & 63) * 2, 16, 1024);
                 umma_f16(tbase + TM_A, ad, bd, id, s > 0);
             }
             umma_commit(bar_mma);
         }
         mma_pending = true;
 
-        // ---------------------------------------------------------------- pass 2: K+, Q+, K_end
-        {
-            float pp[2] = {1.f, 1.f};
+        // ---------------------------------------------------------------- K+, Q+, K_end
+        //   K+ = k e^{Gamma}, Q+ = q e^{Gamma}, K_end = k e^{Gamma_end - Gamma}
 #pragma unroll
-            for (int lr = 0; lr < 16; ++lr) {
-                const int r = 16 * b + lr;
-                const float2 kk = unpack_bf16(ld32(reinterpret_cast<const uint8_t*>(ks), (r * kD + ch) * 2));
-                const float2 qq = unpack_bf16(ld32(reinterpret_cast<const uint8_t*>(qs), (r * kD + ch) * 2));
-                const float k0 = r < L ? kk.x : 0.f, k1 = r < L ? kk.y : 0.f;
-                pp[0] *= av[lr][0];
-                pp[1] *= av[lr][1];
-                const float e0 = Fb[0] * pp[0], e1 = Fb[1] * pp[1];
-                st32(sm, OFF_KP + sw128_off(64, r, ch), pack_bf16(k0 * e0, k1 * e1));
-                st32(sm, OFF_QT + sw128_off(64, r, ch), pack_bf16(qq.x * e0, qq.y * e1));
-                st32(sm, OFF_KE + sw128_off(64, r, ch),
-                     pack_bf16(k0 * sg[lr][0] * Gb[0], k1 * sg[lr][1] * Gb[1]));
+        for (int j = 0; j < 8; ++j) {
+            const int r = rbase + j;
+            float4 k4 = ld_bf16x4(ks + (r * kD + ch0) * 2);
+            const float4 q4 = ld_bf16x4(qs + (r * kD + ch0) * 2);
+            if (r >= L) k4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            float e[4], x[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                e[i] = F[i] * (hh == 0 ? pre[j][i] : own[i] * pre[j][i]);
+                x[i] = G[i] * (hh == 0 ? suf[j][i] * own[i] : suf[j][i]);
             }
+            const uint32_t o64 = toff(64, rb8, j);
+            st_bf16x4(sm + OFF_KP + o64, k4.x * e[0], k4.y * e[1], k4.z * e[2], k4.w * e[3]);
+            st_bf16x4(sm + OFF_QT + o64, q4.x * e[0], q4.y * e[1], q4.z * e[2], q4.w * e[3]);
+            st_bf16x4(sm + OFF_KE + o64, k4.x * x[0], k4.y * x[1], k4.z * x[2], k4.w * x[3]);
         }
         fence_proxy_async();
         __syncthreads();   // q, k, log g of chunk c fully consumed
-        if (tid == 0 && c + 1 < nchunks) issue_tma(c + 1);
-        tma_pending = c + 1 < nchunks;
-        tma_chunk = c + 1;
+        if (c + 1 < nchunks) {
+            if (tid == 0) issue_in(c + 1);
+            in_pending = true;
+            in_chunk = c + 1;
+        }
 
         // ---------------------------------------------------------------- assemble A_kk, A_qk
         if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
@@ -409,86 +455,66 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int r = 32 * (qd & 1) + lane;
             const int a = r >> 4;
             const float br = beta_s[r];
+            // write 16 consecutive entries (i0 .. i0+15) of row r
+            auto put16 = [&](int i0, const float* x) {
+                if (is_q) {
+                    st_bf16x8(sm + OFF_AQK + sw128_off(64, r, i0), x);
+                    st_bf16x8(sm + OFF_AQK + sw128_off(64, r, i0 + 8), x + 8);
+                } else {
+                    float4* dst = reinterpret_cast<float4*>(Lb + r * kLdl + i0);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m)
+                        dst[m] = make_float4(br * x[4 * m], br * x[4 * m + 1], br * x[4 * m + 2],
+                                             br * x[4 * m + 3]);
+                }
+            };
             if (hf == 0) {
-                // diagonal block (and zeros for the blocks after it)
+                // this row's diagonal block, masked to i < r (A_kk) or i <= r (A_qk)
                 float v[32];
                 tmem_ld32(tbase + lane_q + TM_A + 32 * (qd & 1), v);
                 tmem_ld_wait();
-                const bool second = (a & 1) != 0;   // this row's block inside the 32 columns
+                float x[16];
 #pragma unroll
-                for (int j = 0; j < 16; j += 2) {
+                for (int j = 0; j < 16; ++j) {
                     const int i = 16 * a + j;
-                    float x0 = second ? v[16 + j] : v[j];
-                    float x1 = second ? v[17 + j] : v[j + 1];
-                    if (is_q) {
-                        x0 = (i <= r) ? x0 : 0.f;
-                        x1 = (i + 1 <= r) ? x1 : 0.f;
-                        st32(sm, OFF_AQK + sw128_off(64, r, i), pack_bf16(x0, x1));
-                    } else {
-                        Lb[r * kLds + i] = (i < r) ? br * x0 : 0.f;
-                        Lb[r * kLds + i + 1] = (i + 1 < r) ? br * x1 : 0.f;
-                    }
+                    const float val = (a & 1) ? v[16 + j] : v[j];
+                    x[j] = (is_q ? i <= r : i < r) ? val : 0.f;
                 }
-                for (int i = 16 * (a + 1); i < kC; i += 2) {
-                    if (is_q) {
-                        st32(sm, OFF_AQK + sw128_off(64, r, i), 0u);
-                    } else {
-                        Lb[r * kLds + i] = 0.f;
-                        Lb[r * kLds + i + 1] = 0.f;
-                    }
-                }
+                put16(16 * a, x);
+            } else if ((qd & 1) == 0) {
+                float w[16];
+                tmem_ld16(tbase + lane_q + TM_A + 64 + cross_off(1), w);   // block 1: i in 0..15
+                tmem_ld_wait();
+                if (a == 1) put16(0, w);
             } else {
-                // columns from earlier blocks
                 float v[32];
-                auto put = [&](int i, float x0, float x1) {
-                    if (is_q) {
-                        st32(sm, OFF_AQK + sw128_off(64, r, i), pack_bf16(x0, x1));
-                    } else {
-                        Lb[r * kLds + i] = br * x0;
-                        Lb[r * kLds + i + 1] = br * x1;
-                    }
-                };
-                if ((qd & 1) == 0) {
-                    float w[16];
-                    tmem_ld16(tbase + lane_q + TM_A + 64, w);   // row block 1: i in block 0
-                    tmem_ld_wait();
-                    if (a == 1) {
-#pragma unroll
-                        for (int j = 0; j < 16; j += 2) put(j, w[j], w[j + 1]);
-                    }
-                } else {
-                    tmem_ld32(tbase + lane_q + TM_A + 80, v);   // row block 2: i in 0..31
-                    tmem_ld_wait();
-                    if (a == 2) {
-#pragma unroll
-                        for (int j = 0; j < 32; j += 2) put(j, v[j], v[j + 1]);
-                    }
-                    tmem_ld32(tbase + lane_q + TM_A + 112, v);  // row block 3: i in 0..31
-                    tmem_ld_wait();
-                    if (a == 3) {
-#pragma unroll
-                        for (int j = 0; j < 32; j += 2) put(j, v[j], v[j + 1]);
-                    }
-                    float w[16];
-                    tmem_ld16(tbase + lane_q + TM_A + 144, w);  // row block 3: i in 32..47
-                    tmem_ld_wait();
-                    if (a == 3) {
-#pragma unroll
-                        for (int j = 0; j < 16; j += 2) put(32 + j, w[j], w[j + 1]);
-                    }
+                tmem_ld32(tbase + lane_q + TM_A + 64 + cross_off(2), v);   // block 2: i in 0..31
+                tmem_ld_wait();
+                if (a == 2) {
+                    put16(0, v);
+                    put16(16, v + 16);
                 }
+                tmem_ld32(tbase + lane_q + TM_A + 64 + cross_off(3), v);   // block 3: i in 0..31
+                tmem_ld_wait();
+                if (a == 3) {
+                    put16(0, v);
+                    put16(16, v + 16);
+                }
+                float w[16];
+                tmem_ld16(tbase + lane_q + TM_A + 64 + cross_off(3) + 32, w);   // i in 32..47
+                tmem_ld_wait();
+                if (a == 3) put16(32, w);
             }
         }
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
 
-        // ---------------------------------------------------------------- UT solve (fp32)
+        // ---------------------------------------------------------------- UT transform
         {
             const float* Lb = reinterpret_cast<const float*>(sm + OFF_LB);
             float* Mb = reinterpret_cast<float*>(sm + OFF_MB);
-            float* Yb = reinterpret_cast<float*>(sm + OFF_YB);
-            // diagonal 16x16 blocks: forward substitution, one column per thread
+            // diagonal 16x16 blocks of (I + L)^-1: forward substitution, one column per thread
             if (tid < 64) {
                 const int base = 16 * (tid >> 4), j = tid & 15;
                 float acc[16], x[16];
@@ -499,63 +525,99 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     x[k] = (k == j) ? 1.f : (k < j ? 0.f : -acc[k]);
 #pragma unroll
                     for (int i = k + 1; i < 16; ++i)
-                        acc[i] = fmaf(Lb[(base + i) * kLds + base + k], x[k], acc[i]);
+                        acc[i] = fmaf(Lb[(base + i) * kLdl + base + k], x[k], acc[i]);
                 }
 #pragma unroll
-                for (int i = 0; i < 16; ++i) Mb[(base + i) * kLds + base + j] = x[i];
+                for (int i = 0; i < 16; ++i) Mb[(base + i) * kLdm + base + j] = x[i];
             }
             __syncthreads();
-            // off-diagonal blocks by distance d = a - b:
-            //   Y = sum_{kk in blocks b..a-1} L[a-block rows][kk] M[kk][b-block cols],  M_ab = -M_aa Y
+            // off-diagonal blocks, by distance d = a - b, one warp per block (tf32 mma.sync):
+            //   Y = sum_{kk in blocks b..a-1} L[a-block rows][kk] M[kk][b-block cols]
+            //   M_ab = -M_aa Y
+            const int g = lane >> 2, t = lane & 3;
+            float* ys = reinterpret_cast<float*>(sm + OFF_YS) + warp * 16 * 17;
 #pragma unroll 1
             for (int d = 1; d < 4; ++d) {
-                const int npairs = 4 - d;
-                for (int e = tid; e < npairs * 256; e += kThreads) {
-                    const int pi = e >> 8, p = (e >> 4) & 15, qq = e & 15;
-                    const int bb = pi, aa = pi + d;
-                    float s = 0.f;
-                    for (int kk = 16 * bb; kk < 16 * aa; ++kk)
-                        s = fmaf(Lb[(16 * aa + p) * kLds + kk], Mb[kk * kLds + 16 * bb + qq], s);
-                    Yb[(pi * 16 + p) * 17 + qq] = s;
-                }
-                __syncthreads();
-                for (int e = tid; e < npairs * 256; e += kThreads) {
-                    const int pi = e >> 8, p = (e >> 4) & 15, qq = e & 15;
-                    const int bb = pi, aa = pi + d;
-                    float s = 0.f;
+                if (warp < 4 - d) {
+                    const int bb = warp, aa = warp + d;
+                    float y[2][4] = {};
+                    for (int kk = 16 * bb; kk < 16 * aa; kk += 8) {
+                        const float* la = Lb + (16 * aa + g) * kLdl + kk + t;
+                        const uint32_t A[4] = {f2tf(la[0]), f2tf(la[8 * kLdl]), f2tf(la[4]),
+                                               f2tf(la[8 * kLdl + 4])};
 #pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        s = fmaf(Mb[(16 * aa + p) * kLds + 16 * aa + k], Yb[(pi * 16 + k) * 17 + qq], s);
-                    Mb[(16 * aa + p) * kLds + 16 * bb + qq] = -s;
+                        for (int nt = 0; nt < 2; ++nt) {
+                            const float* mb = Mb + (kk + t) * kLdm + 16 * bb + 8 * nt + g;
+                            const uint32_t B[2] = {f2tf(mb[0]), f2tf(mb[4 * kLdm])};
+                            mma_tf32_16x8x8(y[nt], A, B);
+                        }
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        ys[g * 17 + 8 * nt + 2 * t] = y[nt][0];
+                        ys[g * 17 + 8 * nt + 2 * t + 1] = y[nt][1];
+                        ys[(g + 8) * 17 + 8 * nt + 2 * t] = y[nt][2];
+                        ys[(g + 8) * 17 + 8 * nt + 2 * t + 1] = y[nt][3];
+                    }
+                    __syncwarp();
+                    float z[2][4] = {};
+#pragma unroll
+                    for (int ks2 = 0; ks2 < 2; ++ks2) {
+                        const float* ma = Mb + (16 * aa + g) * kLdm + 16 * aa + 8 * ks2 + t;
+                        const uint32_t A[4] = {f2tf(ma[0]), f2tf(ma[8 * kLdm]), f2tf(ma[4]),
+                                               f2tf(ma[8 * kLdm + 4])};
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt) {
+                            const uint32_t B[2] = {f2tf(ys[(8 * ks2 + t) * 17 + 8 * nt + g]),
+                                                   f2tf(ys[(8 * ks2 + t + 4) * 17 + 8 * nt + g])};
+                            mma_tf32_16x8x8(z[nt], A, B);
+                        }
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        float* mo = Mb + (16 * aa + g) * kLdm + 16 * bb + 8 * nt + 2 * t;
+                        mo[0] = -z[nt][0];
+                        mo[1] = -z[nt][1];
+                        mo[8 * kLdm] = -z[nt][2];
+                        mo[8 * kLdm + 1] = -z[nt][3];
+                    }
+                    __syncwarp();
                 }
                 __syncthreads();
             }
-            // T = M diag(beta), lower triangle, bf16 K-major
+            // T = (I + L)^-1 diag(beta): lower triangle, bf16 K-major
             {
                 const int r = tid >> 2, seg = tid & 3;
+                float x[16];
 #pragma unroll
-                for (int j = 0; j < 16; j += 2) {
+                for (int j = 0; j < 16; ++j) {
                     const int i = 16 * seg + j;
-                    const float x0 = (i <= r) ? Mb[r * kLds + i] * beta_s[i] : 0.f;
-                    const float x1 = (i + 1 <= r) ? Mb[r * kLds + i + 1] * beta_s[i + 1] : 0.f;
-                    st32(sm, OFF_T + sw128_off(64, r, i), pack_bf16(x0, x1));
+                    x[j] = (i <= r) ? Mb[r * kLdm + i] * beta_s[i] : 0.f;
                 }
+                st_bf16x8(sm + OFF_T + sw128_off(64, r, 16 * seg), x);
+                st_bf16x8(sm + OFF_T + sw128_off(64, r, 16 * seg + 8), x + 8);
             }
         }
         fence_proxy_async();
         __syncthreads();
 
         // ---------------------------------------------------------------- MMA: W = T K+, U~ = T V
+        if (!wait_all(bar_v, c & 1)) { aborted = true; break; }
+        v_pending = false;
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t idw = idesc_bf16(64, 128, 0, 1), idu = idesc_bf16(64, 64, 0, 1);
+            const uint32_t idw = idesc_bf16(64, 64, 0, 1), idu = idesc_bf16(64, 32, 0, 1);
 #pragma unroll
             for (int s = 0; s < kC / 16; ++s) {
                 const uint64_t ad = sw128_desc(sb + OFF_T + 32 * s, 16, 1024);
-                const uint64_t bw = sw128_desc(sb + OFF_KP + 2048 * s, 8192, 1024);
-                const uint64_t bu = sw128_desc(sb + OFF_V + (c & 1) * 8192 + 2048 * s, 8192, 1024);
-                umma_f16(tbase + TM_W, ad, bw, idw, s > 0);
-                umma_f16(tbase + TM_U, ad, bu, idu, s > 0);
+                umma_f16(tbase + TM_W, ad, sw128_desc(sb + OFF_KP + 2048 * s, 8192, 1024), idw,
+                         s > 0);
+                umma_f16(tbase + TM_W + kLaneHi, ad,
+                         sw128_desc(sb + OFF_KP + 8192 + 2048 * s, 8192, 1024), idw, s > 0);
+                umma_f16(tbase + TM_U, ad, sw64_desc(sb + OFF_V + 1024 * s, 4096, 512), idu,
+                         s > 0);
+                umma_f16(tbase + TM_U + kLaneHi, ad,
+                         sw64_desc(sb + OFF_V + 4096 + 1024 * s, 4096, 512), idu, s > 0);
             }
             umma_commit(bar_mma);
         }
@@ -564,28 +626,25 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ++mma_phase;
         mma_pending = false;
         tc_fence_after();
+        if (c + 1 < nchunks) {   // the V buffer is free again
+            if (tid == 0) issue_v(c + 1);
+            v_pending = true;
+            v_chunk = c + 1;
+        }
+        // lane l of quarter qd: row r = 16 qd + (l mod 16), column half lh = l / 16
+        const int rr = 16 * qd + (lane & 15), lh = lane >> 4;
         {
-            // lanes 0..15 of each quarter hold rows r = 16 qd + lane of the M=64 results
             float v[32];
-            const int r = 16 * qd + (lane & 15);
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int c0 = 64 * hf + 32 * part;
-                tmem_ld32(tbase + lane_q + TM_W + c0, v);
-                tmem_ld_wait();
-                if (lane < 16) {
-#pragma unroll
-                    for (int j = 0; j < 32; j += 2)
-                        st32(sm, OFF_W + sw128_off(64, r, c0 + j), pack_bf16(v[j], v[j + 1]));
-                }
-            }
-            tmem_ld32(tbase + lane_q + TM_U + 32 * hf, v);
+            tmem_ld32(tbase + lane_q + TM_W + 32 * hf, v);   // W[rr][64 lh + 32 hf ..]
+            float u[16];
+            tmem_ld16(tbase + lane_q + TM_U + 16 * hf, u);   // U~[rr][32 lh + 16 hf ..]
             tmem_ld_wait();
-            if (lane < 16) {
 #pragma unroll
-                for (int j = 0; j < 32; j += 2)
-                    st32(sm, OFF_UT + sw128_off(64, r, 32 * hf + j), pack_bf16(v[j], v[j + 1]));
-            }
+            for (int m = 0; m < 4; ++m)
+                st_bf16x8(sm + OFF_W + sw128_off(64, rr, 64 * lh + 32 * hf + 8 * m), v + 8 * m);
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+                st_bf16x8(sm + OFF_UT + lh * 4096 + sw64_off(rr, 16 * hf + 8 * m), u + 8 * m);
         }
         fence_proxy_async();
         tc_fence_before();
@@ -594,14 +653,18 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // ---------------------------------------------------------------- MMA: A_qk W, A_qk U~
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t idw = idesc_bf16(64, 128, 0, 1), idu = idesc_bf16(64, 64, 0, 1);
+            const uint32_t idw = idesc_bf16(64, 64, 0, 1), idu = idesc_bf16(64, 32, 0, 1);
 #pragma unroll
             for (int s = 0; s < kC / 16; ++s) {
                 const uint64_t ad = sw128_desc(sb + OFF_AQK + 32 * s, 16, 1024);
-                const uint64_t bw = sw128_desc(sb + OFF_W + 2048 * s, 8192, 1024);
-                const uint64_t bu = sw128_desc(sb + OFF_UT + 2048 * s, 8192, 1024);
-                umma_f16(tbase + TM_W + kLaneHi, ad, bw, idw, s > 0);
-                umma_f16(tbase + TM_U + kLaneHi, ad, bu, idu, s > 0);
+                umma_f16(tbase + TM_W2, ad, sw128_desc(sb + OFF_W + 2048 * s, 8192, 1024), idw,
+                         s > 0);
+                umma_f16(tbase + TM_W2 + kLaneHi, ad,
+                         sw128_desc(sb + OFF_W + 8192 + 2048 * s, 8192, 1024), idw, s > 0);
+                umma_f16(tbase + TM_U2, ad, sw64_desc(sb + OFF_UT + 1024 * s, 4096, 512), idu,
+                         s > 0);
+                umma_f16(tbase + TM_U2 + kLaneHi, ad,
+                         sw64_desc(sb + OFF_UT + 4096 + 1024 * s, 4096, 512), idu, s > 0);
             }
             umma_commit(bar_mma);
         }
@@ -611,34 +674,31 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mma_pending = false;
         tc_fence_after();
         {
-            // lanes 16..31 hold rows r = 16 qd + lane - 16 of A_qk W: Q~ = Q+ - A_qk W
+            // Q~ = Q+ - A_qk W (in place on the Q+ tile)
             float v[32];
-            const int r = 16 * qd + (lane & 15);
+            tmem_ld32(tbase + lane_q + TM_W2 + 32 * hf, v);
+            tmem_ld_wait();
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int c0 = 64 * hf + 32 * part;
-                tmem_ld32(tbase + lane_q + TM_W + c0, v);
-                tmem_ld_wait();
-                if (lane >= 16) {
-#pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        const uint32_t off = OFF_QT + sw128_off(64, r, c0 + j);
-                        const float2 qp = unpack_bf16(ld32(sm, off));
-                        st32(sm, off, pack_bf16(qp.x - v[j], qp.y - v[j + 1]));
-                    }
-                }
+            for (int m = 0; m < 4; ++m) {
+                uint8_t* p = sm + OFF_QT + sw128_off(64, rr, 64 * lh + 32 * hf + 8 * m);
+                const uint4 qv = *reinterpret_cast<const uint4*>(p);
+                const float2 a0 = unpack_bf16(qv.x), a1 = unpack_bf16(qv.y);
+                const float2 a2 = unpack_bf16(qv.z), a3 = unpack_bf16(qv.w);
+                const float* w = v + 8 * m;
+                *reinterpret_cast<uint4*>(p) =
+                    make_uint4(pack_bf16(a0.x - w[0], a0.y - w[1]), pack_bf16(a1.x - w[2], a1.y - w[3]),
+                               pack_bf16(a2.x - w[4], a2.y - w[5]), pack_bf16(a3.x - w[6], a3.y - w[7]));
             }
         }
-        // ---------------------------------------------------------------- state pass
         {
-            // S (fp32, TMEM) -> bf16 operand; then decay the TMEM copy for the update
+            // state: bf16 operand halves for W S and Q~ S, then decay the fp32 TMEM copy
             float v[32];
             const int cc = 32 * qd + lane;
             tmem_ld32(tbase + lane_q + TM_S + 32 * hf, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 32; j += 2)
-                st32(sm, OFF_S16 + sw128_off(128, cc, 32 * hf + j), pack_bf16(v[j], v[j + 1]));
+            for (int m = 0; m < 4; ++m)
+                st_bf16x8(sm + OFF_S16 + hf * 8192 + sw64_off(cc, 8 * m), v + 8 * m);
             const float dcy = decay_s[cc];
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] *= dcy;
@@ -648,17 +708,24 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
+
+        // ---------------------------------------------------------------- MMA: W S, Q~ S
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t id = idesc_bf16(64, 64, 0, 1);
+            const uint32_t id = idesc_bf16(64, 32, 0, 1);
 #pragma unroll
             for (int s = 0; s < kD / 16; ++s) {
                 const int k0 = 16 * s;
-                const uint64_t aw = sw128_desc(sb + OFF_W + (k0 >> 6) * 8192 + (k0 & 63) * 2, 16, 1024);
-                const uint64_t aq = sw128_desc(sb + OFF_QT + (k0 >> 6) * 8192 + (k0 & 63) * 2, 16, 1024);
-                const uint64_t bs = sw128_desc(sb + OFF_S16 + 2048 * s, 16384, 1024);
-                umma_f16(tbase + TM_B, aw, bs, id, s > 0);
-                umma_f16(tbase + TM_B + kLaneHi, aq, bs, id, s > 0);
+                const uint64_t aw =
+                    sw128_desc(sb + OFF_W + (k0 >> 6) * 8192 + (k0 & 63) * 2, 16, 1024);
+                const uint64_t aq =
+                    sw128_desc(sb + OFF_QT + (k0 >> 6) * 8192 + (k0 & 63) * 2, 16, 1024);
+                const uint64_t b0 = sw64_desc(sb + OFF_S16 + 1024 * s, 8192, 512);
+                const uint64_t b1 = sw64_desc(sb + OFF_S16 + 8192 + 1024 * s, 8192, 512);
+                umma_f16(tbase + TM_B, aw, b0, id, s > 0);
+                umma_f16(tbase + TM_B + kLaneHi, aw, b1, id, s > 0);
+                umma_f16(tbase + TM_B + 32, aq, b0, id, s > 0);
+                umma_f16(tbase + TM_B + 32 + kLaneHi, aq, b1, id, s > 0);
             }
             umma_commit(bar_mma);
         }
@@ -668,35 +735,41 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mma_pending = false;
         tc_fence_after();
         {
-            float ws[32], ut[32];
-            const int r = 16 * qd + (lane & 15);
-            tmem_ld32(tbase + lane_q + TM_B + 32 * hf, ws);
-            tmem_ld32(tbase + lane_q + TM_U + 32 * hf, ut);
-            tmem_ld_wait();
-            if (lane < 16) {
-                // U = U~ - W S
+            float x[32], y[32];
+            if (hf == 0) {
+                // U = U~ - W S  (row rr, value columns 32 lh ..)
+                tmem_ld32(tbase + lane_q + TM_B, x);
+                tmem_ld32(tbase + lane_q + TM_U, y);
+                tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; j += 2)
-                    st32(sm, OFF_U16 + sw128_off(64, r, 32 * hf + j),
-                         pack_bf16(ut[j] - ws[j], ut[j + 1] - ws[j + 1]));
-            } else if (r < L) {
+                for (int j = 0; j < 32; ++j) y[j] -= x[j];
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    st_bf16x8(sm + OFF_U16 + sw128_off(64, rr, 32 * lh + 8 * m), y + 8 * m);
+            } else {
                 // o = O~ + Q~ S
-                uint4* dst = reinterpret_cast<uint4*>(
-                    args.o + ((size_t)(row0 + r) * args.H + h) * kD + dv0 + 32 * hf);
+                tmem_ld32(tbase + lane_q + TM_B + 32, x);
+                tmem_ld32(tbase + lane_q + TM_U2, y);
+                tmem_ld_wait();
+                if (rr < L) {
 #pragma unroll
-                for (int j = 0; j < 32; j += 8) {
-                    uint4 u;
-                    u.x = pack_bf16(ut[j] + ws[j], ut[j + 1] + ws[j + 1]);
-                    u.y = pack_bf16(ut[j + 2] + ws[j + 2], ut[j + 3] + ws[j + 3]);
-                    u.z = pack_bf16(ut[j + 4] + ws[j + 4], ut[j + 5] + ws[j + 5]);
-                    u.w = pack_bf16(ut[j + 6] + ws[j + 6], ut[j + 7] + ws[j + 7]);
-                    dst[j / 8] = u;
+                    for (int j = 0; j < 32; ++j) y[j] += x[j];
+                    uint4* dst = reinterpret_cast<uint4*>(
+                        args.o + ((size_t)(row0 + rr) * args.H + h) * kD + dv0 + 32 * lh);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float* w = y + 8 * m;
+                        dst[m] = make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]),
+                                            pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
+                    }
                 }
             }
         }
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
+
+        // ---------------------------------------------------------------- MMA: S += K_end^T U
         if (tid == 0) {
             tc_fence_after();
             const uint32_t id = idesc_bf16(128, 64, 1, 1);
@@ -716,16 +789,15 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (tid == 0) set_device_error(args.err, DEV_TIMEOUT);
         // wind down: let this CTA's own copies and MMAs finish before TMEM and smem go away
         const long long drain = 1ll << 31;
-        if (tma_pending) mbar_wait(bar_tma, tma_chunk & 1, drain);
+        if (in_pending) mbar_wait(bar_in, in_chunk & 1, drain);
+        if (v_pending) mbar_wait(bar_v, v_chunk & 1, drain);
         if (mma_pending) mbar_wait(bar_mma, mma_phase & 1, drain);
         if (b4_pending) mbar_wait(bar_b4, b4_chunk & 1, drain);
         __syncthreads();
     } else {
-        if (b4_pending) {
-            if (!wait_all(bar_b4, b4_chunk & 1)) {
-                if (tid == 0) set_device_error(args.err, DEV_TIMEOUT);
-                mbar_wait(bar_b4, b4_chunk & 1, 1ll << 31);
-            }
+        if (b4_pending && !wait_all(bar_b4, b4_chunk & 1)) {
+            if (tid == 0) set_device_error(args.err, DEV_TIMEOUT);
+            mbar_wait(bar_b4, b4_chunk & 1, 1ll << 31);
         }
         tc_fence_after();
         if (args.hT) {
@@ -733,7 +805,8 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int cc = 32 * qd + lane;
             tmem_ld32(tbase + lane_q + TM_S + 32 * hf, v);
             tmem_ld_wait();
-            float4* dst = reinterpret_cast<float4*>(args.hT + state_base + (size_t)cc * kD + dv0 + 32 * hf);
+            float4* dst = reinterpret_cast<float4*>(args.hT + state_base + (size_t)cc * kD + dv0 +
+                                                    32 * hf);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
                 dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
@@ -820,8 +893,8 @@ cudaError_t launch_chunk64(const FwdParams& p, cudaStream_t stream) {
                       CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
         (e = make_map(&mg, p.log_g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, p.H, kD,
                       CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
-        (e = make_map(&mv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, kDV,
-                      CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
+        (e = make_map(&mv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, 32,
+                      CU_TENSOR_MAP_SWIZZLE_64B)) != cudaSuccess)
         return e;
     {
         std::lock_guard<std::mutex> lock(g_attr_mu);

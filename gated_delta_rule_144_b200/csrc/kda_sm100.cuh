@@ -195,6 +195,17 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo, uint
     return d;
 }
 
+// Same with 64-byte swizzle (8-row atoms of 512 bytes; 32 bf16 per row).
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)4 << 61;  // SWIZZLE_64B
+    return d;
+}
+
 // Instruction descriptor: bf16 x bf16 -> fp32, dense. a_mn / b_mn: operand is MN-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
@@ -208,6 +219,27 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
 __host__ __device__ constexpr uint32_t sw128_off(int R, int r, int c) {
     return (uint32_t)((c >> 6) * (R * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
                       ((((c & 63) >> 3) ^ (r & 7)) << 4) + (c & 7) * 2);
+}
+
+// Byte offset of element (r, c), c < 32, of a bf16 tile in the 64-byte-swizzled layout: rows of
+// 64 bytes, 16-byte chunks permuted by ((row / 2) mod 4) as TMA SWIZZLE_64B writes them.
+__host__ __device__ constexpr uint32_t sw64_off(int r, int c) {
+    return (uint32_t)(r * 64 + ((((c >> 3) ^ (r >> 1)) & 3) << 4) + (c & 7) * 2);
+}
+
+// ------------------------------------------------------------------ warp-level tf32 MMA
+
+// D (16x8, fp32) += A (16x8, tf32, row) * B (8x8, tf32, col); legacy warp-synchronous MMA used
+// for the 16x16 blocks of the UT transform. Fragment element (row, col) ownership, with
+// g = lane / 4 and t = lane % 4: a = {(g,t), (g+8,t), (g,t+4), (g+8,t+4)}, b = {(t,g), (t+4,g)},
+// d = {(g,2t), (g,2t+1), (g+8,2t), (g+8,2t+1)}.
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4],
+                                                const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
 }  // namespace sm100
