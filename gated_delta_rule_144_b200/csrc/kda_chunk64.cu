@@ -24,8 +24,11 @@
 //
 // Pipeline per chunk (256 threads; thread 0 issues TMA and MMAs):
 //   TMA q, k, log g, v  ->  elementwise decay factors (CUDA cores)  ->  MMA R C^T  ->
-//   assemble A_kk, A_qk  ->  UT solve (fp32, blocked)  ->  MMA T [K+ | V]  ->  MMA A_qk [W | U~]
-//   ->  MMA [W; Q~] S  ->  U, o  ->  MMA S += K_end^T U.
+//   assemble A_kk, A_qk  ->  UT solve (fp32, blocked)  ->  MMA T' = A_qk T  ->
+//   MMA [T; T'] [K+ | V] (W, A_qk W, U~, O~ in one M=128 product)  ->  MMA [W; Q~] S  ->
+//   U, o  ->  MMA S += K_end^T U.
+// Every tcgen05 product is M=128 (full rate): a few large MMAs cost little to issue where many
+// small ones would not.
 // The next chunk's TMA overlaps everything after the elementwise pass. Every mbarrier wait is
 // bounded; on expiry the CTA records KDA_ERR_TIMEOUT, drains its own outstanding copies and MMAs,
 // frees TMEM and exits.
@@ -46,60 +49,60 @@ using namespace sm100;
 
 constexpr int kC = 64;        // tokens per chunk
 constexpr int kD = 128;       // dk = dv
-constexpr int kDV = 64;       // value columns per CTA
-constexpr int kSplit = kD / kDV;
 constexpr int kThreads = 256;
 
-// ---- shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_Q = 0;            // q   [64][128] bf16 row-major (TMA)
-constexpr uint32_t OFF_K = 16384;        // k   [64][128] bf16 row-major (TMA)
-constexpr uint32_t OFF_G = 32768;        // log g [64][128] f32 row-major (TMA)
-constexpr uint32_t OFF_V = 65536;        // v   2 x [64][32] bf16, 64B-swizzled halves (TMA)
-constexpr uint32_t OFF_R = 73728;        // R   [128][128] bf16 (K-major A of R C^T)
-constexpr uint32_t OFF_C = OFF_R + 32768;  // C [160][128] bf16 (K-major B of R C^T)
-//   after R C^T completes, the R/C region is reused:
-constexpr uint32_t OFF_LB = OFF_R;              // L = diag(beta) A_kk, f32 [64][kLdl]
-constexpr uint32_t OFF_MB = OFF_R + 17408;      // (I + L)^-1, f32 [64][kLdm]
-constexpr uint32_t OFF_YS = OFF_R + 35840;      // per-warp 16x16 scratch of the solve
-constexpr uint32_t OFF_T = OFF_R + 39936;       // T  [64][64] bf16 (K-major A)
-constexpr uint32_t OFF_UT = OFF_R + 48128;      // U~ 2 x [64][32] bf16 (MN-major B halves)
-constexpr uint32_t OFF_S16 = OFF_R;             // S  2 x [128][32] bf16 (MN-major B halves)
-constexpr uint32_t OFF_U16 = OFF_R + 16384;     // U  [64][64] bf16 (MN-major B)
-constexpr uint32_t OFF_AQK = OFF_C + 40960;     // A_qk [64][64] bf16 (K-major A), own region
-constexpr uint32_t OFF_KP = OFF_AQK + 8192;     // K+ [64][128] bf16 (MN-major B)
-constexpr uint32_t OFF_W = OFF_KP + 16384;      // W  [64][128] bf16 (K-major A / MN-major B)
-constexpr uint32_t OFF_QT = OFF_W + 16384;      // Q+ then Q~ [64][128] bf16 (K-major A)
-constexpr uint32_t OFF_KE = OFF_QT + 16384;     // K_end [64][128] bf16 (MN-major A)
-constexpr uint32_t OFF_MISC = OFF_KE + 16384;
-constexpr uint32_t OFF_BETA = OFF_MISC;         // f32 [64]
-constexpr uint32_t OFF_DECAY = OFF_MISC + 256;  // f32 [128]
-constexpr uint32_t OFF_LOUP = OFF_MISC + 768;   // f32 [4 blocks][2 halves][128]
-constexpr uint32_t OFF_BAR = OFF_MISC + 4864;   // 5 mbarriers
-constexpr uint32_t OFF_TMEM = OFF_BAR + 64;     // TMEM base address
-constexpr uint32_t kSmemUsed = OFF_TMEM + 16;
-constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
+// Shared memory and TMEM layout for a CTA that owns DV value columns (64: half a head, for
+// workloads with few sequence-head chains; 128: a whole head, which halves the intra-chunk work
+// per value column and doubles the N of every state-step product at the same number of MMAs).
+template <int DV>
+struct Layout {
+    static constexpr int kDV = DV;
+    static constexpr int kSplit = kD / DV;   // CTAs per (sequence, head)
+    static constexpr int kPanels = DV / 64;  // 64-column panels of V, S and U
+    // shared memory (bytes from a 1024-aligned base)
+    static constexpr uint32_t OFF_Q = 0;          // q   [64][128] bf16 row-major (TMA)
+    static constexpr uint32_t OFF_K = 16384;      // k   [64][128] bf16 row-major (TMA)
+    static constexpr uint32_t OFF_G = 32768;      // log g [64][128] f32 row-major (TMA)
+    static constexpr uint32_t OFF_KPV = 65536;    // [K+ | V] [64][128 + DV] MN-major B panels
+    static constexpr uint32_t OFF_R = OFF_KPV + 8192u * (2 + kPanels);  // R [128][128] K-major A
+    static constexpr uint32_t OFF_C = OFF_R + 32768;                    // C [160][128] K-major B
+    //   after R C^T completes, the R/C region is reused:
+    static constexpr uint32_t OFF_LB = OFF_R;           // L = diag(beta) A_kk, f32 [64][kLdl]
+    static constexpr uint32_t OFF_MB = OFF_R + 17408;   // (I + L)^-1, f32 [64][kLdm]
+    static constexpr uint32_t OFF_YS = OFF_R + 35840;   // per-warp 16x16 scratch of the solve
+    static constexpr uint32_t OFF_TT = OFF_R + 40960;   // [T; T'] [128][64] bf16 (K-major A;
+                                                        //   rows 0-63 also the MN-major B of T')
+    static constexpr uint32_t OFF_ZA = OFF_R + 57344;   // [0; A_qk] [128][64] bf16 (K-major A)
+    static constexpr uint32_t OFF_S16 = OFF_R;          // S [128][DV] bf16 (MN-major B panels)
+    static constexpr uint32_t OFF_U16 = OFF_R + 16384u * kPanels;  // U [64][DV] (MN-major B)
+    static constexpr uint32_t OFF_WQ = OFF_C + 40960;   // [W; Q+ -> Q~] [128][128] (K-major A)
+    static constexpr uint32_t OFF_KE = OFF_WQ + 32768;  // K_end [64][128] bf16 (MN-major A)
+    static constexpr uint32_t OFF_MISC = OFF_KE + 16384;
+    static constexpr uint32_t OFF_BETA = OFF_MISC;         // f32 [64]
+    static constexpr uint32_t OFF_DECAY = OFF_MISC + 256;  // f32 [128]
+    static constexpr uint32_t OFF_LOUP = OFF_MISC + 768;   // f32 [4 blocks][2 halves][128]
+    static constexpr uint32_t OFF_BAR = OFF_MISC + 4864;   // 5 mbarriers
+    static constexpr uint32_t OFF_TMEM = OFF_BAR + 64;     // TMEM base address
+    static constexpr uint32_t kSmemBytes = OFF_TMEM + 16 + 1024;  // + alignment slack
+    static_assert(OFF_ZA + 16384 == OFF_C + 40960, "solve buffers fill the R/C region exactly");
+    static_assert(OFF_YS + 3 * 16 * 17 * 4 <= OFF_TT, "solve scratch overlaps [T; T']");
+    static_assert(OFF_U16 + 8192u * kPanels <= OFF_C + 40960, "state-step tiles overflow");
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    // TMEM columns (fp32, 128 lanes; M=128 layout: row m of a product sits in lane m)
+    static constexpr uint32_t TM_A = 0;     // R C^T [128 x 160]; later [T; T'] [K+ | V]:
+                                            //   lanes 0-63: W (cols 0-127), U~ (128 ..)
+                                            //   lanes 64-127: A_qk W (0-127), O~ (128 ..)
+    static constexpr uint32_t TM_TP = 160;  // [0; A_qk] T (lanes 64-127: T' = A_qk T), read
+                                            //   before [T; T'] [K+ | V] overwrites it
+    static constexpr uint32_t TM_B = 128 + DV;  // [W; Q~] S: lanes 0-63 W S, 64-127 Q~ S
+    static constexpr uint32_t TM_S = 128 + 2 * DV;  // state S [128 x DV] fp32
+    static_assert(TM_S + DV <= 512, "TMEM budget");
+    static constexpr uint32_t kTxV = 8192u * kPanels;
+};
 constexpr int kLdl = 68;   // row stride (floats) of L: conflict-free A-fragment loads
 constexpr int kLdm = 72;   // row stride (floats) of M: conflict-free B-fragment loads
-static_assert(OFF_UT + 8192 <= OFF_C + 40960, "solve buffers overflow the R/C region");
-static_assert(OFF_U16 + 8192 <= OFF_T, "state-pass tiles overlap the solve outputs");
-static_assert(OFF_YS + 3 * 16 * 17 * 4 <= OFF_T, "solve scratch overlaps T");
-static_assert(kSmemBytes <= 232448, "shared memory budget");
-
-// ---- TMEM columns (fp32, 128 lanes). M=64 results use lanes {0-15, 32-47, ...} ("lo") and
-// the interleaved {16-31, 48-63, ...} ("hi"); every M=64 product is split in two along N so
-// that both lane halves of every warp carry data.
-constexpr uint32_t TM_A = 0;     // R C^T          [128 x 160]
-constexpr uint32_t TM_W = 160;   // W: cols 0-63 lo, 64-127 hi                     (64 cols)
-constexpr uint32_t TM_U = 224;   // U~: value cols 0-31 lo, 32-63 hi                (32 cols)
-constexpr uint32_t TM_W2 = 256;  // A_qk W, same split as W                         (64 cols)
-constexpr uint32_t TM_U2 = 320;  // O~ = A_qk U~, same split as U~                  (32 cols)
-constexpr uint32_t TM_B = 352;   // W S (+0) and Q~ S (+32), split as U~            (64 cols)
-constexpr uint32_t TM_S = 416;   // state S [128 x 64] fp32
 constexpr uint32_t kTmemCols = 512;
-
 constexpr uint32_t kTxIn = 16384 + 16384 + 32768;
-constexpr uint32_t kTxV = 8192;
-constexpr uint32_t kLaneHi = 16u << 16;   // second M=64 tile interleaved at lane +16
 
 // row offset, inside C[64:], of the columns row block a needs from earlier blocks
 __host__ __device__ constexpr int cross_off(int a) { return a == 1 ? 0 : (a == 2 ? 16 : 48); }
@@ -138,10 +141,22 @@ __device__ __forceinline__ void st_bf16x8(uint8_t* p, const float* v) {
 }
 __device__ __forceinline__ uint32_t f2tf(float x) { return __float_as_uint(x); }
 
+template <int DV>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
                const ChunkArgs args) {
+    using Lay = Layout<DV>;
+    constexpr int kDV = Lay::kDV, kSplit = Lay::kSplit, kPanels = Lay::kPanels;
+    constexpr uint32_t OFF_Q = Lay::OFF_Q, OFF_K = Lay::OFF_K, OFF_G = Lay::OFF_G;
+    constexpr uint32_t OFF_KPV = Lay::OFF_KPV, OFF_R = Lay::OFF_R, OFF_C = Lay::OFF_C;
+    constexpr uint32_t OFF_LB = Lay::OFF_LB, OFF_MB = Lay::OFF_MB, OFF_YS = Lay::OFF_YS;
+    constexpr uint32_t OFF_TT = Lay::OFF_TT, OFF_ZA = Lay::OFF_ZA, OFF_S16 = Lay::OFF_S16;
+    constexpr uint32_t OFF_U16 = Lay::OFF_U16, OFF_WQ = Lay::OFF_WQ, OFF_KE = Lay::OFF_KE;
+    constexpr uint32_t OFF_BETA = Lay::OFF_BETA, OFF_DECAY = Lay::OFF_DECAY;
+    constexpr uint32_t OFF_LOUP = Lay::OFF_LOUP, OFF_BAR = Lay::OFF_BAR, OFF_TMEM = Lay::OFF_TMEM;
+    constexpr uint32_t TM_A = Lay::TM_A, TM_TP = Lay::TM_TP, TM_B = Lay::TM_B, TM_S = Lay::TM_S;
+    constexpr int kHalfCols = kDV / 2;   // value columns per warp in the state read-outs
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -191,10 +206,6 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tmem_alloc(smem_u32(tmem_s), kTmemCols);
         tmem_relinquish();
     }
-    // A_qk lives in its own region: its strictly-upper blocks are zeroed once and never written
-    reinterpret_cast<uint4*>(sm + OFF_AQK)[tid] = make_uint4(0, 0, 0, 0);
-    reinterpret_cast<uint4*>(sm + OFF_AQK)[tid + kThreads] = make_uint4(0, 0, 0, 0);
-    fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -202,13 +213,15 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t lane_q = (uint32_t)(32 * qd) << 16;   // this warp's TMEM lane quarter
     const size_t state_base = ((size_t)n * args.H + h) * kD * kD;
 
-    // initial state: TMEM lane c = 32 qd + lane holds S[c][dv0 + 32 hf .. + 32)
-    {
+    // initial state: TMEM lane c = 32 qd + lane holds S[c][dv0 + kHalfCols hf .. + kHalfCols)
+#pragma unroll
+    for (int p = 0; p < kHalfCols / 32; ++p) {
         float v[32];
         const int c = 32 * qd + lane;
+        const int col = kHalfCols * hf + 32 * p;
         if (args.h0) {
             const float4* src = reinterpret_cast<const float4*>(args.h0 + state_base +
-                                                                (size_t)c * kD + dv0 + 32 * hf);
+                                                                (size_t)c * kD + dv0 + col);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const float4 x = src[i];
@@ -218,7 +231,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0.f;
         }
-        tmem_st32(tbase + lane_q + TM_S + 32 * hf, v);
+        tmem_st32(tbase + lane_q + TM_S + col, v);
         tmem_st_wait();
     }
 
@@ -231,19 +244,26 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     };
     auto issue_v = [&](int c) {
         const int row0 = (int)(t0 + (long long)kC * c);
-        mbar_arrive_expect_tx(bar_v, kTxV);
-        tma_load_3d(sb + OFF_V, &tm_v, bar_v, dv0, h, row0);
-        tma_load_3d(sb + OFF_V + 4096, &tm_v, bar_v, dv0 + 32, h, row0);
+        mbar_arrive_expect_tx(bar_v, Lay::kTxV);
+#pragma unroll
+        for (int p = 0; p < kPanels; ++p)
+            tma_load_3d(sb + OFF_KPV + 16384 + 8192 * p, &tm_v, bar_v, dv0 + 64 * p, h, row0);
     };
+
+    // constant parts of the shared-memory descriptors (the start address is added per MMA)
+    const uint64_t dK = sw128_desc(0, 16, 1024);     // K-major, 128B swizzle
+    const uint64_t dM8 = sw128_desc(0, 8192, 1024);  // MN-major, 128B swizzle, 64-row panels
+    const uint64_t dM16 = sw128_desc(0, 16384, 1024);
 
     // outstanding asynchronous work, drained before exit if a wait expires
     bool in_pending = false, v_pending = false, mma_pending = false, b4_pending = false;
     int in_chunk = 0, v_chunk = 0, b4_chunk = 0;
     uint32_t mma_phase = 0;
     bool aborted = false;
+    // One thread polls; the rest of the CTA waits at the barrier that publishes the outcome.
     auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
-        const bool ok = mbar_wait(bar, parity, args.budget);
-        return __syncthreads_or(!ok) == 0;   // every thread agrees on the outcome
+        const bool ok = tid != 0 || mbar_wait(bar, parity, args.budget);
+        return __syncthreads_or(!ok) == 0;
     };
 
     if (nchunks > 0) {
@@ -256,6 +276,10 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // Failure injection (KDA_DEBUG_STALL_WAIT): a wait on a barrier that nothing signals, with
     // copies in flight, must expire, report KDA_ERR_TIMEOUT and wind down cleanly.
     if (args.debug_stall && !wait_all(bar_never, 0)) aborted = true;
+
+    float beta_next = 0.f;   // beta of the next chunk, row tid (threads tid < 64)
+    if (tid < kC && nchunks > 0 && t0 + tid < t1)
+        beta_next = __bfloat162float(args.beta[(t0 + tid) * args.H + h]);
 
     const uint8_t* qs = sm + OFF_Q;
     const uint8_t* ks = sm + OFF_K;
@@ -284,8 +308,11 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (!wait_all(bar_b4, b4_chunk & 1)) { aborted = true; break; }
             b4_pending = false;
         }
-        if (tid < kC)
-            beta_s[tid] = tid < L ? __bfloat162float(args.beta[(row0 + tid) * args.H + h]) : 0.f;
+        if (tid < kC) beta_s[tid] = beta_next;
+        if (tid < kC && c + 1 < nchunks) {   // prefetch the next chunk's beta
+            const long long r1 = row0 + kC + tid;
+            beta_next = r1 < t1 ? __bfloat162float(args.beta[r1 * args.H + h]) : 0.f;
+        }
 
         // ---------------------------------------------------------------- decay products
         float pre[8][4], suf[8][4];
@@ -401,19 +428,22 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         __syncthreads();
 
         // ---------------------------------------------------------------- MMA: R C^T
-        if (tid == 0) {
+        if (warp == 0) {   // lane 0 issues; the rest of warp 0 waits for it
+            if (lane == 0) {
             tc_fence_after();
             const uint32_t id = idesc_bf16(128, 160, 0, 0);
 #pragma unroll
             for (int s = 0; s < kD / 16; ++s) {
                 const int k0 = 16 * s;
                 const uint64_t ad =
-                    sw128_desc(sb + OFF_R + (k0 >> 6) * 16384 + (k0 & 63) * 2, 16, 1024);
+                    desc_at(dK, sb + OFF_R + (k0 >> 6) * 16384 + (k0 & 63) * 2);
                 const uint64_t bd =
-                    sw128_desc(sb + OFF_C + (k0 >> 6) * 20480 + (k0 & 63) * 2, 16, 1024);
+                    desc_at(dK, sb + OFF_C + (k0 >> 6) * 20480 + (k0 & 63) * 2);
                 umma_f16(tbase + TM_A, ad, bd, id, s > 0);
             }
             umma_commit(bar_mma);
+            }
+            __syncwarp();
         }
         mma_pending = true;
 
@@ -432,8 +462,9 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 x[i] = G[i] * (hh == 0 ? suf[j][i] * own[i] : suf[j][i]);
             }
             const uint32_t o64 = toff(64, rb8, j);
-            st_bf16x4(sm + OFF_KP + o64, k4.x * e[0], k4.y * e[1], k4.z * e[2], k4.w * e[3]);
-            st_bf16x4(sm + OFF_QT + o64, q4.x * e[0], q4.y * e[1], q4.z * e[2], q4.w * e[3]);
+            st_bf16x4(sm + OFF_KPV + o64, k4.x * e[0], k4.y * e[1], k4.z * e[2], k4.w * e[3]);
+            st_bf16x4(sm + OFF_WQ + toff(128, rb8 + 8, j), q4.x * e[0], q4.y * e[1], q4.z * e[2],
+                      q4.w * e[3]);
             st_bf16x4(sm + OFF_KE + o64, k4.x * x[0], k4.y * x[1], k4.z * x[2], k4.w * x[3]);
         }
         fence_proxy_async();
@@ -458,8 +489,8 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // write 16 consecutive entries (i0 .. i0+15) of row r
             auto put16 = [&](int i0, const float* x) {
                 if (is_q) {
-                    st_bf16x8(sm + OFF_AQK + sw128_off(64, r, i0), x);
-                    st_bf16x8(sm + OFF_AQK + sw128_off(64, r, i0 + 8), x + 8);
+                    st_bf16x8(sm + OFF_ZA + sw128_off(128, 64 + r, i0), x);
+                    st_bf16x8(sm + OFF_ZA + sw128_off(128, 64 + r, i0 + 8), x + 8);
                 } else {
                     float4* dst = reinterpret_cast<float4*>(Lb + r * kLdl + i0);
 #pragma unroll
@@ -481,6 +512,16 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     x[j] = (is_q ? i <= r : i < r) ? val : 0.f;
                 }
                 put16(16 * a, x);
+                if (is_q) {   // A_qk is lower triangular: zero the blocks after the diagonal one
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+                    for (int i = 16 * (a + 1); i < kC; i += 8)
+                        *reinterpret_cast<uint4*>(sm + OFF_ZA + sw128_off(128, 64 + r, i)) = z;
+                } else {      // rows 0-63 of [0; A_qk] are zero
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int i = 0; i < kC; i += 8)
+                        *reinterpret_cast<uint4*>(sm + OFF_ZA + sw128_off(128, r, i)) = z;
+                }
             } else if ((qd & 1) == 0) {
                 float w[16];
                 tmem_ld16(tbase + lane_q + TM_A + 64 + cross_off(1), w);   // block 1: i in 0..15
@@ -587,181 +628,178 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             // T = (I + L)^-1 diag(beta): lower triangle, bf16 K-major
             {
-                const int r = tid >> 2, seg = tid & 3;
-                float x[16];
+                const int i = 2 * lane;
+                const float b0 = beta_s[i], b1 = beta_s[i + 1];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int i = 16 * seg + j;
-                    x[j] = (i <= r) ? Mb[r * kLdm + i] * beta_s[i] : 0.f;
+                for (int rr8 = 0; rr8 < 8; ++rr8) {
+                    const int r = 8 * warp + rr8;
+                    const float2 m = *reinterpret_cast<const float2*>(Mb + r * kLdm + i);
+                    const float x0 = (i <= r) ? m.x * b0 : 0.f;
+                    const float x1 = (i + 1 <= r) ? m.y * b1 : 0.f;
+                    *reinterpret_cast<uint32_t*>(sm + OFF_TT + sw128_off(128, r, i)) =
+                        pack_bf16(x0, x1);
                 }
-                st_bf16x8(sm + OFF_T + sw128_off(64, r, 16 * seg), x);
-                st_bf16x8(sm + OFF_T + sw128_off(64, r, 16 * seg + 8), x + 8);
             }
         }
         fence_proxy_async();
         __syncthreads();
 
-        // ---------------------------------------------------------------- MMA: W = T K+, U~ = T V
-        if (!wait_all(bar_v, c & 1)) { aborted = true; break; }
-        v_pending = false;
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t idw = idesc_bf16(64, 64, 0, 1), idu = idesc_bf16(64, 32, 0, 1);
+        // ---------------------------------------------------------------- MMA: T' = A_qk T
+        // [0; A_qk] (128 x 64) times T as the MN-major B operand: lanes 64-127 receive A_qk T.
+        if (warp == 0) {   // lane 0 issues; the rest of warp 0 waits for it
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
-            for (int s = 0; s < kC / 16; ++s) {
-                const uint64_t ad = sw128_desc(sb + OFF_T + 32 * s, 16, 1024);
-                umma_f16(tbase + TM_W, ad, sw128_desc(sb + OFF_KP + 2048 * s, 8192, 1024), idw,
-                         s > 0);
-                umma_f16(tbase + TM_W + kLaneHi, ad,
-                         sw128_desc(sb + OFF_KP + 8192 + 2048 * s, 8192, 1024), idw, s > 0);
-                umma_f16(tbase + TM_U, ad, sw64_desc(sb + OFF_V + 1024 * s, 4096, 512), idu,
-                         s > 0);
-                umma_f16(tbase + TM_U + kLaneHi, ad,
-                         sw64_desc(sb + OFF_V + 4096 + 1024 * s, 4096, 512), idu, s > 0);
+                for (int s = 0; s < kC / 16; ++s)
+                    umma_f16(tbase + TM_TP, desc_at(dK, sb + OFF_ZA + 32 * s),
+                             desc_at(dM8, sb + OFF_TT + 2048 * s), id, s > 0);
+                umma_commit(bar_mma);
             }
-            umma_commit(bar_mma);
+            __syncwarp();
         }
         mma_pending = true;
         if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
         ++mma_phase;
         mma_pending = false;
         tc_fence_after();
-        if (c + 1 < nchunks) {   // the V buffer is free again
-            if (tid == 0) issue_v(c + 1);
-            v_pending = true;
-            v_chunk = c + 1;
-        }
-        // lane l of quarter qd: row r = 16 qd + (l mod 16), column half lh = l / 16
-        const int rr = 16 * qd + (lane & 15), lh = lane >> 4;
-        {
+        if (qd >= 2) {
+            // T' rows r = 32 (qd - 2) + lane  ->  rows 64 + r of [T; T']
             float v[32];
-            tmem_ld32(tbase + lane_q + TM_W + 32 * hf, v);   // W[rr][64 lh + 32 hf ..]
-            float u[16];
-            tmem_ld16(tbase + lane_q + TM_U + 16 * hf, u);   // U~[rr][32 lh + 16 hf ..]
+            const int r = 32 * (qd - 2) + lane;
+            tmem_ld32(tbase + lane_q + TM_TP + 32 * hf, v);
             tmem_ld_wait();
 #pragma unroll
             for (int m = 0; m < 4; ++m)
-                st_bf16x8(sm + OFF_W + sw128_off(64, rr, 64 * lh + 32 * hf + 8 * m), v + 8 * m);
-#pragma unroll
-            for (int m = 0; m < 2; ++m)
-                st_bf16x8(sm + OFF_UT + lh * 4096 + sw64_off(rr, 16 * hf + 8 * m), u + 8 * m);
+                st_bf16x8(sm + OFF_TT + sw128_off(128, 64 + r, 32 * hf + 8 * m), v + 8 * m);
         }
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
 
-        // ---------------------------------------------------------------- MMA: A_qk W, A_qk U~
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t idw = idesc_bf16(64, 64, 0, 1), idu = idesc_bf16(64, 32, 0, 1);
+        // ---------------------------------------------------------------- MMA: [T; T'] [K+ | V]
+        // one M=128, N=192 product: lanes 0-63 get W = T K+ and U~ = T V, lanes 64-127 get
+        // A_qk W = T' K+ and O~ = A_qk U~ = T' V
+        if (!wait_all(bar_v, c & 1)) { aborted = true; break; }
+        v_pending = false;
+        if (warp == 0) {
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 128 + kDV, 0, 1);
 #pragma unroll
-            for (int s = 0; s < kC / 16; ++s) {
-                const uint64_t ad = sw128_desc(sb + OFF_AQK + 32 * s, 16, 1024);
-                umma_f16(tbase + TM_W2, ad, sw128_desc(sb + OFF_W + 2048 * s, 8192, 1024), idw,
-                         s > 0);
-                umma_f16(tbase + TM_W2 + kLaneHi, ad,
-                         sw128_desc(sb + OFF_W + 8192 + 2048 * s, 8192, 1024), idw, s > 0);
-                umma_f16(tbase + TM_U2, ad, sw64_desc(sb + OFF_UT + 1024 * s, 4096, 512), idu,
-                         s > 0);
-                umma_f16(tbase + TM_U2 + kLaneHi, ad,
-                         sw64_desc(sb + OFF_UT + 4096 + 1024 * s, 4096, 512), idu, s > 0);
+                for (int s = 0; s < kC / 16; ++s)
+                    umma_f16(tbase + TM_A, desc_at(dK, sb + OFF_TT + 32 * s),
+                             desc_at(dM8, sb + OFF_KPV + 2048 * s), id, s > 0);
+                umma_commit(bar_mma);
             }
-            umma_commit(bar_mma);
+            __syncwarp();
         }
         mma_pending = true;
         if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
         ++mma_phase;
         mma_pending = false;
         tc_fence_after();
-        {
-            // Q~ = Q+ - A_qk W (in place on the Q+ tile)
-            float v[32];
-            tmem_ld32(tbase + lane_q + TM_W2 + 32 * hf, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                uint8_t* p = sm + OFF_QT + sw128_off(64, rr, 64 * lh + 32 * hf + 8 * m);
-                const uint4 qv = *reinterpret_cast<const uint4*>(p);
-                const float2 a0 = unpack_bf16(qv.x), a1 = unpack_bf16(qv.y);
-                const float2 a2 = unpack_bf16(qv.z), a3 = unpack_bf16(qv.w);
-                const float* w = v + 8 * m;
-                *reinterpret_cast<uint4*>(p) =
-                    make_uint4(pack_bf16(a0.x - w[0], a0.y - w[1]), pack_bf16(a1.x - w[2], a1.y - w[3]),
-                               pack_bf16(a2.x - w[4], a2.y - w[5]), pack_bf16(a3.x - w[6], a3.y - w[7]));
-            }
+        if (c + 1 < nchunks) {   // the V panel is free again
+            if (tid == 0) issue_v(c + 1);
+            v_pending = true;
+            v_chunk = c + 1;
         }
         {
-            // state: bf16 operand halves for W S and Q~ S, then decay the fp32 TMEM copy
+            // quarters 0-1: W rows -> [W; Q~] rows 0-63.  quarters 2-3: Q~ = Q+ - A_qk W in place.
+            // Each warp takes 64 of the 128 columns.
+            const int r = 32 * (qd & 1) + lane;
+            const int row = qd < 2 ? r : 64 + r;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const int c0 = 64 * hf + 32 * part;
+                float v[32];
+                tmem_ld32(tbase + lane_q + TM_A + c0, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    uint8_t* p = sm + OFF_WQ + sw128_off(128, row, c0 + 8 * m);
+                    const float* w = v + 8 * m;
+                    if (qd < 2) {
+                        st_bf16x8(p, w);
+                    } else {
+                        const uint4 qv = *reinterpret_cast<const uint4*>(p);
+                        const float2 a0 = unpack_bf16(qv.x), a1 = unpack_bf16(qv.y);
+                        const float2 a2 = unpack_bf16(qv.z), a3 = unpack_bf16(qv.w);
+                        *reinterpret_cast<uint4*>(p) = make_uint4(
+                            pack_bf16(a0.x - w[0], a0.y - w[1]), pack_bf16(a1.x - w[2], a1.y - w[3]),
+                            pack_bf16(a2.x - w[4], a2.y - w[5]), pack_bf16(a3.x - w[6], a3.y - w[7]));
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int p = 0; p < kHalfCols / 32; ++p) {
+            // state: bf16 operand for [W; Q~] S, then decay the fp32 TMEM copy
             float v[32];
             const int cc = 32 * qd + lane;
-            tmem_ld32(tbase + lane_q + TM_S + 32 * hf, v);
+            const int col = kHalfCols * hf + 32 * p;
+            tmem_ld32(tbase + lane_q + TM_S + col, v);
             tmem_ld_wait();
 #pragma unroll
             for (int m = 0; m < 4; ++m)
-                st_bf16x8(sm + OFF_S16 + hf * 8192 + sw64_off(cc, 8 * m), v + 8 * m);
+                st_bf16x8(sm + OFF_S16 + sw128_off(128, cc, col + 8 * m), v + 8 * m);
             const float dcy = decay_s[cc];
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] *= dcy;
-            tmem_st32(tbase + lane_q + TM_S + 32 * hf, v);
+            tmem_st32(tbase + lane_q + TM_S + col, v);
             tmem_st_wait();
         }
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
 
-        // ---------------------------------------------------------------- MMA: W S, Q~ S
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(64, 32, 0, 1);
+        // ---------------------------------------------------------------- MMA: [W; Q~] S
+        if (warp == 0) {
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, kDV, 0, 1);
 #pragma unroll
-            for (int s = 0; s < kD / 16; ++s) {
-                const int k0 = 16 * s;
-                const uint64_t aw =
-                    sw128_desc(sb + OFF_W + (k0 >> 6) * 8192 + (k0 & 63) * 2, 16, 1024);
-                const uint64_t aq =
-                    sw128_desc(sb + OFF_QT + (k0 >> 6) * 8192 + (k0 & 63) * 2, 16, 1024);
-                const uint64_t b0 = sw64_desc(sb + OFF_S16 + 1024 * s, 8192, 512);
-                const uint64_t b1 = sw64_desc(sb + OFF_S16 + 8192 + 1024 * s, 8192, 512);
-                umma_f16(tbase + TM_B, aw, b0, id, s > 0);
-                umma_f16(tbase + TM_B + kLaneHi, aw, b1, id, s > 0);
-                umma_f16(tbase + TM_B + 32, aq, b0, id, s > 0);
-                umma_f16(tbase + TM_B + 32 + kLaneHi, aq, b1, id, s > 0);
+                for (int s = 0; s < kD / 16; ++s) {
+                    const int k0 = 16 * s;
+                    umma_f16(tbase + TM_B,
+                             desc_at(dK, sb + OFF_WQ + (k0 >> 6) * 16384 + (k0 & 63) * 2),
+                             desc_at(dM16, sb + OFF_S16 + 2048 * s), id, s > 0);
+                }
+                umma_commit(bar_mma);
             }
-            umma_commit(bar_mma);
+            __syncwarp();
         }
         mma_pending = true;
         if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
         ++mma_phase;
         mma_pending = false;
         tc_fence_after();
-        {
+#pragma unroll
+        for (int p = 0; p < kHalfCols / 32; ++p) {
+            // quarters 0-1: U = U~ - W S (rows r, value columns col ..)
+            // quarters 2-3: o = O~ + Q~ S
+            const int r = 32 * (qd & 1) + lane;
+            const int col = kHalfCols * hf + 32 * p;
             float x[32], y[32];
-            if (hf == 0) {
-                // U = U~ - W S  (row rr, value columns 32 lh ..)
-                tmem_ld32(tbase + lane_q + TM_B, x);
-                tmem_ld32(tbase + lane_q + TM_U, y);
-                tmem_ld_wait();
+            tmem_ld32(tbase + lane_q + TM_B + col, x);
+            tmem_ld32(tbase + lane_q + TM_A + 128 + col, y);
+            tmem_ld_wait();
+            if (qd < 2) {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) y[j] -= x[j];
 #pragma unroll
                 for (int m = 0; m < 4; ++m)
-                    st_bf16x8(sm + OFF_U16 + sw128_off(64, rr, 32 * lh + 8 * m), y + 8 * m);
-            } else {
-                // o = O~ + Q~ S
-                tmem_ld32(tbase + lane_q + TM_B + 32, x);
-                tmem_ld32(tbase + lane_q + TM_U2, y);
-                tmem_ld_wait();
-                if (rr < L) {
+                    st_bf16x8(sm + OFF_U16 + sw128_off(64, r, col + 8 * m), y + 8 * m);
+            } else if (r < L) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) y[j] += x[j];
-                    uint4* dst = reinterpret_cast<uint4*>(
-                        args.o + ((size_t)(row0 + rr) * args.H + h) * kD + dv0 + 32 * lh);
+                for (int j = 0; j < 32; ++j) y[j] += x[j];
+                uint4* dst = reinterpret_cast<uint4*>(
+                    args.o + ((size_t)(row0 + r) * args.H + h) * kD + dv0 + col);
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        const float* w = y + 8 * m;
-                        dst[m] = make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]),
-                                            pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
-                    }
+                for (int m = 0; m < 4; ++m) {
+                    const float* w = y + 8 * m;
+                    dst[m] = make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]),
+                                        pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
                 }
             }
         }
@@ -770,16 +808,19 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         __syncthreads();
 
         // ---------------------------------------------------------------- MMA: S += K_end^T U
-        if (tid == 0) {
+        if (warp == 0) {   // lane 0 issues; the rest of warp 0 waits for it
+            if (lane == 0) {
             tc_fence_after();
-            const uint32_t id = idesc_bf16(128, 64, 1, 1);
+            const uint32_t id = idesc_bf16(128, kDV, 1, 1);
 #pragma unroll
             for (int s = 0; s < kC / 16; ++s) {
-                const uint64_t ae = sw128_desc(sb + OFF_KE + 2048 * s, 8192, 1024);
-                const uint64_t bu = sw128_desc(sb + OFF_U16 + 2048 * s, 8192, 1024);
+                const uint64_t ae = desc_at(dM8, sb + OFF_KE + 2048 * s);
+                const uint64_t bu = desc_at(dM8, sb + OFF_U16 + 2048 * s);
                 umma_f16(tbase + TM_S, ae, bu, id, 1);
             }
             umma_commit(bar_b4);
+            }
+            __syncwarp();
         }
         b4_pending = true;
         b4_chunk = c;
@@ -801,15 +842,19 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         tc_fence_after();
         if (args.hT) {
-            float v[32];
-            const int cc = 32 * qd + lane;
-            tmem_ld32(tbase + lane_q + TM_S + 32 * hf, v);
-            tmem_ld_wait();
-            float4* dst = reinterpret_cast<float4*>(args.hT + state_base + (size_t)cc * kD + dv0 +
-                                                    32 * hf);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            for (int p = 0; p < kHalfCols / 32; ++p) {
+                float v[32];
+                const int cc = 32 * qd + lane;
+                const int col = kHalfCols * hf + 32 * p;
+                tmem_ld32(tbase + lane_q + TM_S + col, v);
+                tmem_ld_wait();
+                float4* dst = reinterpret_cast<float4*>(args.hT + state_base + (size_t)cc * kD +
+                                                        dv0 + col);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
         }
     }
     tc_fence_before();
@@ -821,8 +866,6 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
-bool g_attr_set = false;
-std::mutex g_attr_mu;
 
 cudaError_t get_encoder() {
     std::call_once(g_encode_once, [] {
@@ -870,41 +913,22 @@ long long wait_budget() {
     return budget;
 }
 
-}  // namespace
-
-// Compiled in for sm_100a. Availability of the driver's tensor-map encoder is checked at launch
-// (a missing encoder surfaces as a CUDA error there), so path selection stays host-only.
-bool chunk64_available() { return true; }
-
-cudaError_t launch_chunk64(const FwdParams& p, cudaStream_t stream) {
-    cudaError_t e = get_encoder();
+template <int DV>
+cudaError_t launch_width(const FwdParams& p, cudaStream_t stream, const CUtensorMap& mq,
+                         const CUtensorMap& mk, const CUtensorMap& mg, int units) {
+    using Lay = Layout<DV>;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(chunk64_kernel<DV>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)Lay::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    CUtensorMap mv;
+    cudaError_t e = make_map(&mv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B * p.T, p.H, 64,
+                             CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
-    const int rows = p.B * p.T;
-    const int units = p.N * p.H;
-    if (units == 0) return cudaSuccess;
-    if (rows <= 0) {
-        // no tokens: hT = h0 (or zero); the per-token launcher handles it without TMA
-        return launch_recurrent(p, stream);
-    }
-    CUtensorMap mq, mk, mg, mv;
-    if ((e = make_map(&mq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, kD,
-                      CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
-        (e = make_map(&mk, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, kD,
-                      CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
-        (e = make_map(&mg, p.log_g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, p.H, kD,
-                      CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
-        (e = make_map(&mv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, 32,
-                      CU_TENSOR_MAP_SWIZZLE_64B)) != cudaSuccess)
-        return e;
-    {
-        std::lock_guard<std::mutex> lock(g_attr_mu);
-        if (!g_attr_set) {
-            e = cudaFuncSetAttribute(chunk64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)kSmemBytes);
-            if (e != cudaSuccess) return e;
-            g_attr_set = true;
-        }
-    }
     ChunkArgs a;
     a.beta = static_cast<const __nv_bfloat16*>(p.beta);
     a.h0 = p.h0;
@@ -917,10 +941,58 @@ cudaError_t launch_chunk64(const FwdParams& p, cudaStream_t stream) {
     a.budget = wait_budget();
     a.debug_stall = debug_stall();
     a.err = p.err;
-    const long long grid = (long long)units * kSplit;
+    const long long grid = (long long)units * Lay::kSplit;
     if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
-    chunk64_kernel<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(mq, mk, mg, mv, a);
+    chunk64_kernel<DV><<<(unsigned)grid, kThreads, Lay::kSmemBytes, stream>>>(mq, mk, mg, mv, a);
     return cudaGetLastError();
+}
+
+int sm_count() {
+    static int n = [] {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return 148;
+        return v;
+    }();
+    return n;
+}
+
+}  // namespace
+
+// Compiled in for sm_100a. Availability of the driver's tensor-map encoder is checked at launch
+// (a missing encoder surfaces as a CUDA error there), so path selection stays host-only.
+bool chunk64_available() { return true; }
+
+// One CTA per (sequence, head) owning all 128 value columns when there are enough chains to
+// fill the GPU (units > SMs / 2); otherwise two CTAs per chain, 64 value columns each, so that
+// twice as many SMs work on few long sequences.
+cudaError_t launch_chunk64(const FwdParams& p, cudaStream_t stream) {
+    cudaError_t e = get_encoder();
+    if (e != cudaSuccess) return e;
+    const int rows = p.B * p.T;
+    const int units = p.N * p.H;
+    if (units == 0) return cudaSuccess;
+    if (rows <= 0) {
+        // no tokens: hT = h0 (or zero); the per-token launcher handles it without TMA
+        return launch_recurrent(p, stream);
+    }
+    CUtensorMap mq, mk, mg;
+    if ((e = make_map(&mq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, kD,
+                      CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
+        (e = make_map(&mk, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, kD,
+                      CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
+        (e = make_map(&mg, p.log_g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, p.H, kD,
+                      CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess)
+        return e;
+    const int width = chunk64_value_width(p.N, p.H);
+    return width == 128 ? launch_width<128>(p, stream, mq, mk, mg, units)
+                        : launch_width<64>(p, stream, mq, mk, mg, units);
+}
+
+int chunk64_value_width(int N, int H) {
+    const long long units = (long long)N * H;
+    return units * 2 > sm_count() ? 128 : 64;
 }
 
 }  // namespace kda

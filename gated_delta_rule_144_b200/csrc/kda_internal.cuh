@@ -53,6 +53,8 @@ cudaError_t launch_recurrent(const FwdParams& p, cudaStream_t stream);
 cudaError_t launch_decode_d128(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_chunk64(const FwdParams& p, cudaStream_t stream);
 bool chunk64_available();
+// Value columns one chunked-kernel CTA owns for N sequences x H heads (64 or 128).
+int chunk64_value_width(int N, int H);
 
 // Element loads shared by the CUDA-core kernels.
 __device__ __forceinline__ float load_elem(const float* p, int64_t i) { return p[i]; }

@@ -195,6 +195,13 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo, uint
     return d;
 }
 
+// Descriptor from a precomputed constant part: `hi_lbo` holds everything but the start address
+// (sw128_desc(0, lbo, sbo) or sw64_desc(0, lbo, sbo)); the start address (< 256 KB) never
+// carries into the neighbouring fields, so one add builds the descriptor.
+__device__ __forceinline__ uint64_t desc_at(uint64_t hi_lbo, uint32_t addr) {
+    return hi_lbo + (uint64_t)(addr >> 4);
+}
+
 // Same with 64-byte swizzle (8-row atoms of 512 bytes; 32 bf16 per row).
 __device__ __forceinline__ uint64_t sw64_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
     uint64_t d = 0;

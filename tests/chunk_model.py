@@ -112,7 +112,7 @@ def chunk_step(q, k, v, lg, beta, S, L, bf=False, only=None):
             rows = slice(b_blk * BLK, (b_blk + 1) * BLK)
             dst = 64 + CROSS_OFF[a_blk] + b_blk * BLK
             Cm[dst:dst + BLK] = k[rows] * f["sig"][rows] * cross_factor(f, a_blk, b_blk)
-    D = R_("RC")(R) @ R_("RC")(Cm).T                                              # [128, 160] fp32 acc
+    D = (bf16(R) @ bf16(Cm).T) if only == "stacked" else R_("RC")(R) @ R_("RC")(Cm).T                                              # [128, 160] fp32 acc
     Akk = np.zeros((64, 64))
     Aqk = np.zeros((64, 64))
     for r in range(64):
@@ -142,6 +142,21 @@ def chunk_step(q, k, v, lg, beta, S, L, bf=False, only=None):
     Qp = q * eG
     Kend = k * f["sig"] * G[blk_of]
     decay = F[3] * P[3]
+    if only is not None and not isinstance(only, (set, dict)) and only == "stacked":
+        # the kernel's association: T' = A_qk T (bf16 operands, rounded to bf16), then
+        # [W; A_qk W] = [T; T'] K+ and [U~; O~] = [T; T'] V in one product
+        Tb = bf16(Tm)
+        Tp = bf16(bf16(Aqk) @ Tb)
+        W = Tb @ bf16(Kp)
+        Ut = Tb @ v
+        Wb = bf16(W)
+        Qt = bf16(Qp) - Tp @ bf16(Kp)
+        Ot = Tp @ v
+        Sb = bf16(S)
+        U = Ut - Wb @ Sb
+        O = Ot + bf16(Qt) @ Sb
+        S = decay[:, None] * S + bf16(Kend).T @ bf16(U)
+        return O[:L], S
     W = R_("T")(Tm) @ R_("Kp")(Kp)
     Ut = R_("T")(Tm) @ v
     Wb = R_("W")(W)

@@ -64,6 +64,13 @@ def test_ragged_lengths(T):
     _check(synth.prefill_inputs("long-t65536", B=1, T=T, H=2, seed=13 + T))
 
 
+@pytest.mark.parametrize("B,T,H", [(4, 200, 64), (2, 129, 128)])
+def test_many_chains_take_the_full_width_path(B, T, H):
+    """With more (sequence, head) chains than half the SMs, one CTA owns all 128 value columns
+    of a chain; check that variant with h0, batches and ragged lengths."""
+    _check(synth.prefill_inputs("prefill-t4096", B=B, T=T, H=H, h0_std=0.05, seed=17 + T))
+
+
 def test_prefill_t4096_h16_full():
     """The T=4096, H=16 bf16 workload at full size."""
     _check(synth.prefill_inputs("prefill-t4096"))
