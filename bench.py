@@ -182,27 +182,19 @@ def time_launches(fn, steps, stream):
 
 
 def max_over_ranks(x: float, world: int, device):
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from gated_delta_rule_144_b200 import shard
+    return shard.max_over_ranks(x, device) if world > 1 else x
 
 
 def sum_over_ranks(x: float, world: int, device):
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    from gated_delta_rule_144_b200 import shard
+    return shard.sum_over_ranks(x, device) if world > 1 else x
 
 
 def barrier(world):
     if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+        from gated_delta_rule_144_b200 import shard
+        shard.barrier()
 
 
 # ------------------------------------------------------------------------------ our arm
@@ -230,7 +222,8 @@ def run_ours(args):
     wl = synth.WORKLOADS[args.workload]
 
     # ---- headline: prefill on the workload, one batch per rank
-    inp = synth.prefill_inputs(wl, device=dev, seed=1000 + wl.index + 7919 * rank)
+    from gated_delta_rule_144_b200 import shard
+    inp = synth.prefill_inputs(wl, device=dev, seed=shard.rank_seed(1000 + wl.index, rank))
     B, T, H, dk, dv, N = inp["B"], inp["T"], inp["H"], inp["dk"], inp["dv"], inp["N"]
     o = torch.empty((B, T, H, dv), dtype=inp["q"].dtype, device=dev)
     hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
@@ -348,7 +341,8 @@ def run_secondary(kda, synth, args, dev, stream, world, rank):
     out = {}
     hbm_peak, _, _ = measured_peaks()
     # decode: 256 sequences x 32 heads, fp32 128x128 state updated in place every step
-    d = synth.decode_inputs("decode-n256", device=dev, seed=1003 + 7919 * rank)
+    from gated_delta_rule_144_b200 import shard
+    d = synth.decode_inputs("decode-n256", device=dev, seed=shard.rank_seed(1003, rank))
     od = torch.empty_like(d["v"])
 
     def dstep():
@@ -375,7 +369,7 @@ def run_secondary(kda, synth, args, dev, stream, world, rank):
                      "traffic": committed_traffic("kda_decode_d128", "decode-n256")}
     del d, od
     # packed 8-document prefill (H = 32)
-    p = synth.prefill_inputs("packed-8docs", device=dev, seed=1002 + 7919 * rank)
+    p = synth.prefill_inputs("packed-8docs", device=dev, seed=shard.rank_seed(1002, rank))
     o = torch.empty_like(p["v"])
     hT = torch.empty((p["N"], p["H"], 128, 128), dtype=torch.float32, device=dev)
 

@@ -99,16 +99,23 @@ typedef struct {
  *
  * The chunked path (KDA_CHUNK_64) computes in bf16 tensor-core products with fp32 accumulation
  * and an fp32 state. Its within-chunk factorisation needs the summed decay of any 8 consecutive
- * tokens of a 16-token sub-chunk to stay above -80 nats per key channel (e.g. log_g >= -10
- * everywhere); otherwise a factor would leave the float32 range. The kernel detects that case,
- * records KDA_ERR_RANGE in the device error word and still finishes; the per-token path
- * (KDA_CHUNK_PER_TOKEN) has no such limit.
+ * tokens inside a 16-token sub-chunk to stay above about -69 nats per key channel (e.g.
+ * log_g >= -8 everywhere); otherwise a factor would leave the float32 range. The kernel detects
+ * that case (a decay product below 1e-30), records KDA_ERR_RANGE in the device error word and
+ * still finishes; the per-token path (KDA_CHUNK_PER_TOKEN) has no such limit.
  * Returns KDA_OK once the work is enqueued. T = 0 or N = 0 is a valid no-op (hT = h0 or 0).
  */
 kda_status_t kda_fwd(const kda_fwd_desc_t* desc, const void* q, const void* k, const void* v,
                      const float* log_g, const void* beta, const float* h0,
                      const int32_t* cu_seqlens, void* o, float* hT, void* workspace,
                      size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * Path kda_fwd takes for `desc` (has_cu_seqlens: whether cu_seqlens will be non-NULL):
+ * KDA_CHUNK_PER_TOKEN or KDA_CHUNK_64, or the negated kda_status_t when the description is
+ * rejected. Host-only, no CUDA calls.
+ */
+int kda_fwd_algorithm(const kda_fwd_desc_t* desc, int has_cu_seqlens);
 
 /* Scratch bytes kda_fwd needs for `desc` (0 when it needs none). Host-only, no CUDA calls. */
 size_t kda_fwd_workspace_size(const kda_fwd_desc_t* desc);
