@@ -372,10 +372,13 @@ def run_secondary(kda, synth, args, dev, stream, world, rank):
     p = synth.prefill_inputs("packed-8docs", device=dev, seed=shard.rank_seed(1002, rank))
     o = torch.empty_like(p["v"])
     hT = torch.empty((p["N"], p["H"], 128, 128), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(1, kda.fwd_workspace_size(1, p["T"], p["H"], 128, 128, p["N"],
+                                                   torch.bfloat16, args.chunk_size)),
+                     dtype=torch.uint8, device=dev)
 
     def pstep():
         kda.fwd(p["q"], p["k"], p["v"], p["log_g"], p["beta"], cu_seqlens=p["cu_seqlens"],
-                o=o, hT=hT, chunk_size=args.chunk_size)
+                o=o, hT=hT, chunk_size=args.chunk_size, workspace=ws)
 
     for _ in range(max(3, args.warmup)):
         pstep()

@@ -133,9 +133,20 @@ int kda_fwd_algorithm(const kda_fwd_desc_t* desc, int has_cu_seqlens) {
     return path == Path::kChunk64 ? KDA_CHUNK_64 : KDA_CHUNK_PER_TOKEN;
 }
 
+// Packed documents on the chunked path are scheduled longest first; the permutation lives in the
+// caller's workspace (one int32 per document). Nothing else needs scratch.
+static size_t order_bytes(const kda_fwd_desc_t* d, Path path) {
+    const bool packed = d->B == 1 && d->num_seqs >= 2;  // without cu_seqlens num_seqs == B
+    if (path != Path::kChunk64 || !packed || d->num_seqs > kda::kMaxOrderedDocs) return 0;
+    return ((size_t)d->num_seqs * sizeof(int32_t) + 255) / 256 * 256;
+}
+
 size_t kda_fwd_workspace_size(const kda_fwd_desc_t* desc) {
-    (void)desc;
-    return 0;
+    Path path;
+    if (!desc || check_fwd_desc(desc, desc->B == 1 && desc->num_seqs >= 2, &path) != KDA_OK)
+        return 0;
+    t_last_error[0] = 0;
+    return order_bytes(desc, path);
 }
 
 kda_status_t kda_fwd(const kda_fwd_desc_t* d, const void* q, const void* k, const void* v,
@@ -143,8 +154,6 @@ kda_status_t kda_fwd(const kda_fwd_desc_t* d, const void* q, const void* k, cons
                      const int32_t* cu_seqlens, void* o, float* hT, void* workspace,
                      size_t workspace_bytes, kda_stream_t stream) {
     t_last_error[0] = 0;
-    (void)workspace;
-    (void)workspace_bytes;
     Path path;
     kda_status_t st = check_fwd_desc(d, cu_seqlens != nullptr, &path);
     if (st != KDA_OK) return st;
@@ -157,6 +166,11 @@ kda_status_t kda_fwd(const kda_fwd_desc_t* d, const void* q, const void* k, cons
         (st = check_ptr(cu_seqlens, "cu_seqlens", false)))
         return st;
     if (tokens && !beta) return fail(KDA_ERR_INVALID_ARG, "beta is NULL");
+    const size_t need_ws = cu_seqlens ? order_bytes(d, path) : 0;
+    if (need_ws > 0 && (workspace_bytes < need_ws || !workspace || !aligned16(workspace)))
+        return fail(KDA_ERR_INVALID_ARG,
+                    "workspace must be a 16-byte aligned device buffer of %zu bytes "
+                    "(kda_fwd_workspace_size)", need_ws);
     if (!has_units) return KDA_OK;
 
     kda::FwdParams p{};
@@ -164,10 +178,17 @@ kda_status_t kda_fwd(const kda_fwd_desc_t* d, const void* q, const void* k, cons
     p.cu_seqlens = cu_seqlens; p.o = o; p.hT = hT;
     p.B = d->B; p.T = d->T; p.H = d->H; p.dk = d->dk; p.dv = d->dv; p.N = d->num_seqs;
     p.bf16 = d->dtype == KDA_BF16;
+    p.doc_order = nullptr;
     if ((st = device_error_word(&p.err)) != KDA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = path == Path::kChunk64 ? kda::launch_chunk64(p, s)
-                                           : kda::launch_recurrent(p, s);
+    cudaError_t e = cudaSuccess;
+    if (need_ws > 0 && tokens) {
+        int32_t* order = static_cast<int32_t*>(workspace);
+        e = kda::launch_doc_order(cu_seqlens, d->num_seqs, order, s);
+        if (e != cudaSuccess) return cuda_fail(e, "kda_fwd document scheduling");
+        p.doc_order = order;
+    }
+    e = path == Path::kChunk64 ? kda::launch_chunk64(p, s) : kda::launch_recurrent(p, s);
     if (e != cudaSuccess) return cuda_fail(e, "kda_fwd launch");
     return KDA_OK;
 }

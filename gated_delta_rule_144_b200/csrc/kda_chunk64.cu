@@ -108,6 +108,7 @@ constexpr uint32_t kTxIn = 16384 + 16384 + 32768;
 __host__ __device__ constexpr int cross_off(int a) { return a == 1 ? 0 : (a == 2 ? 16 : 48); }
 
 struct ChunkArgs {
+    const int32_t* order;   // nullable: document taken by the k-th (document, head) group
     const __nv_bfloat16* beta;
     const float* h0;
     const int32_t* cu;
@@ -165,7 +166,8 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int qd = warp & 3, hf = warp >> 2;          // TMEM lane quarter, column half
     const int split = blockIdx.x % kSplit;
     const int unit = blockIdx.x / kSplit;
-    const int n = unit / args.H, h = unit % args.H;
+    const int h = unit % args.H;
+    const int n = args.order ? args.order[unit / args.H] : unit / args.H;
     const int dv0 = split * kDV;
 
     long long t0, t1;
@@ -930,6 +932,7 @@ cudaError_t launch_width(const FwdParams& p, cudaStream_t stream, const CUtensor
                              CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
     ChunkArgs a;
+    a.order = p.doc_order;
     a.beta = static_cast<const __nv_bfloat16*>(p.beta);
     a.h0 = p.h0;
     a.cu = p.cu_seqlens;

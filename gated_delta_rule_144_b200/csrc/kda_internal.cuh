@@ -33,6 +33,7 @@ struct FwdParams {
     int B, T, H, dk, dv, N;
     bool bf16;
     unsigned* err;            // device error word
+    const int32_t* doc_order;   // nullable: packed documents in the order CTAs should take them
 };
 
 struct DecodeParams {
@@ -48,7 +49,14 @@ struct DecodeParams {
     unsigned* err;
 };
 
+// Largest number of packed documents the chunked path schedules longest first (above it, CTAs
+// take documents in their packed order).
+constexpr int kMaxOrderedDocs = 2048;
+
 // Launchers (host). Each returns the launch status of its kernel(s).
+// Writes order[0..N) = document indices by decreasing length (ties: lower index first).
+cudaError_t launch_doc_order(const int32_t* cu_seqlens, int N, int32_t* order,
+                             cudaStream_t stream);
 cudaError_t launch_recurrent(const FwdParams& p, cudaStream_t stream);
 cudaError_t launch_decode_d128(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_chunk64(const FwdParams& p, cudaStream_t stream);

@@ -107,7 +107,26 @@ def test_decode_rejects_on_host(L):
 
 def test_workspace_size_is_host_only(L):
     d = _desc()
-    assert L.kda_fwd_workspace_size(ctypes.byref(d)) >= 0
+    assert L.kda_fwd_workspace_size(ctypes.byref(d)) == 0
+    # packed documents on the chunked path: one int32 per document, rounded to 256 bytes
+    d = _desc(num_seqs=8)
+    assert L.kda_fwd_workspace_size(ctypes.byref(d)) == 256
+    d = _desc(num_seqs=300)
+    assert L.kda_fwd_workspace_size(ctypes.byref(d)) == 1280
+    # the exact path needs none
+    d = _desc(num_seqs=8, chunk_size=1)
+    assert L.kda_fwd_workspace_size(ctypes.byref(d)) == 0
+
+
+def test_packed_chunked_call_without_workspace_is_rejected_on_host(L):
+    P = ctypes.c_void_p
+    d = _desc(num_seqs=8)
+    st = L.kda_fwd(ctypes.byref(d), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), None, P(FAKE),
+                   P(FAKE), None, None, 0, None)
+    assert st == 1 and b"workspace" in L.kda_last_error()
+    st = L.kda_fwd(ctypes.byref(d), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), None, P(FAKE),
+                   P(FAKE), None, P(FAKE + 8), 4096, None)   # misaligned workspace
+    assert st == 1 and b"workspace" in L.kda_last_error()
 
 
 def test_python_binding_refuses_cpu_tensors():

@@ -81,6 +81,12 @@ def test_packed_edge_documents():
     _check(synth.prefill_inputs("packed-8docs", lengths=lengths, H=4, h0_std=0.05, seed=14))
 
 
+def test_packed_documents_scheduled_longest_first():
+    """Documents in increasing length: the scheduling permutation is far from the identity."""
+    _check(synth.prefill_inputs("packed-8docs", lengths=[50, 100, 700, 1300, 2, 1301], H=8,
+                                h0_std=0.05, seed=18))
+
+
 def test_packed_8docs_full():
     """The packed 8-document workload (H = 32) at full size, every token and state."""
     _check(synth.prefill_inputs("packed-8docs"))
