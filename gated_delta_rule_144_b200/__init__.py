@@ -19,7 +19,8 @@ from pathlib import Path
 
 import torch
 
-__all__ = ["fwd", "decode_step", "get_device_error", "fwd_workspace_size", "fwd_algorithm",
+__all__ = ["fwd", "fwd_no_alloc", "decode_step", "get_device_error", "fwd_workspace_size",
+           "fwd_algorithm",
            "KdaError",
            "library_path", "lib", "CHUNK_AUTO", "CHUNK_PER_TOKEN", "CHUNK_64"]
 
@@ -64,6 +65,8 @@ def lib():
     p, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     L.kda_fwd.argtypes = [ctypes.POINTER(FwdDesc), p, p, p, p, p, p, p, p, p, p, sz, p]
     L.kda_fwd.restype = i32
+    L.kda_fwd_no_alloc.argtypes = [ctypes.POINTER(FwdDesc), p, p, p, p, p, p, p, p, p, p]
+    L.kda_fwd_no_alloc.restype = i32
     L.kda_fwd_algorithm.argtypes = [ctypes.POINTER(FwdDesc), i32]
     L.kda_fwd_algorithm.restype = i32
     L.kda_fwd_workspace_size.argtypes = [ctypes.POINTER(FwdDesc)]
@@ -197,6 +200,40 @@ def fwd(q, k, v, log_g, beta, h0=None, cu_seqlens=None, *, chunk_size: int = CHU
                            _ptr(beta), _ptr(h0), _ptr(cu_seqlens), _ptr(o), _ptr(hT),
                            _ptr(workspace), ws_bytes, _stream(stream, dev))
     _check(st, "kda_fwd")
+    return o, hT
+
+
+def fwd_no_alloc(q, k, v, log_g, beta, h0, cu_seqlens, o, hT, *, chunk_size: int = CHUNK_AUTO,
+                 stream=None):
+    """``kda_fwd_no_alloc``: the prefill without a workspace, for callers that cannot allocate.
+
+    Every buffer is the caller's: o [B, T, H, dv] and hT [N, H, dk, dv] (or None) must be passed
+    in, and nothing is allocated here or in the library (its scratch is a static device array of
+    KDA_NO_ALLOC_MAX_DOCS = 2048 document slots). Calls overlapping on one GPU race on that array.
+    Same layouts and results as ``fwd``.
+    """
+    lib()
+    _dev(q, "q")
+    dev = q.device
+    B, T, H, dk = q.shape
+    dt = q.dtype
+    _dev(k, "k", dt, (B, T, H, dk), dev)
+    _dev(log_g, "log_g", torch.float32, (B, T, H, dk), dev)
+    _dev(v, "v", dt, None, dev)
+    dv = v.shape[3]
+    _dev(beta, "beta", dt, (B, T, H), dev)
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if cu_seqlens is not None:
+        _dev(cu_seqlens, "cu_seqlens", torch.int32, None, dev)
+    _dev(h0, "h0", torch.float32, (N, H, dk, dv), dev)
+    _dev(o, "o", dt, (B, T, H, dv), dev)
+    _dev(hT, "hT", torch.float32, (N, H, dk, dv), dev)
+    desc = FwdDesc(B, T, H, dk, dv, N, _dtype_code(q), chunk_size)
+    with torch.cuda.device(dev):
+        st = lib().kda_fwd_no_alloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(log_g),
+                                    _ptr(beta), _ptr(h0), _ptr(cu_seqlens), _ptr(o), _ptr(hT),
+                                    _stream(stream, dev))
+    _check(st, "kda_fwd_no_alloc")
     return o, hT
 
 

@@ -107,6 +107,12 @@ kda_status_t check_fwd_desc(const kda_fwd_desc_t* d, bool has_cu, Path* path) {
 
 }  // namespace
 
+namespace kda {
+void set_last_error(const char* msg) {
+    snprintf(t_last_error, sizeof(t_last_error), "%s", msg);
+}
+}  // namespace kda
+
 extern "C" {
 
 int kda_version(void) { return 100; }

@@ -53,6 +53,9 @@ struct DecodeParams {
 // take documents in their packed order).
 constexpr int kMaxOrderedDocs = 2048;
 
+// Record the text kda_last_error() returns on this host thread.
+void set_last_error(const char* msg);
+
 // Launchers (host). Each returns the launch status of its kernel(s).
 // Writes order[0..N) = document indices by decreasing length (ties: lower index first).
 cudaError_t launch_doc_order(const int32_t* cu_seqlens, int N, int32_t* order,

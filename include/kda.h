@@ -121,6 +121,36 @@ int kda_fwd_algorithm(const kda_fwd_desc_t* desc, int has_cu_seqlens);
 size_t kda_fwd_workspace_size(const kda_fwd_desc_t* desc);
 
 /*
+ * kda_fwd_no_alloc - kda_fwd for callers that cannot allocate device memory.
+ *
+ * The source pages have no counterpart for this entry point. It exists for callers that cannot
+ * call cudaMalloc, or any allocator, when they run the prefill. Examples: an engine that reserves
+ * all device memory at start-up and hands kernels only fixed buffers; a plugin host that exposes
+ * no allocator; a serving loop that may not allocate (an allocation can synchronise the device
+ * or fail under memory pressure).
+ *
+ * Same arguments as kda_fwd, without the workspace. The caller still passes every input and
+ * output buffer. The scratch kda_fwd would take from the workspace comes from a static device
+ * array built into the library: KDA_NO_ALLOC_MAX_DOCS int32 document slots (8 KiB), held by
+ * every GPU that loads the library until the process exits. A packed call (cu_seqlens != NULL)
+ * with more documents than that returns KDA_ERR_INVALID_ARG before anything is launched.
+ *
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current. Make that first call before any stream capture.
+ *
+ * All calls on a device share the one array, which keeps the last call's contents. Every call
+ * rewrites the slots it uses before reading them, so nothing needs to start at zero. Calls that
+ * overlap on the GPU (concurrent streams, or several host threads) race on the array: serialise
+ * them, or use kda_fwd with a workspace per stream. Results equal kda_fwd's.
+ * This function allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define KDA_NO_ALLOC_MAX_DOCS 2048
+kda_status_t kda_fwd_no_alloc(const kda_fwd_desc_t* desc, const void* q, const void* k,
+                              const void* v, const float* log_g, const void* beta,
+                              const float* h0, const int32_t* cu_seqlens, void* o, float* hT,
+                              kda_stream_t stream);
+
+/*
  * kda_decode_step - advance N sequences by one token each, updating the state in place.
  *
  *   q, k, log_g : [N, H, dk] (q, k in dtype, log_g float32)    v, o : [N, H, dv] dtype

@@ -129,6 +129,14 @@ def test_packed_chunked_call_without_workspace_is_rejected_on_host(L):
     assert st == 1 and b"workspace" in L.kda_last_error()
 
 
+def test_no_alloc_entry_rejects_more_documents_than_its_scratch_on_host(L):
+    P = ctypes.c_void_p
+    d = _desc(num_seqs=2049)
+    st = L.kda_fwd_no_alloc(ctypes.byref(d), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), None,
+                            P(FAKE), P(FAKE), None, None)
+    assert st == 1 and b"2048" in L.kda_last_error()
+
+
 def test_python_binding_refuses_cpu_tensors():
     import torch
     q = torch.zeros(1, 4, 1, 8)
