@@ -205,6 +205,13 @@ def prefill_bytes(inp) -> int:
     return th * BYTES_PER_TOKEN_HEAD + states * (2 if inp["h0"] is not None else 1)
 
 
+def workspace_for(kda, B, T, H, N, args, dev):
+    """The call's workspace, allocated once outside the timed region (None when 0 bytes)."""
+    size = (kda.fwd_workspace_size_min if args.fused else kda.fwd_workspace_size)(
+        B, T, H, 128, 128, N, torch.bfloat16, args.chunk_size)
+    return torch.empty(size, dtype=torch.uint8, device=dev) if size > 0 else None
+
+
 def run_ours(args):
     import gated_delta_rule_144_b200 as kda
     from gated_delta_rule_144_b200 import synth
@@ -227,10 +234,12 @@ def run_ours(args):
     B, T, H, dk, dv, N = inp["B"], inp["T"], inp["H"], inp["dk"], inp["dv"], inp["N"]
     o = torch.empty((B, T, H, dv), dtype=inp["q"].dtype, device=dev)
     hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    ws = workspace_for(kda, B, T, H, N, args, dev)
 
     def step():
         kda.fwd(inp["q"], inp["k"], inp["v"], inp["log_g"], inp["beta"], h0=inp["h0"],
-                cu_seqlens=inp["cu_seqlens"], o=o, hT=hT, chunk_size=args.chunk_size)
+                cu_seqlens=inp["cu_seqlens"], o=o, hT=hT, chunk_size=args.chunk_size,
+                workspace=ws, fused=args.fused)
 
     for _ in range(args.warmup):
         step()
@@ -259,7 +268,14 @@ def run_ours(args):
     achieved = bytes_launch / (launch_ms / 1e3) / 1e9
     algo = kda.fwd_algorithm(B, T, H, dk, dv, N, inp["q"].dtype, args.chunk_size,
                              varlen=inp["cu_seqlens"] is not None)
-    kernel_name = "kda_chunk64" if algo == kda.CHUNK_64 else "kda_recurrent"
+    packed = inp["cu_seqlens"] is not None
+    if algo != kda.CHUNK_64:
+        kernel_name, launches = "kda_recurrent", 1
+    elif args.fused:
+        kernel_name, launches = "kda_chunk64", 1 + (1 if packed and 2 <= N <= 2048 else 0)
+    else:   # split: intra-chunk kernel + state pass (+ chunk map and document order if packed)
+        kernel_name = "kda_chunk64_intra+kda_chunk_scan"
+        launches = 2 + ((2 if 2 <= N <= 2048 else 1) if packed else 0)
     traffic = committed_traffic(kernel_name, wl.name)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                 "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
@@ -292,7 +308,7 @@ def run_ours(args):
                        "log_g": "-softplus(N(%g,1))" % wl.decay_mu,
                        "parallelism": "dp%d" % world, "l2": "inputs larger than L2",
                        "chunk_size": args.chunk_size, "path": kernel_name},
-            "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
+            "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps * launches,
             "clocks": clk, "cpu_baseline": cpu, "secondary": secondary,
         }
         print(json.dumps(line), flush=True)
@@ -309,6 +325,7 @@ def run_e2e(kda, inp, args, stream, world, dev):
     B, T, H, dv, N, dk = inp["B"], inp["T"], inp["H"], inp["dv"], inp["N"], inp["dk"]
     o = torch.empty((B, T, H, dv), dtype=inp["q"].dtype, device=dev)
     hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    ws = workspace_for(kda, B, T, H, N, args, dev)
     o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     hT_h = torch.empty(hT.shape, dtype=hT.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
@@ -319,7 +336,8 @@ def run_e2e(kda, inp, args, stream, world, dev):
             if host[k] is not None:
                 d_in[k].copy_(host[k], non_blocking=True)
         kda.fwd(d_in["q"], d_in["k"], d_in["v"], d_in["log_g"], d_in["beta"], h0=d_in["h0"],
-                cu_seqlens=d_in["cu_seqlens"], o=o, hT=hT, chunk_size=args.chunk_size)
+                cu_seqlens=d_in["cu_seqlens"], o=o, hT=hT, chunk_size=args.chunk_size,
+                workspace=ws, fused=args.fused)
         o_h.copy_(o, non_blocking=True)
         hT_h.copy_(hT, non_blocking=True)
 
@@ -372,13 +390,11 @@ def run_secondary(kda, synth, args, dev, stream, world, rank):
     p = synth.prefill_inputs("packed-8docs", device=dev, seed=shard.rank_seed(1002, rank))
     o = torch.empty_like(p["v"])
     hT = torch.empty((p["N"], p["H"], 128, 128), dtype=torch.float32, device=dev)
-    ws = torch.empty(max(1, kda.fwd_workspace_size(1, p["T"], p["H"], 128, 128, p["N"],
-                                                   torch.bfloat16, args.chunk_size)),
-                     dtype=torch.uint8, device=dev)
+    ws = workspace_for(kda, 1, p["T"], p["H"], p["N"], args, dev)
 
     def pstep():
         kda.fwd(p["q"], p["k"], p["v"], p["log_g"], p["beta"], cu_seqlens=p["cu_seqlens"],
-                o=o, hT=hT, chunk_size=args.chunk_size, workspace=ws)
+                o=o, hT=hT, chunk_size=args.chunk_size, workspace=ws, fused=args.fused)
 
     for _ in range(max(3, args.warmup)):
         pstep()
@@ -468,8 +484,10 @@ def run_profile_case(args):
         name = args.workload if args.profile_case == "prefill" else "packed-8docs"
         kw = {} if args.profile_tokens <= 0 else {"T": args.profile_tokens}
         p = synth.prefill_inputs(name, device=dev, **kw)
+        ws = workspace_for(kda, p["B"], p["T"], p["H"], p["N"], args, dev)
         fn = lambda: kda.fwd(p["q"], p["k"], p["v"], p["log_g"], p["beta"], h0=p["h0"],
-                             cu_seqlens=p["cu_seqlens"], chunk_size=args.chunk_size)
+                             cu_seqlens=p["cu_seqlens"], chunk_size=args.chunk_size,
+                             workspace=ws, fused=args.fused)
     for _ in range(args.warmup + args.steps):
         fn()
     torch.cuda.synchronize()
@@ -488,6 +506,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long-t65536")
     ap.add_argument("--chunk-size", type=int, default=0)
+    ap.add_argument("--fused", action="store_true",
+                    help="run the fused chunked kernel (minimum workspace) instead of the split path")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-tokens", type=int, default=32768)
     ap.add_argument("--ref-tokens", type=int, default=4096)

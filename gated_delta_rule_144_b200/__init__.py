@@ -20,7 +20,7 @@ from pathlib import Path
 import torch
 
 __all__ = ["fwd", "fwd_no_alloc", "decode_step", "get_device_error", "fwd_workspace_size",
-           "fwd_algorithm",
+           "fwd_workspace_size_min", "fwd_algorithm",
            "KdaError",
            "library_path", "lib", "CHUNK_AUTO", "CHUNK_PER_TOKEN", "CHUNK_64"]
 
@@ -71,6 +71,8 @@ def lib():
     L.kda_fwd_algorithm.restype = i32
     L.kda_fwd_workspace_size.argtypes = [ctypes.POINTER(FwdDesc)]
     L.kda_fwd_workspace_size.restype = sz
+    L.kda_fwd_workspace_size_min.argtypes = [ctypes.POINTER(FwdDesc)]
+    L.kda_fwd_workspace_size_min.restype = sz
     L.kda_decode_step.argtypes = [i32, i32, i32, i32, i32, p, p, p, p, p, p, p, p]
     L.kda_decode_step.restype = i32
     L.kda_get_device_error.argtypes = [p]
@@ -137,6 +139,13 @@ def fwd_algorithm(B, T, H, dk, dv, num_seqs, dtype=torch.bfloat16, chunk_size=0,
     return r
 
 
+def fwd_workspace_size_min(B, T, H, dk, dv, num_seqs, dtype=torch.bfloat16, chunk_size=0) -> int:
+    """Smallest workspace kda_fwd accepts (the fused chunked path's document order)."""
+    d = FwdDesc(B, T, H, dk, dv, num_seqs, KDA_BF16 if dtype == torch.bfloat16 else KDA_F32,
+                chunk_size)
+    return int(lib().kda_fwd_workspace_size_min(ctypes.byref(d)))
+
+
 def fwd_workspace_size(B, T, H, dk, dv, num_seqs, dtype=torch.bfloat16, chunk_size=0) -> int:
     d = FwdDesc(B, T, H, dk, dv, num_seqs, KDA_BF16 if dtype == torch.bfloat16 else KDA_F32,
                 chunk_size)
@@ -144,13 +153,16 @@ def fwd_workspace_size(B, T, H, dk, dv, num_seqs, dtype=torch.bfloat16, chunk_si
 
 
 def fwd(q, k, v, log_g, beta, h0=None, cu_seqlens=None, *, chunk_size: int = CHUNK_AUTO,
-        output_final_state: bool = True, o=None, hT=None, workspace=None, stream=None):
+        output_final_state: bool = True, o=None, hT=None, workspace=None, fused: bool = False,
+        stream=None):
     """Prefill (``kda_fwd``): the recurrence over whole sequences or packed documents.
 
     q, k, log_g: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H]; q/k/v/beta share one dtype
     (bf16 or fp32), log_g is fp32. h0: [N, H, dk, dv] fp32 or None. cu_seqlens: int32 [N + 1]
     on the device (B must be 1) or None. Returns (o [B, T, H, dv], hT [N, H, dk, dv] fp32 or
-    None). Outputs may be passed in preallocated.
+    None). Outputs may be passed in preallocated. The workspace (a uint8 device tensor) is
+    allocated here when not given: kda_fwd_workspace_size bytes (the split chunked path), or,
+    with fused=True, only kda_fwd_workspace_size_min bytes (the fused chunked kernel).
     """
     lib()
     _dev(q, "q")
@@ -187,7 +199,8 @@ def fwd(q, k, v, log_g, beta, h0=None, cu_seqlens=None, *, chunk_size: int = CHU
     else:
         hT = None
     desc = FwdDesc(B, T, H, dk, dv, N, _dtype_code(q), chunk_size)
-    need = int(lib().kda_fwd_workspace_size(ctypes.byref(desc)))
+    need = int((lib().kda_fwd_workspace_size_min if fused else lib().kda_fwd_workspace_size)(
+        ctypes.byref(desc)))
     if need > 0:
         if workspace is None:
             workspace = torch.empty(need, dtype=torch.uint8, device=dev)
@@ -210,7 +223,7 @@ def fwd_no_alloc(q, k, v, log_g, beta, h0, cu_seqlens, o, hT, *, chunk_size: int
     Every buffer is the caller's: o [B, T, H, dv] and hT [N, H, dk, dv] (or None) must be passed
     in, and nothing is allocated here or in the library (its scratch is a static device array of
     KDA_NO_ALLOC_MAX_DOCS = 2048 document slots). Calls overlapping on one GPU race on that array.
-    Same layouts and results as ``fwd``.
+    Same layouts as ``fwd``; the same results as ``fwd(..., fused=True)``.
     """
     lib()
     _dev(q, "q")

@@ -147,7 +147,50 @@ static size_t order_bytes(const kda_fwd_desc_t* d, Path path) {
     return ((size_t)d->num_seqs * sizeof(int32_t) + 255) / 256 * 256;
 }
 
+// Workspace of the split chunked path (intra-chunk kernel + state pass), 256-byte aligned parts.
+struct SplitLayout {
+    size_t order, map, decay, wq, ke, ut, ot, total;
+    long long G;
+    int ncT;
+    bool has_order;
+};
+
+static size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+// packed: the call passes cu_seqlens (records are indexed floor(t0 / 64) + document + chunk).
+static bool split_layout(const kda_fwd_desc_t* d, Path path, bool packed, SplitLayout* L) {
+    if (path != Path::kChunk64 || d->T <= 0 || d->num_seqs <= 0) return false;
+    L->ncT = (d->T + 63) / 64;
+    L->G = packed ? (long long)L->ncT + d->num_seqs : (long long)d->B * L->ncT;
+    const long long R = L->G * d->H;
+    if (R * 128 > 0x7fffffffLL) return false;   // TMA row coordinates are 32-bit
+    L->has_order = packed && d->num_seqs >= 2 && d->num_seqs <= kda::kMaxOrderedDocs;
+    size_t off = 0;
+    L->order = off; off += L->has_order ? up256((size_t)d->num_seqs * 4) : 0;
+    L->map = off;   off += packed ? up256((size_t)L->G * 4) : 0;
+    L->decay = off; off += up256((size_t)R * 512);
+    L->wq = off;    off += (size_t)R * 32768;
+    L->ke = off;    off += (size_t)R * 16384;
+    L->ut = off;    off += (size_t)R * 16384;
+    L->ot = off;    off += (size_t)R * 16384;
+    L->total = off;
+    return true;
+}
+
 size_t kda_fwd_workspace_size(const kda_fwd_desc_t* desc) {
+    Path path;
+    const bool maybe_packed = desc && desc->B == 1;
+    if (!desc || check_fwd_desc(desc, maybe_packed && desc->num_seqs >= 2, &path) != KDA_OK)
+        return 0;
+    t_last_error[0] = 0;
+    SplitLayout L;
+    // B == 1 may come with cu_seqlens: size for the packed record numbering (one record more
+    // per document than a single sequence needs)
+    if (split_layout(desc, path, maybe_packed, &L)) return L.total;
+    return order_bytes(desc, path);
+}
+
+size_t kda_fwd_workspace_size_min(const kda_fwd_desc_t* desc) {
     Path path;
     if (!desc || check_fwd_desc(desc, desc->B == 1 && desc->num_seqs >= 2, &path) != KDA_OK)
         return 0;
@@ -172,7 +215,10 @@ kda_status_t kda_fwd(const kda_fwd_desc_t* d, const void* q, const void* k, cons
         (st = check_ptr(cu_seqlens, "cu_seqlens", false)))
         return st;
     if (tokens && !beta) return fail(KDA_ERR_INVALID_ARG, "beta is NULL");
-    const size_t need_ws = cu_seqlens ? order_bytes(d, path) : 0;
+    SplitLayout L;
+    const bool split = tokens && split_layout(d, path, cu_seqlens != nullptr, &L) && workspace &&
+                       aligned16(workspace) && workspace_bytes >= L.total;
+    const size_t need_ws = (cu_seqlens && !split) ? order_bytes(d, path) : 0;
     if (need_ws > 0 && (workspace_bytes < need_ws || !workspace || !aligned16(workspace)))
         return fail(KDA_ERR_INVALID_ARG,
                     "workspace must be a 16-byte aligned device buffer of %zu bytes "
@@ -188,6 +234,34 @@ kda_status_t kda_fwd(const kda_fwd_desc_t* d, const void* q, const void* k, cons
     if ((st = device_error_word(&p.err)) != KDA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
+    if (split) {
+        uint8_t* w = static_cast<uint8_t*>(workspace);
+        kda::SplitWorkspace ws;
+        ws.wq = reinterpret_cast<__nv_bfloat16*>(w + L.wq);
+        ws.ke = reinterpret_cast<__nv_bfloat16*>(w + L.ke);
+        ws.ut = reinterpret_cast<__nv_bfloat16*>(w + L.ut);
+        ws.ot = reinterpret_cast<__nv_bfloat16*>(w + L.ot);
+        ws.decay = reinterpret_cast<float*>(w + L.decay);
+        ws.map = cu_seqlens ? reinterpret_cast<int32_t*>(w + L.map) : nullptr;
+        ws.G = L.G;
+        ws.ncT = L.ncT;
+        p.split = &ws;
+        if (L.has_order) {
+            int32_t* order = reinterpret_cast<int32_t*>(w + L.order);
+            e = kda::launch_doc_order(cu_seqlens, d->num_seqs, order, s);
+            if (e != cudaSuccess) return cuda_fail(e, "kda_fwd document scheduling");
+            p.doc_order = order;
+        }
+        if (cu_seqlens) {
+            e = kda::launch_chunk_map(cu_seqlens, d->num_seqs, d->T, L.G, ws.map, p.err, s);
+            if (e != cudaSuccess) return cuda_fail(e, "kda_fwd chunk map");
+        }
+        e = kda::launch_chunk64_intra(p, s);
+        if (e != cudaSuccess) return cuda_fail(e, "kda_fwd intra-chunk launch");
+        e = kda::launch_chunk_scan(p, s);
+        if (e != cudaSuccess) return cuda_fail(e, "kda_fwd state-pass launch");
+        return KDA_OK;
+    }
     if (need_ws > 0 && tokens) {
         int32_t* order = static_cast<int32_t*>(workspace);
         e = kda::launch_doc_order(cu_seqlens, d->num_seqs, order, s);

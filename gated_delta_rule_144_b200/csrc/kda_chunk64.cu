@@ -37,10 +37,12 @@
 #include <cudaTypedefs.h>
 
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "kda_internal.cuh"
 #include "kda_sm100.cuh"
+#include "kda_tma.cuh"
 
 namespace kda {
 namespace {
@@ -85,7 +87,7 @@ struct Layout {
     static constexpr uint32_t OFF_TMEM = OFF_BAR + 64;     // TMEM base address
     static constexpr uint32_t kSmemBytes = OFF_TMEM + 16 + 1024;  // + alignment slack
     static_assert(OFF_ZA + 16384 == OFF_C + 40960, "solve buffers fill the R/C region exactly");
-    static_assert(OFF_YS + 3 * 16 * 17 * 4 <= OFF_TT, "solve scratch overlaps [T; T']");
+    static_assert(OFF_YS + 4 * 16 * 17 * 4 <= OFF_TT, "solve scratch overlaps [T; T']");
     static_assert(OFF_U16 + 8192u * kPanels <= OFF_C + 40960, "state-step tiles overflow");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     // TMEM columns (fp32, 128 lanes; M=128 layout: row m of a product sits in lane m)
@@ -109,6 +111,12 @@ __host__ __device__ constexpr int cross_off(int a) { return a == 1 ? 0 : (a == 2
 
 struct ChunkArgs {
     const int32_t* order;   // nullable: document taken by the k-th (document, head) group
+    // intra mode: chunk records (g, head) with g = sequence * ncT + chunk, or, for packed
+    // documents, g = floor(t0 / 64) + document + chunk and map[g] = document (-1: unused)
+    const int32_t* map;
+    float* decay_out;       // [G * H][128]: e^{Gamma_end} of every record
+    long long G;            // chunk records per head
+    int ncT;
     const __nv_bfloat16* beta;
     const float* h0;
     const int32_t* cu;
@@ -142,11 +150,29 @@ __device__ __forceinline__ void st_bf16x8(uint8_t* p, const float* v) {
 }
 __device__ __forceinline__ uint32_t f2tf(float x) { return __float_as_uint(x); }
 
-template <int DV>
+// Output maps of the intra mode (workspace records, row-major bf16, 128-byte swizzle).
+struct IntraMaps {
+    CUtensorMap wq, ke, ut, ot;
+};
+
+// One unit of a CTA's walk: a chunk of 64 rows of one head.
+struct Unit {
+    int h;
+    int L;            // valid rows
+    long long row0;   // first token row
+    long long rec;    // workspace record (intra mode)
+};
+
+// kIntra = false (fused): one CTA per (sequence or document, head, value slice) walks its chunks in
+// order and carries the state in TMEM. kIntra = true: a persistent CTA takes independent
+// (chunk, head) records, computes the chunk's WY factors and stores them for the state pass.
+template <int DV, bool kIntra>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
-               const ChunkArgs args) {
+               const __grid_constant__ IntraMaps omaps, const ChunkArgs args) {
+    static_assert(!kIntra || DV == 128, "the intra mode computes whole heads");
+    constexpr uint32_t kTmemCols = kIntra ? 256 : 512;
     using Lay = Layout<DV>;
     constexpr int kDV = Lay::kDV, kSplit = Lay::kSplit, kPanels = Lay::kPanels;
     constexpr uint32_t OFF_Q = Lay::OFF_Q, OFF_K = Lay::OFF_K, OFF_G = Lay::OFF_G;
@@ -164,14 +190,15 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int qd = warp & 3, hf = warp >> 2;          // TMEM lane quarter, column half
-    const int split = blockIdx.x % kSplit;
-    const int unit = blockIdx.x / kSplit;
-    const int h = unit % args.H;
-    const int n = args.order ? args.order[unit / args.H] : unit / args.H;
+    const int split = kIntra ? 0 : blockIdx.x % kSplit;
+    const int unit = kIntra ? 0 : blockIdx.x / kSplit;
+    int h = kIntra ? 0 : unit % args.H;
+    const int n = kIntra ? 0 : (args.order ? args.order[unit / args.H] : unit / args.H);
     const int dv0 = split * kDV;
 
-    long long t0, t1;
-    if (args.cu) {
+    long long t0 = 0, t1 = 0;
+    if constexpr (kIntra) {
+    } else if (args.cu) {
         t0 = args.cu[n];
         t1 = args.cu[n + 1];
         const bool bad_ends = (n == 0 && t0 != 0) || (n == args.N - 1 && t1 != args.T);
@@ -184,6 +211,48 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         t1 = t0 + args.T;
     }
     const int nchunks = (int)((t1 - t0 + kC - 1) / kC);
+
+    // the walk: chunks of this chain in order (fused), or this CTA's share of the records
+    long long cursor = kIntra ? (long long)blockIdx.x : 0;
+    auto next_unit = [&](Unit& u) -> bool {
+        if constexpr (kIntra) {
+            const long long total = args.G * args.H;
+            while (cursor < total) {
+                const long long idx = cursor;
+                cursor += gridDim.x;
+                const long long g = idx / args.H;
+                u.h = (int)(idx % args.H);
+                u.rec = idx;
+                if (args.cu) {
+                    const int d = args.map[g];
+                    if (d < 0 || d >= args.N) continue;
+                    const long long a = args.cu[d], b = args.cu[d + 1];
+                    if (b <= a || a < 0 || b > args.T) continue;   // reported by the map kernel
+                    const long long cc = g - d - a / kC;
+                    if (cc < 0 || a + kC * cc >= b) continue;
+                    u.row0 = a + kC * cc;
+                    u.L = (int)min((long long)kC, b - u.row0);
+                } else {
+                    const long long s = g / args.ncT, cc = g % args.ncT;
+                    u.row0 = s * args.T + kC * cc;
+                    u.L = (int)min((long long)kC, (long long)args.T - kC * cc);
+                }
+                return true;
+            }
+            return false;
+        } else {
+            if (cursor >= nchunks) return false;
+            u.h = h;
+            u.row0 = t0 + kC * cursor;
+            u.L = (int)min((long long)kC, t1 - u.row0);
+            u.rec = 0;
+            ++cursor;
+            return true;
+        }
+    };
+    Unit cur, nxt;
+    bool has_cur = next_unit(cur);
+    bool has_nxt = has_cur && next_unit(nxt);
 
     float* beta_s = reinterpret_cast<float*>(sm + OFF_BETA);
     float* decay_s = reinterpret_cast<float*>(sm + OFF_DECAY);
@@ -217,7 +286,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
     // initial state: TMEM lane c = 32 qd + lane holds S[c][dv0 + kHalfCols hf .. + kHalfCols)
 #pragma unroll
-    for (int p = 0; p < kHalfCols / 32; ++p) {
+    for (int p = 0; p < (kIntra ? 0 : kHalfCols / 32); ++p) {
         float v[32];
         const int c = 32 * qd + lane;
         const int col = kHalfCols * hf + 32 * p;
@@ -237,19 +306,19 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tmem_st_wait();
     }
 
-    auto issue_in = [&](int c) {
-        const int row0 = (int)(t0 + (long long)kC * c);
+    auto issue_in = [&](const Unit& u) {
+        const int row0 = (int)u.row0;
         mbar_arrive_expect_tx(bar_in, kTxIn);
-        tma_load_3d(sb + OFF_Q, &tm_q, bar_in, 0, h, row0);
-        tma_load_3d(sb + OFF_K, &tm_k, bar_in, 0, h, row0);
-        tma_load_3d(sb + OFF_G, &tm_g, bar_in, 0, h, row0);
+        tma_load_3d(sb + OFF_Q, &tm_q, bar_in, 0, u.h, row0);
+        tma_load_3d(sb + OFF_K, &tm_k, bar_in, 0, u.h, row0);
+        tma_load_3d(sb + OFF_G, &tm_g, bar_in, 0, u.h, row0);
     };
-    auto issue_v = [&](int c) {
-        const int row0 = (int)(t0 + (long long)kC * c);
+    auto issue_v = [&](const Unit& u) {
+        const int row0 = (int)u.row0;
         mbar_arrive_expect_tx(bar_v, Lay::kTxV);
 #pragma unroll
         for (int p = 0; p < kPanels; ++p)
-            tma_load_3d(sb + OFF_KPV + 16384 + 8192 * p, &tm_v, bar_v, dv0 + 64 * p, h, row0);
+            tma_load_3d(sb + OFF_KPV + 16384 + 8192 * p, &tm_v, bar_v, dv0 + 64 * p, u.h, row0);
     };
 
     // constant parts of the shared-memory descriptors (the start address is added per MMA)
@@ -268,10 +337,11 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         return __syncthreads_or(!ok) == 0;
     };
 
-    if (nchunks > 0) {
+    bool stores_pending = false;   // intra mode: bulk stores still reading shared memory
+    if (has_cur) {
         if (tid == 0) {
-            issue_in(0);
-            issue_v(0);
+            issue_in(cur);
+            issue_v(cur);
         }
         in_pending = v_pending = true;
     }
@@ -279,9 +349,10 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // copies in flight, must expire, report KDA_ERR_TIMEOUT and wind down cleanly.
     if (args.debug_stall && !wait_all(bar_never, 0)) aborted = true;
 
-    float beta_next = 0.f;   // beta of the next chunk, row tid (threads tid < 64)
-    if (tid < kC && nchunks > 0 && t0 + tid < t1)
-        beta_next = __bfloat162float(args.beta[(t0 + tid) * args.H + h]);
+    // beta of the next chunk, row tid (threads tid < 64), kept as raw bf16 so that the prefetch
+    // is only waited for when the next chunk begins
+    __nv_bfloat16 beta_next = __float2bfloat16(0.f);
+    if (tid < kC && has_cur && tid < cur.L) beta_next = args.beta[(cur.row0 + tid) * args.H + cur.h];
 
     const uint8_t* qs = sm + OFF_Q;
     const uint8_t* ks = sm + OFF_K;
@@ -299,22 +370,18 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                lo8;
     };
 
-    for (int c = 0; c < nchunks && !aborted; ++c) {
-        const long long row0 = t0 + (long long)kC * c;
-        const int L = (int)min((long long)kC, t1 - row0);
+    for (int c = 0; has_cur && !aborted; ++c) {
+        const long long row0 = cur.row0;
+        const int L = cur.L;
+        h = cur.h;
 
         // ---------------------------------------------------------------- inputs of chunk c
         if (!wait_all(bar_in, c & 1)) { aborted = true; break; }
         in_pending = false;
-        if (b4_pending) {   // the previous state update still reads U and K_end
-            if (!wait_all(bar_b4, b4_chunk & 1)) { aborted = true; break; }
-            b4_pending = false;
-        }
-        if (tid < kC) beta_s[tid] = beta_next;
-        if (tid < kC && c + 1 < nchunks) {   // prefetch the next chunk's beta
-            const long long r1 = row0 + kC + tid;
-            beta_next = r1 < t1 ? __bfloat162float(args.beta[r1 * args.H + h]) : 0.f;
-        }
+        if (tid < kC) beta_s[tid] = __bfloat162float(beta_next);
+        if (tid < kC && has_nxt)   // prefetch the next unit's beta
+            beta_next = tid < nxt.L ? args.beta[(nxt.row0 + tid) * args.H + nxt.h]
+                                    : __float2bfloat16(0.f);
 
         // ---------------------------------------------------------------- decay products
         float pre[8][4], suf[8][4];
@@ -380,8 +447,22 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     if (bb == pb) own[i] = hh == 0 ? up[i] : lo[i];
                 }
             }
-            if (pb == 0 && hh == 0)
+            if (pb == 0 && hh == 0) {
                 *reinterpret_cast<float4*>(decay_s + ch0) = make_float4(dec[0], dec[1], dec[2], dec[3]);
+                if constexpr (kIntra)
+                    *reinterpret_cast<float4*>(args.decay_out + cur.rec * kD + ch0) =
+                        make_float4(dec[0], dec[1], dec[2], dec[3]);
+            }
+        }
+
+        if (b4_pending) {   // the previous state update reads U (R region) and K_end until here
+            if (!wait_all(bar_b4, b4_chunk & 1)) { aborted = true; break; }
+            b4_pending = false;
+        }
+        if (kIntra && stores_pending) {   // the previous record's stores read R, [W; Q~] and K_end
+            if (tid == 0) bulk_wait_read_all();
+            __syncthreads();
+            stores_pending = false;
         }
 
         // ---------------------------------------------------------------- R and C operands
@@ -471,8 +552,8 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         fence_proxy_async();
         __syncthreads();   // q, k, log g of chunk c fully consumed
-        if (c + 1 < nchunks) {
-            if (tid == 0) issue_in(c + 1);
+        if (has_nxt) {
+            if (tid == 0) issue_in(nxt);
             in_pending = true;
             in_chunk = c + 1;
         }
@@ -557,77 +638,105 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         {
             const float* Lb = reinterpret_cast<const float*>(sm + OFF_LB);
             float* Mb = reinterpret_cast<float*>(sm + OFF_MB);
-            // diagonal 16x16 blocks of (I + L)^-1: forward substitution, one column per thread
-            if (tid < 64) {
-                const int base = 16 * (tid >> 4), j = tid & 15;
-                float acc[16], x[16];
+            // diagonal 16x16 blocks of (I + L)^-1: forward substitution for column j of block bk,
+            // x_k = [k = j] - sum_{m<k} L[k][m] x_m, by four threads: part t keeps the running
+            // sums of rows 4t..4t+3 and the owner of row k broadcasts x_k to the other three.
+            // L is zero on and above the diagonal of its diagonal blocks, so every row takes
+            // every update.
+            {
+                // part t owns rows t, t + 4, t + 8, t + 12 (distinct banks for the four parts)
+                const int bk = tid >> 6, j = (tid >> 2) & 15, t = tid & 3;
+                const int base = 16 * bk;
+                const int src0 = lane & ~3;
+                float lr[4][16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+                for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float4 x = *reinterpret_cast<const float4*>(
+                            Lb + (base + t + 4 * ii) * kLdl + base + 4 * m);
+                        lr[ii][4 * m] = x.x;
+                        lr[ii][4 * m + 1] = x.y;
+                        lr[ii][4 * m + 2] = x.z;
+                        lr[ii][4 * m + 3] = x.w;
+                    }
+                float acc[4] = {0.f, 0.f, 0.f, 0.f}, xo[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
-                    x[k] = (k == j) ? 1.f : (k < j ? 0.f : -acc[k]);
+                    const int own = k & 3, kk = k >> 2;
+                    float xk = (k == j ? 1.f : 0.f) - acc[kk];   // meaningful on the owner only
+                    xk = __shfl_sync(0xffffffffu, xk, src0 + own);
+                    if (t == own) xo[kk] = xk;
 #pragma unroll
-                    for (int i = k + 1; i < 16; ++i)
-                        acc[i] = fmaf(Lb[(base + i) * kLdl + base + k], x[k], acc[i]);
+                    for (int ii = 0; ii < 4; ++ii) acc[ii] = fmaf(lr[ii][k], xk, acc[ii]);
                 }
 #pragma unroll
-                for (int i = 0; i < 16; ++i) Mb[(base + i) * kLdm + base + j] = x[i];
+                for (int ii = 0; ii < 4; ++ii) Mb[(base + t + 4 * ii) * kLdm + base + j] = xo[ii];
             }
             __syncthreads();
-            // off-diagonal blocks, by distance d = a - b, one warp per block (tf32 mma.sync):
-            //   Y = sum_{kk in blocks b..a-1} L[a-block rows][kk] M[kk][b-block cols]
-            //   M_ab = -M_aa Y
+            // off-diagonal blocks of M = (I + L)^-1 (tf32 mma.sync, one warp per 16x16 block).
+            //   level 1:  M_{b+1,b} = -M_{b+1,b+1} L_{b+1,b} M_bb
+            //   level 2:  the lower-left 32x32 block, M[32:, :32] = -M[32:, 32:] L[32:, :32] M[:32, :32],
+            //             as Y = L[32:, :32] M[:32, :32] (four blocks) and then -M[32:, 32:] Y
+            //             (blocks (2,0), (3,0), (3,1); (2,1) is known from level 1)
             const int g = lane >> 2, t = lane & 3;
-            float* ys = reinterpret_cast<float*>(sm + OFF_YS) + warp * 16 * 17;
-#pragma unroll 1
-            for (int d = 1; d < 4; ++d) {
-                if (warp < 4 - d) {
-                    const int bb = warp, aa = warp + d;
-                    float y[2][4] = {};
-                    for (int kk = 16 * bb; kk < 16 * aa; kk += 8) {
-                        const float* la = Lb + (16 * aa + g) * kLdl + kk + t;
-                        const uint32_t A[4] = {f2tf(la[0]), f2tf(la[8 * kLdl]), f2tf(la[4]),
-                                               f2tf(la[8 * kLdl + 4])};
-#pragma unroll
-                        for (int nt = 0; nt < 2; ++nt) {
-                            const float* mb = Mb + (kk + t) * kLdm + 16 * bb + 8 * nt + g;
-                            const uint32_t B[2] = {f2tf(mb[0]), f2tf(mb[4 * kLdm])};
-                            mma_tf32_16x8x8(y[nt], A, B);
-                        }
-                    }
+            float* ysb = reinterpret_cast<float*>(sm + OFF_YS);   // four 16x17 scratch blocks
+            // acc += A[0:16, 0:K] B[0:K, 0:16] for fp32 row-major sources
+            auto mm16 = [&](float (&acc)[2][4], const float* A, int lda, const float* B, int ldb,
+                            int K) {
+                for (int kk = 0; kk < K; kk += 8) {
+                    const float* la = A + g * lda + kk + t;
+                    const uint32_t a[4] = {f2tf(la[0]), f2tf(la[8 * lda]), f2tf(la[4]),
+                                           f2tf(la[8 * lda + 4])};
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
-                        ys[g * 17 + 8 * nt + 2 * t] = y[nt][0];
-                        ys[g * 17 + 8 * nt + 2 * t + 1] = y[nt][1];
-                        ys[(g + 8) * 17 + 8 * nt + 2 * t] = y[nt][2];
-                        ys[(g + 8) * 17 + 8 * nt + 2 * t + 1] = y[nt][3];
+                        const float* lb = B + (kk + t) * ldb + 8 * nt + g;
+                        const uint32_t b[2] = {f2tf(lb[0]), f2tf(lb[4 * ldb])};
+                        mma_tf32_16x8x8(acc[nt], a, b);
                     }
-                    __syncwarp();
-                    float z[2][4] = {};
-#pragma unroll
-                    for (int ks2 = 0; ks2 < 2; ++ks2) {
-                        const float* ma = Mb + (16 * aa + g) * kLdm + 16 * aa + 8 * ks2 + t;
-                        const uint32_t A[4] = {f2tf(ma[0]), f2tf(ma[8 * kLdm]), f2tf(ma[4]),
-                                               f2tf(ma[8 * kLdm + 4])};
-#pragma unroll
-                        for (int nt = 0; nt < 2; ++nt) {
-                            const uint32_t B[2] = {f2tf(ys[(8 * ks2 + t) * 17 + 8 * nt + g]),
-                                                   f2tf(ys[(8 * ks2 + t + 4) * 17 + 8 * nt + g])};
-                            mma_tf32_16x8x8(z[nt], A, B);
-                        }
-                    }
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        float* mo = Mb + (16 * aa + g) * kLdm + 16 * bb + 8 * nt + 2 * t;
-                        mo[0] = -z[nt][0];
-                        mo[1] = -z[nt][1];
-                        mo[8 * kLdm] = -z[nt][2];
-                        mo[8 * kLdm + 1] = -z[nt][3];
-                    }
-                    __syncwarp();
                 }
-                __syncthreads();
+            };
+            auto st16 = [&](float* dst, int ld, const float (&z)[2][4], float sign) {
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    dst[g * ld + 8 * nt + 2 * t] = sign * z[nt][0];
+                    dst[g * ld + 8 * nt + 2 * t + 1] = sign * z[nt][1];
+                    dst[(g + 8) * ld + 8 * nt + 2 * t] = sign * z[nt][2];
+                    dst[(g + 8) * ld + 8 * nt + 2 * t + 1] = sign * z[nt][3];
+                }
+            };
+            if (warp < 3) {
+                const int bb = warp, aa = warp + 1;
+                float* ys = ysb + warp * 16 * 17;
+                float y[2][4] = {}, z[2][4] = {};
+                mm16(y, Lb + 16 * aa * kLdl + 16 * bb, kLdl, Mb + 16 * bb * kLdm + 16 * bb, kLdm, 16);
+                st16(ys, 17, y, 1.f);
+                __syncwarp();
+                mm16(z, Mb + 16 * aa * kLdm + 16 * aa, kLdm, ys, 17, 16);
+                st16(Mb + 16 * aa * kLdm + 16 * bb, kLdm, z, -1.f);
             }
+            __syncthreads();
+            if (warp < 4) {   // Y_{ra,cb} = sum over k-blocks cb..1 of L_{ra,k} M_{k,cb}
+                const int ra = 2 + (warp >> 1), cb = warp & 1;
+                float y[2][4] = {};
+                mm16(y, Lb + 16 * ra * kLdl + 16 * cb, kLdl, Mb + 16 * cb * kLdm + 16 * cb, kLdm,
+                     32 - 16 * cb);
+                st16(ysb + warp * 16 * 17, 17, y, 1.f);   // Y_{2,cb} in slot cb, Y_{3,cb} in 2 + cb
+            }
+            __syncthreads();
+            if (warp < 3) {   // warp 0: M_20 = -M_22 Y_20;  warps 1, 2: M_3c = -(M_32 Y_2c + M_33 Y_3c)
+                const int cb = warp == 2 ? 1 : 0;
+                float z[2][4] = {};
+                if (warp == 0) {
+                    mm16(z, Mb + 32 * kLdm + 32, kLdm, ysb, 17, 16);
+                    st16(Mb + 32 * kLdm, kLdm, z, -1.f);
+                } else {
+                    mm16(z, Mb + 48 * kLdm + 32, kLdm, ysb + cb * 16 * 17, 17, 16);
+                    mm16(z, Mb + 48 * kLdm + 48, kLdm, ysb + (2 + cb) * 16 * 17, 17, 16);
+                    st16(Mb + 48 * kLdm + 16 * cb, kLdm, z, -1.f);
+                }
+            }
+            __syncthreads();
             // T = (I + L)^-1 diag(beta): lower triangle, bf16 K-major
             {
                 const int i = 2 * lane;
@@ -687,11 +796,26 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (warp == 0) {
             if (lane == 0) {
                 tc_fence_after();
-                const uint32_t id = idesc_bf16(128, 128 + kDV, 0, 1);
+                if constexpr (kIntra) {
+                    // [T; T'] K+ (W, A_qk W) and, transposed for the state pass, V^T [T; T']^T:
+                    // lane j (value column) gets U~^T (columns 128-191) and O~^T (192-255)
+                    const uint32_t id = idesc_bf16(128, 128, 0, 1);
+                    const uint32_t idt = idesc_bf16(128, 128, 1, 0);
 #pragma unroll
-                for (int s = 0; s < kC / 16; ++s)
-                    umma_f16(tbase + TM_A, desc_at(dK, sb + OFF_TT + 32 * s),
-                             desc_at(dM8, sb + OFF_KPV + 2048 * s), id, s > 0);
+                    for (int s = 0; s < kC / 16; ++s)
+                        umma_f16(tbase + TM_A, desc_at(dK, sb + OFF_TT + 32 * s),
+                                 desc_at(dM8, sb + OFF_KPV + 2048 * s), id, s > 0);
+#pragma unroll
+                    for (int s = 0; s < kC / 16; ++s)
+                        umma_f16(tbase + TM_A + 128, desc_at(dM8, sb + OFF_KPV + 16384 + 2048 * s),
+                                 desc_at(dK, sb + OFF_TT + 32 * s), idt, s > 0);
+                } else {
+                    const uint32_t id = idesc_bf16(128, 128 + kDV, 0, 1);
+#pragma unroll
+                    for (int s = 0; s < kC / 16; ++s)
+                        umma_f16(tbase + TM_A, desc_at(dK, sb + OFF_TT + 32 * s),
+                                 desc_at(dM8, sb + OFF_KPV + 2048 * s), id, s > 0);
+                }
                 umma_commit(bar_mma);
             }
             __syncwarp();
@@ -701,8 +825,8 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ++mma_phase;
         mma_pending = false;
         tc_fence_after();
-        if (c + 1 < nchunks) {   // the V panel is free again
-            if (tid == 0) issue_v(c + 1);
+        if (has_nxt) {   // the V panel is free again
+            if (tid == 0) issue_v(nxt);
             v_pending = true;
             v_chunk = c + 1;
         }
@@ -734,98 +858,132 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
             }
         }
+        if constexpr (kIntra) {
+            // U~^T (TMEM columns 128-191) and O~^T (192-255), lane j = value column, into bf16
+            // staging tiles [128 j][64 tokens] in the R region (128-byte swizzle), then one set
+            // of bulk stores
+            const int jrow = 32 * qd + lane;
+            const uint32_t stage = hf == 0 ? OFF_R : OFF_R + 16384;
 #pragma unroll
-        for (int p = 0; p < kHalfCols / 32; ++p) {
-            // state: bf16 operand for [W; Q~] S, then decay the fp32 TMEM copy
-            float v[32];
-            const int cc = 32 * qd + lane;
-            const int col = kHalfCols * hf + 32 * p;
-            tmem_ld32(tbase + lane_q + TM_S + col, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int m = 0; m < 4; ++m)
-                st_bf16x8(sm + OFF_S16 + sw128_off(128, cc, col + 8 * m), v + 8 * m);
-            const float dcy = decay_s[cc];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] *= dcy;
-            tmem_st32(tbase + lane_q + TM_S + col, v);
-            tmem_st_wait();
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---------------------------------------------------------------- MMA: [W; Q~] S
-        if (warp == 0) {
-            if (lane == 0) {
-                tc_fence_after();
-                const uint32_t id = idesc_bf16(128, kDV, 0, 1);
-#pragma unroll
-                for (int s = 0; s < kD / 16; ++s) {
-                    const int k0 = 16 * s;
-                    umma_f16(tbase + TM_B,
-                             desc_at(dK, sb + OFF_WQ + (k0 >> 6) * 16384 + (k0 & 63) * 2),
-                             desc_at(dM16, sb + OFF_S16 + 2048 * s), id, s > 0);
-                }
-                umma_commit(bar_mma);
-            }
-            __syncwarp();
-        }
-        mma_pending = true;
-        if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
-        ++mma_phase;
-        mma_pending = false;
-        tc_fence_after();
-#pragma unroll
-        for (int p = 0; p < kHalfCols / 32; ++p) {
-            // quarters 0-1: U = U~ - W S (rows r, value columns col ..)
-            // quarters 2-3: o = O~ + Q~ S
-            const int r = 32 * (qd & 1) + lane;
-            const int col = kHalfCols * hf + 32 * p;
-            float x[32], y[32];
-            tmem_ld32(tbase + lane_q + TM_B + col, x);
-            tmem_ld32(tbase + lane_q + TM_A + 128 + col, y);
-            tmem_ld_wait();
-            if (qd < 2) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) y[j] -= x[j];
+            for (int part = 0; part < 2; ++part) {
+                float v[32];
+                tmem_ld32(tbase + lane_q + TM_A + 128 + 64 * hf + 32 * part, v);
+                tmem_ld_wait();
 #pragma unroll
                 for (int m = 0; m < 4; ++m)
-                    st_bf16x8(sm + OFF_U16 + sw128_off(64, r, col + 8 * m), y + 8 * m);
-            } else if (r < L) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) y[j] += x[j];
-                uint4* dst = reinterpret_cast<uint4*>(
-                    args.o + ((size_t)(row0 + r) * args.H + h) * kD + dv0 + col);
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const float* w = y + 8 * m;
-                    dst[m] = make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]),
-                                        pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
+                    st_bf16x8(sm + stage + sw128_off(128, jrow, 32 * part + 8 * m), v + 8 * m);
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                const int rw = (int)(cur.rec * 128), rk = (int)(cur.rec * 64);
+                tma_store_2d(&omaps.wq, sb + OFF_WQ, 0, rw);
+                tma_store_2d(&omaps.wq, sb + OFF_WQ + 16384, 64, rw);
+                tma_store_2d(&omaps.ke, sb + OFF_KE, 0, rk);
+                tma_store_2d(&omaps.ke, sb + OFF_KE + 8192, 64, rk);
+                tma_store_2d(&omaps.ut, sb + OFF_R, 0, rw);
+                tma_store_2d(&omaps.ot, sb + OFF_R + 16384, 0, rw);
+                bulk_commit();
+            }
+            stores_pending = true;
+        } else {
+    #pragma unroll
+            for (int p = 0; p < kHalfCols / 32; ++p) {
+                // state: bf16 operand for [W; Q~] S, then decay the fp32 TMEM copy
+                float v[32];
+                const int cc = 32 * qd + lane;
+                const int col = kHalfCols * hf + 32 * p;
+                tmem_ld32(tbase + lane_q + TM_S + col, v);
+                tmem_ld_wait();
+    #pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    st_bf16x8(sm + OFF_S16 + sw128_off(128, cc, col + 8 * m), v + 8 * m);
+                const float dcy = decay_s[cc];
+    #pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] *= dcy;
+                tmem_st32(tbase + lane_q + TM_S + col, v);
+                tmem_st_wait();
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            __syncthreads();
+
+            // ---------------------------------------------------------------- MMA: [W; Q~] S
+            if (warp == 0) {
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint32_t id = idesc_bf16(128, kDV, 0, 1);
+    #pragma unroll
+                    for (int s = 0; s < kD / 16; ++s) {
+                        const int k0 = 16 * s;
+                        umma_f16(tbase + TM_B,
+                                 desc_at(dK, sb + OFF_WQ + (k0 >> 6) * 16384 + (k0 & 63) * 2),
+                                 desc_at(dM16, sb + OFF_S16 + 2048 * s), id, s > 0);
+                    }
+                    umma_commit(bar_mma);
+                }
+                __syncwarp();
+            }
+            mma_pending = true;
+            if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
+            ++mma_phase;
+            mma_pending = false;
+            tc_fence_after();
+    #pragma unroll
+            for (int p = 0; p < kHalfCols / 32; ++p) {
+                // quarters 0-1: U = U~ - W S (rows r, value columns col ..)
+                // quarters 2-3: o = O~ + Q~ S
+                const int r = 32 * (qd & 1) + lane;
+                const int col = kHalfCols * hf + 32 * p;
+                float x[32], y[32];
+                tmem_ld32(tbase + lane_q + TM_B + col, x);
+                tmem_ld32(tbase + lane_q + TM_A + 128 + col, y);
+                tmem_ld_wait();
+                if (qd < 2) {
+    #pragma unroll
+                    for (int j = 0; j < 32; ++j) y[j] -= x[j];
+    #pragma unroll
+                    for (int m = 0; m < 4; ++m)
+                        st_bf16x8(sm + OFF_U16 + sw128_off(64, r, col + 8 * m), y + 8 * m);
+                } else if (r < L) {
+    #pragma unroll
+                    for (int j = 0; j < 32; ++j) y[j] += x[j];
+                    uint4* dst = reinterpret_cast<uint4*>(
+                        args.o + ((size_t)(row0 + r) * args.H + h) * kD + dv0 + col);
+    #pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float* w = y + 8 * m;
+                        dst[m] = make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]),
+                                            pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
+                    }
                 }
             }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
+            fence_proxy_async();
+            tc_fence_before();
+            __syncthreads();
 
-        // ---------------------------------------------------------------- MMA: S += K_end^T U
-        if (warp == 0) {   // lane 0 issues; the rest of warp 0 waits for it
-            if (lane == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(128, kDV, 1, 1);
-#pragma unroll
-            for (int s = 0; s < kC / 16; ++s) {
-                const uint64_t ae = desc_at(dM8, sb + OFF_KE + 2048 * s);
-                const uint64_t bu = desc_at(dM8, sb + OFF_U16 + 2048 * s);
-                umma_f16(tbase + TM_S, ae, bu, id, 1);
+            // ---------------------------------------------------------------- MMA: S += K_end^T U
+            if (warp == 0) {   // lane 0 issues; the rest of warp 0 waits for it
+                if (lane == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, kDV, 1, 1);
+    #pragma unroll
+                for (int s = 0; s < kC / 16; ++s) {
+                    const uint64_t ae = desc_at(dM8, sb + OFF_KE + 2048 * s);
+                    const uint64_t bu = desc_at(dM8, sb + OFF_U16 + 2048 * s);
+                    umma_f16(tbase + TM_S, ae, bu, id, 1);
+                }
+                umma_commit(bar_b4);
+                }
+                __syncwarp();
             }
-            umma_commit(bar_b4);
-            }
-            __syncwarp();
+            b4_pending = true;
+            b4_chunk = c;
         }
-        b4_pending = true;
-        b4_chunk = c;
+        cur = nxt;
+        has_cur = has_nxt;
+        if (has_cur) has_nxt = next_unit(nxt);
     }
 
     if (aborted) {
@@ -843,7 +1001,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_wait(bar_b4, b4_chunk & 1, 1ll << 31);
         }
         tc_fence_after();
-        if (args.hT) {
+        if (!kIntra && args.hT) {
 #pragma unroll
             for (int p = 0; p < kHalfCols / 32; ++p) {
                 float v[32];
@@ -859,6 +1017,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
         }
     }
+    if (kIntra && tid == 0) bulk_wait_all();   // stores complete before the CTA's smem goes away
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, kTmemCols);
@@ -869,7 +1028,9 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
-cudaError_t get_encoder() {
+}  // namespace
+
+cudaError_t tma_encoder_ready() {
     std::call_once(g_encode_once, [] {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -880,6 +1041,43 @@ cudaError_t get_encoder() {
     });
     return g_encode ? cudaSuccess : cudaErrorNotSupported;
 }
+
+cudaError_t make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
+                        unsigned long long rows, int cols, int box_cols, int box_rows,
+                        CUtensorMapSwizzle sw) {
+    cudaError_t e = tma_encoder_ready();
+    if (e != cudaSuccess) return e;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * elem_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_map_3d_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt,
+                             int elem_bytes, unsigned long long rows, int H, int cols,
+                             int box_rows) {
+    cudaError_t e = tma_encoder_ready();
+    if (e != cudaSuccess) return e;
+    const cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)H, (cuuint64_t)rows};
+    const cuuint64_t strides[2] = {(cuuint64_t)cols * elem_bytes,
+                                   (cuuint64_t)H * cols * elem_bytes};
+    const cuuint32_t box[3] = {(cuuint32_t)cols, 1, (cuuint32_t)box_rows};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = g_encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+namespace {
+
+cudaError_t get_encoder() { return tma_encoder_ready(); }
 
 // [rows, H, 128] row-major tensor, one head's 64-row tile per box
 cudaError_t make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
@@ -915,17 +1113,23 @@ long long wait_budget() {
     return budget;
 }
 
+template <int DV, bool kIntra>
+cudaError_t set_smem_attr() {
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(chunk64_kernel<DV, kIntra>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)Layout<DV>::kSmemBytes);
+    });
+    return attr_err;
+}
+
 template <int DV>
 cudaError_t launch_width(const FwdParams& p, cudaStream_t stream, const CUtensorMap& mq,
                          const CUtensorMap& mk, const CUtensorMap& mg, int units) {
     using Lay = Layout<DV>;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(chunk64_kernel<DV>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)Lay::kSmemBytes);
-    });
+    cudaError_t attr_err = set_smem_attr<DV, false>();
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap mv;
     cudaError_t e = make_map(&mv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B * p.T, p.H, 64,
@@ -946,7 +1150,14 @@ cudaError_t launch_width(const FwdParams& p, cudaStream_t stream, const CUtensor
     a.err = p.err;
     const long long grid = (long long)units * Lay::kSplit;
     if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
-    chunk64_kernel<DV><<<(unsigned)grid, kThreads, Lay::kSmemBytes, stream>>>(mq, mk, mg, mv, a);
+    a.map = nullptr;
+    a.decay_out = nullptr;
+    a.G = 0;
+    a.ncT = 0;
+    IntraMaps none;
+    memset(&none, 0, sizeof(none));
+    chunk64_kernel<DV, false><<<(unsigned)grid, kThreads, Lay::kSmemBytes, stream>>>(
+        mq, mk, mg, mv, none, a);
     return cudaGetLastError();
 }
 
@@ -996,6 +1207,56 @@ cudaError_t launch_chunk64(const FwdParams& p, cudaStream_t stream) {
 int chunk64_value_width(int N, int H) {
     const long long units = (long long)N * H;
     return units * 2 > sm_count() ? 128 : 64;
+}
+
+// Intra-chunk kernel of the split path: a persistent grid (one CTA per SM) takes the (chunk
+// record, head) items in turn and stores each chunk's WY factors into the workspace.
+cudaError_t launch_chunk64_intra(const FwdParams& p, cudaStream_t stream) {
+    const SplitWorkspace& ws = *p.split;
+    cudaError_t e = get_encoder();
+    if (e != cudaSuccess) return e;
+    const int rows = p.B * p.T;
+    const long long items = ws.G * p.H;
+    if (items == 0 || rows <= 0) return cudaSuccess;
+    if (ws.G * p.H * 128 > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    CUtensorMap mq, mk, mg, mv;
+    if ((e = make_map(&mq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, kD,
+                      CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
+        (e = make_map(&mk, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, kD,
+                      CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
+        (e = make_map(&mg, p.log_g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, p.H, kD,
+                      CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
+        (e = make_map(&mv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
+        return e;
+    const unsigned long long R = (unsigned long long)items;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+    IntraMaps om;
+    if ((e = make_map_2d(&om.wq, ws.wq, BF, 2, R * 128, kD, 64, 128, SW)) != cudaSuccess ||
+        (e = make_map_2d(&om.ke, ws.ke, BF, 2, R * 64, kD, 64, 64, SW)) != cudaSuccess ||
+        (e = make_map_2d(&om.ut, ws.ut, BF, 2, R * 128, kC, 64, 128, SW)) != cudaSuccess ||
+        (e = make_map_2d(&om.ot, ws.ot, BF, 2, R * 128, kC, 64, 128, SW)) != cudaSuccess)
+        return e;
+    if ((e = set_smem_attr<128, true>()) != cudaSuccess) return e;
+    ChunkArgs a;
+    memset(&a, 0, sizeof(a));
+    a.beta = static_cast<const __nv_bfloat16*>(p.beta);
+    a.cu = p.cu_seqlens;
+    a.T = p.T;
+    a.H = p.H;
+    a.N = p.N;
+    a.budget = wait_budget();
+    a.debug_stall = debug_stall();
+    a.err = p.err;
+    a.map = ws.map;
+    a.decay_out = ws.decay;
+    a.G = ws.G;
+    a.ncT = ws.ncT;
+    const long long grid = items < sm_count() ? items : sm_count();
+    chunk64_kernel<128, true><<<(unsigned)grid, kThreads, Layout<128>::kSmemBytes, stream>>>(
+        mq, mk, mg, mv, om, a);
+    return cudaGetLastError();
 }
 
 }  // namespace kda

@@ -20,6 +20,22 @@ __device__ __forceinline__ void set_device_error(unsigned* err, unsigned code) {
     atomicCAS(err, 0u, code);
 }
 
+// Workspace of the split chunked prefill: the WY factors of every (chunk record, head), written
+// by the intra-chunk kernel and read by the state pass. Record index = g * H + head, where g is
+// sequence * ncT + chunk (ncT = ceil(T / 64)), or, for packed documents, floor(t0 / 64) +
+// document + chunk (strictly increasing over (document, chunk), so records never collide and
+// g < ncT + N).
+struct SplitWorkspace {
+    __nv_bfloat16* wq;   // [R * 128][128]: rows 0-63 W, 64-127 Q~
+    __nv_bfloat16* ke;   // [R * 64][128]: K_end
+    __nv_bfloat16* ut;   // [R * 128][64]: U~^T (value column, token)
+    __nv_bfloat16* ot;   // [R * 128][64]: O~^T
+    float* decay;        // [R][128]: e^{Gamma_end}
+    int32_t* map;        // [G]: document of chunk record g, -1 if unused (packed only)
+    long long G;         // chunk records per head; R = G * H
+    int ncT;
+};
+
 struct FwdParams {
     const void* q;
     const void* k;
@@ -34,6 +50,7 @@ struct FwdParams {
     bool bf16;
     unsigned* err;            // device error word
     const int32_t* doc_order;   // nullable: packed documents in the order CTAs should take them
+    const SplitWorkspace* split;  // nullable: run the fused kernel instead
 };
 
 struct DecodeParams {
@@ -63,6 +80,12 @@ cudaError_t launch_doc_order(const int32_t* cu_seqlens, int N, int32_t* order,
 cudaError_t launch_recurrent(const FwdParams& p, cudaStream_t stream);
 cudaError_t launch_decode_d128(const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_chunk64(const FwdParams& p, cudaStream_t stream);
+// Split chunked prefill: map[g] for packed documents (sets DEV_BAD_SEQLENS on a malformed
+// cu_seqlens), the intra-chunk kernel over all records, then the state pass over all chains.
+cudaError_t launch_chunk_map(const int32_t* cu_seqlens, int N, int T, long long G, int32_t* map,
+                             unsigned* err, cudaStream_t stream);
+cudaError_t launch_chunk64_intra(const FwdParams& p, cudaStream_t stream);
+cudaError_t launch_chunk_scan(const FwdParams& p, cudaStream_t stream);
 bool chunk64_available();
 // Value columns one chunked-kernel CTA owns for N sequences x H heads (64 or 128).
 int chunk64_value_width(int N, int H);

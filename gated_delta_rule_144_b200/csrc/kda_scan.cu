@@ -1,0 +1,467 @@
+// State pass of the split chunked prefill: the only part of the chunked form that is sequential
+// over chunks.
+//
+// The intra-chunk kernel (chunk64_kernel in its intra mode) has already written, for every chunk
+// of 64 tokens and every head, the chunk's WY factors to the workspace:
+//   [W; Q~] (128 x 128 bf16), K_end (64 x 128 bf16), U~^T and O~^T (128 value columns x 64
+//   tokens, bf16) and the chunk's total decay e^{Gamma_end} (128 fp32).
+// Per (sequence or document, head) this kernel then walks the chunks in order (the WY form of the
+// gated delta rule; GLM-5.3-Flash model card, Kimi Delta Attention snippet, and the state-passing
+// identity it implies):
+//   U = U~ - W S,   o = O~ + Q~ S,   S <- diag(e^{Gamma_end}) S + K_end^T U.
+//
+// Layout: the state is kept transposed, S^T [value column j][key channel c], in TMEM lane j, so
+// both products take their state-side operand from TMEM and no shared-memory write sits on the
+// critical path:
+//   D = S^T [W; Q~]^T    (A = bf16 copy of S^T in TMEM, B = [W; Q~] K-major in shared memory)
+//   S^T += U^T K_end      (A = bf16 U^T in TMEM, B = K_end MN-major in shared memory)
+// 256 threads: warps w and w + 4 share TMEM lane quarter w mod 4 (lane j = value column j) and
+// split the columns of every TMEM row between them. Per chunk c the critical chain is
+//   bf16(S^T) -> D (8 K steps) -> U^T -> S^T += U^T K_end (4 K steps);
+// the decay of S^T, the loads of U~^T and O~^T and the output of chunk c-1 (o = O~ + Q~ S, read
+// from the other of two D buffers, staged in shared memory and written by a TMA store) run while
+// the D product of chunk c is in flight. Thread 0 issues the TMA copies (two stages: chunk c+1
+// arrives while chunk c runs) and the MMAs. Every mbarrier wait is bounded; on expiry the CTA
+// records KDA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "kda_internal.cuh"
+#include "kda_sm100.cuh"
+#include "kda_tma.cuh"
+
+namespace kda {
+namespace {
+
+using namespace sm100;
+
+constexpr int kC = 64;
+constexpr int kD = 128;
+constexpr int kThreads = 256;
+
+// one pipeline stage (bytes from a 1024-aligned stage base)
+constexpr uint32_t ST_WQ = 0;        // [W; Q~] 128 x 128 bf16, K-major SW128: 2 panels of 16 KB
+constexpr uint32_t ST_KE = 32768;    // K_end 64 x 128 bf16, MN-major SW128: 2 panels of 8 KB
+constexpr uint32_t ST_UT = 49152;    // U~^T [128 j][64 tokens] bf16, SW128
+constexpr uint32_t ST_OT = 65536;    // O~^T [128 j][64 tokens] bf16, SW128
+constexpr uint32_t ST_DEC = 81920;   // e^{Gamma_end} [128] f32
+constexpr uint32_t kStage = 82944;   // 81 KB, a multiple of 1024
+constexpr uint32_t kTxStage = 32768 + 3 * 16384 + 512;
+constexpr uint32_t OFF_O = 2 * kStage;       // two output tiles o [64 tokens][128] bf16
+constexpr uint32_t OFF_BAR = OFF_O + 32768;  // full[2], mma1, mma2, never
+constexpr uint32_t OFF_TMEM = OFF_BAR + 64;
+constexpr uint32_t kSmemBytes = OFF_TMEM + 16 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+// TMEM columns (128 lanes = value columns)
+constexpr uint32_t TS = 0;     // S^T fp32 [128 x 128]
+constexpr uint32_t TB = 128;   // bf16 S^T, A operand: 64 columns
+constexpr uint32_t TU = 192;   // bf16 U^T, A operand: 32 columns
+constexpr uint32_t TD = 256;   // two buffers of S^T [W; Q~]^T fp32 (128 columns each):
+                               //   columns 0-63 (W S)^T, 64-127 (Q~ S)^T
+constexpr uint32_t kTmemCols = 512;
+
+struct ScanArgs {
+    const int32_t* order;   // nullable: document taken by the k-th (document, head) group
+    const int32_t* cu;      // nullable
+    const float* h0;
+    float* hT;
+    __nv_bfloat16* o;
+    const float* decay;     // [R][128]
+    int T, H, N, ncT;       // ncT: chunk records per sequence when cu is null
+    long long G;            // chunk records per head
+    long long budget;
+    int debug_stall;
+    unsigned* err;
+};
+
+struct ScanMaps {
+    CUtensorMap wq, ke, ut, ot, o;
+};
+
+__device__ __forceinline__ uint32_t pack2(float x, float y) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(x, y);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float lo_bf(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float hi_bf(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int qd = warp & 3, hs = warp >> 2;   // TMEM lane quarter, column half
+    const int j = 32 * qd + lane;              // value column = TMEM lane
+    const int unit = blockIdx.x;
+    const int h = unit % args.H;
+    const int n = args.order ? args.order[unit / args.H] : unit / args.H;
+
+    long long t0, t1, g0;
+    if (args.cu) {
+        t0 = args.cu[n];
+        t1 = args.cu[n + 1];
+        const bool bad_ends = (n == 0 && t0 != 0) || (n == args.N - 1 && t1 != args.T);
+        if (t1 < t0 || t0 < 0 || t1 > args.T || bad_ends) {
+            if (tid == 0) set_device_error(args.err, DEV_BAD_SEQLENS);
+            return;
+        }
+        g0 = t0 / kC + n;
+    } else {
+        t0 = (long long)n * args.T;
+        t1 = t0 + args.T;
+        g0 = (long long)n * args.ncT;
+    }
+    const int nchunks = (int)((t1 - t0 + kC - 1) / kC);
+    if (g0 + nchunks > args.G) {   // only a malformed cu_seqlens gets here
+        if (tid == 0) set_device_error(args.err, DEV_BAD_SEQLENS);
+        return;
+    }
+
+    uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
+    const uint32_t bar_full0 = sb + OFF_BAR, bar_mma1 = bar_full0 + 16, bar_mma2 = bar_full0 + 24;
+    const uint32_t bar_never = bar_full0 + 32;
+    if (tid == 0) {
+        mbar_init(bar_full0, 1);
+        mbar_init(bar_full0 + 8, 1);
+        mbar_init(bar_mma1, 1);
+        mbar_init(bar_mma2, 1);
+        mbar_init(bar_never, 1);
+        fence_mbar_init();
+        prefetch_tmap(&maps.wq);
+        prefetch_tmap(&maps.ke);
+        prefetch_tmap(&maps.ut);
+        prefetch_tmap(&maps.ot);
+        prefetch_tmap(&maps.o);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_s), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_s;
+    const uint32_t lq = (uint32_t)(32 * qd) << 16;   // this warp's TMEM lane quarter
+    const size_t state_base = ((size_t)n * args.H + h) * kD * kD;
+
+    // initial state, transposed: lane j, column c holds S[c][j]; this thread: c in [64 hs, +64)
+#pragma unroll 1
+    for (int p = 0; p < 2; ++p) {
+        float v[32];
+        const int c0 = 64 * hs + 32 * p;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            v[i] = args.h0 ? args.h0[state_base + (size_t)(c0 + i) * kD + j] : 0.f;
+        tmem_st32(tbase + lq + TS + c0, v);
+    }
+    tmem_st_wait();
+
+    auto issue = [&](int c) {
+        const uint32_t st = sb + (uint32_t)(c & 1) * kStage;
+        const uint32_t bar = bar_full0 + 8 * (c & 1);
+        const long long rec = (g0 + c) * args.H + h;
+        mbar_arrive_expect_tx(bar, kTxStage);
+        tma_load_2d(st + ST_WQ, &maps.wq, bar, 0, (int)(rec * 128));
+        tma_load_2d(st + ST_WQ + 16384, &maps.wq, bar, 64, (int)(rec * 128));
+        tma_load_2d(st + ST_KE, &maps.ke, bar, 0, (int)(rec * 64));
+        tma_load_2d(st + ST_KE + 8192, &maps.ke, bar, 64, (int)(rec * 64));
+        tma_load_2d(st + ST_UT, &maps.ut, bar, 0, (int)(rec * 128));
+        tma_load_2d(st + ST_OT, &maps.ot, bar, 0, (int)(rec * 128));
+        bulk_load(st + ST_DEC, args.decay + rec * kD, 512, bar);
+    };
+
+    const uint64_t dK = sw128_desc(0, 16, 1024);     // K-major, 128B swizzle
+    const uint64_t dM8 = sw128_desc(0, 8192, 1024);  // MN-major, 64-row panels
+    const uint32_t id1 = idesc_bf16(128, 128, 0, 0);
+    const uint32_t id2 = idesc_bf16(128, 128, 0, 1);
+
+    // outstanding asynchronous work, drained before exit if a wait expires
+    int issued = 0;          // chunks whose copies were issued
+    int landed = 0;          // chunks whose copies were waited for
+    bool mma1_pending = false, mma2_pending = false;
+    int mma1_chunk = 0, mma2_chunk = 0;   // chunk of the last commit (its phase parity)
+    bool aborted = false;
+    auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
+        const bool ok = tid != 0 || mbar_wait(bar, parity, args.budget);
+        return __syncthreads_or(!ok) == 0;
+    };
+
+    // o of chunk cc (rows < L): O~^T (this thread's 32 tokens, packed in ob) + (Q~ S)^T from D
+    // buffer cc & 1, staged row-major in output tile cc & 1
+    uint32_t ob[16];
+    auto stage_o = [&](int cc) {
+        float w[32];
+        tmem_ld32(tbase + lq + TD + 128 * (cc & 1) + 64 + 32 * hs, w);
+        tmem_ld_wait();
+        __nv_bfloat16* tile = reinterpret_cast<__nv_bfloat16*>(sm + OFF_O + 16384 * (cc & 1));
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int r = 32 * hs + 2 * i;
+            tile[r * kD + j] = __float2bfloat16_rn(lo_bf(ob[i]) + w[2 * i]);
+            tile[(r + 1) * kD + j] = __float2bfloat16_rn(hi_bf(ob[i]) + w[2 * i + 1]);
+        }
+    };
+    // write staged tile cc to o: one TMA store for a full chunk, row copies for a partial one
+    // (a TMA box would run into the next document's rows). Call after a CTA barrier that
+    // follows fence_proxy_async by the writers.
+    auto flush_o = [&](int cc) {
+        const long long r0 = t0 + (long long)kC * cc;
+        const int L = (int)min((long long)kC, t1 - r0);
+        if (L == kC) {
+            if (tid == 0) {
+                tma_store_3d(&maps.o, sb + OFF_O + 16384 * (cc & 1), 0, h, (int)r0);
+                bulk_commit();
+            }
+        } else {
+            const uint4* src = reinterpret_cast<const uint4*>(sm + OFF_O + 16384 * (cc & 1));
+            for (int i = tid; i < L * 16; i += kThreads) {
+                const int r = i >> 4, q = i & 15;
+                *reinterpret_cast<uint4*>(args.o + ((size_t)(r0 + r) * args.H + h) * kD + 8 * q) =
+                    src[r * 16 + q];
+            }
+        }
+    };
+
+    if (tid == 0) {
+        if (nchunks > 0) issue(0);
+        if (nchunks > 1) issue(1);
+    }
+    issued = min(nchunks, 2);
+    if (args.debug_stall && !wait_all(bar_never, 0)) aborted = true;
+
+    for (int c = 0; c < nchunks && !aborted; ++c) {
+        const uint32_t st = sb + (uint32_t)(c & 1) * kStage;
+        const uint8_t* stp = sm + (size_t)(c & 1) * kStage;
+
+        if (!wait_all(bar_full0 + 8 * (c & 1), (uint32_t)((c >> 1) & 1))) { aborted = true; break; }
+        landed = c + 1;
+        if (mma2_pending) {   // S of chunk c is complete once the previous update has landed
+            if (!wait_all(bar_mma2, (uint32_t)(mma2_chunk & 1))) { aborted = true; break; }
+            mma2_pending = false;
+        }
+        tc_fence_after();
+
+        // ---------------------------------------------------------------- bf16 S^T -> TB
+        float va[32], vb[32];
+        tmem_ld32(tbase + lq + TS + 64 * hs, va);
+        tmem_ld32(tbase + lq + TS + 64 * hs + 32, vb);
+        tmem_ld_wait();
+        {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = pack2(va[2 * i], va[2 * i + 1]);
+            tmem_st16u(tbase + lq + TB + 32 * hs, pk);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = pack2(vb[2 * i], vb[2 * i + 1]);
+            tmem_st16u(tbase + lq + TB + 32 * hs + 16, pk);
+        }
+        tmem_st_wait();
+        // output tile (c-1)&1 is rewritten below; its previous store (chunk c-3) must be done
+        if (tid == 0 && c >= 3) bulk_wait_read_le1();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // stage (c+1)&1 held chunk c-1, fully consumed by now: fetch chunk c+1 into it
+        if (c >= 1 && c + 1 < nchunks) {
+            if (tid == 0) issue(c + 1);
+            issued = c + 2;
+        }
+
+        // ---------------------------------------------------------------- D = S^T [W; Q~]^T
+        if (tid == 0) {
+#pragma unroll
+            for (int s = 0; s < kD / 16; ++s)
+                umma_f16_ts(tbase + TD + 128 * (c & 1), tbase + TB + 8 * s,
+                            desc_at(dK, st + ST_WQ + (s >> 2) * 16384 + (s & 3) * 32), id1, s > 0);
+            umma_commit(bar_mma1);
+        }
+        mma1_pending = true;
+        mma1_chunk = c;
+
+        // ---------------------------------------------------------------- while D runs
+        // decay: TS = S^T diag(e^{Gamma_end}) (the update accumulates into it)
+        {
+            const float* dec = reinterpret_cast<const float*>(stp + ST_DEC) + 64 * hs;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                const float4 d0 = *reinterpret_cast<const float4*>(dec + i);
+                const float4 d1 = *reinterpret_cast<const float4*>(dec + 32 + i);
+                va[i] *= d0.x; va[i + 1] *= d0.y; va[i + 2] *= d0.z; va[i + 3] *= d0.w;
+                vb[i] *= d1.x; vb[i + 1] *= d1.y; vb[i + 2] *= d1.z; vb[i + 3] *= d1.w;
+            }
+            tmem_st32(tbase + lq + TS + 64 * hs, va);
+            tmem_st32(tbase + lq + TS + 64 * hs + 32, vb);
+        }
+        // U~^T of this chunk: row j, tokens [32 hs, +32)
+        uint32_t ub[16];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const uint4 x = *reinterpret_cast<const uint4*>(stp + ST_UT + sw128_off(128, j, 32 * hs + 8 * m));
+            ub[4 * m] = x.x; ub[4 * m + 1] = x.y; ub[4 * m + 2] = x.z; ub[4 * m + 3] = x.w;
+        }
+        if (c >= 1) stage_o(c - 1);
+        tmem_st_wait();
+
+        if (!wait_all(bar_mma1, (uint32_t)(c & 1))) { aborted = true; break; }
+        mma1_pending = false;
+        tc_fence_after();
+
+        // ---------------------------------------------------------------- U^T = U~^T - (W S)^T
+        {
+            float w[32];
+            tmem_ld32(tbase + lq + TD + 128 * (c & 1) + 32 * hs, w);
+            tmem_ld_wait();
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                pk[i] = pack2(lo_bf(ub[i]) - w[2 * i], hi_bf(ub[i]) - w[2 * i + 1]);
+            tmem_st16u(tbase + lq + TU + 16 * hs, pk);
+        }
+        // O~^T of this chunk, for its output at the next step
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const uint4 x = *reinterpret_cast<const uint4*>(stp + ST_OT + sw128_off(128, j, 32 * hs + 8 * m));
+            ob[4 * m] = x.x; ob[4 * m + 1] = x.y; ob[4 * m + 2] = x.z; ob[4 * m + 3] = x.w;
+        }
+        tmem_st_wait();
+        fence_proxy_async();   // output tile c-1 -> TMA store
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---------------------------------------------------------------- S^T += U^T K_end
+        if (tid == 0) {
+#pragma unroll
+            for (int s = 0; s < kC / 16; ++s)
+                umma_f16_ts(tbase + TS, tbase + TU + 8 * s, desc_at(dM8, st + ST_KE + 2048 * s),
+                            id2, 1);
+            umma_commit(bar_mma2);
+        }
+        mma2_pending = true;
+        mma2_chunk = c;
+        if (c >= 1) flush_o(c - 1);
+    }
+
+    if (aborted) {
+        if (tid == 0) set_device_error(args.err, DEV_TIMEOUT);
+        // wind down: this CTA's own copies and MMAs finish before TMEM and smem go away
+        const long long drain = 1ll << 31;
+        for (int c = landed; c < issued; ++c)
+            mbar_wait(bar_full0 + 8 * (c & 1), (uint32_t)((c >> 1) & 1), drain);
+        if (mma1_pending) mbar_wait(bar_mma1, (uint32_t)(mma1_chunk & 1), drain);
+        if (mma2_pending) mbar_wait(bar_mma2, (uint32_t)(mma2_chunk & 1), drain);
+        __syncthreads();
+    } else {
+        if (mma2_pending && !wait_all(bar_mma2, (uint32_t)(mma2_chunk & 1))) {
+            if (tid == 0) set_device_error(args.err, DEV_TIMEOUT);
+            mbar_wait(bar_mma2, (uint32_t)(mma2_chunk & 1), 1ll << 31);
+        }
+        tc_fence_after();
+        if (nchunks > 0) {   // output of the last chunk
+            if (tid == 0 && nchunks >= 3) bulk_wait_read_le1();
+            __syncthreads();
+            stage_o(nchunks - 1);
+            fence_proxy_async();
+            __syncthreads();
+            flush_o(nchunks - 1);
+        }
+        if (args.hT) {
+#pragma unroll 1
+            for (int p = 0; p < 2; ++p) {
+                float v[32];
+                const int c0 = 64 * hs + 32 * p;
+                tmem_ld32(tbase + lq + TS + c0, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) args.hT[state_base + (size_t)(c0 + i) * kD + j] = v[i];
+            }
+        }
+    }
+    if (tid == 0) bulk_wait_all();   // output stores complete before the CTA's smem goes away
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, kTmemCols);
+}
+
+long long scan_wait_budget() {
+    static long long budget = [] {
+        const char* s = std::getenv("KDA_DEBUG_WAIT_CYCLES");
+        if (s && *s) {
+            const long long v = std::atoll(s);
+            if (v > 0) return v;
+        }
+        return 1ll << 31;   // about one second of SM clock
+    }();
+    return budget;
+}
+
+int scan_debug_stall() {
+    static int v = [] {
+        const char* s = std::getenv("KDA_DEBUG_STALL_WAIT");
+        return (s && *s && *s != '0') ? 1 : 0;
+    }();
+    return v;
+}
+
+}  // namespace
+
+// One CTA (4 warps) per (sequence or document, head); packed documents are taken longest first
+// when an order is given.
+cudaError_t launch_chunk_scan(const FwdParams& p, cudaStream_t stream) {
+    const SplitWorkspace& ws = *p.split;
+    const long long units = (long long)p.N * p.H;
+    if (units == 0) return cudaSuccess;
+    if (units > 0x7fffffffLL || ws.G * p.H * 128 > 0x7fffffffLL)
+        return cudaErrorInvalidConfiguration;
+    const unsigned long long R = (unsigned long long)(ws.G * p.H);
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    ScanMaps m;
+    cudaError_t e;
+    if ((e = make_map_2d(&m.wq, ws.wq, BF, 2, R * 128, kD, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) !=
+            cudaSuccess ||
+        (e = make_map_2d(&m.ke, ws.ke, BF, 2, R * 64, kD, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) !=
+            cudaSuccess ||
+        (e = make_map_2d(&m.ut, ws.ut, BF, 2, R * 128, kC, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) !=
+            cudaSuccess ||
+        (e = make_map_2d(&m.ot, ws.ot, BF, 2, R * 128, kC, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) !=
+            cudaSuccess ||
+        (e = make_map_3d_rows(&m.o, p.o, BF, 2, (unsigned long long)p.B * p.T, p.H, kD, kC)) !=
+            cudaSuccess)
+        return e;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(chunk_scan_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)kSmemBytes);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    ScanArgs a;
+    memset(&a, 0, sizeof(a));
+    a.order = p.doc_order;
+    a.cu = p.cu_seqlens;
+    a.h0 = p.h0;
+    a.hT = p.hT;
+    a.o = static_cast<__nv_bfloat16*>(p.o);
+    a.decay = ws.decay;
+    a.T = p.T;
+    a.H = p.H;
+    a.N = p.N;
+    a.ncT = ws.ncT;
+    a.G = ws.G;
+    a.budget = scan_wait_budget();
+    a.debug_stall = scan_debug_stall();
+    a.err = p.err;
+    chunk_scan_kernel<<<(unsigned)units, kThreads, kSmemBytes, stream>>>(m, a);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

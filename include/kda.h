@@ -94,8 +94,15 @@ typedef struct {
  *             (their final state equals their initial state).
  *   o       : output, written for every token.
  *   hT      : [N, H, dk, dv] float32 final state of every sequence/document, or NULL to skip.
- *   workspace, workspace_bytes : scratch owned by the caller; at least
- *             kda_fwd_workspace_size(desc) bytes (may be NULL when that is 0).
+ *   workspace, workspace_bytes : scratch owned by the caller (device memory, 16-byte aligned).
+ *             With at least kda_fwd_workspace_size(desc) bytes the chunked path runs split: an
+ *             intra-chunk kernel computes every chunk's WY factors in parallel over all chunks
+ *             and heads and stores them here (about 80.5 KiB per 64-token chunk and head), then a
+ *             state pass walks each sequence's chunks. With less (but at least
+ *             kda_fwd_workspace_size_min(desc), which is 0 unless documents are packed) one fused
+ *             kernel per (sequence, head) does both, with no intermediate storage. Both give the
+ *             same result up to bf16 rounding of the stored factors. May be NULL when the minimum
+ *             is 0.
  *
  * The chunked path (KDA_CHUNK_64) computes in bf16 tensor-core products with fp32 accumulation
  * and an fp32 state. Its within-chunk factorisation needs the summed decay of any 8 consecutive
@@ -117,8 +124,18 @@ kda_status_t kda_fwd(const kda_fwd_desc_t* desc, const void* q, const void* k, c
  */
 int kda_fwd_algorithm(const kda_fwd_desc_t* desc, int has_cu_seqlens);
 
-/* Scratch bytes kda_fwd needs for `desc` (0 when it needs none). Host-only, no CUDA calls. */
+/*
+ * Workspace bytes for the fastest path kda_fwd has for `desc` (the split chunked path when it
+ * applies; 0 when nothing needs scratch). With B == 1 the size allows for cu_seqlens. Host-only,
+ * no CUDA calls; 0 for a rejected description.
+ */
 size_t kda_fwd_workspace_size(const kda_fwd_desc_t* desc);
+
+/*
+ * Smallest workspace kda_fwd accepts for `desc`: the fused chunked path's document order (one
+ * int32 per packed document, rounded up to 256 bytes; 0 without packed documents). Host-only.
+ */
+size_t kda_fwd_workspace_size_min(const kda_fwd_desc_t* desc);
 
 /*
  * kda_fwd_no_alloc - kda_fwd for callers that cannot allocate device memory.
@@ -141,7 +158,10 @@ size_t kda_fwd_workspace_size(const kda_fwd_desc_t* desc);
  * All calls on a device share the one array, which keeps the last call's contents. Every call
  * rewrites the slots it uses before reading them, so nothing needs to start at zero. Calls that
  * overlap on the GPU (concurrent streams, or several host threads) race on the array: serialise
- * them, or use kda_fwd with a workspace per stream. Results equal kda_fwd's.
+ * them, or use kda_fwd with a workspace per stream. The array is too small for the split
+ * chunked path's workspace, so this entry point runs kda_fwd's fused chunked path: the same
+ * result as kda_fwd given kda_fwd_workspace_size_min bytes, and the same as the split path up to
+ * bf16 rounding of the factors that path stores.
  * This function allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  */
 #define KDA_NO_ALLOC_MAX_DOCS 2048

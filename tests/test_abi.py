@@ -105,17 +105,35 @@ def test_decode_rejects_on_host(L):
     assert L.kda_decode_step(1, 1, 128, 128, 1, *args(o=P(FAKE + 4)), None) == 1
 
 
+def _split_bytes(B, T, H, N, packed):
+    """Split-path workspace: per (64-token chunk record, head) 32 KiB of [W; Q~], 3 x 16 KiB of
+    K_end, U~, O~ and 512 B of decay; plus the record map and document order when packed."""
+    up = lambda x: (x + 255) // 256 * 256
+    ncT = (T + 63) // 64
+    G = ncT + N if packed else B * ncT
+    R = G * H
+    order = up(4 * N) if packed and 2 <= N <= 2048 else 0
+    return order + (up(4 * G) if packed else 0) + up(512 * R) + R * (32768 + 3 * 16384)
+
+
 def test_workspace_size_is_host_only(L):
+    # minimum (fused chunked path): only packed documents need scratch, one int32 each
     d = _desc()
-    assert L.kda_fwd_workspace_size(ctypes.byref(d)) == 0
-    # packed documents on the chunked path: one int32 per document, rounded to 256 bytes
+    assert L.kda_fwd_workspace_size_min(ctypes.byref(d)) == 0
     d = _desc(num_seqs=8)
-    assert L.kda_fwd_workspace_size(ctypes.byref(d)) == 256
+    assert L.kda_fwd_workspace_size_min(ctypes.byref(d)) == 256
     d = _desc(num_seqs=300)
-    assert L.kda_fwd_workspace_size(ctypes.byref(d)) == 1280
+    assert L.kda_fwd_workspace_size_min(ctypes.byref(d)) == 1280
+    # preferred (split chunked path): the stored WY factors of every chunk record and head
+    for kw, packed in (({}, True), ({"num_seqs": 8}, True), ({"num_seqs": 300}, True),
+                       ({"B": 2, "num_seqs": 2, "T": 4096, "H": 16}, False)):
+        d = _desc(**kw)
+        want = _split_bytes(d.B, d.T, d.H, d.num_seqs, packed)
+        assert L.kda_fwd_workspace_size(ctypes.byref(d)) == want, kw
     # the exact path needs none
     d = _desc(num_seqs=8, chunk_size=1)
     assert L.kda_fwd_workspace_size(ctypes.byref(d)) == 0
+    assert L.kda_fwd_workspace_size_min(ctypes.byref(d)) == 0
 
 
 def test_packed_chunked_call_without_workspace_is_rejected_on_host(L):
