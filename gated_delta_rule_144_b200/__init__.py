@@ -199,14 +199,16 @@ def fwd(q, k, v, log_g, beta, h0=None, cu_seqlens=None, *, chunk_size: int = CHU
     else:
         hT = None
     desc = FwdDesc(B, T, H, dk, dv, N, _dtype_code(q), chunk_size)
-    need = int((lib().kda_fwd_workspace_size_min if fused else lib().kda_fwd_workspace_size)(
-        ctypes.byref(desc)))
-    if need > 0:
-        if workspace is None:
+    if workspace is None:
+        need = int((lib().kda_fwd_workspace_size_min if fused else lib().kda_fwd_workspace_size)(
+            ctypes.byref(desc)))
+        if need > 0:
             workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    else:   # the library picks the path the given size allows
         _dev(workspace, "workspace", torch.uint8, None, dev)
+        need = int(lib().kda_fwd_workspace_size_min(ctypes.byref(desc)))
         if workspace.numel() < need:
-            raise ValueError("workspace needs %d bytes" % need)
+            raise ValueError("workspace needs at least %d bytes" % need)
     ws_bytes = 0 if workspace is None else workspace.numel()
     with torch.cuda.device(dev):
         st = lib().kda_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(log_g),

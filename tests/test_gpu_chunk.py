@@ -1,7 +1,9 @@
 """GPU parity of the chunked tcgen05 prefill (bf16, dk = dv = 128) against the float64 oracle.
 
-Sizes escalate from one chunk to the full workloads. Metric: relative L2 over all elements of o
-and of the final states, bound 5e-3 (bf16 inputs).
+Both chunked paths are checked: the split path (intra-chunk kernel over all chunks, then the
+state pass; what kda_fwd runs with a full workspace) and the fused kernel (what it runs with the
+minimum workspace). Sizes escalate from one chunk to the full workloads. Metric: relative L2 over
+all elements of o and of the final states, bound 5e-3 (bf16 inputs).
 """
 
 import os
@@ -28,17 +30,21 @@ def _cuda():
     yield
 
 
-def _run(inp, chunk_size=64):
+PATHS = pytest.mark.parametrize("fused", [False, True], ids=["split", "fused"])
+
+
+def _run(inp, chunk_size=64, fused=False, workspace=None):
     g = to(inp, DEV)
     o, hT = kda.fwd(g["q"], g["k"], g["v"], g["log_g"], g["beta"], h0=g.get("h0"),
-                    cu_seqlens=g.get("cu_seqlens"), chunk_size=chunk_size)
+                    cu_seqlens=g.get("cu_seqlens"), chunk_size=chunk_size, fused=fused,
+                    workspace=workspace)
     torch.cuda.synchronize()
     st = kda.get_device_error()
     return o, hT, st
 
 
-def _check(inp, tol=TOL_BF16):
-    o, hT, st = _run(inp)
+def _check(inp, tol=TOL_BF16, fused=False):
+    o, hT, st = _run(inp, fused=fused)
     assert st == 0, "device error %d" % st
     o_ref, h_ref = oracle_fwd(inp)
     eo, eh = rel_l2(host(o), o_ref), rel_l2(host(hT), h_ref)
@@ -51,45 +57,55 @@ def test_chunk_path_is_selected():
     assert kda.fwd_algorithm(1, 64, 1, 128, 128, 1) == kda.CHUNK_64
 
 
-def test_one_full_chunk():
-    _check(synth.prefill_inputs("prefill-t4096", T=64, H=1, seed=11))
+@PATHS
+def test_one_full_chunk(fused):
+    _check(synth.prefill_inputs("prefill-t4096", T=64, H=1, seed=11), fused=fused)
 
 
-def test_partial_chunks_batch_and_h0():
-    _check(synth.prefill_inputs("prefill-t4096", B=2, T=200, H=3, h0_std=0.1, seed=12))
+@PATHS
+def test_partial_chunks_batch_and_h0(fused):
+    _check(synth.prefill_inputs("prefill-t4096", B=2, T=200, H=3, h0_std=0.1, seed=12), fused=fused)
 
 
 @pytest.mark.parametrize("T", [1, 63, 65, 127, 129, 333])
-def test_ragged_lengths(T):
-    _check(synth.prefill_inputs("long-t65536", B=1, T=T, H=2, seed=13 + T))
+@PATHS
+def test_ragged_lengths(T, fused):
+    _check(synth.prefill_inputs("long-t65536", B=1, T=T, H=2, seed=13 + T), fused=fused)
 
 
 @pytest.mark.parametrize("B,T,H", [(4, 200, 64), (2, 129, 128)])
-def test_many_chains_take_the_full_width_path(B, T, H):
+@PATHS
+def test_many_chains_take_the_full_width_path(B, T, H, fused):
     """With more (sequence, head) chains than half the SMs, one CTA owns all 128 value columns
     of a chain; check that variant with h0, batches and ragged lengths."""
-    _check(synth.prefill_inputs("prefill-t4096", B=B, T=T, H=H, h0_std=0.05, seed=17 + T))
+    _check(synth.prefill_inputs("prefill-t4096", B=B, T=T, H=H, h0_std=0.05, seed=17 + T),
+           fused=fused)
 
 
-def test_prefill_t4096_h16_full():
+@PATHS
+def test_prefill_t4096_h16_full(fused):
     """The T=4096, H=16 bf16 workload at full size."""
-    _check(synth.prefill_inputs("prefill-t4096"))
+    _check(synth.prefill_inputs("prefill-t4096"), fused=fused)
 
 
-def test_packed_edge_documents():
+@PATHS
+def test_packed_edge_documents(fused):
     lengths = [1, 63, 64, 65, 0, 130, 7, 200]
-    _check(synth.prefill_inputs("packed-8docs", lengths=lengths, H=4, h0_std=0.05, seed=14))
+    _check(synth.prefill_inputs("packed-8docs", lengths=lengths, H=4, h0_std=0.05, seed=14),
+           fused=fused)
 
 
-def test_packed_documents_scheduled_longest_first():
+@PATHS
+def test_packed_documents_scheduled_longest_first(fused):
     """Documents in increasing length: the scheduling permutation is far from the identity."""
     _check(synth.prefill_inputs("packed-8docs", lengths=[50, 100, 700, 1300, 2, 1301], H=8,
-                                h0_std=0.05, seed=18))
+                                h0_std=0.05, seed=18), fused=fused)
 
 
-def test_packed_8docs_full():
+@PATHS
+def test_packed_8docs_full(fused):
     """The packed 8-document workload (H = 32) at full size, every token and state."""
-    _check(synth.prefill_inputs("packed-8docs"))
+    _check(synth.prefill_inputs("packed-8docs"), fused=fused)
 
 
 def test_chunked_equals_per_token_path():
@@ -102,12 +118,13 @@ def test_chunked_equals_per_token_path():
     assert rel_l2(host(h1), host(h2)) <= TOL_BF16
 
 
+@PATHS
 @pytest.mark.parametrize("name", ["long-t65536", "long-t65536-slow"])
-def test_long_context_full_size_sampled_heads(name):
+def test_long_context_full_size_sampled_heads(name, fused):
     """B=2, T=65536, H=32 with h0: the GPU runs the whole batch; the oracle recomputes four
     (sequence, head) chains end to end (every token's output and the final state)."""
     inp = synth.prefill_inputs(name, device=DEV)
-    o, hT, st = _run(inp)
+    o, hT, st = _run(inp, fused=fused)
     assert st == 0
     picks = [(0, 0), (0, 31), (1, 7), (1, 20)]
     f = lambda t: t.float().cpu().numpy()
@@ -122,6 +139,25 @@ def test_long_context_full_size_sampled_heads(name):
         worst = (max(worst[0], eo), max(worst[1], eh))
     print("worst rel-L2 o %.3e hT %.3e" % worst)
     assert worst[0] <= TOL_BF16 and worst[1] <= TOL_BF16, worst
+
+
+def test_workspace_size_selects_the_path():
+    """A workspace below kda_fwd_workspace_size (but covering the minimum) runs the fused kernel:
+    bit-identical to fused=True; the full size runs the split path, which agrees within the
+    tolerance (it stores the factors in bf16)."""
+    inp = synth.prefill_inputs("packed-8docs", lengths=[300, 65, 1000], H=4, h0_std=0.02,
+                               seed=19)
+    T, N = inp["T"], inp["N"]
+    full = kda.fwd_workspace_size(1, T, 4, 128, 128, N)
+    small = kda.fwd_workspace_size_min(1, T, 4, 128, 128, N)
+    assert 0 < small < full
+    ws_small = torch.empty(full - 256, dtype=torch.uint8, device=DEV)
+    o1, h1, st1 = _run(inp, workspace=ws_small)
+    o2, h2, st2 = _run(inp, fused=True)
+    o3, h3, st3 = _run(inp)
+    assert st1 == st2 == st3 == 0
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+    assert rel_l2(host(o3), host(o2)) <= TOL_BF16 and rel_l2(host(h3), host(h2)) <= TOL_BF16
 
 
 def test_steep_decay_is_reported_as_range_error():
