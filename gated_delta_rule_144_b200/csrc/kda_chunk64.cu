@@ -338,8 +338,11 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     };
 
     bool stores_pending = false;   // intra mode: bulk stores still reading shared memory
+    // Thread that issues TMA copies: in the intra mode lane 0 of the last warp (the one with the
+    // least elementwise work), so that copy issue never delays thread 0's MMAs.
+    const int copier = kIntra ? kThreads - 32 : 0;
     if (has_cur) {
-        if (tid == 0) {
+        if (tid == copier) {
             issue_in(cur);
             issue_v(cur);
         }
@@ -460,7 +463,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             b4_pending = false;
         }
         if (kIntra && stores_pending) {   // the previous record's stores read R, [W; Q~] and K_end
-            if (tid == 0) bulk_wait_read_all();
+            if (tid == copier) bulk_wait_read_all();
             __syncthreads();
             stores_pending = false;
         }
@@ -553,7 +556,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         fence_proxy_async();
         __syncthreads();   // q, k, log g of chunk c fully consumed
         if (has_nxt) {
-            if (tid == 0) issue_in(nxt);
+            if (tid == copier) issue_in(nxt);
             in_pending = true;
             in_chunk = c + 1;
         }
@@ -826,7 +829,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mma_pending = false;
         tc_fence_after();
         if (has_nxt) {   // the V panel is free again
-            if (tid == 0) issue_v(nxt);
+            if (tid == copier) issue_v(nxt);
             v_pending = true;
             v_chunk = c + 1;
         }
@@ -876,7 +879,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             fence_proxy_async();
             tc_fence_before();
             __syncthreads();
-            if (tid == 0) {
+            if (tid == copier) {
                 const int rw = (int)(cur.rec * 128), rk = (int)(cur.rec * 64);
                 tma_store_2d(&omaps.wq, sb + OFF_WQ, 0, rw);
                 tma_store_2d(&omaps.wq, sb + OFF_WQ + 16384, 64, rw);
@@ -1017,7 +1020,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
         }
     }
-    if (kIntra && tid == 0) bulk_wait_all();   // stores complete before the CTA's smem goes away
+    if (kIntra && tid == copier) bulk_wait_all();   // stores complete before the smem goes away
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, kTmemCols);

@@ -20,8 +20,9 @@
 //   bf16(S^T) -> D (8 K steps) -> U^T -> S^T += U^T K_end (4 K steps);
 // the decay of S^T, the loads of U~^T and O~^T and the output of chunk c-1 (o = O~ + Q~ S, read
 // from the other of two D buffers, staged in shared memory and written by a TMA store) run while
-// the D product of chunk c is in flight. Thread 0 issues the TMA copies (two stages: chunk c+1
-// arrives while chunk c runs) and the MMAs. Every mbarrier wait is bounded; on expiry the CTA
+// the D product of chunk c is in flight. Thread 0 issues the MMAs only; lane 0 of warp 1 issues
+// the TMA loads (two stages: chunk c+1 arrives while chunk c runs) and lane 0 of warp 2 the output
+// stores, so that no copy issue delays an MMA on the critical chain. Every mbarrier wait is bounded; on expiry the CTA
 // records KDA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
 
 #include <cuda.h>
@@ -100,6 +101,7 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int qd = warp & 3, hs = warp >> 2;   // TMEM lane quarter, column half
     const int j = 32 * qd + lane;              // value column = TMEM lane
+    constexpr int kLoader = 32, kStorer = 64;  // threads that issue TMA loads / output stores
     const int unit = blockIdx.x;
     const int h = unit % args.H;
     const int n = args.order ? args.order[unit / args.H] : unit / args.H;
@@ -216,7 +218,7 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         const long long r0 = t0 + (long long)kC * cc;
         const int L = (int)min((long long)kC, t1 - r0);
         if (L == kC) {
-            if (tid == 0) {
+            if (tid == kStorer) {
                 tma_store_3d(&maps.o, sb + OFF_O + 16384 * (cc & 1), 0, h, (int)r0);
                 bulk_commit();
             }
@@ -230,7 +232,7 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         }
     };
 
-    if (tid == 0) {
+    if (tid == kLoader) {
         if (nchunks > 0) issue(0);
         if (nchunks > 1) issue(1);
     }
@@ -265,15 +267,10 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         }
         tmem_st_wait();
         // output tile (c-1)&1 is rewritten below; its previous store (chunk c-3) must be done
-        if (tid == 0 && c >= 3) bulk_wait_read_le1();
+        if (tid == kStorer && c >= 3) bulk_wait_read_le1();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        // stage (c+1)&1 held chunk c-1, fully consumed by now: fetch chunk c+1 into it
-        if (c >= 1 && c + 1 < nchunks) {
-            if (tid == 0) issue(c + 1);
-            issued = c + 2;
-        }
 
         // ---------------------------------------------------------------- D = S^T [W; Q~]^T
         if (tid == 0) {
@@ -285,6 +282,11 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         }
         mma1_pending = true;
         mma1_chunk = c;
+        // stage (c+1)&1 held chunk c-1, fully consumed by now: fetch chunk c+1 into it
+        if (c >= 1 && c + 1 < nchunks) {
+            if (tid == kLoader) issue(c + 1);
+            issued = c + 2;
+        }
 
         // ---------------------------------------------------------------- while D runs
         // decay: TS = S^T diag(e^{Gamma_end}) (the update accumulates into it)
@@ -366,7 +368,7 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         }
         tc_fence_after();
         if (nchunks > 0) {   // output of the last chunk
-            if (tid == 0 && nchunks >= 3) bulk_wait_read_le1();
+            if (tid == kStorer && nchunks >= 3) bulk_wait_read_le1();
             __syncthreads();
             stage_o(nchunks - 1);
             fence_proxy_async();
@@ -385,7 +387,7 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
             }
         }
     }
-    if (tid == 0) bulk_wait_all();   // output stores complete before the CTA's smem goes away
+    if (tid == kStorer) bulk_wait_all();   // output stores complete before the smem goes away
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, kTmemCols);
