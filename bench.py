@@ -136,7 +136,9 @@ class ClockSampler:
 KERNEL_SOURCES = {
     "kda_decode_d128": ["kda_decode.cu", "kda_internal.cuh"],
     "kda_recurrent": ["kda_recurrent.cu", "kda_internal.cuh"],
-    "kda_chunk64": ["kda_chunk64.cu", "kda_sm100.cuh", "kda_internal.cuh"],
+    "kda_chunk64": ["kda_chunk64.cu", "kda_sm100.cuh", "kda_internal.cuh", "kda_tma.cuh"],
+    "kda_chunk64_intra": ["kda_chunk64.cu", "kda_sm100.cuh", "kda_internal.cuh", "kda_tma.cuh"],
+    "kda_chunk_scan": ["kda_scan.cu", "kda_sm100.cuh", "kda_internal.cuh", "kda_tma.cuh"],
 }
 
 
@@ -151,7 +153,11 @@ def source_digest(kernel: str):
 
 
 def committed_traffic(kernel: str, workload: str):
-    """dram read+write bytes per launch from the committed ncu summary, if it is current."""
+    """dram read+write bytes per launch from the committed ncu summary, if it is current. For a
+    path of several kernels ("a+b"), the sum over its kernels, or None if any is missing."""
+    if "+" in kernel:
+        parts = [committed_traffic(k, workload) for k in kernel.split("+")]
+        return None if any(x is None for x in parts) else sum(parts)
     if not PROFILE_TRAFFIC.exists():
         return None
     try:
@@ -280,6 +286,8 @@ def run_ours(args):
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                 "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                 "traffic": traffic, "peak_kind": peak_kind, "kernel": kernel_name,
+                "launch": ("one kda_fwd call: intra-chunk kernel then state pass"
+                           if "+" in kernel_name else "one kda_fwd call"),
                 "algorithmic_bytes_per_launch": bytes_launch,
                 "avg_launch_ms": round(launch_ms, 4),
                 "flops_per_launch": FLOPS_PER_TOKEN_HEAD * B * T * H,
