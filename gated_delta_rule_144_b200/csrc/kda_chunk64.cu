@@ -83,7 +83,7 @@ struct Layout {
     static constexpr uint32_t OFF_BETA = OFF_MISC;         // f32 [64]
     static constexpr uint32_t OFF_DECAY = OFF_MISC + 256;  // f32 [128]
     static constexpr uint32_t OFF_LOUP = OFF_MISC + 768;   // f32 [4 blocks][2 halves][128]
-    static constexpr uint32_t OFF_BAR = OFF_MISC + 4864;   // 5 mbarriers
+    static constexpr uint32_t OFF_BAR = OFF_MISC + 4864;   // 6 mbarriers
     static constexpr uint32_t OFF_TMEM = OFF_BAR + 64;     // TMEM base address
     static constexpr uint32_t kSmemBytes = OFF_TMEM + 16 + 1024;  // + alignment slack
     static_assert(OFF_ZA + 16384 == OFF_C + 40960, "solve buffers fill the R/C region exactly");
@@ -259,7 +259,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     float* loup_s = reinterpret_cast<float*>(sm + OFF_LOUP);
     uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
     const uint32_t bar_in = sb + OFF_BAR, bar_v = bar_in + 8, bar_mma = bar_in + 16;
-    const uint32_t bar_b4 = bar_in + 24, bar_never = bar_in + 32;
+    const uint32_t bar_b4 = bar_in + 24, bar_never = bar_in + 32, bar_wy2 = bar_in + 40;
 
     if (tid == 0) {
         mbar_init(bar_in, 1);
@@ -267,6 +267,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mbar_init(bar_mma, 1);
         mbar_init(bar_b4, 1);
         mbar_init(bar_never, 1);
+        mbar_init(bar_wy2, 1);
         fence_mbar_init();
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
@@ -328,6 +329,8 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
     // outstanding asynchronous work, drained before exit if a wait expires
     bool in_pending = false, v_pending = false, mma_pending = false, b4_pending = false;
+    bool wy2_pending = false;   // intra mode: the transposed WY product (V^T [T; T']^T)
+    int wy2_count = 0;
     int in_chunk = 0, v_chunk = 0, b4_chunk = 0;
     uint32_t mma_phase = 0;
     bool aborted = false;
@@ -463,7 +466,8 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             b4_pending = false;
         }
         if (kIntra && stores_pending) {   // the previous record's stores read R, [W; Q~] and K_end
-            if (tid == copier) bulk_wait_read_all();
+            if (tid == kThreads - 32 || tid == kThreads - 64 || tid == kThreads - 96)
+                bulk_wait_read_all();
             __syncthreads();
             stores_pending = false;
         }
@@ -486,12 +490,10 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     rho[i] = __fdividef(1.f, suf[j][i]);
                     kap[i] = suf[j][i];
                     sig[i] = suf[j][i] * own[i];
-                    range_bad |= suf[j][i] < 1e-30f;
                 } else {
                     rho[i] = pre[j][i];
                     kap[i] = __fdividef(1.f, pre[j][i]);
                     sig[i] = suf[j][i];
-                    range_bad |= pre[j][i] < 1e-30f;
                 }
             }
             st_bf16x4(sm + OFF_R + toff(128, rb8, j), kk[0] * rho[0], kk[1] * rho[1],
@@ -509,7 +511,33 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                           kk[3] * sig[3] * xa[3]);
             }
         }
+        // the reciprocals above stay finite while every factor they invert is >= 1e-30; the
+        // running products only shrink, so the last prefix (upper half) or the first suffix
+        // (lower half) is the smallest
+#pragma unroll
+        for (int i = 0; i < 4; ++i) range_bad |= (hh == 0 ? suf[0][i] : pre[7][i]) < 1e-30f;
         if (range_bad) set_device_error(args.err, DEV_RANGE);
+        //   K+ = k e^{Gamma}, Q+ = q e^{Gamma}, K_end = k e^{Gamma_end - Gamma}
+        auto kplus_pass = [&]() {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = rbase + j;
+                float4 k4 = ld_bf16x4(ks + (r * kD + ch0) * 2);
+                const float4 q4 = ld_bf16x4(qs + (r * kD + ch0) * 2);
+                if (r >= L) k4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                float e[4], x[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    e[i] = F[i] * (hh == 0 ? pre[j][i] : own[i] * pre[j][i]);
+                    x[i] = G[i] * (hh == 0 ? suf[j][i] * own[i] : suf[j][i]);
+                }
+                const uint32_t o64 = toff(64, rb8, j);
+                st_bf16x4(sm + OFF_KPV + o64, k4.x * e[0], k4.y * e[1], k4.z * e[2], k4.w * e[3]);
+                st_bf16x4(sm + OFF_WQ + toff(128, rb8 + 8, j), q4.x * e[0], q4.y * e[1],
+                          q4.z * e[2], q4.w * e[3]);
+                st_bf16x4(sm + OFF_KE + o64, k4.x * x[0], k4.y * x[1], k4.z * x[2], k4.w * x[3]);
+            }
+        };
         fence_proxy_async();
         __syncthreads();
 
@@ -534,25 +562,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mma_pending = true;
 
         // ---------------------------------------------------------------- K+, Q+, K_end
-        //   K+ = k e^{Gamma}, Q+ = q e^{Gamma}, K_end = k e^{Gamma_end - Gamma}
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int r = rbase + j;
-            float4 k4 = ld_bf16x4(ks + (r * kD + ch0) * 2);
-            const float4 q4 = ld_bf16x4(qs + (r * kD + ch0) * 2);
-            if (r >= L) k4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            float e[4], x[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                e[i] = F[i] * (hh == 0 ? pre[j][i] : own[i] * pre[j][i]);
-                x[i] = G[i] * (hh == 0 ? suf[j][i] * own[i] : suf[j][i]);
-            }
-            const uint32_t o64 = toff(64, rb8, j);
-            st_bf16x4(sm + OFF_KPV + o64, k4.x * e[0], k4.y * e[1], k4.z * e[2], k4.w * e[3]);
-            st_bf16x4(sm + OFF_WQ + toff(128, rb8 + 8, j), q4.x * e[0], q4.y * e[1], q4.z * e[2],
-                      q4.w * e[3]);
-            st_bf16x4(sm + OFF_KE + o64, k4.x * x[0], k4.y * x[1], k4.z * x[2], k4.w * x[3]);
-        }
+        kplus_pass();
         fence_proxy_async();
         __syncthreads();   // q, k, log g of chunk c fully consumed
         if (has_nxt) {
@@ -808,27 +818,30 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     for (int s = 0; s < kC / 16; ++s)
                         umma_f16(tbase + TM_A, desc_at(dK, sb + OFF_TT + 32 * s),
                                  desc_at(dM8, sb + OFF_KPV + 2048 * s), id, s > 0);
+                    umma_commit(bar_mma);   // W and A_qk W: read out while the next runs
 #pragma unroll
                     for (int s = 0; s < kC / 16; ++s)
                         umma_f16(tbase + TM_A + 128, desc_at(dM8, sb + OFF_KPV + 16384 + 2048 * s),
                                  desc_at(dK, sb + OFF_TT + 32 * s), idt, s > 0);
+                    umma_commit(bar_wy2);
                 } else {
                     const uint32_t id = idesc_bf16(128, 128 + kDV, 0, 1);
 #pragma unroll
                     for (int s = 0; s < kC / 16; ++s)
                         umma_f16(tbase + TM_A, desc_at(dK, sb + OFF_TT + 32 * s),
                                  desc_at(dM8, sb + OFF_KPV + 2048 * s), id, s > 0);
+                    umma_commit(bar_mma);
                 }
-                umma_commit(bar_mma);
             }
             __syncwarp();
         }
         mma_pending = true;
+        wy2_pending = kIntra;
         if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
         ++mma_phase;
         mma_pending = false;
         tc_fence_after();
-        if (has_nxt) {   // the V panel is free again
+        if (!kIntra && has_nxt) {   // the V panel is free again
             if (tid == copier) issue_v(nxt);
             v_pending = true;
             v_chunk = c + 1;
@@ -862,6 +875,15 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
         }
         if constexpr (kIntra) {
+            if (!wait_all(bar_wy2, wy2_count & 1)) { aborted = true; break; }
+            ++wy2_count;
+            wy2_pending = false;
+            tc_fence_after();
+            if (has_nxt) {   // the V panel is free again
+                if (tid == copier) issue_v(nxt);
+                v_pending = true;
+                v_chunk = c + 1;
+            }
             // U~^T (TMEM columns 128-191) and O~^T (192-255), lane j = value column, into bf16
             // staging tiles [128 j][64 tokens] in the R region (128-byte swizzle), then one set
             // of bulk stores
@@ -879,12 +901,17 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             fence_proxy_async();
             tc_fence_before();
             __syncthreads();
-            if (tid == copier) {
-                const int rw = (int)(cur.rec * 128), rk = (int)(cur.rec * 64);
+            // three issuing threads (lane 0 of warps 5, 6, 7), two stores and one bulk group each
+            const int rw = (int)(cur.rec * 128), rk = (int)(cur.rec * 64);
+            if (tid == kThreads - 32) {
                 tma_store_2d(&omaps.wq, sb + OFF_WQ, 0, rw);
                 tma_store_2d(&omaps.wq, sb + OFF_WQ + 16384, 64, rw);
+                bulk_commit();
+            } else if (tid == kThreads - 64) {
                 tma_store_2d(&omaps.ke, sb + OFF_KE, 0, rk);
                 tma_store_2d(&omaps.ke, sb + OFF_KE + 8192, 64, rk);
+                bulk_commit();
+            } else if (tid == kThreads - 96) {
                 tma_store_2d(&omaps.ut, sb + OFF_R, 0, rw);
                 tma_store_2d(&omaps.ot, sb + OFF_R + 16384, 0, rw);
                 bulk_commit();
@@ -996,6 +1023,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (in_pending) mbar_wait(bar_in, in_chunk & 1, drain);
         if (v_pending) mbar_wait(bar_v, v_chunk & 1, drain);
         if (mma_pending) mbar_wait(bar_mma, mma_phase & 1, drain);
+        if (wy2_pending) mbar_wait(bar_wy2, wy2_count & 1, drain);
         if (b4_pending) mbar_wait(bar_b4, b4_chunk & 1, drain);
         __syncthreads();
     } else {
@@ -1020,7 +1048,8 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
         }
     }
-    if (kIntra && tid == copier) bulk_wait_all();   // stores complete before the smem goes away
+    if (kIntra && (tid == kThreads - 32 || tid == kThreads - 64 || tid == kThreads - 96))
+        bulk_wait_all();   // stores complete before the smem goes away
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, kTmemCols);

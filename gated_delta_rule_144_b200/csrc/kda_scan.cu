@@ -15,14 +15,14 @@
 // critical path:
 //   D = S^T [W; Q~]^T    (A = bf16 copy of S^T in TMEM, B = [W; Q~] K-major in shared memory)
 //   S^T += U^T K_end      (A = bf16 U^T in TMEM, B = K_end MN-major in shared memory)
-// 256 threads: warps w and w + 4 share TMEM lane quarter w mod 4 (lane j = value column j) and
-// split the columns of every TMEM row between them. Per chunk c the critical chain is
+// Eight data warps: warps w and w + 4 share TMEM lane quarter w mod 4 (lane j = value column j)
+// and split the columns of every TMEM row between them. A ninth warp only issues the MMAs, so that
+// no MMA issue waits behind a data warp's work. Per chunk c the critical chain is
 //   bf16(S^T) -> D (8 K steps) -> U^T -> S^T += U^T K_end (4 K steps);
 // the decay of S^T, the loads of U~^T and O~^T and the output of chunk c-1 (o = O~ + Q~ S, read
 // from the other of two D buffers, staged in shared memory and written by a TMA store) run while
-// the D product of chunk c is in flight. Thread 0 issues the MMAs only; lane 0 of warp 1 issues
-// the TMA loads (two stages: chunk c+1 arrives while chunk c runs) and lane 0 of warp 2 the output
-// stores, so that no copy issue delays an MMA on the critical chain. Every mbarrier wait is bounded; on expiry the CTA
+// the D product of chunk c is in flight. Lane 0 of warp 1 issues the TMA loads (two stages: chunk
+// c+1 arrives while chunk c runs) and lane 0 of warp 2 the output stores. Every mbarrier wait is bounded; on expiry the CTA
 // records KDA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
 
 #include <cuda.h>
@@ -43,7 +43,8 @@ using namespace sm100;
 
 constexpr int kC = 64;
 constexpr int kD = 128;
-constexpr int kThreads = 256;
+constexpr int kDataWarps = 8;
+constexpr int kThreads = 32 * kDataWarps + 32;   // + one warp that only issues MMAs
 
 // one pipeline stage (bytes from a 1024-aligned stage base)
 constexpr uint32_t ST_WQ = 0;        // [W; Q~] 128 x 128 bf16, K-major SW128: 2 panels of 16 KB
@@ -102,6 +103,8 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
     const int qd = warp & 3, hs = warp >> 2;   // TMEM lane quarter, column half
     const int j = 32 * qd + lane;              // value column = TMEM lane
     constexpr int kLoader = 32, kStorer = 64;  // threads that issue TMA loads / output stores
+    constexpr int kMma = 32 * kDataWarps;      // thread that issues the MMAs
+    const bool data = warp < kDataWarps;
     const int unit = blockIdx.x;
     const int h = unit % args.H;
     const int n = args.order ? args.order[unit / args.H] : unit / args.H;
@@ -156,7 +159,7 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
 
     // initial state, transposed: lane j, column c holds S[c][j]; this thread: c in [64 hs, +64)
 #pragma unroll 1
-    for (int p = 0; p < 2; ++p) {
+    for (int p = 0; p < (data ? 2 : 0); ++p) {
         float v[32];
         const int c0 = 64 * hs + 32 * p;
 #pragma unroll
@@ -253,10 +256,10 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
 
         // ---------------------------------------------------------------- bf16 S^T -> TB
         float va[32], vb[32];
-        tmem_ld32(tbase + lq + TS + 64 * hs, va);
-        tmem_ld32(tbase + lq + TS + 64 * hs + 32, vb);
-        tmem_ld_wait();
-        {
+        if (data) {
+            tmem_ld32(tbase + lq + TS + 64 * hs, va);
+            tmem_ld32(tbase + lq + TS + 64 * hs + 32, vb);
+            tmem_ld_wait();
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) pk[i] = pack2(va[2 * i], va[2 * i + 1]);
@@ -264,8 +267,8 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) pk[i] = pack2(vb[2 * i], vb[2 * i + 1]);
             tmem_st16u(tbase + lq + TB + 32 * hs + 16, pk);
+            tmem_st_wait();
         }
-        tmem_st_wait();
         // output tile (c-1)&1 is rewritten below; its previous store (chunk c-3) must be done
         if (tid == kStorer && c >= 3) bulk_wait_read_le1();
         tc_fence_before();
@@ -273,7 +276,8 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         tc_fence_after();
 
         // ---------------------------------------------------------------- D = S^T [W; Q~]^T
-        if (tid == 0) {
+        if (tid == kMma) {
+            tc_fence_after();
 #pragma unroll
             for (int s = 0; s < kD / 16; ++s)
                 umma_f16_ts(tbase + TD + 128 * (c & 1), tbase + TB + 8 * s,
@@ -290,7 +294,8 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
 
         // ---------------------------------------------------------------- while D runs
         // decay: TS = S^T diag(e^{Gamma_end}) (the update accumulates into it)
-        {
+        uint32_t ub[16];
+        if (data) {
             const float* dec = reinterpret_cast<const float*>(stp + ST_DEC) + 64 * hs;
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
@@ -301,23 +306,23 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
             }
             tmem_st32(tbase + lq + TS + 64 * hs, va);
             tmem_st32(tbase + lq + TS + 64 * hs + 32, vb);
-        }
-        // U~^T of this chunk: row j, tokens [32 hs, +32)
-        uint32_t ub[16];
+            // U~^T of this chunk: row j, tokens [32 hs, +32)
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const uint4 x = *reinterpret_cast<const uint4*>(stp + ST_UT + sw128_off(128, j, 32 * hs + 8 * m));
-            ub[4 * m] = x.x; ub[4 * m + 1] = x.y; ub[4 * m + 2] = x.z; ub[4 * m + 3] = x.w;
+            for (int m = 0; m < 4; ++m) {
+                const uint4 x = *reinterpret_cast<const uint4*>(
+                    stp + ST_UT + sw128_off(128, j, 32 * hs + 8 * m));
+                ub[4 * m] = x.x; ub[4 * m + 1] = x.y; ub[4 * m + 2] = x.z; ub[4 * m + 3] = x.w;
+            }
+            if (c >= 1) stage_o(c - 1);
+            tmem_st_wait();
         }
-        if (c >= 1) stage_o(c - 1);
-        tmem_st_wait();
 
         if (!wait_all(bar_mma1, (uint32_t)(c & 1))) { aborted = true; break; }
         mma1_pending = false;
         tc_fence_after();
 
         // ---------------------------------------------------------------- U^T = U~^T - (W S)^T
-        {
+        if (data) {
             float w[32];
             tmem_ld32(tbase + lq + TD + 128 * (c & 1) + 32 * hs, w);
             tmem_ld_wait();
@@ -328,19 +333,23 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
             tmem_st16u(tbase + lq + TU + 16 * hs, pk);
         }
         // O~^T of this chunk, for its output at the next step
+        if (data) {
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const uint4 x = *reinterpret_cast<const uint4*>(stp + ST_OT + sw128_off(128, j, 32 * hs + 8 * m));
-            ob[4 * m] = x.x; ob[4 * m + 1] = x.y; ob[4 * m + 2] = x.z; ob[4 * m + 3] = x.w;
+            for (int m = 0; m < 4; ++m) {
+                const uint4 x = *reinterpret_cast<const uint4*>(
+                    stp + ST_OT + sw128_off(128, j, 32 * hs + 8 * m));
+                ob[4 * m] = x.x; ob[4 * m + 1] = x.y; ob[4 * m + 2] = x.z; ob[4 * m + 3] = x.w;
+            }
+            tmem_st_wait();
         }
-        tmem_st_wait();
         fence_proxy_async();   // output tile c-1 -> TMA store
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
 
         // ---------------------------------------------------------------- S^T += U^T K_end
-        if (tid == 0) {
+        if (tid == kMma) {
+            tc_fence_after();
 #pragma unroll
             for (int s = 0; s < kC / 16; ++s)
                 umma_f16_ts(tbase + TS, tbase + TU + 8 * s, desc_at(dM8, st + ST_KE + 2048 * s),
@@ -370,12 +379,12 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         if (nchunks > 0) {   // output of the last chunk
             if (tid == kStorer && nchunks >= 3) bulk_wait_read_le1();
             __syncthreads();
-            stage_o(nchunks - 1);
+            if (data) stage_o(nchunks - 1);
             fence_proxy_async();
             __syncthreads();
             flush_o(nchunks - 1);
         }
-        if (args.hT) {
+        if (args.hT && data) {
 #pragma unroll 1
             for (int p = 0; p < 2; ++p) {
                 float v[32];
