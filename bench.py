@@ -135,6 +135,7 @@ class ClockSampler:
 
 KERNEL_SOURCES = {
     "kda_decode_d128": ["kda_decode.cu", "kda_internal.cuh"],
+    "kda_decode_tokens_d128": ["kda_decode.cu", "kda_internal.cuh"],
     "kda_recurrent": ["kda_recurrent.cu", "kda_internal.cuh"],
     "kda_chunk64": ["kda_chunk64.cu", "kda_sm100.cuh", "kda_internal.cuh", "kda_tma.cuh"],
     "kda_chunk64_intra": ["kda_chunk64.cu", "kda_sm100.cuh", "kda_internal.cuh", "kda_tma.cuh"],
@@ -393,6 +394,33 @@ def run_secondary(kda, synth, args, dev, stream, world, rank):
                      "roofline_frac": round(gbs / hbm_peak, 4), "peak": hbm_peak,
                      "kernel": "kda_decode_d128",
                      "traffic": committed_traffic("kda_decode_d128", "decode-n256")}
+    del d, od
+    # four rows per sequence against the decode state (kda_decode_tokens), in place
+    d = synth.decode_tokens_inputs("decode-rows-n256-t4", device=dev,
+                                   seed=shard.rank_seed(1053, rank))
+    od = torch.empty_like(d["v"])
+
+    def rstep():
+        kda.decode_tokens(d["q"], d["k"], d["v"], d["log_g"], d["beta"], d["S"], o=od)
+
+    for _ in range(max(3, args.warmup)):
+        rstep()
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms, per = time_launches(rstep, steps, stream)
+    barrier(world)
+    ms = max_over_ranks(total_ms, world, dev) / steps
+    state = d["S"].numel() * 4
+    io = sum(d[k].numel() * d[k].element_size() for k in ("q", "k", "v", "log_g", "beta"))
+    io += od.numel() * od.element_size()
+    by = 2 * state + io
+    gbs = by / (ms / 1e3) / 1e9
+    out["decode_rows"] = {"workload": "decode-rows-n256-t4", "N": 256, "T": 4, "H": 32,
+                          "bytes_per_step": by, "ms_per_step": round(ms, 4),
+                          "GB/s": round(gbs * world, 1), "GB/s_per_gpu": round(gbs, 1),
+                          "roofline_frac": round(gbs / hbm_peak, 4), "peak": hbm_peak,
+                          "tokens/s": round(256 * 4 * world / (ms / 1e3), 1),
+                          "kernel": "kda_decode_tokens_d128"}
     del d, od
     # packed 8-document prefill (H = 32)
     p = synth.prefill_inputs("packed-8docs", device=dev, seed=shard.rank_seed(1002, rank))

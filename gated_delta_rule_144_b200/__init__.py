@@ -19,7 +19,8 @@ from pathlib import Path
 
 import torch
 
-__all__ = ["fwd", "fwd_no_alloc", "decode_step", "get_device_error", "fwd_workspace_size",
+__all__ = ["fwd", "fwd_no_alloc", "decode_step", "decode_tokens", "get_device_error",
+           "fwd_workspace_size",
            "fwd_workspace_size_min", "fwd_algorithm",
            "KdaError",
            "library_path", "lib", "CHUNK_AUTO", "CHUNK_PER_TOKEN", "CHUNK_64"]
@@ -75,6 +76,8 @@ def lib():
     L.kda_fwd_workspace_size_min.restype = sz
     L.kda_decode_step.argtypes = [i32, i32, i32, i32, i32, p, p, p, p, p, p, p, p]
     L.kda_decode_step.restype = i32
+    L.kda_decode_tokens.argtypes = [i32, i32, i32, i32, i32, i32, p, p, p, p, p, p, p, p]
+    L.kda_decode_tokens.restype = i32
     L.kda_get_device_error.argtypes = [p]
     L.kda_get_device_error.restype = i32
     L.kda_status_string.argtypes = [i32]
@@ -283,6 +286,41 @@ def decode_step(q, k, v, log_g, beta, S, *, o=None, stream=None):
                                    _ptr(log_g), _ptr(beta), _ptr(S), _ptr(o),
                                    _stream(stream, dev))
     _check(st, "kda_decode_step")
+    return o
+
+
+def decode_tokens(q, k, v, log_g, beta, S, *, o=None, stream=None):
+    """T tokens for each of N sequences from their decode state (``kda_decode_tokens``); S is
+    updated in place to the state after the last token.
+
+    q, k, log_g: [N, T, H, dk]; v: [N, T, H, dv]; beta: [N, T, H]; S: [N, H, dk, dv] fp32.
+    Returns o [N, T, H, dv] in the dtype of q.
+    """
+    lib()
+    _dev(q, "q")
+    dev = q.device
+    if q.dim() != 4:
+        raise ValueError("q must be [N, T, H, dk]")
+    N, T, H, dk = q.shape
+    dt = q.dtype
+    _dtype_code(q)
+    _dev(k, "k", dt, (N, T, H, dk), dev)
+    _dev(log_g, "log_g", torch.float32, (N, T, H, dk), dev)
+    _dev(v, "v", dt, None, dev)
+    if v.dim() != 4 or tuple(v.shape[:3]) != (N, T, H):
+        raise ValueError("v must be [N, T, H, dv]")
+    dv = v.shape[3]
+    _dev(beta, "beta", dt, (N, T, H), dev)
+    _dev(S, "S", torch.float32, (N, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((N, T, H, dv), dtype=dt, device=dev)
+    else:
+        _dev(o, "o", dt, (N, T, H, dv), dev)
+    with torch.cuda.device(dev):
+        st = lib().kda_decode_tokens(N, H, T, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+                                     _ptr(log_g), _ptr(beta), _ptr(S), _ptr(o),
+                                     _stream(stream, dev))
+    _check(st, "kda_decode_tokens")
     return o
 
 

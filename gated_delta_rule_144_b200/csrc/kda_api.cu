@@ -312,6 +312,47 @@ kda_status_t kda_decode_step(int N, int H, int dk, int dv, kda_dtype_t dtype, co
     return KDA_OK;
 }
 
+kda_status_t kda_decode_tokens(int N, int H, int T, int dk, int dv, kda_dtype_t dtype,
+                               const void* q, const void* k, const void* v, const float* log_g,
+                               const void* beta, float* S_inout, void* o, kda_stream_t stream) {
+    t_last_error[0] = 0;
+    if (N < 0 || H < 1 || T < 0 || dk < 1 || dv < 1)
+        return fail(KDA_ERR_INVALID_ARG, "bad sizes N=%d H=%d T=%d dk=%d dv=%d", N, H, T, dk,
+                    dv);
+    if (dtype != KDA_F32 && dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (dk > 256 || dv > 256) return fail(KDA_ERR_UNSUPPORTED, "decode supports dk, dv <= 256");
+    if ((int64_t)N * T * H > (int64_t)1 << 40) return fail(KDA_ERR_INVALID_ARG, "problem too large");
+    kda_status_t st;
+    const bool any = N > 0 && T > 0;
+    if ((st = check_ptr(q, "q", any)) || (st = check_ptr(k, "k", any)) ||
+        (st = check_ptr(v, "v", any)) || (st = check_ptr(log_g, "log_g", any)) ||
+        (st = check_ptr(beta, "beta", any)) || (st = check_ptr(S_inout, "S_inout", any)) ||
+        (st = check_ptr(o, "o", any)))
+        return st;
+    if (!any) return KDA_OK;
+    unsigned* err = nullptr;
+    if ((st = device_error_word(&err)) != KDA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (dk == 128 && dv == 128) {
+        kda::DecodeParams p{q, k, v, log_g, beta, S_inout, o, N, H, dk, dv,
+                            dtype == KDA_BF16, err};
+        e = kda::launch_decode_tokens_d128(p, T, s);
+    } else {
+        // general sizes: the per-token walk over N sequences of T tokens, state in place
+        kda::FwdParams p{};
+        p.q = q; p.k = k; p.v = v; p.log_g = log_g; p.beta = beta; p.h0 = S_inout;
+        p.cu_seqlens = nullptr; p.o = o; p.hT = S_inout;
+        p.B = N; p.T = T; p.H = H; p.dk = dk; p.dv = dv; p.N = N;
+        p.bf16 = dtype == KDA_BF16;
+        p.err = err;
+        e = kda::launch_recurrent(p, s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "kda_decode_tokens launch");
+    return KDA_OK;
+}
+
 kda_status_t kda_get_device_error(kda_stream_t stream) {
     t_last_error[0] = 0;
     unsigned* err = nullptr;

@@ -118,7 +118,122 @@ decode_d128_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     }
 }
 
+// T tokens per (sequence, head) against the same state layout (speculative "verify rows", or a
+// short prefill continuing a decode state): the state is read once, updated T times in
+// registers and written once, so the HBM cost stays one state round trip per call. Token t of
+// sequence n reads row (n * T + t) of the [N, T, H, d] inputs. The inputs of up to kRowGroup
+// tokens are staged in shared memory at once, their loads in flight together with the state's,
+// so the token loop itself waits on no global load and no barrier. The arithmetic of each token
+// is that of decode_d128_kernel, in the same order.
+constexpr int kRowGroup = 8;
+
+template <typename Tin>
+__global__ void __launch_bounds__(128)
+decode_d128_tokens_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                          const Tin* __restrict__ v, const float* __restrict__ log_g,
+                          const Tin* __restrict__ beta, float* __restrict__ S,
+                          Tin* __restrict__ o, int H, int T) {
+    __shared__ __align__(16) float s_q[kRowGroup][kD], s_k[kRowGroup][kD], s_g[kRowGroup][kD],
+        s_v[kRowGroup][kD];
+    __shared__ float s_b[kRowGroup];
+    const int unit = blockIdx.x;  // n * H + h
+    const int n = unit / H, h = unit - n * H;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int phase = lane >> 3;
+    const int col = warp * 32 + (lane & 7) * 4;
+
+    float4* Sp = reinterpret_cast<float4*>(S + (size_t)unit * kD * kD);
+    float4 s[kRowsPerLane];
+#pragma unroll
+    for (int i = 0; i < kRowsPerLane; ++i) {
+        const int r = phase + 4 * i;
+        s[i] = __ldcs(Sp + (r * kD + col) / 4);
+    }
+
+    auto row = [&](int t) { return ((size_t)n * T + t) * H + h; };   // token row index
+    for (int t0 = 0; t0 < T; t0 += kRowGroup) {
+        const int nt = min(kRowGroup, T - t0);
+        if (t0 > 0) __syncthreads();   // the previous group's rows are no longer read
+        for (int u = 0; u < nt; ++u) {
+            const size_t r = row(t0 + u);
+            s_q[u][tid] = load_elem(q, r * kD + tid);
+            s_k[u][tid] = load_elem(k, r * kD + tid);
+            s_g[u][tid] = expf(log_g[r * kD + tid]);
+            s_v[u][tid] = load_elem(v, r * kD + tid);
+        }
+        if (tid < nt) s_b[tid] = load_elem(beta, row(t0 + tid));
+        __syncthreads();
+        for (int u = 0; u < nt; ++u) {
+            const float4 vv = *reinterpret_cast<const float4*>(&s_v[u][col]);
+            const float b = s_b[u];
+            float4 m = make_float4(0.f, 0.f, 0.f, 0.f), p = m;
+            float qk = 0.f;
+#pragma unroll
+            for (int i = 0; i < kRowsPerLane; ++i) {
+                const int r = phase + 4 * i;
+                const float g = s_g[u][r], kr = s_k[u][r], qr = s_q[u][r];
+                s[i].x *= g; s[i].y *= g; s[i].z *= g; s[i].w *= g;
+                m.x = fmaf(kr, s[i].x, m.x); m.y = fmaf(kr, s[i].y, m.y);
+                m.z = fmaf(kr, s[i].z, m.z); m.w = fmaf(kr, s[i].w, m.w);
+                p.x = fmaf(qr, s[i].x, p.x); p.y = fmaf(qr, s[i].y, p.y);
+                p.z = fmaf(qr, s[i].z, p.z); p.w = fmaf(qr, s[i].w, p.w);
+                qk = fmaf(qr, kr, qk);
+            }
+#pragma unroll
+            for (int off = 8; off <= 16; off <<= 1) {
+                m.x += __shfl_xor_sync(0xffffffffu, m.x, off);
+                m.y += __shfl_xor_sync(0xffffffffu, m.y, off);
+                m.z += __shfl_xor_sync(0xffffffffu, m.z, off);
+                m.w += __shfl_xor_sync(0xffffffffu, m.w, off);
+                p.x += __shfl_xor_sync(0xffffffffu, p.x, off);
+                p.y += __shfl_xor_sync(0xffffffffu, p.y, off);
+                p.z += __shfl_xor_sync(0xffffffffu, p.z, off);
+                p.w += __shfl_xor_sync(0xffffffffu, p.w, off);
+                qk += __shfl_xor_sync(0xffffffffu, qk, off);
+            }
+            float4 d;
+            d.x = b * (vv.x - m.x); d.y = b * (vv.y - m.y);
+            d.z = b * (vv.z - m.z); d.w = b * (vv.w - m.w);
+            if (phase == 0) {
+                float4 out;
+                out.x = fmaf(qk, d.x, p.x); out.y = fmaf(qk, d.y, p.y);
+                out.z = fmaf(qk, d.z, p.z); out.w = fmaf(qk, d.w, p.w);
+                store_v4(o + row(t0 + u) * kD + col, out);
+            }
+#pragma unroll
+            for (int i = 0; i < kRowsPerLane; ++i) {
+                const float kr = s_k[u][phase + 4 * i];
+                s[i].x = fmaf(kr, d.x, s[i].x); s[i].y = fmaf(kr, d.y, s[i].y);
+                s[i].z = fmaf(kr, d.z, s[i].z); s[i].w = fmaf(kr, d.w, s[i].w);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < kRowsPerLane; ++i) {
+        const int r = phase + 4 * i;
+        __stcs(Sp + (r * kD + col) / 4, s[i]);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_decode_tokens_d128(const DecodeParams& p, int T, cudaStream_t stream) {
+    const int64_t units = (int64_t)p.N * p.H;
+    if (units == 0 || T <= 0) return cudaSuccess;
+    if (units > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    if (p.bf16)
+        decode_d128_tokens_kernel<__nv_bfloat16><<<(unsigned)units, 128, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(p.q), static_cast<const __nv_bfloat16*>(p.k),
+            static_cast<const __nv_bfloat16*>(p.v), p.log_g,
+            static_cast<const __nv_bfloat16*>(p.beta), p.S, static_cast<__nv_bfloat16*>(p.o),
+            p.H, T);
+    else
+        decode_d128_tokens_kernel<float><<<(unsigned)units, 128, 0, stream>>>(
+            static_cast<const float*>(p.q), static_cast<const float*>(p.k),
+            static_cast<const float*>(p.v), p.log_g, static_cast<const float*>(p.beta), p.S,
+            static_cast<float*>(p.o), p.H, T);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_decode_d128(const DecodeParams& p, cudaStream_t stream) {
     const int64_t units = (int64_t)p.N * p.H;

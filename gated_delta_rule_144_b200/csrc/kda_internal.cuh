@@ -79,6 +79,8 @@ cudaError_t launch_doc_order(const int32_t* cu_seqlens, int N, int32_t* order,
                              cudaStream_t stream);
 cudaError_t launch_recurrent(const FwdParams& p, cudaStream_t stream);
 cudaError_t launch_decode_d128(const DecodeParams& p, cudaStream_t stream);
+// T tokens per sequence ([N, T, H, d] inputs), state read once and written once (d = 128).
+cudaError_t launch_decode_tokens_d128(const DecodeParams& p, int T, cudaStream_t stream);
 cudaError_t launch_chunk64(const FwdParams& p, cudaStream_t stream);
 // Split chunked prefill: map[g] for packed documents (sets DEV_BAD_SEQLENS on a malformed
 // cu_seqlens), the intra-chunk kernel over all records, then the state pass over all chains.

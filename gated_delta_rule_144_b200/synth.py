@@ -61,6 +61,10 @@ WORKLOADS = {
                             h0_std=0.02),
     "long-t65536-slow": Workload("long-t65536-slow", 4, "prefill", B=2, T=65536, H=32,
                                  decay_mu=-2.0, h0_std=0.02),
+    # several rows per sequence against the decode state (verify rows of batched decoding):
+    # the decode workload's sequences and distributions with T = 4 rows each
+    "decode-rows-n256-t4": Workload("decode-rows-n256-t4", 3, "decode", N=256, T=4, H=32,
+                                    state_std=0.02),
 }
 
 _TORCH_DTYPE = {"bf16": torch.bfloat16, "f32": torch.float32}
@@ -139,6 +143,28 @@ def prefill_inputs(w: Workload | str, device="cpu", *, B=None, T=None, H=None, l
     h0 = _normal(gen, (N, H, dk, dv), device, std=hstd) if hstd > 0 else None
     return dict(q=q, k=k, v=v, log_g=log_g, beta=beta, h0=h0, cu_seqlens=cu, lengths=lengths,
                 B=B, T=T, H=H, dk=dk, dv=dv, N=N, dtype=dtype or w.dtype, seed=seed)
+
+
+def decode_tokens_inputs(w: Workload | str = "decode-rows-n256-t4", device="cpu", *, N=None,
+                         T=None, H=None, seed=None, dtype=None, dk=None, dv=None,
+                         decay_mu=None, state_std=None):
+    """Inputs of T decode rows per sequence: q, k, log_g [N, T, H, dk], v [N, T, H, dv],
+    beta [N, T, H] (drawn like a prefill batch of N sequences) and the fp32 state S [N, H, dk, dv]
+    ~ N(0, state_std^2)."""
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    N = N or w.N
+    T = w.T if T is None else T
+    H = H or w.H
+    seed = 1000 + w.index + 50 if seed is None else seed
+    sstd = w.state_std if state_std is None else state_std
+    p = prefill_inputs("prefill-t4096", device, B=N, T=T, H=H, seed=seed,
+                       dtype=dtype or w.dtype, dk=dk or w.dk, dv=dv or w.dv,
+                       decay_mu=w.decay_mu if decay_mu is None else decay_mu, h0_std=sstd)
+    S = p["h0"] if p["h0"] is not None else torch.zeros(
+        (N, H, p["dk"], p["dv"]), dtype=torch.float32, device=device)
+    return dict(q=p["q"], k=p["k"], v=p["v"], log_g=p["log_g"], beta=p["beta"], S=S, N=N, T=T,
+                H=H, dk=p["dk"], dv=p["dv"], dtype=dtype or w.dtype, seed=seed)
 
 
 def decode_inputs(w: Workload | str = "decode-n256", device="cpu", *, N=None, H=None, seed=None,

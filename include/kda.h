@@ -184,6 +184,27 @@ kda_status_t kda_decode_step(int N, int H, int dk, int dv, kda_dtype_t dtype, co
                              float* S_inout, void* o, kda_stream_t stream);
 
 /*
+ * kda_decode_tokens - advance N sequences by T tokens each from their decode state, in place:
+ * the recurrence of the GLM-5.3-Flash model card's Kimi Delta Attention snippet, token by token,
+ * starting from S_inout and leaving the final state there. It serves rows that run against a
+ * decode state several at a time, such as the verify rows of batched decoding (metrale
+ * glm5next_layer, decoder-layer invariants: decode_batched gives verify row t its own slot).
+ * For d = 128 the state crosses HBM once per call (read once, updated T times in registers,
+ * written once), so T tokens cost about what one decode step costs.
+ *
+ *   q, k, log_g : [N, T, H, dk] (q, k in dtype, log_g float32)    v, o : [N, T, H, dv] dtype
+ *   beta        : [N, T, H] dtype
+ *   S_inout     : [N, H, dk, dv] float32, read and overwritten with the state after token T.
+ *   o           : output [N, T, H, dv], row t the read-out after token t.
+ * T = 1 is kda_decode_step (same layouts, same arithmetic order); T = 0 or N = 0 does nothing.
+ * S_inout must not alias any other argument. dk, dv <= 256. Host-checkable errors return before
+ * any launch.
+ */
+kda_status_t kda_decode_tokens(int N, int H, int T, int dk, int dv, kda_dtype_t dtype,
+                               const void* q, const void* k, const void* v, const float* log_g,
+                               const void* beta, float* S_inout, void* o, kda_stream_t stream);
+
+/*
  * kda_get_device_error - synchronise `stream`, then return and clear the sticky device error
  * word (KDA_OK, KDA_ERR_BAD_SEQLENS, KDA_ERR_TIMEOUT or KDA_ERR_RANGE), or KDA_ERR_CUDA if
  * the synchronisation itself failed. The word is per device and shared by all streams.

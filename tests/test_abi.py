@@ -31,7 +31,8 @@ def _declared_functions():
 
 def test_header_declares_the_entry_points():
     names = _declared_functions()
-    for must in ("kda_fwd", "kda_decode_step", "kda_get_device_error", "kda_status_string",
+    for must in ("kda_fwd", "kda_decode_step", "kda_decode_tokens", "kda_get_device_error",
+                 "kda_status_string",
                  "kda_fwd_workspace_size", "kda_last_error", "kda_version"):
         assert must in names
 
@@ -114,6 +115,20 @@ def _split_bytes(B, T, H, N, packed):
     R = G * H
     order = up(4 * N) if packed and 2 <= N <= 2048 else 0
     return order + (up(4 * G) if packed else 0) + up(512 * R) + R * (32768 + 3 * 16384)
+
+
+def test_decode_tokens_rejects_on_host(L):
+    P = ctypes.c_void_p
+    args = lambda **kw: [kw.get(n, P(FAKE)) for n in ("q", "k", "v", "g", "b", "S", "o")]
+    assert L.kda_decode_tokens(1, 1, -1, 128, 128, 1, *args(), None) == 1
+    assert L.kda_decode_tokens(1, 0, 4, 128, 128, 1, *args(), None) == 1
+    assert L.kda_decode_tokens(1, 1, 4, 128, 128, 9, *args(), None) == 1
+    assert L.kda_decode_tokens(1, 1, 4, 512, 128, 1, *args(), None) == 2
+    assert L.kda_decode_tokens(1, 1, 4, 128, 128, 1, *args(S=None), None) == 1
+    assert L.kda_decode_tokens(1, 1, 4, 128, 128, 1, *args(q=P(FAKE + 2)), None) == 1
+    # nothing to do: no pointer is needed
+    assert L.kda_decode_tokens(1, 1, 0, 128, 128, 1, None, None, None, None, None, None, None,
+                               None) == 0
 
 
 def test_workspace_size_is_host_only(L):
