@@ -444,6 +444,35 @@ def run_secondary(kda, synth, args, dev, stream, world, rank):
                              "tokens": p["T"], "ms_per_step": round(ms, 4),
                              "tokens/s": round(p["T"] * world / (ms / 1e3), 1),
                              "roofline_frac": round(by / (ms / 1e3) / 1e9 / hbm_peak, 4)}
+    # gated per-head RMSNorm epilogue on the same workload: kda_fwd_normed against the plain call
+    # followed by the separate norm pass through the Python API
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(shard.rank_seed(1090, rank))
+    gate = torch.randn(o.shape, generator=gen, device=dev).to(o.dtype)
+    nw = torch.rand(128, generator=gen, device=dev) + 0.5
+
+    def nstep():
+        kda.fwd(p["q"], p["k"], p["v"], p["log_g"], p["beta"], cu_seqlens=p["cu_seqlens"],
+                o=o, hT=hT, chunk_size=args.chunk_size, workspace=ws, fused=args.fused,
+                out_norm=(gate, nw, 1e-6))
+
+    def ustep():
+        pstep()
+        kda.out_norm_gated(o, gate, nw, 1e-6, y=o)
+
+    res = {}
+    for name, fn in (("normed", nstep), ("separate", ustep)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        barrier(world)
+        total_ms, _ = time_launches(fn, args.steps, stream)
+        barrier(world)
+        res[name] = round(max_over_ranks(total_ms, world, dev) / args.steps, 4)
+    out["packed_prefill_normed"] = {"workload": "packed-8docs", "epilogue": "gated RMSNorm",
+                                    "ms_normed_call": res["normed"],
+                                    "ms_plain_then_norm": res["separate"],
+                                    "ms_plain": out["packed_prefill"]["ms_per_step"]}
     if kda.get_device_error() != 0:
         raise RuntimeError("device error in the secondary runs")
     return out

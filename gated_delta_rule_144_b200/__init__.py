@@ -19,7 +19,8 @@ from pathlib import Path
 
 import torch
 
-__all__ = ["fwd", "fwd_no_alloc", "decode_step", "decode_tokens", "get_device_error",
+__all__ = ["fwd", "fwd_no_alloc", "out_norm_gated", "decode_step", "decode_tokens",
+           "get_device_error",
            "fwd_workspace_size",
            "fwd_workspace_size_min", "fwd_algorithm",
            "KdaError",
@@ -47,6 +48,10 @@ class FwdDesc(ctypes.Structure):
                 ("dtype", ctypes.c_int), ("chunk_size", ctypes.c_int)]
 
 
+class OutNorm(ctypes.Structure):
+    _fields_ = [("gate", ctypes.c_void_p), ("weight", ctypes.c_void_p), ("eps", ctypes.c_float)]
+
+
 _lib = None
 
 
@@ -66,6 +71,11 @@ def lib():
     p, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     L.kda_fwd.argtypes = [ctypes.POINTER(FwdDesc), p, p, p, p, p, p, p, p, p, p, sz, p]
     L.kda_fwd.restype = i32
+    L.kda_fwd_normed.argtypes = [ctypes.POINTER(FwdDesc), p, p, p, p, p, p, p,
+                                 ctypes.POINTER(OutNorm), p, p, p, sz, p]
+    L.kda_fwd_normed.restype = i32
+    L.kda_out_norm_gated.argtypes = [ctypes.c_longlong, i32, i32, p, p, p, ctypes.c_float, p, p]
+    L.kda_out_norm_gated.restype = i32
     L.kda_fwd_no_alloc.argtypes = [ctypes.POINTER(FwdDesc), p, p, p, p, p, p, p, p, p, p]
     L.kda_fwd_no_alloc.restype = i32
     L.kda_fwd_algorithm.argtypes = [ctypes.POINTER(FwdDesc), i32]
@@ -157,7 +167,7 @@ def fwd_workspace_size(B, T, H, dk, dv, num_seqs, dtype=torch.bfloat16, chunk_si
 
 def fwd(q, k, v, log_g, beta, h0=None, cu_seqlens=None, *, chunk_size: int = CHUNK_AUTO,
         output_final_state: bool = True, o=None, hT=None, workspace=None, fused: bool = False,
-        stream=None):
+        out_norm=None, stream=None):
     """Prefill (``kda_fwd``): the recurrence over whole sequences or packed documents.
 
     q, k, log_g: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H]; q/k/v/beta share one dtype
@@ -166,6 +176,9 @@ def fwd(q, k, v, log_g, beta, h0=None, cu_seqlens=None, *, chunk_size: int = CHU
     None). Outputs may be passed in preallocated. The workspace (a uint8 device tensor) is
     allocated here when not given: kda_fwd_workspace_size bytes (the split chunked path), or,
     with fused=True, only kda_fwd_workspace_size_min bytes (the fused chunked kernel).
+    out_norm = (gate, weight, eps) applies the gated per-head RMSNorm (``kda_fwd_normed``): the
+    returned output is y = o / sqrt(mean(o^2) + eps) * weight * sigmoid(gate); gate is shaped and
+    typed like o, weight is fp32 [dv].
     """
     lib()
     _dev(q, "q")
@@ -213,12 +226,44 @@ def fwd(q, k, v, log_g, beta, h0=None, cu_seqlens=None, *, chunk_size: int = CHU
         if workspace.numel() < need:
             raise ValueError("workspace needs at least %d bytes" % need)
     ws_bytes = 0 if workspace is None else workspace.numel()
+    if out_norm is not None:
+        gate, weight, eps = out_norm
+        _dev(gate, "gate", dt, (B, T, H, dv), dev)
+        _dev(weight, "weight", torch.float32, (dv,), dev)
+        nrm = OutNorm(gate.data_ptr(), weight.data_ptr(), float(eps))
+        with torch.cuda.device(dev):
+            st = lib().kda_fwd_normed(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v),
+                                      _ptr(log_g), _ptr(beta), _ptr(h0), _ptr(cu_seqlens),
+                                      ctypes.byref(nrm), _ptr(o), _ptr(hT), _ptr(workspace),
+                                      ws_bytes, _stream(stream, dev))
+        _check(st, "kda_fwd_normed")
+        return o, hT
     with torch.cuda.device(dev):
         st = lib().kda_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(log_g),
                            _ptr(beta), _ptr(h0), _ptr(cu_seqlens), _ptr(o), _ptr(hT),
                            _ptr(workspace), ws_bytes, _stream(stream, dev))
     _check(st, "kda_fwd")
     return o, hT
+
+
+def out_norm_gated(x, gate, weight, eps: float, *, y=None, stream=None):
+    """The gated per-head RMSNorm alone (``kda_out_norm_gated``) over the last axis of x:
+    y = x / sqrt(mean(x^2) + eps) * weight * sigmoid(gate). y may be x (in place)."""
+    lib()
+    _dev(x, "x")
+    dev = x.device
+    dv = x.shape[-1]
+    _dev(gate, "gate", x.dtype, tuple(x.shape), dev)
+    _dev(weight, "weight", torch.float32, (dv,), dev)
+    if y is None:
+        y = torch.empty_like(x)
+    else:
+        _dev(y, "y", x.dtype, tuple(x.shape), dev)
+    with torch.cuda.device(dev):
+        st = lib().kda_out_norm_gated(x.numel() // dv, dv, _dtype_code(x), _ptr(x), _ptr(gate),
+                                      _ptr(weight), float(eps), _ptr(y), _stream(stream, dev))
+    _check(st, "kda_out_norm_gated")
+    return y
 
 
 def fwd_no_alloc(q, k, v, log_g, beta, h0, cu_seqlens, o, hT, *, chunk_size: int = CHUNK_AUTO,

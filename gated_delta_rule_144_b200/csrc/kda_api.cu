@@ -198,10 +198,12 @@ size_t kda_fwd_workspace_size_min(const kda_fwd_desc_t* desc) {
     return order_bytes(desc, path);
 }
 
-kda_status_t kda_fwd(const kda_fwd_desc_t* d, const void* q, const void* k, const void* v,
-                     const float* log_g, const void* beta, const float* h0,
-                     const int32_t* cu_seqlens, void* o, float* hT, void* workspace,
-                     size_t workspace_bytes, kda_stream_t stream) {
+// kda_fwd with an optional gated RMSNorm epilogue (norm == nullptr: none).
+static kda_status_t fwd_impl(const kda_fwd_desc_t* d, const void* q, const void* k,
+                             const void* v, const float* log_g, const void* beta,
+                             const float* h0, const int32_t* cu_seqlens, void* o, float* hT,
+                             void* workspace, size_t workspace_bytes,
+                             const kda_out_norm_t* norm, kda_stream_t stream) {
     t_last_error[0] = 0;
     Path path;
     kda_status_t st = check_fwd_desc(d, cu_seqlens != nullptr, &path);
@@ -215,6 +217,12 @@ kda_status_t kda_fwd(const kda_fwd_desc_t* d, const void* q, const void* k, cons
         (st = check_ptr(cu_seqlens, "cu_seqlens", false)))
         return st;
     if (tokens && !beta) return fail(KDA_ERR_INVALID_ARG, "beta is NULL");
+    if (norm) {
+        if ((st = check_ptr(norm->gate, "norm gate", tokens)) ||
+            (st = check_ptr(norm->weight, "norm weight", tokens)))
+            return st;
+        if (!(norm->eps >= 0.f)) return fail(KDA_ERR_INVALID_ARG, "norm eps must be >= 0");
+    }
     SplitLayout L;
     const bool split = tokens && split_layout(d, path, cu_seqlens != nullptr, &L) && workspace &&
                        aligned16(workspace) && workspace_bytes >= L.total;
@@ -232,6 +240,14 @@ kda_status_t kda_fwd(const kda_fwd_desc_t* d, const void* q, const void* k, cons
     p.bf16 = d->dtype == KDA_BF16;
     p.doc_order = nullptr;
     if ((st = device_error_word(&p.err)) != KDA_OK) return st;
+    // the epilogue runs as one bandwidth-bound pass after the prefill, on every path (measured
+    // faster than folding it into the split path's state pass, which is latency-bound)
+    auto norm_after = [&]() -> cudaError_t {
+        if (!norm || !tokens) return cudaSuccess;
+        return kda::launch_out_norm_gated(o, norm->gate, norm->weight, norm->eps, o,
+                                          (long long)d->B * d->T * d->H, d->dv, p.bf16,
+                                          reinterpret_cast<cudaStream_t>(stream));
+    };
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
     if (split) {
@@ -260,6 +276,8 @@ kda_status_t kda_fwd(const kda_fwd_desc_t* d, const void* q, const void* k, cons
         if (e != cudaSuccess) return cuda_fail(e, "kda_fwd intra-chunk launch");
         e = kda::launch_chunk_scan(p, s);
         if (e != cudaSuccess) return cuda_fail(e, "kda_fwd state-pass launch");
+        e = norm_after();
+        if (e != cudaSuccess) return cuda_fail(e, "kda_fwd output norm launch");
         return KDA_OK;
     }
     if (need_ws > 0 && tokens) {
@@ -270,6 +288,56 @@ kda_status_t kda_fwd(const kda_fwd_desc_t* d, const void* q, const void* k, cons
     }
     e = path == Path::kChunk64 ? kda::launch_chunk64(p, s) : kda::launch_recurrent(p, s);
     if (e != cudaSuccess) return cuda_fail(e, "kda_fwd launch");
+    e = norm_after();
+    if (e != cudaSuccess) return cuda_fail(e, "kda_fwd output norm launch");
+    return KDA_OK;
+}
+
+kda_status_t kda_fwd(const kda_fwd_desc_t* d, const void* q, const void* k, const void* v,
+                     const float* log_g, const void* beta, const float* h0,
+                     const int32_t* cu_seqlens, void* o, float* hT, void* workspace,
+                     size_t workspace_bytes, kda_stream_t stream) {
+    return fwd_impl(d, q, k, v, log_g, beta, h0, cu_seqlens, o, hT, workspace, workspace_bytes,
+                    nullptr, stream);
+}
+
+kda_status_t kda_fwd_normed(const kda_fwd_desc_t* d, const void* q, const void* k,
+                            const void* v, const float* log_g, const void* beta,
+                            const float* h0, const int32_t* cu_seqlens,
+                            const kda_out_norm_t* norm, void* y, float* hT, void* workspace,
+                            size_t workspace_bytes, kda_stream_t stream) {
+    if (!norm) {
+        t_last_error[0] = 0;
+        return fail(KDA_ERR_INVALID_ARG, "norm is NULL");
+    }
+    if (d && d->dv > 256) {
+        t_last_error[0] = 0;
+        return fail(KDA_ERR_UNSUPPORTED, "the output norm supports dv <= 256");
+    }
+    return fwd_impl(d, q, k, v, log_g, beta, h0, cu_seqlens, y, hT, workspace, workspace_bytes,
+                    norm, stream);
+}
+
+kda_status_t kda_out_norm_gated(long long vectors, int dv, kda_dtype_t dtype, const void* x,
+                                const void* gate, const float* weight, float eps, void* y,
+                                kda_stream_t stream) {
+    t_last_error[0] = 0;
+    if (vectors < 0 || dv < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes vectors=%lld dv=%d",
+                                           vectors, dv);
+    if (dv > 256) return fail(KDA_ERR_UNSUPPORTED, "the output norm supports dv <= 256");
+    if (dtype != KDA_F32 && dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (!(eps >= 0.f)) return fail(KDA_ERR_INVALID_ARG, "eps must be >= 0");
+    kda_status_t st;
+    const bool any = vectors > 0;
+    if ((st = check_ptr(x, "x", any)) || (st = check_ptr(gate, "gate", any)) ||
+        (st = check_ptr(weight, "weight", any)) || (st = check_ptr(y, "y", any)))
+        return st;
+    if (!any) return KDA_OK;
+    cudaError_t e = kda::launch_out_norm_gated(x, gate, weight, eps, y, vectors, dv,
+                                               dtype == KDA_BF16,
+                                               reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kda_out_norm_gated launch");
     return KDA_OK;
 }
 

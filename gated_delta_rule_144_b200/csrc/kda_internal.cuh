@@ -88,6 +88,11 @@ cudaError_t launch_chunk_map(const int32_t* cu_seqlens, int N, int T, long long 
                              unsigned* err, cudaStream_t stream);
 cudaError_t launch_chunk64_intra(const FwdParams& p, cudaStream_t stream);
 cudaError_t launch_chunk_scan(const FwdParams& p, cudaStream_t stream);
+// y = x / sqrt(mean(x^2) + eps) * w * sigmoid(gate) per vector of dv elements (dv <= 256);
+// y may alias x.
+cudaError_t launch_out_norm_gated(const void* x, const void* gate, const float* w, float eps,
+                                  void* y, long long vectors, int dv, bool bf16,
+                                  cudaStream_t stream);
 bool chunk64_available();
 // Value columns one chunked-kernel CTA owns for N sequences x H heads (64 or 128).
 int chunk64_value_width(int N, int H);

@@ -118,6 +118,44 @@ kda_status_t kda_fwd(const kda_fwd_desc_t* desc, const void* q, const void* k, c
                      size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * Gated per-head RMSNorm of the output (NeMo glm5_next layers, _TorchRMSNormGated: normalise
+ * [batch, sequence, heads, head_dim], then gate with a sigmoid; its base Glm5NextRMSNorm keeps
+ * the variance in fp32 and a weight of head_dim entries; metrale glm5next_layer: every norm is
+ * x * w / rms). Per (token, head):
+ *     y = x / sqrt(mean over head_dim of x^2 + eps) * weight * sigmoid(gate).
+ *   gate   : same shape and dtype as the output it gates, device.
+ *   weight : [dv] float32, device, shared by all heads.
+ *   eps    : >= 0.
+ */
+typedef struct {
+    const void* gate;
+    const float* weight;
+    float eps;
+} kda_out_norm_t;
+
+/*
+ * kda_fwd_normed - kda_fwd followed by the gated RMSNorm above, writing y (shaped like o)
+ * instead of o: the prefill writes o into y, then one bandwidth-bound pass normalises y in
+ * place. The norm sees o rounded to the output dtype, as a separate norm module would. Same
+ * arguments, layouts, workspace and errors as kda_fwd; dv <= 256. NULL norm is
+ * KDA_ERR_INVALID_ARG.
+ */
+kda_status_t kda_fwd_normed(const kda_fwd_desc_t* desc, const void* q, const void* k,
+                            const void* v, const float* log_g, const void* beta,
+                            const float* h0, const int32_t* cu_seqlens,
+                            const kda_out_norm_t* norm, void* y, float* hT, void* workspace,
+                            size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * kda_out_norm_gated - the gated RMSNorm on its own: `vectors` vectors of dv elements (for o of
+ * shape [B, T, H, dv], vectors = B * T * H), x and gate in dtype, y in dtype (y may equal x).
+ * dv <= 256. Host-checkable errors return before any launch.
+ */
+kda_status_t kda_out_norm_gated(long long vectors, int dv, kda_dtype_t dtype, const void* x,
+                                const void* gate, const float* weight, float eps, void* y,
+                                kda_stream_t stream);
+
+/*
  * Path kda_fwd takes for `desc` (has_cu_seqlens: whether cu_seqlens will be non-NULL):
  * KDA_CHUNK_PER_TOKEN or KDA_CHUNK_64, or the negated kda_status_t when the description is
  * rejected. Host-only, no CUDA calls.

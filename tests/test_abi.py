@@ -131,6 +131,26 @@ def test_decode_tokens_rejects_on_host(L):
                                None) == 0
 
 
+def test_out_norm_rejects_on_host(L):
+    P = ctypes.c_void_p
+    d = _desc()
+    nrm = kda.OutNorm(FAKE, FAKE, 1e-6)
+    call = lambda desc, norm: L.kda_fwd_normed(ctypes.byref(desc), P(FAKE), P(FAKE), P(FAKE),
+                                               P(FAKE), P(FAKE), None, None, norm, P(FAKE), None,
+                                               None, 0, None)
+    assert call(d, None) == 1                                     # no norm
+    assert call(_desc(dv=512, dtype=kda.KDA_F32), ctypes.byref(nrm)) == 2   # dv > 256
+    bad = kda.OutNorm(FAKE, FAKE, -1.0)
+    assert call(d, ctypes.byref(bad)) == 1                        # eps < 0
+    bad = kda.OutNorm(None, FAKE, 1e-6)
+    assert call(d, ctypes.byref(bad)) == 1                        # no gate
+    assert L.kda_out_norm_gated(4, 300, 1, P(FAKE), P(FAKE), P(FAKE), 1e-6, P(FAKE), None) == 2
+    assert L.kda_out_norm_gated(4, 128, 1, P(FAKE), None, P(FAKE), 1e-6, P(FAKE), None) == 1
+    assert L.kda_out_norm_gated(4, 128, 1, P(FAKE + 2), P(FAKE), P(FAKE), 1e-6, P(FAKE),
+                                None) == 1
+    assert L.kda_out_norm_gated(0, 128, 1, None, None, None, 1e-6, None, None) == 0
+
+
 def test_workspace_size_is_host_only(L):
     # minimum (fused chunked path): only packed documents need scratch, one int32 each
     d = _desc()
