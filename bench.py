@@ -136,6 +136,7 @@ class ClockSampler:
 KERNEL_SOURCES = {
     "kda_decode_d128": ["kda_decode.cu", "kda_internal.cuh"],
     "kda_decode_tokens_d128": ["kda_decode.cu", "kda_internal.cuh"],
+    "kda_out_norm_gated": ["kda_norm.cu", "kda_internal.cuh"],
     "kda_recurrent": ["kda_recurrent.cu", "kda_internal.cuh"],
     "kda_chunk64": ["kda_chunk64.cu", "kda_sm100.cuh", "kda_internal.cuh", "kda_tma.cuh"],
     "kda_chunk64_intra": ["kda_chunk64.cu", "kda_sm100.cuh", "kda_internal.cuh", "kda_tma.cuh"],
@@ -545,6 +546,15 @@ def run_profile_case(args):
     if args.profile_case == "decode":
         d = synth.decode_inputs("decode-n256", device=dev)
         fn = lambda: kda.decode_step(d["q"], d["k"], d["v"], d["log_g"], d["beta"], d["S"])
+    elif args.profile_case == "decode-rows":
+        d = synth.decode_tokens_inputs("decode-rows-n256-t4", device=dev)
+        fn = lambda: kda.decode_tokens(d["q"], d["k"], d["v"], d["log_g"], d["beta"], d["S"])
+    elif args.profile_case == "norm":
+        p = synth.prefill_inputs("packed-8docs", device=dev)
+        o = torch.randn(p["v"].shape, device=dev).to(p["v"].dtype)
+        gate = torch.randn(o.shape, device=dev).to(o.dtype)
+        nw = torch.rand(128, device=dev) + 0.5
+        fn = lambda: kda.out_norm_gated(o, gate, nw, 1e-6)
     else:
         name = args.workload if args.profile_case == "prefill" else "packed-8docs"
         kw = {} if args.profile_tokens <= 0 else {"T": args.profile_tokens}
@@ -578,7 +588,8 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=4096)
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=["prefill", "decode", "packed"], default=None,
+    ap.add_argument("--profile-case", choices=["prefill", "decode", "decode-rows", "packed", "norm"],
+                    default=None,
                     help="run only warm-up + steps launches of one case (for ncu captures)")
     ap.add_argument("--profile-tokens", type=int, default=0,
                     help="with --profile-case prefill: tokens per sequence (0 = workload's)")
