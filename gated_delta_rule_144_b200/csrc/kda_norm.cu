@@ -1,5 +1,5 @@
-// Gated per-head RMSNorm of the KDA output, as a standalone pass (the split chunked prefill fuses
-// the same arithmetic into its output store; this kernel serves every other path).
+// Gated per-head RMSNorm of the KDA output, as a vectorised pass over o after the recurrence (a
+// version folded into the state pass's output store was slower: it lengthened the per-chunk chain).
 //
 // Per (token, head): y = x / sqrt(mean over head_dim of x^2 + eps) * w * sigmoid(gate), with the
 // variance accumulated in fp32 (NeMo glm5_next layers, _TorchRMSNormGated: normalise, then gate
