@@ -83,7 +83,7 @@ struct Layout {
     static constexpr uint32_t OFF_BETA = OFF_MISC;         // f32 [64]
     static constexpr uint32_t OFF_DECAY = OFF_MISC + 256;  // f32 [128]
     static constexpr uint32_t OFF_LOUP = OFF_MISC + 768;   // f32 [4 blocks][2 halves][128]
-    static constexpr uint32_t OFF_BAR = OFF_MISC + 4864;   // 6 mbarriers
+    static constexpr uint32_t OFF_BAR = OFF_MISC + 4864;   // mbarriers
     static constexpr uint32_t OFF_TMEM = OFF_BAR + 64;     // TMEM base address
     static constexpr uint32_t kSmemBytes = OFF_TMEM + 16 + 1024;  // + alignment slack
     static_assert(OFF_ZA + 16384 == OFF_C + 40960, "solve buffers fill the R/C region exactly");
@@ -111,12 +111,6 @@ __host__ __device__ constexpr int cross_off(int a) { return a == 1 ? 0 : (a == 2
 
 struct ChunkArgs {
     const int32_t* order;   // nullable: document taken by the k-th (document, head) group
-    // intra mode: chunk records (g, head) with g = sequence * ncT + chunk, or, for packed
-    // documents, g = floor(t0 / 64) + document + chunk and map[g] = document (-1: unused)
-    const int32_t* map;
-    float* decay_out;       // [G * H][128]: e^{Gamma_end} of every record
-    long long G;            // chunk records per head
-    int ncT;
     const __nv_bfloat16* beta;
     const float* h0;
     const int32_t* cu;
@@ -150,29 +144,20 @@ __device__ __forceinline__ void st_bf16x8(uint8_t* p, const float* v) {
 }
 __device__ __forceinline__ uint32_t f2tf(float x) { return __float_as_uint(x); }
 
-// Output maps of the intra mode (workspace records, row-major bf16, 128-byte swizzle).
-struct IntraMaps {
-    CUtensorMap wq, ke, ut, ot;
-};
-
 // One unit of a CTA's walk: a chunk of 64 rows of one head.
 struct Unit {
     int h;
     int L;            // valid rows
     long long row0;   // first token row
-    long long rec;    // workspace record (intra mode)
 };
 
-// kIntra = false (fused): one CTA per (sequence or document, head, value slice) walks its chunks in
-// order and carries the state in TMEM. kIntra = true: a persistent CTA takes independent
-// (chunk, head) records, computes the chunk's WY factors and stores them for the state pass.
-template <int DV, bool kIntra>
+// One CTA per (sequence or document, head, value slice) walks its chunks in order and carries the
+// state in TMEM.
+template <int DV>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
-               const __grid_constant__ IntraMaps omaps, const ChunkArgs args) {
-    static_assert(!kIntra || DV == 128, "the intra mode computes whole heads");
-    constexpr uint32_t kTmemCols = kIntra ? 256 : 512;
+               const ChunkArgs args) {
     using Lay = Layout<DV>;
     constexpr int kDV = Lay::kDV, kSplit = Lay::kSplit, kPanels = Lay::kPanels;
     constexpr uint32_t OFF_Q = Lay::OFF_Q, OFF_K = Lay::OFF_K, OFF_G = Lay::OFF_G;
@@ -190,15 +175,14 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int qd = warp & 3, hf = warp >> 2;          // TMEM lane quarter, column half
-    const int split = kIntra ? 0 : blockIdx.x % kSplit;
-    const int unit = kIntra ? 0 : blockIdx.x / kSplit;
-    int h = kIntra ? 0 : unit % args.H;
-    const int n = kIntra ? 0 : (args.order ? args.order[unit / args.H] : unit / args.H);
+    const int split = blockIdx.x % kSplit;
+    const int unit = blockIdx.x / kSplit;
+    const int h = unit % args.H;
+    const int n = args.order ? args.order[unit / args.H] : unit / args.H;
     const int dv0 = split * kDV;
 
     long long t0 = 0, t1 = 0;
-    if constexpr (kIntra) {
-    } else if (args.cu) {
+    if (args.cu) {
         t0 = args.cu[n];
         t1 = args.cu[n + 1];
         const bool bad_ends = (n == 0 && t0 != 0) || (n == args.N - 1 && t1 != args.T);
@@ -212,43 +196,15 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     const int nchunks = (int)((t1 - t0 + kC - 1) / kC);
 
-    // the walk: chunks of this chain in order (fused), or this CTA's share of the records
-    long long cursor = kIntra ? (long long)blockIdx.x : 0;
+    // the walk: chunks of this chain in order
+    long long cursor = 0;
     auto next_unit = [&](Unit& u) -> bool {
-        if constexpr (kIntra) {
-            const long long total = args.G * args.H;
-            while (cursor < total) {
-                const long long idx = cursor;
-                cursor += gridDim.x;
-                const long long g = idx / args.H;
-                u.h = (int)(idx % args.H);
-                u.rec = idx;
-                if (args.cu) {
-                    const int d = args.map[g];
-                    if (d < 0 || d >= args.N) continue;
-                    const long long a = args.cu[d], b = args.cu[d + 1];
-                    if (b <= a || a < 0 || b > args.T) continue;   // reported by the map kernel
-                    const long long cc = g - d - a / kC;
-                    if (cc < 0 || a + kC * cc >= b) continue;
-                    u.row0 = a + kC * cc;
-                    u.L = (int)min((long long)kC, b - u.row0);
-                } else {
-                    const long long s = g / args.ncT, cc = g % args.ncT;
-                    u.row0 = s * args.T + kC * cc;
-                    u.L = (int)min((long long)kC, (long long)args.T - kC * cc);
-                }
-                return true;
-            }
-            return false;
-        } else {
-            if (cursor >= nchunks) return false;
-            u.h = h;
-            u.row0 = t0 + kC * cursor;
-            u.L = (int)min((long long)kC, t1 - u.row0);
-            u.rec = 0;
-            ++cursor;
-            return true;
-        }
+        if (cursor >= nchunks) return false;
+        u.h = h;
+        u.row0 = t0 + kC * cursor;
+        u.L = (int)min((long long)kC, t1 - u.row0);
+        ++cursor;
+        return true;
     };
     Unit cur, nxt;
     bool has_cur = next_unit(cur);
@@ -259,7 +215,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     float* loup_s = reinterpret_cast<float*>(sm + OFF_LOUP);
     uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
     const uint32_t bar_in = sb + OFF_BAR, bar_v = bar_in + 8, bar_mma = bar_in + 16;
-    const uint32_t bar_b4 = bar_in + 24, bar_never = bar_in + 32, bar_wy2 = bar_in + 40;
+    const uint32_t bar_b4 = bar_in + 24, bar_never = bar_in + 32;
 
     if (tid == 0) {
         mbar_init(bar_in, 1);
@@ -267,7 +223,6 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mbar_init(bar_mma, 1);
         mbar_init(bar_b4, 1);
         mbar_init(bar_never, 1);
-        mbar_init(bar_wy2, 1);
         fence_mbar_init();
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
@@ -287,7 +242,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
     // initial state: TMEM lane c = 32 qd + lane holds S[c][dv0 + kHalfCols hf .. + kHalfCols)
 #pragma unroll
-    for (int p = 0; p < (kIntra ? 0 : kHalfCols / 32); ++p) {
+    for (int p = 0; p < kHalfCols / 32; ++p) {
         float v[32];
         const int c = 32 * qd + lane;
         const int col = kHalfCols * hf + 32 * p;
@@ -329,8 +284,6 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
     // outstanding asynchronous work, drained before exit if a wait expires
     bool in_pending = false, v_pending = false, mma_pending = false, b4_pending = false;
-    bool wy2_pending = false;   // intra mode: the transposed WY product (V^T [T; T']^T)
-    int wy2_count = 0;
     int in_chunk = 0, v_chunk = 0, b4_chunk = 0;
     uint32_t mma_phase = 0;
     bool aborted = false;
@@ -340,10 +293,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         return __syncthreads_or(!ok) == 0;
     };
 
-    bool stores_pending = false;   // intra mode: bulk stores still reading shared memory
-    // Thread that issues TMA copies: in the intra mode lane 0 of the last warp (the one with the
-    // least elementwise work), so that copy issue never delays thread 0's MMAs.
-    const int copier = kIntra ? kThreads - 32 : 0;
+    const int copier = 0;   // thread that issues the TMA copies
     if (has_cur) {
         if (tid == copier) {
             issue_in(cur);
@@ -379,7 +329,6 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     for (int c = 0; has_cur && !aborted; ++c) {
         const long long row0 = cur.row0;
         const int L = cur.L;
-        h = cur.h;
 
         // ---------------------------------------------------------------- inputs of chunk c
         if (!wait_all(bar_in, c & 1)) { aborted = true; break; }
@@ -453,23 +402,13 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     if (bb == pb) own[i] = hh == 0 ? up[i] : lo[i];
                 }
             }
-            if (pb == 0 && hh == 0) {
+            if (pb == 0 && hh == 0)
                 *reinterpret_cast<float4*>(decay_s + ch0) = make_float4(dec[0], dec[1], dec[2], dec[3]);
-                if constexpr (kIntra)
-                    *reinterpret_cast<float4*>(args.decay_out + cur.rec * kD + ch0) =
-                        make_float4(dec[0], dec[1], dec[2], dec[3]);
-            }
         }
 
         if (b4_pending) {   // the previous state update reads U (R region) and K_end until here
             if (!wait_all(bar_b4, b4_chunk & 1)) { aborted = true; break; }
             b4_pending = false;
-        }
-        if (kIntra && stores_pending) {   // the previous record's stores read R, [W; Q~] and K_end
-            if (tid == kThreads - 32 || tid == kThreads - 64 || tid == kThreads - 96)
-                bulk_wait_read_all();
-            __syncthreads();
-            stores_pending = false;
         }
 
         // ---------------------------------------------------------------- R and C operands
@@ -809,39 +748,21 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (warp == 0) {
             if (lane == 0) {
                 tc_fence_after();
-                if constexpr (kIntra) {
-                    // [T; T'] K+ (W, A_qk W) and, transposed for the state pass, V^T [T; T']^T:
-                    // lane j (value column) gets U~^T (columns 128-191) and O~^T (192-255)
-                    const uint32_t id = idesc_bf16(128, 128, 0, 1);
-                    const uint32_t idt = idesc_bf16(128, 128, 1, 0);
+                const uint32_t id = idesc_bf16(128, 128 + kDV, 0, 1);
 #pragma unroll
-                    for (int s = 0; s < kC / 16; ++s)
-                        umma_f16(tbase + TM_A, desc_at(dK, sb + OFF_TT + 32 * s),
-                                 desc_at(dM8, sb + OFF_KPV + 2048 * s), id, s > 0);
-                    umma_commit(bar_mma);   // W and A_qk W: read out while the next runs
-#pragma unroll
-                    for (int s = 0; s < kC / 16; ++s)
-                        umma_f16(tbase + TM_A + 128, desc_at(dM8, sb + OFF_KPV + 16384 + 2048 * s),
-                                 desc_at(dK, sb + OFF_TT + 32 * s), idt, s > 0);
-                    umma_commit(bar_wy2);
-                } else {
-                    const uint32_t id = idesc_bf16(128, 128 + kDV, 0, 1);
-#pragma unroll
-                    for (int s = 0; s < kC / 16; ++s)
-                        umma_f16(tbase + TM_A, desc_at(dK, sb + OFF_TT + 32 * s),
-                                 desc_at(dM8, sb + OFF_KPV + 2048 * s), id, s > 0);
-                    umma_commit(bar_mma);
-                }
+                for (int s = 0; s < kC / 16; ++s)
+                    umma_f16(tbase + TM_A, desc_at(dK, sb + OFF_TT + 32 * s),
+                             desc_at(dM8, sb + OFF_KPV + 2048 * s), id, s > 0);
+                umma_commit(bar_mma);
             }
             __syncwarp();
         }
         mma_pending = true;
-        wy2_pending = kIntra;
         if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
         ++mma_phase;
         mma_pending = false;
         tc_fence_after();
-        if (!kIntra && has_nxt) {   // the V panel is free again
+        if (has_nxt) {   // the V panel is free again
             if (tid == copier) issue_v(nxt);
             v_pending = true;
             v_chunk = c + 1;
@@ -874,50 +795,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
             }
         }
-        if constexpr (kIntra) {
-            if (!wait_all(bar_wy2, wy2_count & 1)) { aborted = true; break; }
-            ++wy2_count;
-            wy2_pending = false;
-            tc_fence_after();
-            if (has_nxt) {   // the V panel is free again
-                if (tid == copier) issue_v(nxt);
-                v_pending = true;
-                v_chunk = c + 1;
-            }
-            // U~^T (TMEM columns 128-191) and O~^T (192-255), lane j = value column, into bf16
-            // staging tiles [128 j][64 tokens] in the R region (128-byte swizzle), then one set
-            // of bulk stores
-            const int jrow = 32 * qd + lane;
-            const uint32_t stage = hf == 0 ? OFF_R : OFF_R + 16384;
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                float v[32];
-                tmem_ld32(tbase + lane_q + TM_A + 128 + 64 * hf + 32 * part, v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    st_bf16x8(sm + stage + sw128_off(128, jrow, 32 * part + 8 * m), v + 8 * m);
-            }
-            fence_proxy_async();
-            tc_fence_before();
-            __syncthreads();
-            // three issuing threads (lane 0 of warps 5, 6, 7), two stores and one bulk group each
-            const int rw = (int)(cur.rec * 128), rk = (int)(cur.rec * 64);
-            if (tid == kThreads - 32) {
-                tma_store_2d(&omaps.wq, sb + OFF_WQ, 0, rw);
-                tma_store_2d(&omaps.wq, sb + OFF_WQ + 16384, 64, rw);
-                bulk_commit();
-            } else if (tid == kThreads - 64) {
-                tma_store_2d(&omaps.ke, sb + OFF_KE, 0, rk);
-                tma_store_2d(&omaps.ke, sb + OFF_KE + 8192, 64, rk);
-                bulk_commit();
-            } else if (tid == kThreads - 96) {
-                tma_store_2d(&omaps.ut, sb + OFF_R, 0, rw);
-                tma_store_2d(&omaps.ot, sb + OFF_R + 16384, 0, rw);
-                bulk_commit();
-            }
-            stores_pending = true;
-        } else {
+        {
     #pragma unroll
             for (int p = 0; p < kHalfCols / 32; ++p) {
                 // state: bf16 operand for [W; Q~] S, then decay the fp32 TMEM copy
@@ -1023,7 +901,6 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (in_pending) mbar_wait(bar_in, in_chunk & 1, drain);
         if (v_pending) mbar_wait(bar_v, v_chunk & 1, drain);
         if (mma_pending) mbar_wait(bar_mma, mma_phase & 1, drain);
-        if (wy2_pending) mbar_wait(bar_wy2, wy2_count & 1, drain);
         if (b4_pending) mbar_wait(bar_b4, b4_chunk & 1, drain);
         __syncthreads();
     } else {
@@ -1032,7 +909,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_wait(bar_b4, b4_chunk & 1, 1ll << 31);
         }
         tc_fence_after();
-        if (!kIntra && args.hT) {
+        if (args.hT) {
 #pragma unroll
             for (int p = 0; p < kHalfCols / 32; ++p) {
                 float v[32];
@@ -1048,8 +925,6 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
         }
     }
-    if (kIntra && (tid == kThreads - 32 || tid == kThreads - 64 || tid == kThreads - 96))
-        bulk_wait_all();   // stores complete before the smem goes away
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, kTmemCols);
@@ -1090,21 +965,28 @@ cudaError_t make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t make_map_3d_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt,
-                             int elem_bytes, unsigned long long rows, int H, int cols,
-                             int box_rows) {
+cudaError_t make_map_3d_box(CUtensorMap* m, const void* base, CUtensorMapDataType dt,
+                            int elem_bytes, unsigned long long rows, int H, int cols, int box_cols,
+                            int box_rows, CUtensorMapSwizzle sw) {
     cudaError_t e = tma_encoder_ready();
     if (e != cudaSuccess) return e;
     const cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)H, (cuuint64_t)rows};
     const cuuint64_t strides[2] = {(cuuint64_t)cols * elem_bytes,
                                    (cuuint64_t)H * cols * elem_bytes};
-    const cuuint32_t box[3] = {(cuuint32_t)cols, 1, (cuuint32_t)box_rows};
+    const cuuint32_t box[3] = {(cuuint32_t)box_cols, 1, (cuuint32_t)box_rows};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r = g_encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
-                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_map_3d_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt,
+                             int elem_bytes, unsigned long long rows, int H, int cols,
+                             int box_rows) {
+    return make_map_3d_box(m, base, dt, elem_bytes, rows, H, cols, cols, box_rows,
+                           CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 namespace {
@@ -1145,12 +1027,12 @@ long long wait_budget() {
     return budget;
 }
 
-template <int DV, bool kIntra>
+template <int DV>
 cudaError_t set_smem_attr() {
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(chunk64_kernel<DV, kIntra>,
+        attr_err = cudaFuncSetAttribute(chunk64_kernel<DV>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)Layout<DV>::kSmemBytes);
     });
@@ -1161,7 +1043,7 @@ template <int DV>
 cudaError_t launch_width(const FwdParams& p, cudaStream_t stream, const CUtensorMap& mq,
                          const CUtensorMap& mk, const CUtensorMap& mg, int units) {
     using Lay = Layout<DV>;
-    cudaError_t attr_err = set_smem_attr<DV, false>();
+    cudaError_t attr_err = set_smem_attr<DV>();
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap mv;
     cudaError_t e = make_map(&mv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B * p.T, p.H, 64,
@@ -1182,14 +1064,7 @@ cudaError_t launch_width(const FwdParams& p, cudaStream_t stream, const CUtensor
     a.err = p.err;
     const long long grid = (long long)units * Lay::kSplit;
     if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
-    a.map = nullptr;
-    a.decay_out = nullptr;
-    a.G = 0;
-    a.ncT = 0;
-    IntraMaps none;
-    memset(&none, 0, sizeof(none));
-    chunk64_kernel<DV, false><<<(unsigned)grid, kThreads, Lay::kSmemBytes, stream>>>(
-        mq, mk, mg, mv, none, a);
+    chunk64_kernel<DV><<<(unsigned)grid, kThreads, Lay::kSmemBytes, stream>>>(mq, mk, mg, mv, a);
     return cudaGetLastError();
 }
 
@@ -1239,56 +1114,6 @@ cudaError_t launch_chunk64(const FwdParams& p, cudaStream_t stream) {
 int chunk64_value_width(int N, int H) {
     const long long units = (long long)N * H;
     return units * 2 > sm_count() ? 128 : 64;
-}
-
-// Intra-chunk kernel of the split path: a persistent grid (one CTA per SM) takes the (chunk
-// record, head) items in turn and stores each chunk's WY factors into the workspace.
-cudaError_t launch_chunk64_intra(const FwdParams& p, cudaStream_t stream) {
-    const SplitWorkspace& ws = *p.split;
-    cudaError_t e = get_encoder();
-    if (e != cudaSuccess) return e;
-    const int rows = p.B * p.T;
-    const long long items = ws.G * p.H;
-    if (items == 0 || rows <= 0) return cudaSuccess;
-    if (ws.G * p.H * 128 > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    CUtensorMap mq, mk, mg, mv;
-    if ((e = make_map(&mq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, kD,
-                      CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
-        (e = make_map(&mk, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, kD,
-                      CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
-        (e = make_map(&mg, p.log_g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, p.H, kD,
-                      CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
-        (e = make_map(&mv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, p.H, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
-        return e;
-    const unsigned long long R = (unsigned long long)items;
-    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
-    IntraMaps om;
-    if ((e = make_map_2d(&om.wq, ws.wq, BF, 2, R * 128, kD, 64, 128, SW)) != cudaSuccess ||
-        (e = make_map_2d(&om.ke, ws.ke, BF, 2, R * 64, kD, 64, 64, SW)) != cudaSuccess ||
-        (e = make_map_2d(&om.ut, ws.ut, BF, 2, R * 128, kC, 64, 128, SW)) != cudaSuccess ||
-        (e = make_map_2d(&om.ot, ws.ot, BF, 2, R * 128, kC, 64, 128, SW)) != cudaSuccess)
-        return e;
-    if ((e = set_smem_attr<128, true>()) != cudaSuccess) return e;
-    ChunkArgs a;
-    memset(&a, 0, sizeof(a));
-    a.beta = static_cast<const __nv_bfloat16*>(p.beta);
-    a.cu = p.cu_seqlens;
-    a.T = p.T;
-    a.H = p.H;
-    a.N = p.N;
-    a.budget = wait_budget();
-    a.debug_stall = debug_stall();
-    a.err = p.err;
-    a.map = ws.map;
-    a.decay_out = ws.decay;
-    a.G = ws.G;
-    a.ncT = ws.ncT;
-    const long long grid = items < sm_count() ? items : sm_count();
-    chunk64_kernel<128, true><<<(unsigned)grid, kThreads, Layout<128>::kSmemBytes, stream>>>(
-        mq, mk, mg, mv, om, a);
-    return cudaGetLastError();
 }
 
 }  // namespace kda

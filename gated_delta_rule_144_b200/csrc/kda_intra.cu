@@ -1,0 +1,931 @@
+// Intra-chunk kernel of the split chunked prefill: the WY factors of every (chunk, head) record,
+// independent of the state, so all records of all sequences run at once.
+//
+// Per chunk of 64 rows r of one head (WY / UT form of the gated delta rule; GLM-5.3-Flash model
+// card, Kimi Delta Attention snippet), with Gamma the within-chunk cumulative log decay per key
+// channel:
+//   A_kk[r,i] = sum_c k_rc k_ic e^{Gamma_rc - Gamma_ic}  (i < r)    A_qk: same with q_r, i <= r
+//   T  = (I + diag(beta) A_kk)^-1 diag(beta)                          (UT transform, fp32)
+//   W  = T (k e^{Gamma}),  U~ = T v,  Q~ = q e^{Gamma} - A_qk W,  O~ = A_qk U~,
+//   K_end = k e^{Gamma_end - Gamma},  decay = e^{Gamma_end}
+// and the state pass later applies U = U~ - W S, o = O~ + Q~ S, S <- diag(decay) S + K_end^T U.
+// A_kk and A_qk come from one tensor-core product R C^T of separable factors anchored at the
+// middle of each 16-row block (rows of R at their own block's middle, diagonal-block columns at
+// theirs, the columns a later block needs at that later block's middle), so no factor leaves the
+// float32 range while the summed decay of 8 consecutive rows stays above about -69 nats.
+//
+// Occupancy: two CTAs share each SM, so that one CTA's tensor-core waits, barriers and memory
+// latency are covered by the other's CUDA-core work. To fit two CTAs (about 110 KB of shared memory
+// and 256 TMEM columns each), q, k and log g go straight from global memory into registers (the
+// next record's tiles are prefetched into L2 by TMA while this one runs), K_end is written to the
+// workspace from registers, and Q+ = q e^{Gamma} is parked in the workspace slot of Q~ and read
+// back when Q~ = Q+ - A_qk W is formed. Only V (an MMA operand) arrives by TMA into shared memory.
+//
+// Per record (256 threads; thread 0 issues the MMAs, lane 0 of warp 7 the copies):
+//   loads -> decay products -> R, C, K+ (shared), Q+, K_end (global) -> MMA R C^T ->
+//   A_kk, A_qk -> UT solve -> MMA T' = A_qk T -> MMA [T; T'] K+ and V^T [T; T']^T ->
+//   [W; Q~], U~^T, O~^T staged in shared memory -> TMA stores.
+// Every mbarrier wait is bounded; on expiry the CTA records KDA_ERR_TIMEOUT, drains its own
+// copies and MMAs, frees TMEM and exits.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "kda_internal.cuh"
+#include "kda_sm100.cuh"
+#include "kda_tma.cuh"
+
+namespace kda {
+namespace {
+
+using namespace sm100;
+
+constexpr int kC = 64;    // tokens per chunk
+constexpr int kD = 128;   // dk = dv
+constexpr int kThreads = 256;
+
+// shared memory (bytes from a 1024-aligned base)
+constexpr uint32_t OFF_KP = 0;               // K+ [64 tokens][128] bf16, MN-major B (2 x 8 KB)
+constexpr uint32_t OFF_V = 16384;            // V  [64 tokens][128] bf16, MN-major (TMA, SW128)
+constexpr uint32_t OFF_R = 32768;            // R  [128][128] bf16, K-major A (2 x 16 KB)
+constexpr uint32_t OFF_C = OFF_R + 32768;    // C  [160][128] bf16, K-major B (2 x 20 KB)
+//   after R C^T the R/C region holds the solve buffers:
+constexpr uint32_t OFF_LB = OFF_R;           // L = diag(beta) A_kk, f32 [64][kLdl]
+constexpr uint32_t OFF_MB = OFF_R + 17408;   // (I + L)^-1, f32 [64][kLdm]
+constexpr uint32_t OFF_YS = OFF_R + 35840;   // four 16x17 f32 scratch blocks of the solve
+constexpr uint32_t OFF_TT = OFF_R + 40960;   // [T; T'] [128][64] bf16 (K-major A; rows 0-63
+                                             //   also the MN-major B of T')
+constexpr uint32_t OFF_ZA = OFF_R + 57344;   // [0; A_qk] [128][64] bf16 (K-major A)
+//   and, once the WY products have read it, the staging tiles of the stores:
+constexpr uint32_t OFF_SWQ = OFF_R;          // [W; Q~] [128][128] (2 panels x 16 KB)
+constexpr uint32_t OFF_SUT = OFF_R + 32768;  // U~^T [128 value columns][64 tokens]
+constexpr uint32_t OFF_SOT = OFF_R + 49152;  // O~^T [128][64]
+constexpr uint32_t OFF_MISC = OFF_C + 40960;
+constexpr uint32_t OFF_BETA = OFF_MISC;           // f32 [64]
+constexpr uint32_t OFF_LOUP = OFF_MISC + 256;     // f32 [4 blocks][2 halves][128]
+constexpr uint32_t OFF_BAR = OFF_LOUP + 4096;     // mbarriers
+constexpr uint32_t OFF_TMEM = OFF_BAR + 64;       // TMEM base address
+constexpr uint32_t kSmemBytes = OFF_TMEM + 16 + 1024;   // + alignment slack
+static_assert(OFF_ZA + 16384 == OFF_C + 40960, "solve buffers fill the R/C region exactly");
+static_assert(OFF_YS + 4 * 16 * 17 * 4 <= OFF_TT, "solve scratch overlaps [T; T']");
+static_assert(OFF_SWQ + 32768 <= OFF_TT, "[W; Q~] staging must not touch [T; T'] (read by the "
+                                         "second WY product while [W; Q~] is staged)");
+static_assert(OFF_SOT + 16384 <= OFF_MISC, "staging overflows the R/C region");
+static_assert(2 * (kSmemBytes + 1024) <= 233472, "two CTAs per SM");
+// TMEM columns (fp32, 128 lanes; row m of an M = 128 product sits in lane m)
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t TM_A = 0;     // R C^T [128 x 160]; later [T; T'] K+ (0-127) and
+                                 //   V^T [T; T']^T (128-255: U~^T, then O~^T)
+constexpr uint32_t TM_TP = 160;  // [0; A_qk] T (lanes 64-127: T')
+constexpr int kLdl = 68;         // row stride (floats) of L: conflict-free A-fragment loads
+constexpr int kLdm = 72;         // row stride (floats) of M: conflict-free B-fragment loads
+constexpr uint32_t kTxV = 16384;
+
+// row offset, inside C[64:], of the columns row block a needs from earlier blocks
+__host__ __device__ constexpr int cross_off(int a) { return a == 1 ? 0 : (a == 2 ? 16 : 48); }
+
+struct IntraArgs {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* k;
+    const float* g;
+    const __nv_bfloat16* beta;
+    const int32_t* cu;       // nullable: packed documents
+    const int32_t* map;      // packed: document of chunk record g (-1: unused)
+    __nv_bfloat16* wq;       // [R * 128][128]: W, Q~ (Q+ parked there in between)
+    __nv_bfloat16* ke;       // [R * 64][128]: K_end
+    float* decay;            // [R][128]
+    long long G;             // chunk records per head
+    int ncT, T, H, N;
+    long long budget;
+    int debug_stall;         // failure-injection hook: wait on a barrier nothing ever signals
+    unsigned* err;
+};
+
+// q, k, log g, v: [rows, H, 128] maps of one head's 64-row tile (q, k, g for L2 prefetch, v for
+// the shared-memory copy, 64-column boxes); wq, ut, ot: record stores (128-byte swizzle).
+struct IntraMaps {
+    CUtensorMap q, k, g, v, wq, ut, ot;
+};
+
+struct Unit {
+    int h;
+    int L;            // valid rows
+    long long row0;   // first token row
+    long long rec;    // workspace record
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(x, y);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+__device__ __forceinline__ void st_bf16x4(uint8_t* p, float a, float b, float c, float d) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16(a, b), pack_bf16(c, d));
+}
+__device__ __forceinline__ void st_bf16x8(uint8_t* p, const float* v) {
+    *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                              pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+}
+__device__ __forceinline__ uint32_t f2tf(float x) { return __float_as_uint(x); }
+
+__device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+// Orders this thread's generic-proxy writes (shared and global) before later async-proxy
+// accesses (TMA stores) issued after a barrier.
+__device__ __forceinline__ void fence_proxy_async_all() {
+    asm volatile("fence.proxy.async;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int qd = warp & 3, hf = warp >> 2;          // TMEM lane quarter, column half
+    const int H = args.H;
+
+    // this CTA's records: blockIdx.x, + gridDim.x, ... (record = g * H + head)
+    long long cursor = blockIdx.x;
+    auto next_unit = [&](Unit& u) -> bool {
+        const long long total = args.G * H;
+        while (cursor < total) {
+            const long long idx = cursor;
+            cursor += gridDim.x;
+            const long long g = idx / H;
+            u.h = (int)(idx % H);
+            u.rec = idx;
+            if (args.cu) {
+                const int d = args.map[g];
+                if (d < 0 || d >= args.N) continue;
+                const long long a = args.cu[d], b = args.cu[d + 1];
+                if (b <= a || a < 0 || b > args.T) continue;   // reported by the map kernel
+                const long long cc = g - d - a / kC;
+                if (cc < 0 || a + kC * cc >= b) continue;
+                u.row0 = a + kC * cc;
+                u.L = (int)min((long long)kC, b - u.row0);
+            } else {
+                const long long s = g / args.ncT, cc = g % args.ncT;
+                u.row0 = s * args.T + kC * cc;
+                u.L = (int)min((long long)kC, (long long)args.T - kC * cc);
+            }
+            return true;
+        }
+        return false;
+    };
+    Unit cur;
+    bool has_cur = next_unit(cur);
+
+    float* beta_s = reinterpret_cast<float*>(sm + OFF_BETA);
+    float* loup_s = reinterpret_cast<float*>(sm + OFF_LOUP);
+    uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
+    const uint32_t bar_v = sb + OFF_BAR, bar_mma = bar_v + 8, bar_wy2 = bar_v + 16;
+    const uint32_t bar_never = bar_v + 24;
+    // lane 0 of the last warp issues copies and the [W; Q~] stores; warps 5 and 6 the others
+    const int copier = kThreads - 32;
+
+    if (tid == 0) {
+        mbar_init(bar_v, 1);
+        mbar_init(bar_mma, 1);
+        mbar_init(bar_wy2, 1);
+        mbar_init(bar_never, 1);
+        fence_mbar_init();
+    }
+    if (tid == copier) {
+        prefetch_tmap(&maps.q);
+        prefetch_tmap(&maps.k);
+        prefetch_tmap(&maps.g);
+        prefetch_tmap(&maps.v);
+        prefetch_tmap(&maps.wq);
+        prefetch_tmap(&maps.ut);
+        prefetch_tmap(&maps.ot);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_s), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_s;
+    const uint32_t lane_q = (uint32_t)(32 * qd) << 16;   // this warp's TMEM lane quarter
+
+    auto issue_v = [&](const Unit& u) {
+        mbar_arrive_expect_tx(bar_v, kTxV);
+        tma_load_3d(sb + OFF_V, &maps.v, bar_v, 0, u.h, (int)u.row0);
+        tma_load_3d(sb + OFF_V + 8192, &maps.v, bar_v, 64, u.h, (int)u.row0);
+    };
+    auto prefetch_inputs = [&](const Unit& u) {
+        const int row0 = (int)u.row0;
+        tma_prefetch_3d(&maps.q, 0, u.h, row0);
+        tma_prefetch_3d(&maps.k, 0, u.h, row0);
+        tma_prefetch_3d(&maps.g, 0, u.h, row0);
+        tma_prefetch_3d(&maps.v, 0, u.h, row0);
+        tma_prefetch_3d(&maps.v, 64, u.h, row0);
+    };
+
+    // constant parts of the shared-memory descriptors (the start address is added per MMA)
+    const uint64_t dK = sw128_desc(0, 16, 1024);     // K-major, 128B swizzle
+    const uint64_t dM8 = sw128_desc(0, 8192, 1024);  // MN-major, 128B swizzle, 64-row panels
+
+    bool v_pending = false, mma_pending = false, wy2_pending = false, stores_pending = false;
+    int v_count = 0, wy2_count = 0;
+    uint32_t mma_phase = 0;
+    bool aborted = false;
+    // One thread polls; the rest of the CTA waits at the barrier that publishes the outcome.
+    auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
+        const bool ok = tid != 0 || mbar_wait_sleep(bar, parity, args.budget);
+        return __syncthreads_or(!ok) == 0;
+    };
+
+    if (has_cur && tid == copier) prefetch_inputs(cur);
+    // Failure injection (KDA_DEBUG_STALL_WAIT): a wait on a barrier that nothing signals must
+    // expire, report KDA_ERR_TIMEOUT and wind down cleanly.
+    if (args.debug_stall && !wait_all(bar_never, 0)) aborted = true;
+
+    // elementwise thread mapping: 16-row block pb, half hh (rows 0-7 / 8-15), channels ch0..+3
+    const int pb = warp >> 1, hh = warp & 1;
+    const int ch0 = 4 * lane;
+    const int rbase = 16 * pb + 8 * hh;
+    const int rb8 = 2 * pb + hh;
+    const uint32_t lh4 = (uint32_t)(((lane & 15) >> 1) << 4);   // 16-byte chunk within a row
+    const uint32_t lo8 = (uint32_t)((lane & 1) * 8);
+    // byte offset of (row 8*rb + j, channels ch0..ch0+3) in a 128-column tile of R rows
+    auto toff = [&](int R, int rb, int j) -> uint32_t {
+        return (uint32_t)((lane >> 4) * R * 128 + rb * 1024 + j * 128) + (lh4 ^ (uint32_t)(j << 4)) +
+               lo8;
+    };
+    const size_t row_stride = (size_t)H * kD;   // elements between consecutive tokens
+
+    for (int c = 0; has_cur && !aborted; ++c) {
+        const long long row0 = cur.row0;
+        const int L = cur.L;
+        const int h = cur.h;
+        const long long rec = cur.rec;
+
+        // V of this record (its panel is free: the previous record's products have completed);
+        // the next record's inputs go to L2 while this one runs
+        if (tid == copier) {
+            issue_v(cur);
+            const long long saved = cursor;   // look one record ahead without consuming it
+            Unit ahead;
+            if (next_unit(ahead)) prefetch_inputs(ahead);
+            cursor = saved;
+        }
+        v_pending = true;
+        if (tid < kC)
+            beta_s[tid] = tid < L ? __bfloat162float(args.beta[(row0 + tid) * H + h]) : 0.f;
+
+        // ---------------------------------------------------------------- loads of this record
+        // rows >= L (past the end of the chunk's document) read as log g = 0, k = q = 0
+        const size_t in_base = ((size_t)row0 * H + h) * kD + ch0;
+        float4 gv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            gv[j] = rbase + j < L ? __ldg(reinterpret_cast<const float4*>(
+                                        args.g + in_base + (size_t)(rbase + j) * row_stride))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+
+        // ---------------------------------------------------------------- decay products
+        // With a_t = e^{log g_t} over this thread's 8 rows: the lower half (hh = 0) keeps the
+        // suffix products y_j = prod_{t > j} a_t, the upper half the prefix products
+        // y_j = prod_{t <= j} a_t; tot = prod over all 8 rows. The other product of each row is
+        // tot / y_j, formed below from the reciprocal that the operands need anyway.
+        float y[8][4], tot[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float run = 1.f;
+            if (hh == 0) {
+#pragma unroll
+                for (int j = 7; j >= 0; --j) {
+                    y[j][i] = run;
+                    const float gl = i == 0 ? gv[j].x : i == 1 ? gv[j].y : i == 2 ? gv[j].z : gv[j].w;
+                    run *= rbase + j < L ? __expf(gl) : 1.f;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float gl = i == 0 ? gv[j].x : i == 1 ? gv[j].y : i == 2 ? gv[j].z : gv[j].w;
+                    run *= rbase + j < L ? __expf(gl) : 1.f;
+                    y[j][i] = run;
+                }
+            }
+            tot[i] = run;
+        }
+        *reinterpret_cast<float4*>(loup_s + (pb * 2 + hh) * kD + ch0) =
+            make_float4(tot[0], tot[1], tot[2], tot[3]);
+        if (stores_pending) {   // the previous record's stores read the staging tiles (R/C region)
+            if (tid == copier || tid == kThreads - 64 || tid == kThreads - 96) bulk_wait_read_all();
+            stores_pending = false;
+        }
+        __syncthreads();
+        // half totals of every block: Lo_b (rows 0-7), Up_b (rows 8-15), P_b = Lo_b Up_b.
+        // F = prod_{b < pb} P_b, G = prod_{b > pb} P_b; XA[a] = Lo_a prod_{pb < b < a} P_b carries
+        // a column of this block to the middle of a later block a; own = Up_pb (lower half) or
+        // Lo_pb (upper half).
+        float Gf[4], cE[4], sf[4], XA[3][4];
+        {
+            float F[4], own[4], dec[4], between[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                F[i] = Gf[i] = dec[i] = between[i] = 1.f;
+                own[i] = 1.f;
+                XA[0][i] = XA[1][i] = XA[2][i] = 0.f;
+            }
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                const float4 lo4 = *reinterpret_cast<const float4*>(loup_s + (bb * 2) * kD + ch0);
+                const float4 up4 = *reinterpret_cast<const float4*>(loup_s + (bb * 2 + 1) * kD + ch0);
+                const float lo[4] = {lo4.x, lo4.y, lo4.z, lo4.w};
+                const float up[4] = {up4.x, up4.y, up4.z, up4.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float Pb = lo[i] * up[i];
+                    dec[i] *= Pb;
+                    if (bb < pb) F[i] *= Pb;
+                    if (bb > pb) {
+                        Gf[i] *= Pb;
+                        if (bb >= 1) XA[bb - 1][i] = lo[i] * between[i];
+                        between[i] *= Pb;
+                    }
+                    if (bb == pb) own[i] = hh == 0 ? up[i] : lo[i];
+                }
+            }
+            if (warp == 0)
+                *reinterpret_cast<float4*>(args.decay + rec * kD + ch0) =
+                    make_float4(dec[0], dec[1], dec[2], dec[3]);
+            // per row, with yi = 1 / y_j:
+            //   lower half: rho = yi, kappa = y_j, sigma = y_j own, e^{Gamma} = F tot yi
+            //   upper half: rho = y_j, kappa = yi, sigma = tot yi, e^{Gamma} = F own y_j
+            // so that sigma = kappa sf and e^{Gamma} = cE rho
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                cE[i] = hh == 0 ? F[i] * tot[i] : F[i] * own[i];
+                sf[i] = hh == 0 ? own[i] : tot[i];
+            }
+        }
+
+        // ---------------------------------------------------------------- operands
+        //   R: k rho, q rho (rho_r = e^{Gamma_r - Gamma_m}, m the middle of r's block)
+        //   C: k kappa (kappa = e^{Gamma_m - Gamma_r}), cross columns k sigma X_a, X_a <= 1
+        //   K+ = k e^{Gamma} (shared), Q+ = q e^{Gamma} (parked in the Q~ slot),
+        //   K_end = k e^{Gamma_end - Gamma} = k G sigma (workspace)
+        {
+            bool range_bad = false;
+            __nv_bfloat16* qplus = args.wq + ((size_t)rec * 128 + 64) * kD + ch0;
+            __nv_bfloat16* kend = args.ke + (size_t)rec * kC * kD + ch0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = rbase + j;
+                const bool ok = r < L;
+                const size_t off = in_base + (size_t)r * row_stride;
+                const uint2 kv = ok ? __ldg(reinterpret_cast<const uint2*>(args.k + off))
+                                    : make_uint2(0u, 0u);
+                const uint2 qv = ok ? __ldg(reinterpret_cast<const uint2*>(args.q + off))
+                                    : make_uint2(0u, 0u);
+                const float2 k01 = unpack_bf16(kv.x), k23 = unpack_bf16(kv.y);
+                const float2 q01 = unpack_bf16(qv.x), q23 = unpack_bf16(qv.y);
+                const float kk[4] = {k01.x, k01.y, k23.x, k23.y};
+                const float qq[4] = {q01.x, q01.y, q23.x, q23.y};
+                float rho[4], kap[4], sig[4], e[4], x[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float yv = y[j][i];
+                    const float yi = __fdividef(1.f, yv);
+                    rho[i] = hh == 0 ? yi : yv;
+                    kap[i] = hh == 0 ? yv : yi;
+                    sig[i] = kap[i] * sf[i];
+                    e[i] = cE[i] * rho[i];
+                    x[i] = Gf[i] * sig[i];
+                }
+                st_bf16x4(sm + OFF_R + toff(128, rb8, j), kk[0] * rho[0], kk[1] * rho[1],
+                          kk[2] * rho[2], kk[3] * rho[3]);
+                st_bf16x4(sm + OFF_R + toff(128, rb8 + 8, j), qq[0] * rho[0], qq[1] * rho[1],
+                          qq[2] * rho[2], qq[3] * rho[3]);
+                st_bf16x4(sm + OFF_C + toff(160, rb8, j), kk[0] * kap[0], kk[1] * kap[1],
+                          kk[2] * kap[2], kk[3] * kap[3]);
+#pragma unroll
+                for (int a = 1; a < 4; ++a) {
+                    if (a <= pb) continue;
+                    const float* xa = XA[a - 1];
+                    st_bf16x4(sm + OFF_C + toff(160, rb8 + 8 + cross_off(a) / 8, j),
+                              kk[0] * sig[0] * xa[0], kk[1] * sig[1] * xa[1],
+                              kk[2] * sig[2] * xa[2], kk[3] * sig[3] * xa[3]);
+                }
+                st_bf16x4(sm + OFF_KP + toff(64, rb8, j), kk[0] * e[0], kk[1] * e[1],
+                          kk[2] * e[2], kk[3] * e[3]);
+                *reinterpret_cast<uint2*>(qplus + (size_t)r * kD) =
+                    make_uint2(pack_bf16(qq[0] * e[0], qq[1] * e[1]),
+                               pack_bf16(qq[2] * e[2], qq[3] * e[3]));
+                *reinterpret_cast<uint2*>(kend + (size_t)r * kD) =
+                    make_uint2(pack_bf16(kk[0] * x[0], kk[1] * x[1]),
+                               pack_bf16(kk[2] * x[2], kk[3] * x[3]));
+            }
+            // the reciprocals stay finite while every factor they invert is >= 1e-30; the running
+            // products only shrink, so the first suffix (lower half) or the last prefix (upper
+            // half) is the smallest
+#pragma unroll
+            for (int i = 0; i < 4; ++i) range_bad |= (hh == 0 ? y[0][i] : y[7][i]) < 1e-30f;
+            if (range_bad) set_device_error(args.err, DEV_RANGE);
+        }
+        fence_proxy_async();
+        __syncthreads();
+
+        // ---------------------------------------------------------------- MMA: R C^T
+        if (warp == 0) {   // lane 0 issues; the rest of warp 0 waits for it
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 160, 0, 0);
+#pragma unroll
+                for (int s = 0; s < kD / 16; ++s) {
+                    const int k0 = 16 * s;
+                    const uint64_t ad = desc_at(dK, sb + OFF_R + (k0 >> 6) * 16384 + (k0 & 63) * 2);
+                    const uint64_t bd = desc_at(dK, sb + OFF_C + (k0 >> 6) * 20480 + (k0 & 63) * 2);
+                    umma_f16(tbase + TM_A, ad, bd, id, s > 0);
+                }
+                umma_commit(bar_mma);
+            }
+            __syncwarp();
+        }
+        mma_pending = true;
+
+        // ---------------------------------------------------------------- assemble A_kk, A_qk
+        if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
+        ++mma_phase;
+        mma_pending = false;
+        tc_fence_after();
+        {
+            float* Lb = reinterpret_cast<float*>(sm + OFF_LB);
+            const bool is_q = qd >= 2;
+            const int r = 32 * (qd & 1) + lane;
+            const int a = r >> 4;
+            const float br = beta_s[r];
+            // write 16 consecutive entries (i0 .. i0+15) of row r
+            auto put16 = [&](int i0, const float* x) {
+                if (is_q) {
+                    st_bf16x8(sm + OFF_ZA + sw128_off(128, 64 + r, i0), x);
+                    st_bf16x8(sm + OFF_ZA + sw128_off(128, 64 + r, i0 + 8), x + 8);
+                } else {
+                    float4* dst = reinterpret_cast<float4*>(Lb + r * kLdl + i0);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m)
+                        dst[m] = make_float4(br * x[4 * m], br * x[4 * m + 1], br * x[4 * m + 2],
+                                             br * x[4 * m + 3]);
+                }
+            };
+            if (hf == 0) {
+                // this row's diagonal block, masked to i < r (A_kk) or i <= r (A_qk)
+                float v[32];
+                tmem_ld32(tbase + lane_q + TM_A + 32 * (qd & 1), v);
+                tmem_ld_wait();
+                float x[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int i = 16 * a + j;
+                    const float val = (a & 1) ? v[16 + j] : v[j];
+                    x[j] = (is_q ? i <= r : i < r) ? val : 0.f;
+                }
+                put16(16 * a, x);
+                const uint4 z = make_uint4(0, 0, 0, 0);
+                if (is_q) {   // A_qk is lower triangular: zero the blocks after the diagonal one
+                    for (int i = 16 * (a + 1); i < kC; i += 8)
+                        *reinterpret_cast<uint4*>(sm + OFF_ZA + sw128_off(128, 64 + r, i)) = z;
+                } else {      // rows 0-63 of [0; A_qk] are zero
+#pragma unroll
+                    for (int i = 0; i < kC; i += 8)
+                        *reinterpret_cast<uint4*>(sm + OFF_ZA + sw128_off(128, r, i)) = z;
+                }
+            } else if ((qd & 1) == 0) {
+                float w[16];
+                tmem_ld16(tbase + lane_q + TM_A + 64 + cross_off(1), w);   // block 1: i in 0..15
+                tmem_ld_wait();
+                if (a == 1) put16(0, w);
+            } else {
+                float v[32];
+                tmem_ld32(tbase + lane_q + TM_A + 64 + cross_off(2), v);   // block 2: i in 0..31
+                tmem_ld_wait();
+                if (a == 2) {
+                    put16(0, v);
+                    put16(16, v + 16);
+                }
+                tmem_ld32(tbase + lane_q + TM_A + 64 + cross_off(3), v);   // block 3: i in 0..31
+                tmem_ld_wait();
+                if (a == 3) {
+                    put16(0, v);
+                    put16(16, v + 16);
+                }
+                float w[16];
+                tmem_ld16(tbase + lane_q + TM_A + 64 + cross_off(3) + 32, w);   // i in 32..47
+                tmem_ld_wait();
+                if (a == 3) put16(32, w);
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---------------------------------------------------------------- UT transform
+        {
+            const float* Lb = reinterpret_cast<const float*>(sm + OFF_LB);
+            float* Mb = reinterpret_cast<float*>(sm + OFF_MB);
+            // diagonal 16x16 blocks of (I + L)^-1: forward substitution for column j of block bk,
+            // x_k = [k = j] - sum_{m<k} L[k][m] x_m, by four threads: part t keeps the running
+            // sums of rows t, t + 4, t + 8, t + 12 and the owner of row k broadcasts x_k to the
+            // other three. L is zero on and above the diagonal of its diagonal blocks, so every
+            // row takes every update.
+            {
+                const int bk = tid >> 6, j = (tid >> 2) & 15, t = tid & 3;
+                const int base = 16 * bk;
+                const int src0 = lane & ~3;
+                float lr[4][16];
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float4 x = *reinterpret_cast<const float4*>(
+                            Lb + (base + t + 4 * ii) * kLdl + base + 4 * m);
+                        lr[ii][4 * m] = x.x;
+                        lr[ii][4 * m + 1] = x.y;
+                        lr[ii][4 * m + 2] = x.z;
+                        lr[ii][4 * m + 3] = x.w;
+                    }
+                float acc[4] = {0.f, 0.f, 0.f, 0.f}, xo[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int own = k & 3, kk = k >> 2;
+                    float xk = (k == j ? 1.f : 0.f) - acc[kk];   // meaningful on the owner only
+                    xk = __shfl_sync(0xffffffffu, xk, src0 + own);
+                    if (t == own) xo[kk] = xk;
+#pragma unroll
+                    for (int ii = 0; ii < 4; ++ii) acc[ii] = fmaf(lr[ii][k], xk, acc[ii]);
+                }
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii) Mb[(base + t + 4 * ii) * kLdm + base + j] = xo[ii];
+            }
+            __syncthreads();
+            // off-diagonal blocks of M = (I + L)^-1 (tf32 mma.sync, one warp per 16x16 block).
+            //   level 1:  M_{b+1,b} = -M_{b+1,b+1} L_{b+1,b} M_bb
+            //   level 2:  the lower-left 32x32 block, M[32:, :32] = -M[32:, 32:] L[32:, :32] M[:32, :32],
+            //             as Y = L[32:, :32] M[:32, :32] (four blocks) and then -M[32:, 32:] Y
+            //             (blocks (2,0), (3,0), (3,1); (2,1) is known from level 1)
+            const int g = lane >> 2, t = lane & 3;
+            float* ysb = reinterpret_cast<float*>(sm + OFF_YS);
+            // acc += A[0:16, 0:K] B[0:K, 0:16] for fp32 row-major sources
+            auto mm16 = [&](float (&acc)[2][4], const float* A, int lda, const float* B, int ldb,
+                            int K) {
+                for (int kk = 0; kk < K; kk += 8) {
+                    const float* la = A + g * lda + kk + t;
+                    const uint32_t a[4] = {f2tf(la[0]), f2tf(la[8 * lda]), f2tf(la[4]),
+                                           f2tf(la[8 * lda + 4])};
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const float* lb = B + (kk + t) * ldb + 8 * nt + g;
+                        const uint32_t b[2] = {f2tf(lb[0]), f2tf(lb[4 * ldb])};
+                        mma_tf32_16x8x8(acc[nt], a, b);
+                    }
+                }
+            };
+            auto st16 = [&](float* dst, int ld, const float (&z)[2][4], float sign) {
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    dst[g * ld + 8 * nt + 2 * t] = sign * z[nt][0];
+                    dst[g * ld + 8 * nt + 2 * t + 1] = sign * z[nt][1];
+                    dst[(g + 8) * ld + 8 * nt + 2 * t] = sign * z[nt][2];
+                    dst[(g + 8) * ld + 8 * nt + 2 * t + 1] = sign * z[nt][3];
+                }
+            };
+            if (warp < 3) {
+                const int bb = warp, aa = warp + 1;
+                float* ys = ysb + warp * 16 * 17;
+                float yy[2][4] = {}, z[2][4] = {};
+                mm16(yy, Lb + 16 * aa * kLdl + 16 * bb, kLdl, Mb + 16 * bb * kLdm + 16 * bb, kLdm, 16);
+                st16(ys, 17, yy, 1.f);
+                __syncwarp();
+                mm16(z, Mb + 16 * aa * kLdm + 16 * aa, kLdm, ys, 17, 16);
+                st16(Mb + 16 * aa * kLdm + 16 * bb, kLdm, z, -1.f);
+            }
+            __syncthreads();
+            if (warp < 4) {   // Y_{ra,cb} = sum over k-blocks cb..1 of L_{ra,k} M_{k,cb}
+                const int ra = 2 + (warp >> 1), cb = warp & 1;
+                float yy[2][4] = {};
+                mm16(yy, Lb + 16 * ra * kLdl + 16 * cb, kLdl, Mb + 16 * cb * kLdm + 16 * cb, kLdm,
+                     32 - 16 * cb);
+                st16(ysb + warp * 16 * 17, 17, yy, 1.f);   // Y_{2,cb} in slot cb, Y_{3,cb} in 2 + cb
+            }
+            __syncthreads();
+            if (warp < 3) {   // warp 0: M_20 = -M_22 Y_20;  warps 1, 2: M_3c = -(M_32 Y_2c + M_33 Y_3c)
+                const int cb = warp == 2 ? 1 : 0;
+                float z[2][4] = {};
+                if (warp == 0) {
+                    mm16(z, Mb + 32 * kLdm + 32, kLdm, ysb, 17, 16);
+                    st16(Mb + 32 * kLdm, kLdm, z, -1.f);
+                } else {
+                    mm16(z, Mb + 48 * kLdm + 32, kLdm, ysb + cb * 16 * 17, 17, 16);
+                    mm16(z, Mb + 48 * kLdm + 48, kLdm, ysb + (2 + cb) * 16 * 17, 17, 16);
+                    st16(Mb + 48 * kLdm + 16 * cb, kLdm, z, -1.f);
+                }
+            }
+            __syncthreads();
+            // T = (I + L)^-1 diag(beta): lower triangle, bf16 K-major
+            {
+                const int i = 2 * lane;
+                const float b0 = beta_s[i], b1 = beta_s[i + 1];
+#pragma unroll
+                for (int rr8 = 0; rr8 < 8; ++rr8) {
+                    const int r = 8 * warp + rr8;
+                    const float2 m = *reinterpret_cast<const float2*>(Mb + r * kLdm + i);
+                    const float x0 = (i <= r) ? m.x * b0 : 0.f;
+                    const float x1 = (i + 1 <= r) ? m.y * b1 : 0.f;
+                    *reinterpret_cast<uint32_t*>(sm + OFF_TT + sw128_off(128, r, i)) =
+                        pack_bf16(x0, x1);
+                }
+            }
+        }
+        fence_proxy_async();
+        __syncthreads();
+
+        // ---------------------------------------------------------------- MMA: T' = A_qk T
+        // [0; A_qk] (128 x 64) times T as the MN-major B operand: lanes 64-127 receive A_qk T.
+        if (warp == 0) {
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 64, 0, 1);
+#pragma unroll
+                for (int s = 0; s < kC / 16; ++s)
+                    umma_f16(tbase + TM_TP, desc_at(dK, sb + OFF_ZA + 32 * s),
+                             desc_at(dM8, sb + OFF_TT + 2048 * s), id, s > 0);
+                umma_commit(bar_mma);
+            }
+            __syncwarp();
+        }
+        mma_pending = true;
+        if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
+        ++mma_phase;
+        mma_pending = false;
+        tc_fence_after();
+        if (qd >= 2) {
+            // T' rows r = 32 (qd - 2) + lane  ->  rows 64 + r of [T; T']
+            float v[32];
+            const int r = 32 * (qd - 2) + lane;
+            tmem_ld32(tbase + lane_q + TM_TP + 32 * hf, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                st_bf16x8(sm + OFF_TT + sw128_off(128, 64 + r, 32 * hf + 8 * m), v + 8 * m);
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---------------------------------------------------------------- MMA: WY products
+        // [T; T'] K+ (lanes 0-63: W, 64-127: A_qk W) and, transposed for the state pass,
+        // V^T [T; T']^T (lane j = value column: U~^T in columns 128-191, O~^T in 192-255)
+        if (!wait_all(bar_v, v_count & 1)) { aborted = true; break; }
+        ++v_count;
+        v_pending = false;
+        if (warp == 0) {
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 128, 0, 1);
+                const uint32_t idt = idesc_bf16(128, 128, 1, 0);
+#pragma unroll
+                for (int s = 0; s < kC / 16; ++s)
+                    umma_f16(tbase + TM_A, desc_at(dK, sb + OFF_TT + 32 * s),
+                             desc_at(dM8, sb + OFF_KP + 2048 * s), id, s > 0);
+                umma_commit(bar_mma);   // W and A_qk W: read out while the next group runs
+#pragma unroll
+                for (int s = 0; s < kC / 16; ++s)
+                    umma_f16(tbase + TM_A + 128, desc_at(dM8, sb + OFF_V + 2048 * s),
+                             desc_at(dK, sb + OFF_TT + 32 * s), idt, s > 0);
+                umma_commit(bar_wy2);
+            }
+            __syncwarp();
+        }
+        mma_pending = wy2_pending = true;
+        if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
+        ++mma_phase;
+        mma_pending = false;
+        tc_fence_after();
+        {
+            // quarters 0-1: W rows -> [W; Q~] rows 0-63.  quarters 2-3: Q~ = Q+ - A_qk W, with
+            // Q+ read back from the workspace. Each warp takes 64 of the 128 columns.
+            const int r = 32 * (qd & 1) + lane;
+            const int row = qd < 2 ? r : 64 + r;
+            const uint4* qp = reinterpret_cast<const uint4*>(
+                args.wq + ((size_t)rec * 128 + 64 + r) * kD + 64 * hf);
+#pragma unroll
+            for (int part = 0; part < 4; ++part) {
+                const int c0 = 64 * hf + 16 * part;
+                uint4 qv2[2];
+                if (qd >= 2) {
+                    qv2[0] = __ldcg(qp + 2 * part);
+                    qv2[1] = __ldcg(qp + 2 * part + 1);
+                }
+                float v[16];
+                tmem_ld16(tbase + lane_q + TM_A + c0, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    uint8_t* p = sm + OFF_SWQ + sw128_off(128, row, c0 + 8 * m);
+                    const float* w = v + 8 * m;
+                    if (qd < 2) {
+                        st_bf16x8(p, w);
+                    } else {
+                        const float2 a0 = unpack_bf16(qv2[m].x), a1 = unpack_bf16(qv2[m].y);
+                        const float2 a2 = unpack_bf16(qv2[m].z), a3 = unpack_bf16(qv2[m].w);
+                        *reinterpret_cast<uint4*>(p) = make_uint4(
+                            pack_bf16(a0.x - w[0], a0.y - w[1]), pack_bf16(a1.x - w[2], a1.y - w[3]),
+                            pack_bf16(a2.x - w[4], a2.y - w[5]), pack_bf16(a3.x - w[6], a3.y - w[7]));
+                    }
+                }
+            }
+        }
+        if (!wait_all(bar_wy2, wy2_count & 1)) { aborted = true; break; }
+        ++wy2_count;
+        wy2_pending = false;
+        tc_fence_after();
+        {
+            // U~^T (TMEM columns 128-191) and O~^T (192-255), lane j = value column, into bf16
+            // staging tiles [128 j][64 tokens] (128-byte swizzle)
+            const int jrow = 32 * qd + lane;
+            const uint32_t stage = hf == 0 ? OFF_SUT : OFF_SOT;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                float v[32];
+                tmem_ld32(tbase + lane_q + TM_A + 128 + 64 * hf + 32 * part, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    st_bf16x8(sm + stage + sw128_off(128, jrow, 32 * part + 8 * m), v + 8 * m);
+            }
+        }
+        // shared staging tiles and the Q+ parked in the workspace, before the async-proxy stores
+        fence_proxy_async_all();
+        tc_fence_before();
+        __syncthreads();
+        {
+            const int rw = (int)(rec * 128);
+            if (tid == copier) {
+                tma_store_2d(&maps.wq, sb + OFF_SWQ, 0, rw);
+                tma_store_2d(&maps.wq, sb + OFF_SWQ + 16384, 64, rw);
+                bulk_commit();
+            } else if (tid == kThreads - 64) {
+                tma_store_2d(&maps.ut, sb + OFF_SUT, 0, rw);
+                bulk_commit();
+            } else if (tid == kThreads - 96) {
+                tma_store_2d(&maps.ot, sb + OFF_SOT, 0, rw);
+                bulk_commit();
+            }
+            stores_pending = true;
+        }
+        has_cur = next_unit(cur);
+    }
+
+    if (aborted) {
+        if (tid == 0) set_device_error(args.err, DEV_TIMEOUT);
+        // wind down: let this CTA's own copies and MMAs finish before TMEM and smem go away
+        const long long drain = 1ll << 31;
+        if (v_pending && tid == 0) mbar_wait(bar_v, v_count & 1, drain);
+        if (mma_pending && tid == 0) mbar_wait(bar_mma, mma_phase & 1, drain);
+        if (wy2_pending && tid == 0) mbar_wait(bar_wy2, wy2_count & 1, drain);
+    }
+    if (tid == copier || tid == kThreads - 64 || tid == kThreads - 96)
+        bulk_wait_all();   // stores complete before the smem goes away
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, kTmemCols);
+}
+
+// ------------------------------------------------------------------ host side
+
+// [rows, H, 128] row-major tensor, one head's 64-row tile per box of box_inner columns
+cudaError_t make_rows_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt,
+                          int elem_bytes, long long rows, int H, int box_inner,
+                          CUtensorMapSwizzle sw) {
+    return make_map_3d_box(m, base, dt, elem_bytes, (unsigned long long)rows, H, kD, box_inner,
+                           kC, sw);
+}
+
+long long wait_budget() {
+    static long long budget = [] {
+        const char* s = std::getenv("KDA_DEBUG_WAIT_CYCLES");
+        if (s && *s) {
+            const long long v = std::atoll(s);
+            if (v > 0) return v;
+        }
+        return 1ll << 31;   // about one second of SM clock
+    }();
+    return budget;
+}
+
+int debug_stall() {
+    static int v = [] {
+        const char* s = std::getenv("KDA_DEBUG_STALL_WAIT");
+        return (s && *s && *s != '0') ? 1 : 0;
+    }();
+    return v;
+}
+
+// resident CTAs of intra_kernel across the GPU: as many per SM as its registers and shared
+// memory allow (two on B200), by the SM's own limits and by the runtime's occupancy query,
+// whichever is larger. A CTA beyond the resident count would only start later, never wait on
+// another, so an overestimate costs time, not correctness.
+cudaError_t intra_grid_cap(int* cap) {
+    static std::once_flag once;
+    static cudaError_t err = cudaSuccess;
+    static int value = 0;
+    std::call_once(once, [] {
+        err = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)kSmemBytes);
+        if (err != cudaSuccess) return;
+        err = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                   (int)cudaSharedmemCarveoutMaxShared);
+        if (err != cudaSuccess) return;
+        int dev = 0, sms = 0, smem_sm = 0, smem_rsv = 0, regs_sm = 0, per_sm = 0;
+        cudaFuncAttributes fa;
+        if ((err = cudaGetDevice(&dev)) != cudaSuccess ||
+            (err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) !=
+                cudaSuccess ||
+            (err = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor,
+                                          dev)) != cudaSuccess ||
+            (err = cudaDeviceGetAttribute(&smem_rsv, cudaDevAttrReservedSharedMemoryPerBlock,
+                                          dev)) != cudaSuccess ||
+            (err = cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor,
+                                          dev)) != cudaSuccess ||
+            (err = cudaFuncGetAttributes(&fa, intra_kernel)) != cudaSuccess ||
+            (err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, intra_kernel, kThreads,
+                                                                 kSmemBytes)) != cudaSuccess)
+            return;
+        const int by_smem = smem_sm / ((int)kSmemBytes + fa.sharedSizeBytes + smem_rsv);
+        const int by_regs = fa.numRegs > 0 ? regs_sm / (fa.numRegs * kThreads) : 1;
+        int fit = by_smem < by_regs ? by_smem : by_regs;
+        if (fit > 2) fit = 2;   // __launch_bounds__ sizes the kernel for two
+        if (per_sm < fit) per_sm = fit;
+        value = sms * (per_sm > 0 ? per_sm : 1);
+    });
+    *cap = value;
+    return err;
+}
+
+}  // namespace
+
+cudaError_t launch_chunk64_intra(const FwdParams& p, cudaStream_t stream) {
+    const SplitWorkspace& ws = *p.split;
+    cudaError_t e = tma_encoder_ready();
+    if (e != cudaSuccess) return e;
+    const long long rows = (long long)p.B * p.T;
+    const long long items = ws.G * p.H;
+    if (items == 0 || rows <= 0) return cudaSuccess;
+    if (items * 128 > 0x7fffffffLL || rows > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const auto F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const auto SWN = CU_TENSOR_MAP_SWIZZLE_NONE;
+    const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+    IntraMaps m;
+    const unsigned long long R = (unsigned long long)items;
+    if ((e = make_rows_map(&m.q, p.q, BF, 2, rows, p.H, kD, SWN)) != cudaSuccess ||
+        (e = make_rows_map(&m.k, p.k, BF, 2, rows, p.H, kD, SWN)) != cudaSuccess ||
+        (e = make_rows_map(&m.g, p.log_g, F32, 4, rows, p.H, kD, SWN)) != cudaSuccess ||
+        (e = make_rows_map(&m.v, p.v, BF, 2, rows, p.H, 64, SW)) != cudaSuccess ||
+        (e = make_map_2d(&m.wq, ws.wq, BF, 2, R * 128, kD, 64, 128, SW)) != cudaSuccess ||
+        (e = make_map_2d(&m.ut, ws.ut, BF, 2, R * 128, kC, 64, 128, SW)) != cudaSuccess ||
+        (e = make_map_2d(&m.ot, ws.ot, BF, 2, R * 128, kC, 64, 128, SW)) != cudaSuccess)
+        return e;
+    int cap = 0;
+    if ((e = intra_grid_cap(&cap)) != cudaSuccess) return e;
+    IntraArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = static_cast<const __nv_bfloat16*>(p.q);
+    a.k = static_cast<const __nv_bfloat16*>(p.k);
+    a.g = p.log_g;
+    a.beta = static_cast<const __nv_bfloat16*>(p.beta);
+    a.cu = p.cu_seqlens;
+    a.map = ws.map;
+    a.wq = ws.wq;
+    a.ke = ws.ke;
+    a.decay = ws.decay;
+    a.G = ws.G;
+    a.ncT = ws.ncT;
+    a.T = p.T;
+    a.H = p.H;
+    a.N = p.N;
+    a.budget = wait_budget();
+    a.debug_stall = debug_stall();
+    a.err = p.err;
+    const long long grid = items < cap ? items : cap;
+    intra_kernel<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(m, a);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

@@ -1,7 +1,7 @@
 // State pass of the split chunked prefill: the only part of the chunked form that is sequential
 // over chunks.
 //
-// The intra-chunk kernel (chunk64_kernel in its intra mode) has already written, for every chunk
+// The intra-chunk kernel (intra_kernel, kda_intra.cu) has already written, for every chunk
 // of 64 tokens and every head, the chunk's WY factors to the workspace:
 //   [W; Q~] (128 x 128 bf16), K_end (64 x 128 bf16), U~^T and O~^T (128 value columns x 64
 //   tokens, bf16) and the chunk's total decay e^{Gamma_end} (128 fp32).

@@ -46,11 +46,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return done != 0;
 }
 
+// try_wait that may suspend the thread until the phase completes (or about a millisecond
+// passes), instead of returning after the system's default time: a waiting thread then takes no
+// issue slots from the warps of other CTAs on the SM.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity), "r"(1000000u)
+        : "memory");
+    return done != 0;
+}
+
 // Wait for the phase with the given parity to complete, giving up after `budget` SM clock
 // cycles. Returns false on timeout (the caller records the error and winds down).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long budget) {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > budget) return false;
+    }
+    return true;
+}
+
+// The same with the suspending try_wait (for throughput kernels that share an SM).
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, long long budget) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait_sleep(bar, parity)) {
         if (clock64() - t0 > budget) return false;
     }
     return true;

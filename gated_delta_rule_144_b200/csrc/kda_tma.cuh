@@ -14,7 +14,12 @@ cudaError_t make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt
                         unsigned long long rows, int cols, int box_cols, int box_rows,
                         CUtensorMapSwizzle sw);
 
-// Token-major [rows][H][cols] tensor (one head's rows), box of box_rows rows x cols, no swizzle.
+// Token-major [rows][H][cols] tensor (one head's rows), box of box_rows rows x box_cols columns.
+cudaError_t make_map_3d_box(CUtensorMap* m, const void* base, CUtensorMapDataType dt,
+                            int elem_bytes, unsigned long long rows, int H, int cols, int box_cols,
+                            int box_rows, CUtensorMapSwizzle sw);
+
+// The same with whole rows per box (box_cols = cols) and no swizzle.
 cudaError_t make_map_3d_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt,
                              int elem_bytes, unsigned long long rows, int H, int cols,
                              int box_rows);
