@@ -16,14 +16,16 @@
 //
 // Occupancy: two CTAs share each SM, so that one CTA's tensor-core waits, barriers and memory
 // latency are covered by the other's CUDA-core work. To fit two CTAs (about 110 KB of shared memory
-// and 256 TMEM columns each), q, k and log g go straight from global memory into registers (the
-// next record's tiles are prefetched into L2 by TMA while this one runs), K_end is written to the
-// workspace from registers, and Q+ = q e^{Gamma} is parked in the workspace slot of Q~ and read
-// back when Q~ = Q+ - A_qk W is formed. Only V (an MMA operand) arrives by TMA into shared memory.
+// and 256 TMEM columns each) the tiles share space: k and q arrive by TMA where R's rows go and are
+// overwritten in place by k rho and q rho, log g arrives in the K+ / V region and is consumed before
+// K+ and V are written there, the R/C region then holds the UT solve and finally the store staging.
+// K_end is written to the workspace from registers, and Q+ = q e^{Gamma} is parked in the workspace
+// slot of Q~ and read back when Q~ = Q+ - A_qk W is formed. The next record's input tiles are
+// prefetched into L2 while this one runs.
 //
 // Per record (256 threads; thread 0 issues the MMAs, lane 0 of warp 7 the copies):
-//   loads -> decay products -> R, C, K+ (shared), Q+, K_end (global) -> MMA R C^T ->
-//   A_kk, A_qk -> UT solve -> MMA T' = A_qk T -> MMA [T; T'] K+ and V^T [T; T']^T ->
+//   TMA k, q, log g -> decay products -> TMA V; R, C, K+ (shared), Q+, K_end (global) ->
+//   MMA R C^T -> A_kk, A_qk -> UT solve -> MMA T' = A_qk T -> MMA [T; T'] K+ and V^T [T; T']^T ->
 //   [W; Q~], U~^T, O~^T staged in shared memory -> TMA stores.
 // Every mbarrier wait is bounded; on expiry the CTA records KDA_ERR_TIMEOUT, drains its own
 // copies and MMAs, frees TMEM and exits.
@@ -84,6 +86,9 @@ constexpr uint32_t TM_TP = 160;  // [0; A_qk] T (lanes 64-127: T')
 constexpr int kLdl = 68;         // row stride (floats) of L: conflict-free A-fragment loads
 constexpr int kLdm = 72;         // row stride (floats) of M: conflict-free B-fragment loads
 constexpr uint32_t kTxV = 16384;
+constexpr uint32_t kTxIn = 16384 + 16384 + 32768;   // k, q (bf16) and log g (fp32) tiles
+constexpr uint32_t OFF_G = 0;   // log g [64][128] f32 row-major, in the K+ / V region until the
+                                //   decay products have read it
 
 // row offset, inside C[64:], of the columns row block a needs from earlier blocks
 __host__ __device__ constexpr int cross_off(int a) { return a == 1 ? 0 : (a == 2 ? 16 : 48); }
@@ -105,8 +110,9 @@ struct IntraArgs {
     unsigned* err;
 };
 
-// q, k, log g, v: [rows, H, 128] maps of one head's 64-row tile (q, k, g for L2 prefetch, v for
-// the shared-memory copy, 64-column boxes); wq, ut, ot: record stores (128-byte swizzle).
+// q, k, v: [rows, H, 128] maps of one head's 64-row tile in 64-column boxes (128-byte swizzle);
+// log g: the same with whole 128-column rows, no swizzle; wq, ut, ot: record stores (128-byte
+// swizzle).
 struct IntraMaps {
     CUtensorMap q, k, g, v, wq, ut, ot;
 };
@@ -191,7 +197,7 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
     float* loup_s = reinterpret_cast<float*>(sm + OFF_LOUP);
     uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
     const uint32_t bar_v = sb + OFF_BAR, bar_mma = bar_v + 8, bar_wy2 = bar_v + 16;
-    const uint32_t bar_never = bar_v + 24;
+    const uint32_t bar_never = bar_v + 24, bar_in = bar_v + 32;
     // lane 0 of the last warp issues copies and the [W; Q~] stores; warps 5 and 6 the others
     const int copier = kThreads - 32;
 
@@ -200,6 +206,7 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         mbar_init(bar_mma, 1);
         mbar_init(bar_wy2, 1);
         mbar_init(bar_never, 1);
+        mbar_init(bar_in, 1);
         fence_mbar_init();
     }
     if (tid == copier) {
@@ -226,10 +233,24 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         tma_load_3d(sb + OFF_V, &maps.v, bar_v, 0, u.h, (int)u.row0);
         tma_load_3d(sb + OFF_V + 8192, &maps.v, bar_v, 64, u.h, (int)u.row0);
     };
+    // q and k land where R's k rows (0-63) and q rows (64-127) go, one 64-column panel per box,
+    // so that each thread overwrites its own elements with k rho and q rho; log g lands in the
+    // K+ / V region, which it leaves before K+ and V are written
+    auto issue_in = [&](const Unit& u) {
+        const int row0 = (int)u.row0;
+        mbar_arrive_expect_tx(bar_in, kTxIn);
+        tma_load_3d(sb + OFF_R, &maps.k, bar_in, 0, u.h, row0);
+        tma_load_3d(sb + OFF_R + 16384, &maps.k, bar_in, 64, u.h, row0);
+        tma_load_3d(sb + OFF_R + 8192, &maps.q, bar_in, 0, u.h, row0);
+        tma_load_3d(sb + OFF_R + 16384 + 8192, &maps.q, bar_in, 64, u.h, row0);
+        tma_load_3d(sb + OFF_G, &maps.g, bar_in, 0, u.h, row0);
+    };
     auto prefetch_inputs = [&](const Unit& u) {
         const int row0 = (int)u.row0;
         tma_prefetch_3d(&maps.q, 0, u.h, row0);
+        tma_prefetch_3d(&maps.q, 64, u.h, row0);
         tma_prefetch_3d(&maps.k, 0, u.h, row0);
+        tma_prefetch_3d(&maps.k, 64, u.h, row0);
         tma_prefetch_3d(&maps.g, 0, u.h, row0);
         tma_prefetch_3d(&maps.v, 0, u.h, row0);
         tma_prefetch_3d(&maps.v, 64, u.h, row0);
@@ -240,7 +261,8 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
     const uint64_t dM8 = sw128_desc(0, 8192, 1024);  // MN-major, 128B swizzle, 64-row panels
 
     bool v_pending = false, mma_pending = false, wy2_pending = false, stores_pending = false;
-    int v_count = 0, wy2_count = 0;
+    bool in_pending = false;
+    int v_count = 0, wy2_count = 0, in_count = 0;
     uint32_t mma_phase = 0;
     bool aborted = false;
     // One thread polls; the rest of the CTA waits at the barrier that publishes the outcome.
@@ -266,7 +288,7 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         return (uint32_t)((lane >> 4) * R * 128 + rb * 1024 + j * 128) + (lh4 ^ (uint32_t)(j << 4)) +
                lo8;
     };
-    const size_t row_stride = (size_t)H * kD;   // elements between consecutive tokens
+    const float* gs = reinterpret_cast<const float*>(sm + OFF_G);
 
     for (int c = 0; has_cur && !aborted; ++c) {
         const long long row0 = cur.row0;
@@ -274,28 +296,26 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         const int h = cur.h;
         const long long rec = cur.rec;
 
-        // V of this record (its panel is free: the previous record's products have completed);
-        // the next record's inputs go to L2 while this one runs
+        // inputs of this record: the previous record's products have completed (K+ / V region
+        // free) and, after the wait below, its stores have read the staging tiles (R/C region)
+        if (stores_pending) {
+            if (tid == copier || tid == kThreads - 64 || tid == kThreads - 96) bulk_wait_read_all();
+            __syncthreads();
+            stores_pending = false;
+        }
         if (tid == copier) {
-            issue_v(cur);
+            issue_in(cur);
             const long long saved = cursor;   // look one record ahead without consuming it
             Unit ahead;
             if (next_unit(ahead)) prefetch_inputs(ahead);
             cursor = saved;
         }
-        v_pending = true;
+        in_pending = true;
         if (tid < kC)
             beta_s[tid] = tid < L ? __bfloat162float(args.beta[(row0 + tid) * H + h]) : 0.f;
-
-        // ---------------------------------------------------------------- loads of this record
-        // rows >= L (past the end of the chunk's document) read as log g = 0, k = q = 0
-        const size_t in_base = ((size_t)row0 * H + h) * kD + ch0;
-        float4 gv[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            gv[j] = rbase + j < L ? __ldg(reinterpret_cast<const float4*>(
-                                        args.g + in_base + (size_t)(rbase + j) * row_stride))
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (!wait_all(bar_in, in_count & 1)) { aborted = true; break; }
+        ++in_count;
+        in_pending = false;
 
         // ---------------------------------------------------------------- decay products
         // With a_t = e^{log g_t} over this thread's 8 rows: the lower half (hh = 0) keeps the
@@ -303,6 +323,9 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         // y_j = prod_{t <= j} a_t; tot = prod over all 8 rows. The other product of each row is
         // tot / y_j, formed below from the reciprocal that the operands need anyway.
         float y[8][4], tot[4];
+        float4 g4[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) g4[j] = *reinterpret_cast<const float4*>(gs + (rbase + j) * kD + ch0);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             float run = 1.f;
@@ -310,13 +333,13 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
 #pragma unroll
                 for (int j = 7; j >= 0; --j) {
                     y[j][i] = run;
-                    const float gl = i == 0 ? gv[j].x : i == 1 ? gv[j].y : i == 2 ? gv[j].z : gv[j].w;
+                    const float gl = i == 0 ? g4[j].x : i == 1 ? g4[j].y : i == 2 ? g4[j].z : g4[j].w;
                     run *= rbase + j < L ? __expf(gl) : 1.f;
                 }
             } else {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    const float gl = i == 0 ? gv[j].x : i == 1 ? gv[j].y : i == 2 ? gv[j].z : gv[j].w;
+                    const float gl = i == 0 ? g4[j].x : i == 1 ? g4[j].y : i == 2 ? g4[j].z : g4[j].w;
                     run *= rbase + j < L ? __expf(gl) : 1.f;
                     y[j][i] = run;
                 }
@@ -325,11 +348,9 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         }
         *reinterpret_cast<float4*>(loup_s + (pb * 2 + hh) * kD + ch0) =
             make_float4(tot[0], tot[1], tot[2], tot[3]);
-        if (stores_pending) {   // the previous record's stores read the staging tiles (R/C region)
-            if (tid == copier || tid == kThreads - 64 || tid == kThreads - 96) bulk_wait_read_all();
-            stores_pending = false;
-        }
-        __syncthreads();
+        __syncthreads();   // log g consumed: the K+ / V region is free for V and K+
+        if (tid == copier) issue_v(cur);
+        v_pending = true;
         // half totals of every block: Lo_b (rows 0-7), Up_b (rows 8-15), P_b = Lo_b Up_b.
         // F = prod_{b < pb} P_b, G = prod_{b > pb} P_b; XA[a] = Lo_a prod_{pb < b < a} P_b carries
         // a column of this block to the middle of a later block a; own = Up_pb (lower half) or
@@ -388,11 +409,11 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int r = rbase + j;
-                const bool ok = r < L;
-                const size_t off = in_base + (size_t)r * row_stride;
-                const uint2 kv = ok ? __ldg(reinterpret_cast<const uint2*>(args.k + off))
+                const bool ok = r < L;   // rows past the document read as k = q = 0
+                const uint32_t ok_ = toff(128, rb8, j), oq_ = toff(128, rb8 + 8, j);
+                const uint2 kv = ok ? *reinterpret_cast<const uint2*>(sm + OFF_R + ok_)
                                     : make_uint2(0u, 0u);
-                const uint2 qv = ok ? __ldg(reinterpret_cast<const uint2*>(args.q + off))
+                const uint2 qv = ok ? *reinterpret_cast<const uint2*>(sm + OFF_R + oq_)
                                     : make_uint2(0u, 0u);
                 const float2 k01 = unpack_bf16(kv.x), k23 = unpack_bf16(kv.y);
                 const float2 q01 = unpack_bf16(qv.x), q23 = unpack_bf16(qv.y);
@@ -796,6 +817,7 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         if (tid == 0) set_device_error(args.err, DEV_TIMEOUT);
         // wind down: let this CTA's own copies and MMAs finish before TMEM and smem go away
         const long long drain = 1ll << 31;
+        if (in_pending && tid == 0) mbar_wait(bar_in, in_count & 1, drain);
         if (v_pending && tid == 0) mbar_wait(bar_v, v_count & 1, drain);
         if (mma_pending && tid == 0) mbar_wait(bar_mma, mma_phase & 1, drain);
         if (wy2_pending && tid == 0) mbar_wait(bar_wy2, wy2_count & 1, drain);
@@ -894,8 +916,8 @@ cudaError_t launch_chunk64_intra(const FwdParams& p, cudaStream_t stream) {
     const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
     IntraMaps m;
     const unsigned long long R = (unsigned long long)items;
-    if ((e = make_rows_map(&m.q, p.q, BF, 2, rows, p.H, kD, SWN)) != cudaSuccess ||
-        (e = make_rows_map(&m.k, p.k, BF, 2, rows, p.H, kD, SWN)) != cudaSuccess ||
+    if ((e = make_rows_map(&m.q, p.q, BF, 2, rows, p.H, 64, SW)) != cudaSuccess ||
+        (e = make_rows_map(&m.k, p.k, BF, 2, rows, p.H, 64, SW)) != cudaSuccess ||
         (e = make_rows_map(&m.g, p.log_g, F32, 4, rows, p.H, kD, SWN)) != cudaSuccess ||
         (e = make_rows_map(&m.v, p.v, BF, 2, rows, p.H, 64, SW)) != cudaSuccess ||
         (e = make_map_2d(&m.wq, ws.wq, BF, 2, R * 128, kD, 64, 128, SW)) != cudaSuccess ||
