@@ -145,12 +145,16 @@ KERNEL_SOURCES = {
 
 
 def source_digest(kernel: str):
-    """Digest of the sources a kernel is built from (its profile is stale once they change)."""
+    """Digest of the sources a kernel is built from, with their per-file compiler flags (its
+    profile is stale once either changes)."""
+    from gated_delta_rule_144_b200.build import FILE_FLAGS
     h = hashlib.sha256()
     for name in KERNEL_SOURCES.get(kernel, []):
         p = ROOT / "gated_delta_rule_144_b200" / "csrc" / name
         h.update(name.encode())
         h.update(p.read_bytes() if p.exists() else b"")
+        if FILE_FLAGS.get(name):
+            h.update(" ".join(FILE_FLAGS[name]).encode())
     return h.hexdigest()[:16]
 
 

@@ -29,6 +29,16 @@ FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xptxas", "-v
          "--expt-relaxed-constexpr", "-I", str(INCLUDE), "-I", str(CSRC)]
 
 
+# Per-file flags. The chunked kernels evaluate one exponential and one reciprocal per operand
+# element through the MUFU unit; flushing subnormals lets those intrinsics compile without their
+# subnormal fix-ups (14 % fewer instructions in the intra-chunk kernel). Nothing they compute is
+# meant to be subnormal: decay products below 1e-30 are already reported as out of range.
+FILE_FLAGS = {
+    "kda_intra.cu": ["-ftz=true"],
+    "kda_chunk64.cu": ["-ftz=true"],
+}
+
+
 def nvcc() -> str:
     for cand in (os.environ.get("NVCC"), shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
         if cand and Path(cand).exists():
@@ -48,12 +58,12 @@ def up_to_date() -> bool:
     if not LIB.exists():
         return False
     t = LIB.stat().st_mtime
-    return all(p.stat().st_mtime <= t for p in _deps())
+    return all(p.stat().st_mtime <= t for p in _deps()) and Path(__file__).stat().st_mtime <= t
 
 
 def _compile(src: Path, verbose: bool) -> tuple[Path, str]:
     obj = BUILD / (src.stem + ".o")
-    cmd = [nvcc(), *ARCH, *FLAGS, "-c", str(src), "-o", str(obj)]
+    cmd = [nvcc(), *ARCH, *FLAGS, *FILE_FLAGS.get(src.name, []), "-c", str(src), "-o", str(obj)]
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
