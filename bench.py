@@ -285,9 +285,12 @@ def run_ours(args):
         kernel_name, launches = "kda_recurrent", 1
     elif args.fused:
         kernel_name, launches = "kda_chunk64", 1 + (1 if packed and 2 <= N <= 2048 else 0)
-    else:   # split: intra-chunk kernel + state pass (+ chunk map and document order if packed)
+    else:   # split: intra-chunk kernel + state pass per chunk segment (+ chunk map and document
+        # order if packed)
         kernel_name = "kda_chunk64_intra+kda_chunk_scan"
-        launches = 2 + ((2 if 2 <= N <= 2048 else 1) if packed else 0)
+        segs = kda.fwd_split_segments(B, T, H, dk, dv, N, inp["q"].dtype, args.chunk_size,
+                                      varlen=packed)
+        launches = 2 * segs + ((2 if 2 <= N <= 2048 else 1) if packed else 0)
     traffic = committed_traffic(kernel_name, wl.name)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                 "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),

@@ -80,6 +80,8 @@ def lib():
     L.kda_fwd_no_alloc.restype = i32
     L.kda_fwd_algorithm.argtypes = [ctypes.POINTER(FwdDesc), i32]
     L.kda_fwd_algorithm.restype = i32
+    L.kda_fwd_split_segments.argtypes = [ctypes.POINTER(FwdDesc), i32]
+    L.kda_fwd_split_segments.restype = i32
     L.kda_fwd_workspace_size.argtypes = [ctypes.POINTER(FwdDesc)]
     L.kda_fwd_workspace_size.restype = sz
     L.kda_fwd_workspace_size_min.argtypes = [ctypes.POINTER(FwdDesc)]
@@ -149,6 +151,17 @@ def fwd_algorithm(B, T, H, dk, dv, num_seqs, dtype=torch.bfloat16, chunk_size=0,
     r = int(lib().kda_fwd_algorithm(ctypes.byref(d), int(varlen)))
     if r < 0:
         _check(-r, "kda_fwd_algorithm")
+    return r
+
+
+def fwd_split_segments(B, T, H, dk, dv, num_seqs, dtype=torch.bfloat16, chunk_size=0,
+                       varlen=False) -> int:
+    """Chunk segments the split chunked path runs (two kernel launches each)."""
+    d = FwdDesc(B, T, H, dk, dv, num_seqs, KDA_BF16 if dtype == torch.bfloat16 else KDA_F32,
+                chunk_size)
+    r = int(lib().kda_fwd_split_segments(ctypes.byref(d), int(varlen)))
+    if r < 0:
+        _check(-r, "kda_fwd_split_segments")
     return r
 
 

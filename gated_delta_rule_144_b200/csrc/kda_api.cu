@@ -3,10 +3,12 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
 #include "kda.h"
+
 #include "kda_internal.cuh"
 
 namespace {
@@ -132,11 +134,34 @@ const char* kda_status_string(kda_status_t s) {
     return "unknown status";
 }
 
+// Segments of at least 32 chunks, at most 12 (measured on the long-context workload, 1024 chunks
+// per sequence: 1, 4, 8, 12, 16 segments take 5.31, 5.32, 4.89, 4.78, 4.80 ms).
+// KDA_SPLIT_SEGMENTS (1-16, read per call) overrides the count, capped at the chunk count; the
+// result is the same whatever the count (the state crosses segments in fp32).
+static int split_segments(int ncT) {
+    int s = ncT < 64 ? 1 : ncT / 32;
+    if (s > 12) s = 12;
+    if (const char* env = std::getenv("KDA_SPLIT_SEGMENTS")) {
+        const int v = std::atoi(env);
+        if (v >= 1) s = v;
+    }
+    if (s > kda::kMaxSegments) s = kda::kMaxSegments;
+    return s > ncT ? (ncT > 0 ? ncT : 1) : s;
+}
+
 int kda_fwd_algorithm(const kda_fwd_desc_t* desc, int has_cu_seqlens) {
     Path path;
     const kda_status_t st = check_fwd_desc(desc, has_cu_seqlens != 0, &path);
     if (st != KDA_OK) return -(int)st;
     return path == Path::kChunk64 ? KDA_CHUNK_64 : KDA_CHUNK_PER_TOKEN;
+}
+
+int kda_fwd_split_segments(const kda_fwd_desc_t* desc, int has_cu_seqlens) {
+    Path path;
+    const kda_status_t st = check_fwd_desc(desc, has_cu_seqlens != 0, &path);
+    if (st != KDA_OK) return -(int)st;
+    if (path != Path::kChunk64 || has_cu_seqlens || desc->T <= 0) return 1;
+    return split_segments((desc->T + 63) / 64);
 }
 
 // Packed documents on the chunked path are scheduled longest first; the permutation lives in the
@@ -149,7 +174,7 @@ static size_t order_bytes(const kda_fwd_desc_t* d, Path path) {
 
 // Workspace of the split chunked path (intra-chunk kernel + state pass), 256-byte aligned parts.
 struct SplitLayout {
-    size_t order, map, decay, wq, ke, ut, ot, total;
+    size_t order, map, counters, state, decay, wq, ke, ut, ot, total;
     long long G;
     int ncT;
     bool has_order;
@@ -168,6 +193,9 @@ static bool split_layout(const kda_fwd_desc_t* d, Path path, bool packed, SplitL
     size_t off = 0;
     L->order = off; off += L->has_order ? up256((size_t)d->num_seqs * 4) : 0;
     L->map = off;   off += packed ? up256((size_t)L->G * 4) : 0;
+    L->counters = off; off += up256((size_t)kda::kMaxSegments * 8);
+    // state between chunk segments (equal-length sequences): N x H fp32 128 x 128
+    L->state = off; off += packed ? 0 : (size_t)d->num_seqs * d->H * 65536;
     L->decay = off; off += up256((size_t)R * 512);
     L->wq = off;    off += (size_t)R * 32768;
     L->ke = off;    off += (size_t)R * 16384;
@@ -196,6 +224,43 @@ size_t kda_fwd_workspace_size_min(const kda_fwd_desc_t* desc) {
         return 0;
     t_last_error[0] = 0;
     return order_bytes(desc, path);
+}
+
+// Chunk segments of the split path for equal-length sequences with ncT chunks each: the state
+// pass of segment s (one CTA per chain, so at most N x H SMs) runs on a side stream while the
+// intra-chunk kernel works on segment s + 1 with the other SMs. Short sequences run in one.
+// Side stream (highest priority, so that its state-pass CTAs take SMs first when both kernels are
+// ready) and events, one set per host thread and device: concurrent calls from several host
+// threads never share events.
+struct SideStream {
+    cudaStream_t aux = nullptr;
+    cudaEvent_t join = nullptr;
+    cudaEvent_t seg[kda::kMaxSegments] = {};
+};
+static thread_local SideStream t_side[kMaxDevices];
+
+static cudaError_t side_stream(SideStream** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    SideStream& ss = t_side[dev];
+    if (!ss.aux) {
+        int least = 0, greatest = 0;
+        if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
+        cudaStream_t aux;
+        if ((e = cudaStreamCreateWithPriority(&aux, cudaStreamNonBlocking, greatest)) !=
+            cudaSuccess)
+            return e;
+        if ((e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess)
+            return e;
+        for (int i = 0; i < kda::kMaxSegments; ++i)
+            if ((e = cudaEventCreateWithFlags(&ss.seg[i], cudaEventDisableTiming)) != cudaSuccess)
+                return e;
+        ss.aux = aux;
+    }
+    *out = &ss;
+    return cudaSuccess;
 }
 
 // kda_fwd with an optional gated RMSNorm epilogue (norm == nullptr: none).
@@ -259,6 +324,8 @@ static kda_status_t fwd_impl(const kda_fwd_desc_t* d, const void* q, const void*
         ws.ot = reinterpret_cast<__nv_bfloat16*>(w + L.ot);
         ws.decay = reinterpret_cast<float*>(w + L.decay);
         ws.map = cu_seqlens ? reinterpret_cast<int32_t*>(w + L.map) : nullptr;
+        ws.counters = reinterpret_cast<unsigned long long*>(w + L.counters);
+        ws.state = cu_seqlens ? nullptr : reinterpret_cast<float*>(w + L.state);
         ws.G = L.G;
         ws.ncT = L.ncT;
         p.split = &ws;
@@ -272,10 +339,38 @@ static kda_status_t fwd_impl(const kda_fwd_desc_t* d, const void* q, const void*
             e = kda::launch_chunk_map(cu_seqlens, d->num_seqs, d->T, L.G, ws.map, p.err, s);
             if (e != cudaSuccess) return cuda_fail(e, "kda_fwd chunk map");
         }
-        e = kda::launch_chunk64_intra(p, s);
-        if (e != cudaSuccess) return cuda_fail(e, "kda_fwd intra-chunk launch");
-        e = kda::launch_chunk_scan(p, s);
-        if (e != cudaSuccess) return cuda_fail(e, "kda_fwd state-pass launch");
+        const int S = cu_seqlens ? 1 : split_segments(L.ncT);
+        e = cudaMemsetAsync(ws.counters, 0, sizeof(unsigned long long) * S, s);
+        if (e != cudaSuccess) return cuda_fail(e, "kda_fwd workspace counters");
+        if (S == 1) {
+            e = kda::launch_chunk64_intra(p, 0, L.ncT, ws.counters, s);
+            if (e != cudaSuccess) return cuda_fail(e, "kda_fwd intra-chunk launch");
+            e = kda::launch_chunk_scan(p, kda::ScanSegment{0, L.ncT, h0, hT}, s);
+            if (e != cudaSuccess) return cuda_fail(e, "kda_fwd state-pass launch");
+        } else {
+            // intra(0) intra(1) ... on the caller's stream; state(i) on the side stream after
+            // intra(i) and state(i - 1); the caller's stream then waits for the last state pass
+            SideStream* ss = nullptr;
+            if ((e = side_stream(&ss)) != cudaSuccess) return cuda_fail(e, "kda_fwd side stream");
+            cudaError_t first = cudaSuccess;
+            for (int i = 0; i < S && first == cudaSuccess; ++i) {
+                const int cb = (int)((long long)L.ncT * i / S);
+                const int ce = (int)((long long)L.ncT * (i + 1) / S);
+                const kda::ScanSegment seg{cb, ce, i == 0 ? h0 : ws.state,
+                                           i == S - 1 ? hT : ws.state};
+                if ((e = kda::launch_chunk64_intra(p, cb, ce - cb, ws.counters + i, s)) !=
+                        cudaSuccess ||
+                    (e = cudaEventRecord(ss->seg[i], s)) != cudaSuccess ||
+                    (e = cudaStreamWaitEvent(ss->aux, ss->seg[i], 0)) != cudaSuccess ||
+                    (e = kda::launch_chunk_scan(p, seg, ss->aux)) != cudaSuccess)
+                    first = e;
+            }
+            // join even after a failed launch, so that nothing is left pending on the side stream
+            e = cudaEventRecord(ss->join, ss->aux);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
+            if (first != cudaSuccess) return cuda_fail(first, "kda_fwd split launch");
+            if (e != cudaSuccess) return cuda_fail(e, "kda_fwd side stream join");
+        }
         e = norm_after();
         if (e != cudaSuccess) return cuda_fail(e, "kda_fwd output norm launch");
         return KDA_OK;

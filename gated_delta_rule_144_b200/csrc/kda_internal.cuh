@@ -32,8 +32,22 @@ struct SplitWorkspace {
     __nv_bfloat16* ot;   // [R * 128][64]: O~^T
     float* decay;        // [R][128]: e^{Gamma_end}
     int32_t* map;        // [G]: document of chunk record g, -1 if unused (packed only)
+    float* state;        // [N][H][128][128]: state between segments (equal-length sequences only)
+    unsigned long long* counters;   // [kMaxSegments]: record counters of the intra-chunk launches
     long long G;         // chunk records per head; R = G * H
     int ncT;
+};
+
+// The split path may run in up to this many chunk segments (equal-length sequences): the state
+// pass of segment s overlaps the intra-chunk kernel of segment s + 1.
+constexpr int kMaxSegments = 16;
+
+// One launch of the state pass: chunks [c_begin, c_end) of every chain, from the state h0 to the
+// state hT (the caller's, or the workspace's scratch state between segments; either nullable).
+struct ScanSegment {
+    int c_begin, c_end;
+    const float* h0;
+    float* hT;
 };
 
 struct FwdParams {
@@ -86,8 +100,12 @@ cudaError_t launch_chunk64(const FwdParams& p, cudaStream_t stream);
 // cu_seqlens), the intra-chunk kernel over all records, then the state pass over all chains.
 cudaError_t launch_chunk_map(const int32_t* cu_seqlens, int N, int T, long long G, int32_t* map,
                              unsigned* err, cudaStream_t stream);
-cudaError_t launch_chunk64_intra(const FwdParams& p, cudaStream_t stream);
-cudaError_t launch_chunk_scan(const FwdParams& p, cudaStream_t stream);
+// Intra-chunk kernel over the records of chunks [c_begin, c_begin + c_span) of every sequence (all
+// records for packed documents, which are not segmented); CTAs claim records from *counter,
+// which must be zero at launch.
+cudaError_t launch_chunk64_intra(const FwdParams& p, int c_begin, int c_span,
+                                 unsigned long long* counter, cudaStream_t stream);
+cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaStream_t stream);
 // y = x / sqrt(mean(x^2) + eps) * w * sigmoid(gate) per vector of dv elements (dv <= 256);
 // y may alias x.
 cudaError_t launch_out_norm_gated(const void* x, const void* gate, const float* w, float eps,

@@ -71,7 +71,8 @@ constexpr uint32_t OFF_BETA = OFF_MISC;           // f32 [64]
 constexpr uint32_t OFF_LOUP = OFF_MISC + 256;     // f32 [4 blocks][2 halves][128]
 constexpr uint32_t OFF_BAR = OFF_LOUP + 4096;     // mbarriers
 constexpr uint32_t OFF_TMEM = OFF_BAR + 64;       // TMEM base address
-constexpr uint32_t kSmemBytes = OFF_TMEM + 16 + 1024;   // + alignment slack
+constexpr uint32_t OFF_CLAIM = OFF_TMEM + 16;     // two claimed record indices (by parity)
+constexpr uint32_t kSmemBytes = OFF_CLAIM + 16 + 1024;   // + alignment slack
 static_assert(OFF_ZA + 16384 == OFF_C + 40960, "solve buffers fill the R/C region exactly");
 static_assert(OFF_YS + 4 * 16 * 17 * 4 <= OFF_TT, "solve scratch overlaps [T; T']");
 static_assert(OFF_SWQ + 32768 <= OFF_TT, "[W; Q~] staging must not touch [T; T'] (read by the "
@@ -105,6 +106,8 @@ struct IntraArgs {
     float* decay;            // [R][128]
     long long G;             // chunk records per head
     int ncT, T, H, N;
+    int c_begin, c_span;     // equal-length sequences: chunks [c_begin, c_begin + c_span) of each
+    unsigned long long* counter;   // records claimed so far by this launch (zero at launch)
     long long budget;
     int debug_stall;         // failure-injection hook: wait on a barrier nothing ever signals
     unsigned* err;
@@ -162,36 +165,45 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
     const int qd = warp & 3, hf = warp >> 2;          // TMEM lane quarter, column half
     const int H = args.H;
 
-    // this CTA's records: blockIdx.x, + gridDim.x, ... (record = g * H + head)
-    long long cursor = blockIdx.x;
-    auto next_unit = [&](Unit& u) -> bool {
-        const long long total = args.G * H;
-        while (cursor < total) {
-            const long long idx = cursor;
-            cursor += gridDim.x;
+    // Records are claimed one at a time from a counter shared by the launch's CTAs, so that a CTA
+    // that starts late (its SM busy with another kernel) takes fewer records instead of
+    // finishing last. Index idx < total names record (g, head): for packed documents g = idx / H;
+    // for equal-length sequences idx runs over (sequence, chunk in this launch's span, head).
+    const long long total = args.cu ? args.G * H : (long long)args.N * args.c_span * H;
+    auto decode = [&](long long idx, Unit& u) -> bool {
+        u.h = (int)(idx % H);
+        if (args.cu) {
             const long long g = idx / H;
-            u.h = (int)(idx % H);
             u.rec = idx;
-            if (args.cu) {
-                const int d = args.map[g];
-                if (d < 0 || d >= args.N) continue;
-                const long long a = args.cu[d], b = args.cu[d + 1];
-                if (b <= a || a < 0 || b > args.T) continue;   // reported by the map kernel
-                const long long cc = g - d - a / kC;
-                if (cc < 0 || a + kC * cc >= b) continue;
-                u.row0 = a + kC * cc;
-                u.L = (int)min((long long)kC, b - u.row0);
-            } else {
-                const long long s = g / args.ncT, cc = g % args.ncT;
-                u.row0 = s * args.T + kC * cc;
-                u.L = (int)min((long long)kC, (long long)args.T - kC * cc);
-            }
-            return true;
+            const int d = args.map[g];
+            if (d < 0 || d >= args.N) return false;
+            const long long a = args.cu[d], b = args.cu[d + 1];
+            if (b <= a || a < 0 || b > args.T) return false;   // reported by the map kernel
+            const long long cc = g - d - a / kC;
+            if (cc < 0 || a + kC * cc >= b) return false;
+            u.row0 = a + kC * cc;
+            u.L = (int)min((long long)kC, b - u.row0);
+        } else {
+            const long long per_seq = (long long)args.c_span * H;
+            const long long sq = idx / per_seq;
+            const long long cc = args.c_begin + (idx % per_seq) / H;
+            u.rec = (sq * args.ncT + cc) * H + u.h;
+            u.row0 = sq * args.T + kC * cc;
+            u.L = (int)min((long long)kC, (long long)args.T - kC * cc);
         }
-        return false;
+        return true;
     };
+    // next valid record of the launch, or -1 (called by one thread)
+    auto claim = [&]() -> long long {
+        for (;;) {
+            const long long idx = (long long)atomicAdd(args.counter, 1ull);
+            if (idx >= total) return -1;
+            Unit u;
+            if (decode(idx, u)) return idx;
+        }
+    };
+    long long* claim_s = reinterpret_cast<long long*>(sm + OFF_CLAIM);
     Unit cur;
-    bool has_cur = next_unit(cur);
 
     float* beta_s = reinterpret_cast<float*>(sm + OFF_BETA);
     float* loup_s = reinterpret_cast<float*>(sm + OFF_LOUP);
@@ -210,6 +222,7 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         fence_mbar_init();
     }
     if (tid == copier) {
+        claim_s[0] = claim();
         prefetch_tmap(&maps.q);
         prefetch_tmap(&maps.k);
         prefetch_tmap(&maps.g);
@@ -227,6 +240,7 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
     tc_fence_after();
     const uint32_t tbase = *tmem_s;
     const uint32_t lane_q = (uint32_t)(32 * qd) << 16;   // this warp's TMEM lane quarter
+    bool has_cur = claim_s[0] >= 0 && decode(claim_s[0], cur);
 
     auto issue_v = [&](const Unit& u) {
         mbar_arrive_expect_tx(bar_v, kTxV);
@@ -305,10 +319,10 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         }
         if (tid == copier) {
             issue_in(cur);
-            const long long saved = cursor;   // look one record ahead without consuming it
+            const long long nx = claim();   // the record after this one, published by parity
+            claim_s[(c + 1) & 1] = nx;
             Unit ahead;
-            if (next_unit(ahead)) prefetch_inputs(ahead);
-            cursor = saved;
+            if (nx >= 0 && decode(nx, ahead)) prefetch_inputs(ahead);
         }
         in_pending = true;
         if (tid < kC)
@@ -810,7 +824,10 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
             }
             stores_pending = true;
         }
-        has_cur = next_unit(cur);
+        {
+            const long long nx = claim_s[(c + 1) & 1];   // written at this record's start
+            has_cur = nx >= 0 && decode(nx, cur);
+        }
     }
 
     if (aborted) {
@@ -902,20 +919,22 @@ cudaError_t intra_grid_cap(int* cap) {
 
 }  // namespace
 
-cudaError_t launch_chunk64_intra(const FwdParams& p, cudaStream_t stream) {
+cudaError_t launch_chunk64_intra(const FwdParams& p, int c_begin, int c_span,
+                                 unsigned long long* counter, cudaStream_t stream) {
     const SplitWorkspace& ws = *p.split;
     cudaError_t e = tma_encoder_ready();
     if (e != cudaSuccess) return e;
     const long long rows = (long long)p.B * p.T;
-    const long long items = ws.G * p.H;
+    const long long items = p.cu_seqlens ? ws.G * p.H : (long long)p.N * c_span * p.H;
     if (items == 0 || rows <= 0) return cudaSuccess;
-    if (items * 128 > 0x7fffffffLL || rows > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    if (ws.G * p.H * 128 > 0x7fffffffLL || rows > 0x7fffffffLL)
+        return cudaErrorInvalidConfiguration;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const auto F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const auto SWN = CU_TENSOR_MAP_SWIZZLE_NONE;
     const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
     IntraMaps m;
-    const unsigned long long R = (unsigned long long)items;
+    const unsigned long long R = (unsigned long long)(ws.G * p.H);
     if ((e = make_rows_map(&m.q, p.q, BF, 2, rows, p.H, 64, SW)) != cudaSuccess ||
         (e = make_rows_map(&m.k, p.k, BF, 2, rows, p.H, 64, SW)) != cudaSuccess ||
         (e = make_rows_map(&m.g, p.log_g, F32, 4, rows, p.H, kD, SWN)) != cudaSuccess ||
@@ -939,6 +958,9 @@ cudaError_t launch_chunk64_intra(const FwdParams& p, cudaStream_t stream) {
     a.decay = ws.decay;
     a.G = ws.G;
     a.ncT = ws.ncT;
+    a.c_begin = c_begin;
+    a.c_span = c_span;
+    a.counter = counter;
     a.T = p.T;
     a.H = p.H;
     a.N = p.N;

@@ -71,8 +71,9 @@ constexpr uint32_t kTmemCols = 512;
 struct ScanArgs {
     const int32_t* order;   // nullable: document taken by the k-th (document, head) group
     const int32_t* cu;      // nullable
-    const float* h0;
-    float* hT;
+    const float* h0;        // state at chunk c_begin (nullable: zero)
+    float* hT;              // state after chunk c_end - 1 (nullable: not written)
+    int c_begin, c_end;     // chunks of every chain this launch walks
     __nv_bfloat16* o;
     const float* decay;     // [R][128]
     int T, H, N, ncT;       // ncT: chunk records per sequence when cu is null
@@ -124,11 +125,18 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         t1 = t0 + args.T;
         g0 = (long long)n * args.ncT;
     }
-    const int nchunks = (int)((t1 - t0 + kC - 1) / kC);
-    if (g0 + nchunks > args.G) {   // only a malformed cu_seqlens gets here
+    if (g0 + (t1 - t0 + kC - 1) / kC > args.G) {   // only a malformed cu_seqlens gets here
         if (tid == 0) set_device_error(args.err, DEV_BAD_SEQLENS);
         return;
     }
+    {   // this launch's segment of the chain: chunks [c_begin, c_end), possibly empty
+        const long long sb0 = min(t1, t0 + (long long)kC * args.c_begin);
+        const long long sb1 = min(t1, t0 + (long long)kC * args.c_end);
+        g0 += (sb0 - t0 + kC - 1) / kC;
+        t0 = sb0;
+        t1 = max(sb0, sb1);
+    }
+    const int nchunks = (int)((t1 - t0 + kC - 1) / kC);
 
     uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
     const uint32_t bar_full0 = sb + OFF_BAR, bar_mma1 = bar_full0 + 16, bar_mma2 = bar_full0 + 24;
@@ -426,7 +434,7 @@ int scan_debug_stall() {
 
 // One CTA (4 warps) per (sequence or document, head); packed documents are taken longest first
 // when an order is given.
-cudaError_t launch_chunk_scan(const FwdParams& p, cudaStream_t stream) {
+cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaStream_t stream) {
     const SplitWorkspace& ws = *p.split;
     const long long units = (long long)p.N * p.H;
     if (units == 0) return cudaSuccess;
@@ -459,8 +467,10 @@ cudaError_t launch_chunk_scan(const FwdParams& p, cudaStream_t stream) {
     memset(&a, 0, sizeof(a));
     a.order = p.doc_order;
     a.cu = p.cu_seqlens;
-    a.h0 = p.h0;
-    a.hT = p.hT;
+    a.h0 = seg.h0;
+    a.hT = seg.hT;
+    a.c_begin = seg.c_begin;
+    a.c_end = seg.c_end;
     a.o = static_cast<__nv_bfloat16*>(p.o);
     a.decay = ws.decay;
     a.T = p.T;

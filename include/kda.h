@@ -98,7 +98,12 @@ typedef struct {
  *             With at least kda_fwd_workspace_size(desc) bytes the chunked path runs split: an
  *             intra-chunk kernel computes every chunk's WY factors in parallel over all chunks
  *             and heads and stores them here (about 80.5 KiB per 64-token chunk and head), then a
- *             state pass walks each sequence's chunks. With less (but at least
+ *             state pass walks each sequence's chunks. For equal-length sequences of 64 chunks
+ *             or more the two run in chunk segments (up to 12; KDA_SPLIT_SEGMENTS, 1-16,
+ *             overrides): the state pass of one segment runs on an internal high-priority stream
+ *             while the intra-chunk kernel works on the next, and the caller's stream waits for
+ *             both before the call's later work; the state between segments (64 KiB per sequence
+ *             and head) is kept in the workspace. With less workspace (but at least
  *             kda_fwd_workspace_size_min(desc), which is 0 unless documents are packed) one fused
  *             kernel per (sequence, head) does both, with no intermediate storage. Both give the
  *             same result up to bf16 rounding of the stored factors. May be NULL when the minimum
@@ -161,6 +166,14 @@ kda_status_t kda_out_norm_gated(long long vectors, int dv, kda_dtype_t dtype, co
  * rejected. Host-only, no CUDA calls.
  */
 int kda_fwd_algorithm(const kda_fwd_desc_t* desc, int has_cu_seqlens);
+
+/*
+ * Number of chunk segments kda_fwd's split chunked path runs for `desc` (each one launch of the
+ * intra-chunk kernel and one of the state pass): 1 for packed documents, short sequences or the
+ * per-token path, else as described under kda_fwd's workspace. Reads KDA_SPLIT_SEGMENTS like
+ * kda_fwd does. Host-only, no CUDA calls; the negated kda_status_t for a rejected description.
+ */
+int kda_fwd_split_segments(const kda_fwd_desc_t* desc, int has_cu_seqlens);
 
 /*
  * Workspace bytes for the fastest path kda_fwd has for `desc` (the split chunked path when it

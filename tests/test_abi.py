@@ -108,13 +108,17 @@ def test_decode_rejects_on_host(L):
 
 def _split_bytes(B, T, H, N, packed):
     """Split-path workspace: per (64-token chunk record, head) 32 KiB of [W; Q~], 3 x 16 KiB of
-    K_end, U~, O~ and 512 B of decay; plus the record map and document order when packed."""
+    K_end, U~, O~ and 512 B of decay; 256 B of record counters (one per chunk segment, at most
+    16); the record map and document order when packed, else one fp32 128 x 128 state per
+    (sequence, head) carried between chunk segments."""
     up = lambda x: (x + 255) // 256 * 256
     ncT = (T + 63) // 64
     G = ncT + N if packed else B * ncT
     R = G * H
     order = up(4 * N) if packed and 2 <= N <= 2048 else 0
-    return order + (up(4 * G) if packed else 0) + up(512 * R) + R * (32768 + 3 * 16384)
+    state = 0 if packed else N * H * 128 * 128 * 4
+    return (order + (up(4 * G) if packed else 0) + up(8 * 16) + state + up(512 * R) +
+            R * (32768 + 3 * 16384))
 
 
 def test_decode_tokens_rejects_on_host(L):
@@ -169,6 +173,24 @@ def test_workspace_size_is_host_only(L):
     d = _desc(num_seqs=8, chunk_size=1)
     assert L.kda_fwd_workspace_size(ctypes.byref(d)) == 0
     assert L.kda_fwd_workspace_size_min(ctypes.byref(d)) == 0
+
+
+def test_split_segments_rule(L, monkeypatch):
+    """Equal-length sequences of 64 chunks or more run in segments of at least 32 chunks, at most
+    12; packed documents, short sequences and the per-token path in one; the environment
+    override is capped at 16 and at the chunk count."""
+    L.kda_fwd_split_segments.restype = ctypes.c_int
+    seg = lambda T, varlen=0, **kw: L.kda_fwd_split_segments(ctypes.byref(_desc(T=T, **kw)),
+                                                             varlen)
+    monkeypatch.delenv("KDA_SPLIT_SEGMENTS", raising=False)
+    assert seg(64 * 63) == 1 and seg(64 * 64) == 2 and seg(64 * 64 + 1) == 2
+    assert seg(64 * 101) == 3 and seg(65536) == 12 and seg(1 << 20) == 12
+    assert seg(65536, varlen=1, B=1, num_seqs=4) == 1
+    assert seg(65536, chunk_size=1) == 1
+    monkeypatch.setenv("KDA_SPLIT_SEGMENTS", "40")
+    assert seg(65536) == 16 and seg(64 * 3) == 3
+    monkeypatch.setenv("KDA_SPLIT_SEGMENTS", "1")
+    assert seg(65536) == 1
 
 
 def test_packed_chunked_call_without_workspace_is_rejected_on_host(L):

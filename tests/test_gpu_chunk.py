@@ -141,6 +141,29 @@ def test_long_context_full_size_sampled_heads(name, fused):
     assert worst[0] <= TOL_BF16 and worst[1] <= TOL_BF16, worst
 
 
+def test_segmented_split_path_uneven_segments():
+    """Equal-length sequences of 101 chunks (the last one partial) run the split path in three
+    chunk segments of 33, 34 and 34 chunks, the state crossing each boundary through the
+    workspace: o and hT against the oracle."""
+    _check(synth.prefill_inputs("long-t65536", B=2, T=64 * 100 + 17, H=2, h0_std=0.05, seed=23))
+
+
+def test_segment_count_does_not_change_the_result(monkeypatch):
+    """The state crosses segment boundaries in fp32 and every chunk runs the same code, so any
+    segment count gives bit-identical o and hT."""
+    inp = to(synth.prefill_inputs("long-t65536", B=1, T=64 * 70 + 5, H=3, h0_std=0.05, seed=29),
+             DEV)
+    outs = []
+    for segs in ("1", "2", "5", "8"):
+        monkeypatch.setenv("KDA_SPLIT_SEGMENTS", segs)
+        o, hT = kda.fwd(inp["q"], inp["k"], inp["v"], inp["log_g"], inp["beta"], h0=inp["h0"])
+        torch.cuda.synchronize()
+        outs.append((o.clone(), hT.clone()))
+    assert kda.get_device_error() == 0
+    for o, hT in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(hT, outs[0][1])
+
+
 def test_workspace_size_selects_the_path():
     """A workspace below kda_fwd_workspace_size (but covering the minimum) runs the fused kernel:
     bit-identical to fused=True; the full size runs the split path, which agrees within the
