@@ -403,11 +403,17 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
             // per row, with yi = 1 / y_j:
             //   lower half: rho = yi, kappa = y_j, sigma = y_j own, e^{Gamma} = F tot yi
             //   upper half: rho = y_j, kappa = yi, sigma = tot yi, e^{Gamma} = F own y_j
-            // so that sigma = kappa sf and e^{Gamma} = cE rho
+            // so that sigma = kappa sf and e^{Gamma} = cE rho; the products below are taken from
+            // k rho, q rho and k kappa: K+ = (k rho) cE, Q+ = (q rho) cE, K_end = (k kappa) sf G,
+            // cross columns (k kappa) sf X_a
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 cE[i] = hh == 0 ? F[i] * tot[i] : F[i] * own[i];
                 sf[i] = hh == 0 ? own[i] : tot[i];
+                Gf[i] *= sf[i];
+                XA[0][i] *= sf[i];
+                XA[1][i] *= sf[i];
+                XA[2][i] *= sf[i];
             }
         }
 
@@ -433,39 +439,35 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
                 const float2 q01 = unpack_bf16(qv.x), q23 = unpack_bf16(qv.y);
                 const float kk[4] = {k01.x, k01.y, k23.x, k23.y};
                 const float qq[4] = {q01.x, q01.y, q23.x, q23.y};
-                float rho[4], kap[4], sig[4], e[4], x[4];
+                float kr[4], qr[4], kc[4];   // k rho, q rho, k kappa
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const float yv = y[j][i];
                     const float yi = __fdividef(1.f, yv);
-                    rho[i] = hh == 0 ? yi : yv;
-                    kap[i] = hh == 0 ? yv : yi;
-                    sig[i] = kap[i] * sf[i];
-                    e[i] = cE[i] * rho[i];
-                    x[i] = Gf[i] * sig[i];
+                    const float rho = hh == 0 ? yi : yv;
+                    const float kap = hh == 0 ? yv : yi;
+                    kr[i] = kk[i] * rho;
+                    qr[i] = qq[i] * rho;
+                    kc[i] = kk[i] * kap;
                 }
-                st_bf16x4(sm + OFF_R + toff(128, rb8, j), kk[0] * rho[0], kk[1] * rho[1],
-                          kk[2] * rho[2], kk[3] * rho[3]);
-                st_bf16x4(sm + OFF_R + toff(128, rb8 + 8, j), qq[0] * rho[0], qq[1] * rho[1],
-                          qq[2] * rho[2], qq[3] * rho[3]);
-                st_bf16x4(sm + OFF_C + toff(160, rb8, j), kk[0] * kap[0], kk[1] * kap[1],
-                          kk[2] * kap[2], kk[3] * kap[3]);
+                st_bf16x4(sm + OFF_R + toff(128, rb8, j), kr[0], kr[1], kr[2], kr[3]);
+                st_bf16x4(sm + OFF_R + toff(128, rb8 + 8, j), qr[0], qr[1], qr[2], qr[3]);
+                st_bf16x4(sm + OFF_C + toff(160, rb8, j), kc[0], kc[1], kc[2], kc[3]);
 #pragma unroll
                 for (int a = 1; a < 4; ++a) {
                     if (a <= pb) continue;
-                    const float* xa = XA[a - 1];
+                    const float* xa = XA[a - 1];   // sf X_a
                     st_bf16x4(sm + OFF_C + toff(160, rb8 + 8 + cross_off(a) / 8, j),
-                              kk[0] * sig[0] * xa[0], kk[1] * sig[1] * xa[1],
-                              kk[2] * sig[2] * xa[2], kk[3] * sig[3] * xa[3]);
+                              kc[0] * xa[0], kc[1] * xa[1], kc[2] * xa[2], kc[3] * xa[3]);
                 }
-                st_bf16x4(sm + OFF_KP + toff(64, rb8, j), kk[0] * e[0], kk[1] * e[1],
-                          kk[2] * e[2], kk[3] * e[3]);
+                st_bf16x4(sm + OFF_KP + toff(64, rb8, j), kr[0] * cE[0], kr[1] * cE[1],
+                          kr[2] * cE[2], kr[3] * cE[3]);
                 *reinterpret_cast<uint2*>(qplus + (size_t)r * kD) =
-                    make_uint2(pack_bf16(qq[0] * e[0], qq[1] * e[1]),
-                               pack_bf16(qq[2] * e[2], qq[3] * e[3]));
-                *reinterpret_cast<uint2*>(kend + (size_t)r * kD) =
-                    make_uint2(pack_bf16(kk[0] * x[0], kk[1] * x[1]),
-                               pack_bf16(kk[2] * x[2], kk[3] * x[3]));
+                    make_uint2(pack_bf16(qr[0] * cE[0], qr[1] * cE[1]),
+                               pack_bf16(qr[2] * cE[2], qr[3] * cE[3]));
+                *reinterpret_cast<uint2*>(kend + (size_t)r * kD) =   // Gf holds sf G
+                    make_uint2(pack_bf16(kc[0] * Gf[0], kc[1] * Gf[1]),
+                               pack_bf16(kc[2] * Gf[2], kc[3] * Gf[3]));
             }
             // the reciprocals stay finite while every factor they invert is >= 1e-30; the running
             // products only shrink, so the first suffix (lower half) or the last prefix (upper
