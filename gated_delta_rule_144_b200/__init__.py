@@ -76,6 +76,10 @@ def lib():
     L.kda_fwd_normed.restype = i32
     L.kda_out_norm_gated.argtypes = [ctypes.c_longlong, i32, i32, p, p, p, ctypes.c_float, p, p]
     L.kda_out_norm_gated.restype = i32
+    L.kda_bwd.argtypes = [ctypes.POINTER(FwdDesc)] + [p] * 16 + [ctypes.c_size_t, p]
+    L.kda_bwd.restype = i32
+    L.kda_bwd_workspace_size.argtypes = [ctypes.POINTER(FwdDesc)]
+    L.kda_bwd_workspace_size.restype = ctypes.c_size_t
     L.kda_fwd_no_alloc.argtypes = [ctypes.POINTER(FwdDesc), p, p, p, p, p, p, p, p, p, p]
     L.kda_fwd_no_alloc.restype = i32
     L.kda_fwd_algorithm.argtypes = [ctypes.POINTER(FwdDesc), i32]
@@ -257,6 +261,64 @@ def fwd(q, k, v, log_g, beta, h0=None, cu_seqlens=None, *, chunk_size: int = CHU
                            _ptr(workspace), ws_bytes, _stream(stream, dev))
     _check(st, "kda_fwd")
     return o, hT
+
+
+def bwd_workspace_size(B, T, H, dk, dv, num_seqs, dtype=torch.bfloat16) -> int:
+    d = FwdDesc(B, T, H, dk, dv, num_seqs, KDA_BF16 if dtype == torch.bfloat16 else KDA_F32, 0)
+    return int(lib().kda_bwd_workspace_size(ctypes.byref(d)))
+
+
+def bwd(q, k, v, log_g, beta, do, h0=None, dhT=None, cu_seqlens=None, *, workspace=None,
+        stream=None):
+    """Gradients of the recurrence (``kda_bwd``) for upstream gradients do (of o) and dhT (of
+    the final states, or None): returns (dq, dk, dv, dlog_g, dbeta, dh0), all fp32, shaped like
+    (q, k, v, log_g, beta, h0 [N, H, dk, dv]). Forward arguments as for ``fwd``; dk = dv = 128."""
+    lib()
+    _dev(q, "q")
+    dev = q.device
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, dk]")
+    B, T, H, dk = q.shape
+    dt = q.dtype
+    _dtype_code(q)
+    _dev(k, "k", dt, (B, T, H, dk), dev)
+    _dev(log_g, "log_g", torch.float32, (B, T, H, dk), dev)
+    _dev(v, "v", dt, None, dev)
+    if v.dim() != 4 or tuple(v.shape[:3]) != (B, T, H):
+        raise ValueError("v must be [B, T, H, dv]")
+    dv = v.shape[3]
+    _dev(beta, "beta", dt, (B, T, H), dev)
+    _dev(do, "do", dt, (B, T, H, dv), dev)
+    if cu_seqlens is not None:
+        _dev(cu_seqlens, "cu_seqlens", torch.int32, None, dev)
+        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+            raise ValueError("cu_seqlens must be a 1-D int32 tensor of N + 1 offsets")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    _dev(h0, "h0", torch.float32, (N, H, dk, dv), dev)
+    _dev(dhT, "dhT", torch.float32, (N, H, dk, dv), dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    grads = (torch.empty((B, T, H, dk), **f32), torch.empty((B, T, H, dk), **f32),
+             torch.empty((B, T, H, dv), **f32), torch.empty((B, T, H, dk), **f32),
+             torch.empty((B, T, H), **f32), torch.empty((N, H, dk, dv), **f32))
+    desc = FwdDesc(B, T, H, dk, dv, N, _dtype_code(q), 0)
+    need = int(lib().kda_bwd_workspace_size(ctypes.byref(desc)))
+    if workspace is None:
+        if need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    else:
+        _dev(workspace, "workspace", torch.uint8, None, dev)
+        if workspace.numel() < need:
+            raise ValueError("workspace needs at least %d bytes" % need)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    with torch.cuda.device(dev):
+        st = lib().kda_bwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(log_g),
+                           _ptr(beta), _ptr(h0), _ptr(cu_seqlens), _ptr(do), _ptr(dhT),
+                           *[_ptr(g) for g in grads], _ptr(workspace), ws_bytes,
+                           _stream(stream, dev))
+    _check(st, "kda_bwd")
+    return grads
 
 
 def out_norm_gated(x, gate, weight, eps: float, *, y=None, stream=None):

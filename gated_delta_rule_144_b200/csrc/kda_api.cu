@@ -413,6 +413,69 @@ kda_status_t kda_fwd_normed(const kda_fwd_desc_t* d, const void* q, const void* 
                     norm, stream);
 }
 
+static kda_status_t check_bwd_desc(const kda_fwd_desc_t* d, bool has_cu) {
+    Path path;
+    kda_status_t st = check_fwd_desc(d, has_cu, &path);
+    if (st != KDA_OK) return st;
+    if (d->dk != 128 || d->dv != 128)
+        return fail(KDA_ERR_UNSUPPORTED, "kda_bwd supports dk = dv = 128 (got %d, %d)", d->dk,
+                    d->dv);
+    return KDA_OK;
+}
+
+size_t kda_bwd_workspace_size(const kda_fwd_desc_t* desc) {
+    if (!desc || check_bwd_desc(desc, desc->B == 1 && desc->num_seqs >= 2) != KDA_OK) return 0;
+    t_last_error[0] = 0;
+    if (desc->T <= 0 || desc->num_seqs <= 0) return 0;
+    return kda::bwd_workspace_bytes((long long)desc->num_seqs * desc->H, desc->T);
+}
+
+kda_status_t kda_bwd(const kda_fwd_desc_t* d, const void* q, const void* k, const void* v,
+                     const float* log_g, const void* beta, const float* h0,
+                     const int32_t* cu_seqlens, const void* dout, const float* dhT, float* dq,
+                     float* dk, float* dv, float* dlog_g, float* dbeta, float* dh0,
+                     void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+    t_last_error[0] = 0;
+    kda_status_t st = check_bwd_desc(d, cu_seqlens != nullptr);
+    if (st != KDA_OK) return st;
+    const bool tokens = (int64_t)d->B * d->T > 0;
+    if ((st = check_ptr(q, "q", tokens)) || (st = check_ptr(k, "k", tokens)) ||
+        (st = check_ptr(v, "v", tokens)) || (st = check_ptr(log_g, "log_g", tokens)) ||
+        (st = check_ptr(beta, "beta", false)) || (st = check_ptr(dout, "do", tokens)) ||
+        (st = check_ptr(dq, "dq", tokens)) || (st = check_ptr(dk, "dk", tokens)) ||
+        (st = check_ptr(dv, "dv", tokens)) || (st = check_ptr(dlog_g, "dlog_g", tokens)) ||
+        (st = check_ptr(dbeta, "dbeta", false)) || (st = check_ptr(h0, "h0", false)) ||
+        (st = check_ptr(dhT, "dhT", false)) || (st = check_ptr(dh0, "dh0", false)) ||
+        (st = check_ptr(cu_seqlens, "cu_seqlens", false)))
+        return st;
+    if (tokens && (!beta || !dbeta)) return fail(KDA_ERR_INVALID_ARG, "beta or dbeta is NULL");
+    const long long chains = (long long)d->num_seqs * d->H;
+    const size_t need = (tokens && chains > 0) ? kda::bwd_workspace_bytes(chains, d->T) : 0;
+    if (need > 0 && (!workspace || !aligned16(workspace) || workspace_bytes < need))
+        return fail(KDA_ERR_INVALID_ARG,
+                    "workspace must be a 16-byte aligned device buffer of %zu bytes "
+                    "(kda_bwd_workspace_size)", need);
+    if (chains == 0) return KDA_OK;
+    if (!tokens) {   // no tokens: dh0 = dhT (or zero)
+        if (!dh0) return KDA_OK;
+        cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+        const size_t bytes = (size_t)chains * 128 * 128 * sizeof(float);
+        cudaError_t e = dhT ? cudaMemcpyAsync(dh0, dhT, bytes, cudaMemcpyDeviceToDevice, s)
+                            : cudaMemsetAsync(dh0, 0, bytes, s);
+        return e == cudaSuccess ? KDA_OK : cuda_fail(e, "kda_bwd dh0");
+    }
+    kda::BwdParams p{};
+    p.q = q; p.k = k; p.v = v; p.beta = beta; p.dout = dout; p.log_g = log_g; p.h0 = h0;
+    p.dhT = dhT; p.cu_seqlens = cu_seqlens; p.dq = dq; p.dk = dk; p.dv = dv; p.dlog_g = dlog_g;
+    p.dbeta = dbeta; p.dh0 = dh0; p.workspace = workspace;
+    p.T = d->T; p.H = d->H; p.N = d->num_seqs;
+    p.bf16 = d->dtype == KDA_BF16;
+    if ((st = device_error_word(&p.err)) != KDA_OK) return st;
+    cudaError_t e = kda::launch_bwd(p, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kda_bwd launch");
+    return KDA_OK;
+}
+
 kda_status_t kda_out_norm_gated(long long vectors, int dv, kda_dtype_t dtype, const void* x,
                                 const void* gate, const float* weight, float eps, void* y,
                                 kda_stream_t stream) {

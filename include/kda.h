@@ -152,6 +152,36 @@ kda_status_t kda_fwd_normed(const kda_fwd_desc_t* desc, const void* q, const voi
                             size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * kda_bwd - gradients of the recurrence, for training (NeMo glm5_next layers, `_torch_recurrent_kda`
+ * is a differentiable reference KDA; this is the derivative of kda_fwd's recurrence). For
+ * upstream gradients do (of o) and dhT (of the final states), computes the gradients of
+ * L = sum <do, o> + <dhT, hT>:
+ *   dq, dk    : [B, T, H, dk] float32      dv       : [B, T, H, dv] float32
+ *   dlog_g    : [B, T, H, dk] float32      dbeta    : [B, T, H] float32
+ *   dh0       : [N, H, dk, dv] float32, or NULL to skip.
+ * The forward arguments (desc, q, k, v, log_g, beta, h0, cu_seqlens) are as for kda_fwd; do has
+ * the layout and dtype of o; dhT is [N, H, dk, dv] float32 or NULL (zero). dk = dv = 128
+ * (KDA_ERR_UNSUPPORTED otherwise); desc->chunk_size is ignored. Every gradient is computed in
+ * fp32 from the exact per-token recurrence; one CTA per (sequence or document, head) runs the
+ * forward storing the state every 64 tokens, then walks each 64-token chunk backwards after
+ * re-running its forward. The workspace (kda_bwd_workspace_size bytes, 16-byte aligned, device)
+ * holds those states. Host-checkable errors return before any launch; a malformed cu_seqlens is
+ * reported through kda_get_device_error.
+ */
+kda_status_t kda_bwd(const kda_fwd_desc_t* desc, const void* q, const void* k, const void* v,
+                     const float* log_g, const void* beta, const float* h0,
+                     const int32_t* cu_seqlens, const void* dout, const float* dhT, float* dq,
+                     float* dk, float* dv, float* dlog_g, float* dbeta, float* dh0,
+                     void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * Workspace bytes kda_bwd needs for `desc`: per (sequence or document, head), one 64 KiB state
+ * per 64 tokens of T plus one, one 64-token chunk of states and its read-outs. Host-only; 0 for
+ * a rejected description or no tokens.
+ */
+size_t kda_bwd_workspace_size(const kda_fwd_desc_t* desc);
+
+/*
  * kda_out_norm_gated - the gated RMSNorm on its own: `vectors` vectors of dv elements (for o of
  * shape [B, T, H, dv], vectors = B * T * H), x and gate in dtype, y in dtype (y may equal x).
  * dv <= 256. Host-checkable errors return before any launch.

@@ -193,6 +193,33 @@ def test_split_segments_rule(L, monkeypatch):
     assert seg(65536) == 1
 
 
+def test_bwd_workspace_size_and_host_rejections(L):
+    """kda_bwd: per (sequence or document, head) one 64 KiB state per 64 tokens plus one, a
+    64-token chunk of states and 64 x 2 x 128 fp32 read-outs; dk = dv = 128 only; missing
+    pointers and a short workspace are rejected before any launch."""
+    L.kda_bwd_workspace_size.restype = ctypes.c_size_t
+    for kw in (dict(B=2, T=150, H=2, num_seqs=2), dict(B=1, T=200, H=2, num_seqs=3),
+               dict(B=1, T=64, H=1, num_seqs=1)):
+        d = _desc(**kw)
+        chains = kw["num_seqs"] * kw["H"]
+        nck = (kw["T"] + 63) // 64 + 1
+        want = chains * ((nck + 64) * 128 * 128 + 64 * 2 * 128) * 4
+        assert L.kda_bwd_workspace_size(ctypes.byref(d)) == want, kw
+    assert L.kda_bwd_workspace_size(ctypes.byref(_desc(dk=64))) == 0
+    P = ctypes.c_void_p
+    F = P(FAKE)
+
+    def bwd(desc, dout=F, ws=F, ws_bytes=1 << 40):
+        return L.kda_bwd(ctypes.byref(desc), F, F, F, F, F, None, None, dout, None, F, F, F, F,
+                         F, None, ws, ctypes.c_size_t(ws_bytes), None)
+    assert bwd(_desc(dk=64)) == 2
+    assert bwd(_desc(dv=64)) == 2
+    assert bwd(_desc(), dout=None) == 1 and b"do" in L.kda_last_error()
+    assert bwd(_desc(), ws=None) == 1 and b"workspace" in L.kda_last_error()
+    assert bwd(_desc(), ws_bytes=1024) == 1
+    assert bwd(_desc(), dout=P(FAKE + 4)) == 1   # misaligned
+
+
 def test_packed_chunked_call_without_workspace_is_rejected_on_host(L):
     P = ctypes.c_void_p
     d = _desc(num_seqs=8)
