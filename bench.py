@@ -481,6 +481,40 @@ def run_secondary(kda, synth, args, dev, stream, world, rank):
                                     "ms_normed_call": res["normed"],
                                     "ms_plain_then_norm": res["separate"],
                                     "ms_plain": out["packed_prefill"]["ms_per_step"]}
+    # gradients (kda_bwd) on the T=4096, H=16 workload: upstream do and dhT drawn once
+    b = synth.prefill_inputs("prefill-t4096", device=dev, seed=shard.rank_seed(1001, rank))
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(shard.rank_seed(1095, rank))
+    bdo = torch.randn(b["v"].shape, generator=gen, device=dev).to(b["v"].dtype)
+    bdh = torch.randn((b["N"], b["H"], 128, 128), generator=gen, device=dev)
+    bws = torch.empty(kda.bwd_workspace_size(b["B"], b["T"], b["H"], 128, 128, b["N"],
+                                             b["q"].dtype), dtype=torch.uint8, device=dev)
+
+    def bstep():
+        kda.bwd(b["q"], b["k"], b["v"], b["log_g"], b["beta"], bdo, h0=b["h0"], dhT=bdh,
+                workspace=bws)
+
+    bsteps = max(1, min(args.steps, 5))
+    for _ in range(3):
+        bstep()
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms, _ = time_launches(bstep, bsteps, stream)
+    barrier(world)
+    ms = max_over_ranks(total_ms, world, dev) / bsteps
+    th = b["B"] * b["T"] * b["H"]
+    # algorithmic bytes: q, k, v, do (dtype) and log g, beta read; dq, dk, dv, dlog_g (fp32) and
+    # dbeta written; h0, dhT read and dh0 written per chain
+    esz = b["q"].element_size()
+    states = (2 + (b["h0"] is not None)) * b["N"] * b["H"] * STATE_BYTES
+    by = th * (4 * 128 * esz + 128 * 4 + esz + 4 * 128 * 4 + 4) + states
+    out["bwd"] = {"workload": "prefill-t4096", "B": b["B"], "T": b["T"], "H": b["H"],
+                  "ms_per_step": round(ms, 4),
+                  "tokens/s": round(b["B"] * b["T"] * world / (ms / 1e3), 1),
+                  "bytes_per_step": by,
+                  "roofline_frac": round(by / (ms / 1e3) / 1e9 / hbm_peak, 5),
+                  "kernel": "kda_bwd (fp32 CUDA cores, one CTA per chain)"}
+    del b, bdo, bdh, bws
     if kda.get_device_error() != 0:
         raise RuntimeError("device error in the secondary runs")
     return out

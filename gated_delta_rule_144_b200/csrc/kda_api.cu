@@ -9,6 +9,7 @@
 
 #include "kda.h"
 
+#include "kda_bwd.cuh"
 #include "kda_internal.cuh"
 
 namespace {

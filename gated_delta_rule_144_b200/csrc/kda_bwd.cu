@@ -24,7 +24,7 @@
 
 #include <cstdint>
 
-#include "kda_internal.cuh"
+#include "kda_bwd.cuh"
 
 namespace kda {
 namespace {
