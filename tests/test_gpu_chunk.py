@@ -197,10 +197,11 @@ def test_steep_decay_is_reported_as_range_error():
 
 
 def test_expired_wait_reports_timeout_and_context_survives():
-    """Failure injection: with KDA_DEBUG_STALL_WAIT set, every CTA waits (bounded by a 2M-cycle
-    budget, about a millisecond) on a barrier that nothing signals while its first copy is in
-    flight. The kernel must report KDA_ERR_TIMEOUT, drain its own copy, free TMEM and return;
-    the context must stay usable. Runs in a child process: the hooks are read once per process."""
+    """Failure injection: with KDA_DEBUG_STALL_WAIT set, every CTA of the split path's two
+    kernels waits (bounded by a 2M-cycle budget, about a millisecond) on a barrier that nothing
+    signals; the state pass has its first record copies in flight at that point. Each kernel
+    must report KDA_ERR_TIMEOUT, drain its own copies, free TMEM and return; the context must
+    stay usable. Runs in a child process: the hooks are read once per process."""
     code = (
         "import torch, gated_delta_rule_144_b200 as kda\n"
         "from gated_delta_rule_144_b200 import synth\n"
