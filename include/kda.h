@@ -23,8 +23,11 @@
  * Conventions for every entry point
  *   - All tensors are dense, contiguous, row-major, in DEVICE memory unless stated otherwise, and
  *     every base pointer must be 16-byte aligned.
- *   - The caller owns all memory. The library allocates nothing, keeps no per-call state and is
- *     safe to call from several host threads on different streams.
+ *   - The caller owns all memory. The library allocates no device memory, keeps no per-call
+ *     state and is safe to call from several host threads on different streams. The one thing it
+ *     creates: on the first segmented split-path kda_fwd call (see kda_fwd) from a host thread on
+ *     a device, one internal stream and 17 events for that thread and device, kept for the
+ *     thread's lifetime.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default stream).
  *   - Problems visible on the host (null or misaligned pointers, bad sizes, unsupported
  *     combinations) return an error before anything is launched. Problems only the device can
