@@ -8,10 +8,10 @@
 // Glm5NextTextLinearAttention; NeMo AutoModel glm5_next layers page, `_torch_recurrent_kda`):
 // for every (sequence, head) the state S is a dk x dv matrix, and for each token t in order
 //
-//     S      <- diag(g_t) S            (the snippet's `state * g_i`: decay along the key axis)
-//     m      <- k_t^T S                (the snippet's `(state * k_i[..., None]).sum(-2)`)
-//     delta  <- beta_t (v_t - m)       (the snippet's `(v_i - kv_mem) * b_i`)
-//     S      <- S + k_t delta^T        (the snippet's `k_i.unsqueeze(-1) * delta.unsqueeze(-2)`)
+//     S      <- diag(g_t) S            (the snippet scales the state by the gate, key axis)
+//     m      <- k_t^T S                (the snippet reads the state through k, summing keys)
+//     delta  <- beta_t (v_t - m)       (the snippet's error term: value minus read, times beta)
+//     S      <- S + k_t delta^T        (the snippet's rank-one write of k and delta)
 //     o_t    <- S^T q_t                (read-out after the write, no 1/sqrt(dk) scale)
 //
 // with g_t = exp(log_g_t) per key channel. Packed variable-length input (cu_seqlens) restarts
