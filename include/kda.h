@@ -13,10 +13,10 @@
  *     o_t    = S^T q_t                     (read-out after the write; no 1/sqrt(dk) scale)
  *
  * Packed variable-length input restarts the state at every document boundary (NeMo AutoModel
- * glm5_next layers page: `_torch_recurrent_kda(q, k, v, g, beta, cu_seqlens)` "packed
- * boundaries reset the recurrent state"; `Glm5NextLinearAttention.forward` runs KDA "without
- * crossing documents"). The gate arrives in log space as float32, as returned by
- * `Glm5NextKDAFp32Params.forward` ("log-decay gates [batch, sequence, heads, head_dim]").
+ * glm5_next layers page: the docstring of `_torch_recurrent_kda(q, k, v, g, beta, cu_seqlens)`
+ * says the state resets at packed boundaries, and `Glm5NextLinearAttention.forward` keeps KDA
+ * within each document). The gate arrives in log space as float32: `Glm5NextKDAFp32Params.forward`
+ * returns log-decay gates shaped [batch, sequence, heads, head_dim].
  * Decode advances a per-sequence state by one token (metrale glm5next_layer page: KDA decode
  * takes a KdaSeqState).
  *

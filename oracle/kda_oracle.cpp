@@ -15,8 +15,8 @@
 //     o_t    <- S^T q_t                (read-out after the write, no 1/sqrt(dk) scale)
 //
 // with g_t = exp(log_g_t) per key channel. Packed variable-length input (cu_seqlens) restarts
-// the state at every document boundary ("packed boundaries reset the recurrent state", NeMo
-// `_torch_recurrent_kda`). The state starts from h0 (or zero) and the final state of each
+// the state at every document boundary (the NeMo `_torch_recurrent_kda` docstring: the state
+// resets at packed boundaries). The state starts from h0 (or zero) and the final state of each
 // sequence or document is returned.
 //
 // All arithmetic is float64; exp is std::exp. Inputs arrive as float32 arrays that hold exactly
