@@ -341,6 +341,24 @@ def out_norm_gated(x, gate, weight, eps: float, *, y=None, stream=None):
     return y
 
 
+def _prefill_shapes(q, k, v, log_g, beta, cu_seqlens):
+    """(B, T, H, dk, dv, N) of a prefill call; raises ValueError on inconsistent shapes."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, dk]")
+    B, T, H, dk = q.shape
+    if tuple(k.shape) != (B, T, H, dk) or tuple(log_g.shape) != (B, T, H, dk):
+        raise ValueError("k and log_g must be shaped like q, [B, T, H, dk]")
+    if v.dim() != 4 or tuple(v.shape[:3]) != (B, T, H):
+        raise ValueError("v must be [B, T, H, dv]")
+    if tuple(beta.shape) != (B, T, H):
+        raise ValueError("beta must be [B, T, H]")
+    if cu_seqlens is None:
+        return B, T, H, dk, v.shape[3], B
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor of N + 1 offsets")
+    return B, T, H, dk, v.shape[3], cu_seqlens.numel() - 1
+
+
 def fwd_no_alloc(q, k, v, log_g, beta, h0, cu_seqlens, o, hT, *, chunk_size: int = CHUNK_AUTO,
                  stream=None):
     """``kda_fwd_no_alloc``: the prefill without a workspace, for callers that cannot allocate.
@@ -351,21 +369,26 @@ def fwd_no_alloc(q, k, v, log_g, beta, h0, cu_seqlens, o, hT, *, chunk_size: int
     Same layouts as ``fwd``; the same results as ``fwd(..., fused=True)``.
     """
     lib()
+    # shapes first (no device needed): the library reads v, o and hT with the sizes taken from q
+    B, T, H, dk, dv, N = _prefill_shapes(q, k, v, log_g, beta, cu_seqlens)
+    for t, name, shape in ((h0, "h0", (N, H, dk, dv)), (o, "o", (B, T, H, dv)),
+                           (hT, "hT", (N, H, dk, dv))):
+        if t is not None and tuple(t.shape) != shape:
+            raise ValueError("%s must have shape %s, got %s" % (name, shape, tuple(t.shape)))
+    if o is None:
+        raise ValueError("o must be passed in (this entry point allocates nothing)")
     _dev(q, "q")
     dev = q.device
-    B, T, H, dk = q.shape
     dt = q.dtype
-    _dev(k, "k", dt, (B, T, H, dk), dev)
-    _dev(log_g, "log_g", torch.float32, (B, T, H, dk), dev)
+    _dtype_code(q)
+    _dev(k, "k", dt, None, dev)
+    _dev(log_g, "log_g", torch.float32, None, dev)
     _dev(v, "v", dt, None, dev)
-    dv = v.shape[3]
-    _dev(beta, "beta", dt, (B, T, H), dev)
-    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
-    if cu_seqlens is not None:
-        _dev(cu_seqlens, "cu_seqlens", torch.int32, None, dev)
-    _dev(h0, "h0", torch.float32, (N, H, dk, dv), dev)
-    _dev(o, "o", dt, (B, T, H, dv), dev)
-    _dev(hT, "hT", torch.float32, (N, H, dk, dv), dev)
+    _dev(beta, "beta", dt, None, dev)
+    _dev(cu_seqlens, "cu_seqlens", torch.int32, None, dev)
+    _dev(h0, "h0", torch.float32, None, dev)
+    _dev(o, "o", dt, None, dev)
+    _dev(hT, "hT", torch.float32, None, dev)
     desc = FwdDesc(B, T, H, dk, dv, N, _dtype_code(q), chunk_size)
     with torch.cuda.device(dev):
         st = lib().kda_fwd_no_alloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(log_g),

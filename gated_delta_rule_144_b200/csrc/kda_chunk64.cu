@@ -1029,14 +1029,12 @@ long long wait_budget() {
 
 template <int DV>
 cudaError_t set_smem_attr() {
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(chunk64_kernel<DV>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)Layout<DV>::kSmemBytes);
+    static PerDevice attr;
+    return attr.run([](int) {
+        return cudaFuncSetAttribute(chunk64_kernel<DV>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)Layout<DV>::kSmemBytes);
     });
-    return attr_err;
 }
 
 template <int DV>
@@ -1068,15 +1066,20 @@ cudaError_t launch_width(const FwdParams& p, cudaStream_t stream, const CUtensor
     return cudaGetLastError();
 }
 
+// SMs of the current device (148 on B200), queried once per device.
 int sm_count() {
-    static int n = [] {
-        int dev = 0, v = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return 148;
-        return v;
-    }();
-    return n;
+    static PerDevice once;
+    static int count[PerDevice::kMax];
+    int dev = 0;
+    const cudaError_t e = once.run(
+        [](int d) {
+            int v = 0;
+            const cudaError_t r = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, d);
+            count[d] = (r == cudaSuccess && v > 0) ? v : 148;
+            return cudaSuccess;
+        },
+        &dev);
+    return e == cudaSuccess ? count[dev] : 148;
 }
 
 }  // namespace

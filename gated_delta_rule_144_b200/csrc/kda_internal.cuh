@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace kda {
 
 // Codes the kernels store into the sticky device error word (same values as kda_status_t).
@@ -114,6 +116,34 @@ cudaError_t launch_out_norm_gated(const void* x, const void* gate, const float* 
 bool chunk64_available();
 // Value columns one chunked-kernel CTA owns for N sequences x H heads (64 or 128).
 int chunk64_value_width(int N, int H);
+
+// One-time set-up per device (kernel attributes, occupancy queries): `fn(device)` runs once for
+// each device index, with that device current, and its status is kept for later calls. Kernel
+// attributes such as the dynamic shared-memory limit belong to a device's context, so a process
+// that launches on several devices needs them set on each.
+class PerDevice {
+  public:
+    static constexpr int kMax = 64;
+    template <class F>
+    cudaError_t run(F&& fn, int* dev_out = nullptr) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= kMax) return cudaErrorInvalidDevice;
+        if (dev_out) *dev_out = dev;
+        std::lock_guard<std::mutex> lock(mu_);
+        if (!done_[dev]) {
+            err_[dev] = fn(dev);
+            done_[dev] = true;
+        }
+        return err_[dev];
+    }
+
+  private:
+    std::mutex mu_;
+    bool done_[kMax] = {};
+    cudaError_t err_[kMax] = {};
+};
 
 // Element loads shared by the CUDA-core kernels.
 __device__ __forceinline__ float load_elem(const float* p, int64_t i) { return p[i]; }

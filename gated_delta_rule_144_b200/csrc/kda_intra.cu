@@ -883,39 +883,41 @@ int debug_stall() {
 // whichever is larger. A CTA beyond the resident count would only start later, never wait on
 // another, so an overestimate costs time, not correctness.
 cudaError_t intra_grid_cap(int* cap) {
-    static std::once_flag once;
-    static cudaError_t err = cudaSuccess;
-    static int value = 0;
-    std::call_once(once, [] {
-        err = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)kSmemBytes);
-        if (err != cudaSuccess) return;
-        err = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                   (int)cudaSharedmemCarveoutMaxShared);
-        if (err != cudaSuccess) return;
-        int dev = 0, sms = 0, smem_sm = 0, smem_rsv = 0, regs_sm = 0, per_sm = 0;
-        cudaFuncAttributes fa;
-        if ((err = cudaGetDevice(&dev)) != cudaSuccess ||
-            (err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) !=
-                cudaSuccess ||
-            (err = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor,
-                                          dev)) != cudaSuccess ||
-            (err = cudaDeviceGetAttribute(&smem_rsv, cudaDevAttrReservedSharedMemoryPerBlock,
-                                          dev)) != cudaSuccess ||
-            (err = cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor,
-                                          dev)) != cudaSuccess ||
-            (err = cudaFuncGetAttributes(&fa, intra_kernel)) != cudaSuccess ||
-            (err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, intra_kernel, kThreads,
-                                                                 kSmemBytes)) != cudaSuccess)
-            return;
-        const int by_smem = smem_sm / ((int)kSmemBytes + fa.sharedSizeBytes + smem_rsv);
-        const int by_regs = fa.numRegs > 0 ? regs_sm / (fa.numRegs * kThreads) : 1;
-        int fit = by_smem < by_regs ? by_smem : by_regs;
-        if (fit > 2) fit = 2;   // __launch_bounds__ sizes the kernel for two
-        if (per_sm < fit) per_sm = fit;
-        value = sms * (per_sm > 0 ? per_sm : 1);
-    });
-    *cap = value;
+    static PerDevice once;
+    static int value[PerDevice::kMax];
+    int dev = 0;
+    const cudaError_t err = once.run(
+        [](int d) {
+            cudaError_t e = cudaFuncSetAttribute(
+                intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+            if (e != cudaSuccess) return e;
+            e = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared);
+            if (e != cudaSuccess) return e;
+            int sms = 0, smem_sm = 0, smem_rsv = 0, regs_sm = 0, per_sm = 0;
+            cudaFuncAttributes fa;
+            if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, d)) !=
+                    cudaSuccess ||
+                (e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor,
+                                            d)) != cudaSuccess ||
+                (e = cudaDeviceGetAttribute(&smem_rsv, cudaDevAttrReservedSharedMemoryPerBlock,
+                                            d)) != cudaSuccess ||
+                (e = cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor,
+                                            d)) != cudaSuccess ||
+                (e = cudaFuncGetAttributes(&fa, intra_kernel)) != cudaSuccess ||
+                (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, intra_kernel, kThreads,
+                                                                   kSmemBytes)) != cudaSuccess)
+                return e;
+            const int by_smem = smem_sm / ((int)kSmemBytes + fa.sharedSizeBytes + smem_rsv);
+            const int by_regs = fa.numRegs > 0 ? regs_sm / (fa.numRegs * kThreads) : 1;
+            int fit = by_smem < by_regs ? by_smem : by_regs;
+            if (fit > 2) fit = 2;   // __launch_bounds__ sizes the kernel for two
+            if (per_sm < fit) per_sm = fit;
+            value[d] = sms * (per_sm > 0 ? per_sm : 1);
+            return cudaSuccess;
+        },
+        &dev);
+    *cap = err == cudaSuccess ? value[dev] : 0;
     return err;
 }
 

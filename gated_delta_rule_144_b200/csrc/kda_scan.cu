@@ -455,12 +455,10 @@ cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaSt
         (e = make_map_3d_rows(&m.o, p.o, BF, 2, (unsigned long long)p.B * p.T, p.H, kD, kC)) !=
             cudaSuccess)
         return e;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(chunk_scan_kernel,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)kSmemBytes);
+    static PerDevice attr;
+    const cudaError_t attr_err = attr.run([](int) {
+        return cudaFuncSetAttribute(chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kSmemBytes);
     });
     if (attr_err != cudaSuccess) return attr_err;
     ScanArgs a;

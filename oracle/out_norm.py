@@ -13,7 +13,7 @@ Passages it follows:
 
 Reading (the formula is not printed): per (token, head), rms = sqrt(mean over head_dim of x^2 +
 eps) and y = x / rms * w * sigmoid(gate), with w of head_dim entries shared by all heads and
-gate of the same shape as x. Pinned in tests/test_oracle_pins.py.
+gate of the same shape as x. Pinned in tests/test_oracle_out_norm.py.
 """
 
 from __future__ import annotations

@@ -246,3 +246,28 @@ def test_python_binding_refuses_cpu_tensors():
         kda.fwd(q, q, q, q, torch.zeros(1, 4, 1))
     with pytest.raises(ValueError, match="CUDA tensor"):
         kda.decode_step(q[0], q[0], q[0], q[0], torch.zeros(4, 1), torch.zeros(4, 1, 8, 8))
+
+
+def test_no_alloc_binding_checks_shapes_before_any_launch():
+    """fwd_no_alloc reads v, o and hT with the sizes taken from q: a v shorter in T or H, an o or
+    hT of the wrong shape, or a malformed cu_seqlens must raise before the library is called."""
+    import torch
+    B, T, H, d = 1, 8, 2, 16
+    q = torch.zeros(B, T, H, d, dtype=torch.bfloat16)
+    g = torch.zeros(B, T, H, d)
+    beta = torch.zeros(B, T, H, dtype=torch.bfloat16)
+    o = torch.zeros(B, T, H, d, dtype=torch.bfloat16)
+    hT = torch.zeros(B, H, d, d)
+    short_t = torch.zeros(B, T - 1, H, d, dtype=torch.bfloat16)
+    short_h = torch.zeros(B, T, H - 1, d, dtype=torch.bfloat16)
+    for v in (short_t, short_h, torch.zeros(T, H, d, dtype=torch.bfloat16)):
+        with pytest.raises(ValueError, match="v must be"):
+            kda.fwd_no_alloc(q, q, v, g, beta, None, None, o, hT)
+    with pytest.raises(ValueError, match="q must be"):
+        kda.fwd_no_alloc(q[0], q, q, g, beta, None, None, o, hT)
+    with pytest.raises(ValueError, match="o must have shape"):
+        kda.fwd_no_alloc(q, q, q, g, beta, None, None, o[:, :4], hT)
+    with pytest.raises(ValueError, match="hT must have shape"):
+        kda.fwd_no_alloc(q, q, q, g, beta, None, None, o, hT[:, :1])
+    with pytest.raises(ValueError, match="cu_seqlens"):
+        kda.fwd_no_alloc(q, q, q, g, beta, None, torch.zeros((2, 2), dtype=torch.int32), o, None)

@@ -118,27 +118,51 @@ def test_chunked_equals_per_token_path():
     assert rel_l2(host(h1), host(h2)) <= TOL_BF16
 
 
-@PATHS
 @pytest.mark.parametrize("name", ["long-t65536", "long-t65536-slow"])
-def test_long_context_full_size_sampled_heads(name, fused):
-    """B=2, T=65536, H=32 with h0: the GPU runs the whole batch; the oracle recomputes four
-    (sequence, head) chains end to end (every token's output and the final state)."""
+def test_long_context_full_size_every_chain(name):
+    """B=2, T=65536, H=32 with h0, at full size on both chunked paths: every one of the 64
+    (sequence, head) chains is recomputed by the oracle end to end (every token's output and the
+    final state) and compared element by element. The bound holds per chain, which is stricter
+    than the relative L2 over the whole tensor (reported too). The oracle runs eight heads of one
+    sequence at a time to bound host memory."""
     inp = synth.prefill_inputs(name, device=DEV)
-    o, hT, st = _run(inp, fused=fused)
-    assert st == 0
-    picks = [(0, 0), (0, 31), (1, 7), (1, 20)]
+    outs = {}
+    for fused in (False, True):
+        o, hT, st = _run(inp, fused=fused)
+        assert st == 0, "device error %d" % st
+        outs["fused" if fused else "split"] = (o, hT)
     f = lambda t: t.float().cpu().numpy()
-    worst = (0.0, 0.0)
-    for n, h in picks:
-        sl = lambda t: f(t[n:n + 1, :, h:h + 1])
-        o_ref, h_ref = oracle.kda_fwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]),
-                                      sl(inp["log_g"]), f(inp["beta"][n:n + 1, :, h:h + 1]),
-                                      h0=f(inp["h0"][n:n + 1, h:h + 1]))
-        eo = rel_l2(f(o[n:n + 1, :, h:h + 1]), o_ref)
-        eh = rel_l2(f(hT[n:n + 1, h:h + 1]), h_ref)
-        worst = (max(worst[0], eo), max(worst[1], eh))
-    print("worst rel-L2 o %.3e hT %.3e" % worst)
-    assert worst[0] <= TOL_BF16 and worst[1] <= TOL_BF16, worst
+    B, T, H = inp["q"].shape[:3]
+    worst = {p: (0.0, 0.0, None) for p in outs}
+    sq = {p: [0.0, 0.0] for p in outs}   # squared error over the whole tensor, per path
+    ref_sq = [0.0, 0.0]
+    group = 8
+    for n in range(B):
+        for h0_ in range(0, H, group):
+            hs = slice(h0_, h0_ + group)
+            o_ref, h_ref = oracle.kda_fwd(f(inp["q"][n:n + 1, :, hs]), f(inp["k"][n:n + 1, :, hs]),
+                                          f(inp["v"][n:n + 1, :, hs]),
+                                          f(inp["log_g"][n:n + 1, :, hs]),
+                                          f(inp["beta"][n:n + 1, :, hs]),
+                                          h0=f(inp["h0"][n:n + 1, hs]))
+            ref_sq[0] += float(np.sum(o_ref ** 2))
+            ref_sq[1] += float(np.sum(h_ref ** 2))
+            for path, (o, hT) in outs.items():
+                og = f(o[n:n + 1, :, hs]).astype(np.float64)
+                hg = f(hT[n:n + 1, hs]).astype(np.float64)
+                sq[path][0] += float(np.sum((og - o_ref) ** 2))
+                sq[path][1] += float(np.sum((hg - h_ref) ** 2))
+                for j in range(group):
+                    eo = rel_l2(og[:, :, j], o_ref[:, :, j])
+                    eh = rel_l2(hg[:, j], h_ref[:, j])
+                    w = worst[path]
+                    worst[path] = (max(w[0], eo), max(w[1], eh),
+                                   (n, h0_ + j) if eo > w[0] else w[2])
+    for path in outs:
+        whole = (np.sqrt(sq[path][0] / ref_sq[0]), np.sqrt(sq[path][1] / ref_sq[1]))
+        print("%s %s: worst chain rel-L2 o %.3e (chain %s) hT %.3e; whole tensor o %.3e hT %.3e"
+              % (name, path, worst[path][0], worst[path][2], worst[path][1], *whole))
+        assert worst[path][0] <= TOL_BF16 and worst[path][1] <= TOL_BF16, (path, worst[path])
 
 
 def test_segmented_split_path_uneven_segments():
