@@ -130,7 +130,7 @@ const char* kda_status_string(kda_status_t s) {
         case KDA_ERR_CUDA: return "CUDA runtime error";
         case KDA_ERR_TIMEOUT: return "device pipeline wait timed out";
         case KDA_ERR_BAD_SEQLENS: return "malformed cu_seqlens";
-        case KDA_ERR_RANGE: return "decay too steep for the chunked path";
+        case KDA_ERR_RANGE: return "decay out of range (reserved; no longer raised)";
     }
     return "unknown status";
 }

@@ -119,6 +119,7 @@ struct ChunkArgs {
     int T, H, N;
     long long budget;
     int debug_stall;   // failure-injection hook: wait on a barrier nothing ever signals
+    int force_direct;  // test hook: every chunk takes the steep-decay (direct) path
     unsigned* err;
 };
 
@@ -150,6 +151,151 @@ struct Unit {
     int L;            // valid rows
     long long row0;   // first token row
 };
+
+// Steep-decay path of one chunk (all 256 threads; called in place of the R and C operands, the
+// R C^T product, the K+ pass and the assembly when some product of 8 consecutive decays falls
+// below 1e-30, where the anchored factors would leave the float32 range). Gamma is formed in log
+// space, A_kk and A_qk are summed directly as sum_c k_rc k_ic e^{Gamma_rc - Gamma_ic} (exponent
+// <= 0 for i <= r), and K+, Q+, K_end come from e^{Gamma} and e^{Gamma_end - Gamma} (both <= 1):
+// nothing overflows, and factors below the float range become zero, as their true values are
+// negligible. On return (after a CTA barrier, q, k and log g consumed) L = diag(beta) A_kk,
+// [0; A_qk], K+, Q+ and K_end are in their buffers exactly as the fast path leaves them. Not
+// inlined, so that its registers do not weigh on the fast path.
+template <int DV>
+__device__ __noinline__ void steep_chunk(uint8_t* sm, int L) {
+    using Lay = Layout<DV>;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int pb = warp >> 1, hh = warp & 1;
+    const int ch0 = 4 * lane;
+    const int rbase = 16 * pb + 8 * hh;
+    const int rb8 = 2 * pb + hh;
+    const uint32_t lh4 = (uint32_t)(((lane & 15) >> 1) << 4);
+    const uint32_t lo8 = (uint32_t)((lane & 1) * 8);
+    auto toff = [&](int R, int rb, int j) -> uint32_t {
+        return (uint32_t)((lane >> 4) * R * 128 + rb * 1024 + j * 128) + (lh4 ^ (uint32_t)(j << 4)) +
+               lo8;
+    };
+    const uint8_t* qs = sm + Lay::OFF_Q;   // q, k: [64][128] bf16 row-major
+    const uint8_t* ks = sm + Lay::OFF_K;
+    float* gsw = reinterpret_cast<float*>(sm + Lay::OFF_G);    // log g -> Gamma, in place
+    float* hsum = reinterpret_cast<float*>(sm + Lay::OFF_C);   // [8 half blocks][128]
+    const float* beta_s = reinterpret_cast<const float*>(sm + Lay::OFF_BETA);
+    float cg[8][4];
+    {
+        float run[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 x = *reinterpret_cast<const float4*>(gsw + (rbase + j) * kD + ch0);
+            const bool ok = rbase + j < L;   // rows past the document do not decay
+            run[0] += ok ? x.x : 0.f;
+            run[1] += ok ? x.y : 0.f;
+            run[2] += ok ? x.z : 0.f;
+            run[3] += ok ? x.w : 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) cg[j][i] = run[i];
+        }
+        *reinterpret_cast<float4*>(hsum + rb8 * kD + ch0) =
+            make_float4(run[0], run[1], run[2], run[3]);
+    }
+    __syncthreads();
+    float gend[4] = {0.f, 0.f, 0.f, 0.f}, goff[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int hb = 0; hb < 8; ++hb) {
+        const float4 x = *reinterpret_cast<const float4*>(hsum + hb * kD + ch0);
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            gend[i] += xs[i];
+            if (hb < rb8) goff[i] += xs[i];
+        }
+    }
+    // this thread's Gamma rows back into the tile; its K+, Q+ and K_end elements
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int r = rbase + j;
+        const bool ok = r < L;
+        float G4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) G4[i] = goff[i] + cg[j][i];
+        *reinterpret_cast<float4*>(gsw + r * kD + ch0) = make_float4(G4[0], G4[1], G4[2], G4[3]);
+        float4 k4 = ld_bf16x4(ks + (r * kD + ch0) * 2);
+        float4 q4 = ld_bf16x4(qs + (r * kD + ch0) * 2);
+        if (!ok) k4 = q4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        float e[4], eb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            e[i] = __expf(G4[i]);
+            eb[i] = __expf(gend[i] - G4[i]);
+        }
+        const uint32_t o64 = toff(64, rb8, j);
+        st_bf16x4(sm + Lay::OFF_KPV + o64, k4.x * e[0], k4.y * e[1], k4.z * e[2], k4.w * e[3]);
+        st_bf16x4(sm + Lay::OFF_WQ + toff(128, rb8 + 8, j), q4.x * e[0], q4.y * e[1],
+                  q4.z * e[2], q4.w * e[3]);
+        st_bf16x4(sm + Lay::OFF_KE + o64, k4.x * eb[0], k4.y * eb[1], k4.z * eb[2], k4.w * eb[3]);
+    }
+    __syncthreads();
+    // A_kk, A_qk: thread (R4, I4) sums the 4 x 4 block of rows 4 R4.., columns 4 I4.. over the
+    // key channels (each thread starts at its own channel offset, so that the Gamma loads of a
+    // warp spread over the banks); rows past the document read as k = q = 0
+    const int R4 = tid >> 4, I4 = tid & 15;
+    float akk[4][4], aqk[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) akk[a][b] = aqk[a][b] = 0.f;
+    if (I4 <= R4) {
+        float mr[4], mi[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            mr[a] = 4 * R4 + a < L ? 1.f : 0.f;
+            mi[a] = 4 * I4 + a < L ? 1.f : 0.f;
+        }
+#pragma unroll 1
+        for (int cc = 0; cc < kD; ++cc) {
+            const int c = (cc + 2 * I4) & (kD - 1);
+            float Gr[4], Gi[4], kr[4], qr[4], ki[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int r = 4 * R4 + a, i = 4 * I4 + a;
+                Gr[a] = gsw[r * kD + c];
+                Gi[a] = gsw[i * kD + c];
+                kr[a] = mr[a] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                                    ks + (r * kD + c) * 2));
+                qr[a] = mr[a] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                                    qs + (r * kD + c) * 2));
+                ki[a] = mi[a] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                                    ks + (i * kD + c) * 2));
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const float e = __expf(fminf(Gr[a] - Gi[b], 0.f)) * ki[b];
+                    akk[a][b] = fmaf(kr[a], e, akk[a][b]);
+                    aqk[a][b] = fmaf(qr[a], e, aqk[a][b]);
+                }
+        }
+    }
+    // L = diag(beta) A_kk (i < r) and [0; A_qk] (A_qk, i <= r, in rows 64 + r; zeros above the
+    // diagonal and in rows 0-63); the R/C region holds neither q, k nor log g in this kernel
+    float* Lb = reinterpret_cast<float*>(sm + Lay::OFF_LB);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const int r = 4 * R4 + a;
+        const float br = beta_s[r];
+        float x[4], y[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            x[b] = 4 * I4 + b < r ? br * akk[a][b] : 0.f;
+            y[b] = 4 * I4 + b <= r ? aqk[a][b] : 0.f;
+        }
+        *reinterpret_cast<float4*>(Lb + r * kLdl + 4 * I4) = make_float4(x[0], x[1], x[2], x[3]);
+        st_bf16x4(sm + Lay::OFF_ZA + sw128_off(128, 64 + r, 4 * I4), y[0], y[1], y[2], y[3]);
+        *reinterpret_cast<uint2*>(sm + Lay::OFF_ZA + sw128_off(128, r, 4 * I4)) = make_uint2(0u, 0u);
+    }
+    fence_proxy_async();
+    __syncthreads();   // q, k and log g of this chunk fully consumed
+}
 
 // One CTA per (sequence or document, head, value slice) walks its chunks in order and carries the
 // state in TMEM.
@@ -368,7 +514,13 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             *reinterpret_cast<float4*>(loup_s + (pb * 2 + hh) * kD + ch0) =
                 make_float4(pre[7][0], pre[7][1], pre[7][2], pre[7][3]);
         }
-        __syncthreads();
+        // The anchored factors below invert these running products; they stay finite while
+        // every product is >= 1e-30. The products only shrink, so the last prefix (upper half)
+        // or the first suffix (lower half) is the smallest. A chunk with a steeper decay
+        // anywhere takes the direct path (steep_chunk) instead.
+#pragma unroll
+        for (int i = 0; i < 4; ++i) range_bad |= (hh == 0 ? suf[0][i] : pre[7][i]) < 1e-30f;
+        const bool steep = __syncthreads_or(range_bad || args.force_direct) != 0;
         // half totals of every block: Lo_b (rows 0-7), Up_b (rows 8-15), P_b = Lo_b Up_b.
         // F = prod_{b < pb} P_b, G = prod_{b > pb} P_b; XA[a] = Lo_a prod_{pb < b < a} P_b is the
         // factor that carries a column of this block to the middle of a later block a.
@@ -411,6 +563,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             b4_pending = false;
         }
 
+        if (!steep) {
         // ---------------------------------------------------------------- R and C operands
         //   rho_r = e^{Gamma_r - Gamma_m}, kappa_r = e^{Gamma_m - Gamma_r} (m: block middle)
         //   sigma_r = e^{Gamma_end(b) - Gamma_r}, cross columns k sigma X_a, X_a <= 1
@@ -450,12 +603,6 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                           kk[3] * sig[3] * xa[3]);
             }
         }
-        // the reciprocals above stay finite while every factor they invert is >= 1e-30; the
-        // running products only shrink, so the last prefix (upper half) or the first suffix
-        // (lower half) is the smallest
-#pragma unroll
-        for (int i = 0; i < 4; ++i) range_bad |= (hh == 0 ? suf[0][i] : pre[7][i]) < 1e-30f;
-        if (range_bad) set_device_error(args.err, DEV_RANGE);
         //   K+ = k e^{Gamma}, Q+ = q e^{Gamma}, K_end = k e^{Gamma_end - Gamma}
         auto kplus_pass = [&]() {
 #pragma unroll
@@ -504,11 +651,15 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         kplus_pass();
         fence_proxy_async();
         __syncthreads();   // q, k, log g of chunk c fully consumed
+        } else {
+            steep_chunk<DV>(sm, L);   // ends with a barrier: q, k, log g of chunk c consumed
+        }
         if (has_nxt) {
             if (tid == copier) issue_in(nxt);
             in_pending = true;
             in_chunk = c + 1;
         }
+        if (!steep) {
 
         // ---------------------------------------------------------------- assemble A_kk, A_qk
         if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
@@ -581,6 +732,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 tmem_ld_wait();
                 if (a == 3) put16(32, w);
             }
+        }
         }
         fence_proxy_async();
         tc_fence_before();
@@ -1015,6 +1167,16 @@ int debug_stall() {
     return v;
 }
 
+// KDA_DEBUG_FORCE_DIRECT=1 (read once per process): every chunk takes the steep-decay path, so
+// that tests can check that path against the oracle on ordinary inputs.
+int force_direct() {
+    static int v = [] {
+        const char* s = std::getenv("KDA_DEBUG_FORCE_DIRECT");
+        return (s && *s && *s != '0') ? 1 : 0;
+    }();
+    return v;
+}
+
 long long wait_budget() {
     static long long budget = [] {
         const char* s = std::getenv("KDA_DEBUG_WAIT_CYCLES");
@@ -1059,6 +1221,7 @@ cudaError_t launch_width(const FwdParams& p, cudaStream_t stream, const CUtensor
     a.N = p.N;
     a.budget = wait_budget();
     a.debug_stall = debug_stall();
+    a.force_direct = force_direct();
     a.err = p.err;
     const long long grid = (long long)units * Lay::kSplit;
     if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;

@@ -14,7 +14,7 @@ enum DeviceError : unsigned {
     DEV_OK = 0,
     DEV_TIMEOUT = 4,
     DEV_BAD_SEQLENS = 5,
-    DEV_RANGE = 6,
+    DEV_RANGE = 6,   // reserved: steep decays take the chunked kernels' direct path instead
 };
 
 // The first error sticks; later ones are dropped.

@@ -67,6 +67,9 @@ constexpr uint32_t OFF_SWQ = OFF_R;          // [W; Q~] [128][128] (2 panels x 1
 constexpr uint32_t OFF_SUT = OFF_R + 32768;  // U~^T [128 value columns][64 tokens]
 constexpr uint32_t OFF_SOT = OFF_R + 49152;  // O~^T [128][64]
 constexpr uint32_t OFF_MISC = OFF_C + 40960;
+// (steep-decay path only: half-block sums at OFF_C and K+ staged at OFF_C + 4096, both below
+// OFF_ZA, which that path writes at the same time)
+static_assert(OFF_C + 4096 + 16384 <= OFF_ZA, "steep-path scratch overlaps [0; A_qk]");
 constexpr uint32_t OFF_BETA = OFF_MISC;           // f32 [64]
 constexpr uint32_t OFF_LOUP = OFF_MISC + 256;     // f32 [4 blocks][2 halves][128]
 constexpr uint32_t OFF_BAR = OFF_LOUP + 4096;     // mbarriers
@@ -110,6 +113,7 @@ struct IntraArgs {
     unsigned long long* counter;   // records claimed so far by this launch (zero at launch)
     long long budget;
     int debug_stall;         // failure-injection hook: wait on a barrier nothing ever signals
+    int force_direct;        // test hook: every record takes the steep-decay (direct) path
     unsigned* err;
 };
 
@@ -153,6 +157,173 @@ __device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int c0, int c1
 // accesses (TMA stores) issued after a barrier.
 __device__ __forceinline__ void fence_proxy_async_all() {
     asm volatile("fence.proxy.async;" ::: "memory");
+}
+
+// Steep-decay path of one record (all 256 threads; called in place of the operand pass, the
+// R C^T product and the assembly when some product of 8 consecutive decays falls below 1e-30).
+// On entry: k, q (bf16) in R's rows, log g (f32) in its tile, beta in shared memory. On return
+// (after a CTA barrier): L = diag(beta) A_kk, [0; A_qk] and K+ in their buffers, Q+ and K_end in
+// the workspace, exactly as the fast path leaves them. Not inlined, so that its registers do not
+// weigh on the fast path.
+__device__ __noinline__ void steep_chunk(uint8_t* sm, int L, long long rec, __nv_bfloat16* wq,
+                                         __nv_bfloat16* ke) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int pb = warp >> 1, hh = warp & 1;
+    const int ch0 = 4 * lane;
+    const int rbase = 16 * pb + 8 * hh;
+    const int rb8 = 2 * pb + hh;
+    const uint32_t lh4 = (uint32_t)(((lane & 15) >> 1) << 4);
+    const uint32_t lo8 = (uint32_t)((lane & 1) * 8);
+    auto toff = [&](int R, int rb, int j) -> uint32_t {
+        return (uint32_t)((lane >> 4) * R * 128 + rb * 1024 + j * 128) + (lh4 ^ (uint32_t)(j << 4)) +
+               lo8;
+    };
+    const float* gs = reinterpret_cast<const float*>(sm + OFF_G);
+    const float* beta_s = reinterpret_cast<const float*>(sm + OFF_BETA);
+    // A chunk whose decay over some 8 rows exceeds the anchored factors' range. Gamma is
+    // formed in log space, A_kk and A_qk are summed directly as
+    //   sum_c k_rc k_ic e^{Gamma_rc - Gamma_ic}   (exponent <= 0 for i <= r),
+    // and K+, Q+, K_end from e^{Gamma} and e^{Gamma_end - Gamma} (both <= 1), so nothing
+    // overflows; factors below the float range become zero, as their true values are
+    // negligible. The buffers then look as after the fast path's assembly, and the UT
+    // transform and the WY products run unchanged.
+    float* gsw = reinterpret_cast<float*>(sm + OFF_G);     // log g -> Gamma, in place
+    float* hsum = reinterpret_cast<float*>(sm + OFF_C);    // [8 half blocks][128]
+    float cg[8][4];
+    {
+        float run[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 x = *reinterpret_cast<const float4*>(gs + (rbase + j) * kD + ch0);
+            const bool ok = rbase + j < L;   // rows past the document do not decay
+            run[0] += ok ? x.x : 0.f;
+            run[1] += ok ? x.y : 0.f;
+            run[2] += ok ? x.z : 0.f;
+            run[3] += ok ? x.w : 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) cg[j][i] = run[i];
+        }
+        *reinterpret_cast<float4*>(hsum + rb8 * kD + ch0) =
+            make_float4(run[0], run[1], run[2], run[3]);
+    }
+    __syncthreads();
+    float gend[4] = {0.f, 0.f, 0.f, 0.f}, goff[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int hb = 0; hb < 8; ++hb) {
+        const float4 x = *reinterpret_cast<const float4*>(hsum + hb * kD + ch0);
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            gend[i] += xs[i];
+            if (hb < rb8) goff[i] += xs[i];
+        }
+    }
+    // this thread's Gamma rows back into the tile; its K+, Q+ and K_end elements (K+
+    // staged in the free part of C until the log g tile under K+'s tile is read)
+    uint8_t* kp_stage = sm + OFF_C + 4096;
+    {
+        __nv_bfloat16* qplus = wq + ((size_t)rec * 128 + 64) * kD + ch0;
+        __nv_bfloat16* kend = ke + (size_t)rec * kC * kD + ch0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int r = rbase + j;
+            const bool ok = r < L;
+            float G4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) G4[i] = goff[i] + cg[j][i];
+            *reinterpret_cast<float4*>(gsw + r * kD + ch0) =
+                make_float4(G4[0], G4[1], G4[2], G4[3]);
+            const uint2 kv = ok ? *reinterpret_cast<const uint2*>(sm + OFF_R + toff(128, rb8, j))
+                                : make_uint2(0u, 0u);
+            const uint2 qv = ok ? *reinterpret_cast<const uint2*>(sm + OFF_R + toff(128, rb8 + 8, j))
+                                : make_uint2(0u, 0u);
+            const float2 k01 = unpack_bf16(kv.x), k23 = unpack_bf16(kv.y);
+            const float2 q01 = unpack_bf16(qv.x), q23 = unpack_bf16(qv.y);
+            const float kk[4] = {k01.x, k01.y, k23.x, k23.y};
+            const float qq[4] = {q01.x, q01.y, q23.x, q23.y};
+            float e[4], eb[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                e[i] = __expf(G4[i]);
+                eb[i] = __expf(gend[i] - G4[i]);
+            }
+            *reinterpret_cast<uint2*>(kp_stage + toff(64, rb8, j)) =
+                make_uint2(pack_bf16(kk[0] * e[0], kk[1] * e[1]),
+                           pack_bf16(kk[2] * e[2], kk[3] * e[3]));
+            *reinterpret_cast<uint2*>(qplus + (size_t)r * kD) =
+                make_uint2(pack_bf16(qq[0] * e[0], qq[1] * e[1]),
+                           pack_bf16(qq[2] * e[2], qq[3] * e[3]));
+            *reinterpret_cast<uint2*>(kend + (size_t)r * kD) =
+                make_uint2(pack_bf16(kk[0] * eb[0], kk[1] * eb[1]),
+                           pack_bf16(kk[2] * eb[2], kk[3] * eb[3]));
+        }
+    }
+    __syncthreads();
+    // A_kk, A_qk: thread (R4, I4) sums the 4 x 4 block of rows 4 R4.., columns 4 I4..
+    // over the key channels (each thread starts at its own channel offset, so that the
+    // Gamma and k loads of a warp spread over the banks)
+    const int R4 = tid >> 4, I4 = tid & 15;
+    float akk[4][4], aqk[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) akk[a][b] = aqk[a][b] = 0.f;
+    if (I4 <= R4) {
+#pragma unroll 1
+        for (int cc = 0; cc < kD; ++cc) {
+            const int c = (cc + 2 * I4) & (kD - 1);
+            float Gr[4], Gi[4], kr[4], qr[4], ki[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int r = 4 * R4 + a, i = 4 * I4 + a;
+                Gr[a] = gsw[r * kD + c];
+                Gi[a] = gsw[i * kD + c];
+                kr[a] = __bfloat162float(
+                    *reinterpret_cast<const __nv_bfloat16*>(sm + OFF_R + sw128_off(128, r, c)));
+                qr[a] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                    sm + OFF_R + sw128_off(128, 64 + r, c)));
+                ki[a] = __bfloat162float(
+                    *reinterpret_cast<const __nv_bfloat16*>(sm + OFF_R + sw128_off(128, i, c)));
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const float e = __expf(fminf(Gr[a] - Gi[b], 0.f)) * ki[b];
+                    akk[a][b] = fmaf(kr[a], e, akk[a][b]);
+                    aqk[a][b] = fmaf(qr[a], e, aqk[a][b]);
+                }
+        }
+    }
+    // [0; A_qk]: A_qk (i <= r) in rows 64 + r, zeros above the diagonal and in rows 0-63
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const int r = 4 * R4 + a;
+        float x[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) x[b] = 4 * I4 + b <= r ? aqk[a][b] : 0.f;
+        st_bf16x4(sm + OFF_ZA + sw128_off(128, 64 + r, 4 * I4), x[0], x[1], x[2], x[3]);
+        *reinterpret_cast<uint2*>(sm + OFF_ZA + sw128_off(128, r, 4 * I4)) =
+            make_uint2(0u, 0u);
+    }
+    __syncthreads();   // k, q and Gamma fully read: R and the log g tile may be reused
+    {
+        float* Lb = reinterpret_cast<float*>(sm + OFF_LB);
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const int r = 4 * R4 + a;
+            const float br = beta_s[r];
+            float x[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) x[b] = 4 * I4 + b < r ? br * akk[a][b] : 0.f;
+            *reinterpret_cast<float4*>(Lb + r * kLdl + 4 * I4) =
+                make_float4(x[0], x[1], x[2], x[3]);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint2*>(sm + OFF_KP + toff(64, rb8, j)) =
+                *reinterpret_cast<const uint2*>(kp_stage + toff(64, rb8, j));
+    }
 }
 
 __global__ void __launch_bounds__(kThreads, 2)
@@ -362,9 +533,19 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         }
         *reinterpret_cast<float4*>(loup_s + (pb * 2 + hh) * kD + ch0) =
             make_float4(tot[0], tot[1], tot[2], tot[3]);
-        __syncthreads();   // log g consumed: the K+ / V region is free for V and K+
-        if (tid == copier) issue_v(cur);
-        v_pending = true;
+        // The anchored factors invert these running products; they stay finite while every
+        // product is >= 1e-30. The products only shrink, so the first suffix (lower half) or the
+        // last prefix (upper half) is the smallest. A chunk with a steeper decay anywhere takes
+        // the direct path below instead.
+        bool range_bad = false;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) range_bad |= (hh == 0 ? y[0][i] : y[7][i]) < 1e-30f;
+        const bool steep = __syncthreads_or(range_bad || args.force_direct) != 0;
+        // log g consumed (unless steep): the K+ / V region is free for V and K+
+        if (!steep) {
+            if (tid == copier) issue_v(cur);
+            v_pending = true;
+        }
         // half totals of every block: Lo_b (rows 0-7), Up_b (rows 8-15), P_b = Lo_b Up_b.
         // F = prod_{b < pb} P_b, G = prod_{b > pb} P_b; XA[a] = Lo_a prod_{pb < b < a} P_b carries
         // a column of this block to the middle of a later block a; own = Up_pb (lower half) or
@@ -422,8 +603,7 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         //   C: k kappa (kappa = e^{Gamma_m - Gamma_r}), cross columns k sigma X_a, X_a <= 1
         //   K+ = k e^{Gamma} (shared), Q+ = q e^{Gamma} (parked in the Q~ slot),
         //   K_end = k e^{Gamma_end - Gamma} = k G sigma (workspace)
-        {
-            bool range_bad = false;
+        if (!steep) {
             __nv_bfloat16* qplus = args.wq + ((size_t)rec * 128 + 64) * kD + ch0;
             __nv_bfloat16* kend = args.ke + (size_t)rec * kC * kD + ch0;
 #pragma unroll
@@ -469,13 +649,8 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
                     make_uint2(pack_bf16(kc[0] * Gf[0], kc[1] * Gf[1]),
                                pack_bf16(kc[2] * Gf[2], kc[3] * Gf[3]));
             }
-            // the reciprocals stay finite while every factor they invert is >= 1e-30; the running
-            // products only shrink, so the first suffix (lower half) or the last prefix (upper
-            // half) is the smallest
-#pragma unroll
-            for (int i = 0; i < 4; ++i) range_bad |= (hh == 0 ? y[0][i] : y[7][i]) < 1e-30f;
-            if (range_bad) set_device_error(args.err, DEV_RANGE);
         }
+        if (!steep) {
         fence_proxy_async();
         __syncthreads();
 
@@ -567,6 +742,12 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
                 tmem_ld_wait();
                 if (a == 3) put16(32, w);
             }
+        }
+        } else {
+            // ------------------------------------------------------------ steep decay: direct
+            steep_chunk(sm, L, rec, args.wq, args.ke);
+            if (tid == copier) issue_v(cur);
+            v_pending = true;
         }
         fence_proxy_async();
         tc_fence_before();
@@ -878,6 +1059,16 @@ int debug_stall() {
     return v;
 }
 
+// KDA_DEBUG_FORCE_DIRECT=1 (read once per process): every chunk takes the steep-decay path, so
+// that tests can check that path against the oracle on ordinary inputs.
+int force_direct() {
+    static int v = [] {
+        const char* s = std::getenv("KDA_DEBUG_FORCE_DIRECT");
+        return (s && *s && *s != '0') ? 1 : 0;
+    }();
+    return v;
+}
+
 // resident CTAs of intra_kernel across the GPU: as many per SM as its registers and shared
 // memory allow (two on B200), by the SM's own limits and by the runtime's occupancy query,
 // whichever is larger. A CTA beyond the resident count would only start later, never wait on
@@ -970,6 +1161,7 @@ cudaError_t launch_chunk64_intra(const FwdParams& p, int c_begin, int c_span,
     a.N = p.N;
     a.budget = wait_budget();
     a.debug_stall = debug_stall();
+    a.force_direct = force_direct();
     a.err = p.err;
     const long long grid = items < cap ? items : cap;
     intra_kernel<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(m, a);

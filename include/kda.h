@@ -54,7 +54,7 @@ typedef enum {
     KDA_ERR_CUDA = 3,         /* a CUDA runtime call failed; kda_last_error() has the text     */
     KDA_ERR_TIMEOUT = 4,      /* device: a bounded pipeline wait expired (kernel gave up)      */
     KDA_ERR_BAD_SEQLENS = 5,  /* device: cu_seqlens not non-decreasing from 0 to T             */
-    KDA_ERR_RANGE = 6         /* device: decay too steep for the chunked path (see kda_fwd)    */
+    KDA_ERR_RANGE = 6         /* reserved: no longer raised (steep decays take a direct path)  */
 } kda_status_t;
 
 typedef enum {
@@ -113,11 +113,11 @@ typedef struct {
  *             is 0.
  *
  * The chunked path (KDA_CHUNK_64) computes in bf16 tensor-core products with fp32 accumulation
- * and an fp32 state. Its within-chunk factorisation needs the summed decay of any 8 consecutive
- * tokens inside a 16-token sub-chunk to stay above about -69 nats per key channel (e.g.
- * log_g >= -8 everywhere); otherwise a factor would leave the float32 range. The kernel detects
- * that case (a decay product below 1e-30), records KDA_ERR_RANGE in the device error word and
- * still finishes; the per-token path (KDA_CHUNK_PER_TOKEN) has no such limit.
+ * and an fp32 state. Its fast within-chunk factorisation holds while the summed decay of any 8
+ * consecutive tokens inside a 16-token sub-chunk stays above about -69 nats per key channel;
+ * a chunk with a steeper decay (a decay product below 1e-30) is evaluated directly instead
+ * (cumulative log decay, A_kk and A_qk summed with one exponential per term), at a few times the
+ * cost of a fast chunk. Any finite log_g <= 0 is therefore accepted on every path.
  * Returns KDA_OK once the work is enqueued. T = 0 or N = 0 is a valid no-op (hT = h0 or 0).
  */
 kda_status_t kda_fwd(const kda_fwd_desc_t* desc, const void* q, const void* k, const void* v,
@@ -290,7 +290,7 @@ kda_status_t kda_decode_tokens(int N, int H, int T, int dk, int dv, kda_dtype_t 
 
 /*
  * kda_get_device_error - synchronise `stream`, then return and clear the sticky device error
- * word (KDA_OK, KDA_ERR_BAD_SEQLENS, KDA_ERR_TIMEOUT or KDA_ERR_RANGE), or KDA_ERR_CUDA if
+ * word (KDA_OK, KDA_ERR_BAD_SEQLENS or KDA_ERR_TIMEOUT), or KDA_ERR_CUDA if
  * the synchronisation itself failed. The word is per device and shared by all streams.
  */
 kda_status_t kda_get_device_error(kda_stream_t stream);

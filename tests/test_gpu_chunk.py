@@ -207,17 +207,64 @@ def test_workspace_size_selects_the_path():
     assert rel_l2(host(o3), host(o2)) <= TOL_BF16 and rel_l2(host(h3), host(h2)) <= TOL_BF16
 
 
-def test_steep_decay_is_reported_as_range_error():
-    """log g = -30 per token leaves the chunk factorisation's float32 range: KDA_ERR_RANGE."""
-    inp = synth.prefill_inputs("prefill-t4096", T=64, H=1, seed=16)
+@PATHS
+def test_steep_decay_everywhere(fused):
+    """log g = -30 per token: every chunk's decay over 8 rows leaves the anchored factors' float32
+    range, so every chunk takes the direct path; o and hT against the oracle."""
+    inp = synth.prefill_inputs("prefill-t4096", B=2, T=200, H=2, h0_std=0.05, seed=16)
     inp["log_g"] = torch.full_like(inp["log_g"], -30.0)
-    _, _, st = _run(inp)
-    assert st == 6
-    # the per-token path has no such limit
-    o, hT, st = _run(inp, chunk_size=1)
-    assert st == 0
-    o_ref, h_ref = oracle_fwd(inp)
-    assert rel_l2(host(o), o_ref) <= TOL_BF16
+    _check(inp, fused=fused)
+
+
+@PATHS
+def test_steep_and_gentle_chunks_in_one_chain(fused):
+    """Ordinary gates with a few steep rows (log g from -40 to -200 in scattered rows and
+    channels): the chunks that hold them take the direct path, the others the anchored factors,
+    within one chain and one launch; packed documents, one of them ending inside a steep chunk."""
+    inp = synth.prefill_inputs("packed-8docs", lengths=[64 * 5 + 17, 70, 300], H=3, h0_std=0.05,
+                               seed=26)
+    g = torch.Generator().manual_seed(27)
+    lg = inp["log_g"]
+    T = lg.shape[1]
+    rows = torch.randint(0, T, (12,), generator=g)
+    for r in rows.tolist():
+        ch = torch.randint(0, 128, (8,), generator=g)
+        lg[0, r, :, ch] = -40.0 - 160.0 * torch.rand((lg.shape[2], 8), generator=g)
+    _check(inp, fused=fused)
+
+
+def test_direct_path_forced_on_ordinary_inputs():
+    """KDA_DEBUG_FORCE_DIRECT=1 sends every chunk of both chunked paths through the steep-decay
+    path: on ordinary inputs (packed documents with h0, and a batch ending in a partial chunk) it
+    must meet the oracle like the anchored factors do. Runs in a child process (the hook is read
+    once per process)."""
+    code = (
+        "import torch, gated_delta_rule_144_b200 as kda, sys\n"
+        "sys.path.insert(0, 'tests')\n"
+        "from gated_delta_rule_144_b200 import synth\n"
+        "from kda_testutil import oracle_fwd, rel_l2, host, to\n"
+        "cases = [synth.prefill_inputs('packed-8docs', lengths=[700, 1, 64, 300], H=4,\n"
+        "                              h0_std=0.05, seed=24),\n"
+        "         synth.prefill_inputs('long-t65536', B=2, T=64 * 9 + 5, H=2, seed=25)]\n"
+        "worst = 0.0\n"
+        "for inp in cases:\n"
+        "    o_ref, h_ref = oracle_fwd(inp)\n"
+        "    g = to(inp, 'cuda:0')\n"
+        "    for fused in (False, True):\n"
+        "        o, hT = kda.fwd(g['q'], g['k'], g['v'], g['log_g'], g['beta'], h0=g['h0'],\n"
+        "                        cu_seqlens=g['cu_seqlens'], fused=fused)\n"
+        "        torch.cuda.synchronize()\n"
+        "        assert kda.get_device_error() == 0\n"
+        "        worst = max(worst, rel_l2(host(o), o_ref), rel_l2(host(hT), h_ref))\n"
+        "print('WORST', worst)\n")
+    env = dict(os.environ, KDA_DEBUG_FORCE_DIRECT="1")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], env=env, cwd=root, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    worst = float([x for x in r.stdout.splitlines() if x.startswith("WORST")][-1].split()[1])
+    print("direct path, worst rel-L2 %.3e" % worst)
+    assert worst <= TOL_BF16
 
 
 def test_expired_wait_reports_timeout_and_context_survives():
