@@ -175,7 +175,7 @@ static size_t order_bytes(const kda_fwd_desc_t* d, Path path) {
 
 // Workspace of the split chunked path (intra-chunk kernel + state pass), 256-byte aligned parts.
 struct SplitLayout {
-    size_t order, map, counters, state, decay, wq, ke, ut, ot, total;
+    size_t order, map, counters, state, decay, wq, ke, ut, aq, total;
     long long G;
     int ncT;
     bool has_order;
@@ -201,7 +201,7 @@ static bool split_layout(const kda_fwd_desc_t* d, Path path, bool packed, SplitL
     L->wq = off;    off += (size_t)R * 32768;
     L->ke = off;    off += (size_t)R * 16384;
     L->ut = off;    off += (size_t)R * 16384;
-    L->ot = off;    off += (size_t)R * 16384;
+    L->aq = off;    off += (size_t)R * 8192;
     L->total = off;
     return true;
 }
@@ -322,7 +322,7 @@ static kda_status_t fwd_impl(const kda_fwd_desc_t* d, const void* q, const void*
         ws.wq = reinterpret_cast<__nv_bfloat16*>(w + L.wq);
         ws.ke = reinterpret_cast<__nv_bfloat16*>(w + L.ke);
         ws.ut = reinterpret_cast<__nv_bfloat16*>(w + L.ut);
-        ws.ot = reinterpret_cast<__nv_bfloat16*>(w + L.ot);
+        ws.aq = reinterpret_cast<__nv_bfloat16*>(w + L.aq);
         ws.decay = reinterpret_cast<float*>(w + L.decay);
         ws.map = cu_seqlens ? reinterpret_cast<int32_t*>(w + L.map) : nullptr;
         ws.counters = reinterpret_cast<unsigned long long*>(w + L.counters);

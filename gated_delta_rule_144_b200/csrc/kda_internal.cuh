@@ -28,10 +28,10 @@ __device__ __forceinline__ void set_device_error(unsigned* err, unsigned code) {
 // document + chunk (strictly increasing over (document, chunk), so records never collide and
 // g < ncT + N).
 struct SplitWorkspace {
-    __nv_bfloat16* wq;   // [R * 128][128]: rows 0-63 W, 64-127 Q~
+    __nv_bfloat16* wq;   // [R * 128][128]: rows 0-63 W, 64-127 Q+
     __nv_bfloat16* ke;   // [R * 64][128]: K_end
     __nv_bfloat16* ut;   // [R * 128][64]: U~^T (value column, token)
-    __nv_bfloat16* ot;   // [R * 128][64]: O~^T
+    __nv_bfloat16* aq;   // [R * 64][64]: A_qk (row r, column i; zero above the diagonal)
     float* decay;        // [R][128]: e^{Gamma_end}
     int32_t* map;        // [G]: document of chunk record g, -1 if unused (packed only)
     float* state;        // [N][H][128][128]: state between segments (equal-length sequences only)

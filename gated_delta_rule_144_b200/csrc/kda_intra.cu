@@ -6,27 +6,27 @@
 // channel:
 //   A_kk[r,i] = sum_c k_rc k_ic e^{Gamma_rc - Gamma_ic}  (i < r)    A_qk: same with q_r, i <= r
 //   T  = (I + diag(beta) A_kk)^-1 diag(beta)                          (UT transform, fp32)
-//   W  = T (k e^{Gamma}),  U~ = T v,  Q~ = q e^{Gamma} - A_qk W,  O~ = A_qk U~,
+//   W  = T (k e^{Gamma}),  U~ = T v,  Q+ = q e^{Gamma},
 //   K_end = k e^{Gamma_end - Gamma},  decay = e^{Gamma_end}
-// and the state pass later applies U = U~ - W S, o = O~ + Q~ S, S <- diag(decay) S + K_end^T U.
+// and the state pass later applies U = U~ - W S, o = Q+ S + A_qk U, S <- diag(decay) S + K_end^T U.
 // A_kk and A_qk come from one tensor-core product R C^T of separable factors anchored at the
 // middle of each 16-row block (rows of R at their own block's middle, diagonal-block columns at
 // theirs, the columns a later block needs at that later block's middle), so no factor leaves the
-// float32 range while the summed decay of 8 consecutive rows stays above about -69 nats.
+// float32 range while the summed decay of 8 consecutive rows stays above about -69 nats; a chunk
+// with a steeper decay is evaluated directly (steep_chunk).
 //
 // Occupancy: two CTAs share each SM, so that one CTA's tensor-core waits, barriers and memory
 // latency are covered by the other's CUDA-core work. To fit two CTAs (about 110 KB of shared memory
 // and 256 TMEM columns each) the tiles share space: k and q arrive by TMA where R's rows go and are
 // overwritten in place by k rho and q rho, log g arrives in the K+ / V region and is consumed before
 // K+ and V are written there, the R/C region then holds the UT solve and finally the store staging.
-// K_end is written to the workspace from registers, and Q+ = q e^{Gamma} is parked in the workspace
-// slot of Q~ and read back when Q~ = Q+ - A_qk W is formed. The next record's input tiles are
+// Q+ and K_end go from registers straight to the workspace. The next record's input tiles are
 // prefetched into L2 while this one runs.
 //
 // Per record (256 threads; thread 0 issues the MMAs, lane 0 of warp 7 the copies):
 //   TMA k, q, log g -> decay products -> TMA V; R, C, K+ (shared), Q+, K_end (global) ->
-//   MMA R C^T -> A_kk, A_qk -> UT solve -> MMA T' = A_qk T -> MMA [T; T'] K+ and V^T [T; T']^T ->
-//   [W; Q~], U~^T, O~^T staged in shared memory -> TMA stores.
+//   MMA R C^T -> A_kk, A_qk (TMA store of A_qk) -> UT solve -> MMA [T; -] K+ and V^T T^T ->
+//   W, U~^T staged in shared memory -> TMA stores.
 // Every mbarrier wait is bounded; on expiry the CTA records KDA_ERR_TIMEOUT, drains its own
 // copies and MMAs, frees TMEM and exits.
 
@@ -59,13 +59,14 @@ constexpr uint32_t OFF_C = OFF_R + 32768;    // C  [160][128] bf16, K-major B (2
 constexpr uint32_t OFF_LB = OFF_R;           // L = diag(beta) A_kk, f32 [64][kLdl]
 constexpr uint32_t OFF_MB = OFF_R + 17408;   // (I + L)^-1, f32 [64][kLdm]
 constexpr uint32_t OFF_YS = OFF_R + 35840;   // four 16x17 f32 scratch blocks of the solve
-constexpr uint32_t OFF_TT = OFF_R + 40960;   // [T; T'] [128][64] bf16 (K-major A; rows 0-63
-                                             //   also the MN-major B of T')
-constexpr uint32_t OFF_ZA = OFF_R + 57344;   // [0; A_qk] [128][64] bf16 (K-major A)
-//   and, once the WY products have read it, the staging tiles of the stores:
-constexpr uint32_t OFF_SWQ = OFF_R;          // [W; Q~] [128][128] (2 panels x 16 KB)
-constexpr uint32_t OFF_SUT = OFF_R + 32768;  // U~^T [128 value columns][64 tokens]
-constexpr uint32_t OFF_SOT = OFF_R + 49152;  // O~^T [128][64]
+constexpr uint32_t OFF_TT = OFF_R + 40960;   // [T; -] [128][64] bf16 (K-major A of the first WY
+                                             //   product, rows 64-127 unused; rows 0-63 also the
+                                             //   K-major B of the second)
+constexpr uint32_t OFF_ZA = OFF_R + 57344;   // [0; A_qk] [128][64] bf16: rows 64-127 are the
+                                             //   record's A_qk tile, stored from here by TMA
+//   and, once the UT solve is done with them, the staging tiles of the stores:
+constexpr uint32_t OFF_SW = OFF_R;           // W [64][128] (2 panels x 8 KB)
+constexpr uint32_t OFF_SUT = OFF_R + 16384;  // U~^T [128 value columns][64 tokens]
 constexpr uint32_t OFF_MISC = OFF_C + 40960;
 // (steep-decay path only: half-block sums at OFF_C and K+ staged at OFF_C + 4096, both below
 // OFF_ZA, which that path writes at the same time)
@@ -78,15 +79,13 @@ constexpr uint32_t OFF_CLAIM = OFF_TMEM + 16;     // two claimed record indices 
 constexpr uint32_t kSmemBytes = OFF_CLAIM + 16 + 1024;   // + alignment slack
 static_assert(OFF_ZA + 16384 == OFF_C + 40960, "solve buffers fill the R/C region exactly");
 static_assert(OFF_YS + 4 * 16 * 17 * 4 <= OFF_TT, "solve scratch overlaps [T; T']");
-static_assert(OFF_SWQ + 32768 <= OFF_TT, "[W; Q~] staging must not touch [T; T'] (read by the "
-                                         "second WY product while [W; Q~] is staged)");
-static_assert(OFF_SOT + 16384 <= OFF_MISC, "staging overflows the R/C region");
+static_assert(OFF_SUT + 16384 <= OFF_TT, "staging must not touch [T; -] (read by the second WY "
+                                        "product while W is staged) or A_qk (stored meanwhile)");
 static_assert(2 * (kSmemBytes + 1024) <= 233472, "two CTAs per SM");
 // TMEM columns (fp32, 128 lanes; row m of an M = 128 product sits in lane m)
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t TM_A = 0;     // R C^T [128 x 160]; later [T; T'] K+ (0-127) and
-                                 //   V^T [T; T']^T (128-255: U~^T, then O~^T)
-constexpr uint32_t TM_TP = 160;  // [0; A_qk] T (lanes 64-127: T')
+constexpr uint32_t TM_A = 0;     // R C^T [128 x 160]; later [T; -] K+ (0-127, W in lanes
+                                 //   0-63) and V^T T^T (128-191: U~^T)
 constexpr int kLdl = 68;         // row stride (floats) of L: conflict-free A-fragment loads
 constexpr int kLdm = 72;         // row stride (floats) of M: conflict-free B-fragment loads
 constexpr uint32_t kTxV = 16384;
@@ -104,7 +103,7 @@ struct IntraArgs {
     const __nv_bfloat16* beta;
     const int32_t* cu;       // nullable: packed documents
     const int32_t* map;      // packed: document of chunk record g (-1: unused)
-    __nv_bfloat16* wq;       // [R * 128][128]: W, Q~ (Q+ parked there in between)
+    __nv_bfloat16* wq;       // [R * 128][128]: W (rows 0-63, TMA), Q+ (rows 64-127, stores)
     __nv_bfloat16* ke;       // [R * 64][128]: K_end
     float* decay;            // [R][128]
     long long G;             // chunk records per head
@@ -118,10 +117,10 @@ struct IntraArgs {
 };
 
 // q, k, v: [rows, H, 128] maps of one head's 64-row tile in 64-column boxes (128-byte swizzle);
-// log g: the same with whole 128-column rows, no swizzle; wq, ut, ot: record stores (128-byte
-// swizzle).
+// log g: the same with whole 128-column rows, no swizzle; w (the W rows of the [W; Q+] record
+// tile), ut, aq: record stores (128-byte swizzle).
 struct IntraMaps {
-    CUtensorMap q, k, g, v, wq, ut, ot;
+    CUtensorMap q, k, g, v, w, ut, aq;
 };
 
 struct Unit {
@@ -152,11 +151,6 @@ __device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int c0, int c1
                      reinterpret_cast<uint64_t>(tmap)),
                  "r"(c0), "r"(c1), "r"(c2)
                  : "memory");
-}
-// Orders this thread's generic-proxy writes (shared and global) before later async-proxy
-// accesses (TMA stores) issued after a barrier.
-__device__ __forceinline__ void fence_proxy_async_all() {
-    asm volatile("fence.proxy.async;" ::: "memory");
 }
 
 // Steep-decay path of one record (all 256 threads; called in place of the operand pass, the
@@ -295,7 +289,7 @@ __device__ __noinline__ void steep_chunk(uint8_t* sm, int L, long long rec, __nv
                 }
         }
     }
-    // [0; A_qk]: A_qk (i <= r) in rows 64 + r, zeros above the diagonal and in rows 0-63
+    // A_qk (i <= r) in rows 64 + r of [0; A_qk], zeros above the diagonal
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
         const int r = 4 * R4 + a;
@@ -303,8 +297,6 @@ __device__ __noinline__ void steep_chunk(uint8_t* sm, int L, long long rec, __nv
 #pragma unroll
         for (int b = 0; b < 4; ++b) x[b] = 4 * I4 + b <= r ? aqk[a][b] : 0.f;
         st_bf16x4(sm + OFF_ZA + sw128_off(128, 64 + r, 4 * I4), x[0], x[1], x[2], x[3]);
-        *reinterpret_cast<uint2*>(sm + OFF_ZA + sw128_off(128, r, 4 * I4)) =
-            make_uint2(0u, 0u);
     }
     __syncthreads();   // k, q and Gamma fully read: R and the log g tile may be reused
     {
@@ -398,9 +390,9 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         prefetch_tmap(&maps.k);
         prefetch_tmap(&maps.g);
         prefetch_tmap(&maps.v);
-        prefetch_tmap(&maps.wq);
+        prefetch_tmap(&maps.w);
         prefetch_tmap(&maps.ut);
-        prefetch_tmap(&maps.ot);
+        prefetch_tmap(&maps.aq);
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(tmem_s), kTmemCols);
@@ -601,8 +593,8 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         // ---------------------------------------------------------------- operands
         //   R: k rho, q rho (rho_r = e^{Gamma_r - Gamma_m}, m the middle of r's block)
         //   C: k kappa (kappa = e^{Gamma_m - Gamma_r}), cross columns k sigma X_a, X_a <= 1
-        //   K+ = k e^{Gamma} (shared), Q+ = q e^{Gamma} (parked in the Q~ slot),
-        //   K_end = k e^{Gamma_end - Gamma} = k G sigma (workspace)
+        //   K+ = k e^{Gamma} (shared), Q+ = q e^{Gamma} and K_end = k e^{Gamma_end - Gamma} =
+        //   k G sigma (workspace)
         if (!steep) {
             __nv_bfloat16* qplus = args.wq + ((size_t)rec * 128 + 64) * kD + ch0;
             __nv_bfloat16* kend = args.ke + (size_t)rec * kC * kD + ch0;
@@ -709,14 +701,10 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
                     x[j] = (is_q ? i <= r : i < r) ? val : 0.f;
                 }
                 put16(16 * a, x);
-                const uint4 z = make_uint4(0, 0, 0, 0);
                 if (is_q) {   // A_qk is lower triangular: zero the blocks after the diagonal one
+                    const uint4 z = make_uint4(0, 0, 0, 0);
                     for (int i = 16 * (a + 1); i < kC; i += 8)
                         *reinterpret_cast<uint4*>(sm + OFF_ZA + sw128_off(128, 64 + r, i)) = z;
-                } else {      // rows 0-63 of [0; A_qk] are zero
-#pragma unroll
-                    for (int i = 0; i < kC; i += 8)
-                        *reinterpret_cast<uint4*>(sm + OFF_ZA + sw128_off(128, r, i)) = z;
                 }
             } else if ((qd & 1) == 0) {
                 float w[16];
@@ -752,6 +740,12 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
+        // A_qk (rows 64-127 of [0; A_qk]) is final: store it while the UT transform runs
+        if (tid == kThreads - 96) {
+            tma_store_2d(&maps.aq, sb + OFF_ZA + 8192, 0, (int)(rec * 64));
+            bulk_commit();
+        }
+        stores_pending = true;
 
         // ---------------------------------------------------------------- UT transform
         {
@@ -873,42 +867,10 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         fence_proxy_async();
         __syncthreads();
 
-        // ---------------------------------------------------------------- MMA: T' = A_qk T
-        // [0; A_qk] (128 x 64) times T as the MN-major B operand: lanes 64-127 receive A_qk T.
-        if (warp == 0) {
-            if (lane == 0) {
-                tc_fence_after();
-                const uint32_t id = idesc_bf16(128, 64, 0, 1);
-#pragma unroll
-                for (int s = 0; s < kC / 16; ++s)
-                    umma_f16(tbase + TM_TP, desc_at(dK, sb + OFF_ZA + 32 * s),
-                             desc_at(dM8, sb + OFF_TT + 2048 * s), id, s > 0);
-                umma_commit(bar_mma);
-            }
-            __syncwarp();
-        }
-        mma_pending = true;
-        if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
-        ++mma_phase;
-        mma_pending = false;
-        tc_fence_after();
-        if (qd >= 2) {
-            // T' rows r = 32 (qd - 2) + lane  ->  rows 64 + r of [T; T']
-            float v[32];
-            const int r = 32 * (qd - 2) + lane;
-            tmem_ld32(tbase + lane_q + TM_TP + 32 * hf, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int m = 0; m < 4; ++m)
-                st_bf16x8(sm + OFF_TT + sw128_off(128, 64 + r, 32 * hf + 8 * m), v + 8 * m);
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-
         // ---------------------------------------------------------------- MMA: WY products
-        // [T; T'] K+ (lanes 0-63: W, 64-127: A_qk W) and, transposed for the state pass,
-        // V^T [T; T']^T (lane j = value column: U~^T in columns 128-191, O~^T in 192-255)
+        // [T; -] K+ (lanes 0-63: W; rows 64-127 of the A operand are never read out) and,
+        // transposed for the state pass, V^T T^T (lane j = value column: U~^T in columns
+        // 128-191)
         if (!wait_all(bar_v, v_count & 1)) { aborted = true; break; }
         ++v_count;
         v_pending = false;
@@ -916,12 +878,12 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
             if (lane == 0) {
                 tc_fence_after();
                 const uint32_t id = idesc_bf16(128, 128, 0, 1);
-                const uint32_t idt = idesc_bf16(128, 128, 1, 0);
+                const uint32_t idt = idesc_bf16(128, 64, 1, 0);
 #pragma unroll
                 for (int s = 0; s < kC / 16; ++s)
                     umma_f16(tbase + TM_A, desc_at(dK, sb + OFF_TT + 32 * s),
                              desc_at(dM8, sb + OFF_KP + 2048 * s), id, s > 0);
-                umma_commit(bar_mma);   // W and A_qk W: read out while the next group runs
+                umma_commit(bar_mma);   // W: read out while the next product runs
 #pragma unroll
                 for (int s = 0; s < kC / 16; ++s)
                     umma_f16(tbase + TM_A + 128, desc_at(dM8, sb + OFF_V + 2048 * s),
@@ -935,38 +897,18 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         ++mma_phase;
         mma_pending = false;
         tc_fence_after();
-        {
-            // quarters 0-1: W rows -> [W; Q~] rows 0-63.  quarters 2-3: Q~ = Q+ - A_qk W, with
-            // Q+ read back from the workspace. Each warp takes 64 of the 128 columns.
-            const int r = 32 * (qd & 1) + lane;
-            const int row = qd < 2 ? r : 64 + r;
-            const uint4* qp = reinterpret_cast<const uint4*>(
-                args.wq + ((size_t)rec * 128 + 64 + r) * kD + 64 * hf);
+        if (qd < 2) {
+            // W rows r = 32 qd + lane (TMEM lanes 0-63); each warp takes 64 of the 128 columns
+            const int r = 32 * qd + lane;
 #pragma unroll
-            for (int part = 0; part < 4; ++part) {
-                const int c0 = 64 * hf + 16 * part;
-                uint4 qv2[2];
-                if (qd >= 2) {
-                    qv2[0] = __ldcg(qp + 2 * part);
-                    qv2[1] = __ldcg(qp + 2 * part + 1);
-                }
-                float v[16];
-                tmem_ld16(tbase + lane_q + TM_A + c0, v);
+            for (int part = 0; part < 2; ++part) {
+                const int c0 = 64 * hf + 32 * part;
+                float v[32];
+                tmem_ld32(tbase + lane_q + TM_A + c0, v);
                 tmem_ld_wait();
 #pragma unroll
-                for (int m = 0; m < 2; ++m) {
-                    uint8_t* p = sm + OFF_SWQ + sw128_off(128, row, c0 + 8 * m);
-                    const float* w = v + 8 * m;
-                    if (qd < 2) {
-                        st_bf16x8(p, w);
-                    } else {
-                        const float2 a0 = unpack_bf16(qv2[m].x), a1 = unpack_bf16(qv2[m].y);
-                        const float2 a2 = unpack_bf16(qv2[m].z), a3 = unpack_bf16(qv2[m].w);
-                        *reinterpret_cast<uint4*>(p) = make_uint4(
-                            pack_bf16(a0.x - w[0], a0.y - w[1]), pack_bf16(a1.x - w[2], a1.y - w[3]),
-                            pack_bf16(a2.x - w[4], a2.y - w[5]), pack_bf16(a3.x - w[6], a3.y - w[7]));
-                    }
-                }
+                for (int m = 0; m < 4; ++m)
+                    st_bf16x8(sm + OFF_SW + sw128_off(64, r, c0 + 8 * m), v + 8 * m);
             }
         }
         if (!wait_all(bar_wy2, wy2_count & 1)) { aborted = true; break; }
@@ -974,35 +916,27 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         wy2_pending = false;
         tc_fence_after();
         {
-            // U~^T (TMEM columns 128-191) and O~^T (192-255), lane j = value column, into bf16
-            // staging tiles [128 j][64 tokens] (128-byte swizzle)
+            // U~^T (TMEM columns 128-191), lane j = value column, into the bf16 staging tile
+            // [128 j][64 tokens] (128-byte swizzle); each warp takes 32 of the 64 tokens
             const int jrow = 32 * qd + lane;
-            const uint32_t stage = hf == 0 ? OFF_SUT : OFF_SOT;
+            float v[32];
+            tmem_ld32(tbase + lane_q + TM_A + 128 + 32 * hf, v);
+            tmem_ld_wait();
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                float v[32];
-                tmem_ld32(tbase + lane_q + TM_A + 128 + 64 * hf + 32 * part, v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    st_bf16x8(sm + stage + sw128_off(128, jrow, 32 * part + 8 * m), v + 8 * m);
-            }
+            for (int m = 0; m < 4; ++m)
+                st_bf16x8(sm + OFF_SUT + sw128_off(128, jrow, 32 * hf + 8 * m), v + 8 * m);
         }
-        // shared staging tiles and the Q+ parked in the workspace, before the async-proxy stores
-        fence_proxy_async_all();
+        // shared staging tiles before the async-proxy stores
+        fence_proxy_async();
         tc_fence_before();
         __syncthreads();
         {
-            const int rw = (int)(rec * 128);
             if (tid == copier) {
-                tma_store_2d(&maps.wq, sb + OFF_SWQ, 0, rw);
-                tma_store_2d(&maps.wq, sb + OFF_SWQ + 16384, 64, rw);
+                tma_store_2d(&maps.w, sb + OFF_SW, 0, (int)(rec * 128));
+                tma_store_2d(&maps.w, sb + OFF_SW + 8192, 64, (int)(rec * 128));
                 bulk_commit();
             } else if (tid == kThreads - 64) {
-                tma_store_2d(&maps.ut, sb + OFF_SUT, 0, rw);
-                bulk_commit();
-            } else if (tid == kThreads - 96) {
-                tma_store_2d(&maps.ot, sb + OFF_SOT, 0, rw);
+                tma_store_2d(&maps.ut, sb + OFF_SUT, 0, (int)(rec * 128));
                 bulk_commit();
             }
             stores_pending = true;
@@ -1134,9 +1068,9 @@ cudaError_t launch_chunk64_intra(const FwdParams& p, int c_begin, int c_span,
         (e = make_rows_map(&m.k, p.k, BF, 2, rows, p.H, 64, SW)) != cudaSuccess ||
         (e = make_rows_map(&m.g, p.log_g, F32, 4, rows, p.H, kD, SWN)) != cudaSuccess ||
         (e = make_rows_map(&m.v, p.v, BF, 2, rows, p.H, 64, SW)) != cudaSuccess ||
-        (e = make_map_2d(&m.wq, ws.wq, BF, 2, R * 128, kD, 64, 128, SW)) != cudaSuccess ||
+        (e = make_map_2d(&m.w, ws.wq, BF, 2, R * 128, kD, 64, 64, SW)) != cudaSuccess ||
         (e = make_map_2d(&m.ut, ws.ut, BF, 2, R * 128, kC, 64, 128, SW)) != cudaSuccess ||
-        (e = make_map_2d(&m.ot, ws.ot, BF, 2, R * 128, kC, 64, 128, SW)) != cudaSuccess)
+        (e = make_map_2d(&m.aq, ws.aq, BF, 2, R * 64, kC, 64, 64, SW)) != cudaSuccess)
         return e;
     int cap = 0;
     if ((e = intra_grid_cap(&cap)) != cudaSuccess) return e;

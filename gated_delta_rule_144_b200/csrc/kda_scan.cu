@@ -3,27 +3,29 @@
 //
 // The intra-chunk kernel (intra_kernel, kda_intra.cu) has already written, for every chunk
 // of 64 tokens and every head, the chunk's WY factors to the workspace:
-//   [W; Q~] (128 x 128 bf16), K_end (64 x 128 bf16), U~^T and O~^T (128 value columns x 64
-//   tokens, bf16) and the chunk's total decay e^{Gamma_end} (128 fp32).
+//   [W; Q+] (128 x 128 bf16), K_end (64 x 128 bf16), U~^T (128 value columns x 64 tokens, bf16),
+//   A_qk (64 x 64 bf16) and the chunk's total decay e^{Gamma_end} (128 fp32).
 // Per (sequence or document, head) this kernel then walks the chunks in order (the WY form of the
 // gated delta rule; GLM-5.3-Flash model card, Kimi Delta Attention snippet, and the state-passing
 // identity it implies):
-//   U = U~ - W S,   o = O~ + Q~ S,   S <- diag(e^{Gamma_end}) S + K_end^T U.
+//   U = U~ - W S,   o = Q+ S + A_qk U,   S <- diag(e^{Gamma_end}) S + K_end^T U.
 //
 // Layout: the state is kept transposed, S^T [value column j][key channel c], in TMEM lane j, so
-// both products take their state-side operand from TMEM and no shared-memory write sits on the
+// every product takes its state-side operand from TMEM and no shared-memory write sits on the
 // critical path:
-//   D = S^T [W; Q~]^T    (A = bf16 copy of S^T in TMEM, B = [W; Q~] K-major in shared memory)
+//   D = S^T [W; Q+]^T     (A = bf16 copy of S^T in TMEM, B = [W; Q+] K-major in shared memory)
 //   S^T += U^T K_end      (A = bf16 U^T in TMEM, B = K_end MN-major in shared memory)
+//   o^T = (Q+ S)^T + U^T A_qk^T   (accumulated into D's second half; A = U^T, B = A_qk K-major)
 // Eight data warps: warps w and w + 4 share TMEM lane quarter w mod 4 (lane j = value column j)
 // and split the columns of every TMEM row between them. A ninth warp only issues the MMAs, so that
 // no MMA issue waits behind a data warp's work. Per chunk c the critical chain is
 //   bf16(S^T) -> D (8 K steps) -> U^T -> S^T += U^T K_end (4 K steps);
-// the decay of S^T, the loads of U~^T and O~^T and the output of chunk c-1 (o = O~ + Q~ S, read
-// from the other of two D buffers, staged in shared memory and written by a TMA store) run while
-// the D product of chunk c is in flight. Lane 0 of warp 1 issues the TMA loads (two stages: chunk
-// c+1 arrives while chunk c runs) and lane 0 of warp 2 the output stores. Every mbarrier wait is bounded; on expiry the CTA
-// records KDA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
+// the o product follows the update in the tensor pipe, off the chain. The decay of S^T, the load of
+// U~^T and the output of chunk c-1 (read from the other of two D buffers, staged in shared memory
+// and written by a TMA store) run while the D product of chunk c is in flight. Lane 0 of warp 1
+// issues the TMA loads (two stages: chunk c+1 arrives while chunk c runs) and lane 0 of warp 2 the
+// output stores. Every mbarrier wait is bounded; on expiry the CTA records KDA_ERR_TIMEOUT, drains
+// its own copies and MMAs, frees TMEM and exits.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -50,12 +52,12 @@ constexpr int kThreads = 32 * kDataWarps + 32;   // + one warp that only issues 
 constexpr uint32_t ST_WQ = 0;        // [W; Q~] 128 x 128 bf16, K-major SW128: 2 panels of 16 KB
 constexpr uint32_t ST_KE = 32768;    // K_end 64 x 128 bf16, MN-major SW128: 2 panels of 8 KB
 constexpr uint32_t ST_UT = 49152;    // U~^T [128 j][64 tokens] bf16, SW128
-constexpr uint32_t ST_OT = 65536;    // O~^T [128 j][64 tokens] bf16, SW128
-constexpr uint32_t ST_DEC = 81920;   // e^{Gamma_end} [128] f32
-constexpr uint32_t kStage = 82944;   // 81 KB, a multiple of 1024
-constexpr uint32_t kTxStage = 32768 + 3 * 16384 + 512;
+constexpr uint32_t ST_AQ = 65536;    // A_qk [64 r][64 i] bf16, K-major SW128
+constexpr uint32_t ST_DEC = 73728;   // e^{Gamma_end} [128] f32
+constexpr uint32_t kStage = 74752;   // 73 KB, a multiple of 1024
+constexpr uint32_t kTxStage = 32768 + 2 * 16384 + 8192 + 512;
 constexpr uint32_t OFF_O = 2 * kStage;       // two output tiles o [64 tokens][128] bf16
-constexpr uint32_t OFF_BAR = OFF_O + 32768;  // full[2], mma1, mma2, never
+constexpr uint32_t OFF_BAR = OFF_O + 32768;  // full[2], mma1, mma2, never, mma3
 constexpr uint32_t OFF_TMEM = OFF_BAR + 64;
 constexpr uint32_t kSmemBytes = OFF_TMEM + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -64,8 +66,8 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 constexpr uint32_t TS = 0;     // S^T fp32 [128 x 128]
 constexpr uint32_t TB = 128;   // bf16 S^T, A operand: 64 columns
 constexpr uint32_t TU = 192;   // bf16 U^T, A operand: 32 columns
-constexpr uint32_t TD = 256;   // two buffers of S^T [W; Q~]^T fp32 (128 columns each):
-                               //   columns 0-63 (W S)^T, 64-127 (Q~ S)^T
+constexpr uint32_t TD = 256;   // two buffers of S^T [W; Q+]^T fp32 (128 columns each):
+                               //   columns 0-63 (W S)^T, 64-127 (Q+ S)^T, then o^T
 constexpr uint32_t kTmemCols = 512;
 
 struct ScanArgs {
@@ -84,7 +86,7 @@ struct ScanArgs {
 };
 
 struct ScanMaps {
-    CUtensorMap wq, ke, ut, ot, o;
+    CUtensorMap wq, ke, ut, aq, o;
 };
 
 __device__ __forceinline__ uint32_t pack2(float x, float y) {
@@ -140,18 +142,19 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
 
     uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
     const uint32_t bar_full0 = sb + OFF_BAR, bar_mma1 = bar_full0 + 16, bar_mma2 = bar_full0 + 24;
-    const uint32_t bar_never = bar_full0 + 32;
+    const uint32_t bar_never = bar_full0 + 32, bar_mma3 = bar_full0 + 40;
     if (tid == 0) {
         mbar_init(bar_full0, 1);
         mbar_init(bar_full0 + 8, 1);
         mbar_init(bar_mma1, 1);
         mbar_init(bar_mma2, 1);
         mbar_init(bar_never, 1);
+        mbar_init(bar_mma3, 1);
         fence_mbar_init();
         prefetch_tmap(&maps.wq);
         prefetch_tmap(&maps.ke);
         prefetch_tmap(&maps.ut);
-        prefetch_tmap(&maps.ot);
+        prefetch_tmap(&maps.aq);
         prefetch_tmap(&maps.o);
     }
     if (warp == 0) {
@@ -187,7 +190,7 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         tma_load_2d(st + ST_KE, &maps.ke, bar, 0, (int)(rec * 64));
         tma_load_2d(st + ST_KE + 8192, &maps.ke, bar, 64, (int)(rec * 64));
         tma_load_2d(st + ST_UT, &maps.ut, bar, 0, (int)(rec * 128));
-        tma_load_2d(st + ST_OT, &maps.ot, bar, 0, (int)(rec * 128));
+        tma_load_2d(st + ST_AQ, &maps.aq, bar, 0, (int)(rec * 64));
         bulk_load(st + ST_DEC, args.decay + rec * kD, 512, bar);
     };
 
@@ -195,32 +198,34 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
     const uint64_t dM8 = sw128_desc(0, 8192, 1024);  // MN-major, 64-row panels
     const uint32_t id1 = idesc_bf16(128, 128, 0, 0);
     const uint32_t id2 = idesc_bf16(128, 128, 0, 1);
+    const uint32_t id3 = idesc_bf16(128, 64, 0, 0);
 
     // outstanding asynchronous work, drained before exit if a wait expires
     int issued = 0;          // chunks whose copies were issued
     int landed = 0;          // chunks whose copies were waited for
-    bool mma1_pending = false, mma2_pending = false;
-    int mma1_chunk = 0, mma2_chunk = 0;   // chunk of the last commit (its phase parity)
+    bool mma1_pending = false, mma2_pending = false, mma3_pending = false;
+    int mma1_chunk = 0, mma2_chunk = 0, mma3_chunk = 0;   // chunk of the last commit (parity)
     bool aborted = false;
-    auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
+    // One thread polls; the rest of the CTA waits at the barrier that publishes the outcome (and
+    // any failure a thread has recorded in `also_bad` since the last barrier).
+    auto wait_all = [&](uint32_t bar, uint32_t parity, bool also_bad = false) -> bool {
         const bool ok = tid != 0 || mbar_wait(bar, parity, args.budget);
-        return __syncthreads_or(!ok) == 0;
+        return __syncthreads_or(!ok || also_bad) == 0;
     };
 
-    // o of chunk cc (rows < L): O~^T (this thread's 32 tokens, packed in ob) + (Q~ S)^T from D
-    // buffer cc & 1, staged row-major in output tile cc & 1
-    uint32_t ob[16];
-    auto stage_o = [&](int cc) {
+    // o of chunk cc (rows < L): o^T = (Q+ S)^T + U^T A_qk^T from D buffer cc & 1 (this thread's
+    // 32 tokens), staged row-major in output tile cc & 1. Waits (every data thread, bounded) for
+    // the o product of chunk cc; returns false if that wait expired.
+    auto stage_o = [&](int cc) -> bool {
+        const bool ok = mbar_wait(bar_mma3, (uint32_t)(cc & 1), args.budget);
+        tc_fence_after();
         float w[32];
         tmem_ld32(tbase + lq + TD + 128 * (cc & 1) + 64 + 32 * hs, w);
         tmem_ld_wait();
         __nv_bfloat16* tile = reinterpret_cast<__nv_bfloat16*>(sm + OFF_O + 16384 * (cc & 1));
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int r = 32 * hs + 2 * i;
-            tile[r * kD + j] = __float2bfloat16_rn(lo_bf(ob[i]) + w[2 * i]);
-            tile[(r + 1) * kD + j] = __float2bfloat16_rn(hi_bf(ob[i]) + w[2 * i + 1]);
-        }
+        for (int i = 0; i < 32; ++i) tile[(32 * hs + i) * kD + j] = __float2bfloat16_rn(w[i]);
+        return ok;
     };
     // write staged tile cc to o: one TMA store for a full chunk, row copies for a partial one
     // (a TMA box would run into the next document's rows). Call after a CTA barrier that
@@ -294,15 +299,11 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         }
         mma1_pending = true;
         mma1_chunk = c;
-        // stage (c+1)&1 held chunk c-1, fully consumed by now: fetch chunk c+1 into it
-        if (c >= 1 && c + 1 < nchunks) {
-            if (tid == kLoader) issue(c + 1);
-            issued = c + 2;
-        }
 
         // ---------------------------------------------------------------- while D runs
         // decay: TS = S^T diag(e^{Gamma_end}) (the update accumulates into it)
         uint32_t ub[16];
+        bool o_bad = false;
         if (data) {
             const float* dec = reinterpret_cast<const float*>(stp + ST_DEC) + 64 * hs;
 #pragma unroll
@@ -321,11 +322,17 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
                     stp + ST_UT + sw128_off(128, j, 32 * hs + 8 * m));
                 ub[4 * m] = x.x; ub[4 * m + 1] = x.y; ub[4 * m + 2] = x.z; ub[4 * m + 3] = x.w;
             }
-            if (c >= 1) stage_o(c - 1);
+            if (c >= 1) o_bad = !stage_o(c - 1);
+            // stage (c+1)&1 held chunk c-1, read by its update (waited for at this chunk's start)
+            // and its o product (waited for in stage_o): fetch chunk c+1 into it
+            if (tid == kLoader && !o_bad && c >= 1 && c + 1 < nchunks) issue(c + 1);
             tmem_st_wait();
         }
+        if (c >= 1 && c + 1 < nchunks) issued = c + 2;   // (a wait that expired aborts below;
+                                                         //  the drain's wait is bounded)
+        if (c >= 1) mma3_pending = false;   // (waited for above, or the CTA aborts below)
 
-        if (!wait_all(bar_mma1, (uint32_t)(c & 1))) { aborted = true; break; }
+        if (!wait_all(bar_mma1, (uint32_t)(c & 1), o_bad)) { aborted = true; break; }
         mma1_pending = false;
         tc_fence_after();
 
@@ -340,16 +347,7 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
                 pk[i] = pack2(lo_bf(ub[i]) - w[2 * i], hi_bf(ub[i]) - w[2 * i + 1]);
             tmem_st16u(tbase + lq + TU + 16 * hs, pk);
         }
-        // O~^T of this chunk, for its output at the next step
-        if (data) {
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const uint4 x = *reinterpret_cast<const uint4*>(
-                    stp + ST_OT + sw128_off(128, j, 32 * hs + 8 * m));
-                ob[4 * m] = x.x; ob[4 * m + 1] = x.y; ob[4 * m + 2] = x.z; ob[4 * m + 3] = x.w;
-            }
-            tmem_st_wait();
-        }
+        if (data) tmem_st_wait();
         fence_proxy_async();   // output tile c-1 -> TMA store
         tc_fence_before();
         __syncthreads();
@@ -363,9 +361,15 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
                 umma_f16_ts(tbase + TS, tbase + TU + 8 * s, desc_at(dM8, st + ST_KE + 2048 * s),
                             id2, 1);
             umma_commit(bar_mma2);
+            // o^T = (Q+ S)^T + U^T A_qk^T, behind the update in the pipe (off the chain)
+#pragma unroll
+            for (int s = 0; s < kC / 16; ++s)
+                umma_f16_ts(tbase + TD + 128 * (c & 1) + 64, tbase + TU + 8 * s,
+                            desc_at(dK, st + ST_AQ + 32 * s), id3, 1);
+            umma_commit(bar_mma3);
         }
-        mma2_pending = true;
-        mma2_chunk = c;
+        mma2_pending = mma3_pending = true;
+        mma2_chunk = mma3_chunk = c;
         if (c >= 1) flush_o(c - 1);
     }
 
@@ -377,6 +381,7 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
             mbar_wait(bar_full0 + 8 * (c & 1), (uint32_t)((c >> 1) & 1), drain);
         if (mma1_pending) mbar_wait(bar_mma1, (uint32_t)(mma1_chunk & 1), drain);
         if (mma2_pending) mbar_wait(bar_mma2, (uint32_t)(mma2_chunk & 1), drain);
+        if (mma3_pending) mbar_wait(bar_mma3, (uint32_t)(mma3_chunk & 1), drain);
         __syncthreads();
     } else {
         if (mma2_pending && !wait_all(bar_mma2, (uint32_t)(mma2_chunk & 1))) {
@@ -387,10 +392,15 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         if (nchunks > 0) {   // output of the last chunk
             if (tid == kStorer && nchunks >= 3) bulk_wait_read_le1();
             __syncthreads();
-            if (data) stage_o(nchunks - 1);
+            bool bad = false;
+            if (data) bad = !stage_o(nchunks - 1);
             fence_proxy_async();
-            __syncthreads();
-            flush_o(nchunks - 1);
+            if (__syncthreads_or(bad)) {
+                if (tid == 0) set_device_error(args.err, DEV_TIMEOUT);
+                mbar_wait(bar_mma3, (uint32_t)((nchunks - 1) & 1), 1ll << 31);
+            } else {
+                flush_o(nchunks - 1);
+            }
         }
         if (args.hT && data) {
 #pragma unroll 1
@@ -450,7 +460,7 @@ cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaSt
             cudaSuccess ||
         (e = make_map_2d(&m.ut, ws.ut, BF, 2, R * 128, kC, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) !=
             cudaSuccess ||
-        (e = make_map_2d(&m.ot, ws.ot, BF, 2, R * 128, kC, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) !=
+        (e = make_map_2d(&m.aq, ws.aq, BF, 2, R * 64, kC, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) !=
             cudaSuccess ||
         (e = make_map_3d_rows(&m.o, p.o, BF, 2, (unsigned long long)p.B * p.T, p.H, kD, kC)) !=
             cudaSuccess)

@@ -100,7 +100,7 @@ typedef struct {
  *   workspace, workspace_bytes : scratch owned by the caller (device memory, 16-byte aligned).
  *             With at least kda_fwd_workspace_size(desc) bytes the chunked path runs split: an
  *             intra-chunk kernel computes every chunk's WY factors in parallel over all chunks
- *             and heads and stores them here (about 80.5 KiB per 64-token chunk and head), then a
+ *             and heads and stores them here (about 72.5 KiB per 64-token chunk and head), then a
  *             state pass walks each sequence's chunks. For equal-length sequences of 64 chunks
  *             or more the two run in chunk segments (up to 12; KDA_SPLIT_SEGMENTS, 1-16,
  *             overrides): the state pass of one segment runs on an internal high-priority stream

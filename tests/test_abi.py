@@ -107,10 +107,10 @@ def test_decode_rejects_on_host(L):
 
 
 def _split_bytes(B, T, H, N, packed):
-    """Split-path workspace: per (64-token chunk record, head) 32 KiB of [W; Q~], 3 x 16 KiB of
-    K_end, U~, O~ and 512 B of decay; 256 B of record counters (one per chunk segment, at most
-    16); the record map and document order when packed, else one fp32 128 x 128 state per
-    (sequence, head) carried between chunk segments."""
+    """Split-path workspace: per (64-token chunk record, head) 32 KiB of [W; Q+], 2 x 16 KiB of
+    K_end and U~, 8 KiB of A_qk and 512 B of decay; 256 B of record counters (one per chunk
+    segment, at most 16); the record map and document order when packed, else one fp32 128 x 128
+    state per (sequence, head) carried between chunk segments."""
     up = lambda x: (x + 255) // 256 * 256
     ncT = (T + 63) // 64
     G = ncT + N if packed else B * ncT
@@ -118,7 +118,7 @@ def _split_bytes(B, T, H, N, packed):
     order = up(4 * N) if packed and 2 <= N <= 2048 else 0
     state = 0 if packed else N * H * 128 * 128 * 4
     return (order + (up(4 * G) if packed else 0) + up(8 * 16) + state + up(512 * R) +
-            R * (32768 + 3 * 16384))
+            R * (32768 + 2 * 16384 + 8192))
 
 
 def test_decode_tokens_rejects_on_host(L):
