@@ -36,6 +36,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "kda_internal.cuh"
 #include "kda_sm100.cuh"
@@ -145,6 +146,15 @@ __device__ __forceinline__ void st_bf16x8(uint8_t* p, const float* v) {
                                               pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
 }
 __device__ __forceinline__ uint32_t f2tf(float x) { return __float_as_uint(x); }
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 mul4(float4 a, float4 b) {
+    return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
+}
+// Two bf16 products (round to nearest) of the bf16 pair packed in u with the pair f.
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t u, __nv_bfloat162 f) {
+    __nv_bfloat162 x = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&u), f);
+    return *reinterpret_cast<uint32_t*>(&x);
+}
 
 __device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int c0, int c1, int c2) {
     asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
@@ -499,39 +509,54 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         // suffix products y_j = prod_{t > j} a_t, the upper half the prefix products
         // y_j = prod_{t <= j} a_t; tot = prod over all 8 rows. The other product of each row is
         // tot / y_j, formed below from the reciprocal that the operands need anyway.
+        // (This kernel is bound partly by instruction fetch: one copy of each phase, with
+        // selects where the half or the row mask differs, runs faster than copies specialised
+        // per half or for full chunks.)
         float y[8][4], tot[4];
-        float4 g4[8];
+        bool range_bad = false;
+        {
+            float a[8][4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) g4[j] = *reinterpret_cast<const float4*>(gs + (rbase + j) * kD + ch0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float run = 1.f;
+            for (int j = 0; j < 8; ++j) {
+                const float4 g = *reinterpret_cast<const float4*>(gs + (rbase + j) * kD + ch0);
+                const bool ok = rbase + j < L;   // rows past the document: a = 1
+                a[j][0] = ok ? __expf(g.x) : 1.f;
+                a[j][1] = ok ? __expf(g.y) : 1.f;
+                a[j][2] = ok ? __expf(g.z) : 1.f;
+                a[j][3] = ok ? __expf(g.w) : 1.f;
+            }
+            // The anchored factors invert these running products; they stay finite while every
+            // product is >= 1e-30. The products only shrink, so the first suffix (lower half) or
+            // the last prefix (upper half) is the smallest. A chunk with a steeper decay anywhere
+            // takes the direct path (steep_chunk) instead.
             if (hh == 0) {
 #pragma unroll
-                for (int j = 7; j >= 0; --j) {
-                    y[j][i] = run;
-                    const float gl = i == 0 ? g4[j].x : i == 1 ? g4[j].y : i == 2 ? g4[j].z : g4[j].w;
-                    run *= rbase + j < L ? __expf(gl) : 1.f;
+                for (int i = 0; i < 4; ++i) {
+                    float run = 1.f;
+#pragma unroll
+                    for (int j = 7; j >= 0; --j) {
+                        y[j][i] = run;
+                        run *= a[j][i];
+                    }
+                    tot[i] = run;
+                    range_bad |= y[0][i] < 1e-30f;
                 }
             } else {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float gl = i == 0 ? g4[j].x : i == 1 ? g4[j].y : i == 2 ? g4[j].z : g4[j].w;
-                    run *= rbase + j < L ? __expf(gl) : 1.f;
-                    y[j][i] = run;
+                for (int i = 0; i < 4; ++i) {
+                    float run = 1.f;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        run *= a[j][i];
+                        y[j][i] = run;
+                    }
+                    tot[i] = run;
+                    range_bad |= y[7][i] < 1e-30f;
                 }
             }
-            tot[i] = run;
         }
-        *reinterpret_cast<float4*>(loup_s + (pb * 2 + hh) * kD + ch0) =
+        *reinterpret_cast<float4*>(loup_s + rb8 * kD + ch0) =
             make_float4(tot[0], tot[1], tot[2], tot[3]);
-        // The anchored factors invert these running products; they stay finite while every
-        // product is >= 1e-30. The products only shrink, so the first suffix (lower half) or the
-        // last prefix (upper half) is the smallest. A chunk with a steeper decay anywhere takes
-        // the direct path below instead.
-        bool range_bad = false;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) range_bad |= (hh == 0 ? y[0][i] : y[7][i]) < 1e-30f;
         const bool steep = __syncthreads_or(range_bad || args.force_direct) != 0;
         // log g consumed (unless steep): the K+ / V region is free for V and K+
         if (!steep) {
@@ -541,53 +566,38 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         // half totals of every block: Lo_b (rows 0-7), Up_b (rows 8-15), P_b = Lo_b Up_b.
         // F = prod_{b < pb} P_b, G = prod_{b > pb} P_b; XA[a] = Lo_a prod_{pb < b < a} P_b carries
         // a column of this block to the middle of a later block a; own = Up_pb (lower half) or
-        // Lo_pb (upper half).
-        float Gf[4], cE[4], sf[4], XA[3][4];
+        // Lo_pb (upper half). pb is the same for a whole warp: each warp runs only its block's
+        // case, with no per-block predication.
+        float4 F, G, XA[3];
+        const float4 own = ld4(loup_s + (rb8 ^ 1) * kD + ch0);
         {
-            float F[4], own[4], dec[4], between[4];
+            float4 P[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                F[i] = Gf[i] = dec[i] = between[i] = 1.f;
-                own[i] = 1.f;
-                XA[0][i] = XA[1][i] = XA[2][i] = 0.f;
-            }
+            for (int bb = 0; bb < 4; ++bb)
+                P[bb] = mul4(ld4(loup_s + (2 * bb) * kD + ch0), ld4(loup_s + (2 * bb + 1) * kD + ch0));
+            auto setup = [&](auto pb_c) {
+                constexpr int PB = decltype(pb_c)::value;
+                F = G = make_float4(1.f, 1.f, 1.f, 1.f);
 #pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-                const float4 lo4 = *reinterpret_cast<const float4*>(loup_s + (bb * 2) * kD + ch0);
-                const float4 up4 = *reinterpret_cast<const float4*>(loup_s + (bb * 2 + 1) * kD + ch0);
-                const float lo[4] = {lo4.x, lo4.y, lo4.z, lo4.w};
-                const float up[4] = {up4.x, up4.y, up4.z, up4.w};
+                for (int bb = 0; bb < PB; ++bb) F = mul4(F, P[bb]);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float Pb = lo[i] * up[i];
-                    dec[i] *= Pb;
-                    if (bb < pb) F[i] *= Pb;
-                    if (bb > pb) {
-                        Gf[i] *= Pb;
-                        if (bb >= 1) XA[bb - 1][i] = lo[i] * between[i];
-                        between[i] *= Pb;
-                    }
-                    if (bb == pb) own[i] = hh == 0 ? up[i] : lo[i];
+                for (int bb = PB + 1; bb < 4; ++bb) G = mul4(G, P[bb]);
+                float4 between = make_float4(1.f, 1.f, 1.f, 1.f);
+#pragma unroll
+                for (int aa = PB + 1; aa < 4; ++aa) {
+                    XA[aa - 1] = mul4(ld4(loup_s + (2 * aa) * kD + ch0), between);
+                    between = mul4(between, P[aa]);
                 }
+            };
+            switch (pb) {
+                case 0: setup(std::integral_constant<int, 0>{}); break;
+                case 1: setup(std::integral_constant<int, 1>{}); break;
+                case 2: setup(std::integral_constant<int, 2>{}); break;
+                default: setup(std::integral_constant<int, 3>{}); break;
             }
             if (warp == 0)
                 *reinterpret_cast<float4*>(args.decay + rec * kD + ch0) =
-                    make_float4(dec[0], dec[1], dec[2], dec[3]);
-            // per row, with yi = 1 / y_j:
-            //   lower half: rho = yi, kappa = y_j, sigma = y_j own, e^{Gamma} = F tot yi
-            //   upper half: rho = y_j, kappa = yi, sigma = tot yi, e^{Gamma} = F own y_j
-            // so that sigma = kappa sf and e^{Gamma} = cE rho; the products below are taken from
-            // k rho, q rho and k kappa: K+ = (k rho) cE, Q+ = (q rho) cE, K_end = (k kappa) sf G,
-            // cross columns (k kappa) sf X_a
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                cE[i] = hh == 0 ? F[i] * tot[i] : F[i] * own[i];
-                sf[i] = hh == 0 ? own[i] : tot[i];
-                Gf[i] *= sf[i];
-                XA[0][i] *= sf[i];
-                XA[1][i] *= sf[i];
-                XA[2][i] *= sf[i];
-            }
+                    mul4(mul4(P[0], P[1]), mul4(P[2], P[3]));
         }
 
         // ---------------------------------------------------------------- operands
@@ -595,51 +605,76 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         //   C: k kappa (kappa = e^{Gamma_m - Gamma_r}), cross columns k sigma X_a, X_a <= 1
         //   K+ = k e^{Gamma} (shared), Q+ = q e^{Gamma} and K_end = k e^{Gamma_end - Gamma} =
         //   k G sigma (workspace)
+        // Per row, with yi = 1 / y_j:
+        //   lower half: rho = yi, kappa = y_j, sigma = y_j own, e^{Gamma} = F tot yi
+        //   upper half: rho = y_j, kappa = yi, sigma = tot yi, e^{Gamma} = F own y_j
+        // so that sigma = kappa sf and e^{Gamma} = cE rho, with sf = own (lower) or tot (upper)
+        // and cE = F tot (lower) or F own (upper). R, C and K_end take fp32 products of k rho,
+        // q rho, k kappa; K+ and Q+ are the bf16 products of the rounded k rho, q rho with cE
+        // (one bf16x2 multiply per two elements: the extra rounding does not move the result
+        // measurably, where rounding the factors of R, C or K_end would).
         if (!steep) {
             __nv_bfloat16* qplus = args.wq + ((size_t)rec * 128 + 64) * kD + ch0;
             __nv_bfloat16* kend = args.ke + (size_t)rec * kC * kD + ch0;
+            {
+                const bool kUpper = hh != 0;
+                const float totv[4] = {tot[0], tot[1], tot[2], tot[3]};
+                const float4 sf4 = kUpper ? make_float4(totv[0], totv[1], totv[2], totv[3]) : own;
+                const float4 cE4 = kUpper ? mul4(F, own) : mul4(F, make_float4(totv[0], totv[1],
+                                                                                totv[2], totv[3]));
+                const float4 gf4 = mul4(G, sf4);
+                const float gf[4] = {gf4.x, gf4.y, gf4.z, gf4.w};
+                float xa[3][4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int r = rbase + j;
-                const bool ok = r < L;   // rows past the document read as k = q = 0
-                const uint32_t ok_ = toff(128, rb8, j), oq_ = toff(128, rb8 + 8, j);
-                const uint2 kv = ok ? *reinterpret_cast<const uint2*>(sm + OFF_R + ok_)
-                                    : make_uint2(0u, 0u);
-                const uint2 qv = ok ? *reinterpret_cast<const uint2*>(sm + OFF_R + oq_)
-                                    : make_uint2(0u, 0u);
-                const float2 k01 = unpack_bf16(kv.x), k23 = unpack_bf16(kv.y);
-                const float2 q01 = unpack_bf16(qv.x), q23 = unpack_bf16(qv.y);
-                const float kk[4] = {k01.x, k01.y, k23.x, k23.y};
-                const float qq[4] = {q01.x, q01.y, q23.x, q23.y};
-                float kr[4], qr[4], kc[4];   // k rho, q rho, k kappa
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float yv = y[j][i];
-                    const float yi = __fdividef(1.f, yv);
-                    const float rho = hh == 0 ? yi : yv;
-                    const float kap = hh == 0 ? yv : yi;
-                    kr[i] = kk[i] * rho;
-                    qr[i] = qq[i] * rho;
-                    kc[i] = kk[i] * kap;
+                for (int aa = 0; aa < 3; ++aa) {
+                    const float4 x = mul4(XA[aa], sf4);
+                    xa[aa][0] = x.x; xa[aa][1] = x.y; xa[aa][2] = x.z; xa[aa][3] = x.w;
                 }
-                st_bf16x4(sm + OFF_R + toff(128, rb8, j), kr[0], kr[1], kr[2], kr[3]);
-                st_bf16x4(sm + OFF_R + toff(128, rb8 + 8, j), qr[0], qr[1], qr[2], qr[3]);
-                st_bf16x4(sm + OFF_C + toff(160, rb8, j), kc[0], kc[1], kc[2], kc[3]);
+                const __nv_bfloat162 cE01 = __floats2bfloat162_rn(cE4.x, cE4.y);
+                const __nv_bfloat162 cE23 = __floats2bfloat162_rn(cE4.z, cE4.w);
 #pragma unroll
-                for (int a = 1; a < 4; ++a) {
-                    if (a <= pb) continue;
-                    const float* xa = XA[a - 1];   // sf X_a
-                    st_bf16x4(sm + OFF_C + toff(160, rb8 + 8 + cross_off(a) / 8, j),
-                              kc[0] * xa[0], kc[1] * xa[1], kc[2] * xa[2], kc[3] * xa[3]);
+                for (int j = 0; j < 8; ++j) {
+                    const int r = rbase + j;
+                    const bool ok = r < L;   // rows past the document read as k = q = 0
+                    const uint2 kv = ok ? *reinterpret_cast<const uint2*>(sm + OFF_R + toff(128, rb8, j))
+                                        : make_uint2(0u, 0u);
+                    const uint2 qv = ok ? *reinterpret_cast<const uint2*>(sm + OFF_R + toff(128, rb8 + 8, j))
+                                        : make_uint2(0u, 0u);
+                    const float2 k01 = unpack_bf16(kv.x), k23 = unpack_bf16(kv.y);
+                    const float2 q01 = unpack_bf16(qv.x), q23 = unpack_bf16(qv.y);
+                    const float kk[4] = {k01.x, k01.y, k23.x, k23.y};
+                    const float qq[4] = {q01.x, q01.y, q23.x, q23.y};
+                    float kr[4], qr[4], kc[4];   // k rho, q rho, k kappa
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float yv = y[j][i];
+                        const float yi = __fdividef(1.f, yv);
+                        const float rho = kUpper ? yv : yi;
+                        const float kap = kUpper ? yi : yv;
+                        kr[i] = kk[i] * rho;
+                        qr[i] = qq[i] * rho;
+                        kc[i] = kk[i] * kap;
+                    }
+                    const uint2 krb = make_uint2(pack_bf16(kr[0], kr[1]), pack_bf16(kr[2], kr[3]));
+                    const uint2 qrb = make_uint2(pack_bf16(qr[0], qr[1]), pack_bf16(qr[2], qr[3]));
+                    *reinterpret_cast<uint2*>(sm + OFF_R + toff(128, rb8, j)) = krb;
+                    *reinterpret_cast<uint2*>(sm + OFF_R + toff(128, rb8 + 8, j)) = qrb;
+                    st_bf16x4(sm + OFF_C + toff(160, rb8, j), kc[0], kc[1], kc[2], kc[3]);
+#pragma unroll
+                    for (int aa = 1; aa < 4; ++aa) {
+                        if (aa <= pb) continue;
+                        const float* x = xa[aa - 1];   // sf X_a
+                        st_bf16x4(sm + OFF_C + toff(160, rb8 + 8 + cross_off(aa) / 8, j),
+                                  kc[0] * x[0], kc[1] * x[1], kc[2] * x[2], kc[3] * x[3]);
+                    }
+                    *reinterpret_cast<uint2*>(sm + OFF_KP + toff(64, rb8, j)) =
+                        make_uint2(hmul2_u32(krb.x, cE01), hmul2_u32(krb.y, cE23));
+                    *reinterpret_cast<uint2*>(qplus + (size_t)r * kD) =
+                        make_uint2(hmul2_u32(qrb.x, cE01), hmul2_u32(qrb.y, cE23));
+                    *reinterpret_cast<uint2*>(kend + (size_t)r * kD) =
+                        make_uint2(pack_bf16(kc[0] * gf[0], kc[1] * gf[1]),
+                                   pack_bf16(kc[2] * gf[2], kc[3] * gf[3]));
                 }
-                st_bf16x4(sm + OFF_KP + toff(64, rb8, j), kr[0] * cE[0], kr[1] * cE[1],
-                          kr[2] * cE[2], kr[3] * cE[3]);
-                *reinterpret_cast<uint2*>(qplus + (size_t)r * kD) =
-                    make_uint2(pack_bf16(qr[0] * cE[0], qr[1] * cE[1]),
-                               pack_bf16(qr[2] * cE[2], qr[3] * cE[3]));
-                *reinterpret_cast<uint2*>(kend + (size_t)r * kD) =   // Gf holds sf G
-                    make_uint2(pack_bf16(kc[0] * Gf[0], kc[1] * Gf[1]),
-                               pack_bf16(kc[2] * Gf[2], kc[3] * Gf[3]));
             }
         }
         if (!steep) {

@@ -22,9 +22,9 @@
 //   bf16(S^T) -> D (8 K steps) -> U^T -> S^T += U^T K_end (4 K steps);
 // the o product follows the update in the tensor pipe, off the chain. The decay of S^T, the load of
 // U~^T and the output of chunk c-1 (read from the other of two D buffers, staged in shared memory
-// and written by a TMA store) run while the D product of chunk c is in flight. Lane 0 of warp 1
-// issues the TMA loads (two stages: chunk c+1 arrives while chunk c runs) and lane 0 of warp 2 the
-// output stores. Every mbarrier wait is bounded; on expiry the CTA records KDA_ERR_TIMEOUT, drains
+// and written by a TMA store) run while the D product of chunk c is in flight. The MMA-issuing
+// thread also issues the TMA loads, while the D product runs (two stages: chunk c+1 arrives while
+// chunk c runs), and lane 0 of warp 2 the output stores. Every mbarrier wait is bounded; on expiry the CTA records KDA_ERR_TIMEOUT, drains
 // its own copies and MMAs, frees TMEM and exits.
 
 #include <cuda.h>
@@ -105,8 +105,8 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int qd = warp & 3, hs = warp >> 2;   // TMEM lane quarter, column half
     const int j = 32 * qd + lane;              // value column = TMEM lane
-    constexpr int kLoader = 32, kStorer = 64;  // threads that issue TMA loads / output stores
-    constexpr int kMma = 32 * kDataWarps;      // thread that issues the MMAs
+    constexpr int kStorer = 64;                // thread that issues the output stores
+    constexpr int kMma = 32 * kDataWarps;      // thread that issues the MMAs and the TMA loads
     const bool data = warp < kDataWarps;
     const int unit = blockIdx.x;
     const int h = unit % args.H;
@@ -248,7 +248,7 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         }
     };
 
-    if (tid == kLoader) {
+    if (tid == kMma) {
         if (nchunks > 0) issue(0);
         if (nchunks > 1) issue(1);
     }
@@ -288,7 +288,8 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         __syncthreads();
         tc_fence_after();
 
-        // ---------------------------------------------------------------- D = S^T [W; Q~]^T
+        // ---------------------------------------------------------------- D = S^T [W; Q+]^T
+        bool o_bad = false;
         if (tid == kMma) {
             tc_fence_after();
 #pragma unroll
@@ -296,14 +297,23 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
                 umma_f16_ts(tbase + TD + 128 * (c & 1), tbase + TB + 8 * s,
                             desc_at(dK, st + ST_WQ + (s >> 2) * 16384 + (s & 3) * 32), id1, s > 0);
             umma_commit(bar_mma1);
+            // Stage (c+1)&1 held chunk c-1, read by its update (waited for at this chunk's start)
+            // and its o product: once that is done, fetch chunk c+1 into it. This thread issues
+            // nothing else until the D product is waited for, so the copies (about 100 cycles to
+            // issue each) cost the chain nothing.
+            if (c >= 1 && c + 1 < nchunks) {
+                if (mbar_wait(bar_mma3, (uint32_t)((c - 1) & 1), args.budget)) issue(c + 1);
+                else o_bad = true;
+            }
         }
+        if (c >= 1 && c + 1 < nchunks) issued = c + 2;   // (an expired wait aborts below; the
+                                                         //  drain's waits are bounded)
         mma1_pending = true;
         mma1_chunk = c;
 
         // ---------------------------------------------------------------- while D runs
         // decay: TS = S^T diag(e^{Gamma_end}) (the update accumulates into it)
         uint32_t ub[16];
-        bool o_bad = false;
         if (data) {
             const float* dec = reinterpret_cast<const float*>(stp + ST_DEC) + 64 * hs;
 #pragma unroll
@@ -323,13 +333,8 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
                 ub[4 * m] = x.x; ub[4 * m + 1] = x.y; ub[4 * m + 2] = x.z; ub[4 * m + 3] = x.w;
             }
             if (c >= 1) o_bad = !stage_o(c - 1);
-            // stage (c+1)&1 held chunk c-1, read by its update (waited for at this chunk's start)
-            // and its o product (waited for in stage_o): fetch chunk c+1 into it
-            if (tid == kLoader && !o_bad && c >= 1 && c + 1 < nchunks) issue(c + 1);
             tmem_st_wait();
         }
-        if (c >= 1 && c + 1 < nchunks) issued = c + 2;   // (a wait that expired aborts below;
-                                                         //  the drain's wait is bounded)
         if (c >= 1) mma3_pending = false;   // (waited for above, or the CTA aborts below)
 
         if (!wait_all(bar_mma1, (uint32_t)(c & 1), o_bad)) { aborted = true; break; }
