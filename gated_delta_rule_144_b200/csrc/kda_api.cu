@@ -306,8 +306,8 @@ static kda_status_t fwd_impl(const kda_fwd_desc_t* d, const void* q, const void*
     p.bf16 = d->dtype == KDA_BF16;
     p.doc_order = nullptr;
     if ((st = device_error_word(&p.err)) != KDA_OK) return st;
-    // the epilogue runs as one bandwidth-bound pass after the prefill, on every path (measured
-    // faster than folding it into the split path's state pass, which is latency-bound)
+    // the epilogue: on the split path the state pass's epilogue warps apply it to the fp32 o as
+    // they store it; the other paths run it as one bandwidth-bound pass over o afterwards
     auto norm_after = [&]() -> cudaError_t {
         if (!norm || !tokens) return cudaSuccess;
         return kda::launch_out_norm_gated(o, norm->gate, norm->weight, norm->eps, o,
@@ -340,13 +340,21 @@ static kda_status_t fwd_impl(const kda_fwd_desc_t* d, const void* q, const void*
             e = kda::launch_chunk_map(cu_seqlens, d->num_seqs, d->T, L.G, ws.map, p.err, s);
             if (e != cudaSuccess) return cuda_fail(e, "kda_fwd chunk map");
         }
+        kda::ScanNorm sn{};
+        const kda::ScanNorm* snp = nullptr;
+        if (norm) {
+            sn.gate = norm->gate;
+            sn.weight = norm->weight;
+            sn.eps = norm->eps;
+            snp = &sn;
+        }
         const int S = cu_seqlens ? 1 : split_segments(L.ncT);
         e = cudaMemsetAsync(ws.counters, 0, sizeof(unsigned long long) * S, s);
         if (e != cudaSuccess) return cuda_fail(e, "kda_fwd workspace counters");
         if (S == 1) {
             e = kda::launch_chunk64_intra(p, 0, L.ncT, ws.counters, s);
             if (e != cudaSuccess) return cuda_fail(e, "kda_fwd intra-chunk launch");
-            e = kda::launch_chunk_scan(p, kda::ScanSegment{0, L.ncT, h0, hT}, s);
+            e = kda::launch_chunk_scan(p, kda::ScanSegment{0, L.ncT, h0, hT}, s, snp);
             if (e != cudaSuccess) return cuda_fail(e, "kda_fwd state-pass launch");
         } else {
             // intra(0) intra(1) ... on the caller's stream; state(i) on the side stream after
@@ -363,7 +371,7 @@ static kda_status_t fwd_impl(const kda_fwd_desc_t* d, const void* q, const void*
                         cudaSuccess ||
                     (e = cudaEventRecord(ss->seg[i], s)) != cudaSuccess ||
                     (e = cudaStreamWaitEvent(ss->aux, ss->seg[i], 0)) != cudaSuccess ||
-                    (e = kda::launch_chunk_scan(p, seg, ss->aux)) != cudaSuccess)
+                    (e = kda::launch_chunk_scan(p, seg, ss->aux, snp)) != cudaSuccess)
                     first = e;
             }
             // join even after a failed launch, so that nothing is left pending on the side stream
@@ -372,8 +380,6 @@ static kda_status_t fwd_impl(const kda_fwd_desc_t* d, const void* q, const void*
             if (first != cudaSuccess) return cuda_fail(first, "kda_fwd split launch");
             if (e != cudaSuccess) return cuda_fail(e, "kda_fwd side stream join");
         }
-        e = norm_after();
-        if (e != cudaSuccess) return cuda_fail(e, "kda_fwd output norm launch");
         return KDA_OK;
     }
     if (need_ws > 0 && tokens) {

@@ -107,7 +107,15 @@ cudaError_t launch_chunk_map(const int32_t* cu_seqlens, int N, int T, long long 
 // which must be zero at launch.
 cudaError_t launch_chunk64_intra(const FwdParams& p, int c_begin, int c_span,
                                  unsigned long long* counter, cudaStream_t stream);
-cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaStream_t stream);
+// Gated RMSNorm applied by the state pass to its output (y = o / sqrt(mean(o^2) + eps) * weight *
+// sigmoid(gate) per (token, head)), instead of a separate pass over o.
+struct ScanNorm {
+    const void* gate;      // shaped and typed like o
+    const float* weight;   // [128]
+    float eps;
+};
+cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaStream_t stream,
+                              const ScanNorm* norm = nullptr);
 // y = x / sqrt(mean(x^2) + eps) * w * sigmoid(gate) per vector of dv elements (dv <= 256);
 // y may alias x.
 cudaError_t launch_out_norm_gated(const void* x, const void* gate, const float* w, float eps,

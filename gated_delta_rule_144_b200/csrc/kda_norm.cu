@@ -13,6 +13,11 @@ namespace {
 
 constexpr int kWarps = 8;
 
+// sigmoid(g) = 1 / (1 + e^{-g}) with the fast exponential and reciprocal intrinsics (about 2 ulp
+// each); exactly the arithmetic of the state pass's fused epilogue (kda_scan.cu), so that both
+// give the same bits.
+__device__ __forceinline__ float sigmoid_fast(float g) { return __fdividef(1.f, 1.f + __expf(-g)); }
+
 __device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
     const float4 x = *reinterpret_cast<const float4*>(p);
     v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
@@ -77,11 +82,11 @@ out_norm_gated_kernel(const T* x, const T* __restrict__ gate, const float* __res
             const float4 wv = *reinterpret_cast<const float4*>(w + c);
             const float ws[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) out[e] = xv[i][e] * inv * ws[e] / (1.f + __expf(-g[e]));
+            for (int e = 0; e < 4; ++e) out[e] = xv[i][e] * inv * ws[e] * sigmoid_fast(g[e]);
             store4(y + base + c, out);
         } else {
             const float g = load_elem(gate, base + c);
-            store_elem(y, base + c, xv[i][0] * inv * w[c] / (1.f + __expf(-g)));
+            store_elem(y, base + c, xv[i][0] * inv * w[c] * sigmoid_fast(g));
         }
     }
 }

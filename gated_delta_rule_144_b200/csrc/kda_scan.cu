@@ -9,6 +9,9 @@
 // gated delta rule; GLM-5.3-Flash model card, Kimi Delta Attention snippet, and the state-passing
 // identity it implies):
 //   U = U~ - W S,   o = Q+ S + A_qk U,   S <- diag(e^{Gamma_end}) S + K_end^T U.
+// With a gated RMSNorm epilogue (NeMo glm5_next layers, _TorchRMSNormGated) the kernel writes
+// y = o / sqrt(mean over the head's value columns of o^2 + eps) * w * sigmoid(gate) instead of o,
+// from o rounded to bf16, in the same arithmetic as the separate pass (kda_norm.cu).
 //
 // Layout: the state is kept transposed, S^T [value column j][key channel c], in TMEM lane j, so
 // every product takes its state-side operand from TMEM and no shared-memory write sits on the
@@ -16,16 +19,25 @@
 //   D = S^T [W; Q+]^T     (A = bf16 copy of S^T in TMEM, B = [W; Q+] K-major in shared memory)
 //   S^T += U^T K_end      (A = bf16 U^T in TMEM, B = K_end MN-major in shared memory)
 //   o^T = (Q+ S)^T + U^T A_qk^T   (accumulated into D's second half; A = U^T, B = A_qk K-major)
-// Eight data warps: warps w and w + 4 share TMEM lane quarter w mod 4 (lane j = value column j)
-// and split the columns of every TMEM row between them. A ninth warp only issues the MMAs, so that
-// no MMA issue waits behind a data warp's work. Per chunk c the critical chain is
-//   bf16(S^T) -> D (8 K steps) -> U^T -> S^T += U^T K_end (4 K steps);
-// the o product follows the update in the tensor pipe, off the chain. The decay of S^T, the load of
-// U~^T and the output of chunk c-1 (read from the other of two D buffers, staged in shared memory
-// and written by a TMA store) run while the D product of chunk c is in flight. The MMA-issuing
-// thread also issues the TMA loads, while the D product runs (two stages: chunk c+1 arrives while
-// chunk c runs), and lane 0 of warp 2 the output stores. Every mbarrier wait is bounded; on expiry the CTA records KDA_ERR_TIMEOUT, drains
-// its own copies and MMAs, frees TMEM and exits.
+//
+// Roles (14 warps):
+//   - 8 chain warps walk the chunks: warps w and w + 4 share TMEM lane quarter w mod 4 (lane j =
+//     value column j) and split the columns of every TMEM row between them. Per chunk c the chain
+//     is bf16(S^T) -> D (8 K steps) -> U^T = U~^T - (W S)^T -> S^T += U^T K_end (4 K steps); the
+//     decay of S^T and the load of U~^T run while D is in flight.
+//   - 1 MMA warp: one thread issues every tcgen05.mma.
+//   - 4 epilogue warps (one per lane quarter) take o of chunk c out of TMEM once its product is
+//     done, stage it row-major in shared memory (applying the norm when asked, with the gate
+//     tile of chunk c fetched by TMA a chunk ahead) and store it, so that none of the output's
+//     work sits on the chain. The D buffers are double-buffered: the MMA thread issues chunk c's
+//     D product once the epilogue has read chunk c-2's.
+//   - 1 loader warp: one thread issues the TMA copies of the records (two stages): chunk c+2's
+//     as soon as chunk c's o product is done, which frees chunk c's stage (its update precedes
+//     it), a whole chunk before they are needed (a record takes about 2.5 K cycles to land,
+//     and issuing its copies about 650).
+// The chain warps and the MMA warp synchronise with named barrier 1, the epilogue warps with named
+// barrier 2, and the two groups only through mbarriers. Every mbarrier wait is bounded; on expiry
+// the CTA records KDA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -46,19 +58,28 @@ using namespace sm100;
 constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr int kDataWarps = 8;
-constexpr int kThreads = 32 * kDataWarps + 32;   // + one warp that only issues MMAs
+constexpr int kEpiWarps = 4;
+constexpr int kChainThreads = 32 * kDataWarps + 32;          // chain warps + the MMA warp
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = kChainThreads + kEpiThreads + 32;     // + the loader warp
+constexpr int kMma = 32 * kDataWarps;    // thread that issues the MMAs
+constexpr int kEpi0 = kChainThreads;     // first epilogue thread (issues the output stores)
+constexpr int kLoader = kChainThreads + kEpiThreads;   // thread that issues the record copies
+constexpr uint32_t kBarChain = 1, kBarEpi = 2;   // named barriers (0 is __syncthreads)
 
 // one pipeline stage (bytes from a 1024-aligned stage base)
-constexpr uint32_t ST_WQ = 0;        // [W; Q~] 128 x 128 bf16, K-major SW128: 2 panels of 16 KB
+constexpr uint32_t ST_WQ = 0;        // [W; Q+] 128 x 128 bf16, K-major SW128: 2 panels of 16 KB
 constexpr uint32_t ST_KE = 32768;    // K_end 64 x 128 bf16, MN-major SW128: 2 panels of 8 KB
 constexpr uint32_t ST_UT = 49152;    // U~^T [128 j][64 tokens] bf16, SW128
 constexpr uint32_t ST_AQ = 65536;    // A_qk [64 r][64 i] bf16, K-major SW128
 constexpr uint32_t ST_DEC = 73728;   // e^{Gamma_end} [128] f32
 constexpr uint32_t kStage = 74752;   // 73 KB, a multiple of 1024
 constexpr uint32_t kTxStage = 32768 + 2 * 16384 + 8192 + 512;
-constexpr uint32_t OFF_O = 2 * kStage;       // two output tiles o [64 tokens][128] bf16
-constexpr uint32_t OFF_BAR = OFF_O + 32768;  // full[2], mma1, mma2, never, mma3
-constexpr uint32_t OFF_TMEM = OFF_BAR + 64;
+constexpr uint32_t OFF_G = 2 * kStage;       // two norm gate tiles [64 tokens][128] bf16
+constexpr uint32_t OFF_Y = OFF_G + 32768;    // two output tiles [64 tokens][128] bf16
+constexpr uint32_t OFF_BAR = OFF_Y + 32768;  // mbarriers
+constexpr uint32_t OFF_FLAG = OFF_BAR + 128; // set when the chain aborts
+constexpr uint32_t OFF_TMEM = OFF_FLAG + 16;
 constexpr uint32_t kSmemBytes = OFF_TMEM + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -76,8 +97,11 @@ struct ScanArgs {
     const float* h0;        // state at chunk c_begin (nullable: zero)
     float* hT;              // state after chunk c_end - 1 (nullable: not written)
     int c_begin, c_end;     // chunks of every chain this launch walks
-    __nv_bfloat16* o;
+    __nv_bfloat16* o;       // o, or y with the norm
     const float* decay;     // [R][128]
+    const __nv_bfloat16* gate;   // norm gate, shaped like o (nullable: no norm)
+    const float* nw;             // norm weight [128]
+    float eps;
     int T, H, N, ncT;       // ncT: chunk records per sequence when cu is null
     long long G;            // chunk records per head
     long long budget;
@@ -86,7 +110,7 @@ struct ScanArgs {
 };
 
 struct ScanMaps {
-    CUtensorMap wq, ke, ut, aq, o;
+    CUtensorMap wq, ke, ut, aq, o, g;   // g: the norm gate, shaped like o (unused without it)
 };
 
 __device__ __forceinline__ uint32_t pack2(float x, float y) {
@@ -96,6 +120,26 @@ __device__ __forceinline__ uint32_t pack2(float x, float y) {
 __device__ __forceinline__ float lo_bf(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float hi_bf(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 
+// Named barrier over `count` threads (a multiple of 32), and the same with an OR of `pred`.
+__device__ __forceinline__ void bar_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool bar_or(uint32_t id, uint32_t count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
     extern __shared__ uint8_t smem_raw[];
@@ -103,11 +147,12 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
                                              ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int qd = warp & 3, hs = warp >> 2;   // TMEM lane quarter, column half
+    const int qd = warp & 3;                   // TMEM lane quarter (every role)
+    const int hs = (warp >> 2) & 1;            // chain warps: column half
     const int j = 32 * qd + lane;              // value column = TMEM lane
-    constexpr int kStorer = 64;                // thread that issues the output stores
-    constexpr int kMma = 32 * kDataWarps;      // thread that issues the MMAs and the TMA loads
     const bool data = warp < kDataWarps;
+    const bool epi = tid >= kEpi0 && tid < kLoader;
+    const bool loader = tid >= kLoader;
     const int unit = blockIdx.x;
     const int h = unit % args.H;
     const int n = args.order ? args.order[unit / args.H] : unit / args.H;
@@ -141,21 +186,33 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
     const int nchunks = (int)((t1 - t0 + kC - 1) / kC);
 
     uint32_t* tmem_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
-    const uint32_t bar_full0 = sb + OFF_BAR, bar_mma1 = bar_full0 + 16, bar_mma2 = bar_full0 + 24;
-    const uint32_t bar_never = bar_full0 + 32, bar_mma3 = bar_full0 + 40;
+    volatile int* abort_s = reinterpret_cast<volatile int*>(sm + OFF_FLAG);
+    const uint32_t bar_full0 = sb + OFF_BAR;                       // + 8 (c & 1)
+    const uint32_t bar_mma1 = bar_full0 + 16, bar_mma2 = bar_full0 + 24;
+    const uint32_t bar_never = bar_full0 + 32;
+    const uint32_t bar_o0 = bar_full0 + 40;      // + 8 (c & 1): o product of chunk c done
+    const uint32_t bar_dfree0 = bar_full0 + 56;  // + 8 (c & 1): epilogue has read D buffer c & 1
+    const uint32_t bar_gate0 = bar_full0 + 72;   // + 8 (c & 1): gate tile of chunk c landed
     if (tid == 0) {
         mbar_init(bar_full0, 1);
         mbar_init(bar_full0 + 8, 1);
         mbar_init(bar_mma1, 1);
         mbar_init(bar_mma2, 1);
         mbar_init(bar_never, 1);
-        mbar_init(bar_mma3, 1);
+        mbar_init(bar_o0, 1);
+        mbar_init(bar_o0 + 8, 1);
+        mbar_init(bar_dfree0, kEpiThreads);
+        mbar_init(bar_dfree0 + 8, kEpiThreads);
+        mbar_init(bar_gate0, 1);
+        mbar_init(bar_gate0 + 8, 1);
+        *abort_s = 0;
         fence_mbar_init();
         prefetch_tmap(&maps.wq);
         prefetch_tmap(&maps.ke);
         prefetch_tmap(&maps.ut);
         prefetch_tmap(&maps.aq);
         prefetch_tmap(&maps.o);
+        if (args.gate) prefetch_tmap(&maps.g);
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(tmem_s), kTmemCols);
@@ -180,6 +237,7 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
     }
     tmem_st_wait();
 
+    // records of chunk c into stage c & 1 (issued by the loader thread)
     auto issue = [&](int c) {
         const uint32_t st = sb + (uint32_t)(c & 1) * kStage;
         const uint32_t bar = bar_full0 + 8 * (c & 1);
@@ -194,232 +252,321 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         bulk_load(st + ST_DEC, args.decay + rec * kD, 512, bar);
     };
 
-    const uint64_t dK = sw128_desc(0, 16, 1024);     // K-major, 128B swizzle
-    const uint64_t dM8 = sw128_desc(0, 8192, 1024);  // MN-major, 64-row panels
-    const uint32_t id1 = idesc_bf16(128, 128, 0, 0);
-    const uint32_t id2 = idesc_bf16(128, 128, 0, 1);
-    const uint32_t id3 = idesc_bf16(128, 64, 0, 0);
-
-    // outstanding asynchronous work, drained before exit if a wait expires
-    int issued = 0;          // chunks whose copies were issued
-    int landed = 0;          // chunks whose copies were waited for
-    bool mma1_pending = false, mma2_pending = false, mma3_pending = false;
-    int mma1_chunk = 0, mma2_chunk = 0, mma3_chunk = 0;   // chunk of the last commit (parity)
-    bool aborted = false;
-    // One thread polls; the rest of the CTA waits at the barrier that publishes the outcome (and
-    // any failure a thread has recorded in `also_bad` since the last barrier).
-    auto wait_all = [&](uint32_t bar, uint32_t parity, bool also_bad = false) -> bool {
-        const bool ok = tid != 0 || mbar_wait(bar, parity, args.budget);
-        return __syncthreads_or(!ok || also_bad) == 0;
-    };
-
-    // o of chunk cc (rows < L): o^T = (Q+ S)^T + U^T A_qk^T from D buffer cc & 1 (this thread's
-    // 32 tokens), staged row-major in output tile cc & 1. Waits (every data thread, bounded) for
-    // the o product of chunk cc; returns false if that wait expired.
-    auto stage_o = [&](int cc) -> bool {
-        const bool ok = mbar_wait(bar_mma3, (uint32_t)(cc & 1), args.budget);
-        tc_fence_after();
-        float w[32];
-        tmem_ld32(tbase + lq + TD + 128 * (cc & 1) + 64 + 32 * hs, w);
-        tmem_ld_wait();
-        __nv_bfloat16* tile = reinterpret_cast<__nv_bfloat16*>(sm + OFF_O + 16384 * (cc & 1));
-#pragma unroll
-        for (int i = 0; i < 32; ++i) tile[(32 * hs + i) * kD + j] = __float2bfloat16_rn(w[i]);
-        return ok;
-    };
-    // write staged tile cc to o: one TMA store for a full chunk, row copies for a partial one
-    // (a TMA box would run into the next document's rows). Call after a CTA barrier that
-    // follows fence_proxy_async by the writers.
-    auto flush_o = [&](int cc) {
-        const long long r0 = t0 + (long long)kC * cc;
-        const int L = (int)min((long long)kC, t1 - r0);
-        if (L == kC) {
-            if (tid == kStorer) {
-                tma_store_3d(&maps.o, sb + OFF_O + 16384 * (cc & 1), 0, h, (int)r0);
-                bulk_commit();
+    if (loader) {
+        // ============================================================ loader warp
+        // chunk c's stage is free once its o product is done (its update precedes it): chunk
+        // c+2's records go there. After a chain abort the wait expires and the loader stops.
+        if (tid == kLoader) {
+            int last0 = -1, last1 = -1;   // the chunk whose records went last into each stage
+            if (nchunks > 0) issue(0), last0 = 0;
+            if (nchunks > 1) issue(1), last1 = 1;
+            for (int c = 0; c + 2 < nchunks; ++c) {
+                if (!mbar_wait(bar_o0 + 8 * (c & 1), (uint32_t)((c >> 1) & 1), args.budget)) break;
+                issue(c + 2);
+                if (c & 1) last1 = c + 2;
+                else last0 = c + 2;
             }
-        } else {
-            const uint4* src = reinterpret_cast<const uint4*>(sm + OFF_O + 16384 * (cc & 1));
-            for (int i = tid; i < L * 16; i += kThreads) {
-                const int r = i >> 4, q = i & 15;
-                *reinterpret_cast<uint4*>(args.o + ((size_t)(r0 + r) * args.H + h) * kD + 8 * q) =
-                    src[r * 16 + q];
-            }
+            // copies still in flight land before the smem goes away (bounded; earlier copies
+            // were waited for by the chain, and a completed phase returns at once)
+            if (last0 >= 0) mbar_wait(bar_full0, (uint32_t)((last0 >> 1) & 1), 1ll << 31);
+            if (last1 >= 0) mbar_wait(bar_full0 + 8, (uint32_t)((last1 >> 1) & 1), 1ll << 31);
         }
-    };
+    } else if (!epi) {
+        // ============================================================ chain warps and MMA warp
+        const uint64_t dK = sw128_desc(0, 16, 1024);     // K-major, 128B swizzle
+        const uint64_t dM8 = sw128_desc(0, 8192, 1024);  // MN-major, 64-row panels
+        const uint32_t id1 = idesc_bf16(128, 128, 0, 0);
+        const uint32_t id2 = idesc_bf16(128, 128, 0, 1);
+        const uint32_t id3 = idesc_bf16(128, 64, 0, 0);
 
-    if (tid == kMma) {
-        if (nchunks > 0) issue(0);
-        if (nchunks > 1) issue(1);
-    }
-    issued = min(nchunks, 2);
-    if (args.debug_stall && !wait_all(bar_never, 0)) aborted = true;
+        // outstanding MMAs, drained before exit if a wait expires (the record copies are the
+        // epilogue's to drain)
+        bool mma1_pending = false, mma2_pending = false, o_pending = false;
+        int mma1_chunk = 0, mma2_chunk = 0, o_chunk = 0;   // chunk of the last commit
+        bool aborted = false;
+        // thread 0 polls; the chain waits at the barrier that publishes the outcome (and any
+        // failure a thread has recorded in `also_bad` since the last barrier)
+        auto wait_chain = [&](uint32_t bar, uint32_t parity, bool also_bad) -> bool {
+            const bool ok = tid != 0 || mbar_wait(bar, parity, args.budget);
+            return !bar_or(kBarChain, kChainThreads, !ok || also_bad);
+        };
 
-    for (int c = 0; c < nchunks && !aborted; ++c) {
-        const uint32_t st = sb + (uint32_t)(c & 1) * kStage;
-        const uint8_t* stp = sm + (size_t)(c & 1) * kStage;
+        if (args.debug_stall && !wait_chain(bar_never, 0, false)) aborted = true;
 
-        if (!wait_all(bar_full0 + 8 * (c & 1), (uint32_t)((c >> 1) & 1))) { aborted = true; break; }
-        landed = c + 1;
-        if (mma2_pending) {   // S of chunk c is complete once the previous update has landed
-            if (!wait_all(bar_mma2, (uint32_t)(mma2_chunk & 1))) { aborted = true; break; }
+        for (int c = 0; c < nchunks && !aborted; ++c) {
+            const uint32_t st = sb + (uint32_t)(c & 1) * kStage;
+            const uint8_t* stp = sm + (size_t)(c & 1) * kStage;
+
+            // records of chunk c landed; S of chunk c complete once the previous update has
+            bool ok = true;
+            if (tid == 0) {
+                ok = mbar_wait(bar_full0 + 8 * (c & 1), (uint32_t)((c >> 1) & 1), args.budget);
+                if (ok && mma2_pending)
+                    ok = mbar_wait(bar_mma2, (uint32_t)(mma2_chunk & 1), args.budget);
+            }
+            if (bar_or(kBarChain, kChainThreads, !ok)) { aborted = true; break; }
             mma2_pending = false;
-        }
-        tc_fence_after();
-
-        // ---------------------------------------------------------------- bf16 S^T -> TB
-        float va[32], vb[32];
-        if (data) {
-            tmem_ld32(tbase + lq + TS + 64 * hs, va);
-            tmem_ld32(tbase + lq + TS + 64 * hs + 32, vb);
-            tmem_ld_wait();
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pk[i] = pack2(va[2 * i], va[2 * i + 1]);
-            tmem_st16u(tbase + lq + TB + 32 * hs, pk);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pk[i] = pack2(vb[2 * i], vb[2 * i + 1]);
-            tmem_st16u(tbase + lq + TB + 32 * hs + 16, pk);
-            tmem_st_wait();
-        }
-        // output tile (c-1)&1 is rewritten below; its previous store (chunk c-3) must be done
-        if (tid == kStorer && c >= 3) bulk_wait_read_le1();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-
-        // ---------------------------------------------------------------- D = S^T [W; Q+]^T
-        bool o_bad = false;
-        if (tid == kMma) {
             tc_fence_after();
+
+            // ------------------------------------------------------------ bf16 S^T -> TB
+            if (data) {
+                float va[32], vb[32];
+                tmem_ld32(tbase + lq + TS + 64 * hs, va);
+                tmem_ld32(tbase + lq + TS + 64 * hs + 32, vb);
+                tmem_ld_wait();
+                uint32_t pk[16];
 #pragma unroll
-            for (int s = 0; s < kD / 16; ++s)
-                umma_f16_ts(tbase + TD + 128 * (c & 1), tbase + TB + 8 * s,
-                            desc_at(dK, st + ST_WQ + (s >> 2) * 16384 + (s & 3) * 32), id1, s > 0);
-            umma_commit(bar_mma1);
-            // Stage (c+1)&1 held chunk c-1, read by its update (waited for at this chunk's start)
-            // and its o product: once that is done, fetch chunk c+1 into it. This thread issues
-            // nothing else until the D product is waited for, so the copies (about 100 cycles to
-            // issue each) cost the chain nothing.
-            if (c >= 1 && c + 1 < nchunks) {
-                if (mbar_wait(bar_mma3, (uint32_t)((c - 1) & 1), args.budget)) issue(c + 1);
-                else o_bad = true;
+                for (int i = 0; i < 16; ++i) pk[i] = pack2(va[2 * i], va[2 * i + 1]);
+                tmem_st16u(tbase + lq + TB + 32 * hs, pk);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk[i] = pack2(vb[2 * i], vb[2 * i + 1]);
+                tmem_st16u(tbase + lq + TB + 32 * hs + 16, pk);
+                tmem_st_wait();
             }
-        }
-        if (c >= 1 && c + 1 < nchunks) issued = c + 2;   // (an expired wait aborts below; the
-                                                         //  drain's waits are bounded)
-        mma1_pending = true;
-        mma1_chunk = c;
-
-        // ---------------------------------------------------------------- while D runs
-        // decay: TS = S^T diag(e^{Gamma_end}) (the update accumulates into it)
-        uint32_t ub[16];
-        if (data) {
-            const float* dec = reinterpret_cast<const float*>(stp + ST_DEC) + 64 * hs;
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-                const float4 d0 = *reinterpret_cast<const float4*>(dec + i);
-                const float4 d1 = *reinterpret_cast<const float4*>(dec + 32 + i);
-                va[i] *= d0.x; va[i + 1] *= d0.y; va[i + 2] *= d0.z; va[i + 3] *= d0.w;
-                vb[i] *= d1.x; vb[i + 1] *= d1.y; vb[i + 2] *= d1.z; vb[i + 3] *= d1.w;
-            }
-            tmem_st32(tbase + lq + TS + 64 * hs, va);
-            tmem_st32(tbase + lq + TS + 64 * hs + 32, vb);
-            // U~^T of this chunk: row j, tokens [32 hs, +32)
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const uint4 x = *reinterpret_cast<const uint4*>(
-                    stp + ST_UT + sw128_off(128, j, 32 * hs + 8 * m));
-                ub[4 * m] = x.x; ub[4 * m + 1] = x.y; ub[4 * m + 2] = x.z; ub[4 * m + 3] = x.w;
-            }
-            if (c >= 1) o_bad = !stage_o(c - 1);
-            tmem_st_wait();
-        }
-        if (c >= 1) mma3_pending = false;   // (waited for above, or the CTA aborts below)
-
-        if (!wait_all(bar_mma1, (uint32_t)(c & 1), o_bad)) { aborted = true; break; }
-        mma1_pending = false;
-        tc_fence_after();
-
-        // ---------------------------------------------------------------- U^T = U~^T - (W S)^T
-        if (data) {
-            float w[32];
-            tmem_ld32(tbase + lq + TD + 128 * (c & 1) + 32 * hs, w);
-            tmem_ld_wait();
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                pk[i] = pack2(lo_bf(ub[i]) - w[2 * i], hi_bf(ub[i]) - w[2 * i + 1]);
-            tmem_st16u(tbase + lq + TU + 16 * hs, pk);
-        }
-        if (data) tmem_st_wait();
-        fence_proxy_async();   // output tile c-1 -> TMA store
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-
-        // ---------------------------------------------------------------- S^T += U^T K_end
-        if (tid == kMma) {
+            tc_fence_before();
+            bar_sync(kBarChain, kChainThreads);
             tc_fence_after();
-#pragma unroll
-            for (int s = 0; s < kC / 16; ++s)
-                umma_f16_ts(tbase + TS, tbase + TU + 8 * s, desc_at(dM8, st + ST_KE + 2048 * s),
-                            id2, 1);
-            umma_commit(bar_mma2);
-            // o^T = (Q+ S)^T + U^T A_qk^T, behind the update in the pipe (off the chain)
-#pragma unroll
-            for (int s = 0; s < kC / 16; ++s)
-                umma_f16_ts(tbase + TD + 128 * (c & 1) + 64, tbase + TU + 8 * s,
-                            desc_at(dK, st + ST_AQ + 32 * s), id3, 1);
-            umma_commit(bar_mma3);
-        }
-        mma2_pending = mma3_pending = true;
-        mma2_chunk = mma3_chunk = c;
-        if (c >= 1) flush_o(c - 1);
-    }
 
-    if (aborted) {
-        if (tid == 0) set_device_error(args.err, DEV_TIMEOUT);
-        // wind down: this CTA's own copies and MMAs finish before TMEM and smem go away
-        const long long drain = 1ll << 31;
-        for (int c = landed; c < issued; ++c)
-            mbar_wait(bar_full0 + 8 * (c & 1), (uint32_t)((c >> 1) & 1), drain);
-        if (mma1_pending) mbar_wait(bar_mma1, (uint32_t)(mma1_chunk & 1), drain);
-        if (mma2_pending) mbar_wait(bar_mma2, (uint32_t)(mma2_chunk & 1), drain);
-        if (mma3_pending) mbar_wait(bar_mma3, (uint32_t)(mma3_chunk & 1), drain);
-        __syncthreads();
-    } else {
-        if (mma2_pending && !wait_all(bar_mma2, (uint32_t)(mma2_chunk & 1))) {
-            if (tid == 0) set_device_error(args.err, DEV_TIMEOUT);
-            mbar_wait(bar_mma2, (uint32_t)(mma2_chunk & 1), 1ll << 31);
-        }
-        tc_fence_after();
-        if (nchunks > 0) {   // output of the last chunk
-            if (tid == kStorer && nchunks >= 3) bulk_wait_read_le1();
-            __syncthreads();
-            bool bad = false;
-            if (data) bad = !stage_o(nchunks - 1);
-            fence_proxy_async();
-            if (__syncthreads_or(bad)) {
-                if (tid == 0) set_device_error(args.err, DEV_TIMEOUT);
-                mbar_wait(bar_mma3, (uint32_t)((nchunks - 1) & 1), 1ll << 31);
-            } else {
-                flush_o(nchunks - 1);
+            // ------------------------------------------------------------ D = S^T [W; Q+]^T
+            bool mma_bad = false;
+            if (tid == kMma) {
+                // D buffer c & 1 last held chunk c-2's product: wait until the epilogue has
+                // read its o (long done in steady state)
+                if (c >= 2)
+                    mma_bad = !mbar_wait(bar_dfree0 + 8 * (c & 1), (uint32_t)(((c - 2) >> 1) & 1),
+                                         args.budget);
+                if (!mma_bad) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int s = 0; s < kD / 16; ++s)
+                        umma_f16_ts(tbase + TD + 128 * (c & 1), tbase + TB + 8 * s,
+                                    desc_at(dK, st + ST_WQ + (s >> 2) * 16384 + (s & 3) * 32),
+                                    id1, s > 0);
+                    umma_commit(bar_mma1);
+                }
             }
-        }
-        if (args.hT && data) {
-#pragma unroll 1
-            for (int p = 0; p < 2; ++p) {
-                float v[32];
-                const int c0 = 64 * hs + 32 * p;
-                tmem_ld32(tbase + lq + TS + c0, v);
+            mma1_pending = true;
+            mma1_chunk = c;
+
+            // ------------------------------------------------------------ while D runs
+            // decay: TS = S^T diag(e^{Gamma_end}) (the update accumulates into it); U~^T rows
+            uint32_t ub[16];
+            if (data) {
+                float va[32], vb[32];
+                tmem_ld32(tbase + lq + TS + 64 * hs, va);
+                tmem_ld32(tbase + lq + TS + 64 * hs + 32, vb);
+                const float* dec = reinterpret_cast<const float*>(stp + ST_DEC) + 64 * hs;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const uint4 x = *reinterpret_cast<const uint4*>(
+                        stp + ST_UT + sw128_off(128, j, 32 * hs + 8 * m));
+                    ub[4 * m] = x.x; ub[4 * m + 1] = x.y; ub[4 * m + 2] = x.z; ub[4 * m + 3] = x.w;
+                }
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) args.hT[state_base + (size_t)(c0 + i) * kD + j] = v[i];
+                for (int i = 0; i < 32; i += 4) {
+                    const float4 d0 = *reinterpret_cast<const float4*>(dec + i);
+                    const float4 d1 = *reinterpret_cast<const float4*>(dec + 32 + i);
+                    va[i] *= d0.x; va[i + 1] *= d0.y; va[i + 2] *= d0.z; va[i + 3] *= d0.w;
+                    vb[i] *= d1.x; vb[i + 1] *= d1.y; vb[i + 2] *= d1.z; vb[i + 3] *= d1.w;
+                }
+                tmem_st32(tbase + lq + TS + 64 * hs, va);
+                tmem_st32(tbase + lq + TS + 64 * hs + 32, vb);
+                tmem_st_wait();
+            }
+
+            if (!wait_chain(bar_mma1, (uint32_t)(c & 1), mma_bad)) { aborted = true; break; }
+            mma1_pending = false;
+            tc_fence_after();
+
+            // ------------------------------------------------------------ U^T = U~^T - (W S)^T
+            if (data) {
+                float w[32];
+                tmem_ld32(tbase + lq + TD + 128 * (c & 1) + 32 * hs, w);
+                tmem_ld_wait();
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack2(lo_bf(ub[i]) - w[2 * i], hi_bf(ub[i]) - w[2 * i + 1]);
+                tmem_st16u(tbase + lq + TU + 16 * hs, pk);
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            bar_sync(kBarChain, kChainThreads);
+            tc_fence_after();
+
+            // ------------------------------------------------------------ S^T += U^T K_end
+            if (tid == kMma) {
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < kC / 16; ++s)
+                    umma_f16_ts(tbase + TS, tbase + TU + 8 * s,
+                                desc_at(dM8, st + ST_KE + 2048 * s), id2, 1);
+                umma_commit(bar_mma2);
+                // o^T = (Q+ S)^T + U^T A_qk^T, behind the update in the pipe (off the chain)
+#pragma unroll
+                for (int s = 0; s < kC / 16; ++s)
+                    umma_f16_ts(tbase + TD + 128 * (c & 1) + 64, tbase + TU + 8 * s,
+                                desc_at(dK, st + ST_AQ + 32 * s), id3, 1);
+                umma_commit(bar_o0 + 8 * (c & 1));
+            }
+            mma2_pending = o_pending = true;
+            mma2_chunk = o_chunk = c;
+        }
+
+        if (aborted) {
+            if (tid == 0) set_device_error(args.err, DEV_TIMEOUT);
+            *abort_s = 1;
+            // wind down: this CTA's own copies and MMAs finish before TMEM and smem go away
+            const long long drain = 1ll << 31;
+            if (tid == kMma) {
+                if (mma1_pending) mbar_wait(bar_mma1, (uint32_t)(mma1_chunk & 1), drain);
+                if (mma2_pending) mbar_wait(bar_mma2, (uint32_t)(mma2_chunk & 1), drain);
+                if (o_pending)
+                    mbar_wait(bar_o0 + 8 * (o_chunk & 1), (uint32_t)((o_chunk >> 1) & 1), drain);
+            }
+        } else {
+            bool ok = true;
+            if (tid == 0 && mma2_pending)
+                ok = mbar_wait(bar_mma2, (uint32_t)(mma2_chunk & 1), args.budget);
+            if (bar_or(kBarChain, kChainThreads, !ok)) {
+                if (tid == 0) set_device_error(args.err, DEV_TIMEOUT);
+                *abort_s = 1;
+                if (tid == kMma) mbar_wait(bar_mma2, (uint32_t)(mma2_chunk & 1), 1ll << 31);
+            } else {
+                tc_fence_after();
+                if (args.hT && data) {
+#pragma unroll 1
+                    for (int p = 0; p < 2; ++p) {
+                        float v[32];
+                        const int c0 = 64 * hs + 32 * p;
+                        tmem_ld32(tbase + lq + TS + c0, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            args.hT[state_base + (size_t)(c0 + i) * kD + j] = v[i];
+                    }
+                }
             }
         }
+    } else {
+        // ============================================================ epilogue warps
+        const int et = tid - kEpi0;   // 0..127
+        const int ew = et >> 5;       // 0..3: rows 16 ew .. 16 ew + 15 of the norm pass
+        const bool norm = args.gate != nullptr;
+        float wv[4] = {0.f, 0.f, 0.f, 0.f};
+        if (norm) {
+            const float4 x = *reinterpret_cast<const float4*>(args.nw + 4 * lane);
+            wv[0] = x.x; wv[1] = x.y; wv[2] = x.z; wv[3] = x.w;
+        }
+        // gate tile of chunk cc (one 64-row box of this head; rows past the document are read
+        // but not used) into gate buffer cc & 1
+        auto issue_gate = [&](int cc) {
+            const uint32_t bar = bar_gate0 + 8 * (cc & 1);
+            mbar_arrive_expect_tx(bar, 16384);
+            tma_load_3d(sb + OFF_G + 16384 * (cc & 1), &maps.g, bar, 0, h,
+                        (int)(t0 + (long long)kC * cc));
+        };
+        int gate_issued = 0, gate_landed = 0;
+        if (norm && et == 0 && nchunks > 0) issue_gate(0);
+        if (norm) gate_issued = min(nchunks, 1);
+
+        for (int c = 0; c < nchunks; ++c) {
+            // o product of chunk c done (every epilogue thread polls, bounded; after a chain
+            // abort the wait expires and the epilogue stops)
+            const bool ok =
+                mbar_wait(bar_o0 + 8 * (c & 1), (uint32_t)((c >> 1) & 1), args.budget);
+            if (bar_or(kBarEpi, kEpiThreads, !ok)) {
+                if (et == 0 && !*abort_s) set_device_error(args.err, DEV_TIMEOUT);
+                break;
+            }
+            // the gate of chunk c+1 goes into the buffer chunk c-1's norm finished reading
+            if (norm && c + 1 < nchunks) {
+                if (et == 0) issue_gate(c + 1);
+                gate_issued = c + 2;
+            }
+            tc_fence_after();
+            float v[64];   // o^T row j: tokens 0..63 of value column j
+            {
+                float a[32], b[32];
+                tmem_ld32(tbase + lq + TD + 128 * (c & 1) + 64, a);
+                tmem_ld32(tbase + lq + TD + 128 * (c & 1) + 96, b);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    v[i] = a[i];
+                    v[32 + i] = b[i];
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar_dfree0 + 8 * (c & 1));   // D buffer c & 1 may be overwritten now
+            // output tile c & 1 was last stored for chunk c-2: that store must have read it
+            if (et == 0 && c >= 2) bulk_wait_read_le1();
+            bar_sync(kBarEpi, kEpiThreads);
+            __nv_bfloat16* tile = reinterpret_cast<__nv_bfloat16*>(sm + OFF_Y + 16384 * (c & 1));
+            const long long r0 = t0 + (long long)kC * c;
+            const int L = (int)min((long long)kC, t1 - r0);
+#pragma unroll
+            for (int t = 0; t < kC; ++t) tile[t * kD + j] = __float2bfloat16_rn(v[t]);
+            if (norm) {
+                const bool gok =
+                    mbar_wait(bar_gate0 + 8 * (c & 1), (uint32_t)((c >> 1) & 1), args.budget);
+                gate_landed = c + 1;
+                if (bar_or(kBarEpi, kEpiThreads, !gok)) {   // also: the tile is complete
+                    if (et == 0) set_device_error(args.err, DEV_TIMEOUT);
+                    break;
+                }
+                const __nv_bfloat16* gt =
+                    reinterpret_cast<const __nv_bfloat16*>(sm + OFF_G + 16384 * (c & 1));
+                // one warp per 16 rows, lane l on columns 4 l .. 4 l + 3, in place; the same
+                // arithmetic as the separate pass (kda_norm.cu)
+#pragma unroll 8
+                for (int rr = 0; rr < 16; ++rr) {
+                    const int t = 16 * ew + rr;
+                    const uint2 u = *reinterpret_cast<const uint2*>(tile + t * kD + 4 * lane);
+                    const float x[4] = {lo_bf(u.x), hi_bf(u.x), lo_bf(u.y), hi_bf(u.y)};
+                    float ss = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+                    for (int off = 16; off >= 1; off >>= 1)
+                        ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                    const float inv = rsqrtf(ss / (float)kD + args.eps);
+                    const uint2 gu = *reinterpret_cast<const uint2*>(gt + t * kD + 4 * lane);
+                    const float g[4] = {lo_bf(gu.x), hi_bf(gu.x), lo_bf(gu.y), hi_bf(gu.y)};
+                    float y[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        y[e] = x[e] * inv * wv[e] * __fdividef(1.f, 1.f + __expf(-g[e]));
+                    *reinterpret_cast<uint2*>(tile + t * kD + 4 * lane) =
+                        make_uint2(pack2(y[0], y[1]), pack2(y[2], y[3]));
+                }
+            }
+            fence_proxy_async();   // tile -> TMA store
+            bar_sync(kBarEpi, kEpiThreads);
+            // one TMA store for a full chunk, row copies for a partial one (a TMA box would run
+            // into the next document's rows)
+            if (L == kC) {
+                if (et == 0) {
+                    tma_store_3d(&maps.o, smem_u32(tile), 0, h, (int)r0);
+                    bulk_commit();
+                }
+            } else {
+                const uint4* src = reinterpret_cast<const uint4*>(tile);
+                for (int i = et; i < L * 16; i += kEpiThreads) {
+                    const int r = i >> 4, q = i & 15;
+                    *reinterpret_cast<uint4*>(args.o + ((size_t)(r0 + r) * args.H + h) * kD +
+                                              8 * q) = src[r * 16 + q];
+                }
+            }
+        }
+        if (et == 0) {
+            // gate copies still in flight land before the smem goes away (bounded)
+            for (int cc = gate_landed; cc < gate_issued; ++cc)
+                mbar_wait(bar_gate0 + 8 * (cc & 1), (uint32_t)((cc >> 1) & 1), 1ll << 31);
+            bulk_wait_all();   // output stores complete before the smem goes away
+        }
     }
-    if (tid == kStorer) bulk_wait_all();   // output stores complete before the smem goes away
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, kTmemCols);
@@ -447,9 +594,10 @@ int scan_debug_stall() {
 
 }  // namespace
 
-// One CTA (4 warps) per (sequence or document, head); packed documents are taken longest first
+// One CTA (14 warps) per (sequence or document, head); packed documents are taken longest first
 // when an order is given.
-cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaStream_t stream) {
+cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaStream_t stream,
+                              const ScanNorm* norm) {
     const SplitWorkspace& ws = *p.split;
     const long long units = (long long)p.N * p.H;
     if (units == 0) return cudaSuccess;
@@ -470,6 +618,13 @@ cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaSt
         (e = make_map_3d_rows(&m.o, p.o, BF, 2, (unsigned long long)p.B * p.T, p.H, kD, kC)) !=
             cudaSuccess)
         return e;
+    if (norm) {
+        if ((e = make_map_3d_rows(&m.g, norm->gate, BF, 2, (unsigned long long)p.B * p.T, p.H, kD,
+                                  kC)) != cudaSuccess)
+            return e;
+    } else {
+        memset(&m.g, 0, sizeof(m.g));
+    }
     static PerDevice attr;
     const cudaError_t attr_err = attr.run([](int) {
         return cudaFuncSetAttribute(chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -486,6 +641,11 @@ cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaSt
     a.c_end = seg.c_end;
     a.o = static_cast<__nv_bfloat16*>(p.o);
     a.decay = ws.decay;
+    if (norm) {
+        a.gate = static_cast<const __nv_bfloat16*>(norm->gate);
+        a.nw = norm->weight;
+        a.eps = norm->eps;
+    }
     a.T = p.T;
     a.H = p.H;
     a.N = p.N;
