@@ -8,7 +8,9 @@ It shares no code with ``gated_delta_rule_144_b200`` and never imports it.
 card's Kimi Delta Attention snippet, with packed-document resets as in the NeMo glm5_next
 ``_torch_recurrent_kda`` docstring). ``brute.py`` is a second, loop-free evaluation used only to
 pin the first one on tiny inputs. ``out_norm.py`` is the gated per-head RMSNorm of the output and
-``backward.py`` the gradients of the recurrence (the training direction), both float64 NumPy.
+``backward.py`` the gradients of the recurrence (the training direction) and ``short_conv.py`` the
+short causal convolution of the inputs (with optional SiLU and per-head L2 norm), all float64
+NumPy.
 
 Every function here is pinned (tests/test_oracle_pins.py); none is "parity unpinned".
 """
