@@ -528,6 +528,31 @@ def run_secondary(kda, synth, args, dev, stream, world, rank):
                                     "ms_normed_call": res["normed"],
                                     "ms_plain_then_norm": res["separate"],
                                     "ms_plain": out["packed_prefill"]["ms_per_step"]}
+    # the input prologue (kda_short_conv): one projection of the packed workload, [1, T, 32 x 128]
+    # bf16, W = 4 taps, SiLU, L2 norm per head (how q and k enter the recurrence)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(shard.rank_seed(1097, rank))
+    px = torch.randn((1, p["T"], 32 * 128), generator=gen, device=dev).to(torch.bfloat16)
+    pw = torch.randn((32 * 128, 4), generator=gen, device=dev) * 0.5
+    py = torch.empty_like(px)
+
+    def cstep():
+        kda.short_conv(px, pw, p["cu_seqlens"], activation="silu", norm_group=128, y=py)
+
+    for _ in range(3):
+        cstep()
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms, _ = time_launches(cstep, max(args.steps, 20), stream)
+    barrier(world)
+    ms = max_over_ranks(total_ms, world, dev) / max(args.steps, 20)
+    by = 2 * px.numel() * 2 + pw.numel() * 4 + p["cu_seqlens"].numel() * 4
+    out["prologue"] = {"workload": "packed-8docs (one of q, k, v: 32 heads x 128 channels)",
+                       "W": 4, "activation": "silu", "norm_group": 128,
+                       "ms_per_call": round(ms, 4), "bytes_per_call": by,
+                       "roofline_frac": round(by / (ms / 1e3) / 1e9 / hbm_peak, 4),
+                       "kernel": "short_conv_kernel"}
+    del px, pw, py
     # gradients (kda_bwd) on the T=4096, H=16 workload: upstream do and dhT drawn once
     b = synth.prefill_inputs("prefill-t4096", device=dev, seed=shard.rank_seed(1001, rank))
     gen = torch.Generator(device=dev)

@@ -19,7 +19,7 @@ from pathlib import Path
 
 import torch
 
-__all__ = ["fwd", "fwd_no_alloc", "out_norm_gated", "decode_step", "decode_tokens",
+__all__ = ["fwd", "fwd_no_alloc", "out_norm_gated", "short_conv", "decode_step", "decode_tokens",
            "get_device_error",
            "fwd_workspace_size",
            "fwd_workspace_size_min", "fwd_algorithm",
@@ -80,6 +80,9 @@ def lib():
     L.kda_bwd.restype = i32
     L.kda_bwd_workspace_size.argtypes = [ctypes.POINTER(FwdDesc)]
     L.kda_bwd_workspace_size.restype = ctypes.c_size_t
+    L.kda_short_conv.argtypes = [i32, i32, i32, i32, i32, p, p, p, i32, i32, i32, ctypes.c_float,
+                                 p, p]
+    L.kda_short_conv.restype = i32
     L.kda_fwd_no_alloc.argtypes = [ctypes.POINTER(FwdDesc), p, p, p, p, p, p, p, p, p, p]
     L.kda_fwd_no_alloc.restype = i32
     L.kda_fwd_algorithm.argtypes = [ctypes.POINTER(FwdDesc), i32]
@@ -357,6 +360,44 @@ def _prefill_shapes(q, k, v, log_g, beta, cu_seqlens):
     if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
         raise ValueError("cu_seqlens must be a 1-D int32 tensor of N + 1 offsets")
     return B, T, H, dk, v.shape[3], cu_seqlens.numel() - 1
+
+
+def short_conv(x, weight, cu_seqlens=None, *, activation: str = "none", norm_group: int = 0,
+               eps: float = 1e-6, y=None, stream=None):
+    """``kda_short_conv``: the short causal convolution of one input (q, k or v) over
+    [B, T, C] with a reset at packed-document boundaries, then an optional SiLU
+    (activation="silu") and an optional L2 norm of every group of ``norm_group`` channels
+    (norm_group = head_dim gives q or k as kda_fwd takes them). weight: fp32 [C, W], W <= 8.
+    Returns y shaped and typed like x (y must not be x)."""
+    lib()
+    _dev(x, "x")
+    dev = x.device
+    if x.dim() != 3:
+        raise ValueError("x must be [B, T, C]")
+    B, T, C = x.shape
+    _dtype_code(x)
+    _dev(weight, "weight", torch.float32, None, dev)
+    if weight.dim() != 2 or weight.shape[0] != C:
+        raise ValueError("weight must be [C, W]")
+    acts = {"none": 0, "silu": 1}
+    if activation not in acts:
+        raise ValueError("activation must be 'none' or 'silu'")
+    N = B
+    if cu_seqlens is not None:
+        _dev(cu_seqlens, "cu_seqlens", torch.int32, None, dev)
+        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+            raise ValueError("cu_seqlens must be a 1-D int32 tensor of N + 1 offsets")
+        N = cu_seqlens.numel() - 1
+    if y is None:
+        y = torch.empty_like(x)
+    else:
+        _dev(y, "y", x.dtype, tuple(x.shape), dev)
+    with torch.cuda.device(dev):
+        st = lib().kda_short_conv(B, T, C, weight.shape[1], _dtype_code(x), _ptr(x), _ptr(weight),
+                                  _ptr(cu_seqlens), N, acts[activation], int(norm_group),
+                                  float(eps), _ptr(y), _stream(stream, dev))
+    _check(st, "kda_short_conv")
+    return y
 
 
 def fwd_no_alloc(q, k, v, log_g, beta, h0, cu_seqlens, o, hT, *, chunk_size: int = CHUNK_AUTO,

@@ -506,6 +506,48 @@ kda_status_t kda_out_norm_gated(long long vectors, int dv, kda_dtype_t dtype, co
     return KDA_OK;
 }
 
+kda_status_t kda_short_conv(int B, int T, int C, int W, kda_dtype_t dtype, const void* x,
+                            const float* weight, const int32_t* cu_seqlens, int num_seqs,
+                            kda_activation_t act, int norm_group, float eps, void* y,
+                            kda_stream_t stream) {
+    t_last_error[0] = 0;
+    if (B < 1 || T < 0 || C < 1 || num_seqs < 0)
+        return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d C=%d N=%d", B, T, C, num_seqs);
+    if (W < 1 || W > 8) return fail(KDA_ERR_UNSUPPORTED, "kernel width %d (1..8)", W);
+    if (C % 4) return fail(KDA_ERR_UNSUPPORTED, "C = %d is not a multiple of 4", C);
+    if (dtype != KDA_F32 && dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (act != KDA_ACT_NONE && act != KDA_ACT_SILU)
+        return fail(KDA_ERR_INVALID_ARG, "unknown activation %d", (int)act);
+    if (norm_group != 0 && (norm_group < 4 || norm_group > 128 ||
+                            (norm_group & (norm_group - 1)) || C % norm_group))
+        return fail(KDA_ERR_UNSUPPORTED,
+                    "norm_group %d (0, or a power of two from 4 to 128 dividing C)", norm_group);
+    if (!(eps >= 0.f)) return fail(KDA_ERR_INVALID_ARG, "eps must be >= 0");
+    if (cu_seqlens && B != 1) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens requires B == 1");
+    if (cu_seqlens && num_seqs < 1)
+        return fail(KDA_ERR_INVALID_ARG, "cu_seqlens needs num_seqs >= 1");
+    if ((int64_t)B * T * C > (int64_t)1 << 40) return fail(KDA_ERR_INVALID_ARG, "problem too large");
+    kda_status_t st;
+    const bool any = (int64_t)B * T > 0;
+    if ((st = check_ptr(x, "x", any)) || (st = check_ptr(weight, "weight", any)) ||
+        (st = check_ptr(y, "y", any)) || (st = check_ptr(cu_seqlens, "cu_seqlens", false)))
+        return st;
+    if (!any) return KDA_OK;
+    const size_t esz = dtype == KDA_BF16 ? 2 : 4;
+    const uintptr_t xb = reinterpret_cast<uintptr_t>(x), yb = reinterpret_cast<uintptr_t>(y);
+    const size_t bytes = (size_t)B * T * C * esz;
+    if (xb < yb + bytes && yb < xb + bytes)
+        return fail(KDA_ERR_INVALID_ARG, "y overlaps x (the window reads earlier rows of x)");
+    unsigned* err = nullptr;
+    if ((st = device_error_word(&err)) != KDA_OK) return st;
+    cudaError_t e = kda::launch_short_conv(x, weight, cu_seqlens, num_seqs, y, B, T, C, W,
+                                           dtype == KDA_BF16, (int)act, norm_group, eps, err,
+                                           reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kda_short_conv launch");
+    return KDA_OK;
+}
+
 kda_status_t kda_decode_step(int N, int H, int dk, int dv, kda_dtype_t dtype, const void* q,
                              const void* k, const void* v, const float* log_g, const void* beta,
                              float* S_inout, void* o, kda_stream_t stream) {

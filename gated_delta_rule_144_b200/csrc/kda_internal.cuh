@@ -121,6 +121,11 @@ cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaSt
 cudaError_t launch_out_norm_gated(const void* x, const void* gate, const float* w, float eps,
                                   void* y, long long vectors, int dv, bool bf16,
                                   cudaStream_t stream);
+// Short causal convolution with document resets, optional SiLU (act = 1) and L2 norm per group
+// of `group` channels (0: none); x, y [B, T, C]; w [C][W], 1 <= W <= 8.
+cudaError_t launch_short_conv(const void* x, const float* w, const int32_t* cu, int N, void* y,
+                              int B, int T, int C, int W, bool bf16, int act, int group, float eps,
+                              unsigned* err, cudaStream_t stream);
 bool chunk64_available();
 // Value columns one chunked-kernel CTA owns for N sequences x H heads (64 or 128).
 int chunk64_value_width(int N, int H);

@@ -194,6 +194,33 @@ kda_status_t kda_out_norm_gated(long long vectors, int dv, kda_dtype_t dtype, co
                                 kda_stream_t stream);
 
 /*
+ * kda_short_conv - the input prologue of the recurrence: the short causal convolution of q, k or
+ * v with a reset at packed-document boundaries, an optional SiLU and an optional L2 norm per
+ * group of channels, in one pass (NeMo glm5_next layers, _TorchShortConvolution: a depthwise
+ * causal Conv1d over [batch, sequence, channels] that resets at packed boundaries;
+ * Glm5NextLinearAttention holds one each for q, k and v, of linear_conv_kernel_dim taps). Per
+ * channel c and token t of a document starting at s:
+ *     y[t, c] = sum_{j < W} weight[c, j] x[t - (W - 1) + j, c]     (positions before s: zero)
+ * then, with act = KDA_ACT_SILU, y <- y * sigmoid(y), and, with norm_group = g > 0,
+ * y <- y / sqrt(sum over its group of y^2 + eps) for every group of g consecutive channels
+ * (g = head_dim normalises each head vector, the form in which q and k enter kda_fwd).
+ *   x, y       : [B, T, C] in dtype (C = heads * head_dim), device, 16-byte aligned; y must not
+ *                overlap x.
+ *   weight     : [C, W] float32, device; 1 <= W <= 8.
+ *   cu_seqlens : int32 [num_seqs + 1] on the device (B must be 1), or NULL (each batch row is
+ *                one document).
+ *   C % 4 == 0; norm_group is 0 or one of 4, 8, ..., 128 and divides C.
+ * Host-checkable errors return before any launch; a malformed cu_seqlens sets
+ * KDA_ERR_BAD_SEQLENS in the device error word. The pages do not print the activation: it is
+ * off unless asked for.
+ */
+typedef enum { KDA_ACT_NONE = 0, KDA_ACT_SILU = 1 } kda_activation_t;
+kda_status_t kda_short_conv(int B, int T, int C, int W, kda_dtype_t dtype, const void* x,
+                            const float* weight, const int32_t* cu_seqlens, int num_seqs,
+                            kda_activation_t act, int norm_group, float eps, void* y,
+                            kda_stream_t stream);
+
+/*
  * Path kda_fwd takes for `desc` (has_cu_seqlens: whether cu_seqlens will be non-NULL):
  * KDA_CHUNK_PER_TOKEN or KDA_CHUNK_64, or the negated kda_status_t when the description is
  * rejected. Host-only, no CUDA calls.

@@ -271,3 +271,26 @@ def test_no_alloc_binding_checks_shapes_before_any_launch():
         kda.fwd_no_alloc(q, q, q, g, beta, None, None, o, hT[:, :1])
     with pytest.raises(ValueError, match="cu_seqlens"):
         kda.fwd_no_alloc(q, q, q, g, beta, None, torch.zeros((2, 2), dtype=torch.int32), o, None)
+
+
+def test_short_conv_rejects_on_host(L):
+    P = ctypes.c_void_p
+    ok = dict(B=1, T=16, C=256, W=4, dtype=kda.KDA_BF16, x=P(FAKE), w=P(FAKE), cu=None, N=1,
+              act=0, group=128, eps=1e-6, y=P(FAKE + 0x100000))
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return L.kda_short_conv(a["B"], a["T"], a["C"], a["W"], a["dtype"], a["x"], a["w"],
+                                a["cu"], a["N"], a["act"], a["group"], a["eps"], a["y"], None)
+
+    assert call(W=0) == 2 and call(W=9) == 2
+    assert call(C=258) == 2                      # not a multiple of 4
+    assert call(group=12) == 2 and call(group=256) == 2 and call(C=192, group=128) == 2
+    assert call(act=3) == 1
+    assert call(eps=-1.0) == 1
+    assert call(x=None) == 1 and call(x=P(FAKE + 4)) == 1
+    assert call(y=P(FAKE + 64)) == 1             # overlaps x
+    assert b"overlaps" in L.kda_last_error()
+    assert call(B=2, cu=P(FAKE)) == 1            # cu_seqlens needs B == 1
+    assert call(T=0) == 0                        # no tokens: nothing to do
