@@ -152,11 +152,12 @@ short_conv_kernel(const ConvArgs a) {
             for (int e = 0; e < 4; ++e) xw[i][e] = 0.f;
         }
     }
+    // pass 1: the convolution of every token of the run (outputs depend on inputs only), SiLU
+    float v[kRun][4];
 #pragma unroll
     for (int r = 0; r < kRun; ++r) {
         const int t = t_begin + r;
-        if (t >= t_end) break;
-        if (t >= next_start) {   // a new document starts at t: the window restarts from zero
+        if (t >= next_start && t < t_end) {   // a new document starts at t: restart the window
             while (d + 1 < a.N && a.cu[d + 1] <= t) ++d;
             doc_start = a.cu[d];
             next_start = a.cu[d + 1];
@@ -167,29 +168,17 @@ short_conv_kernel(const ConvArgs a) {
         }
         float xt[4];
         unpack4(raw[r], xt);
-        float v[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             float s = 0.f;
 #pragma unroll
             for (int i = 0; i < W - 1; ++i) s = fmaf(w[e][i], xw[i][e], s);
-            v[e] = fmaf(w[e][W - 1], xt[e], s);
+            v[r][e] = fmaf(w[e][W - 1], xt[e], s);
         }
         if (a.act == 1) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) v[e] = __fdividef(v[e], 1.f + __expf(-v[e]));
+            for (int e = 0; e < 4; ++e) v[r][e] = __fdividef(v[r][e], 1.f + __expf(-v[r][e]));
         }
-        if (a.group > 0) {
-            float ss = 0.f;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) ss = fmaf(v[e], v[e], ss);
-            for (int off = 1; off < a.group / 4; off <<= 1)
-                ss += __shfl_xor_sync(0xffffffffu, ss, off);
-            const float inv = rsqrtf(ss + a.eps);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) v[e] *= inv;
-        }
-        if (active) store4(y + base + (size_t)t * row, v);
 #pragma unroll
         for (int i = 0; i + 1 < W - 1; ++i)
 #pragma unroll
@@ -199,6 +188,30 @@ short_conv_kernel(const ConvArgs a) {
             for (int e = 0; e < 4; ++e) xw[W > 1 ? W - 2 : 0][e] = xt[e];
         }
     }
+    // pass 2: the group norms of all the run's tokens at once (independent shuffle chains)
+    if (a.group > 0) {
+        float ss[kRun];
+#pragma unroll
+        for (int r = 0; r < kRun; ++r) {
+            ss[r] = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) ss[r] = fmaf(v[r][e], v[r][e], ss[r]);
+        }
+        for (int off = 1; off < a.group / 4; off <<= 1) {
+#pragma unroll
+            for (int r = 0; r < kRun; ++r) ss[r] += __shfl_xor_sync(0xffffffffu, ss[r], off);
+        }
+#pragma unroll
+        for (int r = 0; r < kRun; ++r) {
+            const float inv = rsqrtf(ss[r] + a.eps);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[r][e] *= inv;
+        }
+    }
+    // pass 3: stores
+#pragma unroll
+    for (int r = 0; r < kRun; ++r)
+        if (active && t_begin + r < t_end) store4(y + base + (size_t)(t_begin + r) * row, v[r]);
 }
 
 template <typename T>
