@@ -12,7 +12,8 @@ pin the first one on tiny inputs. ``out_norm.py`` is the gated per-head RMSNorm 
 short causal convolution of the inputs (with optional SiLU and per-head L2 norm), all float64
 NumPy.
 
-Every function here is pinned (tests/test_oracle_pins.py); none is "parity unpinned".
+Every function here is pinned (tests/test_oracle_pins.py, test_oracle_backward.py,
+test_oracle_out_norm.py, test_oracle_short_conv.py); none is "parity unpinned".
 """
 
 from __future__ import annotations
