@@ -671,6 +671,13 @@ def run_profile_case(args):
         bdh = torch.randn((b["N"], b["H"], 128, 128), generator=gen, device=dev)
         fn = lambda: kda.bwd(b["q"], b["k"], b["v"], b["log_g"], b["beta"], bdo, h0=b["h0"],
                              dhT=bdh)
+    elif args.profile_case == "conv":
+        p = synth.prefill_inputs("packed-8docs", device=dev)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(1097)
+        px = torch.randn((1, p["T"], 32 * 128), generator=gen, device=dev).to(torch.bfloat16)
+        pw = torch.randn((32 * 128, 4), generator=gen, device=dev) * 0.5
+        fn = lambda: kda.short_conv(px, pw, p["cu_seqlens"], activation="silu", norm_group=128)
     elif args.profile_case == "norm":
         p = synth.prefill_inputs("packed-8docs", device=dev)
         o = torch.randn(p["v"].shape, device=dev).to(p["v"].dtype)
@@ -711,7 +718,7 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case",
-                    choices=["prefill", "decode", "decode-rows", "packed", "norm", "bwd"],
+                    choices=["prefill", "decode", "decode-rows", "packed", "norm", "bwd", "conv"],
                     default=None,
                     help="run only warm-up + steps launches of one case (for ncu captures)")
     ap.add_argument("--profile-tokens", type=int, default=0,
