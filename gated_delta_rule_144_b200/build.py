@@ -30,12 +30,15 @@ FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xptxas", "-v
 
 
 # Per-file flags. The chunked kernels evaluate one exponential and one reciprocal per operand
-# element through the MUFU unit; flushing subnormals lets those intrinsics compile without their
-# subnormal fix-ups (14 % fewer instructions in the intra-chunk kernel). Nothing they compute is
-# meant to be subnormal: decay products below 1e-30 are already reported as out of range.
+# element through the MUFU unit, the prologue two per element (its SiLU); flushing subnormals lets
+# those intrinsics compile without their subnormal fix-ups (14 % fewer instructions in the
+# intra-chunk kernel). Nothing they compute is meant to be subnormal: chunks whose decay products
+# fall below 1e-30 take the direct path, and a prologue output below 1.2e-38 is zero to any
+# tolerance the inputs' precision allows.
 FILE_FLAGS = {
     "kda_intra.cu": ["-ftz=true"],
     "kda_chunk64.cu": ["-ftz=true"],
+    "kda_conv.cu": ["-ftz=true"],
 }
 
 

@@ -10,57 +10,90 @@
 // each group of g consecutive channels (g = head_dim normalises each head vector, as the
 // recurrence's q and k arrive).
 //
-// Work split: a warp owns 128 consecutive channels (4 per lane: 8-byte bf16 / 16-byte fp32
-// accesses, a warp row access is 256 or 512 contiguous bytes) and a run of kRun consecutive tokens
-// of one batch row; it keeps the last W - 1 input rows of its channels in registers, so each input
-// row is read once per run (plus W - 1 rows of halo at the run's start), the run's rows all
-// loaded before the first is used. A group norm of g channels is a shuffle reduction over g / 4
-// lanes.
+// Work split: a warp owns 32 * CH consecutive channels (CH = 4 per lane) and a segment of 64
+// consecutive tokens of one batch row, which it streams through in blocks of rows: the next
+// block's rows are in flight while the current one is computed, and the last W - 1 input rows of
+// its channels stay in registers, so each input row is read once (plus W - 1 rows of halo at the
+// segment's start). A block inside one document is computed without branches, so that its rows'
+// conv, SiLU and norm chains interleave; a block with a document start or the segment's end goes
+// row by row. A group norm of g channels is a shuffle reduction over g / CH lanes.
 
 #include <cstdint>
-#include <type_traits>
 
 #include "kda_internal.cuh"
 
 namespace kda {
 namespace {
 
-// tokens per warp: the run's rows are held in registers (16 bf16 rows, 8 fp32 rows)
-template <typename T>
-constexpr int run_of() { return sizeof(T) == 2 ? 16 : 8; }
-constexpr int kWarps = 8;     // warps per block
+constexpr int kWarps = 4;     // warps per block
+// channels per lane: 8-byte bf16 / 16-byte fp32 accesses, a warp row is 256 or 512 contiguous
+// bytes (eight per lane measured 5 % slower: its registers allow fewer warps per SM)
+constexpr int kCh = 4;
 
-__device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
-    const float4 x = *reinterpret_cast<const float4*>(p);
-    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+// A lane's CH consecutive channels of one row, as raw words (CH * sizeof(T) bytes: 8, 16 or 32).
+template <typename T, int CH>
+struct Row {
+    static constexpr int kWords = CH * (int)sizeof(T) / 4;
+    uint32_t u[kWords];
+    __device__ __forceinline__ void zero() {
+#pragma unroll
+        for (int i = 0; i < kWords; ++i) u[i] = 0u;
+    }
+    __device__ __forceinline__ void load(const T* p) {
+        if constexpr (kWords == 2) {
+            const uint2 x = *reinterpret_cast<const uint2*>(p);
+            u[0] = x.x; u[1] = x.y;
+        } else {
+#pragma unroll
+            for (int i = 0; i < kWords; i += 4) {
+                const uint4 x = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint32_t*>(p) + i);
+                u[i] = x.x; u[i + 1] = x.y; u[i + 2] = x.z; u[i + 3] = x.w;
+            }
+        }
+    }
+    __device__ __forceinline__ void unpack(float (&v)[CH]) const {
+        if constexpr (sizeof(T) == 2) {
+#pragma unroll
+            for (int i = 0; i < kWords; ++i) {
+                v[2 * i] = __uint_as_float(u[i] << 16);
+                v[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < CH; ++i) v[i] = __uint_as_float(u[i]);
+        }
+    }
+};
+
+template <typename T, int CH>
+__device__ __forceinline__ void store_row(T* p, const float (&v)[CH]) {
+    if constexpr (sizeof(T) == 2) {
+        uint32_t w[CH / 2];
+#pragma unroll
+        for (int i = 0; i < CH / 2; ++i) {
+            __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t*>(&b);
+        }
+        if constexpr (CH == 4) {
+            *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
+        } else {
+            *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < CH; i += 4)
+            *reinterpret_cast<float4*>(p + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+    }
 }
-__device__ __forceinline__ void load4(const __nv_bfloat16* p, float (&v)[4]) {
-    const uint2 u = *reinterpret_cast<const uint2*>(p);
-    v[0] = __uint_as_float(u.x << 16);
-    v[1] = __uint_as_float(u.x & 0xffff0000u);
-    v[2] = __uint_as_float(u.y << 16);
-    v[3] = __uint_as_float(u.y & 0xffff0000u);
-}
-__device__ __forceinline__ void unpack4(const uint2& u, float (&v)[4]) {
-    v[0] = __uint_as_float(u.x << 16);
-    v[1] = __uint_as_float(u.x & 0xffff0000u);
-    v[2] = __uint_as_float(u.y << 16);
-    v[3] = __uint_as_float(u.y & 0xffff0000u);
-}
-__device__ __forceinline__ void unpack4(const uint4& u, float (&v)[4]) {
-    v[0] = __uint_as_float(u.x);
-    v[1] = __uint_as_float(u.y);
-    v[2] = __uint_as_float(u.z);
-    v[3] = __uint_as_float(u.w);
-}
-__device__ __forceinline__ void store4(float* p, const float (&v)[4]) {
-    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-}
-__device__ __forceinline__ void store4(__nv_bfloat16* p, const float (&v)[4]) {
-    __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
-    __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
-    *reinterpret_cast<uint2*>(p) =
-        make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+
+// x sigmoid(x), with the fast exponential and division (subnormals flushed in this file)
+__device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.f + __expf(-x)); }
+
+// tokens per warp item, and input rows in flight per lane (64 bytes of loads per lane)
+constexpr int kSeg = 64;
+template <typename T, int CH>
+constexpr int ahead_of() {
+    return 64 / (CH * (int)sizeof(T)) < 2 ? 2 : 64 / (CH * (int)sizeof(T));
 }
 
 struct ConvArgs {
@@ -71,59 +104,54 @@ struct ConvArgs {
     void* y;
     int B, T, C;
     int act;                 // 0: none, 1: SiLU
-    int group;               // 0 or the channels of one norm group (divides 128 and C)
+    int group;               // 0 or the channels of one norm group (>= CH; divides C)
     float eps;
     unsigned* err;
 };
 
-template <typename T, int W>
+template <typename T, int W, int CH>
 __global__ void __launch_bounds__(32 * kWarps)
 short_conv_kernel(const ConvArgs a) {
-    constexpr int kRun = run_of<T>();
+    constexpr int kAhead = ahead_of<T, CH>();
+    constexpr int kSpan = 32 * CH;   // channels per warp
+    constexpr int kHalo = W > 1 ? W - 1 : 1;
     const int lane = threadIdx.x & 31;
     const long long warp_id = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
-    const int cgroups = (a.C + 127) / 128;
-    const int runs = (a.T + kRun - 1) / kRun;
-    const long long items = (long long)a.B * runs * cgroups;
+    const int cgroups = (a.C + kSpan - 1) / kSpan;
+    const int segs = (a.T + kSeg - 1) / kSeg;
+    const long long items = (long long)a.B * segs * cgroups;
     if (warp_id >= items) return;
     const int cg = (int)(warp_id % cgroups);
     const long long rr = warp_id / cgroups;
-    const int b = (int)(rr / runs);
-    const int t_begin = (int)(rr % runs) * kRun;
-    const int t_end = min(a.T, t_begin + kRun);
-    const int c0 = 128 * cg + 4 * lane;
-    const bool active = c0 < a.C;   // C % 4 == 0: a lane is wholly in or out
-    const T* x = static_cast<const T*>(a.x);
-    T* y = static_cast<T*>(a.y);
-
-    float w[4][W];
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-#pragma unroll
-        for (int j = 0; j < W; ++j) w[e][j] = active ? a.w[(size_t)(c0 + e) * W + j] : 0.f;
-
-    // every input row of the run and its W - 1 rows of halo are loaded first, before the
-    // document lookup below (a few dependent loads of cu_seqlens), so that all of them are in
-    // flight together
+    const int b = (int)(rr / segs);
+    const int t_begin = (int)(rr % segs) * kSeg;
+    const int t_end = min(a.T, t_begin + kSeg);
+    const int c0 = kSpan * cg + CH * lane;
+    const bool active = c0 < a.C;   // C % CH == 0: a lane is wholly in or out
     const size_t row = (size_t)a.C;
-    const size_t base = (size_t)b * a.T * row + c0;
-    using Raw = typename std::conditional<sizeof(T) == 2, uint2, uint4>::type;
-    Raw raw[kRun], halo[W > 1 ? W - 1 : 1];
+    const T* xb = static_cast<const T*>(a.x) + (size_t)b * a.T * row + c0;
+    T* yb = static_cast<T*>(a.y) + (size_t)b * a.T * row + c0;
+
+    // the W - 1 halo rows and the first kAhead rows go out before anything waits on memory
+    Row<T, CH> halo[kHalo], raw[kAhead];
 #pragma unroll
     for (int i = 0; i < W - 1; ++i) {
         const int p = t_begin - (W - 1) + i;
-        halo[i] = Raw{};
-        if (active && p >= 0)
-            halo[i] = *reinterpret_cast<const Raw*>(x + base + (size_t)p * row);
+        halo[i].zero();
+        if (active && p >= 0) halo[i].load(xb + (size_t)p * row);
     }
 #pragma unroll
-    for (int r = 0; r < kRun; ++r) {
-        raw[r] = Raw{};
-        if (active && t_begin + r < t_end)
-            raw[r] = *reinterpret_cast<const Raw*>(x + base + (size_t)(t_begin + r) * row);
+    for (int j = 0; j < kAhead; ++j) {
+        raw[j].zero();
+        if (active && t_begin + j < t_end) raw[j].load(xb + (size_t)(t_begin + j) * row);
     }
+    float w[CH][W];
+#pragma unroll
+    for (int e = 0; e < CH; ++e)
+#pragma unroll
+        for (int j = 0; j < W; ++j) w[e][j] = active ? a.w[(size_t)(c0 + e) * W + j] : 0.f;
 
-    // document of the run's first token (packed row), and where the next one starts
+    // document of the segment's first token (packed row), and where the next one starts
     int doc_start = 0, next_start = a.T;
     int d = 0;
     if (a.cu) {
@@ -143,92 +171,157 @@ short_conv_kernel(const ConvArgs a) {
         }
     }
     // window: xw[i] holds the input at position t - (W - 1) + i, zero before the document start
-    float xw[W > 1 ? W - 1 : 1][4];
+    float xw[kHalo][CH];
 #pragma unroll
     for (int i = 0; i < W - 1; ++i) {
-        unpack4(halo[i], xw[i]);
+        halo[i].unpack(xw[i]);
         if (t_begin - (W - 1) + i < doc_start) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) xw[i][e] = 0.f;
+            for (int e = 0; e < CH; ++e) xw[i][e] = 0.f;
         }
     }
-    // pass 1: the convolution of every token of the run (outputs depend on inputs only), SiLU
-    float v[kRun][4];
+    const int lanes_per_group = a.group / CH;
+    for (int t0 = t_begin; t0 < t_end; t0 += kAhead) {
+        if (t0 + kAhead <= t_end && t0 + kAhead <= next_start) {
+            // the common case: kAhead whole rows inside one document, computed branch-free so
+            // that their conv, SiLU and norm chains interleave
+            float v[kAhead][CH];
 #pragma unroll
-    for (int r = 0; r < kRun; ++r) {
-        const int t = t_begin + r;
-        if (t >= next_start && t < t_end) {   // a new document starts at t: restart the window
-            while (d + 1 < a.N && a.cu[d + 1] <= t) ++d;
-            doc_start = a.cu[d];
-            next_start = a.cu[d + 1];
+            for (int j = 0; j < kAhead; ++j) {
+                float xt[CH];
+                raw[j].unpack(xt);
+                if (active && t0 + j + kAhead < t_end)
+                    raw[j].load(xb + (size_t)(t0 + j + kAhead) * row);
 #pragma unroll
-            for (int i = 0; i < W - 1; ++i)
+                for (int e = 0; e < CH; ++e) {
+                    float s = 0.f;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) xw[i][e] = 0.f;
+                    for (int i = 0; i < W - 1; ++i) s = fmaf(w[e][i], xw[i][e], s);
+                    v[j][e] = fmaf(w[e][W - 1], xt[e], s);
+                }
+#pragma unroll
+                for (int i = 0; i + 1 < W - 1; ++i)
+#pragma unroll
+                    for (int e = 0; e < CH; ++e) xw[i][e] = xw[i + 1][e];
+                if (W > 1) {
+#pragma unroll
+                    for (int e = 0; e < CH; ++e) xw[kHalo - 1][e] = xt[e];
+                }
+            }
+            if (a.act == 1) {
+#pragma unroll
+                for (int j = 0; j < kAhead; ++j)
+#pragma unroll
+                    for (int e = 0; e < CH; ++e) v[j][e] = silu(v[j][e]);
+            }
+            if (lanes_per_group > 0) {
+                float ss[kAhead];
+#pragma unroll
+                for (int j = 0; j < kAhead; ++j) {
+                    ss[j] = 0.f;
+#pragma unroll
+                    for (int e = 0; e < CH; ++e) ss[j] = fmaf(v[j][e], v[j][e], ss[j]);
+                }
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    if (off < lanes_per_group) {
+#pragma unroll
+                        for (int j = 0; j < kAhead; ++j)
+                            ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], off);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < kAhead; ++j) {
+                    const float inv = rsqrtf(ss[j] + a.eps);
+#pragma unroll
+                    for (int e = 0; e < CH; ++e) v[j][e] *= inv;
+                }
+            }
+            if (active) {
+#pragma unroll
+                for (int j = 0; j < kAhead; ++j)
+                    store_row<T, CH>(yb + (size_t)(t0 + j) * row, v[j]);
+            }
+            continue;
         }
-        float xt[4];
-        unpack4(raw[r], xt);
+        // a document boundary or the segment's end falls in this block: row by row
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float s = 0.f;
+        for (int j = 0; j < kAhead; ++j) {
+            const int t = t0 + j;
+            if (t >= t_end) break;
+            float xt[CH];
+            raw[j].unpack(xt);
+            // the row kAhead further on takes this row's registers
+            if (active && t + kAhead < t_end) raw[j].load(xb + (size_t)(t + kAhead) * row);
+            if (t >= next_start) {   // a new document starts at t: restart the window
+                while (d + 1 < a.N && a.cu[d + 1] <= t) ++d;
+                next_start = a.cu[d + 1];
 #pragma unroll
-            for (int i = 0; i < W - 1; ++i) s = fmaf(w[e][i], xw[i][e], s);
-            v[r][e] = fmaf(w[e][W - 1], xt[e], s);
-        }
-        if (a.act == 1) {
+                for (int i = 0; i < W - 1; ++i)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) v[r][e] = __fdividef(v[r][e], 1.f + __expf(-v[r][e]));
-        }
+                    for (int e = 0; e < CH; ++e) xw[i][e] = 0.f;
+            }
+            float v[CH];
 #pragma unroll
-        for (int i = 0; i + 1 < W - 1; ++i)
+            for (int e = 0; e < CH; ++e) {
+                float s = 0.f;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) xw[i][e] = xw[i + 1][e];
-        if (W > 1) {
+                for (int i = 0; i < W - 1; ++i) s = fmaf(w[e][i], xw[i][e], s);
+                v[e] = fmaf(w[e][W - 1], xt[e], s);
+            }
+            if (a.act == 1) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) xw[W > 1 ? W - 2 : 0][e] = xt[e];
+                for (int e = 0; e < CH; ++e) v[e] = silu(v[e]);
+            }
+            if (lanes_per_group > 0) {
+                float ss = 0.f;
+#pragma unroll
+                for (int e = 0; e < CH; ++e) ss = fmaf(v[e], v[e], ss);
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1)
+                    if (off < lanes_per_group) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                const float inv = rsqrtf(ss + a.eps);
+#pragma unroll
+                for (int e = 0; e < CH; ++e) v[e] *= inv;
+            }
+            if (active) store_row<T, CH>(yb + (size_t)t * row, v);
+#pragma unroll
+            for (int i = 0; i + 1 < W - 1; ++i)
+#pragma unroll
+                for (int e = 0; e < CH; ++e) xw[i][e] = xw[i + 1][e];
+            if (W > 1) {
+#pragma unroll
+                for (int e = 0; e < CH; ++e) xw[kHalo - 1][e] = xt[e];
+            }
         }
     }
-    // pass 2: the group norms of all the run's tokens at once (independent shuffle chains)
-    if (a.group > 0) {
-        float ss[kRun];
-#pragma unroll
-        for (int r = 0; r < kRun; ++r) {
-            ss[r] = 0.f;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) ss[r] = fmaf(v[r][e], v[r][e], ss[r]);
-        }
-        for (int off = 1; off < a.group / 4; off <<= 1) {
-#pragma unroll
-            for (int r = 0; r < kRun; ++r) ss[r] += __shfl_xor_sync(0xffffffffu, ss[r], off);
-        }
-#pragma unroll
-        for (int r = 0; r < kRun; ++r) {
-            const float inv = rsqrtf(ss[r] + a.eps);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) v[r][e] *= inv;
-        }
-    }
-    // pass 3: stores
-#pragma unroll
-    for (int r = 0; r < kRun; ++r)
-        if (active && t_begin + r < t_end) store4(y + base + (size_t)(t_begin + r) * row, v[r]);
 }
 
-template <typename T>
+template <typename T, int CH>
 cudaError_t launch_typed(const ConvArgs& a, int W, unsigned blocks, cudaStream_t s) {
     const unsigned th = 32 * kWarps;
     switch (W) {
-        case 1: short_conv_kernel<T, 1><<<blocks, th, 0, s>>>(a); break;
-        case 2: short_conv_kernel<T, 2><<<blocks, th, 0, s>>>(a); break;
-        case 3: short_conv_kernel<T, 3><<<blocks, th, 0, s>>>(a); break;
-        case 4: short_conv_kernel<T, 4><<<blocks, th, 0, s>>>(a); break;
-        case 5: short_conv_kernel<T, 5><<<blocks, th, 0, s>>>(a); break;
-        case 6: short_conv_kernel<T, 6><<<blocks, th, 0, s>>>(a); break;
-        case 7: short_conv_kernel<T, 7><<<blocks, th, 0, s>>>(a); break;
-        case 8: short_conv_kernel<T, 8><<<blocks, th, 0, s>>>(a); break;
+        case 1: short_conv_kernel<T, 1, CH><<<blocks, th, 0, s>>>(a); break;
+        case 2: short_conv_kernel<T, 2, CH><<<blocks, th, 0, s>>>(a); break;
+        case 3: short_conv_kernel<T, 3, CH><<<blocks, th, 0, s>>>(a); break;
+        case 4: short_conv_kernel<T, 4, CH><<<blocks, th, 0, s>>>(a); break;
+        case 5: short_conv_kernel<T, 5, CH><<<blocks, th, 0, s>>>(a); break;
+        case 6: short_conv_kernel<T, 6, CH><<<blocks, th, 0, s>>>(a); break;
+        case 7: short_conv_kernel<T, 7, CH><<<blocks, th, 0, s>>>(a); break;
+        case 8: short_conv_kernel<T, 8, CH><<<blocks, th, 0, s>>>(a); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
+}
+
+template <typename T, int CH>
+cudaError_t launch_ch(const ConvArgs& a, int W, cudaStream_t stream) {
+    const long long items =
+        (long long)a.B * ((a.T + kSeg - 1) / kSeg) * ((a.C + 32 * CH - 1) / (32 * CH));
+    if (items <= 0) return cudaSuccess;
+    const long long blocks = (items + kWarps - 1) / kWarps;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    return launch_typed<T, CH>(a, W, (unsigned)blocks, stream);
 }
 
 }  // namespace
@@ -236,14 +329,8 @@ cudaError_t launch_typed(const ConvArgs& a, int W, unsigned blocks, cudaStream_t
 cudaError_t launch_short_conv(const void* x, const float* w, const int32_t* cu, int N, void* y,
                               int B, int T, int C, int W, bool bf16, int act, int group, float eps,
                               unsigned* err, cudaStream_t stream) {
-    const int run = bf16 ? run_of<__nv_bfloat16>() : run_of<float>();
-    const long long items = (long long)B * ((T + run - 1) / run) * ((C + 127) / 128);
-    if (items <= 0) return cudaSuccess;
-    const long long blocks = (items + kWarps - 1) / kWarps;
-    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     ConvArgs a{x, w, cu, N, y, B, T, C, act, group, eps, err};
-    return bf16 ? launch_typed<__nv_bfloat16>(a, W, (unsigned)blocks, stream)
-                : launch_typed<float>(a, W, (unsigned)blocks, stream);
+    return bf16 ? launch_ch<__nv_bfloat16, kCh>(a, W, stream) : launch_ch<float, kCh>(a, W, stream);
 }
 
 }  // namespace kda

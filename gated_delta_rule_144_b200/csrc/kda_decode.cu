@@ -165,9 +165,11 @@ decode_d128_tokens_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                           Tin* __restrict__ o, int H, int T, long long units, unsigned* err) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     float* sbuf = reinterpret_cast<float*>(smem_raw);             // next unit's state
-    __shared__ __align__(16) float s_q[kRowGroup][kD], s_k[kRowGroup][kD], s_g[kRowGroup][kD],
-        s_v[kRowGroup][kD];
-    __shared__ float s_b[kRowGroup];
+    // token rows staged per lane's access order: element r of q, k, g at [r % 4][r / 4], so that a
+    // lane (row phase r % 4) reads its 32 rows as 8 float4; v in natural order; q.k per row
+    __shared__ __align__(16) float s_q[kRowGroup][4][32], s_k[kRowGroup][4][32],
+        s_g[kRowGroup][4][32], s_v[kRowGroup][kD];
+    __shared__ float s_b[kRowGroup], s_qk[kRowGroup];
     __shared__ __align__(8) unsigned long long s_bar;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int phase = lane >> 3;
@@ -221,28 +223,53 @@ decode_d128_tokens_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
             if (t0 > 0) __syncthreads();   // the previous group's rows are no longer read
             for (int u = 0; u < nt; ++u) {
                 const size_t r = row(t0 + u);
-                s_q[u][tid] = load_elem(q, r * kD + tid);
-                s_k[u][tid] = load_elem(k, r * kD + tid);
-                s_g[u][tid] = expf(log_g[r * kD + tid]);
+                const float qv = load_elem(q, r * kD + tid), kv = load_elem(k, r * kD + tid);
+                s_q[u][tid & 3][tid >> 2] = qv;
+                s_k[u][tid & 3][tid >> 2] = kv;
+                s_g[u][tid & 3][tid >> 2] = expf(log_g[r * kD + tid]);
                 s_v[u][tid] = load_elem(v, r * kD + tid);
             }
             if (tid < nt) s_b[tid] = load_elem(beta, row(t0 + tid));
             __syncthreads();
+            // q.k per row, once (warp u % 4 for row u), in the single step's order: lane l sums
+            // rows l / 8 + 4 i over i, then a butterfly over the four row phases
+            if ((lane & 7) == 0) {
+                for (int u = warp; u < nt; u += 4) {
+                    float qk = 0.f;
+#pragma unroll
+                    for (int i = 0; i < kRowsPerLane; ++i)
+                        qk = fmaf(s_q[u][phase][i], s_k[u][phase][i], qk);
+                    // combine the four phases as xor 8, then 16 would: (0 + 1) + (2 + 3)
+                    const unsigned lanes = 0x01010101u;
+                    const float a0 = __shfl_sync(lanes, qk, 0), a1 = __shfl_sync(lanes, qk, 8);
+                    const float a2 = __shfl_sync(lanes, qk, 16), a3 = __shfl_sync(lanes, qk, 24);
+                    if (lane == 0) s_qk[u] = (a0 + a1) + (a2 + a3);
+                }
+            }
+            __syncthreads();
             for (int u = 0; u < nt; ++u) {
                 const float4 vv = *reinterpret_cast<const float4*>(&s_v[u][col]);
                 const float b = s_b[u];
+                const float qk = s_qk[u];
                 float4 m = make_float4(0.f, 0.f, 0.f, 0.f), p = m;
-                float qk = 0.f;
+                const float4* g4 = reinterpret_cast<const float4*>(s_g[u][phase]);
+                const float4* k4 = reinterpret_cast<const float4*>(s_k[u][phase]);
+                const float4* q4 = reinterpret_cast<const float4*>(s_q[u][phase]);
 #pragma unroll
-                for (int i = 0; i < kRowsPerLane; ++i) {
-                    const int r = phase + 4 * i;
-                    const float g = s_g[u][r], kr = s_k[u][r], qr = s_q[u][r];
-                    s[i].x *= g; s[i].y *= g; s[i].z *= g; s[i].w *= g;
-                    m.x = fmaf(kr, s[i].x, m.x); m.y = fmaf(kr, s[i].y, m.y);
-                    m.z = fmaf(kr, s[i].z, m.z); m.w = fmaf(kr, s[i].w, m.w);
-                    p.x = fmaf(qr, s[i].x, p.x); p.y = fmaf(qr, s[i].y, p.y);
-                    p.z = fmaf(qr, s[i].z, p.z); p.w = fmaf(qr, s[i].w, p.w);
-                    qk = fmaf(qr, kr, qk);
+                for (int i4 = 0; i4 < kRowsPerLane / 4; ++i4) {
+                    const float4 gg = g4[i4], kk = k4[i4], qq = q4[i4];
+                    const float ga[4] = {gg.x, gg.y, gg.z, gg.w}, ka[4] = {kk.x, kk.y, kk.z, kk.w},
+                                qa[4] = {qq.x, qq.y, qq.z, qq.w};
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int i = 4 * i4 + jj;
+                        const float g = ga[jj], kr = ka[jj], qr = qa[jj];
+                        s[i].x *= g; s[i].y *= g; s[i].z *= g; s[i].w *= g;
+                        m.x = fmaf(kr, s[i].x, m.x); m.y = fmaf(kr, s[i].y, m.y);
+                        m.z = fmaf(kr, s[i].z, m.z); m.w = fmaf(kr, s[i].w, m.w);
+                        p.x = fmaf(qr, s[i].x, p.x); p.y = fmaf(qr, s[i].y, p.y);
+                        p.z = fmaf(qr, s[i].z, p.z); p.w = fmaf(qr, s[i].w, p.w);
+                    }
                 }
 #pragma unroll
                 for (int off = 8; off <= 16; off <<= 1) {
@@ -254,7 +281,6 @@ decode_d128_tokens_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                     p.y += __shfl_xor_sync(0xffffffffu, p.y, off);
                     p.z += __shfl_xor_sync(0xffffffffu, p.z, off);
                     p.w += __shfl_xor_sync(0xffffffffu, p.w, off);
-                    qk += __shfl_xor_sync(0xffffffffu, qk, off);
                 }
                 float4 d;
                 d.x = b * (vv.x - m.x); d.y = b * (vv.y - m.y);
@@ -266,10 +292,16 @@ decode_d128_tokens_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                     store_v4(o + row(t0 + u) * kD + col, out);
                 }
 #pragma unroll
-                for (int i = 0; i < kRowsPerLane; ++i) {
-                    const float kr = s_k[u][phase + 4 * i];
-                    s[i].x = fmaf(kr, d.x, s[i].x); s[i].y = fmaf(kr, d.y, s[i].y);
-                    s[i].z = fmaf(kr, d.z, s[i].z); s[i].w = fmaf(kr, d.w, s[i].w);
+                for (int i4 = 0; i4 < kRowsPerLane / 4; ++i4) {
+                    const float4 kk = k4[i4];
+                    const float ka[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int i = 4 * i4 + jj;
+                        const float kr = ka[jj];
+                        s[i].x = fmaf(kr, d.x, s[i].x); s[i].y = fmaf(kr, d.y, s[i].y);
+                        s[i].z = fmaf(kr, d.z, s[i].z); s[i].w = fmaf(kr, d.w, s[i].w);
+                    }
                 }
             }
         }

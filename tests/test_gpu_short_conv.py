@@ -66,6 +66,20 @@ def test_batch_rows_and_a_partial_channel_warp(dtype, tol):
     assert rel_l2(host(y), ref) <= tol
 
 
+@pytest.mark.parametrize("dtype,tol", [(torch.bfloat16, TOL_BF16), (torch.float32, TOL_F32)],
+                         ids=["bf16", "fp32"])
+def test_partial_warp_span_and_one_lane_groups(dtype, tol):
+    """C = 100 channels (a warp's 128-channel span is partly idle) and a norm group of 4 (one lane
+    per group, no shuffles); packed documents, W = 2."""
+    lengths = [9, 30, 1, 20]
+    x, w, cu = _inputs(1, sum(lengths), 100, 2, dtype, 9, lengths)
+    y = kda.short_conv(x.to(DEV), w.to(DEV), cu.to(DEV), activation="silu", norm_group=4)
+    torch.cuda.synchronize()
+    assert kda.get_device_error() == 0
+    ref = oracle_conv(host(x), host(w), cu.numpy(), activation="silu", norm_group=4)
+    assert rel_l2(host(y), ref) <= tol
+
+
 def test_packed_8docs_shape_full_size():
     """The packed 8-document workload's q shape (28937 tokens, 32 heads x 128 channels), W = 4,
     SiLU and a per-head L2 norm, every element against the oracle."""
