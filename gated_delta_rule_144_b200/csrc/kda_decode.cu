@@ -149,12 +149,15 @@ __device__ __forceinline__ bool bar_try(uint32_t bar, uint32_t parity) {
         : "memory");
     return done != 0;
 }
-// bounded wait (about a second of SM clock): false on expiry
+// bounded wait (about a second of SM clock): false on expiry; the clock (a slow read) only once
+// the first test has failed
 __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
+    if (bar_try(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!bar_try(bar, parity))
+    for (;;) {
+        if (bar_try(bar, parity)) return true;
         if (clock64() - t0 > (1ll << 31)) return false;
-    return true;
+    }
 }
 
 template <typename Tin>

@@ -23,7 +23,7 @@
 // Q+ and K_end go from registers straight to the workspace. The next record's input tiles are
 // prefetched into L2 while this one runs.
 //
-// Per record (256 threads; thread 0 issues the MMAs, lane 0 of warp 7 the copies):
+// Per record (256 threads; warp 0 issues the MMAs, lane 0 of warp 7 the copies):
 //   TMA k, q, log g -> decay products -> TMA V; R, C, K+ (shared), Q+, K_end (global) ->
 //   MMA R C^T -> A_kk, A_qk (TMA store of A_qk) -> UT solve -> MMA [T; -] K+ and V^T T^T ->
 //   W, U~^T staged in shared memory -> TMA stores.
@@ -682,20 +682,17 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         __syncthreads();
 
         // ---------------------------------------------------------------- MMA: R C^T
-        if (warp == 0) {   // lane 0 issues; the rest of warp 0 waits for it
-            if (lane == 0) {
-                tc_fence_after();
-                const uint32_t id = idesc_bf16(128, 160, 0, 0);
+        if (warp == 0) {   // the whole warp runs the issue code; one elected lane issues
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, 160, 0, 0);
 #pragma unroll
-                for (int s = 0; s < kD / 16; ++s) {
-                    const int k0 = 16 * s;
-                    const uint64_t ad = desc_at(dK, sb + OFF_R + (k0 >> 6) * 16384 + (k0 & 63) * 2);
-                    const uint64_t bd = desc_at(dK, sb + OFF_C + (k0 >> 6) * 20480 + (k0 & 63) * 2);
-                    umma_f16(tbase + TM_A, ad, bd, id, s > 0);
-                }
-                umma_commit(bar_mma);
+            for (int s = 0; s < kD / 16; ++s) {
+                const int k0 = 16 * s;
+                const uint64_t ad = desc_at(dK, sb + OFF_R + (k0 >> 6) * 16384 + (k0 & 63) * 2);
+                const uint64_t bd = desc_at(dK, sb + OFF_C + (k0 >> 6) * 20480 + (k0 & 63) * 2);
+                umma_f16_warp(tbase + TM_A, ad, bd, id, s > 0);
             }
-            __syncwarp();
+            umma_commit_warp(bar_mma);
         }
         mma_pending = true;
 
@@ -910,22 +907,19 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
         ++v_count;
         v_pending = false;
         if (warp == 0) {
-            if (lane == 0) {
-                tc_fence_after();
-                const uint32_t id = idesc_bf16(128, 128, 0, 1);
-                const uint32_t idt = idesc_bf16(128, 64, 1, 0);
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, 128, 0, 1);
+            const uint32_t idt = idesc_bf16(128, 64, 1, 0);
 #pragma unroll
-                for (int s = 0; s < kC / 16; ++s)
-                    umma_f16(tbase + TM_A, desc_at(dK, sb + OFF_TT + 32 * s),
-                             desc_at(dM8, sb + OFF_KP + 2048 * s), id, s > 0);
-                umma_commit(bar_mma);   // W: read out while the next product runs
+            for (int s = 0; s < kC / 16; ++s)
+                umma_f16_warp(tbase + TM_A, desc_at(dK, sb + OFF_TT + 32 * s),
+                              desc_at(dM8, sb + OFF_KP + 2048 * s), id, s > 0);
+            umma_commit_warp(bar_mma);   // W: read out while the next product runs
 #pragma unroll
-                for (int s = 0; s < kC / 16; ++s)
-                    umma_f16(tbase + TM_A + 128, desc_at(dM8, sb + OFF_V + 2048 * s),
-                             desc_at(dK, sb + OFF_TT + 32 * s), idt, s > 0);
-                umma_commit(bar_wy2);
-            }
-            __syncwarp();
+            for (int s = 0; s < kC / 16; ++s)
+                umma_f16_warp(tbase + TM_A + 128, desc_at(dM8, sb + OFF_V + 2048 * s),
+                              desc_at(dK, sb + OFF_TT + 32 * s), idt, s > 0);
+            umma_commit_warp(bar_wy2);
         }
         mma_pending = wy2_pending = true;
         if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }

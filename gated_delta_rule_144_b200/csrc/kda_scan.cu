@@ -23,9 +23,11 @@
 // Roles (14 warps):
 //   - 8 chain warps walk the chunks: warps w and w + 4 share TMEM lane quarter w mod 4 (lane j =
 //     value column j) and split the columns of every TMEM row between them. Per chunk c the chain
-//     is bf16(S^T) -> D (8 K steps) -> U^T = U~^T - (W S)^T -> S^T += U^T K_end (4 K steps); the
+//     is bf16(S^T) -> (W S)^T (8 K steps; the (Q+ S)^T half of D follows it in the pipe, off the
+//     chain) -> U^T = U~^T - (W S)^T -> S^T += U^T K_end (4 K steps); the
 //     decay of S^T and the load of U~^T run while D is in flight.
-//   - 1 MMA warp: one thread issues every tcgen05.mma.
+//   - 1 MMA warp: issues every tcgen05.mma (the whole warp runs the issue code, one elected lane
+//     issues, so that the operands stay warp-uniform).
 //   - 4 epilogue warps (one per lane quarter) take o of chunk c out of TMEM once its product is
 //     done, stage it row-major in shared memory (applying the norm when asked, with the gate
 //     tile of chunk c fetched by TMA a chunk ahead) and store it, so that none of the output's
@@ -62,7 +64,8 @@ constexpr int kEpiWarps = 4;
 constexpr int kChainThreads = 32 * kDataWarps + 32;          // chain warps + the MMA warp
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kThreads = kChainThreads + kEpiThreads + 32;     // + the loader warp
-constexpr int kMma = 32 * kDataWarps;    // thread that issues the MMAs
+constexpr int kMma = 32 * kDataWarps;    // first thread of the warp that issues the MMAs
+constexpr int kMmaWarp = kDataWarps;
 constexpr int kEpi0 = kChainThreads;     // first epilogue thread (issues the output stores)
 constexpr int kLoader = kChainThreads + kEpiThreads;   // thread that issues the record copies
 constexpr uint32_t kBarChain = 1, kBarEpi = 2;   // named barriers (0 is __syncthreads)
@@ -275,9 +278,8 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         // ============================================================ chain warps and MMA warp
         const uint64_t dK = sw128_desc(0, 16, 1024);     // K-major, 128B swizzle
         const uint64_t dM8 = sw128_desc(0, 8192, 1024);  // MN-major, 64-row panels
-        const uint32_t id1 = idesc_bf16(128, 128, 0, 0);
+        const uint32_t id_half = idesc_bf16(128, 64, 0, 0);   // D halves and the o product
         const uint32_t id2 = idesc_bf16(128, 128, 0, 1);
-        const uint32_t id3 = idesc_bf16(128, 64, 0, 0);
 
         // outstanding MMAs, drained before exit if a wait expires (the record copies are the
         // epilogue's to drain)
@@ -329,27 +331,37 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
 
             // ------------------------------------------------------------ D = S^T [W; Q+]^T
             bool mma_bad = false;
-            if (tid == kMma) {
+            if (warp == kMmaWarp) {
                 // D buffer c & 1 last held chunk c-2's product: wait until the epilogue has
                 // read its o (long done in steady state)
-                if (c >= 2)
+                if (c >= 2 && lane == 0)
                     mma_bad = !mbar_wait(bar_dfree0 + 8 * (c & 1), (uint32_t)(((c - 2) >> 1) & 1),
                                          args.budget);
+                mma_bad = __shfl_sync(0xffffffffu, mma_bad, 0);
                 if (!mma_bad) {
                     tc_fence_after();
+                    // (W S)^T first, committed on its own: the chain needs only this half; the
+                    // (Q+ S)^T half follows in the pipe while the chain forms U
 #pragma unroll
                     for (int s = 0; s < kD / 16; ++s)
-                        umma_f16_ts(tbase + TD + 128 * (c & 1), tbase + TB + 8 * s,
-                                    desc_at(dK, st + ST_WQ + (s >> 2) * 16384 + (s & 3) * 32),
-                                    id1, s > 0);
-                    umma_commit(bar_mma1);
+                        umma_f16_ts_warp(tbase + TD + 128 * (c & 1), tbase + TB + 8 * s,
+                                         desc_at(dK, st + ST_WQ + (s >> 2) * 16384 + (s & 3) * 32),
+                                         id_half, s > 0);
+                    umma_commit_warp(bar_mma1);
+#pragma unroll
+                    for (int s = 0; s < kD / 16; ++s)
+                        umma_f16_ts_warp(
+                            tbase + TD + 128 * (c & 1) + 64, tbase + TB + 8 * s,
+                            desc_at(dK, st + ST_WQ + 8192 + (s >> 2) * 16384 + (s & 3) * 32),
+                            id_half, s > 0);
                 }
             }
             mma1_pending = true;
             mma1_chunk = c;
 
             // ------------------------------------------------------------ while D runs
-            // decay: TS = S^T diag(e^{Gamma_end}) (the update accumulates into it); U~^T rows
+            // decay: S^T diag(e^{Gamma_end}) in registers (stored into TS, where the update
+            // accumulates, with U^T below); U~^T rows
             uint32_t ub[16];
             if (data) {
                 float va[32], vb[32];
@@ -396,19 +408,19 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
             tc_fence_after();
 
             // ------------------------------------------------------------ S^T += U^T K_end
-            if (tid == kMma) {
+            if (warp == kMmaWarp) {
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < kC / 16; ++s)
-                    umma_f16_ts(tbase + TS, tbase + TU + 8 * s,
-                                desc_at(dM8, st + ST_KE + 2048 * s), id2, 1);
-                umma_commit(bar_mma2);
+                    umma_f16_ts_warp(tbase + TS, tbase + TU + 8 * s,
+                                     desc_at(dM8, st + ST_KE + 2048 * s), id2, 1);
+                umma_commit_warp(bar_mma2);
                 // o^T = (Q+ S)^T + U^T A_qk^T, behind the update in the pipe (off the chain)
 #pragma unroll
                 for (int s = 0; s < kC / 16; ++s)
-                    umma_f16_ts(tbase + TD + 128 * (c & 1) + 64, tbase + TU + 8 * s,
-                                desc_at(dK, st + ST_AQ + 32 * s), id3, 1);
-                umma_commit(bar_o0 + 8 * (c & 1));
+                    umma_f16_ts_warp(tbase + TD + 128 * (c & 1) + 64, tbase + TU + 8 * s,
+                                     desc_at(dK, st + ST_AQ + 32 * s), id_half, 1);
+                umma_commit_warp(bar_o0 + 8 * (c & 1));
             }
             mma2_pending = o_pending = true;
             mma2_chunk = o_chunk = c;

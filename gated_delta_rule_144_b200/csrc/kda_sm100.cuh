@@ -63,21 +63,28 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 
 // Wait for the phase with the given parity to complete, giving up after `budget` SM clock
 // cycles. Returns false on timeout (the caller records the error and winds down).
+// The clock is read only once the first test has failed: on B200 a clock64() read costs about
+// 170 cycles, against about 10 for a try_wait that finds the phase complete, and most waits on a
+// critical chain find it so.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long budget) {
+    if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
         if (clock64() - t0 > budget) return false;
     }
-    return true;
 }
 
 // The same with the suspending try_wait (for throughput kernels that share an SM).
 __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, long long budget) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait_sleep(bar, parity)) {
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity)) return true;
         if (clock64() - t0 > budget) return false;
     }
-    return true;
 }
 
 // ------------------------------------------------------------------ TMA
@@ -192,6 +199,41 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// The same two products issued from a whole converged warp: every lane executes the call with
+// the same (warp-uniform) operands and one elected lane issues the instruction. Issued this way
+// the operands stay in uniform registers; measured on B200, 8 back-to-back M = 128, N = 128
+// products issue in about 350 cycles this way against about 475 from a single thread (and 690
+// from a single thread in a loop that is not unrolled).
+__device__ __forceinline__ void umma_f16_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_f16_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// umma_commit from a whole converged warp (one elected lane commits).
+__device__ __forceinline__ void umma_commit_warp(uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+            bar)
         : "memory");
 }
 
