@@ -299,19 +299,19 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
             const uint32_t st = sb + (uint32_t)(c & 1) * kStage;
             const uint8_t* stp = sm + (size_t)(c & 1) * kStage;
 
-            // records of chunk c landed; S of chunk c complete once the previous update has
+            // records of chunk c landed; S of chunk c complete once the previous update has.
+            // Every chain thread waits itself (bounded) and the outcome is agreed on at the
+            // barrier after the conversion, so no barrier of its own sits on the chain.
             bool ok = true;
-            if (tid == 0) {
+            if (data) {
                 ok = mbar_wait(bar_full0 + 8 * (c & 1), (uint32_t)((c >> 1) & 1), args.budget);
                 if (ok && mma2_pending)
                     ok = mbar_wait(bar_mma2, (uint32_t)(mma2_chunk & 1), args.budget);
+                tc_fence_after();
             }
-            if (bar_or(kBarChain, kChainThreads, !ok)) { aborted = true; break; }
-            mma2_pending = false;
-            tc_fence_after();
 
             // ------------------------------------------------------------ bf16 S^T -> TB
-            if (data) {
+            if (data && ok) {
                 float va[32], vb[32];
                 tmem_ld32(tbase + lq + TS + 64 * hs, va);
                 tmem_ld32(tbase + lq + TS + 64 * hs + 32, vb);
@@ -326,7 +326,8 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
                 tmem_st_wait();
             }
             tc_fence_before();
-            bar_sync(kBarChain, kChainThreads);
+            if (bar_or(kBarChain, kChainThreads, !ok)) { aborted = true; break; }
+            mma2_pending = false;
             tc_fence_after();
 
             // ------------------------------------------------------------ D = S^T [W; Q+]^T
@@ -387,12 +388,15 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
                 tmem_st_wait();
             }
 
-            if (!wait_chain(bar_mma1, (uint32_t)(c & 1), mma_bad)) { aborted = true; break; }
-            mma1_pending = false;
-            tc_fence_after();
+            // (W S)^T done: again each chain thread waits itself, agreed on at the next barrier
+            bool ok1 = true;
+            if (data) {
+                ok1 = mbar_wait(bar_mma1, (uint32_t)(c & 1), args.budget);
+                tc_fence_after();
+            }
 
             // ------------------------------------------------------------ U^T = U~^T - (W S)^T
-            if (data) {
+            if (data && ok1) {
                 float w[32];
                 tmem_ld32(tbase + lq + TD + 128 * (c & 1) + 32 * hs, w);
                 tmem_ld_wait();
@@ -404,7 +408,8 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
                 tmem_st_wait();
             }
             tc_fence_before();
-            bar_sync(kBarChain, kChainThreads);
+            if (bar_or(kBarChain, kChainThreads, !ok1 || mma_bad)) { aborted = true; break; }
+            mma1_pending = false;
             tc_fence_after();
 
             // ------------------------------------------------------------ S^T += U^T K_end
