@@ -169,9 +169,12 @@ decode_d128_tokens_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     float* sbuf = reinterpret_cast<float*>(smem_raw);             // next unit's state
     // token rows staged per lane's access order: element r of q, k, g at [r % 4][r / 4], so that a
-    // lane (row phase r % 4) reads its 32 rows as 8 float4; v in natural order; q.k per row
-    __shared__ __align__(16) float s_q[kRowGroup][4][32], s_k[kRowGroup][4][32],
-        s_g[kRowGroup][4][32], s_v[kRowGroup][kD];
+    // lane (row phase r % 4) reads its 32 rows as 8 float4; the phases 36 floats apart, so that
+    // a warp's four phases fall in different banks (32 apart they would share them, four ways);
+    // v in natural order; q.k per row
+    constexpr int kPh = 36;
+    __shared__ __align__(16) float s_q[kRowGroup][4][kPh], s_k[kRowGroup][4][kPh],
+        s_g[kRowGroup][4][kPh], s_v[kRowGroup][kD];
     __shared__ float s_b[kRowGroup], s_qk[kRowGroup];
     __shared__ __align__(8) unsigned long long s_bar;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;

@@ -344,9 +344,29 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
     // for equal-length sequences idx runs over (sequence, chunk in this launch's span, head).
     const long long total = args.cu ? args.G * H : (long long)args.N * args.c_span * H;
     auto decode = [&](long long idx, Unit& u) -> bool {
-        u.h = (int)(idx % H);
+        // q = idx / H, and for equal-length sequences sequence sq, chunk-in-span cr = q / c_span,
+        // q % c_span: 32-bit divisions whenever the launch's indices fit (a 64-bit division is a
+        // long software sequence, and every thread decodes each record)
+        long long q, sq = 0, cr = 0;
+        if (total <= 0x7fffffffLL) {
+            const uint32_t i32 = (uint32_t)idx, h32 = (uint32_t)H, q32 = i32 / h32;
+            u.h = (int)(i32 - q32 * h32);
+            q = q32;
+            if (!args.cu) {
+                const uint32_t cs = (uint32_t)args.c_span, s32 = q32 / cs;
+                sq = s32;
+                cr = q32 - s32 * cs;
+            }
+        } else {
+            u.h = (int)(idx % H);
+            q = idx / H;
+            if (!args.cu) {
+                sq = q / args.c_span;
+                cr = q % args.c_span;
+            }
+        }
         if (args.cu) {
-            const long long g = idx / H;
+            const long long g = q;
             u.rec = idx;
             const int d = args.map[g];
             if (d < 0 || d >= args.N) return false;
@@ -357,9 +377,7 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
             u.row0 = a + kC * cc;
             u.L = (int)min((long long)kC, b - u.row0);
         } else {
-            const long long per_seq = (long long)args.c_span * H;
-            const long long sq = idx / per_seq;
-            const long long cc = args.c_begin + (idx % per_seq) / H;
+            const long long cc = args.c_begin + cr;
             u.rec = (sq * args.ncT + cc) * H + u.h;
             u.row0 = sq * args.T + kC * cc;
             u.L = (int)min((long long)kC, (long long)args.T - kC * cc);

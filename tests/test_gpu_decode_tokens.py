@@ -37,9 +37,10 @@ def _run(inp):
     return o, S
 
 
-@pytest.mark.parametrize("T", [1, 2, 4, 7])
+@pytest.mark.parametrize("T", [1, 2, 4, 7, 8, 9, 20])
 @pytest.mark.parametrize("dtype,tol", [("bf16", TOL_BF16), ("f32", TOL_F32)])
 def test_rows_match_the_oracle(T, dtype, tol):
+    """T up to 8 arrives with the state (prefetched rows); 9 and 20 add groups read later."""
     inp = synth.decode_tokens_inputs(N=6, T=T, H=3, dtype=dtype, seed=60 + T, device=DEV)
     o, S = _run(inp)
     o_ref, S_ref = _oracle(inp, inp["S"])
@@ -56,12 +57,13 @@ def test_general_head_sizes_take_the_per_token_walk(dk, dv):
     assert rel_l2(host(o), o_ref) <= TOL_F32 and rel_l2(host(S), S_ref) <= TOL_F32
 
 
+@pytest.mark.parametrize("T,N,H", [(5, 8, 4), (11, 40, 8)])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_rows_equal_successive_decode_steps_bit_for_bit(dtype):
+def test_rows_equal_successive_decode_steps_bit_for_bit(dtype, T, N, H):
     """T rows in one call = T calls of kda_decode_step: the state stays fp32 in registers between
-    rows exactly as it would in memory, and each row's arithmetic runs in the same order."""
-    T = 5
-    inp = synth.decode_tokens_inputs(N=8, T=T, H=4, dtype=dtype, seed=80, device=DEV)
+    rows exactly as it would in memory, and each row's arithmetic runs in the same order. 40 x 8
+    units exceed the persistent grid, so blocks walk several units with prefetched rows."""
+    inp = synth.decode_tokens_inputs(N=N, T=T, H=H, dtype=dtype, seed=80, device=DEV)
     o, S = _run(inp)
     S2 = inp["S"].clone()
     for t in range(T):
