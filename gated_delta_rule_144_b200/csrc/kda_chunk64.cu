@@ -628,8 +628,7 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         __syncthreads();
 
         // ---------------------------------------------------------------- MMA: R C^T
-        if (warp == 0) {   // lane 0 issues; the rest of warp 0 waits for it
-            if (lane == 0) {
+        if (warp == 0) {   // the whole warp runs the issue code; one elected lane issues
             tc_fence_after();
             const uint32_t id = idesc_bf16(128, 160, 0, 0);
 #pragma unroll
@@ -639,11 +638,9 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     desc_at(dK, sb + OFF_R + (k0 >> 6) * 16384 + (k0 & 63) * 2);
                 const uint64_t bd =
                     desc_at(dK, sb + OFF_C + (k0 >> 6) * 20480 + (k0 & 63) * 2);
-                umma_f16(tbase + TM_A, ad, bd, id, s > 0);
+                umma_f16_warp(tbase + TM_A, ad, bd, id, s > 0);
             }
-            umma_commit(bar_mma);
-            }
-            __syncwarp();
+            umma_commit_warp(bar_mma);
         }
         mma_pending = true;
 
@@ -861,17 +858,14 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
         // ---------------------------------------------------------------- MMA: T' = A_qk T
         // [0; A_qk] (128 x 64) times T as the MN-major B operand: lanes 64-127 receive A_qk T.
-        if (warp == 0) {   // lane 0 issues; the rest of warp 0 waits for it
-            if (lane == 0) {
-                tc_fence_after();
-                const uint32_t id = idesc_bf16(128, 64, 0, 1);
+        if (warp == 0) {   // the whole warp runs the issue code; one elected lane issues
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
-                for (int s = 0; s < kC / 16; ++s)
-                    umma_f16(tbase + TM_TP, desc_at(dK, sb + OFF_ZA + 32 * s),
-                             desc_at(dM8, sb + OFF_TT + 2048 * s), id, s > 0);
-                umma_commit(bar_mma);
-            }
-            __syncwarp();
+            for (int s = 0; s < kC / 16; ++s)
+                umma_f16_warp(tbase + TM_TP, desc_at(dK, sb + OFF_ZA + 32 * s),
+                              desc_at(dM8, sb + OFF_TT + 2048 * s), id, s > 0);
+            umma_commit_warp(bar_mma);
         }
         mma_pending = true;
         if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
@@ -898,16 +892,13 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (!wait_all(bar_v, c & 1)) { aborted = true; break; }
         v_pending = false;
         if (warp == 0) {
-            if (lane == 0) {
                 tc_fence_after();
                 const uint32_t id = idesc_bf16(128, 128 + kDV, 0, 1);
 #pragma unroll
                 for (int s = 0; s < kC / 16; ++s)
-                    umma_f16(tbase + TM_A, desc_at(dK, sb + OFF_TT + 32 * s),
-                             desc_at(dM8, sb + OFF_KPV + 2048 * s), id, s > 0);
-                umma_commit(bar_mma);
-            }
-            __syncwarp();
+                    umma_f16_warp(tbase + TM_A, desc_at(dK, sb + OFF_TT + 32 * s),
+                                  desc_at(dM8, sb + OFF_KPV + 2048 * s), id, s > 0);
+                umma_commit_warp(bar_mma);
         }
         mma_pending = true;
         if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
@@ -971,19 +962,16 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
             // ---------------------------------------------------------------- MMA: [W; Q~] S
             if (warp == 0) {
-                if (lane == 0) {
-                    tc_fence_after();
-                    const uint32_t id = idesc_bf16(128, kDV, 0, 1);
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, kDV, 0, 1);
     #pragma unroll
-                    for (int s = 0; s < kD / 16; ++s) {
-                        const int k0 = 16 * s;
-                        umma_f16(tbase + TM_B,
-                                 desc_at(dK, sb + OFF_WQ + (k0 >> 6) * 16384 + (k0 & 63) * 2),
-                                 desc_at(dM16, sb + OFF_S16 + 2048 * s), id, s > 0);
-                    }
-                    umma_commit(bar_mma);
+                for (int s = 0; s < kD / 16; ++s) {
+                    const int k0 = 16 * s;
+                    umma_f16_warp(tbase + TM_B,
+                                  desc_at(dK, sb + OFF_WQ + (k0 >> 6) * 16384 + (k0 & 63) * 2),
+                                  desc_at(dM16, sb + OFF_S16 + 2048 * s), id, s > 0);
                 }
-                __syncwarp();
+                umma_commit_warp(bar_mma);
             }
             mma_pending = true;
             if (!wait_all(bar_mma, mma_phase & 1)) { aborted = true; break; }
@@ -1024,19 +1012,16 @@ chunk64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             __syncthreads();
 
             // ---------------------------------------------------------------- MMA: S += K_end^T U
-            if (warp == 0) {   // lane 0 issues; the rest of warp 0 waits for it
-                if (lane == 0) {
+            if (warp == 0) {   // the whole warp runs the issue code; one elected lane issues
                 tc_fence_after();
                 const uint32_t id = idesc_bf16(128, kDV, 1, 1);
     #pragma unroll
                 for (int s = 0; s < kC / 16; ++s) {
                     const uint64_t ae = desc_at(dM8, sb + OFF_KE + 2048 * s);
                     const uint64_t bu = desc_at(dM8, sb + OFF_U16 + 2048 * s);
-                    umma_f16(tbase + TM_S, ae, bu, id, 1);
+                    umma_f16_warp(tbase + TM_S, ae, bu, id, 1);
                 }
-                umma_commit(bar_b4);
-                }
-                __syncwarp();
+                umma_commit_warp(bar_b4);
             }
             b4_pending = true;
             b4_chunk = c;
