@@ -141,6 +141,7 @@ KERNEL_SOURCES = {
     "kda_chunk64": ["kda_chunk64.cu", "kda_sm100.cuh", "kda_internal.cuh", "kda_tma.cuh"],
     "kda_chunk64_intra": ["kda_intra.cu", "kda_sm100.cuh", "kda_internal.cuh", "kda_tma.cuh"],
     "kda_chunk_scan": ["kda_scan.cu", "kda_sm100.cuh", "kda_internal.cuh", "kda_tma.cuh"],
+    "kda_short_conv": ["kda_conv.cu", "kda_internal.cuh"],
 }
 
 
@@ -443,7 +444,9 @@ def run_secondary(kda, synth, args, dev, stream, world, rank):
                           "GB/s": round(gbs * world, 1), "GB/s_per_gpu": round(gbs, 1),
                           "roofline_frac": round(gbs / hbm_peak, 4), "peak": hbm_peak,
                           "tokens/s": round(256 * 4 * world / (ms / 1e3), 1),
-                          "kernel": "kda_decode_tokens_d128"}
+                          "kernel": "kda_decode_tokens_d128",
+                          "traffic": committed_traffic("kda_decode_tokens_d128",
+                                                       "decode-rows-n256-t4")}
     del d, od
     # packed 8-document prefill (H = 32)
     p = synth.prefill_inputs("packed-8docs", device=dev, seed=shard.rank_seed(1002, rank))
@@ -551,7 +554,8 @@ def run_secondary(kda, synth, args, dev, stream, world, rank):
                        "W": 4, "activation": "silu", "norm_group": 128,
                        "ms_per_call": round(ms, 4), "bytes_per_call": by,
                        "roofline_frac": round(by / (ms / 1e3) / 1e9 / hbm_peak, 4),
-                       "kernel": "short_conv_kernel"}
+                       "kernel": "short_conv_kernel",
+                       "traffic": committed_traffic("kda_short_conv", "packed-8docs")}
     del px, pw, py
     # gradients (kda_bwd) on the T=4096, H=16 workload: upstream do and dhT drawn once
     b = synth.prefill_inputs("prefill-t4096", device=dev, seed=shard.rank_seed(1001, rank))
