@@ -19,7 +19,12 @@
 // Threads: 512 per chain; thread (r, q) owns row r of S and of dS, columns 32 q .. 32 q + 31.
 // Sums over columns (dq, dk, dlog_g) are two shuffles among the four threads of a row; sums over
 // rows (m, dd) are a reduce-scatter over the 8 rows of a warp (each lane keeps 4 columns) and a
-// sum over the 16 warps in shared memory. Plain fp32 arithmetic and expf, no tensor cores: this
+// sum over the 16 warps in shared memory. The kernel's own copies of the state (checkpoints, the
+// chunk's per-token states) interleave the threads' elements, so that every warp access to them
+// is one contiguous 128-byte line (a thread's 32 consecutive floats would touch 32 lines per warp
+// instruction: measured 14 K of a token's 26 K cycles); the staged per-column vectors are padded
+// so that the four column groups of a warp read different banks; the next token's inputs are
+// fetched into registers a step ahead. Plain fp32 arithmetic and expf, no tensor cores: this
 // kernel is the correct first version of the training direction, not yet its fast one.
 
 #include <cstdint>
@@ -33,6 +38,11 @@ constexpr int kD = 128;
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kCk = 64;   // tokens per checkpointed chunk
+constexpr int kDp = kD + kD / 32;   // padded per-column vectors: entry c at c + c / 32
+
+// Entry c of a per-column vector in shared memory. Thread (r, q) reads entries 32 q + i of its
+// column group; one word of padding per 32 puts the four groups of a warp in different banks.
+__device__ __forceinline__ int pc(int c) { return c + (c >> 5); }
 
 struct BwdArgs {
     const void* q;
@@ -59,7 +69,7 @@ struct BwdArgs {
 
 template <typename E>
 __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const BwdArgs a) {
-    __shared__ float q_s[kD], k_s[kD], g_s[kD], v_s[kD], do_s[kD], m_s[kD], d_s[kD], x_s[kD];
+    __shared__ float q_s[kD], k_s[kD], g_s[kD], v_s[kD], do_s[kDp], m_s[kDp], d_s[kDp], x_s[kDp];
     __shared__ float part[kWarps * kD];
     __shared__ float beta_s, db_s[4];
 
@@ -99,22 +109,48 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const BwdArgs a) {
     float* cs = a.chunk_s + (size_t)chain * kCk * mat;
     float* cmd = a.chunk_md + (size_t)chain * kCk * 2 * kD;
     const size_t my = (size_t)r * kD + c0;   // this thread's 32 elements in a 128 x 128 matrix
+    // the same 32 elements in the kernel's own copies (checkpoints, the chunk's states): element i
+    // of every thread side by side, so that a warp's access is 128 contiguous bytes
+    auto ti = [&](int i) { return (size_t)i * kThreads + tid; };
 
-    // inputs of token row `row` into shared memory (threads < 128, one channel each)
-    auto stage = [&](long long row, bool backward) {
-        __syncthreads();   // the previous step has finished reading the staged values
+    // Inputs of token row `row` into shared memory (threads < 128, one channel each). The next
+    // row staged (forward, re-run and backward walks included) is fetched into registers right
+    // after, so its loads are in flight during this step; a row that was not fetched ahead is
+    // loaded on the spot.
+    float nk = 0.f, nlg = 0.f, nv = 0.f, nq = 0.f, ndo = 0.f, nb = 0.f;
+    long long n_row = -1;
+    bool n_bwd = false;
+    auto fetch = [&](long long row, bool backward) {
         if (tid < kD) {
             const size_t e = ((size_t)row * a.H + h) * kD + tid;
-            k_s[tid] = load_elem(k, e);
-            g_s[tid] = expf(a.log_g[e]);
-            v_s[tid] = load_elem(v, e);
+            nk = load_elem(k, e);
+            nlg = a.log_g[e];
+            nv = load_elem(v, e);
             if (backward) {
-                q_s[tid] = load_elem(q, e);
-                do_s[tid] = load_elem(dout, e);
+                nq = load_elem(q, e);
+                ndo = load_elem(dout, e);
             }
-            if (tid == 0) beta_s = load_elem(beta, (size_t)row * a.H + h);
+            if (tid == 0) nb = load_elem(beta, (size_t)row * a.H + h);
+        }
+        n_row = row;
+        n_bwd = backward;
+    };
+    auto stage = [&](long long row, bool backward, long long next_row, bool next_bwd) {
+        __syncthreads();   // the previous step has finished reading the staged values
+        if (n_row != row || n_bwd != backward) fetch(row, backward);
+        if (tid < kD) {
+            k_s[tid] = nk;
+            g_s[tid] = expf(nlg);
+            v_s[tid] = nv;
+            if (backward) {
+                q_s[tid] = nq;
+                do_s[pc(tid)] = ndo;
+            }
+            if (tid == 0) beta_s = nb;
         }
         __syncthreads();
+        if (next_row >= 0) fetch(next_row, next_bwd);
+        else n_row = -1;
     };
     // out[c] = sum over rows of f(i) (i: this thread's column 32 qq + i); the result lands in
     // shared memory for every thread after the call
@@ -142,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const BwdArgs a) {
             float s = 0.f;
 #pragma unroll 4
             for (int w = 0; w < kWarps; ++w) s += part[w * kD + tid];
-            out[tid] = s;
+            out[pc(tid)] = s;
         }
         __syncthreads();
     };
@@ -160,10 +196,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const BwdArgs a) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) S[i] *= gr;
         colsum([&](int i) { return kr * S[i]; }, m_s);
-        if (tid < kD) d_s[tid] = beta_s * (v_s[tid] - m_s[tid]);
+        if (tid < kD) d_s[pc(tid)] = beta_s * (v_s[tid] - m_s[pc(tid)]);
         __syncthreads();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) S[i] += kr * d_s[c0 + i];
+        for (int i = 0; i < 32; ++i) S[i] += kr * d_s[pc(c0 + i)];
     };
 
     // ---------------------------------------------------------------- forward, checkpoints
@@ -172,9 +208,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const BwdArgs a) {
     for (long long s = 0; s < L; ++s) {
         if (s % kCk == 0) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ckpt[(size_t)(s / kCk) * mat + my + i] = S[i];
+            for (int i = 0; i < 32; ++i) ckpt[(size_t)(s / kCk) * mat + ti(i)] = S[i];
         }
-        stage(t0 + s, false);
+        // next: the token after, or the first token of the last chunk's re-run
+        stage(t0 + s, false, s + 1 < L ? t0 + s + 1 : t0 + (long long)(nck - 1) * kCk, false);
         forward_step();
     }
 
@@ -186,35 +223,39 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const BwdArgs a) {
         const long long s1 = min(L, s0 + kCk);
         // the chunk's forward again, keeping S_{s-1}, m_s and d_s of every token
 #pragma unroll
-        for (int i = 0; i < 32; ++i) S[i] = ckpt[(size_t)ci * mat + my + i];
+        for (int i = 0; i < 32; ++i) S[i] = ckpt[(size_t)ci * mat + ti(i)];
         for (long long s = s0; s < s1; ++s) {
             const size_t j = (size_t)(s - s0);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) cs[j * mat + my + i] = S[i];
-            stage(t0 + s, false);
+            for (int i = 0; i < 32; ++i) cs[j * mat + ti(i)] = S[i];
+            // next: the token after, or the chunk's last token for the backward walk
+            if (s + 1 < s1) stage(t0 + s, false, t0 + s + 1, false);
+            else stage(t0 + s, false, t0 + s1 - 1, true);
             forward_step();
             if (tid < kD) {
-                cmd[j * 2 * kD + tid] = m_s[tid];
-                cmd[j * 2 * kD + kD + tid] = d_s[tid];
+                cmd[j * 2 * kD + tid] = m_s[pc(tid)];
+                cmd[j * 2 * kD + kD + tid] = d_s[pc(tid)];
             }
         }
         // the chunk's tokens from the last to the first
         for (long long s = s1 - 1; s >= s0; --s) {
             const size_t j = (size_t)(s - s0);
             const long long row = t0 + s;
-            stage(row, true);
+            // next: the token before, or the first token of the previous chunk's re-run
+            if (s > s0) stage(row, true, row - 1, true);
+            else stage(row, true, ci > 0 ? t0 + (long long)(ci - 1) * kCk : -1, false);
             if (tid < kD) {   // written by this same thread in the pass above
-                m_s[tid] = cmd[j * 2 * kD + tid];
-                d_s[tid] = cmd[j * 2 * kD + kD + tid];
+                m_s[pc(tid)] = cmd[j * 2 * kD + tid];
+                d_s[pc(tid)] = cmd[j * 2 * kD + kD + tid];
             }
 #pragma unroll
-            for (int i = 0; i < 32; ++i) S[i] = cs[j * mat + my + i];   // S_{s-1}
+            for (int i = 0; i < 32; ++i) S[i] = cs[j * mat + ti(i)];   // S_{s-1}
             __syncthreads();
             const float gr = g_s[r], kr = k_s[r], qr = q_s[r];
             float pq = 0.f, pk = 0.f;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float dl = d_s[c0 + i], dov = do_s[c0 + i];
+                const float dl = d_s[pc(c0 + i)], dov = do_s[pc(c0 + i)];
                 const float st = gr * S[i] + kr * dl;   // S_s
                 pq = fmaf(st, dov, pq);
                 dS[i] = fmaf(qr, dov, dS[i]);
@@ -223,9 +264,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const BwdArgs a) {
             colsum([&](int i) { return kr * dS[i]; }, x_s);   // dd
             const float bt = beta_s;
             if (tid < kD) {
-                const float dd = x_s[tid];
+                const float dd = x_s[pc(tid)];
                 a.dv[((size_t)row * a.H + h) * kD + tid] = bt * dd;
-                float p = dd * (v_s[tid] - m_s[tid]);
+                float p = dd * (v_s[tid] - m_s[pc(tid)]);
 #pragma unroll
                 for (int off = 16; off >= 1; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
                 if (lane == 0) db_s[warp] = p;
@@ -235,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const BwdArgs a) {
             float pg = 0.f;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float dm = -bt * x_s[c0 + i];
+                const float dm = -bt * x_s[pc(c0 + i)];
                 const float sp = gr * S[i];   // S'_s
                 pk = fmaf(sp, dm, pk);
                 const float dsp = fmaf(kr, dm, dS[i]);
