@@ -135,12 +135,16 @@ const char* kda_status_string(kda_status_t s) {
     return "unknown status";
 }
 
-// Segments of at least 32 chunks, at most 12 (measured on the long-context workload, 1024 chunks
-// per sequence: 1, 4, 8, 12, 16 segments take 5.31, 5.32, 4.89, 4.78, 4.80 ms).
+// Segments of at least 32 chunks, at most 12, and one segment up to 64 chunks. Measured on one
+// B200 (L2 flushed before each call): the long-context workload (1024 chunks per sequence, 64
+// chains) takes 3.84, 3.89, 3.63, 3.71, 3.65 ms at 1, 4, 8, 12, 16 segments; the single-sequence
+// one (64 chunks, 16 chains) 0.154, 0.178, 0.170, 0.168 ms at 1, 2, 3, 4: the next segment's
+// intra-chunk launch takes the SMs before a short state pass can start, so a short chain gains no
+// overlap and pays the side stream's joins.
 // KDA_SPLIT_SEGMENTS (1-16, read per call) overrides the count, capped at the chunk count; the
 // result is the same whatever the count (the state crosses segments in fp32).
 static int split_segments(int ncT) {
-    int s = ncT < 64 ? 1 : ncT / 32;
+    int s = ncT <= 64 ? 1 : ncT / 32;
     if (s > 12) s = 12;
     if (const char* env = std::getenv("KDA_SPLIT_SEGMENTS")) {
         const int v = std::atoi(env);

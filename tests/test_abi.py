@@ -176,14 +176,14 @@ def test_workspace_size_is_host_only(L):
 
 
 def test_split_segments_rule(L, monkeypatch):
-    """Equal-length sequences of 64 chunks or more run in segments of at least 32 chunks, at most
-    12; packed documents, short sequences and the per-token path in one; the environment
-    override is capped at 16 and at the chunk count."""
+    """Equal-length sequences of more than 64 chunks run in segments of at least 32 chunks, at
+    most 12; packed documents, sequences of up to 64 chunks and the per-token path in one; the
+    environment override is capped at 16 and at the chunk count."""
     L.kda_fwd_split_segments.restype = ctypes.c_int
     seg = lambda T, varlen=0, **kw: L.kda_fwd_split_segments(ctypes.byref(_desc(T=T, **kw)),
                                                              varlen)
     monkeypatch.delenv("KDA_SPLIT_SEGMENTS", raising=False)
-    assert seg(64 * 63) == 1 and seg(64 * 64) == 2 and seg(64 * 64 + 1) == 2
+    assert seg(64 * 63) == 1 and seg(64 * 64) == 1 and seg(64 * 64 + 1) == 2
     assert seg(64 * 101) == 3 and seg(65536) == 12 and seg(1 << 20) == 12
     assert seg(65536, varlen=1, B=1, num_seqs=4) == 1
     assert seg(65536, chunk_size=1) == 1
