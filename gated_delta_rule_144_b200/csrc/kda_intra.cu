@@ -762,23 +762,20 @@ intra_kernel(const __grid_constant__ IntraMaps maps, const IntraArgs args) {
                 tmem_ld_wait();
                 if (a == 1) put16(0, w);
             } else {
-                float v[32];
-                tmem_ld32(tbase + lane_q + TM_A + 64 + cross_off(2), v);   // block 2: i in 0..31
-                tmem_ld_wait();
-                if (a == 2) {
-                    put16(0, v);
-                    put16(16, v + 16);
-                }
-                tmem_ld32(tbase + lane_q + TM_A + 64 + cross_off(3), v);   // block 3: i in 0..31
-                tmem_ld_wait();
-                if (a == 3) {
-                    put16(0, v);
-                    put16(16, v + 16);
-                }
-                float w[16];
+                // rows of blocks 2 and 3: all three loads in flight before one wait
+                float v2[32], v3[32], w[16];
+                tmem_ld32(tbase + lane_q + TM_A + 64 + cross_off(2), v2);        // block 2: i 0..31
+                tmem_ld32(tbase + lane_q + TM_A + 64 + cross_off(3), v3);        // block 3: i 0..31
                 tmem_ld16(tbase + lane_q + TM_A + 64 + cross_off(3) + 32, w);   // i in 32..47
                 tmem_ld_wait();
-                if (a == 3) put16(32, w);
+                if (a == 2) {
+                    put16(0, v2);
+                    put16(16, v2 + 16);
+                } else {
+                    put16(0, v3);
+                    put16(16, v3 + 16);
+                    put16(32, w);
+                }
             }
         }
         } else {
