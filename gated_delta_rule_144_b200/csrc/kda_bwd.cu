@@ -10,22 +10,24 @@
 //   dq_t = S_t do_t;   dS += q_t do_t^T;   dd = dS^T k_t;   dbeta_t = <dd, v_t - m_t>;
 //   dv_t = beta_t dd;  dm = -beta_t dd;    dk_t = dS d_t + S'_t dm;   dS' = dS + k_t dm^T;
 //   dlog_g_t = g_t * rowsum(dS' * S_{t-1});   dS = diag(g_t) dS'   (dh0 = dS after the first).
-// The backward needs S_{t-1} at every token in reverse order. One CTA per chain first runs the
-// forward and stores the state at the start of every 64-token chunk (checkpoints, in the
-// workspace); then, chunk by chunk from the last, it re-runs the chunk's forward from its
-// checkpoint, keeping the chunk's states and m_t, d_t in the workspace, and walks the chunk
-// backwards.
+// The backward needs S_{t-1} at every token in reverse order. Each CTA first runs the forward and
+// stores the state at the start of every 64-token chunk (checkpoints, in the workspace); then,
+// chunk by chunk from the last, it re-runs the chunk's forward from its checkpoint, keeping the
+// chunk's states and m_t, d_t in the workspace, and walks the chunk backwards.
 //
-// Threads: 512 per chain; thread (r, q) owns row r of S and of dS, columns 32 q .. 32 q + 31.
-// Sums over columns (dq, dk, dlog_g) are two shuffles among the four threads of a row; sums over
-// rows (m, dd) are a reduce-scatter over the 8 rows of a warp (each lane keeps 4 columns) and a
-// sum over the 16 warps in shared memory. The kernel's own copies of the state (checkpoints, the
-// chunk's per-token states) interleave the threads' elements, so that every warp access to them
-// is one contiguous 128-byte line (a thread's 32 consecutive floats would touch 32 lines per warp
-// instruction: measured 14 K of a token's 26 K cycles); the staged per-column vectors are padded
-// so that the four column groups of a warp read different banks; the next token's inputs are
-// fetched into registers a step ahead. Plain fp32 arithmetic and expf, no tensor cores: this
-// kernel is the correct first version of the training direction, not yet its fast one.
+// Value columns are independent in both directions: column j of S, m, d, dS and dd depends on
+// column j alone. So a chain is split over 16 CTAs of 8 value columns each, which walk their
+// columns with no exchange; only dq, dk, dlog_g (sums over columns) and dbeta are summed over the
+// 16 CTAs, by fp32 atomic adds into outputs the launch zeroes first (the order of those adds is
+// not fixed, so the last bits of dq, dk, dlog_g and dbeta may differ between runs; dv and dh0 are
+// written once).
+//
+// Threads: 128 per CTA; thread r owns row r of the slice's S and dS (8 columns). Sums over
+// columns are in-thread; sums over rows (m, dd) are a reduce-scatter over the 32 rows of a warp
+// (9 shuffles) and a sum over the 4 warps in shared memory. The kernel's own copies of the state interleave the threads' elements, so that every
+// warp access to them is one contiguous 128-byte line; the next token's inputs are fetched into
+// registers a step ahead. Plain fp32 arithmetic and expf, no tensor cores: a per-token kernel,
+// not the chunked one.
 
 #include <cstdint>
 
@@ -35,14 +37,16 @@ namespace kda {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kThreads = 512;
+constexpr int kCk = 64;                 // tokens per checkpointed chunk
+constexpr int kSlices = 16;             // CTAs per chain (8 measured 1.6x slower)
+constexpr int kCols = kD / kSlices;     // value columns per CTA
+constexpr int kPer = 8;                 // columns per thread
+constexpr int kTpr = kCols / kPer;      // threads per row of S: 2 or 1
+constexpr int kThreads = kD * kTpr;
 constexpr int kWarps = kThreads / 32;
-constexpr int kCk = 64;   // tokens per checkpointed chunk
-constexpr int kDp = kD + kD / 32;   // padded per-column vectors: entry c at c + c / 32
-
-// Entry c of a per-column vector in shared memory. Thread (r, q) reads entries 32 q + i of its
-// column group; one word of padding per 32 puts the four groups of a warp in different banks.
-__device__ __forceinline__ int pc(int c) { return c + (c >> 5); }
+constexpr int kSmat = kD * kCols;       // floats of one slice of the state
+static_assert(kTpr == 1 || kTpr == 2, "8 or 16 value columns per CTA");
+static_assert(kPer * kThreads == kSmat, "the threads cover the slice exactly");
 
 struct BwdArgs {
     const void* q;
@@ -54,29 +58,31 @@ struct BwdArgs {
     const float* h0;     // nullable
     const float* dhT;    // nullable
     const int32_t* cu;   // nullable
-    float* dq;
+    float* dq;           // zeroed by the launch: the CTAs of a chain add into dq, dk, dlog_g, dbeta
     float* dk;
     float* dv;
     float* dlog_g;
     float* dbeta;
     float* dh0;          // nullable
-    float* ckpt;         // [chains][nck][128][128]
-    float* chunk_s;      // [chains][kCk][128][128]
-    float* chunk_md;     // [chains][kCk][2][128]
+    float* ckpt;         // [chains][slices][nck][kSmat]
+    float* chunk_s;      // [chains][slices][kCk][kSmat]
+    float* chunk_md;     // [chains][slices][kCk][2][kCols]
     int T, H, N, nck;
     unsigned* err;
 };
 
 template <typename E>
-__global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const BwdArgs a) {
-    __shared__ float q_s[kD], k_s[kD], g_s[kD], v_s[kD], do_s[kDp], m_s[kDp], d_s[kDp], x_s[kDp];
-    __shared__ float part[kWarps * kD];
-    __shared__ float beta_s, db_s[4];
+__global__ void __launch_bounds__(kThreads, 512 / kThreads) bwd_kernel(const BwdArgs a) {
+    __shared__ float q_s[kD], k_s[kD], g_s[kD];
+    __shared__ float v_s[kCols], do_s[kCols], m_s[kCols], d_s[kCols], x_s[kCols];
+    __shared__ float part[kWarps][kCols];
+    __shared__ float beta_s;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int r = tid >> 2, qq = tid & 3;   // row of S, column group
-    const int c0 = 32 * qq;
-    const int chain = blockIdx.x;
+    const int r = tid / kTpr, hc = tid % kTpr;   // row of S, column half
+    const int lc0 = kPer * hc;              // first of this thread's columns within the slice
+    const int chain = blockIdx.x / kSlices, slice = blockIdx.x % kSlices;
+    const int cs0 = kCols * slice;          // first value column of the slice
     const int n = chain / a.H, h = chain % a.H;
     const E* q = static_cast<const E*>(a.q);
     const E* k = static_cast<const E*>(a.k);
@@ -105,30 +111,31 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const BwdArgs a) {
         return;
     }
     const size_t mat = (size_t)kD * kD;
-    float* ckpt = a.ckpt + (size_t)chain * a.nck * mat;
-    float* cs = a.chunk_s + (size_t)chain * kCk * mat;
-    float* cmd = a.chunk_md + (size_t)chain * kCk * 2 * kD;
-    const size_t my = (size_t)r * kD + c0;   // this thread's 32 elements in a 128 x 128 matrix
-    // the same 32 elements in the kernel's own copies (checkpoints, the chunk's states): element i
-    // of every thread side by side, so that a warp's access is 128 contiguous bytes
+    const size_t unit = (size_t)chain * kSlices + slice;
+    float* ckpt = a.ckpt + unit * a.nck * kSmat;
+    float* cs = a.chunk_s + unit * kCk * kSmat;
+    float* cmd = a.chunk_md + unit * kCk * 2 * kCols;
+    // this thread's 8 elements in a caller's 128 x 128 matrix (h0, dhT, dh0)
+    const size_t my = (size_t)r * kD + cs0 + lc0;
+    // the same elements in the kernel's own copies: element i of every thread side by side
     auto ti = [&](int i) { return (size_t)i * kThreads + tid; };
 
-    // Inputs of token row `row` into shared memory (threads < 128, one channel each). The next
-    // row staged (forward, re-run and backward walks included) is fetched into registers right
-    // after, so its loads are in flight during this step; a row that was not fetched ahead is
-    // loaded on the spot.
-    float nk = 0.f, nlg = 0.f, nv = 0.f, nq = 0.f, ndo = 0.f, nb = 0.f;
+    // Inputs of token row `row` into shared memory: threads < 128 one key channel each (k, log g,
+    // q), threads < 16 one of the slice's value columns (v, do). The next row staged is fetched
+    // into registers right after, so its loads are in flight during this step; a row that was
+    // not fetched ahead is loaded on the spot.
+    float nk = 0.f, nlg = 0.f, nq = 0.f, nv = 0.f, ndo = 0.f, nb = 0.f;
     long long n_row = -1;
     bool n_bwd = false;
     auto fetch = [&](long long row, bool backward) {
         if (tid < kD) {
-            const size_t e = ((size_t)row * a.H + h) * kD + tid;
-            nk = load_elem(k, e);
-            nlg = a.log_g[e];
-            nv = load_elem(v, e);
-            if (backward) {
-                nq = load_elem(q, e);
-                ndo = load_elem(dout, e);
+            const size_t e = ((size_t)row * a.H + h) * kD;
+            nk = load_elem(k, e + tid);
+            nlg = a.log_g[e + tid];
+            if (backward) nq = load_elem(q, e + tid);
+            if (tid < kCols) {
+                nv = load_elem(v, e + cs0 + tid);
+                if (backward) ndo = load_elem(dout, e + cs0 + tid);
             }
             if (tid == 0) nb = load_elem(beta, (size_t)row * a.H + h);
         }
@@ -141,10 +148,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const BwdArgs a) {
         if (tid < kD) {
             k_s[tid] = nk;
             g_s[tid] = expf(nlg);
-            v_s[tid] = nv;
-            if (backward) {
-                q_s[tid] = nq;
-                do_s[pc(tid)] = ndo;
+            if (backward) q_s[tid] = nq;
+            if (tid < kCols) {
+                v_s[tid] = nv;
+                if (backward) do_s[tid] = ndo;
             }
             if (tid == 0) beta_s = nb;
         }
@@ -152,63 +159,58 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const BwdArgs a) {
         if (next_row >= 0) fetch(next_row, next_bwd);
         else n_row = -1;
     };
-    // out[c] = sum over rows of f(i) (i: this thread's column 32 qq + i); the result lands in
-    // shared memory for every thread after the call
+    // out[c] = sum over the 128 rows of f(i) (i: this thread's column lc0 + i); the result lands
+    // in shared memory for every thread after the call. Within a warp (16 rows x 2 column halves)
+    // each lane first keeps one column of its half summed over the warp's rows (three halving
+    // exchanges and one plain one), then the 8 warps' partials are added in shared memory.
     auto colsum = [&](auto f, float* out) {
-        float s16[16], s8[8], s4[4];
+        float v8[kPer], s4[4], s2[2];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) v8[i] = f(i);
         const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float lo = f(i), hi = f(16 + i);
-            s16[i] = (b4 ? hi : lo) + __shfl_xor_sync(0xffffffffu, b4 ? lo : hi, 16);
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            s8[i] = (b3 ? s16[8 + i] : s16[i]) +
-                    __shfl_xor_sync(0xffffffffu, b3 ? s16[i] : s16[8 + i], 8);
-#pragma unroll
         for (int i = 0; i < 4; ++i)
-            s4[i] = (b2 ? s8[4 + i] : s8[i]) +
-                    __shfl_xor_sync(0xffffffffu, b2 ? s8[i] : s8[4 + i], 4);
-        const int base = c0 + (b4 ? 16 : 0) + (b3 ? 8 : 0) + (b2 ? 4 : 0);
+            s4[i] = (b4 ? v8[4 + i] : v8[i]) +
+                    __shfl_xor_sync(0xffffffffu, b4 ? v8[i] : v8[4 + i], 16);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) part[warp * kD + base + i] = s4[i];
+        for (int i = 0; i < 2; ++i)
+            s2[i] = (b3 ? s4[2 + i] : s4[i]) +
+                    __shfl_xor_sync(0xffffffffu, b3 ? s4[i] : s4[2 + i], 8);
+        float s1 = (b2 ? s2[1] : s2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? s2[0] : s2[1], 4);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+        if (kTpr == 1) s1 += __shfl_xor_sync(0xffffffffu, s1, 1);   // bit 0 is a row bit too
+        if ((lane & (kTpr == 1 ? 3 : 2)) == 0)
+            part[warp][lc0 + (b4 ? 4 : 0) + (b3 ? 2 : 0) + (b2 ? 1 : 0)] = s1;
         __syncthreads();
-        if (tid < kD) {
+        if (tid < kCols) {
             float s = 0.f;
-#pragma unroll 4
-            for (int w = 0; w < kWarps; ++w) s += part[w * kD + tid];
-            out[pc(tid)] = s;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) s += part[w][tid];
+            out[tid] = s;
         }
         __syncthreads();
-    };
-    // sum over this row's four threads
-    auto rowsum = [&](float x) {
-        x += __shfl_xor_sync(0xffffffffu, x, 1);
-        x += __shfl_xor_sync(0xffffffffu, x, 2);
-        return x;
     };
 
-    float S[32], dS[32];
+    float S[kPer], dS[kPer];
     // forward step on the staged token: S <- S' + k d^T; m and d land in m_s, d_s
     auto forward_step = [&]() {
         const float gr = g_s[r], kr = k_s[r];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) S[i] *= gr;
+        for (int i = 0; i < kPer; ++i) S[i] *= gr;
         colsum([&](int i) { return kr * S[i]; }, m_s);
-        if (tid < kD) d_s[pc(tid)] = beta_s * (v_s[tid] - m_s[pc(tid)]);
+        if (tid < kCols) d_s[tid] = beta_s * (v_s[tid] - m_s[tid]);
         __syncthreads();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) S[i] += kr * d_s[pc(c0 + i)];
+        for (int i = 0; i < kPer; ++i) S[i] += kr * d_s[lc0 + i];
     };
 
     // ---------------------------------------------------------------- forward, checkpoints
 #pragma unroll
-    for (int i = 0; i < 32; ++i) S[i] = a.h0 ? a.h0[(size_t)chain * mat + my + i] : 0.f;
+    for (int i = 0; i < kPer; ++i) S[i] = a.h0 ? a.h0[(size_t)chain * mat + my + i] : 0.f;
     for (long long s = 0; s < L; ++s) {
         if (s % kCk == 0) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ckpt[(size_t)(s / kCk) * mat + ti(i)] = S[i];
+            for (int i = 0; i < kPer; ++i) ckpt[(size_t)(s / kCk) * kSmat + ti(i)] = S[i];
         }
         // next: the token after, or the first token of the last chunk's re-run
         stage(t0 + s, false, s + 1 < L ? t0 + s + 1 : t0 + (long long)(nck - 1) * kCk, false);
@@ -217,24 +219,24 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const BwdArgs a) {
 
     // ---------------------------------------------------------------- backward, chunk by chunk
 #pragma unroll
-    for (int i = 0; i < 32; ++i) dS[i] = a.dhT ? a.dhT[(size_t)chain * mat + my + i] : 0.f;
+    for (int i = 0; i < kPer; ++i) dS[i] = a.dhT ? a.dhT[(size_t)chain * mat + my + i] : 0.f;
     for (int ci = nck - 1; ci >= 0; --ci) {
         const long long s0 = (long long)ci * kCk;
         const long long s1 = min(L, s0 + kCk);
         // the chunk's forward again, keeping S_{s-1}, m_s and d_s of every token
 #pragma unroll
-        for (int i = 0; i < 32; ++i) S[i] = ckpt[(size_t)ci * mat + ti(i)];
+        for (int i = 0; i < kPer; ++i) S[i] = ckpt[(size_t)ci * kSmat + ti(i)];
         for (long long s = s0; s < s1; ++s) {
             const size_t j = (size_t)(s - s0);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) cs[j * mat + ti(i)] = S[i];
+            for (int i = 0; i < kPer; ++i) cs[j * kSmat + ti(i)] = S[i];
             // next: the token after, or the chunk's last token for the backward walk
             if (s + 1 < s1) stage(t0 + s, false, t0 + s + 1, false);
             else stage(t0 + s, false, t0 + s1 - 1, true);
             forward_step();
-            if (tid < kD) {
-                cmd[j * 2 * kD + tid] = m_s[pc(tid)];
-                cmd[j * 2 * kD + kD + tid] = d_s[pc(tid)];
+            if (tid < kCols) {
+                cmd[j * 2 * kCols + tid] = m_s[tid];
+                cmd[j * 2 * kCols + kCols + tid] = d_s[tid];
             }
         }
         // the chunk's tokens from the last to the first
@@ -244,18 +246,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const BwdArgs a) {
             // next: the token before, or the first token of the previous chunk's re-run
             if (s > s0) stage(row, true, row - 1, true);
             else stage(row, true, ci > 0 ? t0 + (long long)(ci - 1) * kCk : -1, false);
-            if (tid < kD) {   // written by this same thread in the pass above
-                m_s[pc(tid)] = cmd[j * 2 * kD + tid];
-                d_s[pc(tid)] = cmd[j * 2 * kD + kD + tid];
+            if (tid < kCols) {   // written by this same thread in the pass above
+                m_s[tid] = cmd[j * 2 * kCols + tid];
+                d_s[tid] = cmd[j * 2 * kCols + kCols + tid];
             }
 #pragma unroll
-            for (int i = 0; i < 32; ++i) S[i] = cs[j * mat + ti(i)];   // S_{s-1}
+            for (int i = 0; i < kPer; ++i) S[i] = cs[j * kSmat + ti(i)];   // S_{s-1}
             __syncthreads();
             const float gr = g_s[r], kr = k_s[r], qr = q_s[r];
             float pq = 0.f, pk = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float dl = d_s[pc(c0 + i)], dov = do_s[pc(c0 + i)];
+            for (int i = 0; i < kPer; ++i) {
+                const float dl = d_s[lc0 + i], dov = do_s[lc0 + i];
                 const float st = gr * S[i] + kr * dl;   // S_s
                 pq = fmaf(st, dov, pq);
                 dS[i] = fmaf(qr, dov, dS[i]);
@@ -263,40 +265,42 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const BwdArgs a) {
             }
             colsum([&](int i) { return kr * dS[i]; }, x_s);   // dd
             const float bt = beta_s;
-            if (tid < kD) {
-                const float dd = x_s[pc(tid)];
-                a.dv[((size_t)row * a.H + h) * kD + tid] = bt * dd;
-                float p = dd * (v_s[tid] - m_s[pc(tid)]);
+            if (tid < kCols) {   // the first lanes of warp 0
+                const float dd = x_s[tid];
+                a.dv[((size_t)row * a.H + h) * kD + cs0 + tid] = bt * dd;
+                float p = dd * (v_s[tid] - m_s[tid]);
 #pragma unroll
-                for (int off = 16; off >= 1; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
-                if (lane == 0) db_s[warp] = p;
+                for (int off = kCols / 2; off >= 1; off >>= 1)
+                    p += __shfl_xor_sync((1u << kCols) - 1u, p, off);
+                if (tid == 0) atomicAdd(a.dbeta + (size_t)row * a.H + h, p);
             }
-            __syncthreads();
-            if (tid == 0) a.dbeta[(size_t)row * a.H + h] = (db_s[0] + db_s[1]) + (db_s[2] + db_s[3]);
             float pg = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float dm = -bt * x_s[pc(c0 + i)];
+            for (int i = 0; i < kPer; ++i) {
+                const float dm = -bt * x_s[lc0 + i];
                 const float sp = gr * S[i];   // S'_s
                 pk = fmaf(sp, dm, pk);
                 const float dsp = fmaf(kr, dm, dS[i]);
                 pg = fmaf(dsp, S[i], pg);
                 dS[i] = gr * dsp;
             }
-            pq = rowsum(pq);
-            pk = rowsum(pk);
-            pg = rowsum(pg);
-            if (qq == 0) {
+            // the row's sums over the slice's columns: this thread's 8 and its partner's
+            if (kTpr == 2) {
+                pq += __shfl_xor_sync(0xffffffffu, pq, 1);
+                pk += __shfl_xor_sync(0xffffffffu, pk, 1);
+                pg += __shfl_xor_sync(0xffffffffu, pg, 1);
+            }
+            if (hc == 0) {
                 const size_t e = ((size_t)row * a.H + h) * kD + r;
-                a.dq[e] = pq;
-                a.dk[e] = pk;
-                a.dlog_g[e] = gr * pg;
+                atomicAdd(a.dq + e, pq);
+                atomicAdd(a.dk + e, pk);
+                atomicAdd(a.dlog_g + e, gr * pg);
             }
         }
     }
     if (a.dh0) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) a.dh0[(size_t)chain * mat + my + i] = dS[i];
+        for (int i = 0; i < kPer; ++i) a.dh0[(size_t)chain * mat + my + i] = dS[i];
     }
 }
 
@@ -310,7 +314,15 @@ size_t bwd_workspace_bytes(long long chains, int T) {
 cudaError_t launch_bwd(const BwdParams& p, cudaStream_t stream) {
     const long long chains = (long long)p.N * p.H;
     if (chains == 0) return cudaSuccess;
-    if (chains > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    if (chains * kSlices > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    // the CTAs of a chain add their slices' parts of dq, dk, dlog_g and dbeta
+    const size_t rows = (size_t)(p.cu_seqlens ? 1 : p.N) * p.T * p.H;
+    cudaError_t e;
+    if ((e = cudaMemsetAsync(p.dq, 0, rows * kD * sizeof(float), stream)) != cudaSuccess ||
+        (e = cudaMemsetAsync(p.dk, 0, rows * kD * sizeof(float), stream)) != cudaSuccess ||
+        (e = cudaMemsetAsync(p.dlog_g, 0, rows * kD * sizeof(float), stream)) != cudaSuccess ||
+        (e = cudaMemsetAsync(p.dbeta, 0, rows * sizeof(float), stream)) != cudaSuccess)
+        return e;
     BwdArgs a;
     a.q = p.q;
     a.k = p.k;
@@ -337,10 +349,11 @@ cudaError_t launch_bwd(const BwdParams& p, cudaStream_t stream) {
     a.N = p.N;
     a.nck = (int)nck;
     a.err = p.err;
+    const unsigned grid = (unsigned)(chains * kSlices);
     if (p.bf16)
-        bwd_kernel<__nv_bfloat16><<<(unsigned)chains, kThreads, 0, stream>>>(a);
+        bwd_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(a);
     else
-        bwd_kernel<float><<<(unsigned)chains, kThreads, 0, stream>>>(a);
+        bwd_kernel<float><<<grid, kThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 
