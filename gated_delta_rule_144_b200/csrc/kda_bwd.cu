@@ -16,15 +16,15 @@
 // chunk's states and m_t, d_t in the workspace, and walks the chunk backwards.
 //
 // Value columns are independent in both directions: column j of S, m, d, dS and dd depends on
-// column j alone. So a chain is split over 16 CTAs of 8 value columns each, which walk their
+// column j alone. So a chain is split over 32 CTAs of 4 value columns each, which walk their
 // columns with no exchange; only dq, dk, dlog_g (sums over columns) and dbeta are summed over the
-// 16 CTAs, by fp32 atomic adds into outputs the launch zeroes first (the order of those adds is
+// 32 CTAs, by fp32 atomic adds into outputs the launch zeroes first (the order of those adds is
 // not fixed, so the last bits of dq, dk, dlog_g and dbeta may differ between runs; dv and dh0 are
 // written once).
 //
-// Threads: 128 per CTA; thread r owns row r of the slice's S and dS (8 columns). Sums over
+// Threads: 128 per CTA; thread r owns row r of the slice's S and dS (4 columns). Sums over
 // columns are in-thread; sums over rows (m, dd) are a reduce-scatter over the 32 rows of a warp
-// (9 shuffles) and a sum over the 4 warps in shared memory. The kernel's own copies of the state interleave the threads' elements, so that every
+// (6 shuffles) and a sum over the 4 warps in shared memory. The kernel's own copies of the state interleave the threads' elements, so that every
 // warp access to them is one contiguous 128-byte line; the next token's inputs are fetched into
 // registers a step ahead. Plain fp32 arithmetic and expf, no tensor cores: a per-token kernel,
 // not the chunked one.
@@ -38,15 +38,13 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kCk = 64;                 // tokens per checkpointed chunk
-constexpr int kSlices = 16;             // CTAs per chain (8 measured 1.6x slower)
-constexpr int kCols = kD / kSlices;     // value columns per CTA
-constexpr int kPer = 8;                 // columns per thread
-constexpr int kTpr = kCols / kPer;      // threads per row of S: 2 or 1
-constexpr int kThreads = kD * kTpr;
+// CTAs per chain (prefill-t4096 on one B200: 8, 16, 32 slices take 19.8, 13.1, 12.1 ms)
+constexpr int kSlices = 32;
+constexpr int kCols = kD / kSlices;     // value columns per CTA, all held by each thread
+constexpr int kThreads = kD;            // one row of the slice per thread
 constexpr int kWarps = kThreads / 32;
 constexpr int kSmat = kD * kCols;       // floats of one slice of the state
-static_assert(kTpr == 1 || kTpr == 2, "8 or 16 value columns per CTA");
-static_assert(kPer * kThreads == kSmat, "the threads cover the slice exactly");
+static_assert(kCols == 4 || kCols == 8, "4 or 8 value columns per CTA");
 
 struct BwdArgs {
     const void* q;
@@ -79,8 +77,7 @@ __global__ void __launch_bounds__(kThreads, 512 / kThreads) bwd_kernel(const Bwd
     __shared__ float beta_s;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int r = tid / kTpr, hc = tid % kTpr;   // row of S, column half
-    const int lc0 = kPer * hc;              // first of this thread's columns within the slice
+    const int r = tid;                      // row of S
     const int chain = blockIdx.x / kSlices, slice = blockIdx.x % kSlices;
     const int cs0 = kCols * slice;          // first value column of the slice
     const int n = chain / a.H, h = chain % a.H;
@@ -116,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 512 / kThreads) bwd_kernel(const Bwd
     float* cs = a.chunk_s + unit * kCk * kSmat;
     float* cmd = a.chunk_md + unit * kCk * 2 * kCols;
     // this thread's 8 elements in a caller's 128 x 128 matrix (h0, dhT, dh0)
-    const size_t my = (size_t)r * kD + cs0 + lc0;
+    const size_t my = (size_t)r * kD + cs0;
     // the same elements in the kernel's own copies: element i of every thread side by side
     auto ti = [&](int i) { return (size_t)i * kThreads + tid; };
 
@@ -159,28 +156,28 @@ __global__ void __launch_bounds__(kThreads, 512 / kThreads) bwd_kernel(const Bwd
         if (next_row >= 0) fetch(next_row, next_bwd);
         else n_row = -1;
     };
-    // out[c] = sum over the 128 rows of f(i) (i: this thread's column lc0 + i); the result lands
-    // in shared memory for every thread after the call. Within a warp (16 rows x 2 column halves)
-    // each lane first keeps one column of its half summed over the warp's rows (three halving
-    // exchanges and one plain one), then the 8 warps' partials are added in shared memory.
+    // out[c] = sum over the 128 rows of f(c); the result lands in shared memory for every thread
+    // after the call. Within a warp (32 rows) each lane first keeps one column summed over a group
+    // of rows (halving exchanges on lane bits 16, 8 (, 4): a lane keeps the upper or lower half of
+    // its columns and adds its partner's), plain exchanges then finish the warp's 32 rows, and the
+    // 4 warps' partials are added in shared memory.
     auto colsum = [&](auto f, float* out) {
-        float v8[kPer], s4[4], s2[2];
+        float c[kCols];
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) v8[i] = f(i);
-        const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+        for (int i = 0; i < kCols; ++i) c[i] = f(i);
+        int col = 0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            s4[i] = (b4 ? v8[4 + i] : v8[i]) +
-                    __shfl_xor_sync(0xffffffffu, b4 ? v8[i] : v8[4 + i], 16);
+        for (int half = kCols / 2, bit = 16; half >= 1; half >>= 1, bit >>= 1) {
+            const bool up = lane & bit;
 #pragma unroll
-        for (int i = 0; i < 2; ++i)
-            s2[i] = (b3 ? s4[2 + i] : s4[i]) +
-                    __shfl_xor_sync(0xffffffffu, b3 ? s4[i] : s4[2 + i], 8);
-        float s1 = (b2 ? s2[1] : s2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? s2[0] : s2[1], 4);
-        s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-        if (kTpr == 1) s1 += __shfl_xor_sync(0xffffffffu, s1, 1);   // bit 0 is a row bit too
-        if ((lane & (kTpr == 1 ? 3 : 2)) == 0)
-            part[warp][lc0 + (b4 ? 4 : 0) + (b3 ? 2 : 0) + (b2 ? 1 : 0)] = s1;
+            for (int i = 0; i < half; ++i)
+                c[i] = (up ? c[half + i] : c[i]) +
+                       __shfl_xor_sync(0xffffffffu, up ? c[i] : c[half + i], bit);
+            if (up) col += half;
+        }
+#pragma unroll
+        for (int bit = 16 / kCols; bit >= 1; bit >>= 1) c[0] += __shfl_xor_sync(0xffffffffu, c[0], bit);
+        if ((lane & (2 * (16 / kCols) - 1)) == 0) part[warp][col] = c[0];
         __syncthreads();
         if (tid < kCols) {
             float s = 0.f;
@@ -191,26 +188,26 @@ __global__ void __launch_bounds__(kThreads, 512 / kThreads) bwd_kernel(const Bwd
         __syncthreads();
     };
 
-    float S[kPer], dS[kPer];
+    float S[kCols], dS[kCols];
     // forward step on the staged token: S <- S' + k d^T; m and d land in m_s, d_s
     auto forward_step = [&]() {
         const float gr = g_s[r], kr = k_s[r];
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) S[i] *= gr;
+        for (int i = 0; i < kCols; ++i) S[i] *= gr;
         colsum([&](int i) { return kr * S[i]; }, m_s);
         if (tid < kCols) d_s[tid] = beta_s * (v_s[tid] - m_s[tid]);
         __syncthreads();
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) S[i] += kr * d_s[lc0 + i];
+        for (int i = 0; i < kCols; ++i) S[i] += kr * d_s[i];
     };
 
     // ---------------------------------------------------------------- forward, checkpoints
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) S[i] = a.h0 ? a.h0[(size_t)chain * mat + my + i] : 0.f;
+    for (int i = 0; i < kCols; ++i) S[i] = a.h0 ? a.h0[(size_t)chain * mat + my + i] : 0.f;
     for (long long s = 0; s < L; ++s) {
         if (s % kCk == 0) {
 #pragma unroll
-            for (int i = 0; i < kPer; ++i) ckpt[(size_t)(s / kCk) * kSmat + ti(i)] = S[i];
+            for (int i = 0; i < kCols; ++i) ckpt[(size_t)(s / kCk) * kSmat + ti(i)] = S[i];
         }
         // next: the token after, or the first token of the last chunk's re-run
         stage(t0 + s, false, s + 1 < L ? t0 + s + 1 : t0 + (long long)(nck - 1) * kCk, false);
@@ -219,17 +216,17 @@ __global__ void __launch_bounds__(kThreads, 512 / kThreads) bwd_kernel(const Bwd
 
     // ---------------------------------------------------------------- backward, chunk by chunk
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) dS[i] = a.dhT ? a.dhT[(size_t)chain * mat + my + i] : 0.f;
+    for (int i = 0; i < kCols; ++i) dS[i] = a.dhT ? a.dhT[(size_t)chain * mat + my + i] : 0.f;
     for (int ci = nck - 1; ci >= 0; --ci) {
         const long long s0 = (long long)ci * kCk;
         const long long s1 = min(L, s0 + kCk);
         // the chunk's forward again, keeping S_{s-1}, m_s and d_s of every token
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) S[i] = ckpt[(size_t)ci * kSmat + ti(i)];
+        for (int i = 0; i < kCols; ++i) S[i] = ckpt[(size_t)ci * kSmat + ti(i)];
         for (long long s = s0; s < s1; ++s) {
             const size_t j = (size_t)(s - s0);
 #pragma unroll
-            for (int i = 0; i < kPer; ++i) cs[j * kSmat + ti(i)] = S[i];
+            for (int i = 0; i < kCols; ++i) cs[j * kSmat + ti(i)] = S[i];
             // next: the token after, or the chunk's last token for the backward walk
             if (s + 1 < s1) stage(t0 + s, false, t0 + s + 1, false);
             else stage(t0 + s, false, t0 + s1 - 1, true);
@@ -251,13 +248,13 @@ __global__ void __launch_bounds__(kThreads, 512 / kThreads) bwd_kernel(const Bwd
                 d_s[tid] = cmd[j * 2 * kCols + kCols + tid];
             }
 #pragma unroll
-            for (int i = 0; i < kPer; ++i) S[i] = cs[j * kSmat + ti(i)];   // S_{s-1}
+            for (int i = 0; i < kCols; ++i) S[i] = cs[j * kSmat + ti(i)];   // S_{s-1}
             __syncthreads();
             const float gr = g_s[r], kr = k_s[r], qr = q_s[r];
             float pq = 0.f, pk = 0.f;
 #pragma unroll
-            for (int i = 0; i < kPer; ++i) {
-                const float dl = d_s[lc0 + i], dov = do_s[lc0 + i];
+            for (int i = 0; i < kCols; ++i) {
+                const float dl = d_s[i], dov = do_s[i];
                 const float st = gr * S[i] + kr * dl;   // S_s
                 pq = fmaf(st, dov, pq);
                 dS[i] = fmaf(qr, dov, dS[i]);
@@ -276,21 +273,15 @@ __global__ void __launch_bounds__(kThreads, 512 / kThreads) bwd_kernel(const Bwd
             }
             float pg = 0.f;
 #pragma unroll
-            for (int i = 0; i < kPer; ++i) {
-                const float dm = -bt * x_s[lc0 + i];
+            for (int i = 0; i < kCols; ++i) {
+                const float dm = -bt * x_s[i];
                 const float sp = gr * S[i];   // S'_s
                 pk = fmaf(sp, dm, pk);
                 const float dsp = fmaf(kr, dm, dS[i]);
                 pg = fmaf(dsp, S[i], pg);
                 dS[i] = gr * dsp;
             }
-            // the row's sums over the slice's columns: this thread's 8 and its partner's
-            if (kTpr == 2) {
-                pq += __shfl_xor_sync(0xffffffffu, pq, 1);
-                pk += __shfl_xor_sync(0xffffffffu, pk, 1);
-                pg += __shfl_xor_sync(0xffffffffu, pg, 1);
-            }
-            if (hc == 0) {
+            {   // this row's sums over the slice's columns
                 const size_t e = ((size_t)row * a.H + h) * kD + r;
                 atomicAdd(a.dq + e, pq);
                 atomicAdd(a.dk + e, pk);
@@ -300,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 512 / kThreads) bwd_kernel(const Bwd
     }
     if (a.dh0) {
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) a.dh0[(size_t)chain * mat + my + i] = dS[i];
+        for (int i = 0; i < kCols; ++i) a.dh0[(size_t)chain * mat + my + i] = dS[i];
     }
 }
 

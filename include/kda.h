@@ -165,11 +165,11 @@ kda_status_t kda_fwd_normed(const kda_fwd_desc_t* desc, const void* q, const voi
  * The forward arguments (desc, q, k, v, log_g, beta, h0, cu_seqlens) are as for kda_fwd; do has
  * the layout and dtype of o; dhT is [N, H, dk, dv] float32 or NULL (zero). dk = dv = 128
  * (KDA_ERR_UNSUPPORTED otherwise); desc->chunk_size is ignored. Every gradient is computed in
- * fp32 from the exact per-token recurrence; 16 CTAs per (sequence or document, head), one per 8
+ * fp32 from the exact per-token recurrence; 32 CTAs per (sequence or document, head), one per 4
  * value columns, run the forward storing the state every 64 tokens, then walk each 64-token chunk
  * backwards after re-running its forward. The workspace (kda_bwd_workspace_size bytes, 16-byte
  * aligned, device) holds those states. dq, dk, dlog_g and dbeta are sums over the value columns:
- * the call zeroes them on the stream and the 16 CTAs add their parts atomically, in no fixed order,
+ * the call zeroes them on the stream and the 32 CTAs add their parts atomically, in no fixed order,
  * so their last bits may differ between runs (dv and dh0 are written once). Host-checkable errors
  * return before any launch; a malformed cu_seqlens is reported through kda_get_device_error.
  */
