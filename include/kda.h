@@ -101,9 +101,9 @@ typedef struct {
  *             With at least kda_fwd_workspace_size(desc) bytes the chunked path runs split: an
  *             intra-chunk kernel computes every chunk's WY factors in parallel over all chunks
  *             and heads and stores them here (about 72.5 KiB per 64-token chunk and head), then a
- *             state pass walks each sequence's chunks. For equal-length sequences of 64 chunks
- *             or more the two run in chunk segments (up to 12; KDA_SPLIT_SEGMENTS, 1-16,
- *             overrides): the state pass of one segment runs on an internal high-priority stream
+ *             state pass walks each sequence's chunks. For equal-length sequences of more than
+ *             64 chunks the two run in chunk segments of at least 32 chunks (up to 12;
+ *             KDA_SPLIT_SEGMENTS, 1-16, overrides): the state pass of one segment runs on an internal high-priority stream
  *             while the intra-chunk kernel works on the next, and the caller's stream waits for
  *             both before the call's later work; the state between segments (64 KiB per sequence
  *             and head) is kept in the workspace. With less workspace (but at least
