@@ -275,7 +275,9 @@ def bwd(q, k, v, log_g, beta, do, h0=None, dhT=None, cu_seqlens=None, *, workspa
         stream=None):
     """Gradients of the recurrence (``kda_bwd``) for upstream gradients do (of o) and dhT (of
     the final states, or None): returns (dq, dk, dv, dlog_g, dbeta, dh0), all fp32, shaped like
-    (q, k, v, log_g, beta, h0 [N, H, dk, dv]). Forward arguments as for ``fwd``; dk = dv = 128."""
+    (q, k, v, log_g, beta, h0 [N, H, dk, dv]). Forward arguments as for ``fwd``; dk = dv = 128.
+    dq, dk, dlog_g and dbeta are sums over value-column slices added atomically, so their last
+    bits may differ between runs; dv and dh0 are reproducible."""
     lib()
     _dev(q, "q")
     dev = q.device
