@@ -519,13 +519,36 @@ def run_secondary(kda, synth, args, dev, stream, world, rank):
     by1 = prefill_bytes(c1)
     segs1 = kda.fwd_split_segments(1, c1["T"], c1["H"], 128, 128, 1, c1["q"].dtype,
                                    args.chunk_size)
+    pscan1 = kda.fwd_scan_segments(1, c1["T"], c1["H"], 128, 128, 1, c1["q"].dtype,
+                                   args.chunk_size)
+    ms1_plain = None
+    if pscan1 >= 3:
+        # the same call with the plain state pass (one chain per SM), for comparison
+        prev = os.environ.get("KDA_SCAN_SEGMENTS")
+        os.environ["KDA_SCAN_SEGMENTS"] = "0"
+        try:
+            for _ in range(3):
+                c1step()
+            torch.cuda.synchronize()
+            barrier(world)
+            perp = time_launches_flushed(c1step, max(args.steps, 20), stream, flush)
+            barrier(world)
+            ms1_plain = round(max_over_ranks(statistics.fmean(perp), world, dev), 5)
+        finally:
+            if prev is None:
+                del os.environ["KDA_SCAN_SEGMENTS"]
+            else:
+                os.environ["KDA_SCAN_SEGMENTS"] = prev
     out["prefill_t4096"] = {"workload": "prefill-t4096", "B": 1, "T": c1["T"], "H": c1["H"],
                             "ms_per_step": round(ms1, 5),
                             "tokens/s": round(c1["T"] * world / (ms1 / 1e3), 1),
                             "bytes_per_step": by1,
                             "roofline_frac": round(by1 / (ms1 / 1e3) / 1e9 / hbm_peak, 4),
                             "l2": "flushed before every launch (256 MiB write)",
+                            "ms_plain_state_pass": ms1_plain,
                             "kernel": "kda_chunk64" if args.fused else
+                            "kda_chunk64_intra+kda_chunk_scan (two-level state pass, %d "
+                            "segments)" % pscan1 if pscan1 >= 3 else
                             "kda_chunk64_intra+kda_chunk_scan (%d segment%s)" % (
                                 segs1, "" if segs1 == 1 else "s")}
     del c1, o1, h1, ws1, flush

@@ -89,6 +89,8 @@ def lib():
     L.kda_fwd_algorithm.restype = i32
     L.kda_fwd_split_segments.argtypes = [ctypes.POINTER(FwdDesc), i32]
     L.kda_fwd_split_segments.restype = i32
+    L.kda_fwd_scan_segments.argtypes = [ctypes.POINTER(FwdDesc), i32]
+    L.kda_fwd_scan_segments.restype = i32
     L.kda_fwd_workspace_size.argtypes = [ctypes.POINTER(FwdDesc)]
     L.kda_fwd_workspace_size.restype = sz
     L.kda_fwd_workspace_size_min.argtypes = [ctypes.POINTER(FwdDesc)]
@@ -169,6 +171,18 @@ def fwd_split_segments(B, T, H, dk, dv, num_seqs, dtype=torch.bfloat16, chunk_si
     r = int(lib().kda_fwd_split_segments(ctypes.byref(d), int(varlen)))
     if r < 0:
         _check(-r, "kda_fwd_split_segments")
+    return r
+
+
+def fwd_scan_segments(B, T, H, dk, dv, num_seqs, dtype=torch.bfloat16, chunk_size=0,
+                      varlen=False) -> int:
+    """Segments of kda_fwd's two-level state pass for this shape (>= 3), or 1 for the plain
+    state pass (``kda_fwd_scan_segments``; host-only, reads KDA_SCAN_SEGMENTS per call)."""
+    d = FwdDesc(B, T, H, dk, dv, num_seqs, KDA_BF16 if dtype == torch.bfloat16 else KDA_F32,
+                chunk_size)
+    r = int(lib().kda_fwd_scan_segments(ctypes.byref(d), int(varlen)))
+    if r < 0:
+        _check(-r, "kda_fwd_scan_segments")
     return r
 
 

@@ -1,6 +1,8 @@
 // C ABI of libkda.so: argument validation, path selection and the device error word.
 // Declarations and the contract of every entry point are in include/kda.h.
 
+#include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -154,6 +156,50 @@ static int split_segments(int ncT) {
     return s > ncT ? (ncT > 0 ? ncT : 1) : s;
 }
 
+// Two-level state pass for equal-length sequences with few chains (the sequential chunk chain,
+// one SM per chain, would leave most SMs idle): P segments of m chunks, P >= 3, or 1 for the
+// plain pass. Phases (one SM per unit): the state pass of segment 0 from h0 (with its outputs),
+// beside the transition maps A_p and zero-start states B_p of segments 1 .. P-2 (2 (P-2) units per
+// chain, no outputs); then S_{p+1} = A_p S_p + B_p in fp32 (P - 2 steps of a 128 x 128 x 128
+// product per chain); then segments 1 .. P-1 at once from their initial states. P minimises a
+// cost model in units of one chunk of the state pass (about 1.6 us on B200): the intra-chunk
+// kernel (about 3.7 units of SM time per record, all SMs), then the phases, each ceil(units /
+// 148) waves of m chunks, plus 1.5 units per combine step and 4 for the launches; the plain pass is
+// intra-chunk kernel + chain (one segment) or the larger of the two (chunk segments overlapping).
+// The two-level pass is used when it models at least 15 % faster. KDA_SCAN_SEGMENTS (read per
+// call) overrides: 0 or 1 = the plain pass, 3 .. 32 = that many segments (capped by the chunks).
+static int scan_segments(int ncT, long long chains) {
+    if (ncT < 3 || chains <= 0 || chains > 148) return 1;
+    auto effective = [&](int P) {   // segments of ceil(ncT / P) chunks, none empty
+        const int m = (ncT + P - 1) / P;
+        return (ncT + m - 1) / m;
+    };
+    if (const char* env = std::getenv("KDA_SCAN_SEGMENTS")) {
+        int v = std::atoi(env);
+        if (v < 3) return 1;
+        if (v > kda::kMaxScanSegments) v = kda::kMaxScanSegments;
+        if (v > ncT) v = ncT;
+        v = effective(v);
+        return v >= 3 ? v : 1;
+    }
+    const double sms = 148.0, ch = (double)chains;
+    const double intra = (double)ncT * ch * 3.7 / sms;
+    const int S = split_segments(ncT);
+    const double plain = S == 1 ? intra + ncT
+                                : std::max(intra * sms / (sms - std::min(ch, 74.0)), (double)ncT);
+    double best = 0.85 * plain;
+    int bestP = 1;
+    for (int P = 3; P <= std::min(ncT, kda::kMaxScanSegments); ++P) {
+        if (effective(P) != P) continue;
+        const int m = (ncT + P - 1) / P;
+        const double w1 = std::ceil((2.0 * (P - 2) + 1.0) * ch / sms);
+        const double w3 = std::ceil((P - 1.0) * ch / sms);
+        const double cost = intra + (w1 + w3) * m + 1.5 * (P - 2) + 4.0;
+        if (cost < best) best = cost, bestP = P;
+    }
+    return bestP;
+}
+
 int kda_fwd_algorithm(const kda_fwd_desc_t* desc, int has_cu_seqlens) {
     Path path;
     const kda_status_t st = check_fwd_desc(desc, has_cu_seqlens != 0, &path);
@@ -166,7 +212,17 @@ int kda_fwd_split_segments(const kda_fwd_desc_t* desc, int has_cu_seqlens) {
     const kda_status_t st = check_fwd_desc(desc, has_cu_seqlens != 0, &path);
     if (st != KDA_OK) return -(int)st;
     if (path != Path::kChunk64 || has_cu_seqlens || desc->T <= 0) return 1;
-    return split_segments((desc->T + 63) / 64);
+    const int ncT = (desc->T + 63) / 64;
+    if (scan_segments(ncT, (long long)desc->num_seqs * desc->H) >= 3) return 1;
+    return split_segments(ncT);
+}
+
+int kda_fwd_scan_segments(const kda_fwd_desc_t* desc, int has_cu_seqlens) {
+    Path path;
+    const kda_status_t st = check_fwd_desc(desc, has_cu_seqlens != 0, &path);
+    if (st != KDA_OK) return -(int)st;
+    if (path != Path::kChunk64 || has_cu_seqlens || desc->T <= 0) return 1;
+    return scan_segments((desc->T + 63) / 64, (long long)desc->num_seqs * desc->H);
 }
 
 // Packed documents on the chunked path are scheduled longest first; the permutation lives in the
@@ -180,8 +236,10 @@ static size_t order_bytes(const kda_fwd_desc_t* d, Path path) {
 // Workspace of the split chunked path (intra-chunk kernel + state pass), 256-byte aligned parts.
 struct SplitLayout {
     size_t order, map, counters, state, decay, wq, ke, ut, aq, total;
+    size_t maps, total_pscan;   // two-level state pass: its states, and the workspace it needs
     long long G;
     int ncT;
+    int P;                      // segments of the two-level state pass (1: the plain pass)
     bool has_order;
 };
 
@@ -207,6 +265,12 @@ static bool split_layout(const kda_fwd_desc_t* d, Path path, bool packed, SplitL
     L->ut = off;    off += (size_t)R * 16384;
     L->aq = off;    off += (size_t)R * 8192;
     L->total = off;
+    // two-level state pass: A_p and B_p of segments 1 .. P-2, then the initial states of
+    // segments 1 .. P-1, each N x H fp32 128 x 128
+    L->P = packed ? 1 : scan_segments(L->ncT, (long long)d->num_seqs * d->H);
+    L->maps = off;
+    if (L->P >= 3) off += (size_t)(3 * L->P - 5) * d->num_seqs * d->H * 65536;
+    L->total_pscan = off;
     return true;
 }
 
@@ -218,8 +282,13 @@ size_t kda_fwd_workspace_size(const kda_fwd_desc_t* desc) {
     t_last_error[0] = 0;
     SplitLayout L;
     // B == 1 may come with cu_seqlens: size for the packed record numbering (one record more
-    // per document than a single sequence needs)
-    if (split_layout(desc, path, maybe_packed, &L)) return L.total;
+    // per document than a single sequence needs), or for the two-level state pass without them
+    if (split_layout(desc, path, maybe_packed, &L)) {
+        size_t t = L.total_pscan;
+        SplitLayout U;
+        if (maybe_packed && split_layout(desc, path, false, &U)) t = std::max(t, U.total_pscan);
+        return t;
+    }
     return order_bytes(desc, path);
 }
 
@@ -296,6 +365,8 @@ static kda_status_t fwd_impl(const kda_fwd_desc_t* d, const void* q, const void*
     SplitLayout L;
     const bool split = tokens && split_layout(d, path, cu_seqlens != nullptr, &L) && workspace &&
                        aligned16(workspace) && workspace_bytes >= L.total;
+    // the two-level state pass when the plan has one and the workspace holds its states
+    const bool pscan = split && !cu_seqlens && L.P >= 3 && workspace_bytes >= L.total_pscan;
     const size_t need_ws = (cu_seqlens && !split) ? order_bytes(d, path) : 0;
     if (need_ws > 0 && (workspace_bytes < need_ws || !workspace || !aligned16(workspace)))
         return fail(KDA_ERR_INVALID_ARG,
@@ -352,10 +423,52 @@ static kda_status_t fwd_impl(const kda_fwd_desc_t* d, const void* q, const void*
             sn.eps = norm->eps;
             snp = &sn;
         }
-        const int S = cu_seqlens ? 1 : split_segments(L.ncT);
+        const int S = cu_seqlens || pscan ? 1 : split_segments(L.ncT);
         e = cudaMemsetAsync(ws.counters, 0, sizeof(unsigned long long) * S, s);
         if (e != cudaSuccess) return cuda_fail(e, "kda_fwd workspace counters");
-        if (S == 1) {
+        if (pscan) {
+            // intra-chunk kernel over every chunk; then segment 0 (side stream) beside the maps
+            // of segments 1 .. P-2 (caller's stream); the segments' initial states; then
+            // segments 1 .. P-1 at once
+            const int P = L.P, m = (L.ncT + P - 1) / P;
+            const size_t states = (size_t)d->num_seqs * d->H * 16384;   // floats per state set
+            float* maps = reinterpret_cast<float*>(w + L.maps);         // A: [P-2], B: [P-2]
+            float* sinit = maps + 2 * (size_t)(P - 2) * states;          // [P-1]
+            SideStream* ss = nullptr;
+            if ((e = side_stream(&ss)) != cudaSuccess) return cuda_fail(e, "kda_fwd side stream");
+            e = kda::launch_chunk64_intra(p, 0, L.ncT, ws.counters, s);
+            if (e != cudaSuccess) return cuda_fail(e, "kda_fwd intra-chunk launch");
+            kda::ScanSegment seg0{0, m, h0, sinit};
+            kda::ScanSegment mid{0, 0, nullptr, maps};
+            mid.seg_m = m;
+            mid.seg_p0 = 1;
+            mid.seg_count = P - 2;
+            mid.groups = 2;
+            mid.nseg = P;
+            mid.ident = true;
+            mid.no_out = true;
+            kda::ScanSegment rest{0, 0, sinit, hT};
+            rest.seg_m = m;
+            rest.seg_p0 = 1;
+            rest.seg_count = P - 1;
+            rest.nseg = P;
+            rest.hT_last = true;
+            cudaError_t first = cudaSuccess;
+            if ((first = cudaEventRecord(ss->seg[0], s)) == cudaSuccess &&
+                (first = cudaStreamWaitEvent(ss->aux, ss->seg[0], 0)) == cudaSuccess &&
+                (first = kda::launch_chunk_scan(p, seg0, ss->aux, snp)) == cudaSuccess)
+                first = kda::launch_chunk_scan(p, mid, s);
+            // join even after a failed launch, so that nothing is left pending on the side stream
+            e = cudaEventRecord(ss->join, ss->aux);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
+            if (first != cudaSuccess) return cuda_fail(first, "kda_fwd state-pass launch");
+            if (e != cudaSuccess) return cuda_fail(e, "kda_fwd side stream join");
+            e = kda::launch_scan_combine(maps, maps + (size_t)(P - 2) * states, sinit,
+                                         d->num_seqs * d->H, P - 2, s);
+            if (e != cudaSuccess) return cuda_fail(e, "kda_fwd segment-state launch");
+            e = kda::launch_chunk_scan(p, rest, s, snp);
+            if (e != cudaSuccess) return cuda_fail(e, "kda_fwd state-pass launch");
+        } else if (S == 1) {
             e = kda::launch_chunk64_intra(p, 0, L.ncT, ws.counters, s);
             if (e != cudaSuccess) return cuda_fail(e, "kda_fwd intra-chunk launch");
             e = kda::launch_chunk_scan(p, kda::ScanSegment{0, L.ncT, h0, hT}, s, snp);

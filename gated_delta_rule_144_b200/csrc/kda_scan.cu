@@ -106,6 +106,10 @@ struct ScanArgs {
     const float* nw;             // norm weight [128]
     float eps;
     int T, H, N, ncT;       // ncT: chunk records per sequence when cu is null
+    // segmented launch (seg_m > 0; equal-length sequences): unit u = (group, segment, chain),
+    // as ScanSegment describes; ident: group 0 starts from S = I with U~ = 0
+    int seg_m, seg_p0, seg_count, nseg;
+    int ident, no_out, hT_last;
     long long G;            // chunk records per head
     long long budget;
     int debug_stall;
@@ -157,8 +161,19 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
     const bool epi = tid >= kEpi0 && tid < kLoader;
     const bool loader = tid >= kLoader;
     const int unit = blockIdx.x;
-    const int h = unit % args.H;
-    const int n = args.order ? args.order[unit / args.H] : unit / args.H;
+    int chain = unit, seg = 0, c_begin = args.c_begin, c_end = args.c_end;
+    bool ident = false;
+    if (args.seg_m > 0) {
+        const int chains = args.N * args.H;
+        chain = unit % chains;
+        const int rest = unit / chains;
+        seg = args.seg_p0 + rest % args.seg_count;
+        ident = args.ident && rest < args.seg_count;
+        c_begin = seg * args.seg_m;
+        c_end = c_begin + args.seg_m;
+    }
+    const int h = chain % args.H;
+    const int n = args.order ? args.order[chain / args.H] : chain / args.H;
 
     long long t0, t1, g0;
     if (args.cu) {
@@ -180,8 +195,8 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
         return;
     }
     {   // this launch's segment of the chain: chunks [c_begin, c_end), possibly empty
-        const long long sb0 = min(t1, t0 + (long long)kC * args.c_begin);
-        const long long sb1 = min(t1, t0 + (long long)kC * args.c_end);
+        const long long sb0 = min(t1, t0 + (long long)kC * c_begin);
+        const long long sb1 = min(t1, t0 + (long long)kC * c_end);
         g0 += (sb0 - t0 + kC - 1) / kC;
         t0 = sb0;
         t1 = max(sb0, sb1);
@@ -227,15 +242,21 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
     const uint32_t tbase = *tmem_s;
     const uint32_t lq = (uint32_t)(32 * qd) << 16;   // this warp's TMEM lane quarter
     const size_t state_base = ((size_t)n * args.H + h) * kD * kD;
+    // a segmented launch keeps its states per unit (the last segment's hT per chain)
+    const size_t h0_base = args.seg_m > 0 ? (size_t)unit * kD * kD : state_base;
+    float* const hT = args.seg_m > 0 && args.hT_last && seg != args.nseg - 1 ? nullptr : args.hT;
+    const size_t hT_base = args.seg_m > 0 && !args.hT_last ? (size_t)unit * kD * kD : state_base;
 
     // initial state, transposed: lane j, column c holds S[c][j]; this thread: c in [64 hs, +64)
+    // (the identity for a transition-map unit)
 #pragma unroll 1
     for (int p = 0; p < (data ? 2 : 0); ++p) {
         float v[32];
         const int c0 = 64 * hs + 32 * p;
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-            v[i] = args.h0 ? args.h0[state_base + (size_t)(c0 + i) * kD + j] : 0.f;
+            v[i] = ident ? (c0 + i == j ? 1.f : 0.f)
+                         : (args.h0 ? args.h0[h0_base + (size_t)(c0 + i) * kD + j] : 0.f);
         tmem_st32(tbase + lq + TS + c0, v);
     }
     tmem_st_wait();
@@ -370,9 +391,10 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
                 tmem_ld32(tbase + lq + TS + 64 * hs + 32, vb);
                 const float* dec = reinterpret_cast<const float*>(stp + ST_DEC) + 64 * hs;
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const uint4 x = *reinterpret_cast<const uint4*>(
-                        stp + ST_UT + sw128_off(128, j, 32 * hs + 8 * m));
+                for (int m = 0; m < 4; ++m) {   // (zero for a transition-map unit)
+                    const uint4 x = ident ? make_uint4(0u, 0u, 0u, 0u)
+                                          : *reinterpret_cast<const uint4*>(
+                                                stp + ST_UT + sw128_off(128, j, 32 * hs + 8 * m));
                     ub[4 * m] = x.x; ub[4 * m + 1] = x.y; ub[4 * m + 2] = x.z; ub[4 * m + 3] = x.w;
                 }
                 tmem_ld_wait();
@@ -452,7 +474,7 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
                 if (tid == kMma) mbar_wait(bar_mma2, (uint32_t)(mma2_chunk & 1), 1ll << 31);
             } else {
                 tc_fence_after();
-                if (args.hT && data) {
+                if (hT && data) {
 #pragma unroll 1
                     for (int p = 0; p < 2; ++p) {
                         float v[32];
@@ -461,7 +483,7 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
                         tmem_ld_wait();
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
-                            args.hT[state_base + (size_t)(c0 + i) * kD + j] = v[i];
+                            hT[hT_base + (size_t)(c0 + i) * kD + j] = v[i];
                     }
                 }
             }
@@ -517,6 +539,7 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
             }
             tc_fence_before();
             mbar_arrive(bar_dfree0 + 8 * (c & 1));   // D buffer c & 1 may be overwritten now
+            if (args.no_out) continue;
             // output tile c & 1 was last stored for chunk c-2: that store must have read it
             if (et == 0 && c >= 2) bulk_wait_read_le1();
             bar_sync(kBarEpi, kEpiThreads);
@@ -589,6 +612,143 @@ chunk_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs args) {
     if (warp == 0) tmem_dealloc(tbase, kTmemCols);
 }
 
+// Initial states of the two-level state pass's segments, S_p = A_{p-1} S_{p-1} + B_{p-1} for
+// p = 1 .. steps (a few 128 x 128 x 128 products per chain, on the critical path once per
+// segment). Block (jb, chain) owns value columns 16 jb .. 16 jb + 15 of one chain (the columns
+// are independent); warp w computes rows 16 w .. 16 w + 15 of them with tensor-core products in
+// 3xTF32: each fp32 operand x = hi + lo with hi = x rounded to tf32 and lo = the rest rounded
+// to tf32, and a b is taken as hi_a hi_b + (lo_a hi_b + hi_a lo_b) (the lo lo term, about 2^-22 of
+// the product, is dropped), each of the three in its own fp32 accumulator (short dependency
+// chains), summed at the end with B_{p-1}. The maps are staged in shared memory by 16-byte
+// asynchronous copies, double-buffered: A_p lands while step p computes, and B_p is read into
+// registers a step ahead. The row strides (132 floats for A, 24 for S) put every fragment read
+// of a warp in distinct banks.
+constexpr int kCombCols = 16;
+constexpr int kCombLdA = 132;
+constexpr int kCombLdS = 24;
+constexpr uint32_t kCombSmem = (uint32_t)(2 * kD * kCombLdA + kD * kCombLdS) * 4;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+    hi = to_tf32(x);
+    lo = to_tf32(x - __uint_as_float(hi));
+}
+
+__global__ void __launch_bounds__(256)
+scan_combine_kernel(const float* __restrict__ amap, const float* __restrict__ bmap,
+                    float* __restrict__ sinit, int chains, int steps) {
+    extern __shared__ float4 comb_raw[];
+    float* As0 = reinterpret_cast<float*>(comb_raw);   // 2 x [128][kCombLdA]: A_{p-1}, A_p
+    float* Ss = As0 + 2 * kD * kCombLdA;                // [128][kCombLdS]: S_{p-1}'s columns
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3, r0 = 16 * warp;
+    const int jb = blockIdx.x, chain = blockIdx.y;
+    const size_t mat = (size_t)kD * kD;
+    const size_t col0 = (size_t)kCombCols * jb;
+    // A_{p-1} into buffer (p - 1) & 1: 16 copies of 16 bytes per thread, one commit group
+    auto stage = [&](int p) {
+        const float* A = amap + ((size_t)(p - 1) * chains + chain) * mat;
+        float* As = As0 + ((p - 1) & 1) * kD * kCombLdA;
+#pragma unroll
+        for (int u = 0; u < kD * kD / 4 / 256; ++u) {
+            const int i = tid + 256 * u, r = i >> 5, q = i & 31;
+            cp_async16(smem_u32(As + r * kCombLdA + 4 * q), A + (size_t)r * kD + 4 * q);
+        }
+        cp_async_commit();
+    };
+    // B_{p-1} of this thread's fragment into bnext
+    float bnext[2][4];
+    auto load_b = [&](int p) {
+        const float* B = bmap + ((size_t)(p - 1) * chains + chain) * mat + col0;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const int col = 8 * nt + 2 * t;
+            const float2 u = *reinterpret_cast<const float2*>(B + (size_t)(r0 + g) * kD + col);
+            const float2 v = *reinterpret_cast<const float2*>(B + (size_t)(r0 + g + 8) * kD + col);
+            bnext[nt][0] = u.x; bnext[nt][1] = u.y; bnext[nt][2] = v.x; bnext[nt][3] = v.y;
+        }
+    };
+    stage(1);
+    load_b(1);
+    for (int i = tid; i < kD * kCombCols / 4; i += 256) {
+        const int r = i >> 2, q = i & 3;
+        *reinterpret_cast<float4*>(Ss + r * kCombLdS + 4 * q) =
+            *reinterpret_cast<const float4*>(sinit + chain * mat + (size_t)r * kD + col0 + 4 * q);
+    }
+    for (int p = 1; p <= steps; ++p) {
+        // the next map goes into the buffer step p - 1 read (released by its closing barrier)
+        if (p < steps) stage(p + 1);
+        const float* As = As0 + ((p - 1) & 1) * kD * kCombLdA;
+        // B_{p-1} (read a step ahead) and the next step's, in the m16n8 fragment layout: rows
+        // r0 + g (+ 8), columns 8 nt + 2 t (+ 1)
+        float bias[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) bias[nt][e] = bnext[nt][e];
+        if (p < steps) load_b(p + 1);
+        float acc[2][4] = {}, acc_x[2][4] = {}, acc_y[2][4] = {};
+        if (p < steps)
+            cp_async_wait<1>();   // this step's map landed (the next one may still be in flight)
+        else
+            cp_async_wait<0>();
+        __syncthreads();   // A_{p-1} staged by every thread, S_{p-1} complete
+#pragma unroll 4
+        for (int kk = 0; kk < kD; kk += 8) {
+            const float* la = As + (r0 + g) * kCombLdA + kk + t;
+            uint32_t ah[4], al[4];
+            split_tf32(la[0], ah[0], al[0]);
+            split_tf32(la[8 * kCombLdA], ah[1], al[1]);
+            split_tf32(la[4], ah[2], al[2]);
+            split_tf32(la[8 * kCombLdA + 4], ah[3], al[3]);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const float* lb = Ss + (kk + t) * kCombLdS + 8 * nt + g;
+                uint32_t bh[2], bl[2];
+                split_tf32(lb[0], bh[0], bl[0]);
+                split_tf32(lb[4 * kCombLdS], bh[1], bl[1]);
+                mma_tf32_16x8x8(acc_x[nt], al, bh);
+                mma_tf32_16x8x8(acc_y[nt], ah, bl);
+                mma_tf32_16x8x8(acc[nt], ah, bh);
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                acc[nt][e] = bias[nt][e] + (acc[nt][e] + (acc_x[nt][e] + acc_y[nt][e]));
+        __syncthreads();   // every warp has read A_{p-1} and S_{p-1}
+        float* out = sinit + ((size_t)p * chains + chain) * mat + col0;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const int col = 8 * nt + 2 * t;
+            *reinterpret_cast<float2*>(Ss + (r0 + g) * kCombLdS + col) =
+                make_float2(acc[nt][0], acc[nt][1]);
+            *reinterpret_cast<float2*>(Ss + (r0 + g + 8) * kCombLdS + col) =
+                make_float2(acc[nt][2], acc[nt][3]);
+            *reinterpret_cast<float2*>(out + (size_t)(r0 + g) * kD + col) =
+                make_float2(acc[nt][0], acc[nt][1]);
+            *reinterpret_cast<float2*>(out + (size_t)(r0 + g + 8) * kD + col) =
+                make_float2(acc[nt][2], acc[nt][3]);
+        }
+    }
+}
+
 long long scan_wait_budget() {
     static long long budget = [] {
         const char* s = std::getenv("KDA_DEBUG_WAIT_CYCLES");
@@ -616,7 +776,8 @@ int scan_debug_stall() {
 cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaStream_t stream,
                               const ScanNorm* norm) {
     const SplitWorkspace& ws = *p.split;
-    const long long units = (long long)p.N * p.H;
+    const long long chains = (long long)p.N * p.H;
+    const long long units = seg.seg_m > 0 ? chains * seg.seg_count * seg.groups : chains;
     if (units == 0) return cudaSuccess;
     if (units > 0x7fffffffLL || ws.G * p.H * 128 > 0x7fffffffLL)
         return cudaErrorInvalidConfiguration;
@@ -656,6 +817,13 @@ cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaSt
     a.hT = seg.hT;
     a.c_begin = seg.c_begin;
     a.c_end = seg.c_end;
+    a.seg_m = seg.seg_m;
+    a.seg_p0 = seg.seg_p0;
+    a.seg_count = seg.seg_count;
+    a.nseg = seg.nseg;
+    a.ident = seg.ident ? 1 : 0;
+    a.no_out = seg.no_out ? 1 : 0;
+    a.hT_last = seg.hT_last ? 1 : 0;
     a.o = static_cast<__nv_bfloat16*>(p.o);
     a.decay = ws.decay;
     if (norm) {
@@ -672,6 +840,21 @@ cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaSt
     a.debug_stall = scan_debug_stall();
     a.err = p.err;
     chunk_scan_kernel<<<(unsigned)units, kThreads, kSmemBytes, stream>>>(m, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scan_combine(const float* amap, const float* bmap, float* sinit, int chains,
+                                int steps, cudaStream_t stream) {
+    if (steps <= 0 || chains <= 0) return cudaSuccess;
+    if (chains > 65535) return cudaErrorInvalidConfiguration;
+    static PerDevice attr;
+    const cudaError_t attr_err = attr.run([](int) {
+        return cudaFuncSetAttribute(scan_combine_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCombSmem);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    scan_combine_kernel<<<dim3(kD / kCombCols, (unsigned)chains), 256, kCombSmem, stream>>>(
+        amap, bmap, sinit, chains, steps);
     return cudaGetLastError();
 }
 

@@ -106,7 +106,13 @@ typedef struct {
  *             KDA_SPLIT_SEGMENTS, 1-16, overrides): the state pass of one segment runs on an internal high-priority stream
  *             while the intra-chunk kernel works on the next, and the caller's stream waits for
  *             both before the call's later work; the state between segments (64 KiB per sequence
- *             and head) is kept in the workspace. With less workspace (but at least
+ *             and head) is kept in the workspace. Equal-length sequences with few chains
+ *             (sequences x heads) and enough chunks instead run a two-level state pass (see
+ *             kda_fwd_scan_segments): the chunks are cut into P segments; the map from a
+ *             segment's initial to its final state is affine, S -> A S + B, so the state pass
+ *             computes A and B of the inner segments beside segment 0, chains the segments'
+ *             initial states in fp32, and then runs every segment at once (3 P - 5 states of
+ *             64 KiB per sequence and head in the workspace). With less workspace (but at least
  *             kda_fwd_workspace_size_min(desc), which is 0 unless documents are packed) one fused
  *             kernel per (sequence, head) does both, with no intermediate storage. Both give the
  *             same result up to bf16 rounding of the stored factors. May be NULL when the minimum
@@ -236,6 +242,18 @@ int kda_fwd_algorithm(const kda_fwd_desc_t* desc, int has_cu_seqlens);
  * kda_fwd does. Host-only, no CUDA calls; the negated kda_status_t for a rejected description.
  */
 int kda_fwd_split_segments(const kda_fwd_desc_t* desc, int has_cu_seqlens);
+
+/*
+ * Segments P of kda_fwd's two-level state pass for `desc` (equal-length sequences): P >= 3 when
+ * the call runs it (with kda_fwd_workspace_size(desc) bytes of workspace), 1 for the plain state
+ * pass (packed documents, many chains, short sequences, the per-token path). P is chosen from a
+ * cost model of the phases; KDA_SCAN_SEGMENTS (read per call) overrides it: 0 or 1 = the plain
+ * pass, 3 to 32 = that many segments of ceil(chunks / P) chunks (fewer when that leaves a
+ * segment empty). Results differ from the plain pass's only by rounding (the segments' initial
+ * states are products of fp32 maps whose factors were rounded to bf16 like the state's).
+ * Host-only, no CUDA calls; the negated kda_status_t for a rejected description.
+ */
+int kda_fwd_scan_segments(const kda_fwd_desc_t* desc, int has_cu_seqlens);
 
 /*
  * Workspace bytes for the fastest path kda_fwd has for `desc` (the split chunked path when it

@@ -183,6 +183,7 @@ def test_split_segments_rule(L, monkeypatch):
     seg = lambda T, varlen=0, **kw: L.kda_fwd_split_segments(ctypes.byref(_desc(T=T, **kw)),
                                                              varlen)
     monkeypatch.delenv("KDA_SPLIT_SEGMENTS", raising=False)
+    monkeypatch.setenv("KDA_SCAN_SEGMENTS", "0")   # the plain state pass (no two-level plan)
     assert seg(64 * 63) == 1 and seg(64 * 64) == 1 and seg(64 * 64 + 1) == 2
     assert seg(64 * 101) == 3 and seg(65536) == 12 and seg(1 << 20) == 12
     assert seg(65536, varlen=1, B=1, num_seqs=4) == 1
@@ -294,3 +295,34 @@ def test_short_conv_rejects_on_host(L):
     assert b"overlaps" in L.kda_last_error()
     assert call(B=2, cu=P(FAKE)) == 1            # cu_seqlens needs B == 1
     assert call(T=0) == 0                        # no tokens: nothing to do
+
+
+def test_scan_segments_rule(L, monkeypatch):
+    """Host plan of the two-level state pass: few chains of many chunks take it, many chains or
+    short sequences the plain pass; KDA_SCAN_SEGMENTS overrides (capped by the chunks, no empty
+    segment); its states grow the workspace; the split path then runs one chunk segment."""
+    monkeypatch.delenv("KDA_SCAN_SEGMENTS", raising=False)
+
+    def plan(B, T, H, cu=0, **kw):
+        return L.kda_fwd_scan_segments(ctypes.byref(_desc(B=B, T=T, H=H, num_seqs=B, **kw)), cu)
+
+    assert plan(1, 4096, 16) >= 3              # 16 chains of 64 chunks
+    assert plan(2, 65536, 32) == 1             # 64 chains: chunk segments overlap instead
+    assert plan(4, 4096, 16) == 1              # 64 chains
+    assert plan(1, 200, 3) == 1                # 4 chunks
+    assert plan(1, 4096, 16, cu=1) == 1        # packed documents
+    assert plan(1, 4096, 16, chunk_size=1) == 1
+    assert plan(1, 4096, 16, dtype=7) < 0      # rejected description
+    d = _desc(B=1, T=4096, H=16, num_seqs=1)
+    assert L.kda_fwd_split_segments(ctypes.byref(d), 0) == 1
+    ws_two_level = L.kda_fwd_workspace_size(ctypes.byref(d))
+    for v, want in (("0", 1), ("1", 1), ("2", 1), ("3", 3), ("5", 5), ("40", 32)):
+        monkeypatch.setenv("KDA_SCAN_SEGMENTS", v)
+        assert plan(1, 4096, 16) == want, v
+    assert plan(1, 64 * 13 + 29, 3) == 14      # 14 chunks: one per segment
+    assert plan(1, 64 * 9, 3) == 9
+    monkeypatch.setenv("KDA_SCAN_SEGMENTS", "7")
+    assert plan(1, 64 * 10, 3) == 5            # 7 asked: segments of 2 chunks, 5 of them
+    monkeypatch.setenv("KDA_SCAN_SEGMENTS", "0")
+    ws_plain = L.kda_fwd_workspace_size(ctypes.byref(d))
+    assert ws_two_level > ws_plain

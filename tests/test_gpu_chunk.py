@@ -165,10 +165,13 @@ def test_long_context_full_size_every_chain(name):
         assert worst[path][0] <= TOL_BF16 and worst[path][1] <= TOL_BF16, (path, worst[path])
 
 
-def test_segmented_split_path_uneven_segments():
+def test_segmented_split_path_uneven_segments(monkeypatch):
     """Equal-length sequences of 101 chunks (the last one partial) run the split path in three
     chunk segments of 33, 34 and 34 chunks, the state crossing each boundary through the
-    workspace: o and hT against the oracle."""
+    workspace: o and hT against the oracle. (The plain state pass: with 4 chains the default
+    plan would take the two-level one.)"""
+    monkeypatch.setenv("KDA_SCAN_SEGMENTS", "0")
+    assert kda.fwd_split_segments(2, 64 * 100 + 17, 2, 128, 128, 2) == 3
     _check(synth.prefill_inputs("long-t65536", B=2, T=64 * 100 + 17, H=2, h0_std=0.05, seed=23))
 
 
@@ -177,6 +180,7 @@ def test_segment_count_does_not_change_the_result(monkeypatch):
     segment count gives bit-identical o and hT."""
     inp = to(synth.prefill_inputs("long-t65536", B=1, T=64 * 70 + 5, H=3, h0_std=0.05, seed=29),
              DEV)
+    monkeypatch.setenv("KDA_SCAN_SEGMENTS", "0")   # the plain state pass, in chunk segments
     outs = []
     for segs in ("1", "2", "5", "8"):
         monkeypatch.setenv("KDA_SPLIT_SEGMENTS", segs)
@@ -186,6 +190,119 @@ def test_segment_count_does_not_change_the_result(monkeypatch):
     assert kda.get_device_error() == 0
     for o, hT in outs[1:]:
         assert torch.equal(o, outs[0][0]) and torch.equal(hT, outs[0][1])
+
+
+@pytest.mark.parametrize("P,expect", [("3", 3), ("4", 4), ("7", 7), ("32", 14)])
+def test_two_level_state_pass_against_the_oracle(P, expect, monkeypatch):
+    """The two-level state pass, forced to P segments (KDA_SCAN_SEGMENTS), on 2 sequences of
+    14 chunks (the last one partial) x 3 heads with h0: segment 0 from h0, the transition maps
+    and zero-start states of the inner segments, their fp32 chain, then the other segments at
+    once; o and hT against the oracle. 32 asked gives one chunk per segment (14 segments). The
+    gates decay slowly (log g = -softplus(N(-5, 1)): the median channel keeps about 0.65 of its
+    state over a chunk), so every segment's initial state weighs on its outputs."""
+    monkeypatch.setenv("KDA_SCAN_SEGMENTS", P)
+    inp = synth.prefill_inputs("prefill-t4096", B=2, T=64 * 13 + 29, H=3, h0_std=0.05,
+                               decay_mu=-5.0, seed=31)
+    assert kda.fwd_scan_segments(2, inp["T"], 3, 128, 128, 2) == expect
+    _check(inp)
+
+
+@pytest.mark.parametrize("P", ["0", "4", "13"])
+def test_two_level_state_pass_carries_h0_exactly_without_writes(P, monkeypatch):
+    """beta = 0: every chunk's map is the pure decay (W = U~ = 0 exactly), so the final state is
+    diag(prod_t g_t) h0 in closed form (the oracle pin beta = 0 => S_T = diag(prod g) S_0). The
+    two-level pass carries h0 through the transition maps alone (A_p = the segment's decay
+    product, B_p = 0, the fp32 chain of the segments' initial states): hT must meet the closed
+    form to fp32 rounding, like the plain pass (P = 0); o against the oracle. The bound, 2e-4,
+    allows for the chunk decays being products of 64 fp32 exponentials each (839 tokens); a
+    segment's decay lost or applied twice would be off by about 45 %."""
+    monkeypatch.setenv("KDA_SCAN_SEGMENTS", P)
+    inp = synth.prefill_inputs("prefill-t4096", B=2, T=64 * 13 + 7, H=2, h0_std=1.0,
+                               decay_mu=-5.0, seed=34)
+    inp["beta"] = torch.zeros_like(inp["beta"])
+    o, hT, st = _run(inp)
+    assert st == 0
+    total = inp["log_g"].double().sum(dim=1)                       # [B, H, dk]
+    closed = torch.exp(total)[..., None] * inp["h0"].double()      # [B, H, dk, dv]
+    eh = rel_l2(host(hT), closed.numpy())
+    o_ref, _ = oracle_fwd(inp)
+    eo = rel_l2(host(o), o_ref)
+    print("P %s: hT vs closed form %.3e, o %.3e" % (P, eh, eo))
+    assert eh <= 2e-4 and eo <= TOL_BF16
+
+
+def test_two_level_state_pass_weak_writes_slow_decay(monkeypatch):
+    """beta scaled by 0.05 and slow gates (log g = -softplus(N(-6, 1))): the state persists over
+    many chunks, so the segments' initial states (the transition maps and zero-start states of
+    the inner segments and their chain) carry most of hT. Forced 5 segments against the oracle and
+    against the plain pass."""
+    inp = synth.prefill_inputs("prefill-t4096", B=1, T=64 * 30 + 11, H=3, h0_std=0.5,
+                               decay_mu=-6.0, seed=35)
+    inp["beta"] = (inp["beta"].float() * 0.05).to(inp["beta"].dtype)
+    monkeypatch.setenv("KDA_SCAN_SEGMENTS", "5")
+    eo, eh = _check(inp)
+    o2, h2, st = _run(inp)
+    monkeypatch.setenv("KDA_SCAN_SEGMENTS", "0")
+    o1, h1, st1 = _run(inp)
+    assert st == 0 and st1 == 0
+    d_o, d_h = rel_l2(host(o2), host(o1)), rel_l2(host(h2), host(h1))
+    print("two-level vs plain: o %.3e hT %.3e" % (d_o, d_h))
+    assert d_o <= TOL_BF16 and d_h <= TOL_BF16
+
+
+def test_two_level_and_plain_state_pass_slow_decay(monkeypatch):
+    """Slow gates (log g = -softplus(N(-6, 1))) over 40 chunks x 4 chains: the two-level pass
+    (default plan) and the plain pass both meet the oracle, and differ from each other only by
+    rounding."""
+    monkeypatch.delenv("KDA_SCAN_SEGMENTS", raising=False)
+    inp = synth.prefill_inputs("prefill-t4096", B=1, T=64 * 40, H=4, h0_std=0.05,
+                               decay_mu=-6.0, seed=33)
+    assert kda.fwd_scan_segments(1, inp["T"], 4, 128, 128, 1) >= 3
+    _check(inp)
+    o2, h2, st = _run(inp)
+    assert st == 0
+    monkeypatch.setenv("KDA_SCAN_SEGMENTS", "0")
+    _check(inp)
+    o1, h1, st = _run(inp)
+    assert st == 0
+    assert not torch.equal(h1, h2)   # the two passes round differently
+    assert rel_l2(host(o2), host(o1)) <= TOL_BF16 and rel_l2(host(h2), host(h1)) <= TOL_BF16
+
+
+def test_two_level_state_pass_without_final_state_and_with_steep_decays(monkeypatch):
+    """Forced two-level pass (5 segments) with output_final_state=False (only o is written; the
+    segments' states stay in the workspace), and with log g = -30 everywhere (every chunk takes
+    the direct path; the transition maps are then all but zero)."""
+    monkeypatch.setenv("KDA_SCAN_SEGMENTS", "5")
+    inp = synth.prefill_inputs("long-t65536", B=1, T=64 * 10, H=2, h0_std=0.05, decay_mu=-5.0,
+                               seed=32)
+    g = to(inp, DEV)
+    o, hT = kda.fwd(g["q"], g["k"], g["v"], g["log_g"], g["beta"], h0=g["h0"],
+                    output_final_state=False)
+    torch.cuda.synchronize()
+    assert hT is None and kda.get_device_error() == 0
+    o_ref, _ = oracle_fwd(inp)
+    assert rel_l2(host(o), o_ref) <= TOL_BF16
+    inp["log_g"] = torch.full_like(inp["log_g"], -30.0)
+    _check(inp)
+
+
+def test_prefill_t4096_two_level_and_plain_state_pass(monkeypatch):
+    """The T=4096, H=16 workload at full size: the default plan takes the two-level state pass
+    (16 chains); it and the plain pass (KDA_SCAN_SEGMENTS=0) both meet the oracle."""
+    monkeypatch.delenv("KDA_SCAN_SEGMENTS", raising=False)
+    inp = synth.prefill_inputs("prefill-t4096")
+    assert kda.fwd_scan_segments(1, 4096, 16, 128, 128, 1) >= 3
+    o_ref, h_ref = oracle_fwd(inp)
+    res = {}
+    for plan in ("default", "0"):
+        if plan == "0":
+            monkeypatch.setenv("KDA_SCAN_SEGMENTS", "0")
+        o, hT, st = _run(inp)
+        assert st == 0
+        res[plan] = (rel_l2(host(o), o_ref), rel_l2(host(hT), h_ref))
+        print(plan, "rel-L2 o %.3e hT %.3e" % res[plan])
+        assert res[plan][0] <= TOL_BF16 and res[plan][1] <= TOL_BF16
 
 
 def test_workspace_size_selects_the_path():
