@@ -140,7 +140,8 @@ KERNEL_SOURCES = {
     "kda_recurrent": ["kda_recurrent.cu", "kda_internal.cuh"],
     "kda_chunk64": ["kda_chunk64.cu", "kda_sm100.cuh", "kda_internal.cuh", "kda_tma.cuh"],
     "kda_chunk64_intra": ["kda_intra.cu", "kda_sm100.cuh", "kda_internal.cuh", "kda_tma.cuh"],
-    "kda_chunk_scan": ["kda_scan.cu", "kda_sm100.cuh", "kda_internal.cuh", "kda_tma.cuh"],
+    "kda_chunk_scan": ["kda_scan.cu", "kda_scan.cuh", "kda_sm100.cuh", "kda_internal.cuh",
+                       "kda_tma.cuh"],
     "kda_short_conv": ["kda_conv.cu", "kda_internal.cuh"],
 }
 

@@ -13,6 +13,7 @@
 
 #include "kda_bwd.cuh"
 #include "kda_internal.cuh"
+#include "kda_scan.cuh"
 
 namespace {
 
@@ -438,26 +439,28 @@ static kda_status_t fwd_impl(const kda_fwd_desc_t* d, const void* q, const void*
             if ((e = side_stream(&ss)) != cudaSuccess) return cuda_fail(e, "kda_fwd side stream");
             e = kda::launch_chunk64_intra(p, 0, L.ncT, ws.counters, s);
             if (e != cudaSuccess) return cuda_fail(e, "kda_fwd intra-chunk launch");
-            kda::ScanSegment seg0{0, m, h0, sinit};
-            kda::ScanSegment mid{0, 0, nullptr, maps};
-            mid.seg_m = m;
-            mid.seg_p0 = 1;
-            mid.seg_count = P - 2;
-            mid.groups = 2;
-            mid.nseg = P;
-            mid.ident = true;
-            mid.no_out = true;
-            kda::ScanSegment rest{0, 0, sinit, hT};
-            rest.seg_m = m;
-            rest.seg_p0 = 1;
-            rest.seg_count = P - 1;
-            rest.nseg = P;
-            rest.hT_last = true;
+            const kda::ScanSegment seg0{0, m, h0, sinit};
+            const kda::ScanSegment mid{0, 0, nullptr, maps};
+            kda::ScanSplit mid_split;
+            mid_split.seg_m = m;
+            mid_split.seg_p0 = 1;
+            mid_split.seg_count = P - 2;
+            mid_split.groups = 2;
+            mid_split.nseg = P;
+            mid_split.ident = true;
+            mid_split.no_out = true;
+            const kda::ScanSegment rest{0, 0, sinit, hT};
+            kda::ScanSplit rest_split;
+            rest_split.seg_m = m;
+            rest_split.seg_p0 = 1;
+            rest_split.seg_count = P - 1;
+            rest_split.nseg = P;
+            rest_split.hT_last = true;
             cudaError_t first = cudaSuccess;
             if ((first = cudaEventRecord(ss->seg[0], s)) == cudaSuccess &&
                 (first = cudaStreamWaitEvent(ss->aux, ss->seg[0], 0)) == cudaSuccess &&
                 (first = kda::launch_chunk_scan(p, seg0, ss->aux, snp)) == cudaSuccess)
-                first = kda::launch_chunk_scan(p, mid, s);
+                first = kda::launch_chunk_scan_split(p, mid, mid_split, s);
             // join even after a failed launch, so that nothing is left pending on the side stream
             e = cudaEventRecord(ss->join, ss->aux);
             if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
@@ -466,7 +469,7 @@ static kda_status_t fwd_impl(const kda_fwd_desc_t* d, const void* q, const void*
             e = kda::launch_scan_combine(maps, maps + (size_t)(P - 2) * states, sinit,
                                          d->num_seqs * d->H, P - 2, s);
             if (e != cudaSuccess) return cuda_fail(e, "kda_fwd segment-state launch");
-            e = kda::launch_chunk_scan(p, rest, s, snp);
+            e = kda::launch_chunk_scan_split(p, rest, rest_split, s, snp);
             if (e != cudaSuccess) return cuda_fail(e, "kda_fwd state-pass launch");
         } else if (S == 1) {
             e = kda::launch_chunk64_intra(p, 0, L.ncT, ws.counters, s);

@@ -44,25 +44,12 @@ struct SplitWorkspace {
 // pass of segment s overlaps the intra-chunk kernel of segment s + 1.
 constexpr int kMaxSegments = 16;
 
-// Two-level state pass (equal-length sequences with few chains): the chunks of every chain are
-// cut into segments of seg_m chunks. The map from a segment's initial state to its final state is
-// affine, S -> A_p S + B_p, so the segments' initial states follow from a short product chain over
-// the segments, after which every segment runs at once.
-constexpr int kMaxScanSegments = 32;
-
 // One launch of the state pass: chunks [c_begin, c_end) of every chain, from the state h0 to the
 // state hT (the caller's, or the workspace's scratch state between segments; either nullable).
-// With seg_m > 0 the launch is segmented instead: unit u = (group, segment, chain), chain =
-// u % (N H), segment = seg_p0 + (u / (N H)) % seg_count, group = u / (N H seg_count), chunks
-// [segment seg_m, (segment + 1) seg_m); h0 and hT are indexed by u (hT_last: only segment
-// nseg - 1 writes hT, at the chain's index). With ident, group 0 starts from S = I with U~ = 0
-// (it computes A_p); no_out suppresses the output stores.
 struct ScanSegment {
     int c_begin, c_end;
     const float* h0;
     float* hT;
-    int seg_m = 0, seg_p0 = 0, seg_count = 0, groups = 1, nseg = 0;
-    bool ident = false, no_out = false, hT_last = false;
 };
 
 struct FwdParams {
@@ -129,13 +116,6 @@ struct ScanNorm {
 };
 cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaStream_t stream,
                               const ScanNorm* norm = nullptr);
-
-// The segments' initial states of the two-level state pass, in fp32:
-//   sinit[p] = amap[p - 1] sinit[p - 1] + bmap[p - 1],  p = 1 .. steps,
-// every array [.][chains][128][128] (row = key channel, column = value column), sinit[0] given.
-cudaError_t launch_scan_combine(const float* amap, const float* bmap, float* sinit, int chains,
-                                int steps, cudaStream_t stream);
-
 // y = x / sqrt(mean(x^2) + eps) * w * sigmoid(gate) per vector of dv elements (dv <= 256);
 // y may alias x.
 cudaError_t launch_out_norm_gated(const void* x, const void* gate, const float* w, float eps,

@@ -49,6 +49,7 @@
 #include <mutex>
 
 #include "kda_internal.cuh"
+#include "kda_scan.cuh"
 #include "kda_sm100.cuh"
 #include "kda_tma.cuh"
 
@@ -107,7 +108,7 @@ struct ScanArgs {
     float eps;
     int T, H, N, ncT;       // ncT: chunk records per sequence when cu is null
     // segmented launch (seg_m > 0; equal-length sequences): unit u = (group, segment, chain),
-    // as ScanSegment describes; ident: group 0 starts from S = I with U~ = 0
+    // as ScanSplit describes; ident: group 0 starts from S = I with U~ = 0
     int seg_m, seg_p0, seg_count, nseg;
     int ident, no_out, hT_last;
     long long G;            // chunk records per head
@@ -775,9 +776,15 @@ int scan_debug_stall() {
 // when an order is given.
 cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaStream_t stream,
                               const ScanNorm* norm) {
+    return launch_chunk_scan_split(p, seg, ScanSplit{}, stream, norm);
+}
+
+cudaError_t launch_chunk_scan_split(const FwdParams& p, const ScanSegment& seg,
+                                    const ScanSplit& split, cudaStream_t stream,
+                                    const ScanNorm* norm) {
     const SplitWorkspace& ws = *p.split;
     const long long chains = (long long)p.N * p.H;
-    const long long units = seg.seg_m > 0 ? chains * seg.seg_count * seg.groups : chains;
+    const long long units = split.seg_m > 0 ? chains * split.seg_count * split.groups : chains;
     if (units == 0) return cudaSuccess;
     if (units > 0x7fffffffLL || ws.G * p.H * 128 > 0x7fffffffLL)
         return cudaErrorInvalidConfiguration;
@@ -817,13 +824,13 @@ cudaError_t launch_chunk_scan(const FwdParams& p, const ScanSegment& seg, cudaSt
     a.hT = seg.hT;
     a.c_begin = seg.c_begin;
     a.c_end = seg.c_end;
-    a.seg_m = seg.seg_m;
-    a.seg_p0 = seg.seg_p0;
-    a.seg_count = seg.seg_count;
-    a.nseg = seg.nseg;
-    a.ident = seg.ident ? 1 : 0;
-    a.no_out = seg.no_out ? 1 : 0;
-    a.hT_last = seg.hT_last ? 1 : 0;
+    a.seg_m = split.seg_m;
+    a.seg_p0 = split.seg_p0;
+    a.seg_count = split.seg_count;
+    a.nseg = split.nseg;
+    a.ident = split.ident ? 1 : 0;
+    a.no_out = split.no_out ? 1 : 0;
+    a.hT_last = split.hT_last ? 1 : 0;
     a.o = static_cast<__nv_bfloat16*>(p.o);
     a.decay = ws.decay;
     if (norm) {
