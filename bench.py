@@ -640,7 +640,7 @@ def run_secondary(kda, synth, args, dev, stream, world, rank):
                   "tokens/s": round(b["B"] * b["T"] * world / (ms / 1e3), 1),
                   "bytes_per_step": by,
                   "roofline_frac": round(by / (ms / 1e3) / 1e9 / hbm_peak, 5),
-                  "kernel": "kda_bwd (fp32 CUDA cores, 32 CTAs per chain: 4 value columns each)"}
+                  "kernel": "kda_bwd (fp32 CUDA cores, 16 warps per chain: 8 value columns each)"}
     del b, bdo, bdh, bws
     if kda.get_device_error() != 0:
         raise RuntimeError("device error in the secondary runs")

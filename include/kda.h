@@ -103,10 +103,10 @@ typedef struct {
  *             and heads and stores them here (about 72.5 KiB per 64-token chunk and head), then a
  *             state pass walks each sequence's chunks. For equal-length sequences of more than
  *             64 chunks the two run in chunk segments of at least 32 chunks (up to 12;
- *             KDA_SPLIT_SEGMENTS, 1-16, overrides): the state pass of one segment runs on an internal high-priority stream
- *             while the intra-chunk kernel works on the next, and the caller's stream waits for
- *             both before the call's later work; the state between segments (64 KiB per sequence
- *             and head) is kept in the workspace. Equal-length sequences with few chains
+ *             KDA_SPLIT_SEGMENTS, 1-16, overrides): the state pass of one segment runs on an
+ *             internal high-priority stream while the intra-chunk kernel works on the next, and
+ *             the caller's stream waits for both before the call's later work; the state between
+ *             segments (64 KiB per sequence and head) is kept in the workspace. Equal-length sequences with few chains
  *             (sequences x heads) and enough chunks instead run a two-level state pass (see
  *             kda_fwd_scan_segments): the chunks are cut into P segments; the map from a
  *             segment's initial to its final state is affine, S -> A S + B, so the state pass
@@ -161,8 +161,9 @@ kda_status_t kda_fwd_normed(const kda_fwd_desc_t* desc, const void* q, const voi
                             size_t workspace_bytes, kda_stream_t stream);
 
 /*
- * kda_bwd - gradients of the recurrence, for training (NeMo glm5_next layers, `_torch_recurrent_kda`
- * is a differentiable reference KDA; this is the derivative of kda_fwd's recurrence). For
+ * kda_bwd - gradients of the recurrence, for training (NeMo glm5_next layers,
+ * `_torch_recurrent_kda` is a differentiable reference KDA; this is the derivative of kda_fwd's
+ * recurrence). For
  * upstream gradients do (of o) and dhT (of the final states), computes the gradients of
  * L = sum <do, o> + <dhT, hT>:
  *   dq, dk    : [B, T, H, dk] float32      dv       : [B, T, H, dv] float32
@@ -171,13 +172,14 @@ kda_status_t kda_fwd_normed(const kda_fwd_desc_t* desc, const void* q, const voi
  * The forward arguments (desc, q, k, v, log_g, beta, h0, cu_seqlens) are as for kda_fwd; do has
  * the layout and dtype of o; dhT is [N, H, dk, dv] float32 or NULL (zero). dk = dv = 128
  * (KDA_ERR_UNSUPPORTED otherwise); desc->chunk_size is ignored. Every gradient is computed in
- * fp32 from the exact per-token recurrence; 32 CTAs per (sequence or document, head), one per 4
+ * fp32 from the exact per-token recurrence; 16 warps per (sequence or document, head), one per 8
  * value columns, run the forward storing the state every 64 tokens, then walk each 64-token chunk
  * backwards after re-running its forward. The workspace (kda_bwd_workspace_size bytes, 16-byte
  * aligned, device) holds those states. dq, dk, dlog_g and dbeta are sums over the value columns:
- * the call zeroes them on the stream and the 32 CTAs add their parts atomically, in no fixed order,
- * so their last bits may differ between runs (dv and dh0 are written once). Host-checkable errors
- * return before any launch; a malformed cu_seqlens is reported through kda_get_device_error.
+ * the call zeroes them on the stream and the 16 warps add their parts atomically, in no fixed
+ * order, so their last bits may differ between runs (dv and dh0 are written once).
+ * Host-checkable errors return before any launch; a malformed cu_seqlens is reported through
+ * kda_get_device_error.
  */
 kda_status_t kda_bwd(const kda_fwd_desc_t* desc, const void* q, const void* k, const void* v,
                      const float* log_g, const void* beta, const float* h0,
