@@ -408,3 +408,42 @@ def test_expired_wait_reports_timeout_and_context_survives():
     st, after = map(int, line.split()[1:])
     assert st == 4
     assert after == 0        # the context stays usable: the exact path runs clean afterwards
+
+
+@pytest.mark.parametrize("plan", ["segments", "two-level"])
+def test_split_call_replays_in_a_cuda_graph(plan, monkeypatch):
+    """The split path's fork and join (state passes on the library's side stream) are event
+    records and waits, so a call can be captured in a CUDA graph. The replay must equal the
+    eager call bit for bit. Chunk segments overlapping the intra-chunk kernel (plain state pass,
+    3 segments) and the two-level state pass (4 segments). The eager call also creates the
+    library's side stream, events and kernel attributes before the capture."""
+    if plan == "segments":
+        monkeypatch.setenv("KDA_SCAN_SEGMENTS", "0")
+        inp = synth.prefill_inputs("long-t65536", B=2, T=64 * 100 + 17, H=2, h0_std=0.05,
+                                   seed=36, device=DEV)
+    else:
+        monkeypatch.setenv("KDA_SCAN_SEGMENTS", "4")
+        inp = synth.prefill_inputs("prefill-t4096", B=1, T=64 * 20 + 5, H=3, h0_std=0.05,
+                                   decay_mu=-3.0, seed=37, device=DEV)
+    B, T, H = inp["B"], inp["T"], inp["H"]
+    if plan == "segments":
+        assert kda.fwd_split_segments(B, T, H, 128, 128, B) == 3
+    else:
+        assert kda.fwd_scan_segments(B, T, H, 128, 128, B) == 4
+    args = (inp["q"], inp["k"], inp["v"], inp["log_g"], inp["beta"])
+    ws = torch.empty(kda.fwd_workspace_size(B, T, H, 128, 128, B), dtype=torch.uint8,
+                     device=DEV)
+    o_ref, h_ref = kda.fwd(*args, h0=inp["h0"], workspace=ws)
+    torch.cuda.synchronize()
+    o = torch.empty_like(o_ref)
+    hT = torch.empty_like(h_ref)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        kda.fwd(*args, h0=inp["h0"], o=o, hT=hT, workspace=ws)
+    o.zero_()
+    hT.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert kda.get_device_error() == 0
+    assert torch.equal(o, o_ref) and torch.equal(hT, h_ref)
+    del graph

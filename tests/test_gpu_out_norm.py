@@ -63,15 +63,22 @@ CASES = [
         "packed-8docs", lengths=[1, 63, 64, 65, 0, 130, 7, 200], H=4, h0_std=0.05, seed=93)),
     ("one sequence, several chunks", lambda: synth.prefill_inputs("long-t65536", B=1, T=513,
                                                                   H=2, seed=94)),
-    # 71 chunks: the split path runs two chunk segments, each state pass applying the norm
+    # 71 chunks: the split path runs two chunk segments, each state pass applying the norm (the
+    # plain state pass: with 4 chains the default plan would take the two-level one)
     ("two chunk segments", lambda: synth.prefill_inputs("long-t65536", B=2, T=64 * 70 + 9, H=2,
-                                                        h0_std=0.05, seed=98)),
+                                                        h0_std=0.05, seed=98), "0"),
+    # the two-level state pass, 4 segments: segment 0 and the last phase apply the norm
+    ("two-level state pass", lambda: synth.prefill_inputs("long-t65536", B=2, T=64 * 20 + 9,
+                                                          H=2, h0_std=0.05, decay_mu=-3.0,
+                                                          seed=99), "4"),
 ]
 
 
 @pytest.mark.parametrize("path", ["split", "fused", "per-token"])
 @pytest.mark.parametrize("case", CASES, ids=lambda c: c[0])
-def test_fwd_normed_matches_the_oracle(case, path):
+def test_fwd_normed_matches_the_oracle(case, path, monkeypatch):
+    if len(case) > 2:   # the state-pass plan this case is about
+        monkeypatch.setenv("KDA_SCAN_SEGMENTS", case[2])
     inp = case[1]()
     g = to(inp, DEV)
     B, T, H = g["B"], g["T"], g["H"]
@@ -105,3 +112,22 @@ def test_normed_call_equals_fwd_then_norm(fused):
     torch.cuda.synchronize()
     assert kda.get_device_error() == 0
     assert torch.equal(y, y2), rel_l2(host(y), host(y2))
+
+
+def test_normed_call_equals_fwd_then_norm_two_level(monkeypatch):
+    """The same identity on the two-level state pass (5 segments forced): segment 0 and the last
+    phase's segments apply the norm to their output tiles; the maps launch writes no output."""
+    monkeypatch.setenv("KDA_SCAN_SEGMENTS", "5")
+    inp = synth.prefill_inputs("long-t65536", B=2, T=64 * 25 + 3, H=3, h0_std=0.05, seed=100,
+                               device=DEV)
+    B, T = inp["B"], inp["T"]
+    assert kda.fwd_scan_segments(B, T, 3, 128, 128, B) == 5
+    gate, w = _gate_weight((B, T, 3, 128), torch.bfloat16, 101)
+    y, h1 = kda.fwd(inp["q"], inp["k"], inp["v"], inp["log_g"], inp["beta"], h0=inp["h0"],
+                    out_norm=(gate, w, EPS))
+    o, h2 = kda.fwd(inp["q"], inp["k"], inp["v"], inp["log_g"], inp["beta"], h0=inp["h0"])
+    y2 = kda.out_norm_gated(o, gate, w, EPS)
+    torch.cuda.synchronize()
+    assert kda.get_device_error() == 0
+    assert torch.equal(y, y2), rel_l2(host(y), host(y2))
+    assert torch.equal(h1, h2)
