@@ -165,9 +165,13 @@ static int split_segments(int ncT) {
 // product per chain); then segments 1 .. P-1 at once from their initial states. P minimises a
 // cost model in units of one chunk of the state pass (about 1.6 us on B200): the intra-chunk
 // kernel (about 3.7 units of SM time per record, all SMs), then the phases, each ceil(units /
-// 148) waves of m chunks, plus 1.5 units per combine step and 4 for the launches; the plain pass is
+// 148) waves of m chunks, plus 2.5 units per combine step and 4 for the launches; the plain pass is
 // intra-chunk kernel + chain (one segment) or the larger of the two (chunk segments overlapping).
-// The two-level pass is used when it models at least 15 % faster. KDA_SCAN_SEGMENTS (read per
+// The two-level pass is used when it models at least 15 % faster. Measured on one B200 (L2
+// flushed, ms per call at P = plain, 3, 4, 5, 6, 7, 8, 10): 1 x 4096 tokens x 16 heads 0.158,
+// 0.147, 0.133, 0.129, 0.127, 0.144, 0.139, 0.141 (the model picks 6); 1 x 16384 x 16 0.543,
+// 0.440, 0.381, 0.354, 0.336, 0.373, 0.359, 0.354 (picks 6); 1 x 8192 x 8 0.260, 0.205, 0.176,
+// 0.162, 0.155, 0.150, 0.145, 0.143 (picks 10). KDA_SCAN_SEGMENTS (read per
 // call) overrides: 0 or 1 = the plain pass, 3 .. 32 = that many segments (capped by the chunks).
 static int scan_segments(int ncT, long long chains) {
     if (ncT < 3 || chains <= 0 || chains > 148) return 1;
@@ -195,7 +199,7 @@ static int scan_segments(int ncT, long long chains) {
         const int m = (ncT + P - 1) / P;
         const double w1 = std::ceil((2.0 * (P - 2) + 1.0) * ch / sms);
         const double w3 = std::ceil((P - 1.0) * ch / sms);
-        const double cost = intra + (w1 + w3) * m + 1.5 * (P - 2) + 4.0;
+        const double cost = intra + (w1 + w3) * m + 2.5 * (P - 2) + 4.0;
         if (cost < best) best = cost, bestP = P;
     }
     return bestP;
