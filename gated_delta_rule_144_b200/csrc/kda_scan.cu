@@ -40,6 +40,12 @@
 // The chain warps and the MMA warp synchronise with named barrier 1, the epilogue warps with named
 // barrier 2, and the two groups only through mbarriers. Every mbarrier wait is bounded; on expiry
 // the CTA records KDA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
+//
+// The same kernel serves the two-level state pass (kda_scan.cuh): a segmented launch gives each
+// CTA one (segment, chain) unit with its own initial and final state, a transition-map unit
+// starts from S = I with U~ taken as 0 (its final state is the segment's map A), and a launch
+// without outputs skips the epilogue's stores. scan_combine_kernel, below, chains the segments'
+// initial states between the launches.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
