@@ -308,6 +308,11 @@ def run_ours(args):
         segs = kda.fwd_split_segments(B, T, H, dk, dv, N, inp["q"].dtype, args.chunk_size,
                                       varlen=packed)
         launches = 2 * segs + ((2 if 2 <= N <= 2048 else 1) if packed else 0)
+        if kda.fwd_scan_segments(B, T, H, dk, dv, N, inp["q"].dtype, args.chunk_size,
+                                 varlen=packed) >= 3:
+            # two-level state pass: intra-chunk kernel, segment 0 and the maps, their chain,
+            # the remaining segments
+            launches = 5
     traffic = committed_traffic(kernel_name, wl.name)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                 "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
@@ -352,41 +357,74 @@ def run_ours(args):
 
 
 def run_e2e(kda, inp, args, stream, world, dev):
-    """Same metric through kda.fwd with pinned host inputs copied in and o, hT copied out."""
+    """Same metric through kda.fwd with pinned host inputs copied in and o, hT copied out, every
+    step. Steps run as a serving loop would run them: step i's inputs go up on one copy stream and
+    its outputs come down on another, so the download of step i overlaps the upload of step i + 1
+    (PCIe is full duplex); the device buffers are double-buffered and events order their reuse.
+    Every step's copies are inside the timed region."""
     keys = ("q", "k", "v", "log_g", "beta", "h0", "cu_seqlens")
     host = {k: (inp[k].cpu().pin_memory() if inp[k] is not None else None) for k in keys}
-    d_in = {k: (torch.empty_like(inp[k]) if inp[k] is not None else None) for k in keys}
+    nbuf = 2
+    d_in = [{k: (torch.empty_like(inp[k]) if inp[k] is not None else None) for k in keys}
+            for _ in range(nbuf)]
     B, T, H, dv, N, dk = inp["B"], inp["T"], inp["H"], inp["dv"], inp["N"], inp["dk"]
-    o = torch.empty((B, T, H, dv), dtype=inp["q"].dtype, device=dev)
-    hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
-    ws = workspace_for(kda, B, T, H, N, args, dev)
-    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    hT_h = torch.empty(hT.shape, dtype=hT.dtype).pin_memory()
+    o = [torch.empty((B, T, H, dv), dtype=inp["q"].dtype, device=dev) for _ in range(nbuf)]
+    hT = [torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev) for _ in range(nbuf)]
+    ws = workspace_for(kda, B, T, H, N, args, dev)   # the calls run in order on `stream`
+    o_h = [torch.empty(o[0].shape, dtype=o[0].dtype).pin_memory() for _ in range(nbuf)]
+    hT_h = [torch.empty(hT[0].shape, dtype=hT[0].dtype).pin_memory() for _ in range(nbuf)]
     h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
-    d2h = o.numel() * o.element_size() + hT.numel() * hT.element_size()
+    d2h = o[0].numel() * o[0].element_size() + hT[0].numel() * hT[0].element_size()
+    s_in = torch.cuda.Stream(device=dev)
+    s_out = torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(nbuf)]     # inputs of buffer b uploaded
+    ev_done = [torch.cuda.Event() for _ in range(nbuf)]   # the call on buffer b finished
+    ev_out = [torch.cuda.Event() for _ in range(nbuf)]    # outputs of buffer b downloaded
 
-    def step():
-        for k in keys:
-            if host[k] is not None:
-                d_in[k].copy_(host[k], non_blocking=True)
-        kda.fwd(d_in["q"], d_in["k"], d_in["v"], d_in["log_g"], d_in["beta"], h0=d_in["h0"],
-                cu_seqlens=d_in["cu_seqlens"], o=o, hT=hT, chunk_size=args.chunk_size,
-                workspace=ws, fused=args.fused)
-        o_h.copy_(o, non_blocking=True)
-        hT_h.copy_(hT, non_blocking=True)
+    def step(i):
+        b = i % nbuf
+        s_in.wait_event(ev_done[b])   # the call two steps back has read these inputs
+        with torch.cuda.stream(s_in):
+            for k in keys:
+                if host[k] is not None:
+                    d_in[b][k].copy_(host[k], non_blocking=True)
+        ev_in[b].record(s_in)
+        stream.wait_event(ev_in[b])
+        stream.wait_event(ev_out[b])  # the outputs two steps back have been read
+        g = d_in[b]
+        kda.fwd(g["q"], g["k"], g["v"], g["log_g"], g["beta"], h0=g["h0"],
+                cu_seqlens=g["cu_seqlens"], o=o[b], hT=hT[b], chunk_size=args.chunk_size,
+                workspace=ws, fused=args.fused, stream=stream)
+        ev_done[b].record(stream)
+        s_out.wait_event(ev_done[b])
+        with torch.cuda.stream(s_out):
+            o_h[b].copy_(o[b], non_blocking=True)
+            hT_h[b].copy_(hT[b], non_blocking=True)
+        ev_out[b].record(s_out)
 
     steps = max(1, min(args.steps, args.e2e_steps))
-    step()
+    for i in range(nbuf):   # warm-up: one step on each buffer
+        step(i)
     torch.cuda.synchronize()
     barrier(world)
-    total_ms, _ = time_launches(step, steps, stream)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(s_in)   # every stream is idle here: the first timed work is the first upload
+    for i in range(nbuf, nbuf + steps):
+        step(i)
+    stream.wait_stream(s_in)
+    stream.wait_stream(s_out)
+    t1.record(stream)
+    t1.synchronize()
+    total_ms = t0.elapsed_time(t1)
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(total_ms, world, dev)
     tokens_all = sum_over_ranks(float(B * T), world, dev)
     return {"value": round(tokens_all * steps / (ms / 1e3), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(ms / steps, 3)}
+            "ms_per_step": round(ms / steps, 3),
+            "pipelined": "download of step i overlaps upload of step i + 1"}
 
 
 def run_secondary(kda, synth, args, dev, stream, world, rank):
